@@ -1,0 +1,326 @@
+/*
+ * bi.h -- C ABI of libbi, batch-invariant inference kernels for NVIDIA B200 (sm_100a).
+ *
+ * What "batch-invariant" means here follows "Defeating Nondeterminism in LLM
+ * Inference" (section "Batch invariance and determinism"): the value computed
+ * for one row (one token) must not depend on how many other rows share the
+ * launch, where in the batch the row sits, how the engine chunked its
+ * sequence, or which run it is. Every kernel behind this header fixes the
+ * floating-point reduction order of each output element as a function of the
+ * reduced length only.
+ *
+ * Conventions shared by every entry point
+ *  - All tensor arguments are DEVICE pointers owned by the caller. bf16 data
+ *    is passed as `void*` (IEEE bfloat16, 2 bytes, round-to-nearest-even).
+ *    Matrices are row-major; leading dimensions (ld*) count ELEMENTS.
+ *  - `stream` is a cudaStream_t passed as `void*` (NULL = legacy stream).
+ *    Every call is asynchronous on that stream; nothing synchronises the host
+ *    except bi_device_status().
+ *  - Arguments are validated on the host before anything is launched. On a
+ *    non-BI_OK return nothing was enqueued and bi_last_error() (thread-local)
+ *    holds a one-line reason.
+ *  - No entry point allocates device memory. Scratch space is a caller-owned
+ *    workspace whose size comes from the matching *_workspace_size query.
+ *  - Data that only the device can see (page ids, slot ids, sequence lengths)
+ *    is range-checked inside the kernels: an out-of-range value skips the
+ *    access and sets a bit of the library's device status word, read with
+ *    bi_device_status(). Kernels never trap and every device-side wait is
+ *    bounded (a timeout also sets a status bit and the kernel returns).
+ *  - No reduction uses atomics, split-K or stream-K; the launch shape never
+ *    depends on the batch size in a way that reaches the arithmetic.
+ */
+#ifndef BI_H_
+#define BI_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BI_OK = 0,
+  BI_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad enum */
+  BI_ERR_SHAPE = 2,       /* size outside what the kernel supports */
+  BI_ERR_ALIGN = 3,       /* pointer or leading dimension misaligned */
+  BI_ERR_WORKSPACE = 4,   /* workspace missing or too small */
+  BI_ERR_UNSUPPORTED = 5, /* no sm_100 device / feature unavailable */
+  BI_ERR_CUDA = 6,        /* a CUDA runtime/driver call failed */
+  BI_ERR_DEVICE_CHECK = 7 /* device status word non-zero (bi_device_status) */
+} bi_status;
+
+typedef enum { BI_BF16 = 0, BI_F32 = 1 } bi_dtype;
+
+/* Fixed geometry. These are compile-time constants on purpose: a tile or split
+ * size chosen at run time from the problem shape would make the reduction order
+ * depend on the batch, which is exactly what the library must not do. */
+#define BI_HEAD_DIM 128   /* attention head dimension d_h */
+#define BI_PAGE_SIZE 16   /* tokens per KV-cache page */
+#define BI_ATTN_TILE 128  /* keys per attention tile, at absolute key offsets */
+#define BI_ATTN_SPLIT 512 /* keys per KV split (fixed split SIZE, not count) */
+#define BI_GEMM_BM 128    /* GEMM output tile rows */
+#define BI_GEMM_BN 256    /* GEMM output tile columns */
+#define BI_GEMM_BK 64     /* GEMM K stage */
+
+/* Device status word bits (bi_device_status). */
+#define BI_DEV_WAIT_TIMEOUT 0x1 /* a bounded mbarrier wait ran out */
+#define BI_DEV_BAD_SLOT 0x2     /* slot_mapping entry outside the cache */
+#define BI_DEV_BAD_PAGE 0x4     /* block_table entry outside the cache */
+#define BI_DEV_BAD_SEQLEN 0x8   /* seq_lens entry outside [n_query, max_kv_len] */
+#define BI_DEV_BAD_TOKEN 0x10   /* token id outside the vocabulary */
+
+/* Thread-local description of the last failure on this host thread. */
+const char* bi_last_error(void);
+
+/* Reads the device status word of the current device into *status (after
+ * synchronising `stream`), and clears it when `clear` is non-zero.
+ * Returns BI_ERR_DEVICE_CHECK when the word was non-zero. */
+bi_status bi_device_status(int32_t* status, int32_t clear, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* RMSNorm.  "Defeating Nondeterminism in LLM Inference", section
+ * "Batch-invariant RMSNorm": the reference definition x * rsqrt(mean(x^2)) *
+ * weight, parallelised with one row per core so that no row's reduction is
+ * ever split. eps is added inside the square root.
+ *
+ *   y[i, :] = bf16( x[i, :] * r_i * gamma ),  r_i = 1 / sqrt(sum_j x_ij^2 / D + eps)
+ *
+ * x [M, D] bf16 row-major (ld = D), gamma [D] bf16, y [M, D] bf16.
+ * The sum of squares is fp32 in an order that depends on D only: each thread
+ * adds its 8-element chunks in sequence, then a warp shuffle tree, then warp
+ * partials in warp order. Needs D % 8 == 0, 8 <= D <= 32768, pointers 16-byte
+ * aligned. M == 0 is a no-op. One CTA per row. */
+bi_status bi_rmsnorm(const void* x, const void* gamma, void* y, int64_t M,
+                     int64_t D, float eps, void* stream);
+
+/* Same reduction, fp32 input rows (the residual stream of bi_forward) and bf16
+ * output. x [M, D] fp32. */
+bi_status bi_rmsnorm_f32in(const float* x, const void* gamma, void* y,
+                           int64_t M, int64_t D, float eps, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* GEMM.  "Defeating Nondeterminism in LLM Inference", section "Batch-invariant
+ * matmul": a data-parallel output tiling with each K reduction inside one
+ * core, one kernel configuration for every shape, no split-K, no stream-K.
+ *
+ *   C[m, n] = sum_k A[m, k] * W[n, k]        (C = A * W^T, nn.Linear layout)
+ *
+ * A [M, K] bf16 (row stride lda), W [N, K] bf16 (row stride ldw), C [M, N]
+ * (row stride ldc) bf16 (c_dtype = BI_BF16, round-to-nearest-even) or fp32
+ * (BI_F32). Products are exact, accumulation is fp32 in tensor memory, one
+ * tcgen05.mma kind::f16 shape (128 x 256 x 16), K walked 0, 16, 32, ... in
+ * order whatever M is. Needs K % 8 == 0, N % 8 == 0, lda/ldw/ldc % 8 == 0,
+ * A, W, C 16-byte aligned. M == 0 or N == 0 is a no-op. K == 0 writes zeros. */
+bi_status bi_gemm(const void* A, int64_t lda, const void* W, int64_t ldw,
+                  void* C, int64_t ldc, int32_t c_dtype, int64_t M, int64_t N,
+                  int64_t K, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Paged KV cache.  "Defeating Nondeterminism in LLM Inference", section
+ * "Batch-invariant attention": the cache and page table are updated BEFORE
+ * the attention kernel runs, so every key is read from the same layout
+ * whether it was cached earlier or belongs to the chunk in flight.
+ *
+ * Layout (one page = BI_PAGE_SIZE tokens, d_h = BI_HEAD_DIM):
+ *   k_cache [num_pages, num_kv_heads, 16, 128] bf16   (key rows, d contiguous)
+ *   v_cache [num_pages, num_kv_heads, 128, 16] bf16   (values stored transposed)
+ * Token slot s = page * 16 + offset. */
+typedef struct {
+  int32_t num_pages;
+  int32_t num_kv_heads;
+  int32_t head_dim;  /* must be BI_HEAD_DIM */
+  int32_t page_size; /* must be BI_PAGE_SIZE */
+} bi_kv_layout;
+
+/* Writes token t's key and value rows (k_new + t*ld_new, num_kv_heads * 128
+ * bf16 each) into slot slot_mapping[t]. A negative slot skips the token
+ * (padding). A slot >= num_pages*16 is skipped and sets BI_DEV_BAD_SLOT.
+ * Pure data movement: the cache holds the exact input bytes. */
+bi_status bi_kv_append(const void* k_new, const void* v_new, int64_t ld_new,
+                       const int32_t* slot_mapping, int64_t n_tok,
+                       void* k_cache, void* v_cache, const bi_kv_layout* kv,
+                       void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Attention over the paged cache, causal, grouped-query (q head h reads kv
+ * head h / (num_q_heads / num_kv_heads)).
+ *
+ * "Defeating Nondeterminism in LLM Inference", section "Batch-invariant
+ * attention": the reduction order for a query must not depend on how many
+ * tokens of its sequence are processed at once, nor on how many are already
+ * cached; decoding needs a split reduction over the keys. The split used
+ * here has a fixed SIZE (BI_ATTN_SPLIT keys at absolute key offsets), so a
+ * query at position p always reduces over splits 0..p/512, each walked in
+ * 128-key tiles at absolute offsets with an online softmax, and the splits
+ * are merged in index order by a separate finishing pass (same section and
+ * "When are atomic adds needed?": split reduction plus a serial finish).
+ *
+ * Per split s and row: S = (q . k_j) * scale in fp32 (tcgen05, bf16 inputs),
+ * keys j > p masked, m' = max(m, rowmax), alpha = exp(m - m'),
+ * P = bf16(exp(S - m')), l = alpha*l + sum(P) (fixed order), O = alpha*O + P.V.
+ * Merge: M = max_s m_s, w_s = exp(m_s - M), out = bf16(sum_s w_s O_s / sum_s
+ * w_s l_s), sums in split order. Decode and prefill run the same kernels, so
+ * a token's output is bitwise equal in both.
+ *
+ * q rows: token t, head h at q + t*ldq + h*128 (bf16). out likewise with ldo.
+ * block_table [B, max_pages_per_seq] int32 (page ids, in key order),
+ * seq_lens [B] int32 = number of keys in the cache for sequence b, INCLUDING
+ * the tokens queried in this call (they were appended first). */
+typedef struct {
+  int32_t num_q_heads;       /* Hq */
+  int32_t num_kv_heads;      /* Hkv; Hq / Hkv must be 1, 2, 4 or 8 */
+  int32_t head_dim;          /* must be BI_HEAD_DIM */
+  int32_t page_size;         /* must be BI_PAGE_SIZE */
+  int32_t num_pages;         /* pages in each cache (device range check) */
+  int32_t max_pages_per_seq; /* row stride of block_table */
+  int32_t max_kv_len;        /* upper bound of seq_lens (grid + workspace) */
+  float scale;               /* softmax scale, e.g. 1/sqrt(128) */
+} bi_attn_shape;
+
+/* Workspace bytes for up to `max_tokens` query tokens with keys up to
+ * shape->max_kv_len: per (token, q head, split) 128 fp32 partial outputs plus
+ * (m, l). */
+bi_status bi_attn_workspace_size(const bi_attn_shape* shape, int64_t max_tokens,
+                                 size_t* bytes);
+
+/* Decode: one query per sequence; q/out row b belongs to sequence b and sits
+ * at position seq_lens[b] - 1. */
+bi_status bi_attn_decode(const void* q, int64_t ldq, const void* k_cache,
+                         const void* v_cache, const int32_t* block_table,
+                         const int32_t* seq_lens, int32_t B,
+                         const bi_attn_shape* shape, void* out, int64_t ldo,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* Prefill (chunked): sequence b owns query rows cu_q[b] .. cu_q[b+1]-1
+ * (cu_q [B+1] int32 on the device, cu_q[0] = 0, cu_q[B] = n_tok); they are its
+ * LAST n_b = cu_q[b+1]-cu_q[b] tokens, so row cu_q[b]+i sits at position
+ * seq_lens[b] - n_b + i. max_q_len bounds n_b (host-side grid size). */
+bi_status bi_attn_prefill(const void* q, int64_t ldq, const int32_t* cu_q,
+                          int32_t max_q_len, int64_t n_tok, const void* k_cache,
+                          const void* v_cache, const int32_t* block_table,
+                          const int32_t* seq_lens, int32_t B,
+                          const bi_attn_shape* shape, void* out, int64_t ldo,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Pointwise steps of the decoder. "Defeating Nondeterminism in LLM
+ * Inference", section "How do we make kernels batch-invariant?": pointwise
+ * operations are batch-invariant as long as every element takes the same code
+ * path; each kernel below has exactly one path per element. */
+
+/* Embedding gather: out[t, :] = float(table[tokens[t], :]), table [V, D] bf16,
+ * out [n_tok, D] fp32 (the residual stream). Bad ids write zeros and set
+ * BI_DEV_BAD_TOKEN. D % 8 == 0. */
+bi_status bi_embed(const int32_t* tokens, int64_t n_tok, const void* table,
+                   int64_t vocab, int64_t D, float* out, void* stream);
+
+/* Rotary embedding in place, rotate-half pairing (i, i + 64) of each 128-wide
+ * head, angle = pos * theta^(-2i/128) evaluated in fp64 on the host into an
+ * fp32 cos/sin table. x row t, head h at x + t*ldx + h*128 (bf16), positions
+ * [n_tok] int32 on the device, < max_pos. Writes bf16(x_i c - x_{i+64} s) and
+ * bf16(x_{i+64} c + x_i s) computed in fp32. cos_sin: [max_pos, 64, 2] fp32
+ * caller-owned table filled by bi_rope_table. */
+bi_status bi_rope_table(float* cos_sin, int32_t max_pos, double theta,
+                        void* stream);
+bi_status bi_rope(void* x, int64_t ldx, int32_t n_heads, const int32_t* positions,
+                  int64_t n_tok, const float* cos_sin, int32_t max_pos,
+                  void* stream);
+
+/* SwiGLU: out[t, i] = bf16( silu(g) * u ), g = gu[t, i], u = gu[t, F + i],
+ * silu(g) = g / (1 + exp(-g)) in fp32. gu [n_tok, 2F] bf16, out [n_tok, F]. */
+bi_status bi_swiglu(const void* gu, int64_t n_tok, int64_t F, void* out,
+                    void* stream);
+
+/* Residual add: x[t, :] += float(d[t, :]) in fp32, d bf16 [n_tok, D]. */
+bi_status bi_residual_add(float* x, const void* d, int64_t n_tok, int64_t D,
+                          void* stream);
+
+/* Greedy token: idx[r] = argmax_j logits[r, j] over fp32 logits [rows, V]
+ * (row stride ld), lowest index on ties. Max is exact, so the result is
+ * order-free. NaN rows return the first NaN's index. */
+bi_status bi_argmax(const float* logits, int64_t rows, int64_t V, int64_t ld,
+                    int32_t* idx, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Dense decoder forward (pre-norm, RMSNorm, RoPE, GQA attention, SwiGLU MLP),
+ * composed only of the kernels above, with an fp32 residual stream and fp32
+ * logits. */
+typedef struct {
+  int32_t n_layers;
+  int32_t d_model;     /* D */
+  int32_t n_q_heads;   /* Hq, head_dim = BI_HEAD_DIM, Hq * 128 == D */
+  int32_t n_kv_heads;  /* Hkv */
+  int32_t d_ff;        /* F */
+  int32_t vocab;       /* V */
+  int32_t max_pos;     /* positions < max_pos */
+  float rms_eps;
+  double rope_theta;
+} bi_model_config;
+
+/* Caller-owned device weights, bf16, nn.Linear layout [out, in]. Per layer l
+ * the arrays hold n_layers consecutive blocks:
+ *   attn_norm [L][D], w_qkv [L][(Hq + 2 Hkv) * 128][D] (rows: q heads, then k
+ *   heads, then v heads), w_o [L][D][Hq * 128], mlp_norm [L][D],
+ *   w_gate_up [L][2F][D] (gate rows, then up rows), w_down [L][D][F];
+ *   embed [V][D], final_norm [D], lm_head [V][D]. */
+typedef struct {
+  const void* embed;
+  const void* attn_norm;
+  const void* w_qkv;
+  const void* w_o;
+  const void* mlp_norm;
+  const void* w_gate_up;
+  const void* w_down;
+  const void* final_norm;
+  const void* lm_head;
+} bi_model_weights;
+
+typedef struct bi_model bi_model;
+
+/* One forward step over n_tok tokens of B sequences (any mix of prefill
+ * chunks and decode tokens). All arrays are device int32:
+ *   tokens [n_tok], positions [n_tok], slot_mapping [n_tok],
+ *   cu_q [B+1] (rows of each sequence, contiguous and in order),
+ *   seq_lens [B] (keys cached after this step), block_table [B][max_pages_per_seq],
+ *   logits_rows [n_logits] (which token rows produce logits).
+ * Host ints: max_q_len bounds cu_q[b+1]-cu_q[b]; max_kv_len bounds seq_lens. */
+typedef struct {
+  const int32_t* tokens;
+  const int32_t* positions;
+  const int32_t* slot_mapping;
+  const int32_t* cu_q;
+  const int32_t* seq_lens;
+  const int32_t* block_table;
+  const int32_t* logits_rows;
+  int64_t n_tok;
+  int32_t B;
+  int32_t max_q_len;
+  int32_t max_kv_len;
+  int32_t max_pages_per_seq;
+  int64_t n_logits;
+} bi_batch;
+
+bi_status bi_model_create(const bi_model_config* cfg, const bi_model_weights* w,
+                          bi_model** out);
+void bi_model_destroy(bi_model* m);
+
+/* Workspace for a step of up to max_tokens tokens, max_logits logit rows and
+ * keys up to max_kv_len. */
+bi_status bi_forward_workspace_size(const bi_model* m, int64_t max_tokens,
+                                    int64_t max_logits, int32_t max_kv_len,
+                                    size_t* bytes);
+
+/* k_cache / v_cache: layout bi_kv_layout with num_layers consecutive caches,
+ * layer l at offset l * num_pages * Hkv * 16 * 128 elements. logits
+ * [n_logits, V] fp32; next_tokens [n_logits] int32 (nullable) = greedy argmax. */
+bi_status bi_forward(const bi_model* m, const bi_batch* batch, void* k_cache,
+                     void* v_cache, int32_t num_pages, float* logits,
+                     int32_t* next_tokens, void* ws, size_t ws_bytes,
+                     void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BI_H_ */

@@ -1,0 +1,27 @@
+"""CPU oracle for the batch-invariant kernels -- TEST INFRASTRUCTURE ONLY.
+
+Nothing on the product path may import, call or link anything in this
+package: only the test suite, the smoke check and the CPU-baseline leg of the
+benchmark use it. It shares no code, header, table or constant with the CUDA
+library; its inputs come from the seeded generators in
+``invariant_deterministic_03_b200.synth`` (which hold none of the method's
+arithmetic), passed in as arrays.
+
+Two independent views of every operation:
+
+* :mod:`oracle.fp64`  -- the plain mathematical definition in float64
+  (numpy; a library matmul serves as the matmul step).
+* :mod:`oracle.ordered` -- the same operations in float32 with one fixed,
+  written-out summation order (plain C in ``ordered.c``: sequential ``fmaf``
+  accumulation), used to show order dependence and to time the CPU baseline.
+
+bf16 tensors cross into the oracle as uint16 bit patterns or as float64
+arrays that hold bf16 values exactly (:func:`oracle.fp64.bf16_bits_to_f64`).
+
+Parity status: every function of :mod:`oracle.fp64` except ``forward`` is
+pinned by ``tests/test_oracle_pins.py`` against closed forms, exact rational
+arithmetic, brute force or the worked examples printed in "Defeating
+Nondeterminism in LLM Inference". ``forward`` is pinned only structurally
+(causality, identity blocks, one-token closed form): the pages print no logits
+for any model, so its end-to-end values are "parity unpinned".
+"""
