@@ -1,0 +1,281 @@
+"""Thin ctypes binding of libbi (include/bi.h) for torch tensors.
+
+Argument marshalling only: every entry point takes device tensors, passes
+their data pointers, sizes and the current CUDA stream to the C ABI and raises
+:class:`BIError` on a non-zero status. No arithmetic of the path runs here and
+there is no CPU fallback: importing this module fails loudly when libbi.so is
+missing, and every call fails on a non-B200 device.
+
+The functions named ``bi_*`` mirror the C entry points (outputs passed in);
+the short names (``rmsnorm``, ``gemm``, ...) allocate their outputs with torch
+and call the same entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbi.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libbi.so is not built ({LIB_PATH}); run "
+                      "`python -m invariant_deterministic_03_b200.build`")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+BI_OK, BI_ERR_INVALID_ARG, BI_ERR_SHAPE, BI_ERR_ALIGN, BI_ERR_WORKSPACE, \
+    BI_ERR_UNSUPPORTED, BI_ERR_CUDA, BI_ERR_DEVICE_CHECK = range(8)
+BI_BF16, BI_F32 = 0, 1
+HEAD_DIM, PAGE_SIZE, ATTN_TILE, ATTN_SPLIT = 128, 16, 128, 512
+GEMM_BM, GEMM_BN, GEMM_BK = 128, 256, 64
+
+_p, _i32, _i64, _f32, _f64, _sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64,
+                                   ctypes.c_float, ctypes.c_double, ctypes.c_size_t)
+
+
+class KVLayout(ctypes.Structure):
+    _fields_ = [("num_pages", _i32), ("num_kv_heads", _i32), ("head_dim", _i32),
+                ("page_size", _i32)]
+
+
+class AttnShape(ctypes.Structure):
+    _fields_ = [("num_q_heads", _i32), ("num_kv_heads", _i32), ("head_dim", _i32),
+                ("page_size", _i32), ("num_pages", _i32), ("max_pages_per_seq", _i32),
+                ("max_kv_len", _i32), ("scale", _f32)]
+
+
+class ModelConfig(ctypes.Structure):
+    _fields_ = [("n_layers", _i32), ("d_model", _i32), ("n_q_heads", _i32),
+                ("n_kv_heads", _i32), ("d_ff", _i32), ("vocab", _i32), ("max_pos", _i32),
+                ("rms_eps", _f32), ("rope_theta", _f64)]
+
+
+class ModelWeights(ctypes.Structure):
+    _fields_ = [(n, _p) for n in ("embed", "attn_norm", "w_qkv", "w_o", "mlp_norm",
+                                  "w_gate_up", "w_down", "final_norm", "lm_head")]
+
+
+class Batch(ctypes.Structure):
+    _fields_ = [("tokens", _p), ("positions", _p), ("slot_mapping", _p), ("cu_q", _p),
+                ("seq_lens", _p), ("block_table", _p), ("logits_rows", _p), ("n_tok", _i64),
+                ("B", _i32), ("max_q_len", _i32), ("max_kv_len", _i32),
+                ("max_pages_per_seq", _i32), ("n_logits", _i64)]
+
+
+_SIGS = {
+    "bi_last_error": (ctypes.c_char_p, []),
+    "bi_device_status": (_i32, [ctypes.POINTER(_i32), _i32, _p]),
+    "bi_rmsnorm": (_i32, [_p, _p, _p, _i64, _i64, _f32, _p]),
+    "bi_rmsnorm_f32in": (_i32, [_p, _p, _p, _i64, _i64, _f32, _p]),
+    "bi_gemm": (_i32, [_p, _i64, _p, _i64, _p, _i64, _i32, _i64, _i64, _i64, _p]),
+    "bi_kv_append": (_i32, [_p, _p, _i64, _p, _i64, _p, _p, ctypes.POINTER(KVLayout), _p]),
+    "bi_attn_workspace_size": (_i32, [ctypes.POINTER(AttnShape), _i64, ctypes.POINTER(_sz)]),
+    "bi_attn_decode": (_i32, [_p, _i64, _p, _p, _p, _p, _i32, ctypes.POINTER(AttnShape), _p,
+                              _i64, _p, _sz, _p]),
+    "bi_attn_prefill": (_i32, [_p, _i64, _p, _i32, _i64, _p, _p, _p, _p, _i32,
+                               ctypes.POINTER(AttnShape), _p, _i64, _p, _sz, _p]),
+    "bi_embed": (_i32, [_p, _i64, _p, _i64, _i64, _p, _p]),
+    "bi_rope_table": (_i32, [_p, _i32, _f64, _p]),
+    "bi_rope": (_i32, [_p, _i64, _i32, _p, _i64, _p, _i32, _p]),
+    "bi_swiglu": (_i32, [_p, _i64, _i64, _p, _p]),
+    "bi_residual_add": (_i32, [_p, _p, _i64, _i64, _p]),
+    "bi_argmax": (_i32, [_p, _i64, _i64, _i64, _p, _p]),
+    "bi_model_create": (_i32, [ctypes.POINTER(ModelConfig), ctypes.POINTER(ModelWeights),
+                               ctypes.POINTER(_p)]),
+    "bi_model_destroy": (None, [_p]),
+    "bi_forward_workspace_size": (_i32, [_p, _i64, _i64, _i32, ctypes.POINTER(_sz)]),
+    "bi_forward": (_i32, [_p, ctypes.POINTER(Batch), _p, _p, _i32, _p, _p, _p, _sz, _p]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+EXPORTS = tuple(_SIGS)
+
+
+class BIError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        msg = lib.bi_last_error().decode(errors="replace")
+        super().__init__(f"{fn} failed with status {status}: {msg}")
+
+
+def _chk(fn: str, st: int) -> None:
+    if st != BI_OK:
+        raise BIError(fn, st)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None) -> int | None:
+    if stream is not None:
+        return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+    return torch.cuda.current_stream().cuda_stream
+
+
+# ------------------------------------------------------------------ entry points
+
+def bi_device_status(clear: bool = True, stream=None) -> int:
+    v = _i32(0)
+    st = lib.bi_device_status(ctypes.byref(v), int(clear), _stream(stream))
+    if st not in (BI_OK, BI_ERR_DEVICE_CHECK):
+        raise BIError("bi_device_status", st)
+    return v.value
+
+
+def bi_rmsnorm(x, gamma, y, eps: float, stream=None) -> None:
+    M, D = x.shape
+    fn = "bi_rmsnorm_f32in" if x.dtype == torch.float32 else "bi_rmsnorm"
+    _chk(fn, getattr(lib, fn)(_ptr(x), _ptr(gamma), _ptr(y), M, D, eps, _stream(stream)))
+
+
+def bi_gemm(A, W, C, stream=None) -> None:
+    """C = A W^T. A [M, K] bf16, W [N, K] bf16, C [M, N] bf16 or fp32 (row strides
+    taken from the tensors)."""
+    M, K = A.shape
+    N = W.shape[0]
+    cdt = BI_F32 if C.dtype == torch.float32 else BI_BF16
+    _chk("bi_gemm", lib.bi_gemm(_ptr(A), A.stride(0), _ptr(W), W.stride(0), _ptr(C), C.stride(0),
+                                cdt, M, N, K, _stream(stream)))
+
+
+def bi_kv_append(k_new, v_new, slot_mapping, k_cache, v_cache, stream=None) -> None:
+    n_tok = k_new.shape[0]
+    kv = KVLayout(k_cache.shape[0], k_cache.shape[1], HEAD_DIM, PAGE_SIZE)
+    ld = k_new.stride(0)
+    _chk("bi_kv_append", lib.bi_kv_append(_ptr(k_new), _ptr(v_new), ld, _ptr(slot_mapping), n_tok,
+                                          _ptr(k_cache), _ptr(v_cache), ctypes.byref(kv),
+                                          _stream(stream)))
+
+
+def attn_shape(num_q_heads, num_kv_heads, num_pages, max_pages_per_seq, max_kv_len,
+               scale=None) -> AttnShape:
+    return AttnShape(num_q_heads, num_kv_heads, HEAD_DIM, PAGE_SIZE, num_pages,
+                     max_pages_per_seq, max_kv_len,
+                     1.0 / math.sqrt(HEAD_DIM) if scale is None else scale)
+
+
+def bi_attn_workspace_size(shape: AttnShape, max_tokens: int) -> int:
+    n = _sz(0)
+    _chk("bi_attn_workspace_size", lib.bi_attn_workspace_size(ctypes.byref(shape), max_tokens,
+                                                              ctypes.byref(n)))
+    return n.value
+
+
+def bi_attn_decode(q, k_cache, v_cache, block_table, seq_lens, shape: AttnShape, out, ws,
+                   stream=None) -> None:
+    B = seq_lens.shape[0]
+    _chk("bi_attn_decode", lib.bi_attn_decode(
+        _ptr(q), q.stride(0), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens), B,
+        ctypes.byref(shape), _ptr(out), out.stride(0), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def bi_attn_prefill(q, cu_q, max_q_len: int, k_cache, v_cache, block_table, seq_lens,
+                    shape: AttnShape, out, ws, stream=None) -> None:
+    B = seq_lens.shape[0]
+    _chk("bi_attn_prefill", lib.bi_attn_prefill(
+        _ptr(q), q.stride(0), _ptr(cu_q), max_q_len, q.shape[0], _ptr(k_cache), _ptr(v_cache),
+        _ptr(block_table), _ptr(seq_lens), B, ctypes.byref(shape), _ptr(out), out.stride(0),
+        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def bi_embed(tokens, table, out, stream=None) -> None:
+    _chk("bi_embed", lib.bi_embed(_ptr(tokens), tokens.shape[0], _ptr(table), table.shape[0],
+                                  table.shape[1], _ptr(out), _stream(stream)))
+
+
+def bi_rope_table(cos_sin, max_pos: int, theta: float, stream=None) -> None:
+    _chk("bi_rope_table", lib.bi_rope_table(_ptr(cos_sin), max_pos, theta, _stream(stream)))
+
+
+def bi_rope(x, n_heads: int, positions, cos_sin, max_pos: int, stream=None) -> None:
+    _chk("bi_rope", lib.bi_rope(_ptr(x), x.stride(0), n_heads, _ptr(positions), x.shape[0],
+                                _ptr(cos_sin), max_pos, _stream(stream)))
+
+
+def bi_swiglu(gu, out, stream=None) -> None:
+    _chk("bi_swiglu", lib.bi_swiglu(_ptr(gu), gu.shape[0], gu.shape[1] // 2, _ptr(out),
+                                    _stream(stream)))
+
+
+def bi_residual_add(x, d, stream=None) -> None:
+    _chk("bi_residual_add", lib.bi_residual_add(_ptr(x), _ptr(d), x.shape[0], x.shape[1],
+                                                _stream(stream)))
+
+
+def bi_argmax(logits, idx, stream=None) -> None:
+    _chk("bi_argmax", lib.bi_argmax(_ptr(logits), logits.shape[0], logits.shape[1],
+                                    logits.stride(0), _ptr(idx), _stream(stream)))
+
+
+# ------------------------------------------------------------------ allocating helpers
+
+def rmsnorm(x, gamma, eps: float):
+    y = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device)
+    bi_rmsnorm(x, gamma, y, eps)
+    return y
+
+
+def gemm(A, W, out_dtype=torch.bfloat16):
+    C = torch.empty((A.shape[0], W.shape[0]), dtype=out_dtype, device=A.device)
+    bi_gemm(A, W, C)
+    return C
+
+
+def new_kv_cache(num_pages: int, num_kv_heads: int, device, n_layers: int = 1, zero=True):
+    """k [L, pages, Hkv, 16, 128] and v [L, pages, Hkv, 128, 16] bf16 (v transposed per page)."""
+    f = torch.zeros if zero else torch.empty
+    k = f((n_layers, num_pages, num_kv_heads, PAGE_SIZE, HEAD_DIM), dtype=torch.bfloat16, device=device)
+    v = f((n_layers, num_pages, num_kv_heads, HEAD_DIM, PAGE_SIZE), dtype=torch.bfloat16, device=device)
+    return k, v
+
+
+class Model:
+    """A bi_model handle over caller-owned device weights (dict of bf16 tensors
+    in nn.Linear layout, as produced by synth.model_weights moved to the GPU)."""
+
+    def __init__(self, cfg: dict, weights: dict):
+        self.cfg = dict(cfg)
+        self.weights = weights  # keep the tensors alive
+        c = ModelConfig(cfg["n_layers"], cfg["d_model"], cfg["n_q_heads"], cfg["n_kv_heads"],
+                        cfg["d_ff"], cfg["vocab"], cfg["max_pos"], cfg["rms_eps"],
+                        cfg["rope_theta"])
+        w = ModelWeights(*[_ptr(weights[n]) for n, _ in ModelWeights._fields_])
+        h = _p(0)
+        _chk("bi_model_create", lib.bi_model_create(ctypes.byref(c), ctypes.byref(w),
+                                                    ctypes.byref(h)))
+        self.handle = h
+
+    def __del__(self):
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            lib.bi_model_destroy(self.handle)
+            self.handle = None
+
+    def workspace_size(self, max_tokens: int, max_logits: int, max_kv_len: int) -> int:
+        n = _sz(0)
+        _chk("bi_forward_workspace_size", lib.bi_forward_workspace_size(
+            self.handle, max_tokens, max_logits, max_kv_len, ctypes.byref(n)))
+        return n.value
+
+    def forward(self, batch: dict, k_cache, v_cache, logits, next_tokens, ws, stream=None):
+        """batch: device int32 tensors tokens, positions, slot_mapping, cu_q,
+        seq_lens, block_table [B, P], logits_rows, plus host ints max_q_len,
+        max_kv_len."""
+        bt = batch["block_table"]
+        b = Batch(_ptr(batch["tokens"]), _ptr(batch["positions"]), _ptr(batch["slot_mapping"]),
+                  _ptr(batch["cu_q"]), _ptr(batch["seq_lens"]), _ptr(bt),
+                  _ptr(batch["logits_rows"]), batch["tokens"].shape[0],
+                  batch["seq_lens"].shape[0], batch["max_q_len"], batch["max_kv_len"],
+                  bt.shape[1], batch["logits_rows"].shape[0])
+        _chk("bi_forward", lib.bi_forward(self.handle, ctypes.byref(b), _ptr(k_cache),
+                                          _ptr(v_cache), k_cache.shape[1], _ptr(logits),
+                                          _ptr(next_tokens), _ptr(ws),
+                                          ws.numel() * ws.element_size(), _stream(stream)))

@@ -1,0 +1,588 @@
+// attention.cu -- batch-invariant paged attention (decode and chunked
+// prefill share every instruction of the per-row arithmetic).
+//
+// "Defeating Nondeterminism in LLM Inference", section "Batch-invariant
+// attention":
+//  - parallelise over queries (FlashAttention-2 style) and reduce over the
+//    keys inside one core;
+//  - the reduction order of a query must be the same whether its sequence is
+//    processed whole, in chunks, or one token at a time (query 1000 with 0 or
+//    999 cached tokens): keys are always read from the paged cache, which is
+//    updated BEFORE this kernel, and walked in 128-key tiles at ABSOLUTE key
+//    offsets (multiples of 128 from key 0);
+//  - decode needs a split reduction over the keys (Split-KV / FlashDecoding).
+//    Here a split is a fixed SIZE of 512 keys at absolute offsets, so a query
+//    at position p always uses splits 0 .. p/512, and a separate finishing
+//    pass merges them in split order (section "When are atomic adds
+//    needed?": split reduction plus a serial finishing reduction).
+//
+// Split kernel: one CTA per (split s, sequence b, query block, kv head g).
+// The CTA's 128 MMA rows are (query, q head of group g) pairs. Per tile:
+//   S  = Q K^T            tcgen05.mma M128 N128 K16 x8, fp32 in TMEM
+//   per row (one thread): m' = max(m, max_j s_j log2e*scale), alpha = 2^(m-m'),
+//        P_j = bf16(2^(s_j - m')), l = alpha*l + sum_j P_j (j = 0..127 in order)
+//   PV = P V              tcgen05.mma M128 N128 K16 x8 (one 16-key page per MMA)
+//   O  = fma(alpha, O, PV) per element, in registers.
+// A row takes part only in tiles whose first key is <= its position, so the
+// update sequence of a row is a function of (position, split) alone.
+// Masked keys get P = 0 by selection (never by arithmetic on -inf), and
+// cache slots at or past the sequence length are zeroed in shared memory so
+// that stale cache contents cannot reach the P.V products.
+#include "common.cuh"
+#include "host.h"
+
+namespace bi {
+namespace attn {
+
+constexpr int HD = BI_HEAD_DIM;        // 128
+constexpr int TILE = BI_ATTN_TILE;     // 128 keys
+constexpr int SPLIT = BI_ATTN_SPLIT;   // 512 keys
+constexpr int PAGE = BI_PAGE_SIZE;     // 16 keys
+constexpr int PAGES_PER_TILE = TILE / PAGE;
+constexpr uint32_t TILE_BYTES = 128 * 128 * 2;  // 32 KB: Q, K, V and P tiles
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_K = TILE_BYTES;          // 2 buffers
+constexpr uint32_t OFF_V = 3 * TILE_BYTES;      // 2 buffers
+constexpr uint32_t OFF_P = 5 * TILE_BYTES;
+constexpr uint32_t OFF_BAR = 6 * TILE_BYTES;
+constexpr size_t SMEM_BYTES = 1024 + 6 * TILE_BYTES + 256;
+constexpr int THREADS = 160;  // warps 0-3: one row each thread; warp 4: TMA + MMA
+constexpr uint32_t TMEM_COLS = 256;  // S at [0,128), PV at [128,256)
+
+struct Params {
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  const int32_t* cu_q;  // null: decode (one query per sequence, row b)
+  float* ws_o;          // [n_tok, Hq, n_split_max, 128]
+  float* ws_ml;         // [n_tok, Hq, n_split_max, 2]
+  int32_t B, Hq, Hkv, G, QR, qblocks, q_box, n_tok;
+  int32_t num_pages, max_pages, max_kv_len, n_split_max;
+  float scale_log2;
+  int32_t* status;
+};
+
+__device__ __forceinline__ void load_kv_tile(const Params& p, const CUtensorMap* tmK,
+                                             const CUtensorMap* tmV, uint8_t* kbuf, uint8_t* vbuf,
+                                             uint64_t* kbar, uint64_t* vbar, int b, int g, int L,
+                                             int tile) {
+  const int32_t k_rows_total = p.num_pages * p.Hkv * PAGE;  // first out-of-range row
+  const int32_t v_rows_total = p.num_pages * p.Hkv * HD;
+  int32_t krow[PAGES_PER_TILE], vrow[PAGES_PER_TILE];
+#pragma unroll
+  for (int i = 0; i < PAGES_PER_TILE; ++i) {
+    const int pidx = tile * PAGES_PER_TILE + i;
+    krow[i] = k_rows_total;  // out of range: TMA fills zeros
+    vrow[i] = v_rows_total;
+    if (pidx * PAGE < L && pidx < p.max_pages) {
+      const int32_t pid = p.block_table[(size_t)b * p.max_pages + pidx];
+      if (pid >= 0 && pid < p.num_pages) {
+        krow[i] = (pid * p.Hkv + g) * PAGE;
+        vrow[i] = (pid * p.Hkv + g) * HD;
+      } else {
+        set_status(p.status, BI_DEV_BAD_PAGE);
+      }
+    } else if (pidx * PAGE < L) {
+      set_status(p.status, BI_DEV_BAD_PAGE);
+    }
+  }
+  mbar_arrive_expect_tx(kbar, TILE_BYTES);
+#pragma unroll
+  for (int i = 0; i < PAGES_PER_TILE; ++i) {
+    tma_load_2d(kbuf + i * 2048, tmK, kbar, 0, krow[i]);
+    tma_load_2d(kbuf + 16384 + i * 2048, tmK, kbar, 64, krow[i]);
+  }
+  mbar_arrive_expect_tx(vbar, TILE_BYTES);
+#pragma unroll
+  for (int i = 0; i < PAGES_PER_TILE; ++i) tma_load_2d(vbuf + i * 4096, tmV, vbar, 0, vrow[i]);
+}
+
+__device__ __forceinline__ void issue_s(uint32_t tmem_s, uint32_t q_addr, uint32_t k_addr) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
+#pragma unroll
+  for (int kk = 0; kk < HD / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+    mma_bf16(tmem_s, smem_desc(q_addr + off, 16, 1024, 2), smem_desc(k_addr + off, 16, 1024, 2),
+             idesc, kk != 0);
+  }
+}
+
+__device__ __forceinline__ void issue_pv(uint32_t tmem_pv, uint32_t p_addr, uint32_t v_addr) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
+#pragma unroll
+  for (int j = 0; j < PAGES_PER_TILE; ++j) {
+    const uint32_t poff = (j >> 2) * 16384 + (j & 3) * 32;
+    // V^T page block j: [128 d rows x 16 keys], 32-byte rows, 32-byte swizzle,
+    // 8-row groups 256 bytes apart.
+    mma_bf16(tmem_pv, smem_desc(p_addr + poff, 16, 1024, 2),
+             smem_desc(v_addr + j * 4096, 16, 256, 6), idesc, j != 0);
+  }
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    attn_split_kernel(const __grid_constant__ CUtensorMap tmQ,
+                      const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const Params p) {
+  const int s = blockIdx.x;
+  const int b = blockIdx.y / p.qblocks;
+  const int jb = blockIdx.y % p.qblocks;
+  const int g = blockIdx.z;
+
+  // ---- which queries and keys this CTA covers (uniform across the CTA)
+  const int L = p.seq_lens[b];
+  int r0, nb;
+  if (p.cu_q) {
+    r0 = p.cu_q[b];
+    nb = p.cu_q[b + 1] - r0;
+  } else {
+    r0 = b;
+    nb = 1;
+  }
+  if (nb <= 0 || jb * p.QR >= nb) return;
+  if (L < nb || L > p.max_kv_len || r0 < 0 || r0 + nb > p.n_tok) {
+    if (threadIdx.x == 0 && s == 0 && g == 0) set_status(p.status, BI_DEV_BAD_SEQLEN);
+    return;
+  }
+  const int q_lo = jb * p.QR;
+  const int q_hi = min(nb, q_lo + p.QR);
+  const int p_last = L - nb + q_hi - 1;
+  const int key_lo = s * SPLIT;
+  if (key_lo > p_last) return;
+  const int key_hi = min((s + 1) * SPLIT, p_last + 1);  // exclusive
+  const int t0 = key_lo / TILE;
+  const int ntiles = (key_hi - 1) / TILE - t0 + 1;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* v_full = bars + 3;    // [2]
+  uint64_t* kv_empty = bars + 5;  // [2]
+  uint64_t* s_full = bars + 7;
+  uint64_t* p_ready = bars + 8;
+  uint64_t* o_full = bars + 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_ready, 128);
+    mbar_init(o_full, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_s = tmem;
+  const uint32_t tmem_pv = tmem + 128;
+  const uint32_t sQ = smem_u32(smem + OFF_Q);
+  const uint32_t sK[2] = {smem_u32(smem + OFF_K), smem_u32(smem + OFF_K + TILE_BYTES)};
+  const uint32_t sV[2] = {smem_u32(smem + OFF_V), smem_u32(smem + OFF_V + TILE_BYTES)};
+  const uint32_t sP = smem_u32(smem + OFF_P);
+
+  if (warp == 4) {
+    // ------------------------------------------------ TMA + MMA control thread
+    if (lane == 0) {
+      bool ok = true;
+      const uint32_t q_bytes = 2u * 64u * 2u * (uint32_t)(p.G * p.q_box);
+      mbar_arrive_expect_tx(q_full, q_bytes);
+      tma_load_3d(smem + OFF_Q, &tmQ, q_full, 0, g * p.G, r0 + q_lo);
+      tma_load_3d(smem + OFF_Q + 16384, &tmQ, q_full, 64, g * p.G, r0 + q_lo);
+      load_kv_tile(p, &tmK, &tmV, smem + OFF_K, smem + OFF_V, &k_full[0], &v_full[0], b, g, L, t0);
+      if (ntiles > 1)
+        load_kv_tile(p, &tmK, &tmV, smem + OFF_K + TILE_BYTES, smem + OFF_V + TILE_BYTES,
+                     &k_full[1], &v_full[1], b, g, L, t0 + 1);
+      ok = mbar_wait(q_full, 0, p.status, abort_flag) &&
+           mbar_wait(&k_full[0], 0, p.status, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(tmem_s, sQ, sK[0]);
+        mma_commit(s_full);
+      }
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const int buf = i & 1;
+        const uint32_t use_par = (uint32_t)(i >> 1) & 1u;
+        if (!mbar_wait(p_ready, (uint32_t)i & 1u, p.status, abort_flag)) break;
+        if (!mbar_wait(&v_full[buf], use_par, p.status, abort_flag)) break;
+        tc_fence_after();
+        issue_pv(tmem_pv, sP, sV[buf]);
+        mma_commit(o_full);
+        mma_commit(&kv_empty[buf]);
+        if (i + 1 < ntiles) {
+          const int nbuf = buf ^ 1;
+          if (!mbar_wait(&k_full[nbuf], (uint32_t)((i + 1) >> 1) & 1u, p.status, abort_flag)) break;
+          tc_fence_after();
+          issue_s(tmem_s, sQ, sK[nbuf]);
+          mma_commit(s_full);
+        }
+        if (i + 2 < ntiles) {
+          if (!mbar_wait(&kv_empty[buf], use_par, p.status, abort_flag)) break;
+          load_kv_tile(p, &tmK, &tmV, smem + OFF_K + buf * TILE_BYTES,
+                       smem + OFF_V + buf * TILE_BYTES, &k_full[buf], &v_full[buf], b, g, L,
+                       t0 + i + 2);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------ one thread per MMA row
+    const int r = threadIdx.x;  // 0..127 == TMEM lane
+    const int qi = r / p.G;
+    const int hj = r - qi * p.G;
+    const int q_idx = q_lo + qi;
+    const int pos = L - nb + q_idx;
+    const bool row_active = (q_idx < q_hi) && (pos >= key_lo);
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    // partial last page: slots >= L of the page holding key L-1 are zeroed in V
+    const int last_page = (L - 1) / PAGE;
+    const int tail = L % PAGE;
+
+    float m = -INFINITY, l = 0.0f;
+    float O[HD];
+#pragma unroll
+    for (int d = 0; d < HD; ++d) O[d] = 0.0f;
+
+    for (int i = 0; i < ntiles; ++i) {
+      const int buf = i & 1;
+      const int kb = (t0 + i) * TILE;
+      const bool need = row_active && kb <= pos;
+      const bool warp_need = __any_sync(0xffffffffu, need);
+      float alpha = 1.0f;
+      if (!mbar_wait(s_full, (uint32_t)i & 1u, p.status, abort_flag)) break;
+      tc_fence_after();
+      if (warp_need) {
+        const int nvalid = need ? min(TILE, pos + 1 - kb) : 0;
+        float m_tile = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t rr[32];
+          tmem_ld32(tmem_s + lane_off + q * 32, rr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (q * 32 + c < nvalid) m_tile = fmaxf(m_tile, __fmul_rn(__uint_as_float(rr[c]), p.scale_log2));
+        }
+        const float m_new = need ? fmaxf(m, m_tile) : 0.0f;
+        if (need) alpha = exp2f(__fsub_rn(m, m_new));
+        float lsum = 0.0f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t rr[32];
+          tmem_ld32(tmem_s + lane_off + q * 32, rr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float pf[2];
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int c = q * 32 + c8 * 8 + e * 2 + h;
+                const float sv = __fmul_rn(__uint_as_float(rr[c8 * 8 + e * 2 + h]), p.scale_log2);
+                const float ev = (c < nvalid) ? exp2f(__fsub_rn(sv, m_new)) : 0.0f;
+                const bf16 pb = __float2bfloat16_rn(ev);
+                pf[h] = __bfloat162float(pb);
+                lsum = __fadd_rn(lsum, pf[h]);
+              }
+              pk[e] = pack_bf16x2(pf[0], pf[1]);  // exact: pf are bf16 values
+            }
+            // key chunk (8 keys) index 0..15 -> half, 16-byte slot, swizzled by row
+            const int chunk = q * 4 + c8;
+            const uint32_t addr = (uint32_t)(chunk >> 3) * 16384u + (uint32_t)r * 128u +
+                                  (uint32_t)(((chunk & 7) ^ (r & 7)) << 4);
+            *reinterpret_cast<uint4*>(smem + OFF_P + addr) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+        if (need) {
+          l = __fadd_rn(__fmul_rn(alpha, l), lsum);
+          m = m_new;
+        }
+      }
+      // zero V slots at or past the sequence end inside this tile's last page
+      if (tail != 0 && last_page / PAGES_PER_TILE == t0 + i) {
+        if (!mbar_wait(&v_full[buf], (uint32_t)(i >> 1) & 1u, p.status, abort_flag)) break;
+        uint8_t* vblk = smem + OFF_V + buf * TILE_BYTES + (last_page % PAGES_PER_TILE) * 4096;
+        const int d = r;  // V^T row
+        for (int slot = tail; slot < PAGE; ++slot) {
+          const uint32_t off = (uint32_t)d * 32u + ((uint32_t)((slot >> 3) ^ ((d >> 2) & 1)) << 4) +
+                               (uint32_t)(slot & 7) * 2u;
+          *reinterpret_cast<uint16_t*>(vblk + off) = 0;
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_ready);
+      if (!mbar_wait(o_full, (uint32_t)i & 1u, p.status, abort_flag)) break;
+      tc_fence_after();
+      if (warp_need) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t rr[32];
+          tmem_ld32(tmem_pv + lane_off + q * 32, rr);
+          tmem_ld_wait();
+          if (need) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) O[q * 32 + c] = __fmaf_rn(alpha, O[q * 32 + c], __uint_as_float(rr[c]));
+          }
+        }
+      }
+    }
+    if (row_active && !*abort_flag) {
+      const size_t idx = ((size_t)(r0 + q_idx) * p.Hq + (size_t)(g * p.G + hj)) * p.n_split_max + s;
+      float4* dst = reinterpret_cast<float4*>(p.ws_o + idx * HD);
+#pragma unroll
+      for (int d4 = 0; d4 < HD / 4; ++d4)
+        dst[d4] = make_float4(O[4 * d4], O[4 * d4 + 1], O[4 * d4 + 2], O[4 * d4 + 3]);
+      *reinterpret_cast<float2*>(p.ws_ml + idx * 2) = make_float2(m, l);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 4) {
+    __syncwarp();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// Finishing pass: one warp per (query token, q head); lane owns 4 of the 128
+// output elements. Splits merged strictly in order s = 0 .. n-1.
+struct CombineParams {
+  const float* ws_o;
+  const float* ws_ml;
+  const int32_t* seq_lens;
+  const int32_t* cu_q;  // null: decode
+  bf16* out;
+  int64_t ldo;
+  int32_t n_tok, B, Hq, n_split_max, max_kv_len;
+};
+
+__global__ void attn_combine_kernel(const CombineParams p) {
+  const int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (wid >= (int64_t)p.n_tok * p.Hq) return;
+  const int tok = (int)(wid / p.Hq);
+  const int h = (int)(wid % p.Hq);
+  int b, nb, qidx;
+  if (p.cu_q) {
+    int lo = 0, hi = p.B;  // find b with cu_q[b] <= tok < cu_q[b+1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (p.cu_q[mid] <= tok) lo = mid; else hi = mid;
+    }
+    b = lo;
+    nb = p.cu_q[b + 1] - p.cu_q[b];
+    qidx = tok - p.cu_q[b];
+    if (p.cu_q[b] < 0 || p.cu_q[b + 1] > p.n_tok) nb = 0;  // malformed cu_q: zeros
+  } else {
+    b = tok;
+    nb = 1;
+    qidx = 0;
+  }
+  const int L = p.seq_lens[b];
+  bf16* dst = p.out + (size_t)tok * p.ldo + (size_t)h * HD + lane * 4;
+  if (L < nb || L > p.max_kv_len || nb <= 0) {  // flagged by the split kernel; write zeros
+    *reinterpret_cast<uint2*>(dst) = make_uint2(0u, 0u);
+    return;
+  }
+  const int pos = L - nb + qidx;
+  const int n = pos / SPLIT + 1;
+  const size_t base = ((size_t)tok * p.Hq + h) * p.n_split_max;
+  float M = -INFINITY;
+  for (int s = 0; s < n; ++s) M = fmaxf(M, p.ws_ml[(base + s) * 2]);
+  float Lsum = 0.0f;
+  float o0 = 0.0f, o1 = 0.0f, o2 = 0.0f, o3 = 0.0f;
+  for (int s = 0; s < n; ++s) {
+    const float2 ml = *reinterpret_cast<const float2*>(p.ws_ml + (base + s) * 2);
+    const float w = exp2f(__fsub_rn(ml.x, M));
+    Lsum = __fmaf_rn(w, ml.y, Lsum);
+    const float4 o = *reinterpret_cast<const float4*>(p.ws_o + (base + s) * HD + lane * 4);
+    o0 = __fmaf_rn(w, o.x, o0);
+    o1 = __fmaf_rn(w, o.y, o1);
+    o2 = __fmaf_rn(w, o.z, o2);
+    o3 = __fmaf_rn(w, o.w, o3);
+  }
+  // + 0.0f turns a -0 into +0, so a zero's sign cannot depend on the split path
+  const float y0 = __fadd_rn(__fdiv_rn(o0, Lsum), 0.0f), y1 = __fadd_rn(__fdiv_rn(o1, Lsum), 0.0f);
+  const float y2 = __fadd_rn(__fdiv_rn(o2, Lsum), 0.0f), y3 = __fadd_rn(__fdiv_rn(o3, Lsum), 0.0f);
+  *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(y0, y1), pack_bf16x2(y2, y3));
+}
+
+static size_t ws_bytes_for(int64_t n_tok, int Hq, int n_split) {
+  const size_t o = (size_t)n_tok * Hq * n_split * HD * sizeof(float);
+  const size_t ml = (size_t)n_tok * Hq * n_split * 2 * sizeof(float);
+  return o + ml;
+}
+
+static bi_status check_shape(const bi_attn_shape* sh) {
+  if (!sh) return fail(BI_ERR_INVALID_ARG, "attention: shape is null");
+  if (sh->head_dim != HD) return fail(BI_ERR_SHAPE, "attention: head_dim must be %d", HD);
+  if (sh->page_size != PAGE) return fail(BI_ERR_SHAPE, "attention: page_size must be %d", PAGE);
+  if (sh->num_q_heads <= 0 || sh->num_kv_heads <= 0 || sh->num_q_heads % sh->num_kv_heads)
+    return fail(BI_ERR_SHAPE, "attention: num_q_heads must be a positive multiple of num_kv_heads");
+  const int G = sh->num_q_heads / sh->num_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return fail(BI_ERR_SHAPE, "attention: q heads per kv head must be 1, 2, 4 or 8 (got %d)", G);
+  if (sh->num_pages <= 0 || sh->max_pages_per_seq <= 0 || sh->max_kv_len <= 0)
+    return fail(BI_ERR_SHAPE, "attention: num_pages, max_pages_per_seq and max_kv_len must be positive");
+  if ((int64_t)sh->num_pages * sh->num_kv_heads * HD > 0x7fffffffll)
+    return fail(BI_ERR_SHAPE, "attention: cache too large for 32-bit TMA coordinates");
+  if (!(sh->scale > 0.0f)) return fail(BI_ERR_INVALID_ARG, "attention: scale must be > 0");
+  return BI_OK;
+}
+
+static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t max_q_len,
+                     int64_t n_tok, const void* k_cache, const void* v_cache,
+                     const int32_t* block_table, const int32_t* seq_lens, int32_t B,
+                     const bi_attn_shape* sh, void* out, int64_t ldo, void* ws, size_t ws_bytes,
+                     cudaStream_t stream) {
+  bi_status st = check_shape(sh);
+  if (st != BI_OK) return st;
+  if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !out)
+    return fail(BI_ERR_INVALID_ARG, "attention: null pointer");
+  if (B < 0 || n_tok < 0 || max_q_len < 0) return fail(BI_ERR_INVALID_ARG, "attention: negative size");
+  const int Hq = sh->num_q_heads, G = sh->num_q_heads / sh->num_kv_heads;
+  if (ldq < (int64_t)Hq * HD || ldo < (int64_t)Hq * HD) return fail(BI_ERR_SHAPE, "attention: ldq/ldo smaller than num_q_heads*128");
+  if (ldq % 8 || ldo % 8) return fail(BI_ERR_ALIGN, "attention: ldq and ldo must be multiples of 8");
+  if (!aligned16(q) || !aligned16(out) || !aligned16(k_cache) || !aligned16(v_cache) || (ws && !aligned16(ws)))
+    return fail(BI_ERR_ALIGN, "attention: pointers must be 16-byte aligned");
+  if (B == 0 || n_tok == 0) return BI_OK;
+  const int n_split = (sh->max_kv_len + SPLIT - 1) / SPLIT;
+  const int QR = 128 / G;
+  const int qblocks = cu_q ? (max_q_len + QR - 1) / QR : 1;
+  if (cu_q && max_q_len <= 0) return fail(BI_ERR_SHAPE, "attention: max_q_len must be positive");
+  if ((int64_t)B * qblocks > 65535) return fail(BI_ERR_SHAPE, "attention: B * ceil(max_q_len / %d) above 65535", QR);
+  if (n_split > 65535) return fail(BI_ERR_SHAPE, "attention: max_kv_len too large");
+  if (n_tok > 0x7fffffffll / Hq) return fail(BI_ERR_SHAPE, "attention: too many tokens");
+  const size_t need = ws_bytes_for(n_tok, Hq, n_split);
+  if (!ws || ws_bytes < need) return fail(BI_ERR_WORKSPACE, "attention: workspace %zu bytes < %zu needed", ws_bytes, need);
+  if ((st = require_sm100()) != BI_OK) return st;
+
+  CUtensorMap tmQ, tmK, tmV;
+  {
+    uint64_t dims[3] = {(uint64_t)HD, (uint64_t)Hq, (uint64_t)n_tok};
+    uint64_t strides[2] = {(uint64_t)HD * 2, (uint64_t)ldq * 2};
+    uint32_t box[3] = {64, (uint32_t)G, cu_q ? (uint32_t)QR : 1u};
+    if ((st = encode_tmap(&tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims,
+                          strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != BI_OK)
+      return st;
+  }
+  {
+    uint64_t dims[2] = {(uint64_t)HD, (uint64_t)sh->num_pages * sh->num_kv_heads * PAGE};
+    uint64_t strides[1] = {(uint64_t)HD * 2};
+    uint32_t box[2] = {64, (uint32_t)PAGE};
+    if ((st = encode_tmap(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(k_cache),
+                          dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != BI_OK)
+      return st;
+  }
+  {
+    uint64_t dims[2] = {(uint64_t)PAGE, (uint64_t)sh->num_pages * sh->num_kv_heads * HD};
+    uint64_t strides[1] = {(uint64_t)PAGE * 2};
+    uint32_t box[2] = {(uint32_t)PAGE, (uint32_t)HD};
+    if ((st = encode_tmap(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(v_cache),
+                          dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B)) != BI_OK)
+      return st;
+  }
+  Params p;
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.cu_q = cu_q;
+  p.ws_o = static_cast<float*>(ws);
+  p.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + (size_t)n_tok * Hq * n_split * HD * sizeof(float));
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = sh->num_kv_heads;
+  p.G = G;
+  p.QR = QR;
+  p.qblocks = qblocks;
+  p.q_box = cu_q ? QR : 1;
+  p.n_tok = (int32_t)n_tok;
+  p.num_pages = sh->num_pages;
+  p.max_pages = sh->max_pages_per_seq;
+  p.max_kv_len = sh->max_kv_len;
+  p.n_split_max = n_split;
+  p.scale_log2 = (float)((double)sh->scale * 1.4426950408889634);  // scale * log2(e)
+  p.status = status_word();
+
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!attr_set[dev & 63]) {
+    cudaError_t e = cudaFuncSetAttribute(attn_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e, "attention: smem attribute");
+    attr_set[dev & 63] = true;
+  }
+  dim3 grid(n_split, B * qblocks, sh->num_kv_heads);
+  attn_split_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
+  BI_CHECK_LAUNCH("attention split launch");
+
+  CombineParams c;
+  c.ws_o = p.ws_o;
+  c.ws_ml = p.ws_ml;
+  c.seq_lens = seq_lens;
+  c.cu_q = cu_q;
+  c.out = static_cast<bf16*>(out);
+  c.ldo = ldo;
+  c.n_tok = (int32_t)n_tok;
+  c.B = B;
+  c.Hq = Hq;
+  c.n_split_max = n_split;
+  c.max_kv_len = sh->max_kv_len;
+  const int64_t warps = n_tok * Hq;
+  const int blocks = (int)((warps + 7) / 8);
+  attn_combine_kernel<<<blocks, 256, 0, stream>>>(c);
+  BI_CHECK_LAUNCH("attention combine launch");
+  return BI_OK;
+}
+
+}  // namespace attn
+}  // namespace bi
+
+using namespace bi;
+
+extern "C" bi_status bi_attn_workspace_size(const bi_attn_shape* shape, int64_t max_tokens,
+                                            size_t* bytes) {
+  bi_status st = attn::check_shape(shape);
+  if (st != BI_OK) return st;
+  if (!bytes || max_tokens < 0) return fail(BI_ERR_INVALID_ARG, "attn_workspace_size: bad arguments");
+  const int n_split = (shape->max_kv_len + attn::SPLIT - 1) / attn::SPLIT;
+  *bytes = attn::ws_bytes_for(max_tokens, shape->num_q_heads, n_split);
+  return BI_OK;
+}
+
+extern "C" bi_status bi_attn_decode(const void* q, int64_t ldq, const void* k_cache,
+                                    const void* v_cache, const int32_t* block_table,
+                                    const int32_t* seq_lens, int32_t B, const bi_attn_shape* shape,
+                                    void* out, int64_t ldo, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  return attn::run(q, ldq, nullptr, 1, B, k_cache, v_cache, block_table, seq_lens, B, shape, out,
+                   ldo, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" bi_status bi_attn_prefill(const void* q, int64_t ldq, const int32_t* cu_q,
+                                     int32_t max_q_len, int64_t n_tok, const void* k_cache,
+                                     const void* v_cache, const int32_t* block_table,
+                                     const int32_t* seq_lens, int32_t B,
+                                     const bi_attn_shape* shape, void* out, int64_t ldo, void* ws,
+                                     size_t ws_bytes, void* stream) {
+  if (!cu_q) return fail(BI_ERR_INVALID_ARG, "attn_prefill: cu_q is null");
+  return attn::run(q, ldq, cu_q, max_q_len, n_tok, k_cache, v_cache, block_table, seq_lens, B,
+                   shape, out, ldo, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}

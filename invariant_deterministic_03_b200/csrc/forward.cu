@@ -1,0 +1,230 @@
+// forward.cu -- one step of a dense pre-norm decoder, composed only of the
+// batch-invariant kernels of this library.
+//
+// Per layer: RMSNorm -> QKV GEMM -> RoPE(q, k) -> KV-cache append -> paged
+// attention (split + ordered merge) -> O GEMM (fp32 out) -> residual add ->
+// RMSNorm -> gate/up GEMM -> SwiGLU -> down GEMM (fp32 out) -> residual add.
+// Then the final RMSNorm of the rows that want logits and the LM-head GEMM
+// with fp32 logits, and optionally the greedy argmax.
+//
+// Every kernel computes each row (token) with an order that depends only on
+// that row's data and, for attention, on its sequence's cache, so a
+// sequence's logits are the same bits whatever else shares the step
+// ("Defeating Nondeterminism in LLM Inference", sections "Batch invariance and
+// determinism" and "How do we make kernels batch-invariant?"). The residual
+// stream is kept in fp32 and the two GEMMs that feed it write fp32 (a reading:
+// the pages fix no activation precision; this keeps the stream's rounding
+// error below the bf16 inputs').
+#include <stdlib.h>
+
+#include "common.cuh"
+#include "host.h"
+
+namespace bi {
+bi_status launch_kv_append(const bf16* k, const bf16* v, int64_t ld_new, const int32_t* slots,
+                           int64_t n_tok, bf16* kc, bf16* vc, int Hkv, int num_pages,
+                           cudaStream_t s);
+bi_status launch_embed(const int32_t* tok, int64_t n_tok, const bf16* table, int64_t vocab,
+                       int64_t D, float* out, cudaStream_t s);
+bi_status launch_rope(bf16* x, int64_t ldx, int n_heads, const int32_t* pos, int64_t n_tok,
+                      const float* cs, int max_pos, cudaStream_t s);
+bi_status launch_swiglu(const bf16* gu, int64_t n_tok, int64_t F, bf16* out, cudaStream_t s);
+bi_status launch_argmax(const float* logits, int64_t rows, int64_t V, int64_t ld, int32_t* idx,
+                        cudaStream_t s);
+
+namespace fwd {
+
+__global__ void add_f32_kernel(float* __restrict__ x, const float* __restrict__ d, int64_t n) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) x[i] = __fadd_rn(x[i], d[i]);
+}
+
+__global__ void gather_rows_kernel(const float* __restrict__ x, const int32_t* __restrict__ rows,
+                                   int64_t n_rows, int64_t n_tok, int D, float* __restrict__ out,
+                                   int32_t* status) {
+  const int64_t r = blockIdx.x;
+  const int32_t src = rows[r];
+  const bool ok = src >= 0 && src < n_tok;
+  if (!ok && threadIdx.x == 0) set_status(status, BI_DEV_BAD_TOKEN);
+  for (int c = threadIdx.x; c < D; c += blockDim.x)
+    out[r * D + c] = ok ? x[(size_t)src * D + c] : 0.0f;
+}
+
+struct Layout {  // workspace carve-up, all offsets 256-byte aligned
+  size_t x, h, qkv, att, t32, gu, act, xl, hl, rope, attn_ws, total;
+  size_t attn_ws_bytes;
+};
+
+static size_t up(size_t v) { return (v + 255) & ~(size_t)255; }
+
+static Layout layout(const bi_model_config& c, int64_t T, int64_t NL, int32_t max_kv_len) {
+  Layout L;
+  const size_t D = c.d_model, F = c.d_ff;
+  const size_t QKV = (size_t)(c.n_q_heads + 2 * c.n_kv_heads) * BI_HEAD_DIM;
+  size_t o = 0;
+  L.x = o; o += up(T * D * 4);
+  L.h = o; o += up(T * D * 2);
+  L.qkv = o; o += up(T * QKV * 2);
+  L.att = o; o += up(T * D * 2);
+  L.t32 = o; o += up(T * D * 4);
+  L.gu = o; o += up(T * 2 * F * 2);
+  L.act = o; o += up(T * F * 2);
+  L.xl = o; o += up(NL * D * 4);
+  L.hl = o; o += up(NL * D * 2);
+  L.rope = o; o += up((size_t)c.max_pos * 64 * 2 * 4);
+  bi_attn_shape sh;
+  sh.num_q_heads = c.n_q_heads;
+  sh.num_kv_heads = c.n_kv_heads;
+  sh.head_dim = BI_HEAD_DIM;
+  sh.page_size = BI_PAGE_SIZE;
+  sh.num_pages = 1;
+  sh.max_pages_per_seq = 1;
+  sh.max_kv_len = max_kv_len > 0 ? max_kv_len : 1;
+  sh.scale = 1.0f;
+  size_t a = 0;
+  bi_attn_workspace_size(&sh, T, &a);
+  L.attn_ws = o; o += up(a);
+  L.attn_ws_bytes = a;
+  L.total = o;
+  return L;
+}
+
+}  // namespace fwd
+}  // namespace bi
+
+struct bi_model {
+  bi_model_config cfg;
+  bi_model_weights w;
+};
+
+using namespace bi;
+
+extern "C" bi_status bi_model_create(const bi_model_config* cfg, const bi_model_weights* w,
+                                     bi_model** out) {
+  if (!cfg || !w || !out) return fail(BI_ERR_INVALID_ARG, "model_create: null argument");
+  const bi_model_config& c = *cfg;
+  if (c.n_layers < 0 || c.d_model <= 0 || c.n_q_heads <= 0 || c.n_kv_heads <= 0 || c.d_ff <= 0 ||
+      c.vocab <= 0 || c.max_pos <= 0)
+    return fail(BI_ERR_INVALID_ARG, "model_create: sizes must be positive");
+  if (c.d_model != c.n_q_heads * BI_HEAD_DIM) return fail(BI_ERR_SHAPE, "model_create: d_model must equal n_q_heads * 128");
+  if (c.n_q_heads % c.n_kv_heads) return fail(BI_ERR_SHAPE, "model_create: n_q_heads must be a multiple of n_kv_heads");
+  const int G = c.n_q_heads / c.n_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return fail(BI_ERR_SHAPE, "model_create: q heads per kv head must be 1, 2, 4 or 8");
+  if (c.d_ff % 8 || c.vocab % 8) return fail(BI_ERR_SHAPE, "model_create: d_ff and vocab must be multiples of 8");
+  if (!(c.rms_eps >= 0.0f) || !(c.rope_theta > 1.0)) return fail(BI_ERR_INVALID_ARG, "model_create: bad eps or rope_theta");
+  if (!w->embed || !w->final_norm || !w->lm_head) return fail(BI_ERR_INVALID_ARG, "model_create: missing weights");
+  if (c.n_layers > 0 && (!w->attn_norm || !w->w_qkv || !w->w_o || !w->mlp_norm || !w->w_gate_up || !w->w_down))
+    return fail(BI_ERR_INVALID_ARG, "model_create: missing layer weights");
+  bi_model* m = static_cast<bi_model*>(malloc(sizeof(bi_model)));
+  if (!m) return fail(BI_ERR_INVALID_ARG, "model_create: out of host memory");
+  m->cfg = c;
+  m->w = *w;
+  *out = m;
+  return BI_OK;
+}
+
+extern "C" void bi_model_destroy(bi_model* m) { free(m); }
+
+extern "C" bi_status bi_forward_workspace_size(const bi_model* m, int64_t max_tokens,
+                                               int64_t max_logits, int32_t max_kv_len,
+                                               size_t* bytes) {
+  if (!m || !bytes || max_tokens < 0 || max_logits < 0 || max_kv_len <= 0)
+    return fail(BI_ERR_INVALID_ARG, "forward_workspace_size: bad arguments");
+  *bytes = fwd::layout(m->cfg, max_tokens, max_logits, max_kv_len).total;
+  return BI_OK;
+}
+
+#define BI_TRY(expr)                     \
+  do {                                   \
+    bi_status st_ = (expr);              \
+    if (st_ != BI_OK) return st_;        \
+  } while (0)
+
+extern "C" bi_status bi_forward(const bi_model* m, const bi_batch* bt, void* k_cache,
+                                void* v_cache, int32_t num_pages, float* logits,
+                                int32_t* next_tokens, void* ws, size_t ws_bytes, void* stream) {
+  if (!m || !bt || !k_cache || !v_cache || !logits || !ws) return fail(BI_ERR_INVALID_ARG, "forward: null argument");
+  const bi_model_config& c = m->cfg;
+  const bi_batch& b = *bt;
+  if (b.n_tok <= 0 || b.B <= 0 || b.n_logits < 0 || b.max_q_len <= 0 || b.max_kv_len <= 0 || b.max_pages_per_seq <= 0 || num_pages <= 0)
+    return fail(BI_ERR_INVALID_ARG, "forward: bad batch sizes");
+  if (!b.tokens || !b.positions || !b.slot_mapping || !b.cu_q || !b.seq_lens || !b.block_table || (b.n_logits && !b.logits_rows))
+    return fail(BI_ERR_INVALID_ARG, "forward: null batch array");
+  if (b.max_kv_len > c.max_pos) return fail(BI_ERR_SHAPE, "forward: max_kv_len above max_pos");
+  const fwd::Layout L = fwd::layout(c, b.n_tok, b.n_logits, b.max_kv_len);
+  if (ws_bytes < L.total) return fail(BI_ERR_WORKSPACE, "forward: workspace %zu < %zu", ws_bytes, L.total);
+  if (!aligned16(ws) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(logits))
+    return fail(BI_ERR_ALIGN, "forward: pointers must be 16-byte aligned");
+  BI_TRY(require_sm100());
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  float* x = reinterpret_cast<float*>(base + L.x);
+  bf16* h = reinterpret_cast<bf16*>(base + L.h);
+  bf16* qkv = reinterpret_cast<bf16*>(base + L.qkv);
+  bf16* att = reinterpret_cast<bf16*>(base + L.att);
+  float* t32 = reinterpret_cast<float*>(base + L.t32);
+  bf16* gu = reinterpret_cast<bf16*>(base + L.gu);
+  bf16* act = reinterpret_cast<bf16*>(base + L.act);
+  float* xl = reinterpret_cast<float*>(base + L.xl);
+  bf16* hl = reinterpret_cast<bf16*>(base + L.hl);
+  float* rope = reinterpret_cast<float*>(base + L.rope);
+  void* attn_ws = base + L.attn_ws;
+
+  const int64_t T = b.n_tok, D = c.d_model, F = c.d_ff;
+  const int Hq = c.n_q_heads, Hkv = c.n_kv_heads;
+  const int64_t QKV = (int64_t)(Hq + 2 * Hkv) * BI_HEAD_DIM;
+  const size_t cache_layer = (size_t)num_pages * Hkv * BI_PAGE_SIZE * BI_HEAD_DIM;
+  const bf16* W = nullptr;
+  (void)W;
+
+  BI_TRY(bi_rope_table(rope, c.max_pos, c.rope_theta, stream));
+  BI_TRY(launch_embed(b.tokens, T, static_cast<const bf16*>(m->w.embed), c.vocab, D, x, s));
+
+  bi_attn_shape sh;
+  sh.num_q_heads = Hq;
+  sh.num_kv_heads = Hkv;
+  sh.head_dim = BI_HEAD_DIM;
+  sh.page_size = BI_PAGE_SIZE;
+  sh.num_pages = num_pages;
+  sh.max_pages_per_seq = b.max_pages_per_seq;
+  sh.max_kv_len = b.max_kv_len;
+  sh.scale = (float)(1.0 / sqrt((double)BI_HEAD_DIM));
+
+  const int64_t add_blocks = (T * D + 255) / 256;
+  for (int l = 0; l < c.n_layers; ++l) {
+    const bf16* attn_norm = static_cast<const bf16*>(m->w.attn_norm) + (size_t)l * D;
+    const bf16* mlp_norm = static_cast<const bf16*>(m->w.mlp_norm) + (size_t)l * D;
+    const bf16* w_qkv = static_cast<const bf16*>(m->w.w_qkv) + (size_t)l * QKV * D;
+    const bf16* w_o = static_cast<const bf16*>(m->w.w_o) + (size_t)l * D * D;
+    const bf16* w_gu = static_cast<const bf16*>(m->w.w_gate_up) + (size_t)l * 2 * F * D;
+    const bf16* w_d = static_cast<const bf16*>(m->w.w_down) + (size_t)l * D * F;
+    bf16* kc = static_cast<bf16*>(k_cache) + (size_t)l * cache_layer;
+    bf16* vc = static_cast<bf16*>(v_cache) + (size_t)l * cache_layer;
+
+    BI_TRY(bi_rmsnorm_f32in(x, attn_norm, h, T, D, c.rms_eps, stream));
+    BI_TRY(bi_gemm(h, D, w_qkv, D, qkv, QKV, BI_BF16, T, QKV, D, stream));
+    BI_TRY(launch_rope(qkv, QKV, Hq, b.positions, T, rope, c.max_pos, s));
+    BI_TRY(launch_rope(qkv + (size_t)Hq * BI_HEAD_DIM, QKV, Hkv, b.positions, T, rope, c.max_pos, s));
+    BI_TRY(launch_kv_append(qkv + (size_t)Hq * BI_HEAD_DIM, qkv + (size_t)(Hq + Hkv) * BI_HEAD_DIM,
+                            QKV, b.slot_mapping, T, kc, vc, Hkv, num_pages, s));
+    BI_TRY(bi_attn_prefill(qkv, QKV, b.cu_q, b.max_q_len, T, kc, vc, b.block_table, b.seq_lens,
+                           b.B, &sh, att, D, attn_ws, L.attn_ws_bytes, stream));
+    BI_TRY(bi_gemm(att, D, w_o, D, t32, D, BI_F32, T, D, D, stream));
+    fwd::add_f32_kernel<<<(unsigned)add_blocks, 256, 0, s>>>(x, t32, T * D);
+    BI_CHECK_LAUNCH("forward residual");
+    BI_TRY(bi_rmsnorm_f32in(x, mlp_norm, h, T, D, c.rms_eps, stream));
+    BI_TRY(bi_gemm(h, D, w_gu, D, gu, 2 * F, BI_BF16, T, 2 * F, D, stream));
+    BI_TRY(launch_swiglu(gu, T, F, act, s));
+    BI_TRY(bi_gemm(act, F, w_d, F, t32, D, BI_F32, T, D, F, stream));
+    fwd::add_f32_kernel<<<(unsigned)add_blocks, 256, 0, s>>>(x, t32, T * D);
+    BI_CHECK_LAUNCH("forward residual");
+  }
+  if (b.n_logits == 0) return BI_OK;
+  fwd::gather_rows_kernel<<<(unsigned)b.n_logits, 256, 0, s>>>(x, b.logits_rows, b.n_logits, T,
+                                                               (int)D, xl, status_word());
+  BI_CHECK_LAUNCH("forward gather");
+  BI_TRY(bi_rmsnorm_f32in(xl, m->w.final_norm, hl, b.n_logits, D, c.rms_eps, stream));
+  BI_TRY(bi_gemm(hl, D, m->w.lm_head, D, logits, c.vocab, BI_F32, b.n_logits, c.vocab, D, stream));
+  if (next_tokens) BI_TRY(launch_argmax(logits, b.n_logits, c.vocab, c.vocab, next_tokens, s));
+  return BI_OK;
+}

@@ -1,0 +1,307 @@
+// gemm.cu -- batch-invariant GEMM on the 5th-generation tensor cores.
+//
+// "Defeating Nondeterminism in LLM Inference", section "Batch-invariant
+// matmul": tile the OUTPUT and keep each element's whole K reduction inside
+// one core; never split K (split-K) nor hand different K ranges of a tile to
+// different cores (stream-K); and compile ONE kernel configuration for every
+// shape, because different tensor-core instructions may reduce in different
+// internal orders.
+//
+// The one configuration (for every M, N, K):
+//   output tile 128 x 256, K stage 64, instruction tcgen05.mma.cta_group::1
+//   .kind::f16 M=128 N=256 K=16 with bf16 operands and an fp32 accumulator in
+//   tensor memory. Element (m, n) is accumulated by the K-steps k = 0, 16, 32,
+//   ... in that order, in one CTA, whatever M and N are. Which CTA computes a
+//   tile (persistent round-robin) changes timing only, never arithmetic.
+//
+// CTA layout (192 threads, one CTA per SM, persistent over tiles):
+//   warp 0      TMA producer: A [128 x 64] and W [256 x 64] tiles, 128-byte
+//               swizzle, into a 4-stage shared-memory ring (mbarrier full/empty)
+//   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators);
+//               lane 0 issues the MMAs and tcgen05.commit's
+//   warps 2..5  epilogue: tcgen05.ld the accumulator row by row (thread = row),
+//               round to bf16 (RNE) or keep fp32, store to global; then free
+//               the accumulator for the tile after next.
+// Every mbarrier wait is bounded (see common.cuh); a timeout sets a status
+// bit and the CTA winds down, releasing its tensor memory.
+#include "common.cuh"
+#include "host.h"
+
+namespace bi {
+namespace gemm {
+
+constexpr int BM = BI_GEMM_BM;  // 128
+constexpr int BN = BI_GEMM_BN;  // 256
+constexpr int BK = BI_GEMM_BK;  // 64 bf16 = 128 bytes = one swizzle row
+constexpr int STAGES = 4;
+constexpr int UMMA_K = 16;
+constexpr uint32_t A_BYTES = BM * BK * 2;  // 16 KB
+constexpr uint32_t B_BYTES = BN * BK * 2;  // 32 KB
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int THREADS = 192;
+constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 256 /*barriers*/;
+
+struct Params {
+  void* C;
+  int64_t ldc;
+  int32_t c_f32;
+  int32_t M, N, K;
+  int32_t m_blocks, n_blocks, k_blocks;
+  int32_t* status;
+};
+
+__device__ __forceinline__ void store_row_chunk(const Params& p, int row, int col0,
+                                                const uint32_t (&r)[32]) {
+  // 32 consecutive columns col0 .. col0+31 of one row; N % 8 == 0, so each
+  // group of 8 columns is either fully inside or fully outside.
+  if (p.c_f32) {
+    float* dst = static_cast<float*>(p.C) + (size_t)row * p.ldc + col0;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      if (col0 + g * 8 < p.N) {
+        float4 a = make_float4(__uint_as_float(r[8 * g + 0]), __uint_as_float(r[8 * g + 1]),
+                               __uint_as_float(r[8 * g + 2]), __uint_as_float(r[8 * g + 3]));
+        float4 b = make_float4(__uint_as_float(r[8 * g + 4]), __uint_as_float(r[8 * g + 5]),
+                               __uint_as_float(r[8 * g + 6]), __uint_as_float(r[8 * g + 7]));
+        *reinterpret_cast<float4*>(dst + 8 * g) = a;
+        *reinterpret_cast<float4*>(dst + 8 * g + 4) = b;
+      }
+    }
+  } else {
+    bf16* dst = static_cast<bf16*>(p.C) + (size_t)row * p.ldc + col0;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      if (col0 + g * 8 < p.N) {
+        uint4 o;
+        o.x = pack_bf16x2(__uint_as_float(r[8 * g + 0]), __uint_as_float(r[8 * g + 1]));
+        o.y = pack_bf16x2(__uint_as_float(r[8 * g + 2]), __uint_as_float(r[8 * g + 3]));
+        o.z = pack_bf16x2(__uint_as_float(r[8 * g + 4]), __uint_as_float(r[8 * g + 5]));
+        o.w = pack_bf16x2(__uint_as_float(r[8 * g + 6]), __uint_as_float(r[8 * g + 7]));
+        *reinterpret_cast<uint4*>(dst + 8 * g) = o;
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  // 128-byte swizzled tiles want 1024-byte aligned bases.
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* tiles = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;   // [2]
+  uint64_t* acc_empty = acc_full + 2;    // [2]
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int num_tiles = p.m_blocks * p.n_blocks;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);  // one arrive per epilogue warp
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_base_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_base_slot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int mb = tile % p.m_blocks, nb = tile / p.m_blocks;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, p.status, abort_flag)) { ok = false; break; }
+          uint8_t* sa = tiles + stage * STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          tma_load_2d(sa, &tmA, &full[stage], kb * BK, mb * BM);
+          tma_load_2d(sa + A_BYTES, &tmB, &full[stage], kb * BK, nb * BN);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {
+        // Let copies already in flight land before the CTA can exit: wait
+        // (bounded) for every stage's last fill.
+        for (int s = 0; s < STAGES; ++s) {
+          long long t0 = clock64();
+          while (!mbar_try_wait(&full[s], 0) && !mbar_try_wait(&full[s], 1) &&
+                 clock64() - t0 < kWaitLimitCycles) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (one thread)
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, p.status, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(tiles + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k) {
+            // Advancing the start address by 32 bytes per 16-element K step
+            // inside the 128-byte swizzle atom; the hardware applies the
+            // swizzle on the absolute address (tile bases are 1024-aligned).
+            uint64_t ad = smem_desc(sa + k * 32, 16, 1024, 2);
+            uint64_t bd = smem_desc(sb + k * 32, 16, 1024, 2);
+            mma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0);
+          }
+          mma_commit(&empty[stage]);  // frees the stage once these MMAs retire
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        mma_commit(&acc_full[acc]);   // accumulator complete
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+    }
+  } else {
+    // ---------------- epilogue warps 2..5: TMEM lanes 32*(warp%4) .. +31
+    const int quarter = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int mb = tile % p.m_blocks, nb = tile / p.m_blocks;
+      if (!mbar_wait(&acc_full[acc], acc_phase, p.status, abort_flag)) break;
+      tc_fence_after();
+      const int row = mb * BM + quarter * 32 + lane;
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        const int col0 = nb * BN + c * 32;
+        if (col0 >= p.N) break;  // uniform across the warp
+        uint32_t r[32];
+        tmem_ld32(taddr + c * 32, r);
+        tmem_ld_wait();
+        if (row < p.M) store_row_chunk(p, row, col0, r);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+__global__ void zero_fill_kernel(void* C, int64_t ldc, int32_t c_f32, int32_t M, int32_t N) {
+  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  int64_t total = (int64_t)M * N;
+  for (; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    int64_t m = i / N, n = i % N;
+    if (c_f32) static_cast<float*>(C)[m * ldc + n] = 0.0f;
+    else static_cast<bf16*>(C)[m * ldc + n] = __float2bfloat16_rn(0.0f);
+  }
+}
+
+}  // namespace gemm
+}  // namespace bi
+
+using namespace bi;
+
+extern "C" bi_status bi_gemm(const void* A, int64_t lda, const void* W, int64_t ldw, void* C,
+                             int64_t ldc, int32_t c_dtype, int64_t M, int64_t N, int64_t K,
+                             void* stream) {
+  if (!A || !W || !C) return fail(BI_ERR_INVALID_ARG, "gemm: null pointer");
+  if (M < 0 || N < 0 || K < 0) return fail(BI_ERR_INVALID_ARG, "gemm: negative size");
+  if (c_dtype != BI_BF16 && c_dtype != BI_F32) return fail(BI_ERR_INVALID_ARG, "gemm: bad c_dtype %d", c_dtype);
+  if (M > (1ll << 30) || N > (1ll << 30) || K > (1ll << 30)) return fail(BI_ERR_SHAPE, "gemm: size above 2^30");
+  if (K % 8 || N % 8) return fail(BI_ERR_SHAPE, "gemm: K (%lld) and N (%lld) must be multiples of 8", (long long)K, (long long)N);
+  if (lda < K || ldw < K || ldc < N) return fail(BI_ERR_SHAPE, "gemm: leading dimension smaller than the row");
+  if (lda % 8 || ldw % 8 || ldc % 8) return fail(BI_ERR_ALIGN, "gemm: leading dimensions must be multiples of 8");
+  if (!aligned16(A) || !aligned16(W) || !aligned16(C)) return fail(BI_ERR_ALIGN, "gemm: pointers must be 16-byte aligned");
+  if (M == 0 || N == 0) return BI_OK;
+  bi_status st = require_sm100();
+  if (st != BI_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int32_t c_f32 = c_dtype == BI_F32;
+  if (K == 0) {
+    gemm::zero_fill_kernel<<<296, 256, 0, s>>>(C, ldc, c_f32, (int32_t)M, (int32_t)N);
+    BI_CHECK_LAUNCH("gemm zero fill");
+    return BI_OK;
+  }
+  CUtensorMap tmA, tmB;
+  {
+    uint64_t dims[2] = {(uint64_t)K, (uint64_t)M};
+    uint64_t strides[1] = {(uint64_t)lda * 2};
+    uint32_t box[2] = {gemm::BK, gemm::BM};
+    if ((st = encode_tmap(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(A), dims,
+                          strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != BI_OK)
+      return st;
+  }
+  {
+    uint64_t dims[2] = {(uint64_t)K, (uint64_t)N};
+    uint64_t strides[1] = {(uint64_t)ldw * 2};
+    uint32_t box[2] = {gemm::BK, gemm::BN};
+    if ((st = encode_tmap(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(W), dims,
+                          strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != BI_OK)
+      return st;
+  }
+  gemm::Params p;
+  p.C = C;
+  p.ldc = ldc;
+  p.c_f32 = c_f32;
+  p.M = (int32_t)M;
+  p.N = (int32_t)N;
+  p.K = (int32_t)K;
+  p.m_blocks = (int32_t)((M + gemm::BM - 1) / gemm::BM);
+  p.n_blocks = (int32_t)((N + gemm::BN - 1) / gemm::BN);
+  p.k_blocks = (int32_t)((K + gemm::BK - 1) / gemm::BK);
+  p.status = status_word();
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!attr_set[dev & 63]) {
+    cudaError_t e = cudaFuncSetAttribute(gemm::gemm_tcgen05_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)gemm::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e, "gemm: smem attribute");
+    attr_set[dev & 63] = true;
+  }
+  const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
+  const int sms = num_sms();
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  gemm::gemm_tcgen05_kernel<<<grid, gemm::THREADS, gemm::SMEM_BYTES, s>>>(tmA, tmB, p);
+  BI_CHECK_LAUNCH("gemm launch");
+  return BI_OK;
+}

@@ -1,0 +1,316 @@
+// pointwise.cu -- the element-wise steps of the decoder and the KV-cache write.
+//
+// "Defeating Nondeterminism in LLM Inference", section "How do we make
+// kernels batch-invariant?": pointwise operations are batch-invariant as long
+// as every element goes through the same code (the page's counter-example is
+// a CPU kernel that vectorises part of an array and not the rest). Each kernel
+// here has one code path per element: no vector/scalar tail split depends on
+// the batch, and every element's arithmetic is written out with explicit
+// rounding intrinsics.
+//
+// The cache write follows section "Batch-invariant attention": the KV cache
+// and page table are updated before attention runs, so attention always reads
+// keys from one layout.
+#include "common.cuh"
+#include "host.h"
+
+namespace bi {
+namespace pw {
+
+// ---- KV append: one warp per (token, kv head). k row -> k_cache[page][g][slot][:],
+// v row -> v_cache[page][g][:][slot] (transposed page block).
+__global__ void kv_append_kernel(const bf16* __restrict__ k_new, const bf16* __restrict__ v_new,
+                                 int64_t ld_new, const int32_t* __restrict__ slots, int64_t n_tok,
+                                 int Hkv, int num_pages, bf16* __restrict__ kc,
+                                 bf16* __restrict__ vc, int32_t* status) {
+  const int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (wid >= n_tok * Hkv) return;
+  const int64_t t = wid / Hkv;
+  const int g = (int)(wid % Hkv);
+  const int32_t slot = slots[t];
+  if (slot < 0) return;  // padding token
+  if (slot >= num_pages * BI_PAGE_SIZE) {
+    if (lane == 0) set_status(status, BI_DEV_BAD_SLOT);
+    return;
+  }
+  const int page = slot / BI_PAGE_SIZE, off = slot % BI_PAGE_SIZE;
+  const bf16* ksrc = k_new + t * ld_new + (int64_t)g * BI_HEAD_DIM;
+  const bf16* vsrc = v_new + t * ld_new + (int64_t)g * BI_HEAD_DIM;
+  const size_t blk = (size_t)page * Hkv + g;
+  // keys: 128 elements = 16 lanes x 16 bytes
+  if (lane < 16) {
+    const uint4 v = reinterpret_cast<const uint4*>(ksrc)[lane];
+    reinterpret_cast<uint4*>(kc + (blk * BI_PAGE_SIZE + off) * BI_HEAD_DIM)[lane] = v;
+  }
+  // values, transposed: element d goes to row d, column `off` of the page block
+  bf16* vdst = vc + blk * BI_HEAD_DIM * BI_PAGE_SIZE + off;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int d = lane * 4 + i;
+    vdst[(size_t)d * BI_PAGE_SIZE] = vsrc[d];
+  }
+}
+
+// ---- embedding gather into the fp32 residual stream
+__global__ void embed_kernel(const int32_t* __restrict__ tokens, const bf16* __restrict__ table,
+                             int64_t vocab, int D, float* __restrict__ out, int32_t* status) {
+  const int64_t t = blockIdx.x;
+  const int32_t id = tokens[t];
+  const bool ok = id >= 0 && id < vocab;
+  if (!ok && threadIdx.x == 0) set_status(status, BI_DEV_BAD_TOKEN);
+  for (int c = threadIdx.x; c < D / 8; c += blockDim.x) {
+    float v[8];
+    if (ok) {
+      const uint4 u = reinterpret_cast<const uint4*>(table + (size_t)id * D)[c];
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(h[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+    }
+    float4* o = reinterpret_cast<float4*>(out + t * (size_t)D + c * 8);
+    o[0] = make_float4(v[0], v[1], v[2], v[3]);
+    o[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+}
+
+// ---- RoPE table: cos/sin of pos * theta^(-2i/128) in fp64, stored as fp32
+__global__ void rope_table_kernel(float* __restrict__ cs, int max_pos, double theta) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)max_pos * 64) return;
+  const int pos = (int)(idx / 64), i = (int)(idx % 64);
+  const double inv_freq = pow(theta, -2.0 * (double)i / (double)BI_HEAD_DIM);
+  const double a = (double)pos * inv_freq;
+  cs[idx * 2] = (float)cos(a);
+  cs[idx * 2 + 1] = (float)sin(a);
+}
+
+// ---- RoPE in place: one thread per (token, head, pair i < 64)
+__global__ void rope_kernel(bf16* __restrict__ x, int64_t ldx, int n_heads,
+                            const int32_t* __restrict__ pos, int64_t n_tok,
+                            const float* __restrict__ cs, int max_pos, int32_t* status) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n_tok * n_heads * 64) return;
+  const int i = (int)(idx % 64);
+  const int64_t th = idx / 64;
+  const int h = (int)(th % n_heads);
+  const int64_t t = th / n_heads;
+  const int p = pos[t];
+  bf16* row = x + t * ldx + (int64_t)h * BI_HEAD_DIM;
+  if (p < 0 || p >= max_pos) {
+    if (i == 0) set_status(status, BI_DEV_BAD_TOKEN);
+    return;
+  }
+  const float c = cs[((size_t)p * 64 + i) * 2], s = cs[((size_t)p * 64 + i) * 2 + 1];
+  const float a = __bfloat162float(row[i]), b = __bfloat162float(row[i + 64]);
+  row[i] = __float2bfloat16_rn(__fsub_rn(__fmul_rn(a, c), __fmul_rn(b, s)));
+  row[i + 64] = __float2bfloat16_rn(__fadd_rn(__fmul_rn(b, c), __fmul_rn(a, s)));
+}
+
+// ---- SwiGLU: out = bf16(silu(g) * u), silu(g) = g / (1 + exp(-g))
+__global__ void swiglu_kernel(const bf16* __restrict__ gu, int64_t n_tok, int64_t F,
+                              bf16* __restrict__ out) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n_tok * F) return;
+  const int64_t t = idx / F, i = idx % F;
+  const float g = __bfloat162float(gu[t * 2 * F + i]);
+  const float u = __bfloat162float(gu[t * 2 * F + F + i]);
+  const float silu = __fdiv_rn(g, __fadd_rn(1.0f, expf(-g)));
+  out[idx] = __float2bfloat16_rn(__fmul_rn(silu, u));
+}
+
+// ---- residual add into the fp32 stream
+__global__ void residual_kernel(float* __restrict__ x, const bf16* __restrict__ d, int64_t n) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n) return;
+  x[idx] = __fadd_rn(x[idx], __bfloat162float(d[idx]));
+}
+
+// ---- argmax per row, lowest index on ties; NaN counts as the largest value
+__device__ __forceinline__ bool better(float a, int ia, float b, int ib) {
+  const bool na = a != a, nb = b != b;
+  if (na || nb) return na && (!nb || ia < ib);
+  if (a != b) return a > b;
+  return ia < ib;
+}
+
+__global__ void argmax_kernel(const float* __restrict__ logits, int64_t V, int64_t ld,
+                              int32_t* __restrict__ idx_out) {
+  __shared__ float sv[32];
+  __shared__ int si[32];
+  const float* row = logits + (size_t)blockIdx.x * ld;
+  float bv = -INFINITY;
+  int bi = 0x7fffffff;
+  for (int64_t j = threadIdx.x; j < V; j += blockDim.x) {
+    const float v = row[j];
+    if (better(v, (int)j, bv, bi)) { bv = v; bi = (int)j; }
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const float ov = __shfl_down_sync(0xffffffffu, bv, off);
+    const int oi = __shfl_down_sync(0xffffffffu, bi, off);
+    if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+  }
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) { sv[w] = bv; si[w] = bi; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int k = 1; k < (int)(blockDim.x >> 5); ++k)
+      if (better(sv[k], si[k], bv, bi)) { bv = sv[k]; bi = si[k]; }
+    idx_out[blockIdx.x] = bi == 0x7fffffff ? 0 : bi;
+  }
+}
+
+}  // namespace pw
+
+bi_status launch_kv_append(const bf16* k, const bf16* v, int64_t ld_new, const int32_t* slots,
+                           int64_t n_tok, bf16* kc, bf16* vc, int Hkv, int num_pages,
+                           cudaStream_t s) {
+  const int64_t warps = n_tok * Hkv;
+  const int64_t blocks = (warps + 7) / 8;
+  pw::kv_append_kernel<<<(unsigned)blocks, 256, 0, s>>>(k, v, ld_new, slots, n_tok, Hkv, num_pages,
+                                                        kc, vc, status_word());
+  BI_CHECK_LAUNCH("kv_append launch");
+  return BI_OK;
+}
+
+bi_status launch_embed(const int32_t* tok, int64_t n_tok, const bf16* table, int64_t vocab,
+                       int64_t D, float* out, cudaStream_t s) {
+  pw::embed_kernel<<<(unsigned)n_tok, 128, 0, s>>>(tok, table, vocab, (int)D, out, status_word());
+  BI_CHECK_LAUNCH("embed launch");
+  return BI_OK;
+}
+
+bi_status launch_rope(bf16* x, int64_t ldx, int n_heads, const int32_t* pos, int64_t n_tok,
+                      const float* cs, int max_pos, cudaStream_t s) {
+  const int64_t n = n_tok * n_heads * 64;
+  pw::rope_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(x, ldx, n_heads, pos, n_tok, cs,
+                                                              max_pos, status_word());
+  BI_CHECK_LAUNCH("rope launch");
+  return BI_OK;
+}
+
+bi_status launch_swiglu(const bf16* gu, int64_t n_tok, int64_t F, bf16* out, cudaStream_t s) {
+  const int64_t n = n_tok * F;
+  pw::swiglu_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(gu, n_tok, F, out);
+  BI_CHECK_LAUNCH("swiglu launch");
+  return BI_OK;
+}
+
+bi_status launch_residual(float* x, const bf16* d, int64_t n, cudaStream_t s) {
+  pw::residual_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(x, d, n);
+  BI_CHECK_LAUNCH("residual launch");
+  return BI_OK;
+}
+
+bi_status launch_argmax(const float* logits, int64_t rows, int64_t V, int64_t ld, int32_t* idx,
+                        cudaStream_t s) {
+  pw::argmax_kernel<<<(unsigned)rows, 256, 0, s>>>(logits, V, ld, idx);
+  BI_CHECK_LAUNCH("argmax launch");
+  return BI_OK;
+}
+
+}  // namespace bi
+
+using namespace bi;
+
+static bi_status check_kv(const bi_kv_layout* kv) {
+  if (!kv) return fail(BI_ERR_INVALID_ARG, "kv layout is null");
+  if (kv->head_dim != BI_HEAD_DIM || kv->page_size != BI_PAGE_SIZE)
+    return fail(BI_ERR_SHAPE, "kv layout: head_dim must be 128 and page_size 16");
+  if (kv->num_pages <= 0 || kv->num_kv_heads <= 0) return fail(BI_ERR_SHAPE, "kv layout: sizes must be positive");
+  if ((int64_t)kv->num_pages * BI_PAGE_SIZE > 0x7fffffffll) return fail(BI_ERR_SHAPE, "kv layout: too many pages");
+  return BI_OK;
+}
+
+extern "C" bi_status bi_kv_append(const void* k_new, const void* v_new, int64_t ld_new,
+                                  const int32_t* slot_mapping, int64_t n_tok, void* k_cache,
+                                  void* v_cache, const bi_kv_layout* kv, void* stream) {
+  bi_status st = check_kv(kv);
+  if (st != BI_OK) return st;
+  if (!k_new || !v_new || !slot_mapping || !k_cache || !v_cache) return fail(BI_ERR_INVALID_ARG, "kv_append: null pointer");
+  if (n_tok < 0) return fail(BI_ERR_INVALID_ARG, "kv_append: negative n_tok");
+  if (ld_new < (int64_t)kv->num_kv_heads * BI_HEAD_DIM) return fail(BI_ERR_SHAPE, "kv_append: ld_new smaller than num_kv_heads*128");
+  if (ld_new % 8 || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(BI_ERR_ALIGN, "kv_append: rows must be 16-byte aligned");
+  if (n_tok == 0) return BI_OK;
+  if ((st = require_sm100()) != BI_OK) return st;
+  return launch_kv_append(static_cast<const bf16*>(k_new), static_cast<const bf16*>(v_new), ld_new,
+                          slot_mapping, n_tok, static_cast<bf16*>(k_cache),
+                          static_cast<bf16*>(v_cache), kv->num_kv_heads, kv->num_pages,
+                          static_cast<cudaStream_t>(stream));
+}
+
+extern "C" bi_status bi_embed(const int32_t* tokens, int64_t n_tok, const void* table,
+                              int64_t vocab, int64_t D, float* out, void* stream) {
+  if (!tokens || !table || !out) return fail(BI_ERR_INVALID_ARG, "embed: null pointer");
+  if (n_tok < 0 || vocab <= 0 || D <= 0) return fail(BI_ERR_INVALID_ARG, "embed: bad sizes");
+  if (D % 8 || !aligned16(table) || !aligned16(out)) return fail(BI_ERR_ALIGN, "embed: D % 8 and 16-byte alignment required");
+  if (n_tok > 0x7fffffffll) return fail(BI_ERR_SHAPE, "embed: too many tokens");
+  if (n_tok == 0) return BI_OK;
+  bi_status st = require_sm100();
+  if (st != BI_OK) return st;
+  return launch_embed(tokens, n_tok, static_cast<const bf16*>(table), vocab, D, out,
+                      static_cast<cudaStream_t>(stream));
+}
+
+extern "C" bi_status bi_rope_table(float* cos_sin, int32_t max_pos, double theta, void* stream) {
+  if (!cos_sin || max_pos <= 0 || !(theta > 1.0)) return fail(BI_ERR_INVALID_ARG, "rope_table: bad arguments");
+  bi_status st = require_sm100();
+  if (st != BI_OK) return st;
+  const int64_t n = (int64_t)max_pos * 64;
+  pw::rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      cos_sin, max_pos, theta);
+  BI_CHECK_LAUNCH("rope_table launch");
+  return BI_OK;
+}
+
+extern "C" bi_status bi_rope(void* x, int64_t ldx, int32_t n_heads, const int32_t* positions,
+                             int64_t n_tok, const float* cos_sin, int32_t max_pos, void* stream) {
+  if (!x || !positions || !cos_sin) return fail(BI_ERR_INVALID_ARG, "rope: null pointer");
+  if (n_tok < 0 || n_heads <= 0 || max_pos <= 0) return fail(BI_ERR_INVALID_ARG, "rope: bad sizes");
+  if (ldx < (int64_t)n_heads * BI_HEAD_DIM) return fail(BI_ERR_SHAPE, "rope: ldx smaller than n_heads*128");
+  if (n_tok == 0) return BI_OK;
+  bi_status st = require_sm100();
+  if (st != BI_OK) return st;
+  return launch_rope(static_cast<bf16*>(x), ldx, n_heads, positions, n_tok, cos_sin, max_pos,
+                     static_cast<cudaStream_t>(stream));
+}
+
+extern "C" bi_status bi_swiglu(const void* gu, int64_t n_tok, int64_t F, void* out, void* stream) {
+  if (!gu || !out) return fail(BI_ERR_INVALID_ARG, "swiglu: null pointer");
+  if (n_tok < 0 || F <= 0) return fail(BI_ERR_INVALID_ARG, "swiglu: bad sizes");
+  if (n_tok == 0) return BI_OK;
+  bi_status st = require_sm100();
+  if (st != BI_OK) return st;
+  return launch_swiglu(static_cast<const bf16*>(gu), n_tok, F, static_cast<bf16*>(out),
+                       static_cast<cudaStream_t>(stream));
+}
+
+extern "C" bi_status bi_residual_add(float* x, const void* d, int64_t n_tok, int64_t D,
+                                     void* stream) {
+  if (!x || !d) return fail(BI_ERR_INVALID_ARG, "residual_add: null pointer");
+  if (n_tok < 0 || D <= 0) return fail(BI_ERR_INVALID_ARG, "residual_add: bad sizes");
+  if (n_tok == 0) return BI_OK;
+  bi_status st = require_sm100();
+  if (st != BI_OK) return st;
+  return launch_residual(x, static_cast<const bf16*>(d), n_tok * D,
+                         static_cast<cudaStream_t>(stream));
+}
+
+extern "C" bi_status bi_argmax(const float* logits, int64_t rows, int64_t V, int64_t ld,
+                               int32_t* idx, void* stream) {
+  if (!logits || !idx) return fail(BI_ERR_INVALID_ARG, "argmax: null pointer");
+  if (rows < 0 || V <= 0 || ld < V) return fail(BI_ERR_INVALID_ARG, "argmax: bad sizes");
+  if (V > 0x7fffffffll || rows > 0x7fffffffll) return fail(BI_ERR_SHAPE, "argmax: too large");
+  if (rows == 0) return BI_OK;
+  bi_status st = require_sm100();
+  if (st != BI_OK) return st;
+  return launch_argmax(logits, rows, V, ld, idx, static_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,163 @@
+// rmsnorm.cu -- batch-invariant RMSNorm, one CTA per row.
+//
+// "Defeating Nondeterminism in LLM Inference", section "Batch-invariant
+// RMSNorm": assign each batch element (row) to one core so that no row's
+// reduction is ever split; the reduction strategy may depend on the reduced
+// length D, never on the number of rows. Small batches simply leave SMs idle.
+//
+// Fixed order of the sum of squares of row i (depends on D only):
+//   1. thread t adds x^2 of its chunks c = t, t + T, t + 2T, ... (8 elements
+//      each, left to right) with fmaf, T = threads per CTA (a function of D);
+//   2. warp shuffle-down tree, offsets 16, 8, 4, 2, 1 (lane 0 ends with the
+//      warp sum);
+//   3. thread 0 adds the warp sums in warp order and forms
+//      r = 1 / sqrtf(ss / D + eps);
+//   4. every element: y = bf16((x * r) * gamma), round to nearest even.
+#include "common.cuh"
+#include "host.h"
+
+namespace bi {
+
+template <typename Tin>
+struct Row8;  // 8 consecutive input elements as fp32
+
+template <>
+struct Row8<bf16> {
+  static __device__ __forceinline__ void load(const bf16* p, float (&v)[8]) {
+    uint4 u = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __bfloat1622float2(h[i]);
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
+    }
+  }
+};
+
+template <>
+struct Row8<float> {
+  static __device__ __forceinline__ void load(const float* p, float (&v)[8]) {
+    float4 a = *reinterpret_cast<const float4*>(p);
+    float4 b = *reinterpret_cast<const float4*>(p + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+};
+
+// CPT = chunks per thread (compile-time so the row stays in registers).
+template <typename Tin, int CPT>
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const Tin* __restrict__ x,
+                                                      const bf16* __restrict__ gamma,
+                                                      bf16* __restrict__ y, int D, float eps) {
+  __shared__ float warp_sum[32];
+  __shared__ float row_scale;
+  const int T = blockDim.x;
+  const int t = threadIdx.x;
+  const int nchunks = D >> 3;
+  const size_t row = blockIdx.x;
+  const Tin* xr = x + row * (size_t)D;
+  bf16* yr = y + row * (size_t)D;
+
+  float v[CPT][8];
+  float ss = 0.0f;
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {
+    int c = t + i * T;
+    if (c < nchunks) {
+      Row8<Tin>::load(xr + c * 8, v[i]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss = fmaf(v[i][e], v[i][e], ss);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) ss += __shfl_down_sync(0xffffffffu, ss, off);
+  const int warp = t >> 5, lane = t & 31;
+  if (lane == 0) warp_sum[warp] = ss;
+  __syncthreads();
+  if (t == 0) {
+    float total = 0.0f;
+    const int nw = T >> 5;
+    for (int w = 0; w < nw; ++w) total = total + warp_sum[w];
+    row_scale = 1.0f / sqrtf(total / (float)D + eps);
+  }
+  __syncthreads();
+  const float r = row_scale;
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {
+    int c = t + i * T;
+    if (c < nchunks) {
+      float g[8];
+      Row8<bf16>::load(gamma + c * 8, g);
+      uint4 o;
+      uint32_t* op = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        op[e] = pack_bf16x2((v[i][2 * e] * r) * g[2 * e], (v[i][2 * e + 1] * r) * g[2 * e + 1]);
+      *reinterpret_cast<uint4*>(yr + c * 8) = o;
+    }
+  }
+}
+
+// Threads per CTA and chunks per thread as a function of D alone.
+static void rms_geometry(int64_t D, int* threads, int* cpt) {
+  int64_t nchunks = D / 8;
+  int64_t T = ((nchunks + 31) / 32) * 32;
+  if (T > 256) T = 256;
+  int64_t c = (nchunks + T - 1) / T;
+  int p = 1;
+  while (p < c) p <<= 1;
+  *threads = (int)T;
+  *cpt = p;
+}
+
+template <typename Tin>
+static bi_status launch_rms(const Tin* x, const bf16* g, bf16* y, int64_t M, int64_t D, float eps,
+                            cudaStream_t s) {
+  int T, cpt;
+  rms_geometry(D, &T, &cpt);
+  dim3 grid((unsigned)M), block(T);
+  switch (cpt) {
+    case 1: rmsnorm_kernel<Tin, 1><<<grid, block, 0, s>>>(x, g, y, (int)D, eps); break;
+    case 2: rmsnorm_kernel<Tin, 2><<<grid, block, 0, s>>>(x, g, y, (int)D, eps); break;
+    case 4: rmsnorm_kernel<Tin, 4><<<grid, block, 0, s>>>(x, g, y, (int)D, eps); break;
+    case 8: rmsnorm_kernel<Tin, 8><<<grid, block, 0, s>>>(x, g, y, (int)D, eps); break;
+    case 16: rmsnorm_kernel<Tin, 16><<<grid, block, 0, s>>>(x, g, y, (int)D, eps); break;
+    default: return fail(BI_ERR_SHAPE, "rmsnorm: D=%lld unsupported", (long long)D);
+  }
+  BI_CHECK_LAUNCH("rmsnorm launch");
+  return BI_OK;
+}
+
+static bi_status check_rms(const void* x, const void* gamma, const void* y, int64_t M, int64_t D,
+                           float eps) {
+  if (!x || !gamma || !y) return fail(BI_ERR_INVALID_ARG, "rmsnorm: null pointer");
+  if (M < 0 || D <= 0) return fail(BI_ERR_INVALID_ARG, "rmsnorm: bad sizes M=%lld D=%lld", (long long)M, (long long)D);
+  if (D % 8 != 0 || D > 32768) return fail(BI_ERR_SHAPE, "rmsnorm: D=%lld must be a multiple of 8 and <= 32768", (long long)D);
+  if (M > 0x7fffffffll) return fail(BI_ERR_SHAPE, "rmsnorm: M=%lld too large", (long long)M);
+  if (!(eps >= 0.0f)) return fail(BI_ERR_INVALID_ARG, "rmsnorm: eps must be >= 0");
+  if (!aligned16(x) || !aligned16(gamma) || !aligned16(y)) return fail(BI_ERR_ALIGN, "rmsnorm: pointers must be 16-byte aligned");
+  return BI_OK;
+}
+
+}  // namespace bi
+
+using namespace bi;
+
+extern "C" bi_status bi_rmsnorm(const void* x, const void* gamma, void* y, int64_t M, int64_t D,
+                                float eps, void* stream) {
+  bi_status st = check_rms(x, gamma, y, M, D, eps);
+  if (st != BI_OK || M == 0) return st;
+  if ((st = require_sm100()) != BI_OK) return st;
+  return launch_rms<bf16>(static_cast<const bf16*>(x), static_cast<const bf16*>(gamma),
+                          static_cast<bf16*>(y), M, D, eps, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" bi_status bi_rmsnorm_f32in(const float* x, const void* gamma, void* y, int64_t M,
+                                      int64_t D, float eps, void* stream) {
+  bi_status st = check_rms(x, gamma, y, M, D, eps);
+  if (st != BI_OK || M == 0) return st;
+  if ((st = require_sm100()) != BI_OK) return st;
+  return launch_rms<float>(x, static_cast<const bf16*>(gamma), static_cast<bf16*>(y), M, D, eps,
+                           static_cast<cudaStream_t>(stream));
+}

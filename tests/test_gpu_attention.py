@@ -1,0 +1,201 @@
+"""Paged attention on the GPU: parity with the fp64 oracle, and bitwise
+equality of every token's output across decode, chunked prefill (chunks of 1,
+64, 512), batch composition and runs ("Defeating Nondeterminism in LLM
+Inference", section "Batch-invariant attention": query 1000 must reduce in the
+same order with 0 or 999 cached tokens). Tolerance: per element
+2^-7 |y| + 2^-7 R with R = sqrt(sum_j (p_j v_j)^2) (kappa = 1 for the bf16
+rounding of the softmax weights)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from invariant_deterministic_03_b200 import synth
+from oracle import fp64
+from tests.checker import check
+from tests.gpu_common import dev, f64, same_bits
+
+pytestmark = pytest.mark.gpu
+D = 128
+SCALE = 1.0 / math.sqrt(D)
+
+
+@pytest.fixture(scope="module")
+def bi(cuda_device):
+    from invariant_deterministic_03_b200 import bi as mod
+    return mod
+
+
+class Seqs:
+    """Per-sequence q/k/v ([L, H, 128] bf16, CPU) and their paged cache."""
+
+    def __init__(self, bi, lens, Hq, Hkv, seed, fill=0.0, spare_pages=3):
+        self.lens, self.Hq, self.Hkv = list(lens), Hq, Hkv
+        self.q = [synth.normal_bf16((L, Hq, D), 1.0, seed * 1000 + 3 * b) for b, L in enumerate(lens)]
+        self.k = [synth.normal_bf16((L, Hkv, D), 1.0, seed * 1000 + 3 * b + 1) for b, L in enumerate(lens)]
+        self.v = [synth.normal_bf16((L, Hkv, D), 1.0, seed * 1000 + 3 * b + 2) for b, L in enumerate(lens)]
+        self.layout = synth.PagedLayout(lens, seed, spare_pages=spare_pages)
+        P = self.layout.num_pages
+        self.kc = torch.full((P, Hkv, 16, D), fill, dtype=torch.bfloat16, device="cuda:0")
+        self.vc = torch.full((P, Hkv, D, 16), fill, dtype=torch.bfloat16, device="cuda:0")
+        for b, L in enumerate(lens):
+            slots = self.layout.slots(b, 0, L)
+            bi.bi_kv_append(dev(self.k[b].reshape(L, -1)), dev(self.v[b].reshape(L, -1)),
+                            dev(slots), self.kc, self.vc)
+        self.bt = dev(self.layout.block_table)
+
+    def shape(self, bi, max_kv_len=None):
+        return bi.attn_shape(self.Hq, self.Hkv, self.layout.num_pages, self.layout.pages_per_seq,
+                             max_kv_len or max(self.lens))
+
+    def oracle(self, b, positions):
+        out, probs = fp64.attention(f64(self.q[b][positions]), f64(self.k[b]), f64(self.v[b]),
+                                    positions, SCALE)
+        R = fp64.attention_reduction_scale(probs, f64(self.v[b]), self.Hq // self.Hkv)
+        return out, R
+
+
+def _decode(bi, S, q_rows, seq_lens, bt, shape):
+    B = q_rows.shape[0]
+    ws = torch.empty(bi.bi_attn_workspace_size(shape, B), dtype=torch.uint8, device="cuda:0")
+    out = torch.empty(B, q_rows.shape[1], dtype=torch.bfloat16, device="cuda:0")
+    bi.bi_attn_decode(q_rows, S.kc, S.vc, bt, dev(torch.tensor(seq_lens, dtype=torch.int32)),
+                      shape, out, ws)
+    return out
+
+
+def _prefill(bi, S, chunks, shape):
+    """chunks: list of (b, start, end) -> one prefill call; returns out rows."""
+    q = torch.cat([S.q[b][s:e].reshape(e - s, -1) for b, s, e in chunks])
+    cu = [0]
+    for _, s, e in chunks:
+        cu.append(cu[-1] + e - s)
+    seq_lens = [e for _, _, e in chunks]
+    bt = S.layout.block_table[[b for b, _, _ in chunks]]
+    n = q.shape[0]
+    ws = torch.empty(bi.bi_attn_workspace_size(shape, n), dtype=torch.uint8, device="cuda:0")
+    out = torch.empty(n, q.shape[1], dtype=torch.bfloat16, device="cuda:0")
+    bi.bi_attn_prefill(dev(q), dev(torch.tensor(cu, dtype=torch.int32)), max(e - s for _, s, e in chunks),
+                       S.kc, S.vc, dev(bt), dev(torch.tensor(seq_lens, dtype=torch.int32)), shape, out, ws)
+    return out
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (8, 8), (16, 8), (64, 8)])
+def test_decode_parity(bi, Hq, Hkv):
+    lens = [1, 16, 17, 200, 512, 513, 700, 1030]
+    S = Seqs(bi, lens, Hq, Hkv, seed=Hq)
+    q_rows = torch.stack([S.q[b][L - 1].reshape(-1) for b, L in enumerate(lens)])
+    out = _decode(bi, S, dev(q_rows), lens, S.bt, S.shape(bi))
+    for b, L in enumerate(lens):
+        o64, R = S.oracle(b, [L - 1])
+        check(f64(out[b]).reshape(1, Hq, D), o64, R, kappa=1.0, what=f"decode b={b} L={L}")
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (8, 8)])
+def test_decode_equals_chunked_prefill(bi, Hq, Hkv):
+    """Every token of a 1100-token sequence: decode (one token, its keys
+    cached) == prefill in chunks of 1, 64 and 512 == whole prefill, bitwise;
+    and each matches the oracle."""
+    L = 1100
+    S = Seqs(bi, [L], Hq, Hkv, seed=7)
+    shape = S.shape(bi)
+    # decode of all positions at once: B = L rows sharing one page table
+    bt_rep = S.bt.repeat(L, 1)
+    q_rows = dev(S.q[0].reshape(L, -1))
+    dec = _decode(bi, S, q_rows, list(range(1, L + 1)), bt_rep, shape)
+    o64, R = S.oracle(0, list(range(L)))
+    check(f64(dec).reshape(L, Hq, D), o64, R, kappa=1.0, what="decode all positions")
+    for chunk in [1, 64, 512, L]:
+        if chunk == 1:
+            starts = list(range(0, L, 97))   # a sample of single-token chunks
+        else:
+            starts = list(range(0, L, chunk))
+        for s0 in starts:
+            e0 = min(L, s0 + chunk)
+            out = _prefill(bi, S, [(0, s0, e0)], shape)
+            assert same_bits(out, dec[s0:e0]), f"chunk {chunk} at {s0}"
+
+
+def test_batch_composition(bi):
+    """A sequence's rows are the same bits alone, co-batched with others of
+    mixed lengths and chunk sizes, and at a different batch position."""
+    lens = [900, 37, 4100, 513, 64]
+    S = Seqs(bi, lens, 32, 8, seed=11)
+    shape = S.shape(bi)
+    alone = _prefill(bi, S, [(0, 600, 900)], shape)
+    mixed = _prefill(bi, S, [(1, 0, 37), (2, 3800, 4100), (0, 600, 900), (3, 512, 513), (4, 0, 64)], shape)
+    assert same_bits(mixed[37 + 300:37 + 300 + 300], alone)
+    mixed2 = _prefill(bi, S, [(0, 600, 900), (4, 0, 64)], shape)
+    assert same_bits(mixed2[:300], alone)
+    o64, R = S.oracle(0, list(range(600, 900)))
+    check(f64(alone).reshape(300, 32, D), o64, R, kappa=1.0, what="prefill chunk")
+    o64, R = S.oracle(2, list(range(3800, 4100)))
+    check(f64(mixed[37:337]).reshape(300, 32, D), o64, R, kappa=1.0, what="prefill long")
+
+
+def test_stale_cache_contents_do_not_leak(bi):
+    """Cache slots past a sequence's end hold NaN: outputs are finite and the
+    same bits as with a zeroed cache."""
+    lens = [5, 300, 1000]
+    Sz = Seqs(bi, lens, 32, 8, seed=21, fill=0.0)
+    Sn = Seqs(bi, lens, 32, 8, seed=21, fill=float("nan"))
+    q_rows = dev(torch.stack([Sz.q[b][L - 1].reshape(-1) for b, L in enumerate(lens)]))
+    oz = _decode(bi, Sz, q_rows, lens, Sz.bt, Sz.shape(bi))
+    on = _decode(bi, Sn, q_rows, lens, Sn.bt, Sn.shape(bi))
+    assert torch.isfinite(on.float()).all()
+    assert same_bits(oz, on)
+    pz = _prefill(bi, Sz, [(1, 250, 300), (2, 0, 1000)], Sz.shape(bi))
+    pn = _prefill(bi, Sn, [(1, 250, 300), (2, 0, 1000)], Sn.shape(bi))
+    assert same_bits(pz, pn)
+
+
+def test_config3_decode(bi):
+    """Batch 32, 32/8 GQA heads, head dim 128, lengths uniform in [1, 8192]
+    (seed 0), pages from a seeded permutation: every output vs the oracle."""
+    lens = synth.attention_lengths(32, 1, 8192, seed=0)
+    S = Seqs(bi, lens, 32, 8, seed=0)
+    q_rows = dev(torch.stack([S.q[b][L - 1].reshape(-1) for b, L in enumerate(lens)]))
+    out = _decode(bi, S, q_rows, lens, S.bt, S.shape(bi, 8192))
+    for b, L in enumerate(lens):
+        o64, R = S.oracle(b, [L - 1])
+        check(f64(out[b]).reshape(1, 32, D), o64, R, kappa=1.0, what=f"config3 b={b} L={L}")
+    # run to run
+    for _ in range(20):
+        assert same_bits(_decode(bi, S, q_rows, lens, S.bt, S.shape(bi, 8192)), out)
+    # the max_kv_len bound (grid size, workspace) does not reach the arithmetic
+    out2 = _decode(bi, S, q_rows, lens, S.bt, S.shape(bi, 16384))
+    assert same_bits(out2, out)
+
+
+def test_kv_append_exact(bi):
+    """The cache holds the exact input bytes at the slot's page and offset
+    (keys row-major, values transposed per page); padding slots are skipped."""
+    lens = [40, 3]
+    S = Seqs(bi, lens, 32, 8, seed=5)
+    for b, L in enumerate(lens):
+        slots = S.layout.slots(b, 0, L).long()
+        page, off = slots // 16, slots % 16
+        k_got = S.kc[page.cuda(), :, off.cuda(), :]          # [L, Hkv, 128]
+        v_got = S.vc[page.cuda(), :, :, off.cuda()]          # [L, Hkv, 128]
+        assert same_bits(k_got.cpu(), S.k[b])
+        assert same_bits(v_got.cpu(), S.v[b])
+    before_k, before_v = S.kc.clone(), S.vc.clone()
+    junk = dev(synth.normal_bf16((2, 8 * D), 1.0, 99))
+    bi.bi_kv_append(junk, junk, dev(torch.tensor([-1, -5], dtype=torch.int32)), S.kc, S.vc)
+    assert same_bits(S.kc, before_k) and same_bits(S.vc, before_v)
+
+
+def test_bad_page_sets_status(bi):
+    """A page id outside the cache is reported through the status word (the
+    kernel reads zeros instead and never touches the bad address)."""
+    S = Seqs(bi, [40], 32, 8, seed=6)
+    bi.bi_device_status(clear=True)
+    bt = S.bt.clone()
+    bt[0, 1] = S.layout.num_pages + 100
+    q_rows = dev(S.q[0][39].reshape(1, -1))
+    out = _decode(bi, S, q_rows, [40], bt, S.shape(bi))
+    torch.cuda.synchronize()
+    st = bi.bi_device_status(clear=True)
+    assert st & 0x4
+    assert torch.isfinite(out.float()).all()
