@@ -1,0 +1,506 @@
+#!/usr/bin/env python
+"""Benchmark of the batch-invariant kernels on B200.
+
+One STEP = the GEMM sweep at the Mistral-7B MLP shapes: bi_gemm for every
+M in {1, 2, 4, ..., 4096} at (K=4096, N=14336) and at (K=14336, N=4096), bf16
+inputs (A ~ N(0,1), W ~ N(0, 0.02^2)), fp32 accumulation, bf16 output, one
+fixed tiling. value = total FLOPs of the step / device time (TFLOP/s), inputs
+resident in HBM; weights rotate over three copies per shape so no launch finds
+its weights in L2 (each copy is 117 MB, L2 is 126 MB).
+
+Also measured in the same run, each against its roofline: paged decode
+attention (32 sequences, GQA 32/8, lengths U[1, 8192]), RMSNorm (65536 x
+4096), and torch.matmul (cuBLAS, not batch-invariant) on the same sweep as the
+cost of invariance.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own replica of
+the sweep (no data-path collective: the work is independent); the job value
+is the sum of all ranks' FLOPs over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "bi_gemm TFLOP/s & bi_attn/RMSNorm GB/s vs roofline; cost vs cuBLAS; bitwise invariance"
+SHAPES = [(4096, 14336), (14336, 4096)]          # (K, N)
+MS = [1 << i for i in range(13)]                 # 1 .. 4096
+COPIES = 3
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="bi", choices=["bi", "reference"])
+    ap.add_argument("--no-extras", action="store_true", help="skip attention/RMSNorm/cuBLAS legs")
+    ap.add_argument("--case", default=None, choices=["gemm", "gemm_m128", "attn", "rmsnorm"],
+                    help="run 3 launches of one kernel on its workload and exit (for profilers)")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def step_flops():
+    return sum(2.0 * M * N * K for K, N in SHAPES for M in MS)
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling every 200 ms while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+        time.sleep(0.3)
+
+    def stop(self) -> dict:
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.f.read().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.f.name)
+        loaded = [s for s in sm if mx and s > 0.3 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- distributed
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- workloads
+
+class Sweep:
+    def __init__(self, bi, torch):
+        self.bi, self.torch = bi, torch
+        dev = "cuda"
+        g = torch.Generator(dev).manual_seed(0)
+        self.A = {K: torch.randn(4096, K, device=dev, generator=g).to(torch.bfloat16) for K, _ in SHAPES}
+        self.W = {(K, N): [(torch.randn(N, K, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+                           for _ in range(COPIES)] for K, N in SHAPES}
+        self.C = torch.empty(4096 * 14336, dtype=torch.bfloat16, device=dev)
+        self.launches = [(K, N, M) for K, N in SHAPES for M in MS]
+
+    def out(self, M, N):
+        return self.C[: M * N].view(M, N)
+
+    def step(self, i0=0):
+        """One pass of the sweep; weight copy rotates launch by launch."""
+        for j, (K, N, M) in enumerate(self.launches):
+            self.bi.bi_gemm(self.A[K][:M], self.W[(K, N)][(i0 + j) % COPIES], self.out(M, N))
+
+    def torch_step(self, i0=0):
+        for j, (K, N, M) in enumerate(self.launches):
+            self.torch.matmul(self.A[K][:M], self.W[(K, N)][(i0 + j) % COPIES].t(), out=self.out(M, N))
+
+
+def time_graph(torch, fn, steps, warmup, world):
+    """Capture one step in a CUDA graph; replay warmup + timed steps."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(2):
+            fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        fn()
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = e0.elapsed_time(e1)
+    del graph
+    return ms
+
+
+def per_launch_ms(torch, launch, reps):
+    """Device time of one launch (mean over reps), events on the launching stream."""
+    launch()
+    torch.cuda.synchronize()
+    ts = []
+    for r in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        launch(r)
+        e1.record()
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return sum(ts) / len(ts)
+
+
+def sweep_table(torch, sw, reps):
+    rows = []
+    for K, N in SHAPES:
+        for M in MS:
+            W = sw.W[(K, N)]
+            A = sw.A[K][:M]
+            C = sw.out(M, N)
+            bi_ms = per_launch_ms(torch, lambda r=0: sw.bi.bi_gemm(A, W[r % COPIES], C), reps)
+            th_ms = per_launch_ms(torch, lambda r=0: torch.matmul(A, W[r % COPIES].t(), out=C), reps)
+            fl = 2.0 * M * N * K
+            by = 2.0 * (M * K + N * K + M * N)
+            rows.append({"K": K, "N": N, "M": M, "bi_ms": bi_ms, "bi_tflops": fl / bi_ms / 1e9,
+                         "bi_gbs": by / bi_ms / 1e6, "cublas_ms": th_ms,
+                         "cublas_tflops": fl / th_ms / 1e9})
+    return rows
+
+
+def same_bits(a, b) -> bool:
+    import torch
+    return a.shape == b.shape and bool(torch.equal(a.contiguous().view(torch.int16),
+                                                   b.contiguous().view(torch.int16)))
+
+
+def invariance_flags(torch, sw):
+    ok_bi, ok_th = True, True
+    for K, N in SHAPES:
+        W = sw.W[(K, N)][0]
+        full = sw.bi.gemm(sw.A[K], W)
+        th_full = torch.matmul(sw.A[K], W.t())
+        for M in (1, 7, 100, 1000):
+            ok_bi &= same_bits(sw.bi.gemm(sw.A[K][:M], W), full[:M])
+            ok_th &= same_bits(torch.matmul(sw.A[K][:M], W.t()), th_full[:M])
+    return {"bi_gemm_rows_bitwise_across_M": bool(ok_bi), "cublas_rows_bitwise_across_M": bool(ok_th)}
+
+
+def attention_leg(bi, torch, synth, reps):
+    """Decode step over 32 sequences, lengths U[1, 8192] (seed 0), GQA 32/8."""
+    lens = synth.attention_lengths(32, 1, 8192, seed=0)
+    Hq, Hkv, D = 32, 8, 128
+    lay = synth.PagedLayout(lens, seed=0)
+    g = torch.Generator("cuda").manual_seed(1)
+    kc = torch.randn(lay.num_pages, Hkv, 16, D, device="cuda", generator=g).to(torch.bfloat16)
+    vc = torch.randn(lay.num_pages, Hkv, D, 16, device="cuda", generator=g).to(torch.bfloat16)
+    q = torch.randn(32, Hq * D, device="cuda", generator=g).to(torch.bfloat16)
+    shape = bi.attn_shape(Hq, Hkv, lay.num_pages, lay.pages_per_seq, 8192)
+    ws = torch.empty(bi.bi_attn_workspace_size(shape, 32), dtype=torch.uint8, device="cuda")
+    out = torch.empty(32, Hq * D, dtype=torch.bfloat16, device="cuda")
+    bt = lay.block_table.cuda()
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    ms = per_launch_ms(torch, lambda r=0: bi.bi_attn_decode(q, kc, vc, bt, sl, shape, out, ws), reps)
+    kv_bytes = sum(lens) * Hkv * D * 2 * 2
+    return {"workload": "decode, B=32, Hq=32, Hkv=8, d=128, L~U[1,8192] seed 0, page 16",
+            "ms": ms, "kv_bytes": kv_bytes, "gbs": kv_bytes / ms / 1e6}
+
+
+def rmsnorm_leg(bi, torch, reps):
+    M, D = 65536, 4096
+    g = torch.Generator("cuda").manual_seed(2)
+    x = torch.randn(M, D, device="cuda", generator=g).to(torch.bfloat16)
+    gamma = torch.rand(D, device="cuda", generator=g).to(torch.bfloat16)
+    y = torch.empty_like(x)
+    ms = per_launch_ms(torch, lambda r=0: bi.bi_rmsnorm(x, gamma, y, 1e-6), reps)
+    by = 4.0 * M * D + 2 * D
+    return {"workload": "M=65536, D=4096 bf16", "ms": ms, "bytes": by, "gbs": by / ms / 1e6}
+
+
+def e2e_leg(bi, torch, sw, steps):
+    """The same sweep through the C-ABI with HOST buffers: per step, each
+    shape's weights and each launch's A rows go host->device from pinned
+    memory and each C comes back device->host, inside the timed region."""
+    hA = {K: sw.A[K].cpu().pin_memory() for K, _ in SHAPES}
+    hW = {(K, N): sw.W[(K, N)][0].cpu().pin_memory() for K, N in SHAPES}
+    hC = torch.empty(4096 * 14336, dtype=torch.bfloat16).pin_memory()
+    dW = {k: torch.empty_like(v[0]) for k, v in sw.W.items()}
+    dA = {K: torch.empty_like(sw.A[K]) for K, _ in SHAPES}
+    h2d = d2h = 0
+    for K, N in SHAPES:
+        h2d += N * K * 2
+        for M in MS:
+            h2d += M * K * 2
+            d2h += M * N * 2
+
+    def one():
+        for K, N in SHAPES:
+            dW[(K, N)].copy_(hW[(K, N)], non_blocking=True)
+            for M in MS:
+                dA[K][:M].copy_(hA[K][:M], non_blocking=True)
+                C = sw.out(M, N)
+                bi.bi_gemm(dA[K][:M], dW[(K, N)], C)
+                hC[: M * N].view(M, N).copy_(C, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return ms, h2d, d2h
+
+
+def cpu_baseline_leg(target_s=10.0):
+    """The oracle's fp64 GEMM (numpy matmul) on a bounded sample of the sweep
+    workload: the first r rows of A for both shapes, r sized for ~10 s."""
+    import numpy as np
+    import torch
+    from oracle import fp64
+    from invariant_deterministic_03_b200 import synth
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
+    except Exception:
+        threads = os.cpu_count()
+    mats = {}
+    for K, N in SHAPES:
+        W = fp64.bf16_bits_to_f64(synth.bf16_bits(synth.normal_bf16((N, K), 0.02, 7)))
+        A = fp64.bf16_bits_to_f64(synth.bf16_bits(synth.normal_bf16((512, K), 1.0, 8)))
+        mats[(K, N)] = (A, W)
+    rows, spent, flops = 8, 0.0, 0.0
+    t_start = time.perf_counter()
+    while spent < target_s and rows <= 512:
+        t0 = time.perf_counter()
+        for (K, N), (A, W) in mats.items():
+            fp64.gemm(A[:rows], W)
+            flops += 2.0 * rows * N * K
+        spent = time.perf_counter() - t_start
+        rows *= 2
+    return {"value": flops / spent / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"oracle fp64 GEMM (numpy matmul) on the first 8..{rows // 2} rows (doubling) of A for "
+                      f"both sweep shapes, {spent:.1f} s of CPU work"}
+
+
+# --------------------------------------------------------------------------- main
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cb = cpu_baseline_leg(target_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)))
+    line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "gemm sweep, Mistral-7B MLP shapes: M in 1..4096 (powers of 2) x "
+                                   "(K=4096,N=14336) and (K=14336,N=4096); oracle runs a bounded row sample",
+                       "world_size": world},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_case(case):
+    """Three launches of one kernel on its bench workload, nothing else timed:
+    the first two warm up, a profiler captures the third (-s 2 -c 1)."""
+    import torch
+    from invariant_deterministic_03_b200 import bi, synth
+    torch.cuda.set_device(0)
+    g = torch.Generator("cuda").manual_seed(0)
+    if case in ("gemm", "gemm_m128"):
+        M = 4096 if case == "gemm" else 128
+        A = torch.randn(M, 4096, device="cuda", generator=g).to(torch.bfloat16)
+        W = (torch.randn(14336, 4096, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+        C = torch.empty(M, 14336, dtype=torch.bfloat16, device="cuda")
+        fn = lambda: bi.bi_gemm(A, W, C)  # noqa: E731
+    elif case == "attn":
+        lens = synth.attention_lengths(32, 1, 8192, seed=0)
+        lay = synth.PagedLayout(lens, seed=0)
+        kc = torch.randn(lay.num_pages, 8, 16, 128, device="cuda", generator=g).to(torch.bfloat16)
+        vc = torch.randn(lay.num_pages, 8, 128, 16, device="cuda", generator=g).to(torch.bfloat16)
+        q = torch.randn(32, 32 * 128, device="cuda", generator=g).to(torch.bfloat16)
+        shape = bi.attn_shape(32, 8, lay.num_pages, lay.pages_per_seq, 8192)
+        ws = torch.empty(bi.bi_attn_workspace_size(shape, 32), dtype=torch.uint8, device="cuda")
+        out = torch.empty(32, 32 * 128, dtype=torch.bfloat16, device="cuda")
+        bt, sl = lay.block_table.cuda(), torch.tensor(lens, dtype=torch.int32, device="cuda")
+        fn = lambda: bi.bi_attn_decode(q, kc, vc, bt, sl, shape, out, ws)  # noqa: E731
+    else:
+        x = torch.randn(65536, 4096, device="cuda", generator=g).to(torch.bfloat16)
+        gamma = torch.rand(4096, device="cuda", generator=g).to(torch.bfloat16)
+        y = torch.empty_like(x)
+        fn = lambda: bi.bi_rmsnorm(x, gamma, y, 1e-6)  # noqa: E731
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    assert bi.bi_device_status(clear=True) == 0
+    print(f"case {case}: ok")
+    return 0
+
+
+def main():
+    args = parse()
+    if args.case:
+        return run_case(args.case)
+    if args.impl == "reference":
+        return run_reference(args)
+    import torch
+    from invariant_deterministic_03_b200 import bi, synth
+
+    world, rank, local = dist_setup(args.gpus)
+    peaks, peak_src = load_peaks()
+    sw = Sweep(bi, torch)
+    flops = step_flops()
+
+    # ---- timed region: K steps of the sweep (one CUDA graph per step)
+    sampler = ClockSampler(local)
+    sampler.start()
+    it = [0]
+
+    def fn():
+        sw.step(it[0])
+
+    ms_total = time_graph(torch, fn, args.steps, args.warmup, world)
+    clocks = sampler.stop()
+    ms_total = max_over_ranks(ms_total, world)
+    ms_step = ms_total / args.steps
+    value = flops * world / (ms_step * 1e-3) / 1e12
+
+    extras = {}
+    table = sweep_table(torch, sw, reps=5)
+    big = [r for r in table if r["M"] >= 1024]
+    big_fl = sum(2.0 * r["M"] * r["N"] * r["K"] for r in big)
+    big_ms = sum(r["bi_ms"] for r in big)
+    achieved = big_fl / big_ms / 1e9
+    peak_t = peaks.get("bf16_tflops_sustained") or peaks.get("bf16_tflops")
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
+                "frac": achieved / peak_t, "traffic": None,
+                "kernel": "bi_gemm (gemm_tcgen05_kernel), launches with M >= 1024 of the sweep",
+                "peak_source": f"{peak_src} bf16 dense sustained",
+                "frac_of_burst": achieved / peaks.get("bf16_tflops", peak_t)}
+    bi_sum = sum(r["bi_ms"] for r in table)
+    th_sum = sum(r["cublas_ms"] for r in table)
+    extras["sweep"] = [{k: (round(v, 4) if isinstance(v, float) else v) for k, v in r.items()} for r in table]
+    extras["cost_vs_cublas"] = {"bi_sweep_ms": bi_sum, "cublas_sweep_ms": th_sum,
+                                "bi_over_cublas_time": bi_sum / th_sum,
+                                "cublas_tflops": flops / th_sum / 1e9}
+    if not args.no_extras:
+        a = attention_leg(bi, torch, synth, reps=10)
+        a["frac"] = a["gbs"] / peaks["hbm_gbs"]
+        r = rmsnorm_leg(bi, torch, reps=10)
+        r["frac"] = r["gbs"] / peaks["hbm_gbs"]
+        extras["attn_decode"] = a
+        extras["rmsnorm"] = r
+        extras["invariance"] = invariance_flags(torch, sw)
+
+    e2e_ms, h2d, d2h = e2e_leg(bi, torch, sw, steps=max(2, min(args.steps, 5)))
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    launches = len(sw.launches) * args.steps
+
+    cpu = None
+    if rank == 0 and world == 1:
+        cpu = cpu_baseline_leg()
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": "gemm sweep, Mistral-7B MLP shapes: M in {1,2,4,...,4096} x "
+                                       "(K=4096,N=14336) and (K=14336,N=4096), bf16 in, fp32 accum, bf16 out",
+                           "l2": "inputs larger than L2: weights rotate over 3 copies of 117 MB per shape",
+                           "tile": "128x256x64, tcgen05 M128 N256 K16, one tiling for all M",
+                           "parallelism": f"replicas x{world}"},
+                "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
+                "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "gpu_launches": launches}
+        line.update(extras)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

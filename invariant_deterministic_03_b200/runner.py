@@ -1,0 +1,109 @@
+"""Host-side bookkeeping for bi_forward: page allocation, batch assembly and a
+greedy decode loop. Index arithmetic only -- every step of the model runs in
+libbi through :class:`invariant_deterministic_03_b200.bi.Model`.
+
+Pages come from a seeded random permutation of the pool, so a sequence's keys
+sit in non-contiguous pages, as in a serving engine under load.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import bi as _bi
+from . import synth
+
+PAGE = 16
+
+
+class PagedKV:
+    """KV caches for every layer plus the page tables of live sequences."""
+
+    def __init__(self, n_layers: int, num_pages: int, n_kv_heads: int, max_pages_per_seq: int,
+                 seed: int = 0, device="cuda:0", zero=True):
+        self.num_pages = num_pages
+        self.max_pages = max_pages_per_seq
+        self.k, self.v = _bi.new_kv_cache(num_pages, n_kv_heads, device, n_layers, zero=zero)
+        self.free = synth.permutation(num_pages, seed).tolist()
+        self.pages: dict[int, list[int]] = {}
+        self.length: dict[int, int] = {}
+
+    def ensure(self, seq: int, length: int) -> None:
+        pg = self.pages.setdefault(seq, [])
+        self.length.setdefault(seq, 0)
+        while len(pg) * PAGE < length:
+            if not self.free:
+                raise RuntimeError("KV cache out of pages")
+            if len(pg) >= self.max_pages:
+                raise RuntimeError("sequence longer than max_pages_per_seq pages")
+            pg.append(self.free.pop(0))
+
+    def slot(self, seq: int, pos: int) -> int:
+        return self.pages[seq][pos // PAGE] * PAGE + pos % PAGE
+
+    def release(self, seq: int) -> None:
+        self.free.extend(self.pages.pop(seq, []))
+        self.length.pop(seq, None)
+
+
+def make_batch(kv: PagedKV, chunks, tokens_of, device="cuda:0"):
+    """chunks: list of (seq, start, end) -- tokens start..end-1 of `seq` are
+    processed in this step (their keys are written, then attended). The keys
+    0..start-1 must already be cached. Returns the device batch dict for
+    Model.forward with one logits row per chunk (its last token)."""
+    toks, pos, slots, cu, lens, rows = [], [], [], [0], [], []
+    for seq, s, e in chunks:
+        if kv.length.get(seq, 0) != s:
+            raise ValueError(f"sequence {seq}: cache holds {kv.length.get(seq, 0)} keys, chunk starts at {s}")
+        kv.ensure(seq, e)
+        t = tokens_of(seq)
+        for p in range(s, e):
+            toks.append(int(t[p]))
+            pos.append(p)
+            slots.append(kv.slot(seq, p))
+        cu.append(cu[-1] + e - s)
+        lens.append(e)
+        rows.append(cu[-1] - 1)
+    bt = torch.full((len(chunks), kv.max_pages), -1, dtype=torch.int32)
+    for i, (seq, _, _) in enumerate(chunks):
+        pg = kv.pages[seq]
+        bt[i, : len(pg)] = torch.tensor(pg, dtype=torch.int32)
+    i32 = lambda x: torch.tensor(x, dtype=torch.int32, device=device)  # noqa: E731
+    batch = {"tokens": i32(toks), "positions": i32(pos), "slot_mapping": i32(slots),
+             "cu_q": i32(cu), "seq_lens": i32(lens), "block_table": bt.to(device),
+             "logits_rows": i32(rows), "max_q_len": max(e - s for _, s, e in chunks),
+             "max_kv_len": max(lens)}
+    return batch
+
+
+def commit(kv: PagedKV, chunks) -> None:
+    """Record that the chunks' keys are now cached."""
+    for seq, _, e in chunks:
+        kv.length[seq] = e
+
+
+class Engine:
+    """A model, its caches and one reusable workspace."""
+
+    def __init__(self, cfg: dict, weights_dev: dict, num_pages: int, max_pages_per_seq: int,
+                 max_tokens: int, max_logits: int, seed: int = 0, device="cuda:0"):
+        self.cfg = cfg
+        self.model = _bi.Model(cfg, weights_dev)
+        self.kv = PagedKV(cfg["n_layers"], num_pages, cfg["n_kv_heads"], max_pages_per_seq,
+                          seed, device)
+        self.device = device
+        self.max_tokens, self.max_logits = max_tokens, max_logits
+        ws = self.model.workspace_size(max_tokens, max_logits, cfg["max_pos"])
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
+
+    def step(self, chunks, tokens_of):
+        """Runs one forward over the chunks; returns (logits [n_chunks, V]
+        fp32, greedy next tokens [n_chunks] int32), both on the device."""
+        b = make_batch(self.kv, chunks, tokens_of, self.device)
+        if b["tokens"].shape[0] > self.max_tokens or len(chunks) > self.max_logits:
+            raise ValueError("batch larger than the workspace")
+        b["max_kv_len"] = self.cfg["max_pos"]   # fixed bound: sizes grid and workspace only
+        logits = torch.empty(len(chunks), self.cfg["vocab"], dtype=torch.float32, device=self.device)
+        nxt = torch.empty(len(chunks), dtype=torch.int32, device=self.device)
+        self.model.forward(b, self.kv.k, self.kv.v, logits, nxt, self.ws)
+        commit(self.kv, chunks)
+        return logits, nxt

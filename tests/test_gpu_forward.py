@@ -1,0 +1,122 @@
+"""bi_forward on the GPU: logits against the fp64 oracle forward (teacher
+forced), and bitwise equality of a sequence's logits and greedy tokens alone,
+co-batched with other requests, prefilled in different chunk sizes, and across
+runs ("Defeating Nondeterminism in LLM Inference", sections "Batch invariance
+and determinism" and "Batch-invariant attention")."""
+import numpy as np
+import pytest
+import torch
+
+from invariant_deterministic_03_b200 import synth
+from oracle import fp64
+from tests.gpu_common import f64, same_bits
+
+pytestmark = pytest.mark.gpu
+
+SMALL = dict(n_layers=2, d_model=256, n_q_heads=2, n_kv_heads=1, d_ff=384, vocab=512,
+             max_pos=2048, rms_eps=1e-6, rope_theta=1e4)
+MID = dict(n_layers=2, d_model=4096, n_q_heads=32, n_kv_heads=8, d_ff=14336, vocab=32000,
+           max_pos=4096, rms_eps=1e-6, rope_theta=1e4)
+
+
+@pytest.fixture(scope="module")
+def bi(cuda_device):
+    from invariant_deterministic_03_b200 import bi as mod
+    return mod
+
+
+def _engine(cfg, w, pages=4096, seed=0, max_tokens=2048, max_logits=64):
+    from invariant_deterministic_03_b200 import runner
+    wd = {k: v.cuda().contiguous() for k, v in w.items()}
+    return runner.Engine(cfg, wd, num_pages=pages, max_pages_per_seq=cfg["max_pos"] // 16,
+                         max_tokens=max_tokens, max_logits=max_logits, seed=seed), wd
+
+
+def _oracle_weights(cfg, w):
+    return fp64.ModelWeights(cfg, {k: synth.bf16_bits(v) for k, v in w.items()})
+
+
+def _prefill_all_logits(eng, seq, toks, chunk):
+    """Feed toks in chunks; return logits of every position [n, V] (one row
+    per step is the chunk's last token, so chunk=1 gives all positions)."""
+    out = []
+    n = len(toks)
+    for s in range(0, n, chunk):
+        e = min(n, s + chunk)
+        lg, _ = eng.step([(seq, s, e)], lambda _s: toks)
+        out.append(lg)
+    return torch.cat(out)
+
+
+@pytest.mark.parametrize("cfg", [SMALL, MID], ids=["small", "mistral-shape-2-layers"])
+def test_forward_parity_teacher_forced(bi, cfg):
+    w = synth.model_weights(cfg, seed=3)
+    n = 40
+    toks = synth.randint(n, 0, cfg["vocab"] - 1, seed=4).tolist()
+    eng, _ = _engine(cfg, w)
+    lg = _prefill_all_logits(eng, 0, toks, 1)          # decode, one token per step
+    ref = fp64.forward(_oracle_weights(cfg, w), toks)  # [n, V]
+    err = np.abs(f64(lg) - ref)
+    assert err.max() <= 1e-2, f"max abs logit error {err.max():.3e}"
+    assert np.linalg.norm(f64(lg) - ref) <= 2 ** -8 * np.linalg.norm(ref)
+
+
+def test_invariance_chunking_and_cobatching(bi):
+    cfg = MID
+    w = synth.model_weights(cfg, seed=5)
+    n = 300
+    toks = synth.randint(n, 0, cfg["vocab"] - 1, seed=6).tolist()
+    # reference: one token at a time (every step a decode step)
+    eng, wd = _engine(cfg, w, seed=1)
+    per_tok = _prefill_all_logits(eng, 0, toks, 1)
+    for chunk, seed in [(64, 2), (256, 3), (300, 4)]:
+        e2, _ = _engine(cfg, w, seed=seed)
+        lg = _prefill_all_logits(e2, 0, toks, chunk)
+        idx = [min(n, s + chunk) - 1 for s in range(0, n, chunk)]
+        assert same_bits(lg, per_tok[idx]), f"chunk {chunk}"
+    # co-batched with other prompts of random lengths, mixed chunk sizes
+    e3, _ = _engine(cfg, w, seed=7)
+    others = {10 + i: synth.randint(L, 0, cfg["vocab"] - 1, seed=20 + i).tolist()
+              for i, L in enumerate([16, 700, 123, 2000 - 1000])}
+    tok_of = lambda s: toks if s == 0 else others[s]   # noqa: E731
+    got = []
+    pos = {s: 0 for s in [0, *others]}
+    step = 0
+    while pos[0] < n:
+        chunks = []
+        for s in [0, *others]:
+            L = n if s == 0 else len(tok_of(s))
+            if pos[s] >= L:
+                continue
+            size = 1 if s == 0 and step % 3 else [1, 37, 64, 200][(s + step) % 4]
+            chunks.append((s, pos[s], min(L, pos[s] + size)))
+        # put sequence 0 at a varying batch position
+        chunks = chunks[step % len(chunks):] + chunks[: step % len(chunks)]
+        lg, _ = e3.step(chunks, tok_of)
+        for i, (s, a, b) in enumerate(chunks):
+            if s == 0:
+                got.append((b - 1, lg[i]))
+            pos[s] = b
+        step += 1
+    for p, row in got:
+        assert same_bits(row, per_tok[p]), f"position {p}"
+
+
+def test_greedy_generation_run_to_run(bi):
+    cfg = MID
+    w = synth.model_weights(cfg, seed=8)
+    prompt = synth.randint(50, 0, cfg["vocab"] - 1, seed=9).tolist()
+    outs = []
+    for rep in range(2):
+        eng, _ = _engine(cfg, w, seed=rep)
+        toks = list(prompt)
+        lg, nxt = eng.step([(0, 0, len(toks))], lambda s: toks)
+        logits = [lg]
+        for _ in range(16):
+            toks.append(int(nxt[0].item()))
+            lg, nxt = eng.step([(0, len(toks) - 1, len(toks))], lambda s: toks)
+            logits.append(lg)
+        outs.append((toks, torch.cat(logits)))
+        assert int(torch.argmax(lg[0]).item()) == int(nxt[0].item())
+    assert outs[0][0] == outs[1][0]
+    assert same_bits(outs[0][1], outs[1][1])
