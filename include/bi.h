@@ -192,6 +192,34 @@ bi_status bi_attn_decode(const void* q, int64_t ldq, const void* k_cache,
                          const bi_attn_shape* shape, void* out, int64_t ldo,
                          void* ws, size_t ws_bytes, void* stream);
 
+/* Decode without a caller workspace. The paper has no counterpart: this entry
+ * point exists for callers that cannot allocate device memory -- for example
+ * a host application whose own pool owns all device memory and forbids later
+ * allocations, or a latency-critical loop that cannot afford cudaMalloc's
+ * implicit device synchronisation. Same arguments and the same kernels (so
+ * the same bits) as bi_attn_decode, minus ws/ws_bytes.
+ *
+ * The scratch is a fixed array of BI_ATTN_NOALLOC_SCRATCH_BYTES (16 MiB) that
+ * is part of the library's device image: every GPU that loads libbi holds it
+ * until the process exits. A call needs
+ * B * num_q_heads * ceil(max_kv_len / 512) * 520 bytes of it (e.g. 32
+ * sequences x 32 heads x 8192 keys = 8.5 MiB); larger calls fail with
+ * BI_ERR_WORKSPACE and launch nothing. Nothing is allocated: no cudaMalloc,
+ * no cudaFree, no allocating library routine.
+ *
+ * The first call on each device looks the array's device address up with
+ * cudaGetSymbolAddress (with that device current) and caches it; make that
+ * first call before any stream capture. Every call on a device shares the one
+ * array and leaves its contents behind (nothing in it needs to start at
+ * zero), so calls that overlap on the GPU -- on different streams, or from
+ * several host threads -- race on it: order them on one stream. */
+#define BI_ATTN_NOALLOC_SCRATCH_BYTES (16u << 20)
+bi_status bi_attn_decode_noalloc(const void* q, int64_t ldq, const void* k_cache,
+                                 const void* v_cache, const int32_t* block_table,
+                                 const int32_t* seq_lens, int32_t B,
+                                 const bi_attn_shape* shape, void* out, int64_t ldo,
+                                 void* stream);
+
 /* Prefill (chunked): sequence b owns query rows cu_q[b] .. cu_q[b+1]-1
  * (cu_q [B+1] int32 on the device, cu_q[0] = 0, cu_q[B] = n_tok); they are its
  * LAST n_b = cu_q[b+1]-cu_q[b] tokens, so row cu_q[b]+i sits at position

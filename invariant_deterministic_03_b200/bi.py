@@ -76,6 +76,8 @@ _SIGS = {
     "bi_attn_workspace_size": (_i32, [ctypes.POINTER(AttnShape), _i64, ctypes.POINTER(_sz)]),
     "bi_attn_decode": (_i32, [_p, _i64, _p, _p, _p, _p, _i32, ctypes.POINTER(AttnShape), _p,
                               _i64, _p, _sz, _p]),
+    "bi_attn_decode_noalloc": (_i32, [_p, _i64, _p, _p, _p, _p, _i32, ctypes.POINTER(AttnShape),
+                                      _p, _i64, _p]),
     "bi_attn_prefill": (_i32, [_p, _i64, _p, _i32, _i64, _p, _p, _p, _p, _i32,
                                ctypes.POINTER(AttnShape), _p, _i64, _p, _sz, _p]),
     "bi_embed": (_i32, [_p, _i64, _p, _i64, _i64, _p, _p]),
@@ -176,6 +178,16 @@ def bi_attn_decode(q, k_cache, v_cache, block_table, seq_lens, shape: AttnShape,
         _ptr(q), q.stride(0), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens), B,
         ctypes.byref(shape), _ptr(out), out.stride(0), _ptr(ws),
         ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def bi_attn_decode_noalloc(q, k_cache, v_cache, block_table, seq_lens, shape: AttnShape, out,
+                           stream=None) -> None:
+    """bi_attn_decode without a workspace argument: for callers that cannot
+    allocate device memory; uses the library's fixed 16 MiB device scratch."""
+    B = seq_lens.shape[0]
+    _chk("bi_attn_decode_noalloc", lib.bi_attn_decode_noalloc(
+        _ptr(q), q.stride(0), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens), B,
+        ctypes.byref(shape), _ptr(out), out.stride(0), _stream(stream)))
 
 
 def bi_attn_prefill(q, cu_q, max_q_len: int, k_cache, v_cache, block_table, seq_lens,
