@@ -40,14 +40,18 @@ constexpr int SPLIT = BI_ATTN_SPLIT;   // 512 keys
 constexpr int PAGE = BI_PAGE_SIZE;     // 16 keys
 constexpr int PAGES_PER_TILE = TILE / PAGE;
 constexpr uint32_t TILE_BYTES = 128 * 128 * 2;  // 32 KB: Q, K, V and P tiles
-constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_K = TILE_BYTES;          // 2 buffers
-constexpr uint32_t OFF_V = 3 * TILE_BYTES;      // 2 buffers
-constexpr uint32_t OFF_P = 5 * TILE_BYTES;
-constexpr uint32_t OFF_BAR = 6 * TILE_BYTES;
-constexpr size_t SMEM_BYTES = 1024 + 6 * TILE_BYTES + 256;
-constexpr int THREADS = 160;  // warps 0-3: one row each thread; warp 4: TMA + MMA
-constexpr uint32_t TMEM_COLS = 256;  // S at [0,128), PV at [128,256)
+constexpr uint32_t OFF_Q = 0;                   // 2 buffers (one per work item in flight)
+constexpr uint32_t OFF_K = 2 * TILE_BYTES;      // 2 buffers
+constexpr uint32_t OFF_V = 4 * TILE_BYTES;      // 2 buffers
+constexpr uint32_t OFF_P = 6 * TILE_BYTES;
+constexpr uint32_t OFF_BAR = 7 * TILE_BYTES;
+constexpr size_t SMEM_BYTES = 1024 + 7 * TILE_BYTES + 256;
+// warps 0-3: one thread per MMA row (softmax, O rescale, partials)
+// warp 4: TMA producer; warp 5: TMEM allocator and MMA issuer
+constexpr int THREADS = 192;
+// tensor memory: S double buffer at columns [0,128) and [128,256), O at [256,384)
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TMEM_O = 256;
 
 struct Params {
   const int32_t* block_table;
@@ -57,9 +61,49 @@ struct Params {
   float* ws_ml;         // [n_tok, Hq, n_split_max, 2]
   int32_t B, Hq, Hkv, G, QR, qblocks, q_box, n_tok;
   int32_t num_pages, max_pages, max_kv_len, n_split_max;
+  int32_t total_items;
   float scale_log2;
   int32_t* status;
 };
+
+// One unit of work: (split s, sequence b, query block, kv head g).
+struct Item {
+  int s, b, g, r0, nb, L, q_lo, q_hi, key_lo, t0, ntiles;
+};
+
+// Work item idx -> its coordinates; false when it has nothing to do. The kv
+// head varies fastest and the split slowest, so the persistent CTAs first take
+// every sequence's first split and empty items gather at the end.
+__device__ __forceinline__ bool item_at(const Params& p, int idx, Item& it, bool report) {
+  it.g = idx % p.Hkv;
+  int rest = idx / p.Hkv;
+  it.b = rest % p.B;
+  rest /= p.B;
+  const int jb = rest % p.qblocks;
+  it.s = rest / p.qblocks;
+  it.L = p.seq_lens[it.b];
+  if (p.cu_q) {
+    it.r0 = p.cu_q[it.b];
+    it.nb = p.cu_q[it.b + 1] - it.r0;
+  } else {
+    it.r0 = it.b;
+    it.nb = 1;
+  }
+  if (it.nb <= 0 || jb * p.QR >= it.nb) return false;
+  if (it.L < it.nb || it.L > p.max_kv_len || it.r0 < 0 || it.r0 + it.nb > p.n_tok) {
+    if (report && it.s == 0 && jb == 0 && it.g == 0) set_status(p.status, BI_DEV_BAD_SEQLEN);
+    return false;
+  }
+  it.q_lo = jb * p.QR;
+  it.q_hi = min(it.nb, it.q_lo + p.QR);
+  const int p_last = it.L - it.nb + it.q_hi - 1;
+  it.key_lo = it.s * SPLIT;
+  if (it.key_lo > p_last) return false;
+  const int key_hi = min((it.s + 1) * SPLIT, p_last + 1);  // exclusive
+  it.t0 = it.key_lo / TILE;
+  it.ntiles = (key_hi - 1) / TILE - it.t0 + 1;
+  return true;
+}
 
 __device__ __forceinline__ void load_kv_tile(const Params& p, const CUtensorMap* tmK,
                                              const CUtensorMap* tmV, uint8_t* kbuf, uint8_t* vbuf,
@@ -106,82 +150,82 @@ __device__ __forceinline__ void issue_s(uint32_t tmem_s, uint32_t q_addr, uint32
   }
 }
 
-__device__ __forceinline__ void issue_pv(uint32_t tmem_pv, uint32_t p_addr, uint32_t v_addr) {
+// O (+)= P V: accumulate = 0 on the first tile of a split, 1 after.
+__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t p_addr, uint32_t v_addr,
+                                         bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
 #pragma unroll
   for (int j = 0; j < PAGES_PER_TILE; ++j) {
     const uint32_t poff = (j >> 2) * 16384 + (j & 3) * 32;
     // V^T page block j: [128 d rows x 16 keys], 32-byte rows, 32-byte swizzle,
     // 8-row groups 256 bytes apart.
-    mma_bf16(tmem_pv, smem_desc(p_addr + poff, 16, 1024, 2),
-             smem_desc(v_addr + j * 4096, 16, 256, 6), idesc, j != 0);
+    mma_bf16(tmem_o, smem_desc(p_addr + poff, 16, 1024, 2),
+             smem_desc(v_addr + j * 4096, 16, 256, 6), idesc, (accumulate || j != 0) ? 1u : 0u);
   }
 }
 
+// Bounded wait for the fills a producer issued into a buffer, so that no copy
+// is still landing in shared memory when an aborted CTA exits.
+__device__ __forceinline__ void drain(uint64_t* bar, int fills) {
+  if (fills <= 0) return;
+  const uint32_t parity = (uint32_t)(fills - 1) & 1u;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity) && clock64() - t0 < kWaitLimitCycles) {
+  }
+}
+
+// Split kernel. Persistent: one CTA per SM walks work items idx = blockIdx.x,
+// blockIdx.x + gridDim.x, ...; the three roles walk the same item sequence.
+// Per tile j (counted across items) the MMA warp issues S(j) = Q K_j^T into
+// S buffer j%2 before P(j-1) V_(j-1), so the next QK^T overlaps the softmax of
+// the current tile.
+//
+// Row arithmetic (thread = row, fixed order, same in decode and prefill):
+//   first tile of the split:  m = max_j s_j (log2 domain, s_j = S_ij * scale*log2e),
+//                             P_j = bf16(2^(s_j - m)), l = sum_j P_j, O = P V
+//   later tiles:              m' = max(m, max_j s_j), alpha = 2^(m - m'),
+//                             P_j = bf16(2^(s_j - m')), l = alpha*l + sum_j P_j,
+//                             O = alpha*O (fp32, skipped when alpha == 1), O += P V (MMA)
+// sums over j run j = 0..127 in order; masked keys have P_j = 0 by selection.
 __global__ void __launch_bounds__(THREADS, 1)
     attn_split_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const Params p) {
-  const int s = blockIdx.x;
-  const int b = blockIdx.y / p.qblocks;
-  const int jb = blockIdx.y % p.qblocks;
-  const int g = blockIdx.z;
-
-  // ---- which queries and keys this CTA covers (uniform across the CTA)
-  const int L = p.seq_lens[b];
-  int r0, nb;
-  if (p.cu_q) {
-    r0 = p.cu_q[b];
-    nb = p.cu_q[b + 1] - r0;
-  } else {
-    r0 = b;
-    nb = 1;
-  }
-  if (nb <= 0 || jb * p.QR >= nb) return;
-  if (L < nb || L > p.max_kv_len || r0 < 0 || r0 + nb > p.n_tok) {
-    if (threadIdx.x == 0 && s == 0 && g == 0) set_status(p.status, BI_DEV_BAD_SEQLEN);
-    return;
-  }
-  const int q_lo = jb * p.QR;
-  const int q_hi = min(nb, q_lo + p.QR);
-  const int p_last = L - nb + q_hi - 1;
-  const int key_lo = s * SPLIT;
-  if (key_lo > p_last) return;
-  const int key_hi = min((s + 1) * SPLIT, p_last + 1);  // exclusive
-  const int t0 = key_lo / TILE;
-  const int ntiles = (key_hi - 1) / TILE - t0 + 1;
-
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [2]
-  uint64_t* v_full = bars + 3;    // [2]
-  uint64_t* kv_empty = bars + 5;  // [2]
-  uint64_t* s_full = bars + 7;
-  uint64_t* p_ready = bars + 8;
-  uint64_t* o_full = bars + 9;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+  uint64_t* q_full = bars + 0;     // [2]
+  uint64_t* q_empty = bars + 2;    // [2]
+  uint64_t* k_full = bars + 4;     // [2]
+  uint64_t* v_full = bars + 6;     // [2]
+  uint64_t* kv_empty = bars + 8;   // [2]
+  uint64_t* s_full = bars + 10;    // [2]
+  uint64_t* s_free = bars + 12;    // [2]
+  uint64_t* p_ready = bars + 14;
+  uint64_t* o_ready = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
       mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
     }
-    mbar_init(s_full, 1);
     mbar_init(p_ready, 128);
-    mbar_init(o_full, 1);
+    mbar_init(o_ready, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 4) {
+  if (warp == 5) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
@@ -189,174 +233,237 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_s = tmem;
-  const uint32_t tmem_pv = tmem + 128;
-  const uint32_t sQ = smem_u32(smem + OFF_Q);
-  const uint32_t sK[2] = {smem_u32(smem + OFF_K), smem_u32(smem + OFF_K + TILE_BYTES)};
-  const uint32_t sV[2] = {smem_u32(smem + OFF_V), smem_u32(smem + OFF_V + TILE_BYTES)};
-  const uint32_t sP = smem_u32(smem + OFF_P);
 
   if (warp == 4) {
-    // ------------------------------------------------ TMA + MMA control thread
+    // ------------------------------------------------ TMA producer
     if (lane == 0) {
-      bool ok = true;
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
       const uint32_t q_bytes = 2u * 64u * 2u * (uint32_t)(p.G * p.q_box);
-      mbar_arrive_expect_tx(q_full, q_bytes);
-      tma_load_3d(smem + OFF_Q, &tmQ, q_full, 0, g * p.G, r0 + q_lo);
-      tma_load_3d(smem + OFF_Q + 16384, &tmQ, q_full, 64, g * p.G, r0 + q_lo);
-      load_kv_tile(p, &tmK, &tmV, smem + OFF_K, smem + OFF_V, &k_full[0], &v_full[0], b, g, L, t0);
-      if (ntiles > 1)
-        load_kv_tile(p, &tmK, &tmV, smem + OFF_K + TILE_BYTES, smem + OFF_V + TILE_BYTES,
-                     &k_full[1], &v_full[1], b, g, L, t0 + 1);
-      ok = mbar_wait(q_full, 0, p.status, abort_flag) &&
-           mbar_wait(&k_full[0], 0, p.status, abort_flag);
-      if (ok) {
-        tc_fence_after();
-        issue_s(tmem_s, sQ, sK[0]);
-        mma_commit(s_full);
+      int qi = 0, kvi = 0;
+      int q_fills[2] = {0, 0}, kv_fills[2] = {0, 0};
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < p.total_items && ok; idx += gridDim.x) {
+        Item it;
+        if (!item_at(p, idx, it, true)) continue;
+        const int qb = qi & 1;
+        if (!mbar_wait(&q_empty[qb], (((uint32_t)qi >> 1) & 1u) ^ 1u, p.status, abort_flag)) { ok = false; break; }
+        uint8_t* qdst = smem + OFF_Q + qb * TILE_BYTES;
+        mbar_arrive_expect_tx(&q_full[qb], q_bytes);
+        tma_load_3d(qdst, &tmQ, &q_full[qb], 0, it.g * p.G, it.r0 + it.q_lo);
+        tma_load_3d(qdst + 16384, &tmQ, &q_full[qb], 64, it.g * p.G, it.r0 + it.q_lo);
+        ++q_fills[qb];
+        ++qi;
+        for (int t = 0; t < it.ntiles; ++t) {
+          const int kb = kvi & 1;
+          if (!mbar_wait(&kv_empty[kb], (((uint32_t)kvi >> 1) & 1u) ^ 1u, p.status, abort_flag)) { ok = false; break; }
+          load_kv_tile(p, &tmK, &tmV, smem + OFF_K + kb * TILE_BYTES, smem + OFF_V + kb * TILE_BYTES,
+                       &k_full[kb], &v_full[kb], it.b, it.g, it.L, it.t0 + t);
+          ++kv_fills[kb];
+          ++kvi;
+        }
       }
-      for (int i = 0; i < ntiles && ok; ++i) {
-        const int buf = i & 1;
-        const uint32_t use_par = (uint32_t)(i >> 1) & 1u;
-        if (!mbar_wait(p_ready, (uint32_t)i & 1u, p.status, abort_flag)) break;
-        if (!mbar_wait(&v_full[buf], use_par, p.status, abort_flag)) break;
+      if (!ok) {
+        for (int i = 0; i < 2; ++i) {
+          drain(&q_full[i], q_fills[i]);
+          drain(&k_full[i], kv_fills[i]);
+          drain(&v_full[i], kv_fills[i]);
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------ MMA issuer (one thread)
+    if (lane == 0) {
+      const uint32_t sQ0 = smem_u32(smem + OFF_Q), sK0 = smem_u32(smem + OFF_K);
+      const uint32_t sV0 = smem_u32(smem + OFF_V), sP = smem_u32(smem + OFF_P);
+      int qi = 0, j = 0;
+      bool ok = true;
+      // P V of the previous tile, issued after the next tile's QK^T
+      bool pend = false, pend_acc = false, pend_last = false;
+      int pend_j = 0, pend_qb = 0;
+      auto issue_pending = [&]() -> bool {
+        const int kb = pend_j & 1;
+        if (!mbar_wait(p_ready, (uint32_t)pend_j & 1u, p.status, abort_flag)) return false;
+        if (!mbar_wait(&v_full[kb], ((uint32_t)pend_j >> 1) & 1u, p.status, abort_flag)) return false;
         tc_fence_after();
-        issue_pv(tmem_pv, sP, sV[buf]);
-        mma_commit(o_full);
-        mma_commit(&kv_empty[buf]);
-        if (i + 1 < ntiles) {
-          const int nbuf = buf ^ 1;
-          if (!mbar_wait(&k_full[nbuf], (uint32_t)((i + 1) >> 1) & 1u, p.status, abort_flag)) break;
+        issue_pv(tmem + TMEM_O, sP, sV0 + kb * TILE_BYTES, pend_acc);
+        mma_commit(o_ready);
+        mma_commit(&kv_empty[kb]);
+        if (pend_last) mma_commit(&q_empty[pend_qb]);
+        pend = false;
+        return true;
+      };
+      for (int idx = blockIdx.x; idx < p.total_items && ok; idx += gridDim.x) {
+        Item it;
+        if (!item_at(p, idx, it, false)) continue;
+        const int qb = qi & 1;
+        if (!mbar_wait(&q_full[qb], ((uint32_t)qi >> 1) & 1u, p.status, abort_flag)) { ok = false; break; }
+        for (int t = 0; t < it.ntiles; ++t, ++j) {
+          const int kb = j & 1;
+          if (!mbar_wait(&k_full[kb], ((uint32_t)j >> 1) & 1u, p.status, abort_flag) ||
+              !mbar_wait(&s_free[kb], (((uint32_t)j >> 1) & 1u) ^ 1u, p.status, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          issue_s(tmem_s, sQ, sK[nbuf]);
-          mma_commit(s_full);
+          issue_s(tmem + kb * 128, sQ0 + qb * TILE_BYTES, sK0 + kb * TILE_BYTES);
+          mma_commit(&s_full[kb]);
+          if (pend && !issue_pending()) { ok = false; break; }
+          pend = true;
+          pend_j = j;
+          pend_acc = t > 0;
+          pend_last = t == it.ntiles - 1;
+          pend_qb = qb;
         }
-        if (i + 2 < ntiles) {
-          if (!mbar_wait(&kv_empty[buf], use_par, p.status, abort_flag)) break;
-          load_kv_tile(p, &tmK, &tmV, smem + OFF_K + buf * TILE_BYTES,
-                       smem + OFF_V + buf * TILE_BYTES, &k_full[buf], &v_full[buf], b, g, L,
-                       t0 + i + 2);
-        }
+        ++qi;
       }
+      if (ok && pend) issue_pending();
     }
   } else {
     // ------------------------------------------------ one thread per MMA row
     const int r = threadIdx.x;  // 0..127 == TMEM lane
-    const int qi = r / p.G;
-    const int hj = r - qi * p.G;
-    const int q_idx = q_lo + qi;
-    const int pos = L - nb + q_idx;
-    const bool row_active = (q_idx < q_hi) && (pos >= key_lo);
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    // partial last page: slots >= L of the page holding key L-1 are zeroed in V
-    const int last_page = (L - 1) / PAGE;
-    const int tail = L % PAGE;
-
-    float m = -INFINITY, l = 0.0f;
-    float O[HD];
+    const int qr = r / p.G;
+    const int hj = r - qr * p.G;
+    int j = 0;
+    bool ok = true;
+    bool o_pending = false;  // o_ready of tile j-1 not yet waited for
+    for (int idx = blockIdx.x; idx < p.total_items && ok; idx += gridDim.x) {
+      Item it;
+      if (!item_at(p, idx, it, false)) continue;
+      const int q_idx = it.q_lo + qr;
+      const int pos = it.L - it.nb + q_idx;
+      const bool row_valid = (q_idx < it.q_hi) && (pos >= it.key_lo);
+      const bool warp_valid = __any_sync(0xffffffffu, row_valid);
+      const int last_page = (it.L - 1) / PAGE;
+      const int tail = it.L % PAGE;
+      float m = -INFINITY, l = 0.0f;
+      for (int t = 0; t < it.ntiles; ++t, ++j) {
+        const int sb = j & 1;
+        const int kb0 = (it.t0 + t) * TILE;
+        const bool need = row_valid && kb0 <= pos;
+        if (!mbar_wait(&s_full[sb], ((uint32_t)j >> 1) & 1u, p.status, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t S[128];
+        if (warp_valid) {
 #pragma unroll
-    for (int d = 0; d < HD; ++d) O[d] = 0.0f;
-
-    for (int i = 0; i < ntiles; ++i) {
-      const int buf = i & 1;
-      const int kb = (t0 + i) * TILE;
-      const bool need = row_active && kb <= pos;
-      const bool warp_need = __any_sync(0xffffffffu, need);
-      float alpha = 1.0f;
-      if (!mbar_wait(s_full, (uint32_t)i & 1u, p.status, abort_flag)) break;
-      tc_fence_after();
-      if (warp_need) {
-        const int nvalid = need ? min(TILE, pos + 1 - kb) : 0;
-        float m_tile = -INFINITY;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t rr[32];
-          tmem_ld32(tmem_s + lane_off + q * 32, rr);
+          for (int q = 0; q < 4; ++q)
+            tmem_ld32(tmem + sb * 128 + lane_off + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&S[q * 32]));
           tmem_ld_wait();
-#pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (q * 32 + c < nvalid) m_tile = fmaxf(m_tile, __fmul_rn(__uint_as_float(rr[c]), p.scale_log2));
         }
-        const float m_new = need ? fmaxf(m, m_tile) : 0.0f;
-        if (need) alpha = exp2f(__fsub_rn(m, m_new));
+        tc_fence_before();
+        mbar_arrive(&s_free[sb]);
+
+        float alpha = 1.0f, m_new = 0.0f;
+        // P is packed (2 bf16 per word) into S[0..63] as S is consumed
+        uint32_t* P = S;
         float lsum = 0.0f;
+        if (warp_valid) {
+          const int nvalid = need ? min(TILE, pos + 1 - kb0) : 0;
+          float m_tile = -INFINITY;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t rr[32];
-          tmem_ld32(tmem_s + lane_off + q * 32, rr);
-          tmem_ld_wait();
+          for (int c = 0; c < 128; ++c)
+            if (c < nvalid) m_tile = fmaxf(m_tile, __fmul_rn(__uint_as_float(S[c]), p.scale_log2));
+          if (need) {
+            m_new = fmaxf(m, m_tile);
+            alpha = exp2f(__fsub_rn(m, m_new));
+          }
 #pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) {
-            uint32_t pk[4];
+          for (int c2 = 0; c2 < 64; ++c2) {
+            float pf[2];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float pf[2];
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const int c = q * 32 + c8 * 8 + e * 2 + h;
-                const float sv = __fmul_rn(__uint_as_float(rr[c8 * 8 + e * 2 + h]), p.scale_log2);
-                const float ev = (c < nvalid) ? exp2f(__fsub_rn(sv, m_new)) : 0.0f;
-                const bf16 pb = __float2bfloat16_rn(ev);
-                pf[h] = __bfloat162float(pb);
-                lsum = __fadd_rn(lsum, pf[h]);
-              }
-              pk[e] = pack_bf16x2(pf[0], pf[1]);  // exact: pf are bf16 values
+            for (int h = 0; h < 2; ++h) {
+              const int c = 2 * c2 + h;
+              const float sv = __fmul_rn(__uint_as_float(S[c]), p.scale_log2);
+              const float ev = (c < nvalid) ? exp2f(__fsub_rn(sv, m_new)) : 0.0f;
+              pf[h] = __bfloat162float(__float2bfloat16_rn(ev));
+              lsum = __fadd_rn(lsum, pf[h]);
             }
-            // key chunk (8 keys) index 0..15 -> half, 16-byte slot, swizzled by row
-            const int chunk = q * 4 + c8;
+            P[c2] = pack_bf16x2(pf[0], pf[1]);  // exact: pf are bf16 values
+          }
+          if (need) {
+            l = (t == 0) ? lsum : __fadd_rn(__fmul_rn(alpha, l), lsum);
+            m = m_new;
+          }
+        }
+        // P V of the previous tile must be done before P and O are touched
+        if (o_pending) {
+          if (!mbar_wait(o_ready, (uint32_t)(j - 1) & 1u, p.status, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          o_pending = false;
+        }
+        if (warp_valid) {
+#pragma unroll
+          for (int chunk = 0; chunk < 16; ++chunk) {
+            // 8 keys per 16-byte chunk; 128-byte swizzle within each 64-key half
             const uint32_t addr = (uint32_t)(chunk >> 3) * 16384u + (uint32_t)r * 128u +
                                   (uint32_t)(((chunk & 7) ^ (r & 7)) << 4);
-            *reinterpret_cast<uint4*>(smem + OFF_P + addr) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(smem + OFF_P + addr) =
+                make_uint4(P[4 * chunk], P[4 * chunk + 1], P[4 * chunk + 2], P[4 * chunk + 3]);
+          }
+          // rescale O in tensor memory (not on the split's first tile, whose P V overwrites O)
+          if (t > 0 && __any_sync(0xffffffffu, need && alpha != 1.0f)) {
+            const float a = need ? alpha : 1.0f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint32_t o[32];
+              tmem_ld32(tmem + TMEM_O + lane_off + q * 32, o);
+              tmem_ld_wait();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__fmul_rn(__uint_as_float(o[c]), a));
+              tmem_st32(tmem + TMEM_O + lane_off + q * 32, o);
+            }
+            tmem_st_wait();
           }
         }
-        if (need) {
-          l = __fadd_rn(__fmul_rn(alpha, l), lsum);
-          m = m_new;
+        // zero V slots at or past the sequence end inside this tile's last page
+        if (tail != 0 && last_page / PAGES_PER_TILE == it.t0 + t) {
+          if (!mbar_wait(&v_full[sb], ((uint32_t)j >> 1) & 1u, p.status, abort_flag)) { ok = false; break; }
+          uint8_t* vblk = smem + OFF_V + sb * TILE_BYTES + (last_page % PAGES_PER_TILE) * 4096;
+          const int d = r;  // V^T row
+          for (int slot = tail; slot < PAGE; ++slot) {
+            const uint32_t off = (uint32_t)d * 32u + ((uint32_t)((slot >> 3) ^ ((d >> 2) & 1)) << 4) +
+                                 (uint32_t)(slot & 7) * 2u;
+            *reinterpret_cast<uint16_t*>(vblk + off) = 0;
+          }
         }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(p_ready);
+        o_pending = true;
       }
-      // zero V slots at or past the sequence end inside this tile's last page
-      if (tail != 0 && last_page / PAGES_PER_TILE == t0 + i) {
-        if (!mbar_wait(&v_full[buf], (uint32_t)(i >> 1) & 1u, p.status, abort_flag)) break;
-        uint8_t* vblk = smem + OFF_V + buf * TILE_BYTES + (last_page % PAGES_PER_TILE) * 4096;
-        const int d = r;  // V^T row
-        for (int slot = tail; slot < PAGE; ++slot) {
-          const uint32_t off = (uint32_t)d * 32u + ((uint32_t)((slot >> 3) ^ ((d >> 2) & 1)) << 4) +
-                               (uint32_t)(slot & 7) * 2u;
-          *reinterpret_cast<uint16_t*>(vblk + off) = 0;
-        }
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(p_ready);
-      if (!mbar_wait(o_full, (uint32_t)i & 1u, p.status, abort_flag)) break;
+      if (!ok) break;
+      // end of the split: unnormalised O, m, l of every valid row
+      if (!mbar_wait(o_ready, (uint32_t)(j - 1) & 1u, p.status, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      if (warp_need) {
+      o_pending = false;
+      if (warp_valid) {
+        float* dst = nullptr;
+        if (row_valid) {
+          const size_t widx = ((size_t)(it.r0 + q_idx) * p.Hq + (size_t)(it.g * p.G + hj)) * p.n_split_max + it.s;
+          dst = p.ws_o + widx * HD;
+          *reinterpret_cast<float2*>(p.ws_ml + widx * 2) = make_float2(m, l);
+        }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          uint32_t rr[32];
-          tmem_ld32(tmem_pv + lane_off + q * 32, rr);
+          uint32_t o[32];
+          tmem_ld32(tmem + TMEM_O + lane_off + q * 32, o);
           tmem_ld_wait();
-          if (need) {
+          if (row_valid) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) O[q * 32 + c] = __fmaf_rn(alpha, O[q * 32 + c], __uint_as_float(rr[c]));
+            for (int c4 = 0; c4 < 8; ++c4)
+              reinterpret_cast<float4*>(dst + q * 32)[c4] =
+                  make_float4(__uint_as_float(o[4 * c4]), __uint_as_float(o[4 * c4 + 1]),
+                              __uint_as_float(o[4 * c4 + 2]), __uint_as_float(o[4 * c4 + 3]));
           }
         }
       }
-    }
-    if (row_active && !*abort_flag) {
-      const size_t idx = ((size_t)(r0 + q_idx) * p.Hq + (size_t)(g * p.G + hj)) * p.n_split_max + s;
-      float4* dst = reinterpret_cast<float4*>(p.ws_o + idx * HD);
-#pragma unroll
-      for (int d4 = 0; d4 < HD / 4; ++d4)
-        dst[d4] = make_float4(O[4 * d4], O[4 * d4 + 1], O[4 * d4 + 2], O[4 * d4 + 3]);
-      *reinterpret_cast<float2*>(p.ws_ml + idx * 2) = make_float2(m, l);
+      tc_fence_before();
     }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 4) {
+  if (warp == 5) {
     __syncwarp();
     tmem_dealloc(tmem, TMEM_COLS);
   }
@@ -467,8 +574,8 @@ static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t ma
   const int QR = 128 / G;
   const int qblocks = cu_q ? (max_q_len + QR - 1) / QR : 1;
   if (cu_q && max_q_len <= 0) return fail(BI_ERR_SHAPE, "attention: max_q_len must be positive");
-  if ((int64_t)B * qblocks > 65535) return fail(BI_ERR_SHAPE, "attention: B * ceil(max_q_len / %d) above 65535", QR);
-  if (n_split > 65535) return fail(BI_ERR_SHAPE, "attention: max_kv_len too large");
+  const int64_t total_items = (int64_t)n_split * B * qblocks * sh->num_kv_heads;
+  if (total_items > 0x7fffffffll) return fail(BI_ERR_SHAPE, "attention: too many work items");
   if (n_tok > 0x7fffffffll / Hq) return fail(BI_ERR_SHAPE, "attention: too many tokens");
   const size_t need = ws_bytes_for(n_tok, Hq, n_split);
   if (!ws || ws_bytes < need) return fail(BI_ERR_WORKSPACE, "attention: workspace %zu bytes < %zu needed", ws_bytes, need);
@@ -517,6 +624,7 @@ static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t ma
   p.max_pages = sh->max_pages_per_seq;
   p.max_kv_len = sh->max_kv_len;
   p.n_split_max = n_split;
+  p.total_items = (int32_t)total_items;
   p.scale_log2 = (float)((double)sh->scale * 1.4426950408889634);  // scale * log2(e)
   p.status = status_word();
 
@@ -529,7 +637,8 @@ static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t ma
     if (e != cudaSuccess) return cuda_fail(e, "attention: smem attribute");
     attr_set[dev & 63] = true;
   }
-  dim3 grid(n_split, B * qblocks, sh->num_kv_heads);
+  const int sms = num_sms();
+  const int grid = (int)(total_items < sms ? total_items : sms);
   attn_split_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
   BI_CHECK_LAUNCH("attention split launch");
 

@@ -48,8 +48,17 @@ def _prefill_all_logits(eng, seq, toks, chunk):
     return torch.cat(out)
 
 
-@pytest.mark.parametrize("cfg", [SMALL, MID], ids=["small", "mistral-shape-2-layers"])
-def test_forward_parity_teacher_forced(bi, cfg):
+# bf16 activations: max |logit - fp64| measured 0.0748 on B200 for MID (40
+# tokens, teacher forced) and 0.0758 by a CPU emulation that rounds the fp64
+# forward to bf16 at the same points, so the gap is the bf16 activation
+# rounding itself; each single rounding point alone exceeds 1e-2 at this
+# width. These bounds guard that level (a real bug moves logits by O(1)).
+BF16_BOUNDS = {"small": (1e-2, 2.0 ** -8), "mistral-shape-2-layers": (0.12, 2.0 ** -5)}
+
+
+@pytest.mark.parametrize("cfg,name", [(SMALL, "small"), (MID, "mistral-shape-2-layers")],
+                         ids=["small", "mistral-shape-2-layers"])
+def test_forward_bf16_vs_fp64_teacher_forced(bi, cfg, name):
     w = synth.model_weights(cfg, seed=3)
     n = 40
     toks = synth.randint(n, 0, cfg["vocab"] - 1, seed=4).tolist()
@@ -57,8 +66,9 @@ def test_forward_parity_teacher_forced(bi, cfg):
     lg = _prefill_all_logits(eng, 0, toks, 1)          # decode, one token per step
     ref = fp64.forward(_oracle_weights(cfg, w), toks)  # [n, V]
     err = np.abs(f64(lg) - ref)
-    assert err.max() <= 1e-2, f"max abs logit error {err.max():.3e}"
-    assert np.linalg.norm(f64(lg) - ref) <= 2 ** -8 * np.linalg.norm(ref)
+    max_abs, grel = BF16_BOUNDS[name]
+    assert err.max() <= max_abs, f"max abs logit error {err.max():.3e}"
+    assert np.linalg.norm(f64(lg) - ref) <= grel * np.linalg.norm(ref)
 
 
 def test_invariance_chunking_and_cobatching(bi):
