@@ -271,9 +271,56 @@ bi_status bi_argmax(const float* logits, int64_t rows, int64_t V, int64_t ld,
                     int32_t* idx, void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* fp32-activation ("upcast") steps. The cross-vendor logit-mismatch paper
+ * (arXiv 2610.05458, abstract) reports that upcasting to FP32 reduces logit
+ * differences at ~3x runtime and that keeping only the MLP in BF16 keeps most
+ * of the gain at ~1.3x. In these steps an fp32 activation that feeds a GEMM is
+ * carried as a bf16 pair hi = bf16(x), lo = bf16(x - hi) (~16 significant
+ * bits); everything else stays fp32. Same batch-invariance rules as above. */
+
+/* C = (A_hi + A_lo) W^T: both terms meet the same bf16 W tile; per output
+ * element, each 64-wide K stage adds its 4 hi K-steps then its 4 lo K-steps,
+ * stages in K order. One fixed configuration for every shape (128 x 256
+ * tile). Same constraints as bi_gemm; A_hi and A_lo share lda. */
+bi_status bi_gemm_x2(const void* A_hi, const void* A_lo, int64_t lda,
+                     const void* W, int64_t ldw, void* C, int64_t ldc,
+                     int32_t c_dtype, int64_t M, int64_t N, int64_t K,
+                     void* stream);
+
+/* RMSNorm of fp32 rows (same fixed reduction order as bi_rmsnorm) written as
+ * a bf16 pair: v = x r gamma in fp32, y_hi = bf16(v), y_lo = bf16(v - y_hi). */
+bi_status bi_rmsnorm_split(const float* x, const void* gamma, void* y_hi,
+                           void* y_lo, int64_t M, int64_t D, float eps,
+                           void* stream);
+
+/* hi[i] = bf16(x[i]), lo[i] = bf16(x[i] - hi[i]) for n fp32 values. */
+bi_status bi_split_bf16x2(const float* x, int64_t n, void* hi, void* lo,
+                          void* stream);
+
+/* fp32 attention over an fp32 paged cache (k and v both
+ * [num_pages, num_kv_heads, 16, 128] fp32). cu_q as in bi_attn_prefill, or
+ * NULL for decode (n_tok == B, row b = sequence b). One warp per (query, q
+ * head, 512-key split): s_j = (q . k_j) scale (lane partial sums over d,
+ * then a shuffle-down tree), p_j = exp(s_j - max), l and O summed over keys
+ * in order; splits merged in order as in bi_attn_prefill. q, out fp32. */
+bi_status bi_attn_f32_workspace_size(const bi_attn_shape* shape,
+                                     int64_t max_tokens, size_t* bytes);
+bi_status bi_attn_f32(const float* q, int64_t ldq, const int32_t* cu_q,
+                      int64_t n_tok, const float* k_cache, const float* v_cache,
+                      const int32_t* block_table, const int32_t* seq_lens,
+                      int32_t B, const bi_attn_shape* shape, float* out,
+                      int64_t ldo, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* Dense decoder forward (pre-norm, RMSNorm, RoPE, GQA attention, SwiGLU MLP),
  * composed only of the kernels above, with an fp32 residual stream and fp32
- * logits. */
+ * logits. precision selects the activation path:
+ *   BI_PREC_BF16      bf16 activations, bf16 KV cache (bi_kv_layout)
+ *   BI_PREC_F32       fp32 activations everywhere, fp32 KV cache
+ *   BI_PREC_BF16_MLP  fp32 activations except the MLP block, fp32 KV cache */
+#define BI_PREC_BF16 0
+#define BI_PREC_F32 1
+#define BI_PREC_BF16_MLP 2
 typedef struct {
   int32_t n_layers;
   int32_t d_model;     /* D */
@@ -284,6 +331,7 @@ typedef struct {
   int32_t max_pos;     /* positions < max_pos */
   float rms_eps;
   double rope_theta;
+  int32_t precision; /* BI_PREC_* */
 } bi_model_config;
 
 /* Caller-owned device weights, bf16, nn.Linear layout [out, in]. Per layer l
@@ -339,8 +387,9 @@ bi_status bi_forward_workspace_size(const bi_model* m, int64_t max_tokens,
                                     int64_t max_logits, int32_t max_kv_len,
                                     size_t* bytes);
 
-/* k_cache / v_cache: layout bi_kv_layout with num_layers consecutive caches,
- * layer l at offset l * num_pages * Hkv * 16 * 128 elements. logits
+/* k_cache / v_cache: num_layers consecutive caches, layer l at offset
+ * l * num_pages * Hkv * 16 * 128 elements; bf16 in bi_kv_layout for
+ * BI_PREC_BF16, fp32 [num_pages, Hkv, 16, 128] (k and v alike) otherwise. logits
  * [n_logits, V] fp32; next_tokens [n_logits] int32 (nullable) = greedy argmax. */
 bi_status bi_forward(const bi_model* m, const bi_batch* batch, void* k_cache,
                      void* v_cache, int32_t num_pages, float* logits,

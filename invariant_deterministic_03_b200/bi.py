@@ -30,6 +30,8 @@ lib = ctypes.CDLL(LIB_PATH)
 BI_OK, BI_ERR_INVALID_ARG, BI_ERR_SHAPE, BI_ERR_ALIGN, BI_ERR_WORKSPACE, \
     BI_ERR_UNSUPPORTED, BI_ERR_CUDA, BI_ERR_DEVICE_CHECK = range(8)
 BI_BF16, BI_F32 = 0, 1
+BI_PREC_BF16, BI_PREC_F32, BI_PREC_BF16_MLP = 0, 1, 2
+PRECISIONS = {"bf16": BI_PREC_BF16, "f32": BI_PREC_F32, "bf16_mlp": BI_PREC_BF16_MLP}
 HEAD_DIM, PAGE_SIZE, ATTN_TILE, ATTN_SPLIT = 128, 16, 128, 512
 GEMM_BM, GEMM_BN, GEMM_BK = 128, 256, 64
 
@@ -51,7 +53,7 @@ class AttnShape(ctypes.Structure):
 class ModelConfig(ctypes.Structure):
     _fields_ = [("n_layers", _i32), ("d_model", _i32), ("n_q_heads", _i32),
                 ("n_kv_heads", _i32), ("d_ff", _i32), ("vocab", _i32), ("max_pos", _i32),
-                ("rms_eps", _f32), ("rope_theta", _f64)]
+                ("rms_eps", _f32), ("rope_theta", _f64), ("precision", _i32)]
 
 
 class ModelWeights(ctypes.Structure):
@@ -80,6 +82,12 @@ _SIGS = {
                                       _p, _i64, _p]),
     "bi_attn_prefill": (_i32, [_p, _i64, _p, _i32, _i64, _p, _p, _p, _p, _i32,
                                ctypes.POINTER(AttnShape), _p, _i64, _p, _sz, _p]),
+    "bi_gemm_x2": (_i32, [_p, _p, _i64, _p, _i64, _p, _i64, _i32, _i64, _i64, _i64, _p]),
+    "bi_rmsnorm_split": (_i32, [_p, _p, _p, _p, _i64, _i64, _f32, _p]),
+    "bi_split_bf16x2": (_i32, [_p, _i64, _p, _p, _p]),
+    "bi_attn_f32_workspace_size": (_i32, [ctypes.POINTER(AttnShape), _i64, ctypes.POINTER(_sz)]),
+    "bi_attn_f32": (_i32, [_p, _i64, _p, _i64, _p, _p, _p, _p, _i32, ctypes.POINTER(AttnShape), _p,
+                           _i64, _p, _sz, _p]),
     "bi_embed": (_i32, [_p, _i64, _p, _i64, _i64, _p, _p]),
     "bi_rope_table": (_i32, [_p, _i32, _f64, _p]),
     "bi_rope": (_i32, [_p, _i64, _i32, _p, _i64, _p, _i32, _p]),
@@ -146,6 +154,42 @@ def bi_gemm(A, W, C, stream=None) -> None:
     cdt = BI_F32 if C.dtype == torch.float32 else BI_BF16
     _chk("bi_gemm", lib.bi_gemm(_ptr(A), A.stride(0), _ptr(W), W.stride(0), _ptr(C), C.stride(0),
                                 cdt, M, N, K, _stream(stream)))
+
+
+def bi_gemm_x2(A_hi, A_lo, W, C, stream=None) -> None:
+    """C = (A_hi + A_lo) W^T (an fp32 activation carried as a bf16 pair)."""
+    M, K = A_hi.shape
+    N = W.shape[0]
+    cdt = BI_F32 if C.dtype == torch.float32 else BI_BF16
+    _chk("bi_gemm_x2", lib.bi_gemm_x2(_ptr(A_hi), _ptr(A_lo), A_hi.stride(0), _ptr(W), W.stride(0),
+                                      _ptr(C), C.stride(0), cdt, M, N, K, _stream(stream)))
+
+
+def bi_rmsnorm_split(x, gamma, y_hi, y_lo, eps: float, stream=None) -> None:
+    M, D = x.shape
+    _chk("bi_rmsnorm_split", lib.bi_rmsnorm_split(_ptr(x), _ptr(gamma), _ptr(y_hi), _ptr(y_lo), M, D,
+                                                  eps, _stream(stream)))
+
+
+def bi_split_bf16x2(x, hi, lo, stream=None) -> None:
+    _chk("bi_split_bf16x2", lib.bi_split_bf16x2(_ptr(x), x.numel(), _ptr(hi), _ptr(lo), _stream(stream)))
+
+
+def bi_attn_f32(q, cu_q, k_cache, v_cache, block_table, seq_lens, shape: AttnShape, out, ws,
+                stream=None) -> None:
+    """fp32 attention; cu_q None means decode (one query per sequence)."""
+    B = seq_lens.shape[0]
+    _chk("bi_attn_f32", lib.bi_attn_f32(
+        _ptr(q), q.stride(0), _ptr(cu_q), q.shape[0], _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+        _ptr(seq_lens), B, ctypes.byref(shape), _ptr(out), out.stride(0), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def bi_attn_f32_workspace_size(shape: AttnShape, max_tokens: int) -> int:
+    n = _sz(0)
+    _chk("bi_attn_f32_workspace_size", lib.bi_attn_f32_workspace_size(ctypes.byref(shape), max_tokens,
+                                                                      ctypes.byref(n)))
+    return n.value
 
 
 def bi_kv_append(k_new, v_new, slot_mapping, k_cache, v_cache, stream=None) -> None:
@@ -242,9 +286,14 @@ def gemm(A, W, out_dtype=torch.bfloat16):
     return C
 
 
-def new_kv_cache(num_pages: int, num_kv_heads: int, device, n_layers: int = 1, zero=True):
-    """k [L, pages, Hkv, 16, 128] and v [L, pages, Hkv, 128, 16] bf16 (v transposed per page)."""
+def new_kv_cache(num_pages: int, num_kv_heads: int, device, n_layers: int = 1, zero=True,
+                 precision: int = BI_PREC_BF16):
+    """bf16 mode: k [L, pages, Hkv, 16, 128] and v [L, pages, Hkv, 128, 16] bf16
+    (v transposed per page). fp32 modes: k and v [L, pages, Hkv, 16, 128] fp32."""
     f = torch.zeros if zero else torch.empty
+    if precision != BI_PREC_BF16:
+        shp = (n_layers, num_pages, num_kv_heads, PAGE_SIZE, HEAD_DIM)
+        return f(shp, dtype=torch.float32, device=device), f(shp, dtype=torch.float32, device=device)
     k = f((n_layers, num_pages, num_kv_heads, PAGE_SIZE, HEAD_DIM), dtype=torch.bfloat16, device=device)
     v = f((n_layers, num_pages, num_kv_heads, HEAD_DIM, PAGE_SIZE), dtype=torch.bfloat16, device=device)
     return k, v
@@ -257,9 +306,11 @@ class Model:
     def __init__(self, cfg: dict, weights: dict):
         self.cfg = dict(cfg)
         self.weights = weights  # keep the tensors alive
+        prec = cfg.get("precision", "bf16")
+        self.precision = PRECISIONS[prec] if isinstance(prec, str) else int(prec)
         c = ModelConfig(cfg["n_layers"], cfg["d_model"], cfg["n_q_heads"], cfg["n_kv_heads"],
                         cfg["d_ff"], cfg["vocab"], cfg["max_pos"], cfg["rms_eps"],
-                        cfg["rope_theta"])
+                        cfg["rope_theta"], self.precision)
         w = ModelWeights(*[_ptr(weights[n]) for n, _ in ModelWeights._fields_])
         h = _p(0)
         _chk("bi_model_create", lib.bi_model_create(ctypes.byref(c), ctypes.byref(w),

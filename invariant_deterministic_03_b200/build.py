@@ -21,7 +21,7 @@ BUILD = os.path.join(CSRC, "_build")
 LIB = os.path.join(HERE, "libbi.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 SOURCES = ["api.cu", "rmsnorm.cu", "gemm.cu", "attention.cu", "attention_noalloc.cu",
-           "pointwise.cu", "forward.cu"]
+           "pointwise.cu", "upcast.cu", "forward.cu"]
 HEADERS = ["common.cuh", "host.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

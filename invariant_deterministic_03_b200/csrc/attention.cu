@@ -45,7 +45,8 @@ constexpr uint32_t OFF_K = 2 * TILE_BYTES;      // 2 buffers
 constexpr uint32_t OFF_V = 4 * TILE_BYTES;      // 2 buffers
 constexpr uint32_t OFF_P = 6 * TILE_BYTES;
 constexpr uint32_t OFF_BAR = 7 * TILE_BYTES;
-constexpr size_t SMEM_BYTES = 1024 + 7 * TILE_BYTES + 256;
+constexpr uint32_t OFF_RING = OFF_BAR + 256;   // producer's page-row ring
+constexpr size_t SMEM_BYTES = 1024 + 7 * TILE_BYTES + 256 + 8 * sizeof(int32_t) * 2 * 8;
 // warps 0-3: one thread per MMA row (softmax, O rescale, partials)
 // warp 4: TMA producer; warp 5: TMEM allocator and MMA issuer
 constexpr int THREADS = 192;
@@ -105,23 +106,28 @@ __device__ __forceinline__ bool item_at(const Params& p, int idx, Item& it, bool
   return true;
 }
 
-__device__ __forceinline__ void load_kv_tile(const Params& p, const CUtensorMap* tmK,
-                                             const CUtensorMap* tmV, uint8_t* kbuf, uint8_t* vbuf,
-                                             uint64_t* kbar, uint64_t* vbar, int b, int g, int L,
-                                             int tile) {
-  const int32_t k_rows_total = p.num_pages * p.Hkv * PAGE;  // first out-of-range row
+// Cache rows of the 8 pages of one 128-key tile (page ids looked up in the
+// sequence's block table). Pages past the sequence end, or with an id outside
+// the cache, get the first out-of-range row: TMA fills those boxes with zeros.
+struct TileRows {
+  int32_t k[PAGES_PER_TILE];
+  int32_t v[PAGES_PER_TILE];
+};
+
+__device__ __forceinline__ void tile_rows(const Params& p, int b, int g, int L, int tile,
+                                          TileRows& r) {
+  const int32_t k_rows_total = p.num_pages * p.Hkv * PAGE;
   const int32_t v_rows_total = p.num_pages * p.Hkv * HD;
-  int32_t krow[PAGES_PER_TILE], vrow[PAGES_PER_TILE];
 #pragma unroll
   for (int i = 0; i < PAGES_PER_TILE; ++i) {
     const int pidx = tile * PAGES_PER_TILE + i;
-    krow[i] = k_rows_total;  // out of range: TMA fills zeros
-    vrow[i] = v_rows_total;
+    r.k[i] = k_rows_total;
+    r.v[i] = v_rows_total;
     if (pidx * PAGE < L && pidx < p.max_pages) {
       const int32_t pid = p.block_table[(size_t)b * p.max_pages + pidx];
       if (pid >= 0 && pid < p.num_pages) {
-        krow[i] = (pid * p.Hkv + g) * PAGE;
-        vrow[i] = (pid * p.Hkv + g) * HD;
+        r.k[i] = (pid * p.Hkv + g) * PAGE;
+        r.v[i] = (pid * p.Hkv + g) * HD;
       } else {
         set_status(p.status, BI_DEV_BAD_PAGE);
       }
@@ -129,16 +135,62 @@ __device__ __forceinline__ void load_kv_tile(const Params& p, const CUtensorMap*
       set_status(p.status, BI_DEV_BAD_PAGE);
     }
   }
+}
+
+__device__ __forceinline__ void prefetch_tile(const Params& p, const CUtensorMap* tmK,
+                                              const CUtensorMap* tmV, const TileRows& r) {
+  const int32_t k_rows_total = p.num_pages * p.Hkv * PAGE;
+#pragma unroll
+  for (int i = 0; i < PAGES_PER_TILE; ++i) {
+    if (r.k[i] < k_rows_total) {
+      tma_prefetch_2d(tmK, 0, r.k[i]);
+      tma_prefetch_2d(tmK, 64, r.k[i]);
+      tma_prefetch_2d(tmV, 0, r.v[i]);
+    }
+  }
+}
+
+__device__ __forceinline__ void load_kv_tile(const CUtensorMap* tmK, const CUtensorMap* tmV,
+                                             uint8_t* kbuf, uint8_t* vbuf, uint64_t* kbar,
+                                             uint64_t* vbar, const TileRows& r) {
   mbar_arrive_expect_tx(kbar, TILE_BYTES);
 #pragma unroll
   for (int i = 0; i < PAGES_PER_TILE; ++i) {
-    tma_load_2d(kbuf + i * 2048, tmK, kbar, 0, krow[i]);
-    tma_load_2d(kbuf + 16384 + i * 2048, tmK, kbar, 64, krow[i]);
+    tma_load_2d(kbuf + i * 2048, tmK, kbar, 0, r.k[i]);
+    tma_load_2d(kbuf + 16384 + i * 2048, tmK, kbar, 64, r.k[i]);
   }
   mbar_arrive_expect_tx(vbar, TILE_BYTES);
 #pragma unroll
-  for (int i = 0; i < PAGES_PER_TILE; ++i) tma_load_2d(vbuf + i * 4096, tmV, vbar, 0, vrow[i]);
+  for (int i = 0; i < PAGES_PER_TILE; ++i) tma_load_2d(vbuf + i * 4096, tmV, vbar, 0, r.v[i]);
 }
+
+// Walks the (item, tile) sequence of one CTA.
+struct Cursor {
+  int idx, t;
+  Item it;
+  bool valid;
+};
+
+__device__ __forceinline__ void cursor_next(const Params& p, Cursor& c) {
+  if (c.valid && ++c.t < c.it.ntiles) return;
+  c.valid = false;
+  c.t = 0;
+  for (c.idx += gridDim.x; c.idx < p.total_items; c.idx += gridDim.x)
+    if (item_at(p, c.idx, c.it, false)) {
+      c.valid = true;
+      return;
+    }
+}
+
+__device__ __forceinline__ void cursor_start(const Params& p, Cursor& c) {
+  c.idx = (int)blockIdx.x - (int)gridDim.x;
+  c.t = 0;
+  c.valid = false;
+  cursor_next(p, c);
+}
+
+constexpr int PF_AHEAD = 4;   // tiles prefetched into L2 ahead of the shared-memory loads
+constexpr int PF_RING = 8;    // ring of looked-up page rows (power of two > PF_AHEAD)
 
 __device__ __forceinline__ void issue_s(uint32_t tmem_s, uint32_t q_addr, uint32_t k_addr) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
@@ -241,9 +293,19 @@ __global__ void __launch_bounds__(THREADS, 1)
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       const uint32_t q_bytes = 2u * 64u * 2u * (uint32_t)(p.G * p.q_box);
+      TileRows* ring = reinterpret_cast<TileRows*>(smem + OFF_RING);
       int qi = 0, kvi = 0;
       int q_fills[2] = {0, 0}, kv_fills[2] = {0, 0};
       bool ok = true;
+      // prefetch cursor runs PF_AHEAD tiles in front of the load cursor
+      Cursor pf;
+      cursor_start(p, pf);
+      int pf_n = 0;  // tiles looked up and prefetched so far
+      for (; pf.valid && pf_n < PF_AHEAD; ++pf_n, cursor_next(p, pf)) {
+        TileRows& r = ring[pf_n & (PF_RING - 1)];
+        tile_rows(p, pf.it.b, pf.it.g, pf.it.L, pf.it.t0 + pf.t, r);
+        prefetch_tile(p, &tmK, &tmV, r);
+      }
       for (int idx = blockIdx.x; idx < p.total_items && ok; idx += gridDim.x) {
         Item it;
         if (!item_at(p, idx, it, true)) continue;
@@ -256,10 +318,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         ++q_fills[qb];
         ++qi;
         for (int t = 0; t < it.ntiles; ++t) {
+          // look up and prefetch the tile PF_AHEAD ahead of this one
+          if (pf.valid) {
+            TileRows& r = ring[pf_n & (PF_RING - 1)];
+            tile_rows(p, pf.it.b, pf.it.g, pf.it.L, pf.it.t0 + pf.t, r);
+            prefetch_tile(p, &tmK, &tmV, r);
+            ++pf_n;
+            cursor_next(p, pf);
+          }
           const int kb = kvi & 1;
           if (!mbar_wait(&kv_empty[kb], (((uint32_t)kvi >> 1) & 1u) ^ 1u, p.status, abort_flag)) { ok = false; break; }
-          load_kv_tile(p, &tmK, &tmV, smem + OFF_K + kb * TILE_BYTES, smem + OFF_V + kb * TILE_BYTES,
-                       &k_full[kb], &v_full[kb], it.b, it.g, it.L, it.t0 + t);
+          load_kv_tile(&tmK, &tmV, smem + OFF_K + kb * TILE_BYTES, smem + OFF_V + kb * TILE_BYTES,
+                       &k_full[kb], &v_full[kb], ring[kvi & (PF_RING - 1)]);
           ++kv_fills[kb];
           ++kvi;
         }

@@ -14,7 +14,9 @@
 // determinism" and "How do we make kernels batch-invariant?"). The residual
 // stream is kept in fp32 and the two GEMMs that feed it write fp32 (a reading:
 // the pages fix no activation precision; this keeps the stream's rounding
-// error below the bf16 inputs').
+// error below the bf16 inputs'). The fp32-activation modes (the cross-vendor
+// paper's FP32 upcast and its BF16-MLP-only variant) swap the attention
+// and/or MLP block for the upcast kernels of upcast.cu.
 #include <stdlib.h>
 
 #include "common.cuh"
@@ -31,6 +33,19 @@ bi_status launch_rope(bf16* x, int64_t ldx, int n_heads, const int32_t* pos, int
 bi_status launch_swiglu(const bf16* gu, int64_t n_tok, int64_t F, bf16* out, cudaStream_t s);
 bi_status launch_argmax(const float* logits, int64_t rows, int64_t V, int64_t ld, int32_t* idx,
                         cudaStream_t s);
+bi_status launch_split(const float* x, int64_t n, bf16* hi, bf16* lo, cudaStream_t s);
+bi_status launch_swiglu_split(const float* gu, int64_t n_tok, int64_t F, bf16* hi, bf16* lo,
+                              cudaStream_t s);
+bi_status launch_rope_f32(float* x, int64_t ldx, int n_heads, const int32_t* pos, int64_t n_tok,
+                          const float* cs, int max_pos, cudaStream_t s);
+bi_status launch_kv_append_f32(const float* k, const float* v, int64_t ld, const int32_t* slots,
+                               int64_t n_tok, float* kc, float* vc, int Hkv, int num_pages,
+                               cudaStream_t s);
+bi_status run_attn_f32(const float* q, int64_t ldq, const int32_t* cu_q, int64_t n_tok,
+                       const float* kc, const float* vc, const int32_t* block_table,
+                       const int32_t* seq_lens, int32_t B, const bi_attn_shape* sh, float* out,
+                       int64_t ldo, void* ws, size_t ws_bytes, cudaStream_t s);
+size_t attn_f32_workspace(int64_t n_tok, int Hq, int max_kv_len);
 
 namespace fwd {
 
@@ -51,7 +66,8 @@ __global__ void gather_rows_kernel(const float* __restrict__ x, const int32_t* _
 }
 
 struct Layout {  // workspace carve-up, all offsets 256-byte aligned
-  size_t x, h, qkv, att, t32, gu, act, xl, hl, rope, attn_ws, total;
+  size_t x, h, h_lo, qkv, qkv32, att, att_lo, att32, t32, gu, gu32, act, act_lo, xl, hl, hl_lo,
+      rope, attn_ws, total;
   size_t attn_ws_bytes;
 };
 
@@ -61,16 +77,24 @@ static Layout layout(const bi_model_config& c, int64_t T, int64_t NL, int32_t ma
   Layout L;
   const size_t D = c.d_model, F = c.d_ff;
   const size_t QKV = (size_t)(c.n_q_heads + 2 * c.n_kv_heads) * BI_HEAD_DIM;
+  const bool f32 = c.precision != BI_PREC_BF16;  // fp32 buffers needed
   size_t o = 0;
   L.x = o; o += up(T * D * 4);
   L.h = o; o += up(T * D * 2);
+  L.h_lo = o; o += f32 ? up(T * D * 2) : 0;
   L.qkv = o; o += up(T * QKV * 2);
+  L.qkv32 = o; o += f32 ? up(T * QKV * 4) : 0;
   L.att = o; o += up(T * D * 2);
+  L.att_lo = o; o += f32 ? up(T * D * 2) : 0;
+  L.att32 = o; o += f32 ? up(T * D * 4) : 0;
   L.t32 = o; o += up(T * D * 4);
   L.gu = o; o += up(T * 2 * F * 2);
+  L.gu32 = o; o += c.precision == BI_PREC_F32 ? up(T * 2 * F * 4) : 0;
   L.act = o; o += up(T * F * 2);
+  L.act_lo = o; o += c.precision == BI_PREC_F32 ? up(T * F * 2) : 0;
   L.xl = o; o += up(NL * D * 4);
   L.hl = o; o += up(NL * D * 2);
+  L.hl_lo = o; o += f32 ? up(NL * D * 2) : 0;
   L.rope = o; o += up((size_t)c.max_pos * 64 * 2 * 4);
   bi_attn_shape sh;
   sh.num_q_heads = c.n_q_heads;
@@ -83,6 +107,8 @@ static Layout layout(const bi_model_config& c, int64_t T, int64_t NL, int32_t ma
   sh.scale = 1.0f;
   size_t a = 0;
   bi_attn_workspace_size(&sh, T, &a);
+  const size_t a32 = attn_f32_workspace(T, c.n_q_heads, sh.max_kv_len);
+  if (a32 > a) a = a32;
   L.attn_ws = o; o += up(a);
   L.attn_ws_bytes = a;
   L.total = o;
@@ -112,6 +138,8 @@ extern "C" bi_status bi_model_create(const bi_model_config* cfg, const bi_model_
   if (G != 1 && G != 2 && G != 4 && G != 8) return fail(BI_ERR_SHAPE, "model_create: q heads per kv head must be 1, 2, 4 or 8");
   if (c.d_ff % 8 || c.vocab % 8) return fail(BI_ERR_SHAPE, "model_create: d_ff and vocab must be multiples of 8");
   if (!(c.rms_eps >= 0.0f) || !(c.rope_theta > 1.0)) return fail(BI_ERR_INVALID_ARG, "model_create: bad eps or rope_theta");
+  if (c.precision != BI_PREC_BF16 && c.precision != BI_PREC_F32 && c.precision != BI_PREC_BF16_MLP)
+    return fail(BI_ERR_INVALID_ARG, "model_create: unknown precision %d", c.precision);
   if (!w->embed || !w->final_norm || !w->lm_head) return fail(BI_ERR_INVALID_ARG, "model_create: missing weights");
   if (c.n_layers > 0 && (!w->attn_norm || !w->w_qkv || !w->w_o || !w->mlp_norm || !w->w_gate_up || !w->w_down))
     return fail(BI_ERR_INVALID_ARG, "model_create: missing layer weights");
@@ -160,22 +188,29 @@ extern "C" bi_status bi_forward(const bi_model* m, const bi_batch* bt, void* k_c
   uint8_t* base = static_cast<uint8_t*>(ws);
   float* x = reinterpret_cast<float*>(base + L.x);
   bf16* h = reinterpret_cast<bf16*>(base + L.h);
+  bf16* h_lo = reinterpret_cast<bf16*>(base + L.h_lo);
   bf16* qkv = reinterpret_cast<bf16*>(base + L.qkv);
+  float* qkv32 = reinterpret_cast<float*>(base + L.qkv32);
   bf16* att = reinterpret_cast<bf16*>(base + L.att);
+  bf16* att_lo = reinterpret_cast<bf16*>(base + L.att_lo);
+  float* att32 = reinterpret_cast<float*>(base + L.att32);
   float* t32 = reinterpret_cast<float*>(base + L.t32);
   bf16* gu = reinterpret_cast<bf16*>(base + L.gu);
+  float* gu32 = reinterpret_cast<float*>(base + L.gu32);
   bf16* act = reinterpret_cast<bf16*>(base + L.act);
+  bf16* act_lo = reinterpret_cast<bf16*>(base + L.act_lo);
   float* xl = reinterpret_cast<float*>(base + L.xl);
   bf16* hl = reinterpret_cast<bf16*>(base + L.hl);
+  bf16* hl_lo = reinterpret_cast<bf16*>(base + L.hl_lo);
   float* rope = reinterpret_cast<float*>(base + L.rope);
   void* attn_ws = base + L.attn_ws;
 
+  const bool attn_f32 = c.precision != BI_PREC_BF16;  // attention block (and LM head) upcast
+  const bool mlp_f32 = c.precision == BI_PREC_F32;    // MLP block upcast
   const int64_t T = b.n_tok, D = c.d_model, F = c.d_ff;
   const int Hq = c.n_q_heads, Hkv = c.n_kv_heads;
   const int64_t QKV = (int64_t)(Hq + 2 * Hkv) * BI_HEAD_DIM;
   const size_t cache_layer = (size_t)num_pages * Hkv * BI_PAGE_SIZE * BI_HEAD_DIM;
-  const bf16* W = nullptr;
-  (void)W;
 
   BI_TRY(bi_rope_table(rope, c.max_pos, c.rope_theta, stream));
   BI_TRY(launch_embed(b.tokens, T, static_cast<const bf16*>(m->w.embed), c.vocab, D, x, s));
@@ -198,24 +233,50 @@ extern "C" bi_status bi_forward(const bi_model* m, const bi_batch* bt, void* k_c
     const bf16* w_o = static_cast<const bf16*>(m->w.w_o) + (size_t)l * D * D;
     const bf16* w_gu = static_cast<const bf16*>(m->w.w_gate_up) + (size_t)l * 2 * F * D;
     const bf16* w_d = static_cast<const bf16*>(m->w.w_down) + (size_t)l * D * F;
-    bf16* kc = static_cast<bf16*>(k_cache) + (size_t)l * cache_layer;
-    bf16* vc = static_cast<bf16*>(v_cache) + (size_t)l * cache_layer;
 
-    BI_TRY(bi_rmsnorm_f32in(x, attn_norm, h, T, D, c.rms_eps, stream));
-    BI_TRY(bi_gemm(h, D, w_qkv, D, qkv, QKV, BI_BF16, T, QKV, D, stream));
-    BI_TRY(launch_rope(qkv, QKV, Hq, b.positions, T, rope, c.max_pos, s));
-    BI_TRY(launch_rope(qkv + (size_t)Hq * BI_HEAD_DIM, QKV, Hkv, b.positions, T, rope, c.max_pos, s));
-    BI_TRY(launch_kv_append(qkv + (size_t)Hq * BI_HEAD_DIM, qkv + (size_t)(Hq + Hkv) * BI_HEAD_DIM,
-                            QKV, b.slot_mapping, T, kc, vc, Hkv, num_pages, s));
-    BI_TRY(bi_attn_prefill(qkv, QKV, b.cu_q, b.max_q_len, T, kc, vc, b.block_table, b.seq_lens,
-                           b.B, &sh, att, D, attn_ws, L.attn_ws_bytes, stream));
-    BI_TRY(bi_gemm(att, D, w_o, D, t32, D, BI_F32, T, D, D, stream));
+    // ---- attention block
+    if (attn_f32) {
+      float* kc = static_cast<float*>(k_cache) + (size_t)l * cache_layer;
+      float* vc = static_cast<float*>(v_cache) + (size_t)l * cache_layer;
+      BI_TRY(bi_rmsnorm_split(x, attn_norm, h, h_lo, T, D, c.rms_eps, stream));
+      BI_TRY(bi_gemm_x2(h, h_lo, D, w_qkv, D, qkv32, QKV, BI_F32, T, QKV, D, stream));
+      BI_TRY(launch_rope_f32(qkv32, QKV, Hq, b.positions, T, rope, c.max_pos, s));
+      BI_TRY(launch_rope_f32(qkv32 + (size_t)Hq * BI_HEAD_DIM, QKV, Hkv, b.positions, T, rope, c.max_pos, s));
+      BI_TRY(launch_kv_append_f32(qkv32 + (size_t)Hq * BI_HEAD_DIM,
+                                  qkv32 + (size_t)(Hq + Hkv) * BI_HEAD_DIM, QKV, b.slot_mapping, T,
+                                  kc, vc, Hkv, num_pages, s));
+      BI_TRY(run_attn_f32(qkv32, QKV, b.cu_q, T, kc, vc, b.block_table, b.seq_lens, b.B, &sh, att32,
+                          D, attn_ws, L.attn_ws_bytes, s));
+      BI_TRY(launch_split(att32, T * D, att, att_lo, s));
+      BI_TRY(bi_gemm_x2(att, att_lo, D, w_o, D, t32, D, BI_F32, T, D, D, stream));
+    } else {
+      bf16* kc = static_cast<bf16*>(k_cache) + (size_t)l * cache_layer;
+      bf16* vc = static_cast<bf16*>(v_cache) + (size_t)l * cache_layer;
+      BI_TRY(bi_rmsnorm_f32in(x, attn_norm, h, T, D, c.rms_eps, stream));
+      BI_TRY(bi_gemm(h, D, w_qkv, D, qkv, QKV, BI_BF16, T, QKV, D, stream));
+      BI_TRY(launch_rope(qkv, QKV, Hq, b.positions, T, rope, c.max_pos, s));
+      BI_TRY(launch_rope(qkv + (size_t)Hq * BI_HEAD_DIM, QKV, Hkv, b.positions, T, rope, c.max_pos, s));
+      BI_TRY(launch_kv_append(qkv + (size_t)Hq * BI_HEAD_DIM, qkv + (size_t)(Hq + Hkv) * BI_HEAD_DIM,
+                              QKV, b.slot_mapping, T, kc, vc, Hkv, num_pages, s));
+      BI_TRY(bi_attn_prefill(qkv, QKV, b.cu_q, b.max_q_len, T, kc, vc, b.block_table, b.seq_lens,
+                             b.B, &sh, att, D, attn_ws, L.attn_ws_bytes, stream));
+      BI_TRY(bi_gemm(att, D, w_o, D, t32, D, BI_F32, T, D, D, stream));
+    }
     fwd::add_f32_kernel<<<(unsigned)add_blocks, 256, 0, s>>>(x, t32, T * D);
     BI_CHECK_LAUNCH("forward residual");
-    BI_TRY(bi_rmsnorm_f32in(x, mlp_norm, h, T, D, c.rms_eps, stream));
-    BI_TRY(bi_gemm(h, D, w_gu, D, gu, 2 * F, BI_BF16, T, 2 * F, D, stream));
-    BI_TRY(launch_swiglu(gu, T, F, act, s));
-    BI_TRY(bi_gemm(act, F, w_d, F, t32, D, BI_F32, T, D, F, stream));
+
+    // ---- MLP block
+    if (mlp_f32) {
+      BI_TRY(bi_rmsnorm_split(x, mlp_norm, h, h_lo, T, D, c.rms_eps, stream));
+      BI_TRY(bi_gemm_x2(h, h_lo, D, w_gu, D, gu32, 2 * F, BI_F32, T, 2 * F, D, stream));
+      BI_TRY(launch_swiglu_split(gu32, T, F, act, act_lo, s));
+      BI_TRY(bi_gemm_x2(act, act_lo, F, w_d, F, t32, D, BI_F32, T, D, F, stream));
+    } else {
+      BI_TRY(bi_rmsnorm_f32in(x, mlp_norm, h, T, D, c.rms_eps, stream));
+      BI_TRY(bi_gemm(h, D, w_gu, D, gu, 2 * F, BI_BF16, T, 2 * F, D, stream));
+      BI_TRY(launch_swiglu(gu, T, F, act, s));
+      BI_TRY(bi_gemm(act, F, w_d, F, t32, D, BI_F32, T, D, F, stream));
+    }
     fwd::add_f32_kernel<<<(unsigned)add_blocks, 256, 0, s>>>(x, t32, T * D);
     BI_CHECK_LAUNCH("forward residual");
   }
@@ -223,8 +284,14 @@ extern "C" bi_status bi_forward(const bi_model* m, const bi_batch* bt, void* k_c
   fwd::gather_rows_kernel<<<(unsigned)b.n_logits, 256, 0, s>>>(x, b.logits_rows, b.n_logits, T,
                                                                (int)D, xl, status_word());
   BI_CHECK_LAUNCH("forward gather");
-  BI_TRY(bi_rmsnorm_f32in(xl, m->w.final_norm, hl, b.n_logits, D, c.rms_eps, stream));
-  BI_TRY(bi_gemm(hl, D, m->w.lm_head, D, logits, c.vocab, BI_F32, b.n_logits, c.vocab, D, stream));
+  if (attn_f32) {
+    BI_TRY(bi_rmsnorm_split(xl, m->w.final_norm, hl, hl_lo, b.n_logits, D, c.rms_eps, stream));
+    BI_TRY(bi_gemm_x2(hl, hl_lo, D, m->w.lm_head, D, logits, c.vocab, BI_F32, b.n_logits, c.vocab, D,
+                      stream));
+  } else {
+    BI_TRY(bi_rmsnorm_f32in(xl, m->w.final_norm, hl, b.n_logits, D, c.rms_eps, stream));
+    BI_TRY(bi_gemm(hl, D, m->w.lm_head, D, logits, c.vocab, BI_F32, b.n_logits, c.vocab, D, stream));
+  }
   if (next_tokens) BI_TRY(launch_argmax(logits, b.n_logits, c.vocab, c.vocab, next_tokens, s));
   return BI_OK;
 }

@@ -33,14 +33,22 @@ namespace gemm {
 constexpr int BM = BI_GEMM_BM;  // 128
 constexpr int BN = BI_GEMM_BN;  // 256
 constexpr int BK = BI_GEMM_BK;  // 64 bf16 = 128 bytes = one swizzle row
-constexpr int STAGES = 4;
 constexpr int UMMA_K = 16;
 constexpr uint32_t A_BYTES = BM * BK * 2;  // 16 KB
 constexpr uint32_t B_BYTES = BN * BK * 2;  // 32 KB
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int THREADS = 192;
-constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 256 /*barriers*/;
+
+// TERMS = number of bf16 A operands summed into the product: 1 for plain
+// bf16 activations, 2 for an activation carried as a hi/lo pair (A = A_hi +
+// A_lo, ~16 significant bits). Both terms meet the same W tile in shared
+// memory, so W is read once.
+template <int TERMS>
+struct Cfg {
+  static constexpr int STAGES = TERMS == 1 ? 4 : 3;
+  static constexpr uint32_t STAGE_BYTES = TERMS * A_BYTES + B_BYTES;
+  static constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 256;
+};
 
 struct Params {
   void* C;
@@ -84,9 +92,13 @@ __device__ __forceinline__ void store_row_chunk(const Params& p, int row, int co
   }
 }
 
+template <int TERMS>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmA2,
                         const __grid_constant__ CUtensorMap tmB, const Params p) {
+  constexpr int STAGES = Cfg<TERMS>::STAGES;
+  constexpr uint32_t STAGE_BYTES = Cfg<TERMS>::STAGE_BYTES;
   extern __shared__ uint8_t smem_raw[];
   // 128-byte swizzled tiles want 1024-byte aligned bases.
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -117,6 +129,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
+    if (TERMS == 2) prefetch_tmap(&tmA2);
     prefetch_tmap(&tmB);
   }
   if (warp == 1) {
@@ -134,6 +147,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      int fills[STAGES];
+      for (int s = 0; s < STAGES; ++s) fills[s] = 0;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int mb = tile % p.m_blocks, nb = tile / p.m_blocks;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
@@ -141,7 +156,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           uint8_t* sa = tiles + stage * STAGE_BYTES;
           mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
           tma_load_2d(sa, &tmA, &full[stage], kb * BK, mb * BM);
-          tma_load_2d(sa + A_BYTES, &tmB, &full[stage], kb * BK, nb * BN);
+          if (TERMS == 2) tma_load_2d(sa + A_BYTES, &tmA2, &full[stage], kb * BK, mb * BM);
+          tma_load_2d(sa + TERMS * A_BYTES, &tmB, &full[stage], kb * BK, nb * BN);
+          ++fills[stage];
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -149,9 +166,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         // Let copies already in flight land before the CTA can exit: wait
         // (bounded) for every stage's last fill.
         for (int s = 0; s < STAGES; ++s) {
-          long long t0 = clock64();
-          while (!mbar_try_wait(&full[s], 0) && !mbar_try_wait(&full[s], 1) &&
-                 clock64() - t0 < kWaitLimitCycles) {
+          if (fills[s] == 0) continue;
+          const uint32_t par = (uint32_t)(fills[s] - 1) & 1u;
+          const long long t0 = clock64();
+          while (!mbar_try_wait(&full[s], par) && clock64() - t0 < kWaitLimitCycles) {
           }
         }
       }
@@ -173,15 +191,18 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(tiles + stage * STAGE_BYTES);
-          const uint32_t sb = sa + A_BYTES;
+          const uint32_t sb = sa + TERMS * A_BYTES;
 #pragma unroll
-          for (int k = 0; k < BK / UMMA_K; ++k) {
-            // Advancing the start address by 32 bytes per 16-element K step
-            // inside the 128-byte swizzle atom; the hardware applies the
-            // swizzle on the absolute address (tile bases are 1024-aligned).
-            uint64_t ad = smem_desc(sa + k * 32, 16, 1024, 2);
-            uint64_t bd = smem_desc(sb + k * 32, 16, 1024, 2);
-            mma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0);
+          for (int term = 0; term < TERMS; ++term) {
+#pragma unroll
+            for (int k = 0; k < BK / UMMA_K; ++k) {
+              // Advancing the start address by 32 bytes per 16-element K step
+              // inside the 128-byte swizzle atom; the hardware applies the
+              // swizzle on the absolute address (tile bases are 1024-aligned).
+              uint64_t ad = smem_desc(sa + term * A_BYTES + k * 32, 16, 1024, 2);
+              uint64_t bd = smem_desc(sb + k * 32, 16, 1024, 2);
+              mma_bf16(d_tmem, ad, bd, idesc, (kb | term | k) != 0);
+            }
           }
           mma_commit(&empty[stage]);  // frees the stage once these MMAs retire
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -239,9 +260,11 @@ __global__ void zero_fill_kernel(void* C, int64_t ldc, int32_t c_f32, int32_t M,
 
 using namespace bi;
 
-extern "C" bi_status bi_gemm(const void* A, int64_t lda, const void* W, int64_t ldw, void* C,
-                             int64_t ldc, int32_t c_dtype, int64_t M, int64_t N, int64_t K,
-                             void* stream) {
+namespace bi {
+namespace gemm {
+
+static bi_status check_args(const void* A, int64_t lda, const void* W, int64_t ldw, const void* C,
+                            int64_t ldc, int32_t c_dtype, int64_t M, int64_t N, int64_t K) {
   if (!A || !W || !C) return fail(BI_ERR_INVALID_ARG, "gemm: null pointer");
   if (M < 0 || N < 0 || K < 0) return fail(BI_ERR_INVALID_ARG, "gemm: negative size");
   if (c_dtype != BI_BF16 && c_dtype != BI_F32) return fail(BI_ERR_INVALID_ARG, "gemm: bad c_dtype %d", c_dtype);
@@ -250,58 +273,95 @@ extern "C" bi_status bi_gemm(const void* A, int64_t lda, const void* W, int64_t 
   if (lda < K || ldw < K || ldc < N) return fail(BI_ERR_SHAPE, "gemm: leading dimension smaller than the row");
   if (lda % 8 || ldw % 8 || ldc % 8) return fail(BI_ERR_ALIGN, "gemm: leading dimensions must be multiples of 8");
   if (!aligned16(A) || !aligned16(W) || !aligned16(C)) return fail(BI_ERR_ALIGN, "gemm: pointers must be 16-byte aligned");
-  if (M == 0 || N == 0) return BI_OK;
-  bi_status st = require_sm100();
-  if (st != BI_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return BI_OK;
+}
+
+template <int TERMS>
+static bi_status launch(const void* A, const void* A2, int64_t lda, const void* W, int64_t ldw,
+                        void* C, int64_t ldc, int32_t c_dtype, int64_t M, int64_t N, int64_t K,
+                        cudaStream_t s) {
+  bi_status st;
   const int32_t c_f32 = c_dtype == BI_F32;
   if (K == 0) {
-    gemm::zero_fill_kernel<<<296, 256, 0, s>>>(C, ldc, c_f32, (int32_t)M, (int32_t)N);
+    zero_fill_kernel<<<296, 256, 0, s>>>(C, ldc, c_f32, (int32_t)M, (int32_t)N);
     BI_CHECK_LAUNCH("gemm zero fill");
     return BI_OK;
   }
-  CUtensorMap tmA, tmB;
+  CUtensorMap tmA, tmA2, tmB;
   {
     uint64_t dims[2] = {(uint64_t)K, (uint64_t)M};
     uint64_t strides[1] = {(uint64_t)lda * 2};
-    uint32_t box[2] = {gemm::BK, gemm::BM};
+    uint32_t box[2] = {BK, BM};
     if ((st = encode_tmap(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(A), dims,
                           strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != BI_OK)
       return st;
+    if (TERMS == 2) {
+      if ((st = encode_tmap(&tmA2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(A2), dims,
+                            strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != BI_OK)
+        return st;
+    } else {
+      tmA2 = tmA;
+    }
   }
   {
     uint64_t dims[2] = {(uint64_t)K, (uint64_t)N};
     uint64_t strides[1] = {(uint64_t)ldw * 2};
-    uint32_t box[2] = {gemm::BK, gemm::BN};
+    uint32_t box[2] = {BK, BN};
     if ((st = encode_tmap(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(W), dims,
                           strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != BI_OK)
       return st;
   }
-  gemm::Params p;
+  Params p;
   p.C = C;
   p.ldc = ldc;
   p.c_f32 = c_f32;
   p.M = (int32_t)M;
   p.N = (int32_t)N;
   p.K = (int32_t)K;
-  p.m_blocks = (int32_t)((M + gemm::BM - 1) / gemm::BM);
-  p.n_blocks = (int32_t)((N + gemm::BN - 1) / gemm::BN);
-  p.k_blocks = (int32_t)((K + gemm::BK - 1) / gemm::BK);
+  p.m_blocks = (int32_t)((M + BM - 1) / BM);
+  p.n_blocks = (int32_t)((N + BN - 1) / BN);
+  p.k_blocks = (int32_t)((K + BK - 1) / BK);
   p.status = status_word();
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (!attr_set[dev & 63]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm::gemm_tcgen05_kernel,
+    cudaError_t e = cudaFuncSetAttribute(gemm_tcgen05_kernel<TERMS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)gemm::SMEM_BYTES);
+                                         (int)Cfg<TERMS>::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e, "gemm: smem attribute");
     attr_set[dev & 63] = true;
   }
   const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
   const int sms = num_sms();
   const int grid = (int)(tiles < sms ? tiles : sms);
-  gemm::gemm_tcgen05_kernel<<<grid, gemm::THREADS, gemm::SMEM_BYTES, s>>>(tmA, tmB, p);
+  gemm_tcgen05_kernel<TERMS><<<grid, THREADS, Cfg<TERMS>::SMEM_BYTES, s>>>(tmA, tmA2, tmB, p);
   BI_CHECK_LAUNCH("gemm launch");
   return BI_OK;
+}
+
+}  // namespace gemm
+}  // namespace bi
+
+extern "C" bi_status bi_gemm(const void* A, int64_t lda, const void* W, int64_t ldw, void* C,
+                             int64_t ldc, int32_t c_dtype, int64_t M, int64_t N, int64_t K,
+                             void* stream) {
+  bi_status st = gemm::check_args(A, lda, W, ldw, C, ldc, c_dtype, M, N, K);
+  if (st != BI_OK || M == 0 || N == 0) return st;
+  if ((st = require_sm100()) != BI_OK) return st;
+  return gemm::launch<1>(A, nullptr, lda, W, ldw, C, ldc, c_dtype, M, N, K,
+                         static_cast<cudaStream_t>(stream));
+}
+
+extern "C" bi_status bi_gemm_x2(const void* A_hi, const void* A_lo, int64_t lda, const void* W,
+                                int64_t ldw, void* C, int64_t ldc, int32_t c_dtype, int64_t M,
+                                int64_t N, int64_t K, void* stream) {
+  bi_status st = gemm::check_args(A_hi, lda, W, ldw, C, ldc, c_dtype, M, N, K);
+  if (st != BI_OK) return st;
+  if (!A_lo) return fail(BI_ERR_INVALID_ARG, "gemm_x2: A_lo is null");
+  if (!aligned16(A_lo)) return fail(BI_ERR_ALIGN, "gemm_x2: A_lo must be 16-byte aligned");
+  if (M == 0 || N == 0) return BI_OK;
+  if ((st = require_sm100()) != BI_OK) return st;
+  return gemm::launch<2>(A_hi, A_lo, lda, W, ldw, C, ldc, c_dtype, M, N, K,
+                         static_cast<cudaStream_t>(stream));
 }

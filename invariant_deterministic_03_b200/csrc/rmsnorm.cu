@@ -46,10 +46,13 @@ struct Row8<float> {
 };
 
 // CPT = chunks per thread (compile-time so the row stays in registers).
-template <typename Tin, int CPT>
+// SPLIT: write the fp32 result as a bf16 pair (y = bf16(v), y_lo = bf16(v - y))
+// for the fp32-activation path; otherwise y = bf16(v).
+template <typename Tin, int CPT, bool SPLIT>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const Tin* __restrict__ x,
                                                       const bf16* __restrict__ gamma,
-                                                      bf16* __restrict__ y, int D, float eps) {
+                                                      bf16* __restrict__ y, bf16* __restrict__ y_lo,
+                                                      int D, float eps) {
   __shared__ float warp_sum[32];
   __shared__ float row_scale;
   const int T = blockDim.x;
@@ -89,12 +92,22 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const Tin* __restrict__ x,
     if (c < nchunks) {
       float g[8];
       Row8<bf16>::load(gamma + c * 8, g);
-      uint4 o;
+      uint4 o, olo;
       uint32_t* op = reinterpret_cast<uint32_t*>(&o);
+      uint32_t* olp = reinterpret_cast<uint32_t*>(&olo);
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        op[e] = pack_bf16x2((v[i][2 * e] * r) * g[2 * e], (v[i][2 * e + 1] * r) * g[2 * e + 1]);
+      for (int e = 0; e < 4; ++e) {
+        const float a = __fmul_rn(__fmul_rn(v[i][2 * e], r), g[2 * e]);
+        const float b = __fmul_rn(__fmul_rn(v[i][2 * e + 1], r), g[2 * e + 1]);
+        op[e] = pack_bf16x2(a, b);
+        if (SPLIT) {
+          const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162*>(&op[e]);
+          const float2 hf = __bfloat1622float2(hb);
+          olp[e] = pack_bf16x2(__fsub_rn(a, hf.x), __fsub_rn(b, hf.y));
+        }
+      }
       *reinterpret_cast<uint4*>(yr + c * 8) = o;
+      if (SPLIT) *reinterpret_cast<uint4*>(y_lo + row * (size_t)D + c * 8) = olo;
     }
   }
 }
@@ -111,18 +124,18 @@ static void rms_geometry(int64_t D, int* threads, int* cpt) {
   *cpt = p;
 }
 
-template <typename Tin>
+template <typename Tin, bool SPLIT = false>
 static bi_status launch_rms(const Tin* x, const bf16* g, bf16* y, int64_t M, int64_t D, float eps,
-                            cudaStream_t s) {
+                            cudaStream_t s, bf16* y_lo = nullptr) {
   int T, cpt;
   rms_geometry(D, &T, &cpt);
   dim3 grid((unsigned)M), block(T);
   switch (cpt) {
-    case 1: rmsnorm_kernel<Tin, 1><<<grid, block, 0, s>>>(x, g, y, (int)D, eps); break;
-    case 2: rmsnorm_kernel<Tin, 2><<<grid, block, 0, s>>>(x, g, y, (int)D, eps); break;
-    case 4: rmsnorm_kernel<Tin, 4><<<grid, block, 0, s>>>(x, g, y, (int)D, eps); break;
-    case 8: rmsnorm_kernel<Tin, 8><<<grid, block, 0, s>>>(x, g, y, (int)D, eps); break;
-    case 16: rmsnorm_kernel<Tin, 16><<<grid, block, 0, s>>>(x, g, y, (int)D, eps); break;
+    case 1: rmsnorm_kernel<Tin, 1, SPLIT><<<grid, block, 0, s>>>(x, g, y, y_lo, (int)D, eps); break;
+    case 2: rmsnorm_kernel<Tin, 2, SPLIT><<<grid, block, 0, s>>>(x, g, y, y_lo, (int)D, eps); break;
+    case 4: rmsnorm_kernel<Tin, 4, SPLIT><<<grid, block, 0, s>>>(x, g, y, y_lo, (int)D, eps); break;
+    case 8: rmsnorm_kernel<Tin, 8, SPLIT><<<grid, block, 0, s>>>(x, g, y, y_lo, (int)D, eps); break;
+    case 16: rmsnorm_kernel<Tin, 16, SPLIT><<<grid, block, 0, s>>>(x, g, y, y_lo, (int)D, eps); break;
     default: return fail(BI_ERR_SHAPE, "rmsnorm: D=%lld unsupported", (long long)D);
   }
   BI_CHECK_LAUNCH("rmsnorm launch");
@@ -160,4 +173,15 @@ extern "C" bi_status bi_rmsnorm_f32in(const float* x, const void* gamma, void* y
   if ((st = require_sm100()) != BI_OK) return st;
   return launch_rms<float>(x, static_cast<const bf16*>(gamma), static_cast<bf16*>(y), M, D, eps,
                            static_cast<cudaStream_t>(stream));
+}
+
+extern "C" bi_status bi_rmsnorm_split(const float* x, const void* gamma, void* y_hi, void* y_lo,
+                                      int64_t M, int64_t D, float eps, void* stream) {
+  bi_status st = check_rms(x, gamma, y_hi, M, D, eps);
+  if (st != BI_OK) return st;
+  if (!y_lo || !aligned16(y_lo)) return fail(BI_ERR_ALIGN, "rmsnorm_split: y_lo null or misaligned");
+  if (M == 0) return BI_OK;
+  if ((st = require_sm100()) != BI_OK) return st;
+  return launch_rms<float, true>(x, static_cast<const bf16*>(gamma), static_cast<bf16*>(y_hi), M, D,
+                                 eps, static_cast<cudaStream_t>(stream), static_cast<bf16*>(y_lo));
 }

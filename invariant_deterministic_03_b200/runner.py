@@ -19,10 +19,11 @@ class PagedKV:
     """KV caches for every layer plus the page tables of live sequences."""
 
     def __init__(self, n_layers: int, num_pages: int, n_kv_heads: int, max_pages_per_seq: int,
-                 seed: int = 0, device="cuda:0", zero=True):
+                 seed: int = 0, device="cuda:0", zero=True, precision: int = 0):
         self.num_pages = num_pages
         self.max_pages = max_pages_per_seq
-        self.k, self.v = _bi.new_kv_cache(num_pages, n_kv_heads, device, n_layers, zero=zero)
+        self.k, self.v = _bi.new_kv_cache(num_pages, n_kv_heads, device, n_layers, zero=zero,
+                                          precision=precision)
         self.free = synth.permutation(num_pages, seed).tolist()
         self.pages: dict[int, list[int]] = {}
         self.length: dict[int, int] = {}
@@ -89,7 +90,7 @@ class Engine:
         self.cfg = cfg
         self.model = _bi.Model(cfg, weights_dev)
         self.kv = PagedKV(cfg["n_layers"], num_pages, cfg["n_kv_heads"], max_pages_per_seq,
-                          seed, device)
+                          seed, device, precision=self.model.precision)
         self.device = device
         self.max_tokens, self.max_logits = max_tokens, max_logits
         ws = self.model.workspace_size(max_tokens, max_logits, cfg["max_pos"])
