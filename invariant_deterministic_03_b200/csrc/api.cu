@@ -25,6 +25,7 @@ bi_status fail(bi_status st, const char* fmt, ...) {
 }
 
 bi_status cuda_fail(cudaError_t e, const char* where) {
+  cudaGetLastError();  // clear a non-sticky error so the caller's next CUDA call is not blamed
   return fail(BI_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
 }
 

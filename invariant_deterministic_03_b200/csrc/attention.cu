@@ -45,8 +45,10 @@ constexpr uint32_t OFF_K = 2 * TILE_BYTES;      // 2 buffers
 constexpr uint32_t OFF_V = 4 * TILE_BYTES;      // 2 buffers
 constexpr uint32_t OFF_P = 6 * TILE_BYTES;
 constexpr uint32_t OFF_BAR = 7 * TILE_BYTES;
-constexpr uint32_t OFF_RING = OFF_BAR + 256;   // producer's page-row ring
-constexpr size_t SMEM_BYTES = 1024 + 7 * TILE_BYTES + 256 + 8 * sizeof(int32_t) * 2 * 8;
+constexpr uint32_t OFF_RING = OFF_BAR + 256;   // producer's page-row ring (16 x 64 B)
+constexpr uint32_t OFF_RED = OFF_RING + 1024;  // decode quarter exchange [2][4 warps][8 heads] fp32
+constexpr size_t SMEM_BYTES = 1024 + 7 * TILE_BYTES + 256 + 1024 + 256;
+static_assert(SMEM_BYTES <= 232448, "attention: shared memory above the 227 KB per-CTA limit");
 // warps 0-3: one thread per MMA row (softmax, O rescale, partials)
 // warp 4: TMA producer; warp 5: TMEM allocator and MMA issuer
 constexpr int THREADS = 192;
@@ -118,22 +120,20 @@ __device__ __forceinline__ void tile_rows(const Params& p, int b, int g, int L, 
                                           TileRows& r) {
   const int32_t k_rows_total = p.num_pages * p.Hkv * PAGE;
   const int32_t v_rows_total = p.num_pages * p.Hkv * HD;
+  const int32_t* bt = p.block_table + (size_t)b * p.max_pages;
+  // all eight entries loaded unconditionally (clamped index, always inside the
+  // row) so the loads go out together; validity is applied afterwards
+  int32_t pid[PAGES_PER_TILE];
+#pragma unroll
+  for (int i = 0; i < PAGES_PER_TILE; ++i) pid[i] = bt[min(tile * PAGES_PER_TILE + i, p.max_pages - 1)];
 #pragma unroll
   for (int i = 0; i < PAGES_PER_TILE; ++i) {
     const int pidx = tile * PAGES_PER_TILE + i;
-    r.k[i] = k_rows_total;
-    r.v[i] = v_rows_total;
-    if (pidx * PAGE < L && pidx < p.max_pages) {
-      const int32_t pid = p.block_table[(size_t)b * p.max_pages + pidx];
-      if (pid >= 0 && pid < p.num_pages) {
-        r.k[i] = (pid * p.Hkv + g) * PAGE;
-        r.v[i] = (pid * p.Hkv + g) * HD;
-      } else {
-        set_status(p.status, BI_DEV_BAD_PAGE);
-      }
-    } else if (pidx * PAGE < L) {
-      set_status(p.status, BI_DEV_BAD_PAGE);
-    }
+    const bool in_seq = pidx * PAGE < L;
+    const bool ok = in_seq && pidx < p.max_pages && pid[i] >= 0 && pid[i] < p.num_pages;
+    r.k[i] = ok ? (pid[i] * p.Hkv + g) * PAGE : k_rows_total;
+    r.v[i] = ok ? (pid[i] * p.Hkv + g) * HD : v_rows_total;
+    if (in_seq && !ok) set_status(p.status, BI_DEV_BAD_PAGE);
   }
 }
 
@@ -148,20 +148,6 @@ __device__ __forceinline__ void prefetch_tile(const Params& p, const CUtensorMap
       tma_prefetch_2d(tmV, 0, r.v[i]);
     }
   }
-}
-
-__device__ __forceinline__ void load_kv_tile(const CUtensorMap* tmK, const CUtensorMap* tmV,
-                                             uint8_t* kbuf, uint8_t* vbuf, uint64_t* kbar,
-                                             uint64_t* vbar, const TileRows& r) {
-  mbar_arrive_expect_tx(kbar, TILE_BYTES);
-#pragma unroll
-  for (int i = 0; i < PAGES_PER_TILE; ++i) {
-    tma_load_2d(kbuf + i * 2048, tmK, kbar, 0, r.k[i]);
-    tma_load_2d(kbuf + 16384 + i * 2048, tmK, kbar, 64, r.k[i]);
-  }
-  mbar_arrive_expect_tx(vbar, TILE_BYTES);
-#pragma unroll
-  for (int i = 0; i < PAGES_PER_TILE; ++i) tma_load_2d(vbuf + i * 4096, tmV, vbar, 0, r.v[i]);
 }
 
 // Walks the (item, tile) sequence of one CTA.
@@ -189,8 +175,8 @@ __device__ __forceinline__ void cursor_start(const Params& p, Cursor& c) {
   cursor_next(p, c);
 }
 
-constexpr int PF_AHEAD = 4;   // tiles prefetched into L2 ahead of the shared-memory loads
-constexpr int PF_RING = 8;    // ring of looked-up page rows (power of two > PF_AHEAD)
+constexpr int PF_AHEAD = 4;   // tiles prefetched into L2 ahead of the K loads
+constexpr int PF_RING = 16;   // looked-up page rows, from the oldest V load to the newest prefetch
 
 __device__ __forceinline__ void issue_s(uint32_t tmem_s, uint32_t q_addr, uint32_t k_addr) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
@@ -216,6 +202,53 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t p_addr, uint3
   }
 }
 
+// 2^x by the hardware approximation (ex2.approx.ftz: relative error below
+// 2^-22, results under 2^-126 flushed to zero). Used identically by every row.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// One quarter (32 keys) of a row's tile: P_c = bf16(2^(S_c * scale_log2 -
+// m)) for c < nvalid (else 0), packed two per word into P[0..15], and the
+// quarter sum of the bf16 values, added left to right. Decode and prefill both
+// build a row from exactly these quarters, so their arithmetic is the same.
+__device__ __forceinline__ float quarter_p(const uint32_t (&S)[32], int nvalid, float neg_m,
+                                           float scale_log2, uint32_t (&P)[16]) {
+  float q = 0.0f;
+#pragma unroll
+  for (int c2 = 0; c2 < 16; ++c2) {
+    // every element is evaluated and masked ones are replaced by zero with a
+    // select, so no branch serialises the loop
+    const float e0 = ex2_approx(__fmaf_rn(__uint_as_float(S[2 * c2]), scale_log2, neg_m));
+    const float e1 = ex2_approx(__fmaf_rn(__uint_as_float(S[2 * c2 + 1]), scale_log2, neg_m));
+    const uint32_t pk = pack_bf16x2(2 * c2 < nvalid ? e0 : 0.0f, 2 * c2 + 1 < nvalid ? e1 : 0.0f);
+    q = __fadd_rn(q, __uint_as_float(pk << 16));          // bf16 of element 2*c2
+    q = __fadd_rn(q, __uint_as_float(pk & 0xffff0000u));  // bf16 of element 2*c2+1
+    P[c2] = pk;
+  }
+  return q;
+}
+
+__device__ __forceinline__ float quarter_max(const uint32_t (&S)[32], int nvalid) {
+  float m = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 32; ++c) m = fmaxf(m, c < nvalid ? __uint_as_float(S[c]) : -INFINITY);
+  return m;
+}
+
+__device__ __forceinline__ void store_p_chunks(uint8_t* p_smem, int row, int quarter,
+                                               const uint32_t (&P)[16]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int chunk = quarter * 4 + k;  // 8 keys per 16-byte chunk
+    const uint32_t addr = (uint32_t)(chunk >> 3) * 16384u + (uint32_t)row * 128u +
+                          (uint32_t)(((chunk & 7) ^ (row & 7)) << 4);
+    *reinterpret_cast<uint4*>(p_smem + addr) = make_uint4(P[4 * k], P[4 * k + 1], P[4 * k + 2], P[4 * k + 3]);
+  }
+}
+
 // Bounded wait for the fills a producer issued into a buffer, so that no copy
 // is still landing in shared memory when an aborted CTA exits.
 __device__ __forceinline__ void drain(uint64_t* bar, int fills) {
@@ -228,9 +261,12 @@ __device__ __forceinline__ void drain(uint64_t* bar, int fills) {
 
 // Split kernel. Persistent: one CTA per SM walks work items idx = blockIdx.x,
 // blockIdx.x + gridDim.x, ...; the three roles walk the same item sequence.
-// Per tile j (counted across items) the MMA warp issues S(j) = Q K_j^T into
-// S buffer j%2 before P(j-1) V_(j-1), so the next QK^T overlaps the softmax of
-// the current tile.
+// Tiles j are counted across items. The producer keeps K and V loads apart
+// (a K buffer is free once its QK^T is done, a V buffer once its PV is done)
+// and the MMA warp issues S(j) = Q K_j^T and O += P_j V_j as soon as each is
+// ready, so loads, QK^T and the softmax of neighbouring tiles overlap.
+// DECODE selects the softmax layout (see below); both layouts run the same
+// per-row arithmetic.
 //
 // Row arithmetic (thread = row, fixed order, same in decode and prefill):
 //   first tile of the split:  m = max_j s_j (log2 domain, s_j = S_ij * scale*log2e),
@@ -239,6 +275,7 @@ __device__ __forceinline__ void drain(uint64_t* bar, int fills) {
 //                             P_j = bf16(2^(s_j - m')), l = alpha*l + sum_j P_j,
 //                             O = alpha*O (fp32, skipped when alpha == 1), O += P V (MMA)
 // sums over j run j = 0..127 in order; masked keys have P_j = 0 by selection.
+template <bool DECODE>
 __global__ void __launch_bounds__(THREADS, 1)
     attn_split_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
@@ -251,12 +288,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* q_empty = bars + 2;    // [2]
   uint64_t* k_full = bars + 4;     // [2]
   uint64_t* v_full = bars + 6;     // [2]
-  uint64_t* kv_empty = bars + 8;   // [2]
-  uint64_t* s_full = bars + 10;    // [2]
-  uint64_t* s_free = bars + 12;    // [2]
-  uint64_t* p_ready = bars + 14;
-  uint64_t* o_ready = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* k_empty = bars + 8;    // [2]
+  uint64_t* v_empty = bars + 10;   // [2]
+  uint64_t* s_full = bars + 12;    // [2]
+  uint64_t* s_free = bars + 14;    // [2]
+  uint64_t* p_ready = bars + 16;
+  uint64_t* o_ready = bars + 17;
+  uint64_t* x_bar = bars + 18;     // decode: quarter exchange among the 4 softmax warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -268,12 +307,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&q_empty[i], 1);
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 128);
     }
     mbar_init(p_ready, 128);
     mbar_init(o_ready, 1);
+    mbar_init(x_bar, 128);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -294,51 +335,93 @@ __global__ void __launch_bounds__(THREADS, 1)
       prefetch_tmap(&tmV);
       const uint32_t q_bytes = 2u * 64u * 2u * (uint32_t)(p.G * p.q_box);
       TileRows* ring = reinterpret_cast<TileRows*>(smem + OFF_RING);
-      int qi = 0, kvi = 0;
-      int q_fills[2] = {0, 0}, kv_fills[2] = {0, 0};
-      bool ok = true;
-      // prefetch cursor runs PF_AHEAD tiles in front of the load cursor
-      Cursor pf;
-      cursor_start(p, pf);
-      int pf_n = 0;  // tiles looked up and prefetched so far
-      for (; pf.valid && pf_n < PF_AHEAD; ++pf_n, cursor_next(p, pf)) {
-        TileRows& r = ring[pf_n & (PF_RING - 1)];
-        tile_rows(p, pf.it.b, pf.it.g, pf.it.L, pf.it.t0 + pf.t, r);
-        prefetch_tile(p, &tmK, &tmV, r);
+      Cursor kc, vc, pf;
+      cursor_start(p, kc);
+      vc = kc;
+      pf = kc;
+      int nk = 0, nv = 0, npf = 0, qi = 0;
+      int q_fills[2] = {0, 0}, k_fills[2] = {0, 0}, v_fills[2] = {0, 0};
+      for (; pf.valid && npf < PF_AHEAD; ++npf, cursor_next(p, pf)) {
+        tile_rows(p, pf.it.b, pf.it.g, pf.it.L, pf.it.t0 + pf.t, ring[npf & (PF_RING - 1)]);
+        prefetch_tile(p, &tmK, &tmV, ring[npf & (PF_RING - 1)]);
       }
-      for (int idx = blockIdx.x; idx < p.total_items && ok; idx += gridDim.x) {
-        Item it;
-        if (!item_at(p, idx, it, true)) continue;
-        const int qb = qi & 1;
-        if (!mbar_wait(&q_empty[qb], (((uint32_t)qi >> 1) & 1u) ^ 1u, p.status, abort_flag)) { ok = false; break; }
-        uint8_t* qdst = smem + OFF_Q + qb * TILE_BYTES;
-        mbar_arrive_expect_tx(&q_full[qb], q_bytes);
-        tma_load_3d(qdst, &tmQ, &q_full[qb], 0, it.g * p.G, it.r0 + it.q_lo);
-        tma_load_3d(qdst + 16384, &tmQ, &q_full[qb], 64, it.g * p.G, it.r0 + it.q_lo);
-        ++q_fills[qb];
-        ++qi;
-        for (int t = 0; t < it.ntiles; ++t) {
-          // look up and prefetch the tile PF_AHEAD ahead of this one
-          if (pf.valid) {
-            TileRows& r = ring[pf_n & (PF_RING - 1)];
-            tile_rows(p, pf.it.b, pf.it.g, pf.it.L, pf.it.t0 + pf.t, r);
-            prefetch_tile(p, &tmK, &tmV, r);
-            ++pf_n;
-            cursor_next(p, pf);
+      bool ok = true;
+      long long t_last = clock64();
+      while ((kc.valid || vc.valid) && ok) {
+        bool progressed = false;
+        if (kc.valid) {
+          const int kb = nk & 1, qb = qi & 1;
+          bool ready = mbar_test(&k_empty[kb], (((uint32_t)nk >> 1) & 1u) ^ 1u);
+          if (ready && kc.t == 0) ready = mbar_test(&q_empty[qb], (((uint32_t)qi >> 1) & 1u) ^ 1u);
+          if (ready) {
+            if (kc.t == 0) {  // first tile of an item: its Q rows
+              uint8_t* qdst = smem + OFF_Q + qb * TILE_BYTES;
+              if (!DECODE) {
+                mbar_arrive_expect_tx(&q_full[qb], q_bytes);
+                tma_load_3d(qdst, &tmQ, &q_full[qb], 0, kc.it.g * p.G, kc.it.r0 + kc.it.q_lo);
+                tma_load_3d(qdst + 16384, &tmQ, &q_full[qb], 64, kc.it.g * p.G, kc.it.r0 + kc.it.q_lo);
+              } else {
+                // the G head rows again at rows 32, 64 and 96 (one copy per softmax warp)
+                mbar_arrive_expect_tx(&q_full[qb], 4u * q_bytes);
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                  tma_load_3d(qdst + w * 32 * 128, &tmQ, &q_full[qb], 0, kc.it.g * p.G, kc.it.r0 + kc.it.q_lo);
+                  tma_load_3d(qdst + 16384 + w * 32 * 128, &tmQ, &q_full[qb], 64, kc.it.g * p.G,
+                              kc.it.r0 + kc.it.q_lo);
+                }
+              }
+              ++q_fills[qb];
+              ++qi;
+            }
+            if (pf.valid) {  // keep the page lookups and L2 prefetches PF_AHEAD tiles ahead
+              tile_rows(p, pf.it.b, pf.it.g, pf.it.L, pf.it.t0 + pf.t, ring[npf & (PF_RING - 1)]);
+              prefetch_tile(p, &tmK, &tmV, ring[npf & (PF_RING - 1)]);
+              ++npf;
+              cursor_next(p, pf);
+            }
+            const TileRows& r = ring[nk & (PF_RING - 1)];
+            uint8_t* kbuf = smem + OFF_K + kb * TILE_BYTES;
+            mbar_arrive_expect_tx(&k_full[kb], TILE_BYTES);
+#pragma unroll
+            for (int i = 0; i < PAGES_PER_TILE; ++i) {
+              tma_load_2d(kbuf + i * 2048, &tmK, &k_full[kb], 0, r.k[i]);
+              tma_load_2d(kbuf + 16384 + i * 2048, &tmK, &k_full[kb], 64, r.k[i]);
+            }
+            ++k_fills[kb];
+            ++nk;
+            cursor_next(p, kc);
+            progressed = true;
           }
-          const int kb = kvi & 1;
-          if (!mbar_wait(&kv_empty[kb], (((uint32_t)kvi >> 1) & 1u) ^ 1u, p.status, abort_flag)) { ok = false; break; }
-          load_kv_tile(&tmK, &tmV, smem + OFF_K + kb * TILE_BYTES, smem + OFF_V + kb * TILE_BYTES,
-                       &k_full[kb], &v_full[kb], ring[kvi & (PF_RING - 1)]);
-          ++kv_fills[kb];
-          ++kvi;
+        }
+        if (vc.valid && nv < nk) {
+          const int vb = nv & 1;
+          if (mbar_test(&v_empty[vb], (((uint32_t)nv >> 1) & 1u) ^ 1u)) {
+            const TileRows& r = ring[nv & (PF_RING - 1)];
+            uint8_t* vbuf = smem + OFF_V + vb * TILE_BYTES;
+            mbar_arrive_expect_tx(&v_full[vb], TILE_BYTES);
+#pragma unroll
+            for (int i = 0; i < PAGES_PER_TILE; ++i) tma_load_2d(vbuf + i * 4096, &tmV, &v_full[vb], 0, r.v[i]);
+            ++v_fills[vb];
+            ++nv;
+            cursor_next(p, vc);
+            progressed = true;
+          }
+        }
+        if (progressed) {
+          t_last = clock64();
+        } else if (__nanosleep(32), *abort_flag) {
+          ok = false;
+        } else if (clock64() - t_last > kWaitLimitCycles) {
+          set_status(p.status, BI_DEV_WAIT_TIMEOUT);
+          *abort_flag = 1;
+          ok = false;
         }
       }
       if (!ok) {
         for (int i = 0; i < 2; ++i) {
           drain(&q_full[i], q_fills[i]);
-          drain(&k_full[i], kv_fills[i]);
-          drain(&v_full[i], kv_fills[i]);
+          drain(&k_full[i], k_fills[i]);
+          drain(&v_full[i], v_fills[i]);
         }
       }
     }
@@ -347,62 +430,90 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       const uint32_t sQ0 = smem_u32(smem + OFF_Q), sK0 = smem_u32(smem + OFF_K);
       const uint32_t sV0 = smem_u32(smem + OFF_V), sP = smem_u32(smem + OFF_P);
-      int qi = 0, j = 0;
+      Cursor sc;
+      cursor_start(p, sc);
+      int nS = 0, nP = 0, qi = 0;
+      // per issued S tile (bit n & 31): P V accumulates, item's last tile, Q buffer
+      uint32_t acc_bits = 0, last_bits = 0, qb_bits = 0;
       bool ok = true;
-      // P V of the previous tile, issued after the next tile's QK^T
-      bool pend = false, pend_acc = false, pend_last = false;
-      int pend_j = 0, pend_qb = 0;
-      auto issue_pending = [&]() -> bool {
-        const int kb = pend_j & 1;
-        if (!mbar_wait(p_ready, (uint32_t)pend_j & 1u, p.status, abort_flag)) return false;
-        if (!mbar_wait(&v_full[kb], ((uint32_t)pend_j >> 1) & 1u, p.status, abort_flag)) return false;
-        tc_fence_after();
-        issue_pv(tmem + TMEM_O, sP, sV0 + kb * TILE_BYTES, pend_acc);
-        mma_commit(o_ready);
-        mma_commit(&kv_empty[kb]);
-        if (pend_last) mma_commit(&q_empty[pend_qb]);
-        pend = false;
-        return true;
-      };
-      for (int idx = blockIdx.x; idx < p.total_items && ok; idx += gridDim.x) {
-        Item it;
-        if (!item_at(p, idx, it, false)) continue;
-        const int qb = qi & 1;
-        if (!mbar_wait(&q_full[qb], ((uint32_t)qi >> 1) & 1u, p.status, abort_flag)) { ok = false; break; }
-        for (int t = 0; t < it.ntiles; ++t, ++j) {
-          const int kb = j & 1;
-          if (!mbar_wait(&k_full[kb], ((uint32_t)j >> 1) & 1u, p.status, abort_flag) ||
-              !mbar_wait(&s_free[kb], (((uint32_t)j >> 1) & 1u) ^ 1u, p.status, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          issue_s(tmem + kb * 128, sQ0 + qb * TILE_BYTES, sK0 + kb * TILE_BYTES);
-          mma_commit(&s_full[kb]);
-          if (pend && !issue_pending()) { ok = false; break; }
-          pend = true;
-          pend_j = j;
-          pend_acc = t > 0;
-          pend_last = t == it.ntiles - 1;
-          pend_qb = qb;
+      long long t_last = clock64();
+      while ((sc.valid || nP < nS) && ok) {
+        bool progressed = false;
+        if (sc.valid && nS - nP < 2) {
+          const int kb = nS & 1, qb = qi & 1;
+          const bool ready = (sc.t != 0 || mbar_test(&q_full[qb], ((uint32_t)qi >> 1) & 1u)) &&
+                             mbar_test(&k_full[kb], ((uint32_t)nS >> 1) & 1u) &&
+                             mbar_test(&s_free[kb], (((uint32_t)nS >> 1) & 1u) ^ 1u);
+          if (ready) {
+            tc_fence_after();
+            issue_s(tmem + kb * 128, sQ0 + qb * TILE_BYTES, sK0 + kb * TILE_BYTES);
+            mma_commit(&s_full[kb]);
+            mma_commit(&k_empty[kb]);
+            const uint32_t bit = 1u << (nS & 31);
+            acc_bits = sc.t > 0 ? (acc_bits | bit) : (acc_bits & ~bit);
+            last_bits = sc.t == sc.it.ntiles - 1 ? (last_bits | bit) : (last_bits & ~bit);
+            qb_bits = qb ? (qb_bits | bit) : (qb_bits & ~bit);
+            if (sc.t == sc.it.ntiles - 1) ++qi;
+            ++nS;
+            cursor_next(p, sc);
+            progressed = true;
+          }
         }
-        ++qi;
+        if (nP < nS) {
+          const int vb = nP & 1;
+          if (mbar_test(p_ready, (uint32_t)nP & 1u) && mbar_test(&v_full[vb], ((uint32_t)nP >> 1) & 1u)) {
+            const uint32_t bit = 1u << (nP & 31);
+            tc_fence_after();
+            issue_pv(tmem + TMEM_O, sP, sV0 + vb * TILE_BYTES, (acc_bits & bit) != 0);
+            mma_commit(o_ready);
+            mma_commit(&v_empty[vb]);
+            if (last_bits & bit) mma_commit(&q_empty[(qb_bits & bit) ? 1 : 0]);
+            ++nP;
+            progressed = true;
+          }
+        }
+        if (progressed) {
+          t_last = clock64();
+        } else if (__nanosleep(32), *abort_flag) {
+          ok = false;
+        } else if (clock64() - t_last > kWaitLimitCycles) {
+          set_status(p.status, BI_DEV_WAIT_TIMEOUT);
+          *abort_flag = 1;
+          ok = false;
+        }
       }
-      if (ok && pend) issue_pending();
     }
   } else {
-    // ------------------------------------------------ one thread per MMA row
+    // ------------------------------------------------ softmax warps 0-3
+    // Prefill layout: thread r owns MMA row r = (query r / G, head r % G) and
+    // all 128 keys of a tile (its four quarters in turn).
+    // Decode layout (one query per item): the item's G head rows are loaded
+    // into rows 32w + i of every warp w (identical rows, identical S), and
+    // warp w computes quarter w (keys 32w .. 32w+31) of every head i < G;
+    // quarter maxima and quarter sums are exchanged through shared memory.
+    constexpr bool decode = DECODE;
     const int r = threadIdx.x;  // 0..127 == TMEM lane
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const int qr = r / p.G;
-    const int hj = r - qr * p.G;
-    int j = 0;
+    const int qr = decode ? 0 : r / p.G;
+    const int hj = decode ? lane : r - qr * p.G;
+    float* red = reinterpret_cast<float*>(smem + OFF_RED);  // [2][4 warps][8 head rows]
+    int j = 0, xc = 0;
     bool ok = true;
     bool o_pending = false;  // o_ready of tile j-1 not yet waited for
+    auto exchange = [&](float v, int which) -> bool {
+      if (lane < 8) red[(which * 4 + warp) * 8 + lane] = v;
+      mbar_arrive(x_bar);
+      const bool done = mbar_wait(x_bar, (uint32_t)xc & 1u, p.status, abort_flag);
+      ++xc;
+      return done;
+    };
     for (int idx = blockIdx.x; idx < p.total_items && ok; idx += gridDim.x) {
       Item it;
       if (!item_at(p, idx, it, false)) continue;
       const int q_idx = it.q_lo + qr;
       const int pos = it.L - it.nb + q_idx;
-      const bool row_valid = (q_idx < it.q_hi) && (pos >= it.key_lo);
-      const bool warp_valid = __any_sync(0xffffffffu, row_valid);
+      const bool row_valid = (decode ? lane < p.G : true) && (q_idx < it.q_hi) && (pos >= it.key_lo);
+      const bool warp_valid = decode ? true : __any_sync(0xffffffffu, row_valid);
       const int last_page = (it.L - 1) / PAGE;
       const int tail = it.L % PAGE;
       float m = -INFINITY, l = 0.0f;
@@ -410,78 +521,112 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int sb = j & 1;
         const int kb0 = (it.t0 + t) * TILE;
         const bool need = row_valid && kb0 <= pos;
+        const int nvalid = need ? min(TILE, pos + 1 - kb0) : 0;
         if (!mbar_wait(&s_full[sb], ((uint32_t)j >> 1) & 1u, p.status, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        uint32_t S[128];
-        if (warp_valid) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            tmem_ld32(tmem + sb * 128 + lane_off + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&S[q * 32]));
-          tmem_ld_wait();
-        }
-        tc_fence_before();
-        mbar_arrive(&s_free[sb]);
-
         float alpha = 1.0f, m_new = 0.0f;
-        // P is packed (2 bf16 per word) into S[0..63] as S is consumed
-        uint32_t* P = S;
-        float lsum = 0.0f;
-        if (warp_valid) {
-          const int nvalid = need ? min(TILE, pos + 1 - kb0) : 0;
-          float m_tile = -INFINITY;
+        if constexpr (decode) {
+          // ---- decode layout: this warp's quarter of every head row
+          uint32_t S[32], P[16];
+          tmem_ld32(tmem + sb * 128 + lane_off + warp * 32, S);
+          tmem_ld_wait();
+          tc_fence_before();
+          mbar_arrive(&s_free[sb]);
+          const int nq = min(32, max(0, nvalid - warp * 32));
+          if (!exchange(quarter_max(S, nq), 0)) { ok = false; break; }
+          float mraw = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c < nvalid) m_tile = fmaxf(m_tile, __fmul_rn(__uint_as_float(S[c]), p.scale_log2));
+          for (int w = 0; w < 4; ++w) mraw = fmaxf(mraw, red[w * 8 + (lane & 7)]);
           if (need) {
-            m_new = fmaxf(m, m_tile);
-            alpha = exp2f(__fsub_rn(m, m_new));
+            m_new = fmaxf(m, __fmul_rn(mraw, p.scale_log2));
+            alpha = ex2_approx(__fsub_rn(m, m_new));
           }
-#pragma unroll
-          for (int c2 = 0; c2 < 64; ++c2) {
-            float pf[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int c = 2 * c2 + h;
-              const float sv = __fmul_rn(__uint_as_float(S[c]), p.scale_log2);
-              const float ev = (c < nvalid) ? exp2f(__fsub_rn(sv, m_new)) : 0.0f;
-              pf[h] = __bfloat162float(__float2bfloat16_rn(ev));
-              lsum = __fadd_rn(lsum, pf[h]);
-            }
-            P[c2] = pack_bf16x2(pf[0], pf[1]);  // exact: pf are bf16 values
-          }
+          const float qs = quarter_p(S, nq, -m_new, p.scale_log2, P);
+          if (!exchange(qs, 1)) { ok = false; break; }
           if (need) {
+            const float lsum = __fadd_rn(__fadd_rn(__fadd_rn(red[32 + lane], red[32 + 8 + lane]),
+                                                   red[32 + 16 + lane]), red[32 + 24 + lane]);
             l = (t == 0) ? lsum : __fadd_rn(__fmul_rn(alpha, l), lsum);
             m = m_new;
           }
-        }
-        // P V of the previous tile must be done before P and O are touched
-        if (o_pending) {
-          if (!mbar_wait(o_ready, (uint32_t)(j - 1) & 1u, p.status, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          o_pending = false;
-        }
-        if (warp_valid) {
-#pragma unroll
-          for (int chunk = 0; chunk < 16; ++chunk) {
-            // 8 keys per 16-byte chunk; 128-byte swizzle within each 64-key half
-            const uint32_t addr = (uint32_t)(chunk >> 3) * 16384u + (uint32_t)r * 128u +
-                                  (uint32_t)(((chunk & 7) ^ (r & 7)) << 4);
-            *reinterpret_cast<uint4*>(smem + OFF_P + addr) =
-                make_uint4(P[4 * chunk], P[4 * chunk + 1], P[4 * chunk + 2], P[4 * chunk + 3]);
+          if (o_pending) {
+            if (!mbar_wait(o_ready, (uint32_t)(j - 1) & 1u, p.status, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            o_pending = false;
           }
-          // rescale O in tensor memory (not on the split's first tile, whose P V overwrites O)
+          if (lane < p.G) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) store_p_chunks(smem + OFF_P, v * 32 + lane, warp, P);
+          }
           if (t > 0 && __any_sync(0xffffffffu, need && alpha != 1.0f)) {
+            uint32_t o[32];
+            tmem_ld32(tmem + TMEM_O + lane_off + warp * 32, o);
+            tmem_ld_wait();
             const float a = need ? alpha : 1.0f;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint32_t o[32];
-              tmem_ld32(tmem + TMEM_O + lane_off + q * 32, o);
-              tmem_ld_wait();
-#pragma unroll
-              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__fmul_rn(__uint_as_float(o[c]), a));
-              tmem_st32(tmem + TMEM_O + lane_off + q * 32, o);
-            }
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__fmul_rn(__uint_as_float(o[c]), a));
+            tmem_st32(tmem + TMEM_O + lane_off + warp * 32, o);
             tmem_st_wait();
+          }
+        } else {
+          // ---- prefill layout: all four quarters of row r
+          uint32_t S[128];
+          if (warp_valid) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              tmem_ld32(tmem + sb * 128 + lane_off + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&S[q * 32]));
+            tmem_ld_wait();
+          }
+          tc_fence_before();
+          mbar_arrive(&s_free[sb]);
+          // P is packed (2 bf16 per word) into S[0..63] as S is consumed
+          uint32_t* P = S;
+          if (warp_valid) {
+            float mraw = -INFINITY;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              mraw = fmaxf(mraw, quarter_max(*reinterpret_cast<uint32_t(*)[32]>(&S[q * 32]),
+                                             min(32, max(0, nvalid - q * 32))));
+            if (need) {
+              m_new = fmaxf(m, __fmul_rn(mraw, p.scale_log2));
+              alpha = ex2_approx(__fsub_rn(m, m_new));
+            }
+            float qs[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              qs[q] = quarter_p(*reinterpret_cast<uint32_t(*)[32]>(&S[q * 32]),
+                                min(32, max(0, nvalid - q * 32)), -m_new, p.scale_log2,
+                                *reinterpret_cast<uint32_t(*)[16]>(&P[q * 16]));
+            if (need) {
+              const float lsum = __fadd_rn(__fadd_rn(__fadd_rn(qs[0], qs[1]), qs[2]), qs[3]);
+              l = (t == 0) ? lsum : __fadd_rn(__fmul_rn(alpha, l), lsum);
+              m = m_new;
+            }
+          }
+          // P V of the previous tile must be done before P and O are touched
+          if (o_pending) {
+            if (!mbar_wait(o_ready, (uint32_t)(j - 1) & 1u, p.status, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            o_pending = false;
+          }
+          if (warp_valid) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              store_p_chunks(smem + OFF_P, r, q, *reinterpret_cast<uint32_t(*)[16]>(&P[q * 16]));
+            // rescale O in tensor memory (not on the split's first tile, whose P V overwrites O)
+            if (t > 0 && __any_sync(0xffffffffu, need && alpha != 1.0f)) {
+              const float a = need ? alpha : 1.0f;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                uint32_t o[32];
+                tmem_ld32(tmem + TMEM_O + lane_off + q * 32, o);
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__fmul_rn(__uint_as_float(o[c]), a));
+                tmem_st32(tmem + TMEM_O + lane_off + q * 32, o);
+              }
+              tmem_st_wait();
+            }
           }
         }
         // zero V slots at or past the sequence end inside this tile's last page
@@ -505,13 +650,23 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!mbar_wait(o_ready, (uint32_t)(j - 1) & 1u, p.status, abort_flag)) { ok = false; break; }
       tc_fence_after();
       o_pending = false;
-      if (warp_valid) {
-        float* dst = nullptr;
+      const size_t widx = ((size_t)(it.r0 + q_idx) * p.Hq + (size_t)(it.g * p.G + hj)) * p.n_split_max + it.s;
+      if constexpr (decode) {
+        uint32_t o[32];
+        tmem_ld32(tmem + TMEM_O + lane_off + warp * 32, o);
+        tmem_ld_wait();
         if (row_valid) {
-          const size_t widx = ((size_t)(it.r0 + q_idx) * p.Hq + (size_t)(it.g * p.G + hj)) * p.n_split_max + it.s;
-          dst = p.ws_o + widx * HD;
-          *reinterpret_cast<float2*>(p.ws_ml + widx * 2) = make_float2(m, l);
+          float* dst = p.ws_o + widx * HD + warp * 32;
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4)
+            reinterpret_cast<float4*>(dst)[c4] =
+                make_float4(__uint_as_float(o[4 * c4]), __uint_as_float(o[4 * c4 + 1]),
+                            __uint_as_float(o[4 * c4 + 2]), __uint_as_float(o[4 * c4 + 3]));
+          if (warp == 0) *reinterpret_cast<float2*>(p.ws_ml + widx * 2) = make_float2(m, l);
         }
+      } else if (warp_valid) {
+        float* dst = p.ws_o + widx * HD;
+        if (row_valid) *reinterpret_cast<float2*>(p.ws_ml + widx * 2) = make_float2(m, l);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint32_t o[32];
@@ -702,14 +857,20 @@ static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t ma
   int dev = 0;
   cudaGetDevice(&dev);
   if (!attr_set[dev & 63]) {
-    cudaError_t e = cudaFuncSetAttribute(attn_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(attn_split_kernel<true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attn_split_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e, "attention: smem attribute");
     attr_set[dev & 63] = true;
   }
   const int sms = num_sms();
   const int grid = (int)(total_items < sms ? total_items : sms);
-  attn_split_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
+  if (cu_q)
+    attn_split_kernel<false><<<grid, THREADS, SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
+  else
+    attn_split_kernel<true><<<grid, THREADS, SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
   BI_CHECK_LAUNCH("attention split launch");
 
   CombineParams c;

@@ -242,7 +242,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
 }
 
 __global__ void zero_fill_kernel(void* C, int64_t ldc, int32_t c_f32, int32_t M, int32_t N) {
