@@ -122,9 +122,13 @@ bi_status bi_gemm(const void* A, int64_t lda, const void* W, int64_t ldw,
  * the attention kernel runs, so every key is read from the same layout
  * whether it was cached earlier or belongs to the chunk in flight.
  *
- * Layout (one page = BI_PAGE_SIZE tokens, d_h = BI_HEAD_DIM):
- *   k_cache [num_pages, num_kv_heads, 16, 128] bf16   (key rows, d contiguous)
- *   v_cache [num_pages, num_kv_heads, 128, 16] bf16   (values stored transposed)
+ * Layout (one page = BI_PAGE_SIZE tokens, d_h = BI_HEAD_DIM): each cache is
+ * num_pages x num_kv_heads blocks of 16 x 128 bf16 (4 KB), block (page, g) at
+ * element offset (page * num_kv_heads + g) * 2048. Inside a block the
+ * elements sit in the tensor core's canonical K-major no-swizzle order (8 x 8
+ * core matrices of 128 bytes), so attention copies a block as one piece:
+ *   k_cache: key (slot o, dim d) at (o/8)*1024 + (d/8)*64 + (o%8)*8 + d%8
+ *   v_cache: value (dim d, slot o) at (d/8)*128 + (o/8)*64 + (d%8)*8 + o%8
  * Token slot s = page * 16 + offset. */
 typedef struct {
   int32_t num_pages;

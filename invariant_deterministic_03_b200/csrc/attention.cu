@@ -28,6 +28,10 @@
 // Masked keys get P = 0 by selection (never by arithmetic on -inf), and
 // cache slots at or past the sequence length are zeroed in shared memory so
 // that stale cache contents cannot reach the P.V products.
+//
+// Each (page, kv head) block of the cache is stored in the tensor core's
+// canonical K-major no-swizzle order (8 x 16-byte core matrices), so a tile is
+// 8 + 8 contiguous 4 KB bulk copies straight into MMA operand layout.
 #include "common.cuh"
 #include "host.h"
 
@@ -45,9 +49,9 @@ constexpr uint32_t OFF_K = 2 * TILE_BYTES;      // 2 buffers
 constexpr uint32_t OFF_V = 4 * TILE_BYTES;      // 2 buffers
 constexpr uint32_t OFF_P = 6 * TILE_BYTES;
 constexpr uint32_t OFF_BAR = 7 * TILE_BYTES;
-constexpr uint32_t OFF_RING = OFF_BAR + 256;   // producer's page-row ring (16 x 64 B)
-constexpr uint32_t OFF_RED = OFF_RING + 1024;  // decode quarter exchange [2][4 warps][8 heads] fp32
-constexpr size_t SMEM_BYTES = 1024 + 7 * TILE_BYTES + 256 + 1024 + 256;
+constexpr uint32_t OFF_RING = OFF_BAR + 256;   // producer's page-id ring (16 x 32 B)
+constexpr uint32_t OFF_RED = OFF_RING + 512;   // decode quarter exchange [2][4 warps][8 heads] fp32
+constexpr size_t SMEM_BYTES = 1024 + 7 * TILE_BYTES + 256 + 512 + 256;
 static_assert(SMEM_BYTES <= 232448, "attention: shared memory above the 227 KB per-CTA limit");
 // warps 0-3: one thread per MMA row (softmax, O rescale, partials)
 // warp 4: TMA producer; warp 5: TMEM allocator and MMA issuer
@@ -57,6 +61,8 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_O = 256;
 
 struct Params {
+  const uint8_t* kc;  // bf16 key cache, 4 KB per (page, kv head) block
+  const uint8_t* vc;  // bf16 value cache, same blocking
   const int32_t* block_table;
   const int32_t* seq_lens;
   const int32_t* cu_q;  // null: decode (one query per sequence, row b)
@@ -108,18 +114,20 @@ __device__ __forceinline__ bool item_at(const Params& p, int idx, Item& it, bool
   return true;
 }
 
-// Cache rows of the 8 pages of one 128-key tile (page ids looked up in the
-// sequence's block table). Pages past the sequence end, or with an id outside
-// the cache, get the first out-of-range row: TMA fills those boxes with zeros.
+// A zero (page, head) block: the source for pages past a sequence's end (and
+// for bad page ids), so the masked keys of a tile always meet zero values.
+__device__ __align__(128) uint8_t g_attn_zero_block[4096];
+
+constexpr uint32_t BLOCK_BYTES = PAGE * HD * 2;  // 4 KB: one (page, kv head) block
+
+// Page ids of the 8 pages of one 128-key tile (looked up in the sequence's
+// block table); -1 marks a page past the sequence end or a bad id.
 struct TileRows {
-  int32_t k[PAGES_PER_TILE];
-  int32_t v[PAGES_PER_TILE];
+  int32_t pid[PAGES_PER_TILE];
 };
 
 __device__ __forceinline__ void tile_rows(const Params& p, int b, int g, int L, int tile,
                                           TileRows& r) {
-  const int32_t k_rows_total = p.num_pages * p.Hkv * PAGE;
-  const int32_t v_rows_total = p.num_pages * p.Hkv * HD;
   const int32_t* bt = p.block_table + (size_t)b * p.max_pages;
   // all eight entries loaded unconditionally (clamped index, always inside the
   // row) so the loads go out together; validity is applied afterwards
@@ -131,23 +139,14 @@ __device__ __forceinline__ void tile_rows(const Params& p, int b, int g, int L, 
     const int pidx = tile * PAGES_PER_TILE + i;
     const bool in_seq = pidx * PAGE < L;
     const bool ok = in_seq && pidx < p.max_pages && pid[i] >= 0 && pid[i] < p.num_pages;
-    r.k[i] = ok ? (pid[i] * p.Hkv + g) * PAGE : k_rows_total;
-    r.v[i] = ok ? (pid[i] * p.Hkv + g) * HD : v_rows_total;
+    r.pid[i] = ok ? pid[i] : -1;
     if (in_seq && !ok) set_status(p.status, BI_DEV_BAD_PAGE);
   }
 }
 
-__device__ __forceinline__ void prefetch_tile(const Params& p, const CUtensorMap* tmK,
-                                              const CUtensorMap* tmV, const TileRows& r) {
-  const int32_t k_rows_total = p.num_pages * p.Hkv * PAGE;
-#pragma unroll
-  for (int i = 0; i < PAGES_PER_TILE; ++i) {
-    if (r.k[i] < k_rows_total) {
-      tma_prefetch_2d(tmK, 0, r.k[i]);
-      tma_prefetch_2d(tmK, 64, r.k[i]);
-      tma_prefetch_2d(tmV, 0, r.v[i]);
-    }
-  }
+__device__ __forceinline__ const uint8_t* block_src(const uint8_t* cache, int32_t pid, int Hkv,
+                                                    int g) {
+  return pid < 0 ? g_attn_zero_block : cache + ((size_t)pid * Hkv + g) * BLOCK_BYTES;
 }
 
 // Walks the (item, tile) sequence of one CTA.
@@ -175,15 +174,19 @@ __device__ __forceinline__ void cursor_start(const Params& p, Cursor& c) {
   cursor_next(p, c);
 }
 
-constexpr int PF_AHEAD = 4;   // tiles prefetched into L2 ahead of the K loads
-constexpr int PF_RING = 16;   // looked-up page rows, from the oldest V load to the newest prefetch
+constexpr int PF_AHEAD = 4;   // page-table lookups run this many tiles ahead of the K loads
+constexpr int PF_RING = 16;   // looked-up page ids, from the oldest V load to the newest lookup
 
+// S = Q K^T. Q: 128 rows x 128 d, 128-byte swizzle in two 64-column halves.
+// K: 8 page blocks of 16 keys, canonical no-swizzle K-major: core matrices of
+// 8 keys x 8 d (128 B), d-chunks 128 B apart (LBO), 8-key groups 2 KB apart
+// (SBO, uniform across the blocks of a tile).
 __device__ __forceinline__ void issue_s(uint32_t tmem_s, uint32_t q_addr, uint32_t k_addr) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
 #pragma unroll
   for (int kk = 0; kk < HD / 16; ++kk) {
-    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-    mma_bf16(tmem_s, smem_desc(q_addr + off, 16, 1024, 2), smem_desc(k_addr + off, 16, 1024, 2),
+    const uint32_t qoff = (kk >> 2) * 16384 + (kk & 3) * 32;
+    mma_bf16(tmem_s, smem_desc(q_addr + qoff, 16, 1024, 2), smem_desc(k_addr + kk * 256, 128, 2048, 0),
              idesc, kk != 0);
   }
 }
@@ -195,10 +198,11 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t p_addr, uint3
 #pragma unroll
   for (int j = 0; j < PAGES_PER_TILE; ++j) {
     const uint32_t poff = (j >> 2) * 16384 + (j & 3) * 32;
-    // V^T page block j: [128 d rows x 16 keys], 32-byte rows, 32-byte swizzle,
-    // 8-row groups 256 bytes apart.
+    // V page block j (16 keys = one K step): canonical no-swizzle K-major with
+    // rows = d: core matrices of 8 d x 8 keys, key-chunks 128 B apart (LBO),
+    // 8-d groups 256 B apart (SBO).
     mma_bf16(tmem_o, smem_desc(p_addr + poff, 16, 1024, 2),
-             smem_desc(v_addr + j * 4096, 16, 256, 6), idesc, (accumulate || j != 0) ? 1u : 0u);
+             smem_desc(v_addr + j * BLOCK_BYTES, 128, 256, 0), idesc, (accumulate || j != 0) ? 1u : 0u);
   }
 }
 
@@ -277,9 +281,7 @@ __device__ __forceinline__ void drain(uint64_t* bar, int fills) {
 // sums over j run j = 0..127 in order; masked keys have P_j = 0 by selection.
 template <bool DECODE>
 __global__ void __launch_bounds__(THREADS, 1)
-    attn_split_kernel(const __grid_constant__ CUtensorMap tmQ,
-                      const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmV, const Params p) {
+    attn_split_kernel(const __grid_constant__ CUtensorMap tmQ, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -331,8 +333,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
       const uint32_t q_bytes = 2u * 64u * 2u * (uint32_t)(p.G * p.q_box);
       TileRows* ring = reinterpret_cast<TileRows*>(smem + OFF_RING);
       Cursor kc, vc, pf;
@@ -341,10 +341,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       pf = kc;
       int nk = 0, nv = 0, npf = 0, qi = 0;
       int q_fills[2] = {0, 0}, k_fills[2] = {0, 0}, v_fills[2] = {0, 0};
-      for (; pf.valid && npf < PF_AHEAD; ++npf, cursor_next(p, pf)) {
+      for (; pf.valid && npf < PF_AHEAD; ++npf, cursor_next(p, pf))
         tile_rows(p, pf.it.b, pf.it.g, pf.it.L, pf.it.t0 + pf.t, ring[npf & (PF_RING - 1)]);
-        prefetch_tile(p, &tmK, &tmV, ring[npf & (PF_RING - 1)]);
-      }
       bool ok = true;
       long long t_last = clock64();
       while ((kc.valid || vc.valid) && ok) {
@@ -373,9 +371,8 @@ __global__ void __launch_bounds__(THREADS, 1)
               ++q_fills[qb];
               ++qi;
             }
-            if (pf.valid) {  // keep the page lookups and L2 prefetches PF_AHEAD tiles ahead
+            if (pf.valid) {  // keep the page lookups PF_AHEAD tiles ahead
               tile_rows(p, pf.it.b, pf.it.g, pf.it.L, pf.it.t0 + pf.t, ring[npf & (PF_RING - 1)]);
-              prefetch_tile(p, &tmK, &tmV, ring[npf & (PF_RING - 1)]);
               ++npf;
               cursor_next(p, pf);
             }
@@ -383,10 +380,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             uint8_t* kbuf = smem + OFF_K + kb * TILE_BYTES;
             mbar_arrive_expect_tx(&k_full[kb], TILE_BYTES);
 #pragma unroll
-            for (int i = 0; i < PAGES_PER_TILE; ++i) {
-              tma_load_2d(kbuf + i * 2048, &tmK, &k_full[kb], 0, r.k[i]);
-              tma_load_2d(kbuf + 16384 + i * 2048, &tmK, &k_full[kb], 64, r.k[i]);
-            }
+            for (int i = 0; i < PAGES_PER_TILE; ++i)
+              bulk_load(kbuf + i * BLOCK_BYTES, block_src(p.kc, r.pid[i], p.Hkv, kc.it.g), BLOCK_BYTES,
+                        &k_full[kb]);
             ++k_fills[kb];
             ++nk;
             cursor_next(p, kc);
@@ -400,7 +396,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             uint8_t* vbuf = smem + OFF_V + vb * TILE_BYTES;
             mbar_arrive_expect_tx(&v_full[vb], TILE_BYTES);
 #pragma unroll
-            for (int i = 0; i < PAGES_PER_TILE; ++i) tma_load_2d(vbuf + i * 4096, &tmV, &v_full[vb], 0, r.v[i]);
+            for (int i = 0; i < PAGES_PER_TILE; ++i)
+              bulk_load(vbuf + i * BLOCK_BYTES, block_src(p.vc, r.pid[i], p.Hkv, vc.it.g), BLOCK_BYTES,
+                        &v_full[vb]);
             ++v_fills[vb];
             ++nv;
             cursor_next(p, vc);
@@ -632,11 +630,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         // zero V slots at or past the sequence end inside this tile's last page
         if (tail != 0 && last_page / PAGES_PER_TILE == it.t0 + t) {
           if (!mbar_wait(&v_full[sb], ((uint32_t)j >> 1) & 1u, p.status, abort_flag)) { ok = false; break; }
-          uint8_t* vblk = smem + OFF_V + sb * TILE_BYTES + (last_page % PAGES_PER_TILE) * 4096;
-          const int d = r;  // V^T row
+          uint8_t* vblk = smem + OFF_V + sb * TILE_BYTES + (last_page % PAGES_PER_TILE) * BLOCK_BYTES;
+          const int d = r;  // value row d of the block
           for (int slot = tail; slot < PAGE; ++slot) {
-            const uint32_t off = (uint32_t)d * 32u + ((uint32_t)((slot >> 3) ^ ((d >> 2) & 1)) << 4) +
-                                 (uint32_t)(slot & 7) * 2u;
+            const uint32_t off = (uint32_t)(d >> 3) * 256u + (uint32_t)(slot >> 3) * 128u +
+                                 (uint32_t)(d & 7) * 16u + (uint32_t)(slot & 7) * 2u;
             *reinterpret_cast<uint16_t*>(vblk + off) = 0;
           }
         }
@@ -773,8 +771,8 @@ static bi_status check_shape(const bi_attn_shape* sh) {
   if (G != 1 && G != 2 && G != 4 && G != 8) return fail(BI_ERR_SHAPE, "attention: q heads per kv head must be 1, 2, 4 or 8 (got %d)", G);
   if (sh->num_pages <= 0 || sh->max_pages_per_seq <= 0 || sh->max_kv_len <= 0)
     return fail(BI_ERR_SHAPE, "attention: num_pages, max_pages_per_seq and max_kv_len must be positive");
-  if ((int64_t)sh->num_pages * sh->num_kv_heads * HD > 0x7fffffffll)
-    return fail(BI_ERR_SHAPE, "attention: cache too large for 32-bit TMA coordinates");
+  if ((int64_t)sh->num_pages * sh->num_kv_heads > 0x7fffffffll / PAGE)
+    return fail(BI_ERR_SHAPE, "attention: cache too large");
   if (!(sh->scale > 0.0f)) return fail(BI_ERR_INVALID_ARG, "attention: scale must be > 0");
   return BI_OK;
 }
@@ -806,7 +804,7 @@ static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t ma
   if (!ws || ws_bytes < need) return fail(BI_ERR_WORKSPACE, "attention: workspace %zu bytes < %zu needed", ws_bytes, need);
   if ((st = require_sm100()) != BI_OK) return st;
 
-  CUtensorMap tmQ, tmK, tmV;
+  CUtensorMap tmQ;
   {
     uint64_t dims[3] = {(uint64_t)HD, (uint64_t)Hq, (uint64_t)n_tok};
     uint64_t strides[2] = {(uint64_t)HD * 2, (uint64_t)ldq * 2};
@@ -815,23 +813,9 @@ static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t ma
                           strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != BI_OK)
       return st;
   }
-  {
-    uint64_t dims[2] = {(uint64_t)HD, (uint64_t)sh->num_pages * sh->num_kv_heads * PAGE};
-    uint64_t strides[1] = {(uint64_t)HD * 2};
-    uint32_t box[2] = {64, (uint32_t)PAGE};
-    if ((st = encode_tmap(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(k_cache),
-                          dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != BI_OK)
-      return st;
-  }
-  {
-    uint64_t dims[2] = {(uint64_t)PAGE, (uint64_t)sh->num_pages * sh->num_kv_heads * HD};
-    uint64_t strides[1] = {(uint64_t)PAGE * 2};
-    uint32_t box[2] = {(uint32_t)PAGE, (uint32_t)HD};
-    if ((st = encode_tmap(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(v_cache),
-                          dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B)) != BI_OK)
-      return st;
-  }
   Params p;
+  p.kc = static_cast<const uint8_t*>(k_cache);
+  p.vc = static_cast<const uint8_t*>(v_cache);
   p.block_table = block_table;
   p.seq_lens = seq_lens;
   p.cu_q = cu_q;
@@ -868,9 +852,9 @@ static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t ma
   const int sms = num_sms();
   const int grid = (int)(total_items < sms ? total_items : sms);
   if (cu_q)
-    attn_split_kernel<false><<<grid, THREADS, SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
+    attn_split_kernel<false><<<grid, THREADS, SMEM_BYTES, stream>>>(tmQ, p);
   else
-    attn_split_kernel<true><<<grid, THREADS, SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
+    attn_split_kernel<true><<<grid, THREADS, SMEM_BYTES, stream>>>(tmQ, p);
   BI_CHECK_LAUNCH("attention split launch");
 
   CombineParams c;

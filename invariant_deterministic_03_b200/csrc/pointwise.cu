@@ -17,8 +17,12 @@
 namespace bi {
 namespace pw {
 
-// ---- KV append: one warp per (token, kv head). k row -> k_cache[page][g][slot][:],
-// v row -> v_cache[page][g][:][slot] (transposed page block).
+// ---- KV append: one warp per (token, kv head). Each (page, kv head) block
+// of 16 keys x 128 d is stored in the tensor core's canonical no-swizzle
+// K-major order, so attention copies it into shared memory as one piece:
+//   keys:   element (slot o, d) at (o/8)*1024 + (d/8)*64 + (o%8)*8 + d%8
+//   values: element (d, slot o) at (d/8)*128 + (o/8)*64 + (d%8)*8 + o%8
+// (element offsets inside the block; 8 x 8 core matrices of 128 bytes).
 __global__ void kv_append_kernel(const bf16* __restrict__ k_new, const bf16* __restrict__ v_new,
                                  int64_t ld_new, const int32_t* __restrict__ slots, int64_t n_tok,
                                  int Hkv, int num_pages, bf16* __restrict__ kc,
@@ -34,21 +38,18 @@ __global__ void kv_append_kernel(const bf16* __restrict__ k_new, const bf16* __r
     if (lane == 0) set_status(status, BI_DEV_BAD_SLOT);
     return;
   }
-  const int page = slot / BI_PAGE_SIZE, off = slot % BI_PAGE_SIZE;
+  const int page = slot / BI_PAGE_SIZE, o = slot % BI_PAGE_SIZE;
   const bf16* ksrc = k_new + t * ld_new + (int64_t)g * BI_HEAD_DIM;
   const bf16* vsrc = v_new + t * ld_new + (int64_t)g * BI_HEAD_DIM;
-  const size_t blk = (size_t)page * Hkv + g;
-  // keys: 128 elements = 16 lanes x 16 bytes
-  if (lane < 16) {
-    const uint4 v = reinterpret_cast<const uint4*>(ksrc)[lane];
-    reinterpret_cast<uint4*>(kc + (blk * BI_PAGE_SIZE + off) * BI_HEAD_DIM)[lane] = v;
-  }
-  // values, transposed: element d goes to row d, column `off` of the page block
-  bf16* vdst = vc + blk * BI_HEAD_DIM * BI_PAGE_SIZE + off;
+  const size_t blk = ((size_t)page * Hkv + g) * (BI_PAGE_SIZE * BI_HEAD_DIM);
+  const int d0 = lane * 4;  // this lane's 4 consecutive d values (one core-matrix row half)
+  const uint2 kv = reinterpret_cast<const uint2*>(ksrc)[lane];
+  *reinterpret_cast<uint2*>(kc + blk + (o >> 3) * 1024 + (d0 >> 3) * 64 + (o & 7) * 8 + (d0 & 7)) = kv;
+  bf16* vdst = vc + blk + (o >> 3) * 64 + (o & 7);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int d = lane * 4 + i;
-    vdst[(size_t)d * BI_PAGE_SIZE] = vsrc[d];
+    const int d = d0 + i;
+    vdst[(d >> 3) * 128 + (d & 7) * 8] = vsrc[d];
   }
 }
 

@@ -168,16 +168,29 @@ def test_config3_decode(bi):
     assert same_bits(out2, out)
 
 
+def _logical_k(kc):
+    """[P, Hkv, 16, 128] in the blocked core-matrix order -> (slot, d)."""
+    P, H = kc.shape[:2]
+    return kc.reshape(P, H, 2, 16, 8, 8).permute(0, 1, 2, 4, 3, 5).reshape(P, H, 16, 128)
+
+
+def _logical_v(vc):
+    """[P, Hkv, 128, 16] in the blocked core-matrix order -> (d, slot)."""
+    P, H = vc.shape[:2]
+    return vc.reshape(P, H, 16, 2, 8, 8).permute(0, 1, 2, 4, 3, 5).reshape(P, H, 128, 16)
+
+
 def test_kv_append_exact(bi):
     """The cache holds the exact input bytes at the slot's page and offset
-    (keys row-major, values transposed per page); padding slots are skipped."""
+    (blocked core-matrix order, see include/bi.h); padding slots are skipped."""
     lens = [40, 3]
     S = Seqs(bi, lens, 32, 8, seed=5)
+    K, V = _logical_k(S.kc), _logical_v(S.vc)
     for b, L in enumerate(lens):
         slots = S.layout.slots(b, 0, L).long()
         page, off = slots // 16, slots % 16
-        k_got = S.kc[page.cuda(), :, off.cuda(), :]          # [L, Hkv, 128]
-        v_got = S.vc[page.cuda(), :, :, off.cuda()]          # [L, Hkv, 128]
+        k_got = K[page.cuda(), :, off.cuda(), :]          # [L, Hkv, 128]
+        v_got = V[page.cuda(), :, :, off.cuda()]          # [L, Hkv, 128]
         assert same_bits(k_got.cpu(), S.k[b])
         assert same_bits(v_got.cpu(), S.v[b])
     before_k, before_v = S.kc.clone(), S.vc.clone()
