@@ -49,7 +49,7 @@ constexpr uint32_t OFF_K = 2 * TILE_BYTES;      // 2 buffers
 constexpr uint32_t OFF_V = 4 * TILE_BYTES;      // 2 buffers
 constexpr uint32_t OFF_P = 6 * TILE_BYTES;
 constexpr uint32_t OFF_BAR = 7 * TILE_BYTES;
-constexpr uint32_t OFF_RING = OFF_BAR + 256;   // producer's page-id ring (16 x 32 B)
+constexpr uint32_t OFF_RING = OFF_BAR + 256;   // producer's page-id ring [16 tiles][8 pages]
 constexpr uint32_t OFF_RED = OFF_RING + 512;   // decode quarter exchange [2][4 warps][8 heads] fp32
 constexpr size_t SMEM_BYTES = 1024 + 7 * TILE_BYTES + 256 + 512 + 256;
 static_assert(SMEM_BYTES <= 232448, "attention: shared memory above the 227 KB per-CTA limit");
@@ -120,28 +120,16 @@ __device__ __align__(128) uint8_t g_attn_zero_block[4096];
 
 constexpr uint32_t BLOCK_BYTES = PAGE * HD * 2;  // 4 KB: one (page, kv head) block
 
-// Page ids of the 8 pages of one 128-key tile (looked up in the sequence's
-// block table); -1 marks a page past the sequence end or a bad id.
-struct TileRows {
-  int32_t pid[PAGES_PER_TILE];
-};
-
-__device__ __forceinline__ void tile_rows(const Params& p, int b, int g, int L, int tile,
-                                          TileRows& r) {
-  const int32_t* bt = p.block_table + (size_t)b * p.max_pages;
-  // all eight entries loaded unconditionally (clamped index, always inside the
-  // row) so the loads go out together; validity is applied afterwards
-  int32_t pid[PAGES_PER_TILE];
-#pragma unroll
-  for (int i = 0; i < PAGES_PER_TILE; ++i) pid[i] = bt[min(tile * PAGES_PER_TILE + i, p.max_pages - 1)];
-#pragma unroll
-  for (int i = 0; i < PAGES_PER_TILE; ++i) {
-    const int pidx = tile * PAGES_PER_TILE + i;
-    const bool in_seq = pidx * PAGE < L;
-    const bool ok = in_seq && pidx < p.max_pages && pid[i] >= 0 && pid[i] < p.num_pages;
-    r.pid[i] = ok ? pid[i] : -1;
-    if (in_seq && !ok) set_status(p.status, BI_DEV_BAD_PAGE);
-  }
+// Page id of page i (0..7) of one 128-key tile, looked up in the sequence's
+// block table; -1 marks a page past the sequence end or a bad id (the entry
+// is read unconditionally at a clamped index, always inside the row).
+__device__ __forceinline__ int32_t tile_page(const Params& p, int b, int L, int tile, int i) {
+  const int pidx = tile * PAGES_PER_TILE + i;
+  const int32_t pid = p.block_table[(size_t)b * p.max_pages + min(pidx, p.max_pages - 1)];
+  const bool in_seq = pidx * PAGE < L;
+  const bool ok = in_seq && pidx < p.max_pages && pid >= 0 && pid < p.num_pages;
+  if (in_seq && !ok) set_status(p.status, BI_DEV_BAD_PAGE);
+  return ok ? pid : -1;
 }
 
 __device__ __forceinline__ const uint8_t* block_src(const uint8_t* cache, int32_t pid, int Hkv,
@@ -176,6 +164,7 @@ __device__ __forceinline__ void cursor_start(const Params& p, Cursor& c) {
 
 constexpr int PF_AHEAD = 4;   // page-table lookups run this many tiles ahead of the K loads
 constexpr int PF_RING = 16;   // looked-up page ids, from the oldest V load to the newest lookup
+static_assert(PF_RING * 8 * 4 <= 512, "page-id ring overflows its region");
 
 // S = Q K^T. Q: 128 rows x 128 d, 128-byte swizzle in two 64-column halves.
 // K: 8 page blocks of 16 keys, canonical no-swizzle K-major: core matrices of
@@ -330,29 +319,36 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 4) {
-    // ------------------------------------------------ TMA producer
-    if (lane == 0) {
-      prefetch_tmap(&tmQ);
-      const uint32_t q_bytes = 2u * 64u * 2u * (uint32_t)(p.G * p.q_box);
-      TileRows* ring = reinterpret_cast<TileRows*>(smem + OFF_RING);
-      Cursor kc, vc, pf;
-      cursor_start(p, kc);
-      vc = kc;
-      pf = kc;
-      int nk = 0, nv = 0, npf = 0, qi = 0;
-      int q_fills[2] = {0, 0}, k_fills[2] = {0, 0}, v_fills[2] = {0, 0};
-      for (; pf.valid && npf < PF_AHEAD; ++npf, cursor_next(p, pf))
-        tile_rows(p, pf.it.b, pf.it.g, pf.it.L, pf.it.t0 + pf.t, ring[npf & (PF_RING - 1)]);
-      bool ok = true;
-      long long t_last = clock64();
-      while ((kc.valid || vc.valid) && ok) {
-        bool progressed = false;
-        if (kc.valid) {
-          const int kb = nk & 1, qb = qi & 1;
-          bool ready = mbar_test(&k_empty[kb], (((uint32_t)nk >> 1) & 1u) ^ 1u);
+    // ------------------------------------------------ producer warp
+    // Lane 0 owns the barriers and the Q loads; lanes 0..7 each look up one
+    // page of a tile and issue that page's 4 KB copy, so a tile's eight
+    // copies go out together. All lanes walk the same cursors.
+    if (lane == 0) prefetch_tmap(&tmQ);
+    const uint32_t q_bytes = 2u * 64u * 2u * (uint32_t)(p.G * p.q_box);
+    int32_t* ring = reinterpret_cast<int32_t*>(smem + OFF_RING);  // [PF_RING][8]
+    Cursor kc, vc, pf;
+    cursor_start(p, kc);
+    vc = kc;
+    pf = kc;
+    int nk = 0, nv = 0, npf = 0, qi = 0;
+    int q_fills[2] = {0, 0}, k_fills[2] = {0, 0}, v_fills[2] = {0, 0};
+    for (; pf.valid && npf < PF_AHEAD; ++npf, cursor_next(p, pf))
+      if (lane < PAGES_PER_TILE)
+        ring[(npf & (PF_RING - 1)) * 8 + lane] = tile_page(p, pf.it.b, pf.it.L, pf.it.t0 + pf.t, lane);
+    bool ok = true;
+    long long t_last = clock64();
+    while ((kc.valid || vc.valid) && ok) {
+      bool progressed = false;
+      if (kc.valid) {
+        const int kb = nk & 1, qb = qi & 1;
+        int ready = 0;
+        if (lane == 0) {
+          ready = mbar_test(&k_empty[kb], (((uint32_t)nk >> 1) & 1u) ^ 1u);
           if (ready && kc.t == 0) ready = mbar_test(&q_empty[qb], (((uint32_t)qi >> 1) & 1u) ^ 1u);
-          if (ready) {
-            if (kc.t == 0) {  // first tile of an item: its Q rows
+        }
+        if (__shfl_sync(0xffffffffu, ready, 0)) {
+          if (kc.t == 0) {  // first tile of an item: its Q rows
+            if (lane == 0) {
               uint8_t* qdst = smem + OFF_Q + qb * TILE_BYTES;
               if (!DECODE) {
                 mbar_arrive_expect_tx(&q_full[qb], q_bytes);
@@ -368,59 +364,64 @@ __global__ void __launch_bounds__(THREADS, 1)
                               kc.it.r0 + kc.it.q_lo);
                 }
               }
-              ++q_fills[qb];
-              ++qi;
             }
-            if (pf.valid) {  // keep the page lookups PF_AHEAD tiles ahead
-              tile_rows(p, pf.it.b, pf.it.g, pf.it.L, pf.it.t0 + pf.t, ring[npf & (PF_RING - 1)]);
-              ++npf;
-              cursor_next(p, pf);
-            }
-            const TileRows& r = ring[nk & (PF_RING - 1)];
-            uint8_t* kbuf = smem + OFF_K + kb * TILE_BYTES;
-            mbar_arrive_expect_tx(&k_full[kb], TILE_BYTES);
-#pragma unroll
-            for (int i = 0; i < PAGES_PER_TILE; ++i)
-              bulk_load(kbuf + i * BLOCK_BYTES, block_src(p.kc, r.pid[i], p.Hkv, kc.it.g), BLOCK_BYTES,
-                        &k_full[kb]);
-            ++k_fills[kb];
-            ++nk;
-            cursor_next(p, kc);
-            progressed = true;
+            ++q_fills[qb];
+            ++qi;
           }
-        }
-        if (vc.valid && nv < nk) {
-          const int vb = nv & 1;
-          if (mbar_test(&v_empty[vb], (((uint32_t)nv >> 1) & 1u) ^ 1u)) {
-            const TileRows& r = ring[nv & (PF_RING - 1)];
-            uint8_t* vbuf = smem + OFF_V + vb * TILE_BYTES;
-            mbar_arrive_expect_tx(&v_full[vb], TILE_BYTES);
-#pragma unroll
-            for (int i = 0; i < PAGES_PER_TILE; ++i)
-              bulk_load(vbuf + i * BLOCK_BYTES, block_src(p.vc, r.pid[i], p.Hkv, vc.it.g), BLOCK_BYTES,
-                        &v_full[vb]);
-            ++v_fills[vb];
-            ++nv;
-            cursor_next(p, vc);
-            progressed = true;
+          if (pf.valid) {  // keep the page lookups PF_AHEAD tiles ahead
+            if (lane < PAGES_PER_TILE)
+              ring[(npf & (PF_RING - 1)) * 8 + lane] = tile_page(p, pf.it.b, pf.it.L, pf.it.t0 + pf.t, lane);
+            ++npf;
+            cursor_next(p, pf);
           }
+          if (lane == 0) mbar_arrive_expect_tx(&k_full[kb], TILE_BYTES);
+          __syncwarp();
+          if (lane < PAGES_PER_TILE)
+            bulk_load(smem + OFF_K + kb * TILE_BYTES + lane * BLOCK_BYTES,
+                      block_src(p.kc, ring[(nk & (PF_RING - 1)) * 8 + lane], p.Hkv, kc.it.g), BLOCK_BYTES,
+                      &k_full[kb]);
+          ++k_fills[kb];
+          ++nk;
+          cursor_next(p, kc);
+          progressed = true;
         }
+      }
+      if (vc.valid && nv < nk) {
+        const int vb = nv & 1;
+        int ready = 0;
+        if (lane == 0) ready = mbar_test(&v_empty[vb], (((uint32_t)nv >> 1) & 1u) ^ 1u);
+        if (__shfl_sync(0xffffffffu, ready, 0)) {
+          if (lane == 0) mbar_arrive_expect_tx(&v_full[vb], TILE_BYTES);
+          __syncwarp();
+          if (lane < PAGES_PER_TILE)
+            bulk_load(smem + OFF_V + vb * TILE_BYTES + lane * BLOCK_BYTES,
+                      block_src(p.vc, ring[(nv & (PF_RING - 1)) * 8 + lane], p.Hkv, vc.it.g), BLOCK_BYTES,
+                      &v_full[vb]);
+          ++v_fills[vb];
+          ++nv;
+          cursor_next(p, vc);
+          progressed = true;
+        }
+      }
+      int stop = 0;
+      if (lane == 0) {
         if (progressed) {
           t_last = clock64();
         } else if (__nanosleep(32), *abort_flag) {
-          ok = false;
+          stop = 1;
         } else if (clock64() - t_last > kWaitLimitCycles) {
           set_status(p.status, BI_DEV_WAIT_TIMEOUT);
           *abort_flag = 1;
-          ok = false;
+          stop = 1;
         }
       }
-      if (!ok) {
-        for (int i = 0; i < 2; ++i) {
-          drain(&q_full[i], q_fills[i]);
-          drain(&k_full[i], k_fills[i]);
-          drain(&v_full[i], v_fills[i]);
-        }
+      if (__shfl_sync(0xffffffffu, stop, 0)) ok = false;
+    }
+    if (!ok && lane == 0) {
+      for (int i = 0; i < 2; ++i) {
+        drain(&q_full[i], q_fills[i]);
+        drain(&k_full[i], k_fills[i]);
+        drain(&v_full[i], v_fills[i]);
       }
     }
   } else if (warp == 5) {
