@@ -121,11 +121,15 @@ __device__ __align__(128) uint8_t g_attn_zero_block[4096];
 constexpr uint32_t BLOCK_BYTES = PAGE * HD * 2;  // 4 KB: one (page, kv head) block
 
 // Page id of page i (0..7) of one 128-key tile, looked up in the sequence's
-// block table; -1 marks a page past the sequence end or a bad id (the entry
-// is read unconditionally at a clamped index, always inside the row).
-__device__ __forceinline__ int32_t tile_page(const Params& p, int b, int L, int tile, int i) {
+// block table; -1 marks a page past the sequence end or a bad id. The entry
+// is read unconditionally at a clamped index (always inside the row), so the
+// load can be issued early and validated later (page_valid).
+__device__ __forceinline__ int32_t tile_page_raw(const Params& p, int b, int tile, int i) {
+  return p.block_table[(size_t)b * p.max_pages + min(tile * PAGES_PER_TILE + i, p.max_pages - 1)];
+}
+
+__device__ __forceinline__ int32_t page_valid(const Params& p, int L, int tile, int i, int32_t pid) {
   const int pidx = tile * PAGES_PER_TILE + i;
-  const int32_t pid = p.block_table[(size_t)b * p.max_pages + min(pidx, p.max_pages - 1)];
   const bool in_seq = pidx * PAGE < L;
   const bool ok = in_seq && pidx < p.max_pages && pid >= 0 && pid < p.num_pages;
   if (in_seq && !ok) set_status(p.status, BI_DEV_BAD_PAGE);
@@ -334,7 +338,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     int q_fills[2] = {0, 0}, k_fills[2] = {0, 0}, v_fills[2] = {0, 0};
     for (; pf.valid && npf < PF_AHEAD; ++npf, cursor_next(p, pf))
       if (lane < PAGES_PER_TILE)
-        ring[(npf & (PF_RING - 1)) * 8 + lane] = tile_page(p, pf.it.b, pf.it.L, pf.it.t0 + pf.t, lane);
+        ring[(npf & (PF_RING - 1)) * 8 + lane] =
+            page_valid(p, pf.it.L, pf.it.t0 + pf.t, lane, tile_page_raw(p, pf.it.b, pf.it.t0 + pf.t, lane));
+    // one lookup in flight: its load is issued now and its result is checked
+    // and stored one K issue later, off the issue path
+    bool la_pending = false;
+    int32_t la_pid = -1;
+    int la_slot = 0, la_L = 0, la_tile = 0;
     bool ok = true;
     long long t_last = clock64();
     while ((kc.valid || vc.valid) && ok) {
@@ -368,9 +378,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             ++q_fills[qb];
             ++qi;
           }
+          if (la_pending) {
+            if (lane < PAGES_PER_TILE) ring[la_slot * 8 + lane] = page_valid(p, la_L, la_tile, lane, la_pid);
+            la_pending = false;
+          }
           if (pf.valid) {  // keep the page lookups PF_AHEAD tiles ahead
-            if (lane < PAGES_PER_TILE)
-              ring[(npf & (PF_RING - 1)) * 8 + lane] = tile_page(p, pf.it.b, pf.it.L, pf.it.t0 + pf.t, lane);
+            la_tile = pf.it.t0 + pf.t;
+            la_L = pf.it.L;
+            la_slot = npf & (PF_RING - 1);
+            la_pid = lane < PAGES_PER_TILE ? tile_page_raw(p, pf.it.b, la_tile, lane) : -1;
+            la_pending = true;
             ++npf;
             cursor_next(p, pf);
           }
