@@ -184,7 +184,10 @@ typedef struct {
 
 /* Workspace bytes for up to `max_tokens` query tokens with keys up to
  * shape->max_kv_len: per (token, q head, split) 128 fp32 partial outputs plus
- * (m, l). */
+ * (m, l), rounded up to 256 bytes, then 256 bytes holding the split kernel's
+ * work-item counter (reset by the call itself, on its stream, before the
+ * launch; it only decides which SM takes which (split, head group) item, never
+ * the order of any sum). One workspace serves one call in flight at a time. */
 bi_status bi_attn_workspace_size(const bi_attn_shape* shape, int64_t max_tokens,
                                  size_t* bytes);
 
@@ -206,8 +209,9 @@ bi_status bi_attn_decode(const void* q, int64_t ldq, const void* k_cache,
  * The scratch is a fixed array of BI_ATTN_NOALLOC_SCRATCH_BYTES (16 MiB) that
  * is part of the library's device image: every GPU that loads libbi holds it
  * until the process exits. A call needs
- * B * num_q_heads * ceil(max_kv_len / 512) * 520 bytes of it (e.g. 32
- * sequences x 32 heads x 8192 keys = 8.5 MiB); larger calls fail with
+ * B * num_q_heads * ceil(max_kv_len / 512) * 520 bytes of it, rounded up
+ * to 256, plus 256 (e.g. 32 sequences x 32 heads x 8192 keys = 8.5 MiB);
+ * larger calls fail with
  * BI_ERR_WORKSPACE and launch nothing. Nothing is allocated: no cudaMalloc,
  * no cudaFree, no allocating library routine.
  *

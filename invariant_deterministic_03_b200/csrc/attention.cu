@@ -51,7 +51,9 @@ constexpr uint32_t OFF_P = 6 * TILE_BYTES;
 constexpr uint32_t OFF_BAR = 7 * TILE_BYTES;
 constexpr uint32_t OFF_RING = OFF_BAR + 256;   // producer's page-id ring [16 tiles][8 pages]
 constexpr uint32_t OFF_RED = OFF_RING + 512;   // decode quarter exchange [2][4 warps][8 heads] fp32
-constexpr size_t SMEM_BYTES = 1024 + 7 * TILE_BYTES + 256 + 512 + 256;
+constexpr int ITEM_RING = 32;                  // claimed work items in flight inside a CTA
+constexpr uint32_t OFF_ITEMS = OFF_RED + 256;  // item ring [32] int32, then one mbarrier per slot
+constexpr size_t SMEM_BYTES = 1024 + 7 * TILE_BYTES + 256 + 512 + 256 + ITEM_RING * 4 + ITEM_RING * 8;
 static_assert(SMEM_BYTES <= 232448, "attention: shared memory above the 227 KB per-CTA limit");
 // warps 0-3: one thread per MMA row (softmax, O rescale, partials)
 // warp 4: TMA producer; warp 5: TMEM allocator and MMA issuer
@@ -71,6 +73,7 @@ struct Params {
   int32_t B, Hq, Hkv, G, QR, qblocks, q_box, n_tok;
   int32_t num_pages, max_pages, max_kv_len, n_split_max;
   int32_t total_items;
+  int32_t* work_counter;  // next unclaimed work item (zeroed before the launch)
   float scale_log2;
   int32_t* status;
 };
@@ -141,29 +144,69 @@ __device__ __forceinline__ const uint8_t* block_src(const uint8_t* cache, int32_
   return pid < 0 ? g_attn_zero_block : cache + ((size_t)pid * Hkv + g) * BLOCK_BYTES;
 }
 
-// Walks the (item, tile) sequence of one CTA.
+// Work items are claimed at run time: the producer's look-ahead cursor takes
+// the next index from a global counter (atomicAdd -- scheduling only, no
+// value is ever reduced through it), skips items with no work, and publishes
+// each claimed item (or -1 at the end) in a shared ring with one mbarrier per
+// slot; every other role walks the ring in order. Which CTA runs an item
+// never reaches its arithmetic. The look-ahead is bounded by the K/V buffers
+// (a dozen items at most), far inside the 32-slot ring.
+__device__ __forceinline__ int claim_item(const Params& p, int lane, Item& it) {
+  while (true) {
+    int v = 0;
+    if (lane == 0) v = atomicAdd(p.work_counter, 1);
+    v = __shfl_sync(0xffffffffu, v, 0);
+    if (v >= p.total_items) return -1;
+    if (item_at(p, v, it, true)) return v;
+  }
+}
+
+// Walks the (item, tile) sequence of this CTA through the item ring.
 struct Cursor {
-  int idx, t;
+  int n, t;  // ring sequence number of the current item, tile within it
   Item it;
   bool valid;
 };
 
-__device__ __forceinline__ void cursor_next(const Params& p, Cursor& c) {
-  if (c.valid && ++c.t < c.it.ntiles) return;
+// Advances to the next tile; on a new item, reads ring entry n (waiting for
+// its publication). Returns false only when a wait timed out.
+__device__ __forceinline__ bool cursor_next(const Params& p, Cursor& c, const int32_t* ring,
+                                            uint64_t* ibar, volatile int* abort_flag) {
+  if (c.valid && ++c.t < c.it.ntiles) return true;
   c.valid = false;
   c.t = 0;
-  for (c.idx += gridDim.x; c.idx < p.total_items; c.idx += gridDim.x)
-    if (item_at(p, c.idx, c.it, false)) {
-      c.valid = true;
-      return;
-    }
+  ++c.n;
+  const int slot = c.n & (ITEM_RING - 1);
+  if (!mbar_wait(&ibar[slot], ((uint32_t)c.n / ITEM_RING) & 1u, p.status, abort_flag)) return false;
+  const int idx = reinterpret_cast<const volatile int32_t*>(ring)[slot];
+  if (idx >= 0) {
+    item_at(p, idx, c.it, false);
+    c.valid = true;
+  }
+  return true;
 }
 
-__device__ __forceinline__ void cursor_start(const Params& p, Cursor& c) {
-  c.idx = (int)blockIdx.x - (int)gridDim.x;
+__device__ __forceinline__ bool cursor_start(const Params& p, Cursor& c, const int32_t* ring,
+                                             uint64_t* ibar, volatile int* abort_flag) {
+  c.n = -1;
   c.t = 0;
   c.valid = false;
-  cursor_next(p, c);
+  return cursor_next(p, c, ring, ibar, abort_flag);
+}
+
+// The producer's look-ahead cursor: claims and publishes items.
+__device__ __forceinline__ void claim_next(const Params& p, Cursor& c, int32_t* ring, uint64_t* ibar,
+                                           int lane) {
+  if (c.valid && ++c.t < c.it.ntiles) return;
+  c.t = 0;
+  ++c.n;
+  const int idx = claim_item(p, lane, c.it);
+  c.valid = idx >= 0;
+  if (lane == 0) {
+    const int slot = c.n & (ITEM_RING - 1);
+    reinterpret_cast<volatile int32_t*>(ring)[slot] = idx;
+    mbar_arrive(&ibar[slot]);
+  }
 }
 
 constexpr int PF_AHEAD = 4;   // page-table lookups run this many tiles ahead of the K loads
@@ -291,6 +334,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* o_ready = bars + 17;
   uint64_t* x_bar = bars + 18;     // decode: quarter exchange among the 4 softmax warps
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+  int32_t* item_ring = reinterpret_cast<int32_t*>(smem + OFF_ITEMS);
+  uint64_t* item_bar = reinterpret_cast<uint64_t*>(smem + OFF_ITEMS + ITEM_RING * 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -310,6 +355,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(p_ready, 128);
     mbar_init(o_ready, 1);
     mbar_init(x_bar, 128);
+    for (int i = 0; i < ITEM_RING; ++i) mbar_init(&item_bar[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -331,12 +377,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t q_bytes = 2u * 64u * 2u * (uint32_t)(p.G * p.q_box);
     int32_t* ring = reinterpret_cast<int32_t*>(smem + OFF_RING);  // [PF_RING][8]
     Cursor kc, vc, pf;
-    cursor_start(p, kc);
+    pf.n = -1;
+    pf.t = 0;
+    pf.valid = false;
+    claim_next(p, pf, item_ring, item_bar, lane);  // publishes ring entry 0
+    bool ok = cursor_start(p, kc, item_ring, item_bar, abort_flag);
     vc = kc;
-    pf = kc;
     int nk = 0, nv = 0, npf = 0, qi = 0;
     int q_fills[2] = {0, 0}, k_fills[2] = {0, 0}, v_fills[2] = {0, 0};
-    for (; pf.valid && npf < PF_AHEAD; ++npf, cursor_next(p, pf))
+    for (; pf.valid && npf < PF_AHEAD; ++npf, claim_next(p, pf, item_ring, item_bar, lane))
       if (lane < PAGES_PER_TILE)
         ring[(npf & (PF_RING - 1)) * 8 + lane] =
             page_valid(p, pf.it.L, pf.it.t0 + pf.t, lane, tile_page_raw(p, pf.it.b, pf.it.t0 + pf.t, lane));
@@ -345,7 +394,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     bool la_pending = false;
     int32_t la_pid = -1;
     int la_slot = 0, la_L = 0, la_tile = 0;
-    bool ok = true;
     long long t_last = clock64();
     while ((kc.valid || vc.valid) && ok) {
       bool progressed = false;
@@ -389,7 +437,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             la_pid = lane < PAGES_PER_TILE ? tile_page_raw(p, pf.it.b, la_tile, lane) : -1;
             la_pending = true;
             ++npf;
-            cursor_next(p, pf);
+            claim_next(p, pf, item_ring, item_bar, lane);
           }
           if (lane == 0) mbar_arrive_expect_tx(&k_full[kb], TILE_BYTES);
           __syncwarp();
@@ -399,7 +447,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                       &k_full[kb]);
           ++k_fills[kb];
           ++nk;
-          cursor_next(p, kc);
+          if (!cursor_next(p, kc, item_ring, item_bar, abort_flag)) ok = false;
           progressed = true;
         }
       }
@@ -416,7 +464,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                       &v_full[vb]);
           ++v_fills[vb];
           ++nv;
-          cursor_next(p, vc);
+          if (!cursor_next(p, vc, item_ring, item_bar, abort_flag)) ok = false;
           progressed = true;
         }
       }
@@ -434,6 +482,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (__shfl_sync(0xffffffffu, stop, 0)) ok = false;
     }
+    // publish the rest of the claims up to the end marker: consumers may still
+    // be waiting for ring entries the look-ahead has not reached
+    while (ok && pf.valid) claim_next(p, pf, item_ring, item_bar, lane);
     if (!ok && lane == 0) {
       for (int i = 0; i < 2; ++i) {
         drain(&q_full[i], q_fills[i]);
@@ -447,11 +498,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t sQ0 = smem_u32(smem + OFF_Q), sK0 = smem_u32(smem + OFF_K);
       const uint32_t sV0 = smem_u32(smem + OFF_V), sP = smem_u32(smem + OFF_P);
       Cursor sc;
-      cursor_start(p, sc);
       int nS = 0, nP = 0, qi = 0;
       // per issued S tile (bit n & 31): P V accumulates, item's last tile, Q buffer
       uint32_t acc_bits = 0, last_bits = 0, qb_bits = 0;
-      bool ok = true;
+      bool ok = cursor_start(p, sc, item_ring, item_bar, abort_flag);
       long long t_last = clock64();
       while ((sc.valid || nP < nS) && ok) {
         bool progressed = false;
@@ -471,7 +521,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             qb_bits = qb ? (qb_bits | bit) : (qb_bits & ~bit);
             if (sc.t == sc.it.ntiles - 1) ++qi;
             ++nS;
-            cursor_next(p, sc);
+            if (!cursor_next(p, sc, item_ring, item_bar, abort_flag)) ok = false;
             progressed = true;
           }
         }
@@ -523,9 +573,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       ++xc;
       return done;
     };
-    for (int idx = blockIdx.x; idx < p.total_items && ok; idx += gridDim.x) {
+    for (int n = 0; ok; ++n) {
+      const int slot = n & (ITEM_RING - 1);
+      if (!mbar_wait(&item_bar[slot], ((uint32_t)n / ITEM_RING) & 1u, p.status, abort_flag)) break;
+      const int idx = reinterpret_cast<const volatile int32_t*>(item_ring)[slot];
+      if (idx < 0) break;
       Item it;
-      if (!item_at(p, idx, it, false)) continue;
+      item_at(p, idx, it, false);
       const int q_idx = it.q_lo + qr;
       const int pos = it.L - it.nb + q_idx;
       const bool row_valid = (decode ? lane < p.G : true) && (q_idx < it.q_hi) && (pos >= it.key_lo);
@@ -773,10 +827,16 @@ __global__ void attn_combine_kernel(const CombineParams p) {
   *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(y0, y1), pack_bf16x2(y2, y3));
 }
 
-static size_t ws_bytes_for(int64_t n_tok, int Hq, int n_split) {
+// partial O [n_tok][Hq][n_split][128] fp32, then (m, l) pairs, then (256-byte
+// aligned) the work-item counter of the split kernel
+static size_t ws_counter_offset(int64_t n_tok, int Hq, int n_split) {
   const size_t o = (size_t)n_tok * Hq * n_split * HD * sizeof(float);
   const size_t ml = (size_t)n_tok * Hq * n_split * 2 * sizeof(float);
-  return o + ml;
+  return (o + ml + 255) & ~(size_t)255;
+}
+
+static size_t ws_bytes_for(int64_t n_tok, int Hq, int n_split) {
+  return ws_counter_offset(n_tok, Hq, n_split) + 256;
 }
 
 static bi_status check_shape(const bi_attn_shape* sh) {
@@ -852,6 +912,7 @@ static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t ma
   p.max_kv_len = sh->max_kv_len;
   p.n_split_max = n_split;
   p.total_items = (int32_t)total_items;
+  p.work_counter = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + ws_counter_offset(n_tok, Hq, n_split));
   p.scale_log2 = (float)((double)sh->scale * 1.4426950408889634);  // scale * log2(e)
   p.status = status_word();
 
@@ -869,6 +930,8 @@ static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t ma
   }
   const int sms = num_sms();
   const int grid = (int)(total_items < sms ? total_items : sms);
+  cudaError_t me = cudaMemsetAsync(p.work_counter, 0, sizeof(int32_t), stream);
+  if (me != cudaSuccess) return cuda_fail(me, "attention: work counter reset");
   if (cu_q)
     attn_split_kernel<false><<<grid, THREADS, SMEM_BYTES, stream>>>(tmQ, p);
   else

@@ -72,11 +72,12 @@ def test_attention_host_checks(bi):
     sh = bi.attn_shape(32, 8, 100, 10, 160)
     n = ctypes.c_size_t(0)
     assert bi.lib.bi_attn_workspace_size(ctypes.byref(sh), 7, ctypes.byref(n)) == bi.BI_OK
-    # 7 tokens x 32 heads x ceil(160/512)=1 split x (128 + 2) floats
-    assert n.value == 7 * 32 * 1 * 130 * 4
+    # 7 tokens x 32 heads x ceil(160/512)=1 split x (128 + 2) floats, rounded
+    # up to 256 bytes, then the 256-byte work counter
+    assert n.value == 7 * 32 * 1 * 130 * 4 + 256
     sh_big = bi.attn_shape(32, 8, 100, 10, 8192)
     assert bi.lib.bi_attn_workspace_size(ctypes.byref(sh_big), 32, ctypes.byref(n)) == bi.BI_OK
-    assert n.value == 32 * 32 * 16 * 130 * 4
+    assert n.value == 32 * 32 * 16 * 130 * 4 + 256
     bad = bi.attn_shape(32, 6, 100, 10, 160)   # 32 % 6 != 0
     assert bi.lib.bi_attn_workspace_size(ctypes.byref(bad), 1, ctypes.byref(n)) == bi.BI_ERR_SHAPE
     g3 = bi.attn_shape(48, 16, 100, 10, 160)   # 3 q heads per kv head unsupported
