@@ -12,11 +12,19 @@
 //   .kind::f16 M=128 N=256 K=16 with bf16 operands and an fp32 accumulator in
 //   tensor memory. Element (m, n) is accumulated by the K-steps k = 0, 16, 32,
 //   ... in that order, in one CTA, whatever M and N are. Which CTA computes a
-//   tile (persistent round-robin) changes timing only, never arithmetic.
+//   tile (persistent round-robin), how many rows an A copy carries and what
+//   is prefetched into L2 change timing only, never arithmetic.
 //
 // CTA layout (192 threads, one CTA per SM, persistent over tiles):
 //   warp 0      TMA producer: A [128 x 64] and W [256 x 64] tiles, 128-byte
-//               swizzle, into a 4-stage shared-memory ring (mbarrier full/empty)
+//               swizzle, into a 4-stage shared-memory ring (mbarrier full/empty).
+//               Small M (every CTA holds at most one tile, W streams through
+//               fewer SMs than the GPU has): W tiles are also prefetched into
+//               L2 W_PREFETCH stages ahead of the loads, and when M <= 128
+//               the A copy carries only the M rows rounded up to 8 (the rest
+//               of the 128-row A stage is never written: the MMA still runs
+//               M=128, and rows past M, never stored, read whatever the stage
+//               held; no row of the product depends on another row).
 //   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators);
 //               lane 0 issues the MMAs and tcgen05.commit's
 //   warps 2..5  epilogue: tcgen05.ld the accumulator row by row (thread = row),
@@ -38,6 +46,7 @@ constexpr uint32_t A_BYTES = BM * BK * 2;  // 16 KB
 constexpr uint32_t B_BYTES = BN * BK * 2;  // 32 KB
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int THREADS = 192;
+constexpr int W_PREFETCH = 8;  // W stages prefetched into L2 ahead of the loads (small M)
 
 // TERMS = number of bf16 A operands summed into the product: 1 for plain
 // bf16 activations, 2 for an activation carried as a hi/lo pair (A = A_hi +
@@ -56,6 +65,8 @@ struct Params {
   int32_t c_f32;
   int32_t M, N, K;
   int32_t m_blocks, n_blocks, k_blocks;
+  int32_t w_prefetch;  // W_PREFETCH or 0 (off)
+  uint32_t a_bytes;    // bytes of one A copy: 128 rows, or M rounded up to 8 when M < 128
   int32_t* status;
 };
 
@@ -99,6 +110,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         const __grid_constant__ CUtensorMap tmB, const Params p) {
   constexpr int STAGES = Cfg<TERMS>::STAGES;
   constexpr uint32_t STAGE_BYTES = Cfg<TERMS>::STAGE_BYTES;
+  const uint32_t tx_bytes = TERMS * p.a_bytes + B_BYTES;
   extern __shared__ uint8_t smem_raw[];
   // 128-byte swizzled tiles want 1024-byte aligned bases.
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -151,10 +163,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int s = 0; s < STAGES; ++s) fills[s] = 0;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int mb = tile % p.m_blocks, nb = tile / p.m_blocks;
+        const int pf = p.w_prefetch;
+        for (int kb = 0; kb < pf && kb < p.k_blocks; ++kb) tma_prefetch_2d(&tmB, kb * BK, nb * BN);
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, p.status, abort_flag)) { ok = false; break; }
+          if (pf && kb + pf < p.k_blocks) tma_prefetch_2d(&tmB, (kb + pf) * BK, nb * BN);
           uint8_t* sa = tiles + stage * STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          mbar_arrive_expect_tx(&full[stage], tx_bytes);
           tma_load_2d(sa, &tmA, &full[stage], kb * BK, mb * BM);
           if (TERMS == 2) tma_load_2d(sa + A_BYTES, &tmA2, &full[stage], kb * BK, mb * BM);
           tma_load_2d(sa + TERMS * A_BYTES, &tmB, &full[stage], kb * BK, nb * BN);
@@ -294,7 +309,8 @@ static bi_status launch(const void* A, const void* A2, int64_t lda, const void* 
   {
     uint64_t dims[2] = {(uint64_t)K, (uint64_t)M};
     uint64_t strides[1] = {(uint64_t)lda * 2};
-    uint32_t box[2] = {BK, BM};
+    const uint32_t a_rows = M < BM ? (uint32_t)((M + 7) / 8 * 8) : (uint32_t)BM;
+    uint32_t box[2] = {BK, a_rows};
     if ((st = encode_tmap(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(A), dims,
                           strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != BI_OK)
       return st;
@@ -338,6 +354,8 @@ static bi_status launch(const void* A, const void* A2, int64_t lda, const void* 
   const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
   const int sms = num_sms();
   const int grid = (int)(tiles < sms ? tiles : sms);
+  p.w_prefetch = tiles <= sms ? W_PREFETCH : 0;
+  p.a_bytes = (uint32_t)(M < BM ? (M + 7) / 8 * 8 : BM) * BK * 2;
   gemm_tcgen05_kernel<TERMS><<<grid, THREADS, Cfg<TERMS>::SMEM_BYTES, s>>>(tmA, tmA2, tmB, p);
   BI_CHECK_LAUNCH("gemm launch");
   return BI_OK;
