@@ -39,6 +39,9 @@ SHAPES = [(4096, 14336), (14336, 4096)]          # (K, N)
 MS = [1 << i for i in range(13)]                 # 1 .. 4096
 COPIES = 3
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# dram__bytes_read.sum + dram__bytes_write.sum of one gemm_tcgen05_kernel<1>
+# launch at M=4096 K=4096 N=14336 (profiles/gemm_tcgen05_m4096_k4096_n14336.md)
+GEMM_TRAFFIC_BYTES = 155.250432e6 + 97.863936e6
 
 
 def parse():
@@ -48,6 +51,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="bi", choices=["bi", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip attention/RMSNorm/cuBLAS legs")
+    ap.add_argument("--study", default=None, choices=["precision"],
+                    help="precision study: all-bf16 vs fp32 upcast vs bf16-MLP-only decoder")
     ap.add_argument("--case", default=None, choices=["gemm", "gemm_m128", "attn", "rmsnorm"],
                     help="run 3 launches of one kernel on its workload and exit (for profilers)")
     return ap.parse_args()
@@ -344,18 +349,17 @@ def cpu_baseline_leg(target_s=10.0):
         W = fp64.bf16_bits_to_f64(synth.bf16_bits(synth.normal_bf16((N, K), 0.02, 7)))
         A = fp64.bf16_bits_to_f64(synth.bf16_bits(synth.normal_bf16((512, K), 1.0, 8)))
         mats[(K, N)] = (A, W)
-    rows, spent, flops = 8, 0.0, 0.0
+    rows, spent, flops, passes = 512, 0.0, 0.0, 0
     t_start = time.perf_counter()
-    while spent < target_s and rows <= 512:
-        t0 = time.perf_counter()
+    while spent < target_s:
         for (K, N), (A, W) in mats.items():
             fp64.gemm(A[:rows], W)
             flops += 2.0 * rows * N * K
+        passes += 1
         spent = time.perf_counter() - t_start
-        rows *= 2
     return {"value": flops / spent / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": f"oracle fp64 GEMM (numpy matmul) on the first 8..{rows // 2} rows (doubling) of A for "
-                      f"both sweep shapes, {spent:.1f} s of CPU work"}
+            "sample": f"oracle fp64 GEMM (numpy matmul) of the first {rows} rows of A against W for both "
+                      f"sweep shapes, repeated {passes} times, {spent:.1f} s of CPU work"}
 
 
 # --------------------------------------------------------------------------- main
@@ -417,8 +421,77 @@ def run_case(case):
     return 0
 
 
+def run_precision_study(n_prompts=512, prompt_len=256, oracle_prompts=4):
+    """4-layer d=2048, 16-head (MHA), FFN 5632, vocab 32000 random-init decoder
+    (std 0.02), 512 random prompts of 256 tokens, run in the three activation
+    precisions. Runtime: the whole workload on the GPU (prefill, device time).
+    Error: logits of every position of `oracle_prompts` prompts against the
+    fp64 oracle forward (teacher forced)."""
+    import numpy as np
+    import torch
+    from invariant_deterministic_03_b200 import runner, synth
+    from oracle import fp64
+    torch.cuda.set_device(0)
+    cfg = dict(n_layers=4, d_model=2048, n_q_heads=16, n_kv_heads=16, d_ff=5632, vocab=32000,
+               max_pos=512, rms_eps=1e-6, rope_theta=1e4)
+    w = synth.model_weights(cfg, seed=11)
+    wd = {k: v.cuda().contiguous() for k, v in w.items()}
+    prompts = [synth.randint(prompt_len, 0, cfg["vocab"] - 1, seed=1000 + i).tolist() for i in range(n_prompts)]
+    per_step = 64
+    out = {"workload": f"{n_prompts} prompts x {prompt_len} tokens, 4 layers d=2048 16 heads FFN 5632 vocab 32000",
+           "modes": {}}
+    ref = [fp64.forward(fp64.ModelWeights(cfg, {k: synth.bf16_bits(v) for k, v in w.items()}), prompts[i])
+           for i in range(oracle_prompts)]
+    for mode in ["bf16", "f32", "bf16_mlp"]:
+        c = dict(cfg, precision=mode)
+        eng = runner.Engine(c, wd, num_pages=per_step * prompt_len // 16 + 64, max_pages_per_seq=prompt_len // 16,
+                            max_tokens=per_step * prompt_len, max_logits=per_step, seed=0)
+        # logits of every position for the oracle prompts: one token per step
+        errs, top1, top5 = [], [], []
+        for i in range(oracle_prompts):
+            lg = torch.cat([eng.step([(10_000 + i, p, p + 1)], lambda s, i=i: prompts[i])[0]
+                            for p in range(prompt_len)])
+            e = np.abs(lg.double().cpu().numpy() - ref[i])
+            errs.append(e)
+            a = torch.from_numpy(ref[i])
+            top1.append((lg.argmax(-1).cpu() == a.argmax(-1)).double().mean().item())
+            t5g = lg.topk(5, dim=-1).indices.cpu()
+            t5r = a.topk(5, dim=-1).indices
+            top5.append(np.mean([len(set(t5g[j].tolist()) & set(t5r[j].tolist())) / 5 for j in range(prompt_len)]))
+            eng.kv.release(10_000 + i)
+        # runtime: the whole workload as prefill, 64 prompts per step
+        eng2 = runner.Engine(c, wd, num_pages=per_step * prompt_len // 16 + 64, max_pages_per_seq=prompt_len // 16,
+                             max_tokens=per_step * prompt_len, max_logits=per_step, seed=1)
+        def one_pass():
+            for s0 in range(0, n_prompts, per_step):
+                chunk = [(s, 0, prompt_len) for s in range(s0, min(n_prompts, s0 + per_step))]
+                eng2.step(chunk, lambda s: prompts[s])
+                for s, _, _ in chunk:
+                    eng2.kv.release(s)
+        one_pass()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        one_pass()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        allerr = np.concatenate([e.ravel() for e in errs])
+        out["modes"][mode] = {"max_abs_logit_err": float(allerr.max()), "mean_abs_logit_err": float(allerr.mean()),
+                              "top1_agreement": float(np.mean(top1)), "top5_overlap": float(np.mean(top5)),
+                              "ms": ms, "tokens_per_s": n_prompts * prompt_len / ms * 1e3}
+    b = out["modes"]["bf16"]["ms"]
+    for m in out["modes"].values():
+        m["runtime_vs_bf16"] = m["ms"] / b
+    out["pages_context"] = "FP32 upcast ~3x runtime, BF16-MLP-only ~1.3x (cross-vendor paper, its own hardware)"
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     args = parse()
+    if args.study == "precision":
+        return run_precision_study()
     if args.case:
         return run_case(args.case)
     if args.impl == "reference":
@@ -450,13 +523,20 @@ def main():
     big = [r for r in table if r["M"] >= 1024]
     big_fl = sum(2.0 * r["M"] * r["N"] * r["K"] for r in big)
     big_ms = sum(r["bi_ms"] for r in big)
-    achieved = big_fl / big_ms / 1e9
     peak_t = peaks.get("bf16_tflops_sustained") or peaks.get("bf16_tflops")
+    # the dominant kernel's largest launch of the step (M=4096, K=4096, N=14336):
+    # the launch the committed ncu capture measured
+    top = [r for r in table if r["M"] == 4096 and r["K"] == 4096][0]
+    achieved = 2.0 * top["M"] * top["N"] * top["K"] / top["bi_ms"] / 1e9
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
-                "frac": achieved / peak_t, "traffic": None,
-                "kernel": "bi_gemm (gemm_tcgen05_kernel), launches with M >= 1024 of the sweep",
+                "frac": achieved / peak_t, "traffic": GEMM_TRAFFIC_BYTES,
+                "kernel": "bi_gemm (gemm_tcgen05_kernel<1>), launch M=4096 K=4096 N=14336",
+                "algorithmic_bytes": 2.0 * (top["M"] * top["K"] + top["N"] * top["K"] + top["M"] * top["N"]),
                 "peak_source": f"{peak_src} bf16 dense sustained",
                 "frac_of_burst": achieved / peaks.get("bf16_tflops", peak_t)}
+    extras["roofline_m_ge_1024"] = {"achieved": big_fl / big_ms / 1e9, "unit": "TFLOP/s",
+                                    "frac": big_fl / big_ms / 1e9 / peak_t,
+                                    "launches": "M in {1024, 2048, 4096} x both shapes"}
     bi_sum = sum(r["bi_ms"] for r in table)
     th_sum = sum(r["cublas_ms"] for r in table)
     extras["sweep"] = [{k: (round(v, 4) if isinstance(v, float) else v) for k, v in r.items()} for r in table]

@@ -59,7 +59,7 @@ def _serve(cfg, wd, others, sched_seed, engine_seed):
             if done[s] < r["plen"]:
                 n = min(int(rng.choice(sizes)), r["plen"] - done[s], budget)
             else:
-                n = 1
+                n = 1 if budget > 0 else 0
             if n <= 0:
                 continue
             chunks.append((s, done[s], done[s] + n))
