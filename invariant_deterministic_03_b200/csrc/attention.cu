@@ -43,18 +43,39 @@ constexpr int TILE = BI_ATTN_TILE;     // 128 keys
 constexpr int SPLIT = BI_ATTN_SPLIT;   // 512 keys
 constexpr int PAGE = BI_PAGE_SIZE;     // 16 keys
 constexpr int PAGES_PER_TILE = TILE / PAGE;
-constexpr uint32_t TILE_BYTES = 128 * 128 * 2;  // 32 KB: Q, K, V and P tiles
-constexpr uint32_t OFF_Q = 0;                   // 2 buffers (one per work item in flight)
-constexpr uint32_t OFF_K = 2 * TILE_BYTES;      // 2 buffers
-constexpr uint32_t OFF_V = 4 * TILE_BYTES;      // 2 buffers
-constexpr uint32_t OFF_P = 6 * TILE_BYTES;
-constexpr uint32_t OFF_BAR = 7 * TILE_BYTES;
-constexpr uint32_t OFF_RING = OFF_BAR + 256;   // producer's page-id ring [16 tiles][8 pages]
-constexpr uint32_t OFF_RED = OFF_RING + 512;   // decode quarter exchange [2][4 warps][8 heads] fp32
-constexpr int ITEM_RING = 32;                  // claimed work items in flight inside a CTA
-constexpr uint32_t OFF_ITEMS = OFF_RED + 256;  // item ring [32] int32, then one mbarrier per slot
-constexpr size_t SMEM_BYTES = 1024 + 7 * TILE_BYTES + 256 + 512 + 256 + ITEM_RING * 4 + ITEM_RING * 8;
-static_assert(SMEM_BYTES <= 232448, "attention: shared memory above the 227 KB per-CTA limit");
+constexpr uint32_t TILE_BYTES = 128 * 128 * 2;  // 32 KB: one K or V tile (128 keys x 128 d)
+constexpr int ITEM_RING = 32;                   // claimed work items in flight inside a CTA
+constexpr int MAX_KV_BUF = 3;
+
+// Shared-memory layout. Prefill: Q (two buffers, one per work item in flight)
+// and P are full 128-row tiles, K and V double buffered. Decode: the MMA rows
+// that matter are the G <= 8 head rows of one query, so Q and P keep just one
+// 8-row core-matrix group per 64-column half and the MMA operand descriptor
+// repeats it for all 16 groups (8-row-group stride 0): the same 128-row MMA
+// reads the same values in every row that matters, and the ~90 KB saved buy a
+// third K and a third V buffer and a second P buffer (so the softmax of tile
+// j+1 can store its P while the P V product of tile j still runs).
+template <bool DECODE>
+struct Lay {
+  static constexpr int NK = DECODE ? 3 : 2;                 // K tile buffers
+  static constexpr int NV = DECODE ? 3 : 2;                 // V tile buffers
+  static constexpr int NP = DECODE ? 2 : 1;                 // P buffers
+  static constexpr uint32_t HALF = DECODE ? 1024 : 16384;   // bytes between the 64-column halves of Q / P
+  static constexpr uint32_t ROW_SBO = DECODE ? 0 : 1024;    // bytes between 8-row groups of Q / P
+  static constexpr uint32_t QP_BYTES = 2 * HALF;            // one Q or P buffer
+  static constexpr uint32_t OFF_K = 0;
+  static constexpr uint32_t OFF_V = OFF_K + NK * TILE_BYTES;
+  static constexpr uint32_t OFF_Q = OFF_V + NV * TILE_BYTES;  // 2 buffers
+  static constexpr uint32_t OFF_P = OFF_Q + 2 * QP_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_P + NP * QP_BYTES;
+  static constexpr uint32_t OFF_RING = OFF_BAR + 256;   // producer's page-id ring [16 tiles][8 pages]
+  static constexpr uint32_t OFF_RED = OFF_RING + 512;   // decode quarter exchange [2][4 warps][8 heads] fp32
+  static constexpr uint32_t OFF_ITEMS = OFF_RED + 256;  // item ring [32] int32, then one mbarrier per slot
+  static constexpr size_t SMEM_BYTES = 1024 + OFF_ITEMS + ITEM_RING * 4 + ITEM_RING * 8;
+  static_assert(NK <= MAX_KV_BUF && NV <= MAX_KV_BUF, "barrier arrays hold 3 K and 3 V buffers");
+  static_assert(OFF_Q % 1024 == 0 && OFF_P % 1024 == 0, "swizzled Q / P tiles need 1 KB alignment");
+  static_assert(SMEM_BYTES <= 232448, "attention: shared memory above the 227 KB per-CTA limit");
+};
 // warps 0-3: one thread per MMA row (softmax, O rescale, partials)
 // warp 4: TMA producer; warp 5: TMEM allocator and MMA issuer
 constexpr int THREADS = 192;
@@ -217,27 +238,31 @@ static_assert(PF_RING * 8 * 4 <= 512, "page-id ring overflows its region");
 // K: 8 page blocks of 16 keys, canonical no-swizzle K-major: core matrices of
 // 8 keys x 8 d (128 B), d-chunks 128 B apart (LBO), 8-key groups 2 KB apart
 // (SBO, uniform across the blocks of a tile).
+template <bool DECODE>
 __device__ __forceinline__ void issue_s(uint32_t tmem_s, uint32_t q_addr, uint32_t k_addr) {
+  using L = Lay<DECODE>;
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
 #pragma unroll
   for (int kk = 0; kk < HD / 16; ++kk) {
-    const uint32_t qoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-    mma_bf16(tmem_s, smem_desc(q_addr + qoff, 16, 1024, 2), smem_desc(k_addr + kk * 256, 128, 2048, 0),
+    const uint32_t qoff = (kk >> 2) * L::HALF + (kk & 3) * 32;
+    mma_bf16(tmem_s, smem_desc(q_addr + qoff, 16, L::ROW_SBO, 2), smem_desc(k_addr + kk * 256, 128, 2048, 0),
              idesc, kk != 0);
   }
 }
 
 // O (+)= P V: accumulate = 0 on the first tile of a split, 1 after.
+template <bool DECODE>
 __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t p_addr, uint32_t v_addr,
                                          bool accumulate) {
+  using L = Lay<DECODE>;
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
 #pragma unroll
   for (int j = 0; j < PAGES_PER_TILE; ++j) {
-    const uint32_t poff = (j >> 2) * 16384 + (j & 3) * 32;
+    const uint32_t poff = (j >> 2) * L::HALF + (j & 3) * 32;
     // V page block j (16 keys = one K step): canonical no-swizzle K-major with
     // rows = d: core matrices of 8 d x 8 keys, key-chunks 128 B apart (LBO),
     // 8-d groups 256 B apart (SBO).
-    mma_bf16(tmem_o, smem_desc(p_addr + poff, 16, 1024, 2),
+    mma_bf16(tmem_o, smem_desc(p_addr + poff, 16, L::ROW_SBO, 2),
              smem_desc(v_addr + j * BLOCK_BYTES, 128, 256, 0), idesc, (accumulate || j != 0) ? 1u : 0u);
   }
 }
@@ -271,6 +296,21 @@ __device__ __forceinline__ float quarter_p(const uint32_t (&S)[32], int nvalid, 
   return q;
 }
 
+// The row's reference maximum for tile t (log2 domain), given the previous
+// reference m and this tile's scaled maximum: the first tile of a split takes
+// its maximum; a later tile keeps m unless the new maximum exceeds it by more
+// than 2^RESCALE_LOG2 (then P values stay below 2^8, exact to bf16 like any
+// others, and O and l need no rescale, so the softmax of the next tile rarely
+// waits for the P V of this one). The choice depends on the row's own values
+// only, and decode and prefill make it identically; the split's final O / l
+// (and the merge, which takes each split's m as its reference) do not depend
+// on which reference was used beyond rounding.
+constexpr float RESCALE_LOG2 = 8.0f;
+__device__ __forceinline__ float new_reference(float m, float tile_max, int t) {
+  const float mc = fmaxf(m, tile_max);
+  return (t > 0 && __fsub_rn(mc, m) <= RESCALE_LOG2) ? m : mc;
+}
+
 __device__ __forceinline__ float quarter_max(const uint32_t (&S)[32], int nvalid) {
   float m = -INFINITY;
 #pragma unroll
@@ -278,12 +318,14 @@ __device__ __forceinline__ float quarter_max(const uint32_t (&S)[32], int nvalid
   return m;
 }
 
-__device__ __forceinline__ void store_p_chunks(uint8_t* p_smem, int row, int quarter,
+// P row `row`, keys 32*quarter .. +31, into the 128-byte-swizzled P tile whose
+// two 64-key halves lie `half` bytes apart.
+__device__ __forceinline__ void store_p_chunks(uint8_t* p_smem, uint32_t half, int row, int quarter,
                                                const uint32_t (&P)[16]) {
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int chunk = quarter * 4 + k;  // 8 keys per 16-byte chunk
-    const uint32_t addr = (uint32_t)(chunk >> 3) * 16384u + (uint32_t)row * 128u +
+    const uint32_t addr = (uint32_t)(chunk >> 3) * half + (uint32_t)row * 128u +
                           (uint32_t)(((chunk & 7) ^ (row & 7)) << 4);
     *reinterpret_cast<uint4*>(p_smem + addr) = make_uint4(P[4 * k], P[4 * k + 1], P[4 * k + 2], P[4 * k + 3]);
   }
@@ -311,31 +353,36 @@ __device__ __forceinline__ void drain(uint64_t* bar, int fills) {
 // Row arithmetic (thread = row, fixed order, same in decode and prefill):
 //   first tile of the split:  m = max_j s_j (log2 domain, s_j = S_ij * scale*log2e),
 //                             P_j = bf16(2^(s_j - m)), l = sum_j P_j, O = P V
-//   later tiles:              m' = max(m, max_j s_j), alpha = 2^(m - m'),
+//   later tiles:              c = max(m, max_j s_j); m' = m if c - m <= 8 else c
+//                             (new_reference), alpha = 2^(m - m'),
 //                             P_j = bf16(2^(s_j - m')), l = alpha*l + sum_j P_j,
 //                             O = alpha*O (fp32, skipped when alpha == 1), O += P V (MMA)
 // sums over j run j = 0..127 in order; masked keys have P_j = 0 by selection.
 template <bool DECODE>
 __global__ void __launch_bounds__(THREADS, 1)
     attn_split_kernel(const __grid_constant__ CUtensorMap tmQ, const Params p) {
+  using L = Lay<DECODE>;
+  constexpr int NK = L::NK, NV = L::NV;
+  constexpr uint32_t OFF_Q = L::OFF_Q, OFF_K = L::OFF_K, OFF_V = L::OFF_V, OFF_P = L::OFF_P;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* q_full = bars + 0;     // [2]
   uint64_t* q_empty = bars + 2;    // [2]
-  uint64_t* k_full = bars + 4;     // [2]
-  uint64_t* v_full = bars + 6;     // [2]
-  uint64_t* k_empty = bars + 8;    // [2]
-  uint64_t* v_empty = bars + 10;   // [2]
-  uint64_t* s_full = bars + 12;    // [2]
-  uint64_t* s_free = bars + 14;    // [2]
-  uint64_t* p_ready = bars + 16;
-  uint64_t* o_ready = bars + 17;
-  uint64_t* x_bar = bars + 18;     // decode: quarter exchange among the 4 softmax warps
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
-  int32_t* item_ring = reinterpret_cast<int32_t*>(smem + OFF_ITEMS);
-  uint64_t* item_bar = reinterpret_cast<uint64_t*>(smem + OFF_ITEMS + ITEM_RING * 4);
+  uint64_t* k_full = bars + 4;     // [NK]
+  uint64_t* k_empty = bars + 7;    // [NK]
+  uint64_t* v_full = bars + 10;    // [NV]
+  uint64_t* v_empty = bars + 13;   // [NV]
+  uint64_t* s_full = bars + 16;    // [2]
+  uint64_t* s_free = bars + 18;    // [2]
+  uint64_t* p_ready = bars + 20;   // [NP]
+  uint64_t* o_ready = bars + 22;   // [NP]: P V of the tile that read P buffer i is done
+  uint64_t* x_bar = bars + 24;     // decode: quarter exchange among the 4 softmax warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 25);
+  static_assert(26 * 8 <= 256, "barrier region");
+  int32_t* item_ring = reinterpret_cast<int32_t*>(smem + L::OFF_ITEMS);
+  uint64_t* item_bar = reinterpret_cast<uint64_t*>(smem + L::OFF_ITEMS + ITEM_RING * 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -345,15 +392,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
-      mbar_init(&k_full[i], 1);
-      mbar_init(&v_full[i], 1);
-      mbar_init(&k_empty[i], 1);
-      mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 128);
     }
-    mbar_init(p_ready, 128);
-    mbar_init(o_ready, 1);
+    for (int i = 0; i < NK; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < NV; ++i) {
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < L::NP; ++i) {
+      mbar_init(&p_ready[i], 128);
+      mbar_init(&o_ready[i], 1);
+    }
     mbar_init(x_bar, 128);
     for (int i = 0; i < ITEM_RING; ++i) mbar_init(&item_bar[i], 1);
     *abort_flag = 0;
@@ -375,7 +428,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // copies go out together. All lanes walk the same cursors.
     if (lane == 0) prefetch_tmap(&tmQ);
     const uint32_t q_bytes = 2u * 64u * 2u * (uint32_t)(p.G * p.q_box);
-    int32_t* ring = reinterpret_cast<int32_t*>(smem + OFF_RING);  // [PF_RING][8]
+    int32_t* ring = reinterpret_cast<int32_t*>(smem + L::OFF_RING);  // [PF_RING][8]
     Cursor kc, vc, pf;
     pf.n = -1;
     pf.t = 0;
@@ -384,7 +437,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     bool ok = cursor_start(p, kc, item_ring, item_bar, abort_flag);
     vc = kc;
     int nk = 0, nv = 0, npf = 0, qi = 0;
-    int q_fills[2] = {0, 0}, k_fills[2] = {0, 0}, v_fills[2] = {0, 0};
+    int q_fills[2] = {0, 0}, k_fills[NK] = {}, v_fills[NV] = {};
     for (; pf.valid && npf < PF_AHEAD; ++npf, claim_next(p, pf, item_ring, item_bar, lane))
       if (lane < PAGES_PER_TILE)
         ring[(npf & (PF_RING - 1)) * 8 + lane] =
@@ -398,30 +451,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     while ((kc.valid || vc.valid) && ok) {
       bool progressed = false;
       if (kc.valid) {
-        const int kb = nk & 1, qb = qi & 1;
+        const int kb = nk % NK, qb = qi & 1;
         int ready = 0;
         if (lane == 0) {
-          ready = mbar_test(&k_empty[kb], (((uint32_t)nk >> 1) & 1u) ^ 1u);
+          ready = mbar_test(&k_empty[kb], (((uint32_t)nk / NK) & 1u) ^ 1u);
           if (ready && kc.t == 0) ready = mbar_test(&q_empty[qb], (((uint32_t)qi >> 1) & 1u) ^ 1u);
         }
         if (__shfl_sync(0xffffffffu, ready, 0)) {
           if (kc.t == 0) {  // first tile of an item: its Q rows
             if (lane == 0) {
-              uint8_t* qdst = smem + OFF_Q + qb * TILE_BYTES;
-              if (!DECODE) {
-                mbar_arrive_expect_tx(&q_full[qb], q_bytes);
-                tma_load_3d(qdst, &tmQ, &q_full[qb], 0, kc.it.g * p.G, kc.it.r0 + kc.it.q_lo);
-                tma_load_3d(qdst + 16384, &tmQ, &q_full[qb], 64, kc.it.g * p.G, kc.it.r0 + kc.it.q_lo);
-              } else {
-                // the G head rows again at rows 32, 64 and 96 (one copy per softmax warp)
-                mbar_arrive_expect_tx(&q_full[qb], 4u * q_bytes);
-#pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                  tma_load_3d(qdst + w * 32 * 128, &tmQ, &q_full[qb], 0, kc.it.g * p.G, kc.it.r0 + kc.it.q_lo);
-                  tma_load_3d(qdst + 16384 + w * 32 * 128, &tmQ, &q_full[qb], 64, kc.it.g * p.G,
-                              kc.it.r0 + kc.it.q_lo);
-                }
-              }
+              // both 64-column halves (decode: the G head rows, which the
+              // MMA descriptor repeats over all 128 rows)
+              uint8_t* qdst = smem + OFF_Q + qb * L::QP_BYTES;
+              mbar_arrive_expect_tx(&q_full[qb], q_bytes);
+              tma_load_3d(qdst, &tmQ, &q_full[qb], 0, kc.it.g * p.G, kc.it.r0 + kc.it.q_lo);
+              tma_load_3d(qdst + L::HALF, &tmQ, &q_full[qb], 64, kc.it.g * p.G, kc.it.r0 + kc.it.q_lo);
             }
             ++q_fills[qb];
             ++qi;
@@ -452,9 +496,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       if (vc.valid && nv < nk) {
-        const int vb = nv & 1;
+        const int vb = nv % NV;
         int ready = 0;
-        if (lane == 0) ready = mbar_test(&v_empty[vb], (((uint32_t)nv >> 1) & 1u) ^ 1u);
+        if (lane == 0) ready = mbar_test(&v_empty[vb], (((uint32_t)nv / NV) & 1u) ^ 1u);
         if (__shfl_sync(0xffffffffu, ready, 0)) {
           if (lane == 0) mbar_arrive_expect_tx(&v_full[vb], TILE_BYTES);
           __syncwarp();
@@ -486,11 +530,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     // be waiting for ring entries the look-ahead has not reached
     while (ok && pf.valid) claim_next(p, pf, item_ring, item_bar, lane);
     if (!ok && lane == 0) {
-      for (int i = 0; i < 2; ++i) {
-        drain(&q_full[i], q_fills[i]);
-        drain(&k_full[i], k_fills[i]);
-        drain(&v_full[i], v_fills[i]);
-      }
+      for (int i = 0; i < 2; ++i) drain(&q_full[i], q_fills[i]);
+      for (int i = 0; i < NK; ++i) drain(&k_full[i], k_fills[i]);
+      for (int i = 0; i < NV; ++i) drain(&v_full[i], v_fills[i]);
     }
   } else if (warp == 5) {
     // ------------------------------------------------ MMA issuer (one thread)
@@ -506,14 +548,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       while ((sc.valid || nP < nS) && ok) {
         bool progressed = false;
         if (sc.valid && nS - nP < 2) {
-          const int kb = nS & 1, qb = qi & 1;
+          const int sb = nS & 1, kb = nS % NK, qb = qi & 1;
           const bool ready = (sc.t != 0 || mbar_test(&q_full[qb], ((uint32_t)qi >> 1) & 1u)) &&
-                             mbar_test(&k_full[kb], ((uint32_t)nS >> 1) & 1u) &&
-                             mbar_test(&s_free[kb], (((uint32_t)nS >> 1) & 1u) ^ 1u);
+                             mbar_test(&k_full[kb], ((uint32_t)nS / NK) & 1u) &&
+                             mbar_test(&s_free[sb], (((uint32_t)nS >> 1) & 1u) ^ 1u);
           if (ready) {
             tc_fence_after();
-            issue_s(tmem + kb * 128, sQ0 + qb * TILE_BYTES, sK0 + kb * TILE_BYTES);
-            mma_commit(&s_full[kb]);
+            issue_s<DECODE>(tmem + sb * 128, sQ0 + qb * L::QP_BYTES, sK0 + kb * TILE_BYTES);
+            mma_commit(&s_full[sb]);
             mma_commit(&k_empty[kb]);
             const uint32_t bit = 1u << (nS & 31);
             acc_bits = sc.t > 0 ? (acc_bits | bit) : (acc_bits & ~bit);
@@ -526,12 +568,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
         if (nP < nS) {
-          const int vb = nP & 1;
-          if (mbar_test(p_ready, (uint32_t)nP & 1u) && mbar_test(&v_full[vb], ((uint32_t)nP >> 1) & 1u)) {
+          const int vb = nP % NV, pb = nP % L::NP;
+          if (mbar_test(&p_ready[pb], ((uint32_t)nP / L::NP) & 1u) &&
+              mbar_test(&v_full[vb], ((uint32_t)nP / NV) & 1u)) {
             const uint32_t bit = 1u << (nP & 31);
             tc_fence_after();
-            issue_pv(tmem + TMEM_O, sP, sV0 + vb * TILE_BYTES, (acc_bits & bit) != 0);
-            mma_commit(o_ready);
+            issue_pv<DECODE>(tmem + TMEM_O, sP + pb * L::QP_BYTES, sV0 + vb * TILE_BYTES, (acc_bits & bit) != 0);
+            mma_commit(&o_ready[pb]);
             mma_commit(&v_empty[vb]);
             if (last_bits & bit) mma_commit(&q_empty[(qb_bits & bit) ? 1 : 0]);
             ++nP;
@@ -562,10 +605,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const int qr = decode ? 0 : r / p.G;
     const int hj = decode ? lane : r - qr * p.G;
-    float* red = reinterpret_cast<float*>(smem + OFF_RED);  // [2][4 warps][8 head rows]
+    float* red = reinterpret_cast<float*>(smem + L::OFF_RED);  // [2][4 warps][8 head rows]
     int j = 0, xc = 0;
     bool ok = true;
-    bool o_pending = false;  // o_ready of tile j-1 not yet waited for
+    // waits until the P V product of tile jj (counted across this CTA's items) is done
+    auto pv_done = [&](int jj) -> bool {
+      if (!mbar_wait(&o_ready[jj % L::NP], ((uint32_t)jj / L::NP) & 1u, p.status, abort_flag)) return false;
+      tc_fence_after();
+      return true;
+    };
     auto exchange = [&](float v, int which) -> bool {
       if (lane < 8) red[(which * 4 + warp) * 8 + lane] = v;
       mbar_arrive(x_bar);
@@ -608,7 +656,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int w = 0; w < 4; ++w) mraw = fmaxf(mraw, red[w * 8 + (lane & 7)]);
           if (need) {
-            m_new = fmaxf(m, __fmul_rn(mraw, p.scale_log2));
+            m_new = new_reference(m, __fmul_rn(mraw, p.scale_log2), t);
             alpha = ex2_approx(__fsub_rn(m, m_new));
           }
           const float qs = quarter_p(S, nq, -m_new, p.scale_log2, P);
@@ -619,16 +667,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             l = (t == 0) ? lsum : __fadd_rn(__fmul_rn(alpha, l), lsum);
             m = m_new;
           }
-          if (o_pending) {
-            if (!mbar_wait(o_ready, (uint32_t)(j - 1) & 1u, p.status, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            o_pending = false;
-          }
-          if (lane < p.G) {
-#pragma unroll
-            for (int v = 0; v < 4; ++v) store_p_chunks(smem + OFF_P, v * 32 + lane, warp, P);
-          }
+          // P buffer j % NP was last read by the P V of tile j - NP
+          if (j >= L::NP && !pv_done(j - L::NP)) { ok = false; break; }
+          if (lane < p.G) store_p_chunks(smem + OFF_P + (j % L::NP) * L::QP_BYTES, L::HALF, lane, warp, P);
           if (t > 0 && __any_sync(0xffffffffu, need && alpha != 1.0f)) {
+            // O may be rescaled only once the P V of tile j-1 has landed in it
+            if (L::NP > 1 && !pv_done(j - 1)) { ok = false; break; }
             uint32_t o[32];
             tmem_ld32(tmem + TMEM_O + lane_off + warp * 32, o);
             tmem_ld_wait();
@@ -658,7 +702,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               mraw = fmaxf(mraw, quarter_max(*reinterpret_cast<uint32_t(*)[32]>(&S[q * 32]),
                                              min(32, max(0, nvalid - q * 32))));
             if (need) {
-              m_new = fmaxf(m, __fmul_rn(mraw, p.scale_log2));
+              m_new = new_reference(m, __fmul_rn(mraw, p.scale_log2), t);
               alpha = ex2_approx(__fsub_rn(m, m_new));
             }
             float qs[4];
@@ -673,16 +717,14 @@ __global__ void __launch_bounds__(THREADS, 1)
               m = m_new;
             }
           }
-          // P V of the previous tile must be done before P and O are touched
-          if (o_pending) {
-            if (!mbar_wait(o_ready, (uint32_t)(j - 1) & 1u, p.status, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            o_pending = false;
-          }
+          // the P V that last read this P buffer (one buffer: tile j-1) must be
+          // done before P and O are touched
+          if (j >= L::NP && !pv_done(j - L::NP)) { ok = false; break; }
+          static_assert(DECODE || L::NP == 1, "prefill rescales O right after the P buffer wait");
           if (warp_valid) {
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-              store_p_chunks(smem + OFF_P, r, q, *reinterpret_cast<uint32_t(*)[16]>(&P[q * 16]));
+              store_p_chunks(smem + OFF_P, L::HALF, r, q, *reinterpret_cast<uint32_t(*)[16]>(&P[q * 16]));
             // rescale O in tensor memory (not on the split's first tile, whose P V overwrites O)
             if (t > 0 && __any_sync(0xffffffffu, need && alpha != 1.0f)) {
               const float a = need ? alpha : 1.0f;
@@ -701,8 +743,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         // zero V slots at or past the sequence end inside this tile's last page
         if (tail != 0 && last_page / PAGES_PER_TILE == it.t0 + t) {
-          if (!mbar_wait(&v_full[sb], ((uint32_t)j >> 1) & 1u, p.status, abort_flag)) { ok = false; break; }
-          uint8_t* vblk = smem + OFF_V + sb * TILE_BYTES + (last_page % PAGES_PER_TILE) * BLOCK_BYTES;
+          const int vb = j % NV;
+          if (!mbar_wait(&v_full[vb], ((uint32_t)j / NV) & 1u, p.status, abort_flag)) { ok = false; break; }
+          uint8_t* vblk = smem + OFF_V + vb * TILE_BYTES + (last_page % PAGES_PER_TILE) * BLOCK_BYTES;
           const int d = r;  // value row d of the block
           for (int slot = tail; slot < PAGE; ++slot) {
             const uint32_t off = (uint32_t)(d >> 3) * 256u + (uint32_t)(slot >> 3) * 128u +
@@ -712,14 +755,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(p_ready);
-        o_pending = true;
+        mbar_arrive(&p_ready[j % L::NP]);
       }
       if (!ok) break;
       // end of the split: unnormalised O, m, l of every valid row
-      if (!mbar_wait(o_ready, (uint32_t)(j - 1) & 1u, p.status, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      o_pending = false;
+      if (!pv_done(j - 1)) { ok = false; break; }
       const size_t widx = ((size_t)(it.r0 + q_idx) * p.Hq + (size_t)(it.g * p.G + hj)) * p.n_split_max + it.s;
       if constexpr (decode) {
         uint32_t o[32];
@@ -920,11 +960,11 @@ static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t ma
   int dev = 0;
   cudaGetDevice(&dev);
   if (!attr_set[dev & 63]) {
-    cudaError_t e = cudaFuncSetAttribute(attn_split_kernel<true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(attn_split_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Lay<true>::SMEM_BYTES);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(attn_split_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)SMEM_BYTES);
+                               (int)Lay<false>::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e, "attention: smem attribute");
     attr_set[dev & 63] = true;
   }
@@ -933,9 +973,9 @@ static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t ma
   cudaError_t me = cudaMemsetAsync(p.work_counter, 0, sizeof(int32_t), stream);
   if (me != cudaSuccess) return cuda_fail(me, "attention: work counter reset");
   if (cu_q)
-    attn_split_kernel<false><<<grid, THREADS, SMEM_BYTES, stream>>>(tmQ, p);
+    attn_split_kernel<false><<<grid, THREADS, Lay<false>::SMEM_BYTES, stream>>>(tmQ, p);
   else
-    attn_split_kernel<true><<<grid, THREADS, SMEM_BYTES, stream>>>(tmQ, p);
+    attn_split_kernel<true><<<grid, THREADS, Lay<true>::SMEM_BYTES, stream>>>(tmQ, p);
   BI_CHECK_LAUNCH("attention split launch");
 
   CombineParams c;
