@@ -53,7 +53,7 @@ def parse():
     ap.add_argument("--no-extras", action="store_true", help="skip attention/RMSNorm/cuBLAS legs")
     ap.add_argument("--study", default=None, choices=["precision"],
                     help="precision study: all-bf16 vs fp32 upcast vs bf16-MLP-only decoder")
-    ap.add_argument("--case", default=None, choices=["gemm", "gemm_m128", "attn", "rmsnorm"],
+    ap.add_argument("--case", default=None, choices=["gemm", "gemm_m128", "attn", "rmsnorm", "forward"],
                     help="run 3 launches of one kernel on its workload and exit (for profilers)")
     return ap.parse_args()
 
@@ -284,6 +284,96 @@ def attention_leg(bi, torch, synth, reps):
             "ms": ms, "kv_bytes": kv_bytes, "gbs": kv_bytes / ms / 1e6}
 
 
+def flash_decode_leg(torch, synth, reps):
+    """The same decode workload through flash-attn's varlen kernel on K/V
+    gathered into contiguous per-sequence rows: a non-invariant cost
+    reference (its split count follows the batch), not part of the path."""
+    try:
+        from flash_attn import flash_attn_varlen_func
+    except Exception as e:  # noqa: BLE001
+        return {"unavailable": f"flash_attn import failed: {type(e).__name__}"}
+    lens = synth.attention_lengths(32, 1, 8192, seed=0)
+    Hq, Hkv, D = 32, 8, 128
+    g = torch.Generator("cuda").manual_seed(1)
+    n = sum(lens)
+    k = torch.randn(n, Hkv, D, device="cuda", generator=g).to(torch.bfloat16)
+    v = torch.randn(n, Hkv, D, device="cuda", generator=g).to(torch.bfloat16)
+    q = torch.randn(32, Hq, D, device="cuda", generator=g).to(torch.bfloat16)
+    cu_k = torch.tensor([0] + list(__import__("itertools").accumulate(lens)), dtype=torch.int32, device="cuda")
+    cu_q = torch.arange(33, dtype=torch.int32, device="cuda")
+    fn = lambda r=0: flash_attn_varlen_func(q, k, v, cu_q, cu_k, 1, max(lens),  # noqa: E731
+                                            softmax_scale=D ** -0.5, causal=False)
+    ms = per_launch_ms(torch, fn, reps)
+    kv_bytes = n * Hkv * D * 2 * 2
+    return {"kernel": "flash_attn_varlen_func (flash-attn 2, contiguous K/V)", "ms": ms,
+            "gbs": kv_bytes / ms / 1e6}
+
+
+FWD_CFG = dict(n_layers=32, d_model=4096, n_q_heads=32, n_kv_heads=8, d_ff=14336, vocab=32000,
+               max_pos=4096, rms_eps=1e-6, rope_theta=1e4)
+
+
+def forward_setup(torch, cfg=FWD_CFG, seed=0):
+    """bi_forward at the Mistral-7B shape with random-init bf16 weights (std
+    0.02, norms 1) drawn on the device, and a serving mix already in the KV
+    cache: 64 requests, one with a 1400-token context and 63 with contexts
+    U[16, 2048] (seed 2). Returns the engine plus two prepared batches: a
+    decode step over all 64 requests (64 tokens) and a prefill step of four
+    fresh 2048-token prompts (8192 tokens)."""
+    from invariant_deterministic_03_b200 import runner, synth
+    g = torch.Generator("cuda").manual_seed(seed)
+    L, D, F, V = cfg["n_layers"], cfg["d_model"], cfg["d_ff"], cfg["vocab"]
+    hq, hkv = cfg["n_q_heads"], cfg["n_kv_heads"]
+
+    def rnd(*shape):
+        out = torch.empty(*shape, dtype=torch.bfloat16, device="cuda")
+        for i in range(shape[0] if len(shape) == 3 else 1):
+            dst = out[i] if len(shape) == 3 else out
+            dst.copy_(torch.randn(*dst.shape, device="cuda", generator=g) * 0.02)
+        return out
+    w = {"embed": rnd(V, D), "lm_head": rnd(V, D),
+         "final_norm": torch.ones(D, dtype=torch.bfloat16, device="cuda"),
+         "attn_norm": torch.ones(L, D, dtype=torch.bfloat16, device="cuda"),
+         "mlp_norm": torch.ones(L, D, dtype=torch.bfloat16, device="cuda"),
+         "w_qkv": rnd(L, (hq + 2 * hkv) * 128, D), "w_o": rnd(L, D, hq * 128),
+         "w_gate_up": rnd(L, 2 * F, D), "w_down": rnd(L, D, F)}
+    ctx = [1400] + synth.randint(63, 16, 2048, seed=2).tolist()
+    fresh = [2048] * 4
+    pages = sum((c + 1 + 15) // 16 for c in ctx) + sum((f + 15) // 16 for f in fresh) + 64
+    eng = runner.Engine(cfg, w, num_pages=pages, max_pages_per_seq=cfg["max_pos"] // 16,
+                        max_tokens=8192, max_logits=64, seed=seed)
+    toks = synth.randint(cfg["max_pos"], 0, V - 1, seed=3).tolist()
+    for s, c in enumerate(ctx):          # contexts already cached (content irrelevant for timing)
+        eng.kv.ensure(s, c + 1)
+        eng.kv.length[s] = c
+    decode = runner.make_batch(eng.kv, [(s, c, c + 1) for s, c in enumerate(ctx)], lambda s: toks)
+    prefill = runner.make_batch(eng.kv, [(100 + i, 0, f) for i, f in enumerate(fresh)], lambda s: toks)
+    for b in (decode, prefill):
+        b["max_kv_len"] = cfg["max_pos"]
+    return eng, w, decode, prefill
+
+
+def forward_leg(torch, reps):
+    eng, w, decode, prefill = forward_setup(torch)
+    out = {"workload": "Mistral-7B shape (32 layers, d 4096, 32/8 heads, FFN 14336, vocab 32000), "
+                       "random-init bf16; decode: 64 requests (contexts 1400 + 63 x U[16,2048]); "
+                       "prefill: 4 x 2048-token prompts",
+           "gflop_per_token_weights": 2.0 * sum(v.numel() for k, v in w.items() if k not in ("embed",)) / 1e9}
+    for name, b in (("decode", decode), ("prefill", prefill)):
+        n_log = b["logits_rows"].shape[0]
+        logits = torch.empty(n_log, FWD_CFG["vocab"], dtype=torch.float32, device="cuda")
+        nxt = torch.empty(n_log, dtype=torch.int32, device="cuda")
+        fn = lambda r=0, b=b, logits=logits, nxt=nxt: eng.model.forward(  # noqa: E731
+            b, eng.kv.k, eng.kv.v, logits, nxt, eng.ws)
+        ms = per_launch_ms(torch, fn, reps)
+        n_tok = b["tokens"].shape[0]
+        out[name] = {"tokens": n_tok, "ms": ms, "tokens_per_s": n_tok / ms * 1e3,
+                     "tflops": n_tok * out["gflop_per_token_weights"] / ms / 1e3}
+    del eng, w
+    torch.cuda.empty_cache()
+    return out
+
+
 def rmsnorm_leg(bi, torch, reps):
     M, D = 65536, 4096
     g = torch.Generator("cuda").manual_seed(2)
@@ -391,6 +481,19 @@ def run_case(case):
     from invariant_deterministic_03_b200 import bi, synth
     torch.cuda.set_device(0)
     g = torch.Generator("cuda").manual_seed(0)
+    if case == "forward":
+        # one decode step and one prefill step of the 7B-shape forward after a
+        # warm-up of each (for a launch list of every kernel they run)
+        eng, _, decode, prefill = forward_setup(torch)
+        for b in (decode, prefill, decode, prefill):
+            n_log = b["logits_rows"].shape[0]
+            logits = torch.empty(n_log, FWD_CFG["vocab"], dtype=torch.float32, device="cuda")
+            nxt = torch.empty(n_log, dtype=torch.int32, device="cuda")
+            eng.model.forward(b, eng.kv.k, eng.kv.v, logits, nxt, eng.ws)
+        torch.cuda.synchronize()
+        assert bi.bi_device_status(clear=True) == 0
+        print("case forward: ok")
+        return 0
     if case in ("gemm", "gemm_m128"):
         M = 4096 if case == "gemm" else 128
         A = torch.randn(M, 4096, device="cuda", generator=g).to(torch.bfloat16)
@@ -546,11 +649,13 @@ def main():
     if not args.no_extras:
         a = attention_leg(bi, torch, synth, reps=10)
         a["frac"] = a["gbs"] / peaks["hbm_gbs"]
+        a["flash_attn_reference"] = flash_decode_leg(torch, synth, reps=10)
         r = rmsnorm_leg(bi, torch, reps=10)
         r["frac"] = r["gbs"] / peaks["hbm_gbs"]
         extras["attn_decode"] = a
         extras["rmsnorm"] = r
         extras["invariance"] = invariance_flags(torch, sw)
+        extras["forward"] = forward_leg(torch, reps=5)
 
     e2e_ms, h2d, d2h = e2e_leg(bi, torch, sw, steps=max(2, min(args.steps, 5)))
     e2e_ms = max_over_ranks(e2e_ms, world)

@@ -50,7 +50,10 @@ typedef enum {
   BI_ERR_DEVICE_CHECK = 7 /* device status word non-zero (bi_device_status) */
 } bi_status;
 
-typedef enum { BI_BF16 = 0, BI_F32 = 1 } bi_dtype;
+/* Output element types of the GEMMs. BI_F32_ADD: C is fp32 and the product
+ * is added to it (C = C + A W^T, one fp32 addition per element after the
+ * whole K reduction), as a residual connection into an fp32 stream. */
+typedef enum { BI_BF16 = 0, BI_F32 = 1, BI_F32_ADD = 2 } bi_dtype;
 
 /* Fixed geometry. These are compile-time constants on purpose: a tile or split
  * size chosen at run time from the problem shape would make the reduction order
@@ -115,6 +118,18 @@ bi_status bi_rmsnorm_f32in(const float* x, const void* gamma, void* y,
 bi_status bi_gemm(const void* A, int64_t lda, const void* W, int64_t ldw,
                   void* C, int64_t ldc, int32_t c_dtype, int64_t M, int64_t N,
                   int64_t K, void* stream);
+
+/* Gate/up projection with the SwiGLU activation in its epilogue. W is
+ * [2F, K] (row stride ldw): gate rows 0..F-1, then up rows F..2F-1, as a
+ * fused nn.Linear. out [M, F] bf16 (row stride ldo):
+ *   g = bf16(A Wg^T), u = bf16(A Wu^T) exactly as bi_gemm computes them,
+ *   out = bf16(g / (1 + e^-g) * u) in fp32 (the same steps as bi_swiglu).
+ * Each 128 x 256 tile holds 128 gate and the matching 128 up columns, so the
+ * per-element reduction is bi_gemm's, whatever M is. Constraints as bi_gemm
+ * with N = F. */
+bi_status bi_gemm_swiglu(const void* A, int64_t lda, const void* W,
+                         int64_t ldw, void* out, int64_t ldo, int64_t M,
+                         int64_t F, int64_t K, void* stream);
 
 /* ------------------------------------------------------------------------ */
 /* Paged KV cache.  "Defeating Nondeterminism in LLM Inference", section

@@ -29,7 +29,7 @@ lib = ctypes.CDLL(LIB_PATH)
 
 BI_OK, BI_ERR_INVALID_ARG, BI_ERR_SHAPE, BI_ERR_ALIGN, BI_ERR_WORKSPACE, \
     BI_ERR_UNSUPPORTED, BI_ERR_CUDA, BI_ERR_DEVICE_CHECK = range(8)
-BI_BF16, BI_F32 = 0, 1
+BI_BF16, BI_F32, BI_F32_ADD = 0, 1, 2
 BI_PREC_BF16, BI_PREC_F32, BI_PREC_BF16_MLP = 0, 1, 2
 PRECISIONS = {"bf16": BI_PREC_BF16, "f32": BI_PREC_F32, "bf16_mlp": BI_PREC_BF16_MLP}
 HEAD_DIM, PAGE_SIZE, ATTN_TILE, ATTN_SPLIT = 128, 16, 128, 512
@@ -74,6 +74,7 @@ _SIGS = {
     "bi_rmsnorm": (_i32, [_p, _p, _p, _i64, _i64, _f32, _p]),
     "bi_rmsnorm_f32in": (_i32, [_p, _p, _p, _i64, _i64, _f32, _p]),
     "bi_gemm": (_i32, [_p, _i64, _p, _i64, _p, _i64, _i32, _i64, _i64, _i64, _p]),
+    "bi_gemm_swiglu": (_i32, [_p, _i64, _p, _i64, _p, _i64, _i64, _i64, _i64, _p]),
     "bi_kv_append": (_i32, [_p, _p, _i64, _p, _i64, _p, _p, ctypes.POINTER(KVLayout), _p]),
     "bi_attn_workspace_size": (_i32, [ctypes.POINTER(AttnShape), _i64, ctypes.POINTER(_sz)]),
     "bi_attn_decode": (_i32, [_p, _i64, _p, _p, _p, _p, _i32, ctypes.POINTER(AttnShape), _p,
@@ -146,21 +147,40 @@ def bi_rmsnorm(x, gamma, y, eps: float, stream=None) -> None:
     _chk(fn, getattr(lib, fn)(_ptr(x), _ptr(gamma), _ptr(y), M, D, eps, _stream(stream)))
 
 
-def bi_gemm(A, W, C, stream=None) -> None:
-    """C = A W^T. A [M, K] bf16, W [N, K] bf16, C [M, N] bf16 or fp32 (row strides
-    taken from the tensors)."""
+def bi_gemm(A, W, C, stream=None, add: bool = False) -> None:
+    """C = A W^T (or, add=True with fp32 C, C += A W^T). A [M, K] bf16, W [N, K]
+    bf16, C [M, N] bf16 or fp32 (row strides taken from the tensors)."""
     M, K = A.shape
     N = W.shape[0]
     cdt = BI_F32 if C.dtype == torch.float32 else BI_BF16
+    if add:
+        if cdt != BI_F32:
+            raise ValueError("bi_gemm(add=True) needs an fp32 C")
+        cdt = BI_F32_ADD
     _chk("bi_gemm", lib.bi_gemm(_ptr(A), A.stride(0), _ptr(W), W.stride(0), _ptr(C), C.stride(0),
                                 cdt, M, N, K, _stream(stream)))
 
 
-def bi_gemm_x2(A_hi, A_lo, W, C, stream=None) -> None:
+def bi_gemm_swiglu(A, W, out, stream=None) -> None:
+    """out = swiglu(A Wg^T, A Wu^T). A [M, K] bf16, W [2F, K] bf16 (gate rows,
+    then up rows), out [M, F] bf16."""
+    M, K = A.shape
+    F = out.shape[1]
+    if W.shape[0] != 2 * F:
+        raise ValueError("bi_gemm_swiglu: W must have 2F rows")
+    _chk("bi_gemm_swiglu", lib.bi_gemm_swiglu(_ptr(A), A.stride(0), _ptr(W), W.stride(0), _ptr(out),
+                                              out.stride(0), M, F, K, _stream(stream)))
+
+
+def bi_gemm_x2(A_hi, A_lo, W, C, stream=None, add: bool = False) -> None:
     """C = (A_hi + A_lo) W^T (an fp32 activation carried as a bf16 pair)."""
     M, K = A_hi.shape
     N = W.shape[0]
     cdt = BI_F32 if C.dtype == torch.float32 else BI_BF16
+    if add:
+        if cdt != BI_F32:
+            raise ValueError("bi_gemm_x2(add=True) needs an fp32 C")
+        cdt = BI_F32_ADD
     _chk("bi_gemm_x2", lib.bi_gemm_x2(_ptr(A_hi), _ptr(A_lo), A_hi.stride(0), _ptr(W), W.stride(0),
                                       _ptr(C), C.stride(0), cdt, M, N, K, _stream(stream)))
 

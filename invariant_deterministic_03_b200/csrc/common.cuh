@@ -32,6 +32,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// SwiGLU of one feature from bf16 gate and up values (passed as floats):
+// silu(g) * u = g / (1 + e^-g) * u in fp32, each step rounded to nearest.
+// The caller rounds the result to bf16. Shared by the pointwise kernel and
+// the GEMM epilogue, so both produce the same bits.
+__device__ __forceinline__ float swiglu_f32(float g, float u) {
+  const float silu = __fdiv_rn(g, __fadd_rn(1.0f, expf(-g)));
+  return __fmul_rn(silu, u);
+}
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

@@ -30,7 +30,6 @@ bi_status launch_embed(const int32_t* tok, int64_t n_tok, const bf16* table, int
                        int64_t D, float* out, cudaStream_t s);
 bi_status launch_rope(bf16* x, int64_t ldx, int n_heads, const int32_t* pos, int64_t n_tok,
                       const float* cs, int max_pos, cudaStream_t s);
-bi_status launch_swiglu(const bf16* gu, int64_t n_tok, int64_t F, bf16* out, cudaStream_t s);
 bi_status launch_argmax(const float* logits, int64_t rows, int64_t V, int64_t ld, int32_t* idx,
                         cudaStream_t s);
 bi_status launch_split(const float* x, int64_t n, bf16* hi, bf16* lo, cudaStream_t s);
@@ -49,11 +48,6 @@ size_t attn_f32_workspace(int64_t n_tok, int Hq, int max_kv_len);
 
 namespace fwd {
 
-__global__ void add_f32_kernel(float* __restrict__ x, const float* __restrict__ d, int64_t n) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) x[i] = __fadd_rn(x[i], d[i]);
-}
-
 __global__ void gather_rows_kernel(const float* __restrict__ x, const int32_t* __restrict__ rows,
                                    int64_t n_rows, int64_t n_tok, int D, float* __restrict__ out,
                                    int32_t* status) {
@@ -66,7 +60,7 @@ __global__ void gather_rows_kernel(const float* __restrict__ x, const int32_t* _
 }
 
 struct Layout {  // workspace carve-up, all offsets 256-byte aligned
-  size_t x, h, h_lo, qkv, qkv32, att, att_lo, att32, t32, gu, gu32, act, act_lo, xl, hl, hl_lo,
+  size_t x, h, h_lo, qkv, qkv32, att, att_lo, att32, gu32, act, act_lo, xl, hl, hl_lo,
       rope, attn_ws, total;
   size_t attn_ws_bytes;
 };
@@ -87,8 +81,6 @@ static Layout layout(const bi_model_config& c, int64_t T, int64_t NL, int32_t ma
   L.att = o; o += up(T * D * 2);
   L.att_lo = o; o += f32 ? up(T * D * 2) : 0;
   L.att32 = o; o += f32 ? up(T * D * 4) : 0;
-  L.t32 = o; o += up(T * D * 4);
-  L.gu = o; o += up(T * 2 * F * 2);
   L.gu32 = o; o += c.precision == BI_PREC_F32 ? up(T * 2 * F * 4) : 0;
   L.act = o; o += up(T * F * 2);
   L.act_lo = o; o += c.precision == BI_PREC_F32 ? up(T * F * 2) : 0;
@@ -194,8 +186,6 @@ extern "C" bi_status bi_forward(const bi_model* m, const bi_batch* bt, void* k_c
   bf16* att = reinterpret_cast<bf16*>(base + L.att);
   bf16* att_lo = reinterpret_cast<bf16*>(base + L.att_lo);
   float* att32 = reinterpret_cast<float*>(base + L.att32);
-  float* t32 = reinterpret_cast<float*>(base + L.t32);
-  bf16* gu = reinterpret_cast<bf16*>(base + L.gu);
   float* gu32 = reinterpret_cast<float*>(base + L.gu32);
   bf16* act = reinterpret_cast<bf16*>(base + L.act);
   bf16* act_lo = reinterpret_cast<bf16*>(base + L.act_lo);
@@ -225,7 +215,6 @@ extern "C" bi_status bi_forward(const bi_model* m, const bi_batch* bt, void* k_c
   sh.max_kv_len = b.max_kv_len;
   sh.scale = (float)(1.0 / sqrt((double)BI_HEAD_DIM));
 
-  const int64_t add_blocks = (T * D + 255) / 256;
   for (int l = 0; l < c.n_layers; ++l) {
     const bf16* attn_norm = static_cast<const bf16*>(m->w.attn_norm) + (size_t)l * D;
     const bf16* mlp_norm = static_cast<const bf16*>(m->w.mlp_norm) + (size_t)l * D;
@@ -248,37 +237,40 @@ extern "C" bi_status bi_forward(const bi_model* m, const bi_batch* bt, void* k_c
       BI_TRY(run_attn_f32(qkv32, QKV, b.cu_q, T, kc, vc, b.block_table, b.seq_lens, b.B, &sh, att32,
                           D, attn_ws, L.attn_ws_bytes, s));
       BI_TRY(launch_split(att32, T * D, att, att_lo, s));
-      BI_TRY(bi_gemm_x2(att, att_lo, D, w_o, D, t32, D, BI_F32, T, D, D, stream));
+      BI_TRY(bi_gemm_x2(att, att_lo, D, w_o, D, x, D, BI_F32_ADD, T, D, D, stream));  // x += O proj
     } else {
       bf16* kc = static_cast<bf16*>(k_cache) + (size_t)l * cache_layer;
       bf16* vc = static_cast<bf16*>(v_cache) + (size_t)l * cache_layer;
       BI_TRY(bi_rmsnorm_f32in(x, attn_norm, h, T, D, c.rms_eps, stream));
       BI_TRY(bi_gemm(h, D, w_qkv, D, qkv, QKV, BI_BF16, T, QKV, D, stream));
-      BI_TRY(launch_rope(qkv, QKV, Hq, b.positions, T, rope, c.max_pos, s));
-      BI_TRY(launch_rope(qkv + (size_t)Hq * BI_HEAD_DIM, QKV, Hkv, b.positions, T, rope, c.max_pos, s));
+      // q and k heads are adjacent in a qkv row: one launch rotates both
+      BI_TRY(launch_rope(qkv, QKV, Hq + Hkv, b.positions, T, rope, c.max_pos, s));
       BI_TRY(launch_kv_append(qkv + (size_t)Hq * BI_HEAD_DIM, qkv + (size_t)(Hq + Hkv) * BI_HEAD_DIM,
                               QKV, b.slot_mapping, T, kc, vc, Hkv, num_pages, s));
-      BI_TRY(bi_attn_prefill(qkv, QKV, b.cu_q, b.max_q_len, T, kc, vc, b.block_table, b.seq_lens,
-                             b.B, &sh, att, D, attn_ws, L.attn_ws_bytes, stream));
-      BI_TRY(bi_gemm(att, D, w_o, D, t32, D, BI_F32, T, D, D, stream));
+      if (T == b.B && b.max_q_len == 1) {
+        // every chunk is one token: the decode kernel, whose rows are the
+        // same bits as the prefill kernel's (same tiles, splits and per-row
+        // arithmetic)
+        BI_TRY(bi_attn_decode(qkv, QKV, kc, vc, b.block_table, b.seq_lens, b.B, &sh, att, D, attn_ws,
+                              L.attn_ws_bytes, stream));
+      } else {
+        BI_TRY(bi_attn_prefill(qkv, QKV, b.cu_q, b.max_q_len, T, kc, vc, b.block_table, b.seq_lens,
+                               b.B, &sh, att, D, attn_ws, L.attn_ws_bytes, stream));
+      }
+      BI_TRY(bi_gemm(att, D, w_o, D, x, D, BI_F32_ADD, T, D, D, stream));  // x += O proj
     }
-    fwd::add_f32_kernel<<<(unsigned)add_blocks, 256, 0, s>>>(x, t32, T * D);
-    BI_CHECK_LAUNCH("forward residual");
 
     // ---- MLP block
     if (mlp_f32) {
       BI_TRY(bi_rmsnorm_split(x, mlp_norm, h, h_lo, T, D, c.rms_eps, stream));
       BI_TRY(bi_gemm_x2(h, h_lo, D, w_gu, D, gu32, 2 * F, BI_F32, T, 2 * F, D, stream));
       BI_TRY(launch_swiglu_split(gu32, T, F, act, act_lo, s));
-      BI_TRY(bi_gemm_x2(act, act_lo, F, w_d, F, t32, D, BI_F32, T, D, F, stream));
+      BI_TRY(bi_gemm_x2(act, act_lo, F, w_d, F, x, D, BI_F32_ADD, T, D, F, stream));  // x += down proj
     } else {
       BI_TRY(bi_rmsnorm_f32in(x, mlp_norm, h, T, D, c.rms_eps, stream));
-      BI_TRY(bi_gemm(h, D, w_gu, D, gu, 2 * F, BI_BF16, T, 2 * F, D, stream));
-      BI_TRY(launch_swiglu(gu, T, F, act, s));
-      BI_TRY(bi_gemm(act, F, w_d, F, t32, D, BI_F32, T, D, F, stream));
+      BI_TRY(bi_gemm_swiglu(h, D, w_gu, D, act, F, T, F, D, stream));  // act = swiglu(gate, up)
+      BI_TRY(bi_gemm(act, F, w_d, F, x, D, BI_F32_ADD, T, D, F, stream));  // x += down proj
     }
-    fwd::add_f32_kernel<<<(unsigned)add_blocks, 256, 0, s>>>(x, t32, T * D);
-    BI_CHECK_LAUNCH("forward residual");
   }
   if (b.n_logits == 0) return BI_OK;
   fwd::gather_rows_kernel<<<(unsigned)b.n_logits, 256, 0, s>>>(x, b.logits_rows, b.n_logits, T,

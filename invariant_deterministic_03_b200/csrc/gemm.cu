@@ -103,7 +103,64 @@ __device__ __forceinline__ void store_row_chunk(const Params& p, int row, int co
   }
 }
 
-template <int TERMS>
+// C[row, col0 .. col0+31] (fp32) += the accumulator chunk, one fp32
+// addition per element.
+__device__ __forceinline__ void add_row_chunk(const Params& p, int row, int col0, const uint32_t (&r)[32]) {
+  float* dst = static_cast<float*>(p.C) + (size_t)row * p.ldc + col0;
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    if (col0 + g * 8 < p.N) {
+      float4 a = *reinterpret_cast<const float4*>(dst + 8 * g);
+      float4 b = *reinterpret_cast<const float4*>(dst + 8 * g + 4);
+      a.x = __fadd_rn(a.x, __uint_as_float(r[8 * g + 0]));
+      a.y = __fadd_rn(a.y, __uint_as_float(r[8 * g + 1]));
+      a.z = __fadd_rn(a.z, __uint_as_float(r[8 * g + 2]));
+      a.w = __fadd_rn(a.w, __uint_as_float(r[8 * g + 3]));
+      b.x = __fadd_rn(b.x, __uint_as_float(r[8 * g + 4]));
+      b.y = __fadd_rn(b.y, __uint_as_float(r[8 * g + 5]));
+      b.z = __fadd_rn(b.z, __uint_as_float(r[8 * g + 6]));
+      b.w = __fadd_rn(b.w, __uint_as_float(r[8 * g + 7]));
+      *reinterpret_cast<float4*>(dst + 8 * g) = a;
+      *reinterpret_cast<float4*>(dst + 8 * g + 4) = b;
+    }
+  }
+}
+
+__device__ __forceinline__ float round_bf16(uint32_t acc) {
+  return __bfloat162float(__float2bfloat16_rn(__uint_as_float(acc)));
+}
+
+// out[row, f0 .. f0+31] = bf16(swiglu(bf16(gate), bf16(up))); F % 8 == 0.
+__device__ __forceinline__ void store_swiglu_chunk(const Params& p, int row, int f0, const uint32_t (&g)[32],
+                                                   const uint32_t (&u)[32]) {
+  bf16* dst = static_cast<bf16*>(p.C) + (size_t)row * p.ldc + f0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (f0 + q * 8 < p.N) {
+      float v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[k] = swiglu_f32(round_bf16(g[8 * q + k]), round_bf16(u[8 * q + k]));
+      uint4 o;
+      o.x = pack_bf16x2(v[0], v[1]);
+      o.y = pack_bf16x2(v[2], v[3]);
+      o.z = pack_bf16x2(v[4], v[5]);
+      o.w = pack_bf16x2(v[6], v[7]);
+      *reinterpret_cast<uint4*>(dst + 8 * q) = o;
+    }
+  }
+}
+
+// Epilogue of a tile (EPI):
+//   EPI_STORE   C = acc, rounded to bf16 (RNE) or kept fp32;
+//   EPI_ADD     C (fp32) = C + acc: one fp32 addition per element after the
+//               whole K reduction (a residual connection in the stream);
+//   EPI_SWIGLU  the tile's 256 accumulator columns are 128 gate features
+//               (W rows f) and the same 128 up features (W rows F + f):
+//               C[m, f] = bf16(swiglu_f32(bf16(g), bf16(u))), the same
+//               rounding points as a bf16 GEMM followed by bi_swiglu.
+constexpr int EPI_STORE = 0, EPI_ADD = 1, EPI_SWIGLU = 2;
+
+template <int TERMS, int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmA2,
@@ -164,15 +221,27 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int mb = tile % p.m_blocks, nb = tile / p.m_blocks;
         const int pf = p.w_prefetch;
-        for (int kb = 0; kb < pf && kb < p.k_blocks; ++kb) tma_prefetch_2d(&tmB, kb * BK, nb * BN);
+        // W rows of this tile: 256 from nb * 256, or (SwiGLU) 128 gate rows
+        // from nb * 128 and the matching 128 up rows from F + nb * 128
+        const int w_row0 = EPI == EPI_SWIGLU ? nb * (BN / 2) : nb * BN;
+        const int w_row1 = p.N + nb * (BN / 2);
+        for (int kb = 0; kb < pf && kb < p.k_blocks; ++kb) {
+          tma_prefetch_2d(&tmB, kb * BK, w_row0);
+          if (EPI == EPI_SWIGLU) tma_prefetch_2d(&tmB, kb * BK, w_row1);
+        }
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, p.status, abort_flag)) { ok = false; break; }
-          if (pf && kb + pf < p.k_blocks) tma_prefetch_2d(&tmB, (kb + pf) * BK, nb * BN);
+          if (pf && kb + pf < p.k_blocks) {
+            tma_prefetch_2d(&tmB, (kb + pf) * BK, w_row0);
+            if (EPI == EPI_SWIGLU) tma_prefetch_2d(&tmB, (kb + pf) * BK, w_row1);
+          }
           uint8_t* sa = tiles + stage * STAGE_BYTES;
           mbar_arrive_expect_tx(&full[stage], tx_bytes);
           tma_load_2d(sa, &tmA, &full[stage], kb * BK, mb * BM);
           if (TERMS == 2) tma_load_2d(sa + A_BYTES, &tmA2, &full[stage], kb * BK, mb * BM);
-          tma_load_2d(sa + TERMS * A_BYTES, &tmB, &full[stage], kb * BK, nb * BN);
+          tma_load_2d(sa + TERMS * A_BYTES, &tmB, &full[stage], kb * BK, w_row0);
+          if (EPI == EPI_SWIGLU)
+            tma_load_2d(sa + TERMS * A_BYTES + B_BYTES / 2, &tmB, &full[stage], kb * BK, w_row1);
           ++fills[stage];
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
@@ -238,14 +307,30 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       const int row = mb * BM + quarter * 32 + lane;
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+      if constexpr (EPI == EPI_SWIGLU) {
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        const int col0 = nb * BN + c * 32;
-        if (col0 >= p.N) break;  // uniform across the warp
-        uint32_t r[32];
-        tmem_ld32(taddr + c * 32, r);
-        tmem_ld_wait();
-        if (row < p.M) store_row_chunk(p, row, col0, r);
+        for (int c = 0; c < BN / 64; ++c) {
+          const int f0 = nb * (BN / 2) + c * 32;
+          if (f0 >= p.N) break;  // uniform across the warp
+          uint32_t g[32], u[32];
+          tmem_ld32(taddr + c * 32, g);
+          tmem_ld32(taddr + BN / 2 + c * 32, u);
+          tmem_ld_wait();
+          if (row < p.M) store_swiglu_chunk(p, row, f0, g, u);
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          const int col0 = nb * BN + c * 32;
+          if (col0 >= p.N) break;  // uniform across the warp
+          uint32_t r[32];
+          tmem_ld32(taddr + c * 32, r);
+          tmem_ld_wait();
+          if (row < p.M) {
+            if constexpr (EPI == EPI_ADD) add_row_chunk(p, row, col0, r);
+            else store_row_chunk(p, row, col0, r);
+          }
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -285,7 +370,8 @@ static bi_status check_args(const void* A, int64_t lda, const void* W, int64_t l
                             int64_t ldc, int32_t c_dtype, int64_t M, int64_t N, int64_t K) {
   if (!A || !W || !C) return fail(BI_ERR_INVALID_ARG, "gemm: null pointer");
   if (M < 0 || N < 0 || K < 0) return fail(BI_ERR_INVALID_ARG, "gemm: negative size");
-  if (c_dtype != BI_BF16 && c_dtype != BI_F32) return fail(BI_ERR_INVALID_ARG, "gemm: bad c_dtype %d", c_dtype);
+  if (c_dtype != BI_BF16 && c_dtype != BI_F32 && c_dtype != BI_F32_ADD)
+    return fail(BI_ERR_INVALID_ARG, "gemm: bad c_dtype %d", c_dtype);
   if (M > (1ll << 30) || N > (1ll << 30) || K > (1ll << 30)) return fail(BI_ERR_SHAPE, "gemm: size above 2^30");
   if (K % 8 || N % 8) return fail(BI_ERR_SHAPE, "gemm: K (%lld) and N (%lld) must be multiples of 8", (long long)K, (long long)N);
   if (lda < K || ldw < K || ldc < N) return fail(BI_ERR_SHAPE, "gemm: leading dimension smaller than the row");
@@ -294,13 +380,16 @@ static bi_status check_args(const void* A, int64_t lda, const void* W, int64_t l
   return BI_OK;
 }
 
-template <int TERMS>
+// N is the output width: the W rows for EPI_STORE / EPI_ADD, the feature
+// count F (W has 2F rows) for EPI_SWIGLU.
+template <int TERMS, int EPI>
 static bi_status launch(const void* A, const void* A2, int64_t lda, const void* W, int64_t ldw,
                         void* C, int64_t ldc, int32_t c_dtype, int64_t M, int64_t N, int64_t K,
                         cudaStream_t s) {
   bi_status st;
-  const int32_t c_f32 = c_dtype == BI_F32;
+  const int32_t c_f32 = c_dtype != BI_BF16;
   if (K == 0) {
+    if (EPI == EPI_ADD) return BI_OK;  // C += 0
     zero_fill_kernel<<<296, 256, 0, s>>>(C, ldc, c_f32, (int32_t)M, (int32_t)N);
     BI_CHECK_LAUNCH("gemm zero fill");
     return BI_OK;
@@ -323,9 +412,9 @@ static bi_status launch(const void* A, const void* A2, int64_t lda, const void* 
     }
   }
   {
-    uint64_t dims[2] = {(uint64_t)K, (uint64_t)N};
+    uint64_t dims[2] = {(uint64_t)K, (uint64_t)(EPI == EPI_SWIGLU ? 2 * N : N)};
     uint64_t strides[1] = {(uint64_t)ldw * 2};
-    uint32_t box[2] = {BK, BN};
+    uint32_t box[2] = {BK, EPI == EPI_SWIGLU ? BN / 2 : BN};
     if ((st = encode_tmap(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(W), dims,
                           strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != BI_OK)
       return st;
@@ -338,14 +427,15 @@ static bi_status launch(const void* A, const void* A2, int64_t lda, const void* 
   p.N = (int32_t)N;
   p.K = (int32_t)K;
   p.m_blocks = (int32_t)((M + BM - 1) / BM);
-  p.n_blocks = (int32_t)((N + BN - 1) / BN);
+  const int64_t cols_per_tile = EPI == EPI_SWIGLU ? BN / 2 : BN;
+  p.n_blocks = (int32_t)((N + cols_per_tile - 1) / cols_per_tile);
   p.k_blocks = (int32_t)((K + BK - 1) / BK);
   p.status = status_word();
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (!attr_set[dev & 63]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tcgen05_kernel<TERMS>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_tcgen05_kernel<TERMS, EPI>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Cfg<TERMS>::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e, "gemm: smem attribute");
@@ -356,7 +446,7 @@ static bi_status launch(const void* A, const void* A2, int64_t lda, const void* 
   const int grid = (int)(tiles < sms ? tiles : sms);
   p.w_prefetch = tiles <= sms ? W_PREFETCH : 0;
   p.a_bytes = (uint32_t)(M < BM ? (M + 7) / 8 * 8 : BM) * BK * 2;
-  gemm_tcgen05_kernel<TERMS><<<grid, THREADS, Cfg<TERMS>::SMEM_BYTES, s>>>(tmA, tmA2, tmB, p);
+  gemm_tcgen05_kernel<TERMS, EPI><<<grid, THREADS, Cfg<TERMS>::SMEM_BYTES, s>>>(tmA, tmA2, tmB, p);
   BI_CHECK_LAUNCH("gemm launch");
   return BI_OK;
 }
@@ -370,8 +460,21 @@ extern "C" bi_status bi_gemm(const void* A, int64_t lda, const void* W, int64_t 
   bi_status st = gemm::check_args(A, lda, W, ldw, C, ldc, c_dtype, M, N, K);
   if (st != BI_OK || M == 0 || N == 0) return st;
   if ((st = require_sm100()) != BI_OK) return st;
-  return gemm::launch<1>(A, nullptr, lda, W, ldw, C, ldc, c_dtype, M, N, K,
-                         static_cast<cudaStream_t>(stream));
+  if (c_dtype == BI_F32_ADD)
+    return gemm::launch<1, gemm::EPI_ADD>(A, nullptr, lda, W, ldw, C, ldc, c_dtype, M, N, K,
+                                          static_cast<cudaStream_t>(stream));
+  return gemm::launch<1, gemm::EPI_STORE>(A, nullptr, lda, W, ldw, C, ldc, c_dtype, M, N, K,
+                                          static_cast<cudaStream_t>(stream));
+}
+
+extern "C" bi_status bi_gemm_swiglu(const void* A, int64_t lda, const void* W, int64_t ldw, void* out,
+                                    int64_t ldo, int64_t M, int64_t F, int64_t K, void* stream) {
+  bi_status st = gemm::check_args(A, lda, W, ldw, out, ldo, BI_BF16, M, F, K);
+  if (st != BI_OK || M == 0 || F == 0) return st;
+  if (F > (1ll << 29)) return fail(BI_ERR_SHAPE, "gemm_swiglu: F above 2^29");
+  if ((st = require_sm100()) != BI_OK) return st;
+  return gemm::launch<1, gemm::EPI_SWIGLU>(A, nullptr, lda, W, ldw, out, ldo, BI_BF16, M, F, K,
+                                           static_cast<cudaStream_t>(stream));
 }
 
 extern "C" bi_status bi_gemm_x2(const void* A_hi, const void* A_lo, int64_t lda, const void* W,
@@ -383,6 +486,9 @@ extern "C" bi_status bi_gemm_x2(const void* A_hi, const void* A_lo, int64_t lda,
   if (!aligned16(A_lo)) return fail(BI_ERR_ALIGN, "gemm_x2: A_lo must be 16-byte aligned");
   if (M == 0 || N == 0) return BI_OK;
   if ((st = require_sm100()) != BI_OK) return st;
-  return gemm::launch<2>(A_hi, A_lo, lda, W, ldw, C, ldc, c_dtype, M, N, K,
-                         static_cast<cudaStream_t>(stream));
+  if (c_dtype == BI_F32_ADD)
+    return gemm::launch<2, gemm::EPI_ADD>(A_hi, A_lo, lda, W, ldw, C, ldc, c_dtype, M, N, K,
+                                          static_cast<cudaStream_t>(stream));
+  return gemm::launch<2, gemm::EPI_STORE>(A_hi, A_lo, lda, W, ldw, C, ldc, c_dtype, M, N, K,
+                                          static_cast<cudaStream_t>(stream));
 }

@@ -93,37 +93,87 @@ __global__ void rope_table_kernel(float* __restrict__ cs, int max_pos, double th
 }
 
 // ---- RoPE in place: one thread per (token, head, pair i < 64)
+// grid (token, head-pair block): each thread rotates 8 consecutive pairs
+// (i, i + 64), i = i0 .. i0+7, of one head with 16-byte accesses (rows
+// 16-byte aligned), or one pair (VEC == 1)
+template <int VEC>
 __global__ void rope_kernel(bf16* __restrict__ x, int64_t ldx, int n_heads,
-                            const int32_t* __restrict__ pos, int64_t n_tok,
-                            const float* __restrict__ cs, int max_pos, int32_t* status) {
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= n_tok * n_heads * 64) return;
-  const int i = (int)(idx % 64);
-  const int64_t th = idx / 64;
-  const int h = (int)(th % n_heads);
-  const int64_t t = th / n_heads;
+                            const int32_t* __restrict__ pos, const float* __restrict__ cs,
+                            int max_pos, int32_t* status) {
+  constexpr int PER_HEAD = 64 / VEC;
+  const int64_t t = blockIdx.x;
+  const int k = blockIdx.y * blockDim.x + threadIdx.x;
+  if (k >= n_heads * PER_HEAD) return;
+  const int h = k / PER_HEAD, i0 = (k % PER_HEAD) * VEC;
   const int p = pos[t];
-  bf16* row = x + t * ldx + (int64_t)h * BI_HEAD_DIM;
   if (p < 0 || p >= max_pos) {
-    if (i == 0) set_status(status, BI_DEV_BAD_TOKEN);
+    if (k == 0) set_status(status, BI_DEV_BAD_TOKEN);
     return;
   }
-  const float c = cs[((size_t)p * 64 + i) * 2], s = cs[((size_t)p * 64 + i) * 2 + 1];
-  const float a = __bfloat162float(row[i]), b = __bfloat162float(row[i + 64]);
-  row[i] = __float2bfloat16_rn(__fsub_rn(__fmul_rn(a, c), __fmul_rn(b, s)));
-  row[i + 64] = __float2bfloat16_rn(__fadd_rn(__fmul_rn(b, c), __fmul_rn(a, s)));
+  bf16* row = x + t * ldx + (int64_t)h * BI_HEAD_DIM;
+  const float* csp = cs + ((size_t)p * 64 + i0) * 2;
+  float a[VEC], b[VEC], c[VEC], sn[VEC];
+  if constexpr (VEC == 8) {
+    const uint4 av = *reinterpret_cast<const uint4*>(row + i0), bv = *reinterpret_cast<const uint4*>(row + i0 + 64);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      a[j] = __bfloat162float(reinterpret_cast<const bf16*>(&av)[j]);
+      b[j] = __bfloat162float(reinterpret_cast<const bf16*>(&bv)[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float4 q = reinterpret_cast<const float4*>(csp)[j];
+      c[2 * j] = q.x;
+      sn[2 * j] = q.y;
+      c[2 * j + 1] = q.z;
+      sn[2 * j + 1] = q.w;
+    }
+  } else {
+    a[0] = __bfloat162float(row[i0]);
+    b[0] = __bfloat162float(row[i0 + 64]);
+    c[0] = csp[0];
+    sn[0] = csp[1];
+  }
+  float ra[VEC], rb[VEC];
+#pragma unroll
+  for (int j = 0; j < VEC; ++j) {
+    ra[j] = __fsub_rn(__fmul_rn(a[j], c[j]), __fmul_rn(b[j], sn[j]));
+    rb[j] = __fadd_rn(__fmul_rn(b[j], c[j]), __fmul_rn(a[j], sn[j]));
+  }
+  if constexpr (VEC == 8) {
+    *reinterpret_cast<uint4*>(row + i0) = make_uint4(pack_bf16x2(ra[0], ra[1]), pack_bf16x2(ra[2], ra[3]),
+                                                     pack_bf16x2(ra[4], ra[5]), pack_bf16x2(ra[6], ra[7]));
+    *reinterpret_cast<uint4*>(row + i0 + 64) = make_uint4(pack_bf16x2(rb[0], rb[1]), pack_bf16x2(rb[2], rb[3]),
+                                                          pack_bf16x2(rb[4], rb[5]), pack_bf16x2(rb[6], rb[7]));
+  } else {
+    row[i0] = __float2bfloat16_rn(ra[0]);
+    row[i0 + 64] = __float2bfloat16_rn(rb[0]);
+  }
 }
 
 // ---- SwiGLU: out = bf16(silu(g) * u), silu(g) = g / (1 + exp(-g))
-__global__ void swiglu_kernel(const bf16* __restrict__ gu, int64_t n_tok, int64_t F,
-                              bf16* __restrict__ out) {
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= n_tok * F) return;
-  const int64_t t = idx / F, i = idx % F;
-  const float g = __bfloat162float(gu[t * 2 * F + i]);
-  const float u = __bfloat162float(gu[t * 2 * F + F + i]);
-  const float silu = __fdiv_rn(g, __fadd_rn(1.0f, expf(-g)));
-  out[idx] = __float2bfloat16_rn(__fmul_rn(silu, u));
+// grid (token, feature block); VEC features per thread: 8 with 16-byte
+// vector access (F % 8 == 0, aligned rows), else 1
+template <int VEC>
+__global__ void swiglu_kernel(const bf16* __restrict__ gu, int64_t F, bf16* __restrict__ out) {
+  const int64_t t = blockIdx.x;
+  const int64_t f = ((int64_t)blockIdx.y * blockDim.x + threadIdx.x) * VEC;
+  if (f >= F) return;
+  const bf16* g = gu + t * 2 * F + f;
+  const bf16* u = g + F;
+  bf16* o = out + t * F + f;
+  if constexpr (VEC == 8) {
+    const uint4 gv = *reinterpret_cast<const uint4*>(g), uv = *reinterpret_cast<const uint4*>(u);
+    const bf16* ge = reinterpret_cast<const bf16*>(&gv);
+    const bf16* ue = reinterpret_cast<const bf16*>(&uv);
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = swiglu_f32(__bfloat162float(ge[k]), __bfloat162float(ue[k]));
+    *reinterpret_cast<uint4*>(o) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                              pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+  } else {
+    o[0] = __float2bfloat16_rn(swiglu_f32(__bfloat162float(g[0]), __bfloat162float(u[0])));
+  }
 }
 
 // ---- residual add into the fp32 stream
@@ -190,16 +240,24 @@ bi_status launch_embed(const int32_t* tok, int64_t n_tok, const bf16* table, int
 
 bi_status launch_rope(bf16* x, int64_t ldx, int n_heads, const int32_t* pos, int64_t n_tok,
                       const float* cs, int max_pos, cudaStream_t s) {
-  const int64_t n = n_tok * n_heads * 64;
-  pw::rope_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(x, ldx, n_heads, pos, n_tok, cs,
-                                                              max_pos, status_word());
+  if (n_tok == 0) return BI_OK;
+  const bool vec = ldx % 8 == 0 && aligned16(x);
+  const int64_t per_tok = (int64_t)n_heads * (vec ? 8 : 64);
+  const dim3 grid((unsigned)n_tok, (unsigned)((per_tok + 255) / 256));
+  if (n_tok > 0x7fffffff || grid.y > 65535) return fail(BI_ERR_SHAPE, "rope: size out of range");
+  if (vec) pw::rope_kernel<8><<<grid, 256, 0, s>>>(x, ldx, n_heads, pos, cs, max_pos, status_word());
+  else pw::rope_kernel<1><<<grid, 256, 0, s>>>(x, ldx, n_heads, pos, cs, max_pos, status_word());
   BI_CHECK_LAUNCH("rope launch");
   return BI_OK;
 }
 
 bi_status launch_swiglu(const bf16* gu, int64_t n_tok, int64_t F, bf16* out, cudaStream_t s) {
-  const int64_t n = n_tok * F;
-  pw::swiglu_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(gu, n_tok, F, out);
+  const bool vec = F % 8 == 0 && aligned16(gu) && aligned16(out);
+  const int64_t per_tok = vec ? F / 8 : F;
+  const dim3 grid((unsigned)n_tok, (unsigned)((per_tok + 255) / 256));
+  if (n_tok > 0x7fffffff || grid.y > 65535) return fail(BI_ERR_SHAPE, "swiglu: size out of range");
+  if (vec) pw::swiglu_kernel<8><<<grid, 256, 0, s>>>(gu, F, out);
+  else pw::swiglu_kernel<1><<<grid, 256, 0, s>>>(gu, F, out);
   BI_CHECK_LAUNCH("swiglu launch");
   return BI_OK;
 }

@@ -120,3 +120,14 @@ def test_model_create_checks(bi):
     bi.lib.bi_model_destroy(h)
     bad = bi.ModelConfig(2, 4000, 32, 8, 14336, 32000, 4096, 1e-6, 1e4)
     assert bi.lib.bi_model_create(ctypes.byref(bad), ctypes.byref(w), ctypes.byref(h)) == bi.BI_ERR_SHAPE
+
+
+def test_gemm_epilogue_host_checks(bi):
+    p = 0x1000
+    g = bi.lib.bi_gemm
+    assert g(p, 64, p, 64, p, 64, bi.BI_F32_ADD, 4, 64, 60, None) == bi.BI_ERR_SHAPE   # K % 8
+    sw = bi.lib.bi_gemm_swiglu
+    assert sw(p, 64, p, 64, p, 60, 4, 60, 64, None) == bi.BI_ERR_SHAPE    # F % 8
+    assert sw(p, 64, p, 64, p, 8, 4, 16, 64, None) == bi.BI_ERR_SHAPE     # ldo < F
+    assert sw(None, 64, p, 64, p, 16, 4, 16, 64, None) == bi.BI_ERR_INVALID_ARG
+    assert sw(p, 64, p, 64, p, 16, 0, 16, 64, None) == bi.BI_OK           # M == 0: nothing to do
