@@ -11,9 +11,23 @@
 //   output tile 128 x 256, K stage 64, instruction tcgen05.mma.cta_group::1
 //   .kind::f16 M=128 N=256 K=16 with bf16 operands and an fp32 accumulator in
 //   tensor memory. Element (m, n) is accumulated by the K-steps k = 0, 16, 32,
-//   ... in that order, in one CTA, whatever M and N are. Which CTA computes a
-//   tile (persistent round-robin), how many rows an A copy carries and what
-//   is prefetched into L2 change timing only, never arithmetic.
+//   ... in that order, whatever M is. Which CTA computes a tile (persistent
+//   round-robin), how many rows an A copy carries and what is prefetched into
+//   L2 change timing only, never arithmetic.
+//
+// Fixed K split (a function of N and K only, never of M): when a weight has
+// few output tiles (N / 256 <= 37), so that small batches would leave most
+// SMs idle, and a long K (>= 8192, so that each half still keeps the tensor
+// cores busy long enough to hide the hand-over below), K is cut once, at
+// k-block ceil(k_blocks / 2). A cluster of two
+// CTAs computes each tile: rank r accumulates its half of K in order in its
+// own tensor memory; each rank finishes half of the tile's columns, taking
+// the other rank's fp32 partial for them through distributed shared memory
+// (32 columns at a time) and forming acc0 + acc1 (one fp32 addition per
+// element; the sum of two values does not depend on their order). Same split, same order, for every M ("Defeating
+// Nondeterminism in LLM Inference", section "Batch-invariant RMSNorm": one
+// reduction strategy with enough parallelism for small batches, used at
+// every batch size).
 //
 // CTA layout (192 threads, one CTA per SM, persistent over tiles):
 //   warp 0      TMA producer: A [128 x 64] and W [256 x 64] tiles, 128-byte
@@ -32,6 +46,8 @@
 //               the accumulator for the tile after next.
 // Every mbarrier wait is bounded (see common.cuh); a timeout sets a status
 // bit and the CTA winds down, releasing its tensor memory.
+#include <mutex>
+
 #include "common.cuh"
 #include "host.h"
 
@@ -47,6 +63,9 @@ constexpr uint32_t B_BYTES = BN * BK * 2;  // 32 KB
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int THREADS = 192;
 constexpr int W_PREFETCH = 8;  // W stages prefetched into L2 ahead of the loads (small M)
+constexpr int SPLIT_MAX_TILES_N = 37;       // weights with at most this many column tiles
+constexpr int SPLIT_MIN_K = 8192;           // and at least this K split K in two
+constexpr uint32_t XFER_SLOT = 128 * 32 * 4;  // one 32-column chunk of a 128-row fp32 accumulator
 
 // TERMS = number of bf16 A operands summed into the product: 1 for plain
 // bf16 activations, 2 for an activation carried as a hi/lo pair (A = A_hi +
@@ -56,7 +75,8 @@ template <int TERMS>
 struct Cfg {
   static constexpr int STAGES = TERMS == 1 ? 4 : 3;
   static constexpr uint32_t STAGE_BYTES = TERMS * A_BYTES + B_BYTES;
-  static constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 256;
+  static constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 2 * XFER_SLOT + 256;
+  static_assert(SMEM_BYTES <= 232448, "gemm: shared memory above the per-CTA limit");
 };
 
 struct Params {
@@ -66,6 +86,8 @@ struct Params {
   int32_t M, N, K;
   int32_t m_blocks, n_blocks, k_blocks;
   int32_t w_prefetch;  // W_PREFETCH or 0 (off)
+  int32_t split;       // CTAs (cluster ranks) per tile: 1, or 2 with K cut in two
+  int32_t kb_per_rank; // k-blocks of rank 0 (rank 1 takes the rest)
   uint32_t a_bytes;    // bytes of one A copy: 128 rows, or M rounded up to 8 when M < 128
   int32_t* status;
 };
@@ -173,16 +195,24 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* tiles = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* xfer = smem + STAGES * STAGE_BYTES;  // [2 slots] partial-accumulator chunks from the peer
+  uint64_t* full = reinterpret_cast<uint64_t*>(xfer + 2 * XFER_SLOT);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;   // [2]
   uint64_t* acc_empty = acc_full + 2;    // [2]
-  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* xfer_full = acc_empty + 2;   // [2] the peer's chunk is in my slot
+  uint64_t* xfer_free = xfer_full + 2;   // [2] the peer has read my chunk from its slot
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(xfer_free + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int num_tiles = p.m_blocks * p.n_blocks;
+  const int CL = p.split;
+  const uint32_t rank = CL > 1 ? cluster_rank() : 0u;
+  const int tile0 = (int)blockIdx.x / CL, tile_step = (int)gridDim.x / CL;
+  const int kb_lo = (int)rank * p.kb_per_rank;
+  const int kb_hi = min(p.k_blocks, kb_lo + p.kb_per_rank);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -191,7 +221,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4);  // one arrive per epilogue warp
+      mbar_init(&acc_empty[a], 4);    // one arrive per epilogue warp
+      mbar_init(&xfer_full[a], 128);  // every epilogue thread of the peer
+      mbar_init(&xfer_free[a], 128);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -207,6 +239,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if (CL > 1) cluster_sync();  // both ranks' barriers initialised before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_base_slot;
 
@@ -218,20 +251,20 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool ok = true;
       int fills[STAGES];
       for (int s = 0; s < STAGES; ++s) fills[s] = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int tile = tile0; tile < num_tiles && ok; tile += tile_step) {
         const int mb = tile % p.m_blocks, nb = tile / p.m_blocks;
         const int pf = p.w_prefetch;
         // W rows of this tile: 256 from nb * 256, or (SwiGLU) 128 gate rows
         // from nb * 128 and the matching 128 up rows from F + nb * 128
         const int w_row0 = EPI == EPI_SWIGLU ? nb * (BN / 2) : nb * BN;
         const int w_row1 = p.N + nb * (BN / 2);
-        for (int kb = 0; kb < pf && kb < p.k_blocks; ++kb) {
+        for (int kb = kb_lo; kb < kb_lo + pf && kb < kb_hi; ++kb) {
           tma_prefetch_2d(&tmB, kb * BK, w_row0);
           if (EPI == EPI_SWIGLU) tma_prefetch_2d(&tmB, kb * BK, w_row1);
         }
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        for (int kb = kb_lo; kb < kb_hi; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, p.status, abort_flag)) { ok = false; break; }
-          if (pf && kb + pf < p.k_blocks) {
+          if (pf && kb + pf < kb_hi) {
             tma_prefetch_2d(&tmB, (kb + pf) * BK, w_row0);
             if (EPI == EPI_SWIGLU) tma_prefetch_2d(&tmB, (kb + pf) * BK, w_row1);
           }
@@ -267,11 +300,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int tile = tile0; tile < num_tiles && ok; tile += tile_step) {
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, p.status, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        for (int kb = kb_lo; kb < kb_hi; ++kb) {
           if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(tiles + stage * STAGE_BYTES);
@@ -285,7 +318,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               // swizzle on the absolute address (tile bases are 1024-aligned).
               uint64_t ad = smem_desc(sa + term * A_BYTES + k * 32, 16, 1024, 2);
               uint64_t bd = smem_desc(sb + k * 32, 16, 1024, 2);
-              mma_bf16(d_tmem, ad, bd, idesc, (kb | term | k) != 0);
+              mma_bf16(d_tmem, ad, bd, idesc, (kb != kb_lo || term != 0 || k != 0));
             }
           }
           mma_commit(&empty[stage]);  // frees the stage once these MMAs retire
@@ -299,36 +332,112 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     // ---------------- epilogue warps 2..5: TMEM lanes 32*(warp%4) .. +31
     const int quarter = warp & 3;
+    const int trow = quarter * 32 + lane;  // accumulator row (TMEM lane) of this thread
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    int nx_out = 0, nx_in = 0;  // chunks sent to / received from the peer rank (slot n & 1)
+    bool ok = true;
+    for (int tile = tile0; tile < num_tiles && ok; tile += tile_step) {
       const int mb = tile % p.m_blocks, nb = tile / p.m_blocks;
       if (!mbar_wait(&acc_full[acc], acc_phase, p.status, abort_flag)) break;
       tc_fence_after();
-      const int row = mb * BM + quarter * 32 + lane;
+      const int row = mb * BM + trow;
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
-      if constexpr (EPI == EPI_SWIGLU) {
-#pragma unroll 1
-        for (int c = 0; c < BN / 64; ++c) {
-          const int f0 = nb * (BN / 2) + c * 32;
-          if (f0 >= p.N) break;  // uniform across the warp
-          uint32_t g[32], u[32];
-          tmem_ld32(taddr + c * 32, g);
-          tmem_ld32(taddr + BN / 2 + c * 32, u);
-          tmem_ld_wait();
-          if (row < p.M) store_swiglu_chunk(p, row, f0, g, u);
+      uint32_t held[32];  // SwiGLU: a gate chunk until its up chunk arrives
+      auto col_of = [&](int c) {
+        return EPI == EPI_SWIGLU ? nb * (BN / 2) + (c & 3) * 32 : nb * BN + c * 32;
+      };
+      // the epilogue of one finished 32-column chunk c (values in r)
+      auto finish = [&](int c, uint32_t (&r)[32]) {
+        if (row >= p.M) return;
+        if constexpr (EPI == EPI_SWIGLU) {
+          if (c >= 4) {
+            store_swiglu_chunk(p, row, col_of(c), held, r);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) held[i] = r[i];
+          }
+        } else if constexpr (EPI == EPI_ADD) {
+          add_row_chunk(p, row, col_of(c), r);
+        } else {
+          store_row_chunk(p, row, col_of(c), r);
         }
-      } else {
+      };
+      if (CL == 1) {
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          const int col0 = nb * BN + c * 32;
-          if (col0 >= p.N) break;  // uniform across the warp
+        for (int q = 0; q < BN / 32; ++q) {
+          // SwiGLU pairs gate chunk c with up chunk c + 4
+          const int c = EPI == EPI_SWIGLU ? ((q & 1) ? 4 + (q >> 1) : (q >> 1)) : q;
+          if (col_of(c) >= p.N) break;  // uniform across the warp
           uint32_t r[32];
           tmem_ld32(taddr + c * 32, r);
           tmem_ld_wait();
-          if (row < p.M) {
-            if constexpr (EPI == EPI_ADD) add_row_chunk(p, row, col0, r);
-            else store_row_chunk(p, row, col0, r);
+          finish(c, r);
+        }
+      } else {
+        // K split across the two ranks: rank r finishes half of the chunks
+        // (acc0 + acc1, one fp32 addition) and sends the other half to its
+        // partner. Chunks owned by rank r, in order: 0-3 / 4-7, or for SwiGLU
+        // gate/up pairs 0,4,1,5 / 2,6,3,7. Sends and receives alternate
+        // S S R S R S R R so that each direction keeps two chunks in flight
+        // in the partner's two slots and neither rank can block the other.
+        auto owned = [&](uint32_t rk, int i) {
+          return EPI == EPI_SWIGLU ? (int)rk * 2 + (i >> 1) + (i & 1) * 4 : (int)rk * 4 + i;
+        };
+        int own[4], oth[4], n_own = 0, n_oth = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int co = owned(rank, i), ct = owned(rank ^ 1u, i);
+          if (col_of(co) < p.N) own[n_own++] = co;  // live chunks: the same test on both ranks
+          if (col_of(ct) < p.N) oth[n_oth++] = ct;
+        }
+        const uint32_t peer = rank ^ 1u;
+        int is = 0, ir = 0;
+#pragma unroll 1
+        for (int step = 0; step < 8 && ok; ++step) {
+          const bool pref_send = step == 0 || step == 1 || step == 3 || step == 5;
+          const bool send = pref_send ? is < n_oth : !(ir < n_own);
+          if (send ? is >= n_oth : ir >= n_own) continue;
+          const int c = send ? oth[is++] : own[ir++];
+          uint32_t r[32];
+          tmem_ld32(taddr + c * 32, r);
+          tmem_ld_wait();
+          if (send) {
+            const int slot = nx_out & 1;  // a slot of the peer's staging area
+            if (!mbar_wait_cluster(&xfer_free[slot], (((uint32_t)nx_out >> 1) & 1u) ^ 1u, p.status,
+                                   abort_flag)) {
+              ok = false;
+              break;
+            }
+            if (row < p.M) {
+              const uint32_t dst = cluster_addr(xfer + slot * XFER_SLOT + trow * 128, peer);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)  // 16-byte units swizzled by row: no bank conflicts
+                st_cluster_v4(dst + ((uint32_t)(j ^ (trow & 7)) << 4), r[4 * j], r[4 * j + 1],
+                              r[4 * j + 2], r[4 * j + 3]);
+            }
+            mbar_arrive_cluster(cluster_addr(&xfer_full[slot], peer));
+            ++nx_out;
+          } else {
+            const int slot = nx_in & 1;
+            if (!mbar_wait_cluster(&xfer_full[slot], ((uint32_t)nx_in >> 1) & 1u, p.status, abort_flag)) {
+              ok = false;
+              break;
+            }
+            if (row < p.M) {
+              const uint8_t* src = xfer + slot * XFER_SLOT + trow * 128;
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const uint4 v = *reinterpret_cast<const uint4*>(src + ((j ^ (trow & 7)) << 4));
+                r[4 * j] = __float_as_uint(__fadd_rn(__uint_as_float(r[4 * j]), __uint_as_float(v.x)));
+                r[4 * j + 1] = __float_as_uint(__fadd_rn(__uint_as_float(r[4 * j + 1]), __uint_as_float(v.y)));
+                r[4 * j + 2] = __float_as_uint(__fadd_rn(__uint_as_float(r[4 * j + 2]), __uint_as_float(v.z)));
+                r[4 * j + 3] = __float_as_uint(__fadd_rn(__uint_as_float(r[4 * j + 3]), __uint_as_float(v.w)));
+              }
+            }
+            mbar_arrive_cluster(cluster_addr(&xfer_free[slot], peer));
+            ++nx_in;
+            finish(c, r);
           }
         }
       }
@@ -341,6 +450,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
+  // no rank leaves while the other may still write into, or arrive on, its
+  // shared memory
+  if (CL > 1) cluster_sync();
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
@@ -377,6 +489,57 @@ static bi_status check_args(const void* A, int64_t lda, const void* W, int64_t l
   if (lda < K || ldw < K || ldc < N) return fail(BI_ERR_SHAPE, "gemm: leading dimension smaller than the row");
   if (lda % 8 || ldw % 8 || ldc % 8) return fail(BI_ERR_ALIGN, "gemm: leading dimensions must be multiples of 8");
   if (!aligned16(A) || !aligned16(W) || !aligned16(C)) return fail(BI_ERR_ALIGN, "gemm: pointers must be 16-byte aligned");
+  return BI_OK;
+}
+
+template <int TERMS, int EPI>
+static bi_status set_smem_attr() {
+  static bool done[64] = {false};
+  static std::mutex mu;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (!done[dev & 63]) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tcgen05_kernel<TERMS, EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Cfg<TERMS>::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e, "gemm: smem attribute");
+    done[dev & 63] = true;
+  }
+  return BI_OK;
+}
+
+// How many two-CTA clusters of this kernel the device runs at once (queried
+// once per device).
+template <int TERMS, int EPI>
+static bi_status pair_clusters(int* out) {
+  static int cache[64] = {0};
+  static std::mutex mu;
+  bi_status st = set_smem_attr<TERMS, EPI>();
+  if (st != BI_OK) return st;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  int& v = cache[dev & 63];
+  if (v == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = Cfg<TERMS>::SMEM_BYTES;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    cudaError_t e = cudaOccupancyMaxActiveClusters(&n, gemm_tcgen05_kernel<TERMS, EPI>, &cfg);
+    if (e != cudaSuccess) return cuda_fail(e, "gemm: cluster occupancy");
+    if (n <= 0) return fail(BI_ERR_UNSUPPORTED, "gemm: no two-CTA cluster fits on this device");
+    v = n;
+  }
+  *out = v;
   return BI_OK;
 }
 
@@ -431,22 +594,36 @@ static bi_status launch(const void* A, const void* A2, int64_t lda, const void* 
   p.n_blocks = (int32_t)((N + cols_per_tile - 1) / cols_per_tile);
   p.k_blocks = (int32_t)((K + BK - 1) / BK);
   p.status = status_word();
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (!attr_set[dev & 63]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tcgen05_kernel<TERMS, EPI>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)Cfg<TERMS>::SMEM_BYTES);
-    if (e != cudaSuccess) return cuda_fail(e, "gemm: smem attribute");
-    attr_set[dev & 63] = true;
-  }
+  if ((st = set_smem_attr<TERMS, EPI>()) != BI_OK) return st;
+  // the K split depends on the weight's shape only, never on M
+  p.split = (p.n_blocks <= SPLIT_MAX_TILES_N && K >= SPLIT_MIN_K) ? 2 : 1;
+  p.kb_per_rank = (p.k_blocks + p.split - 1) / p.split;
   const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
   const int sms = num_sms();
-  const int grid = (int)(tiles < sms ? tiles : sms);
-  p.w_prefetch = tiles <= sms ? W_PREFETCH : 0;
+  p.w_prefetch = tiles * p.split <= sms ? W_PREFETCH : 0;
   p.a_bytes = (uint32_t)(M < BM ? (M + 7) / 8 * 8 : BM) * BK * 2;
-  gemm_tcgen05_kernel<TERMS, EPI><<<grid, THREADS, Cfg<TERMS>::SMEM_BYTES, s>>>(tmA, tmA2, tmB, p);
+  if (p.split == 1) {
+    const int grid = (int)(tiles < sms ? tiles : sms);
+    gemm_tcgen05_kernel<TERMS, EPI><<<grid, THREADS, Cfg<TERMS>::SMEM_BYTES, s>>>(tmA, tmA2, tmB, p);
+  } else {
+    int fit = 0;
+    if ((st = pair_clusters<TERMS, EPI>(&fit)) != BI_OK) return st;
+    const int64_t clusters = tiles < fit ? tiles : fit;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)(2 * clusters));
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = Cfg<TERMS>::SMEM_BYTES;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tcgen05_kernel<TERMS, EPI>, tmA, tmA2, tmB, p);
+    if (e != cudaSuccess) return cuda_fail(e, "gemm: cluster launch");
+  }
   BI_CHECK_LAUNCH("gemm launch");
   return BI_OK;
 }

@@ -127,3 +127,18 @@ def test_linspace_batch_invariance_demo(bi):
     out2 = bi.gemm(a, W, torch.float32)[:1]
     assert (out1 - out2).abs().max().item() == 0.0
     assert same_bits(out1, out2)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 8, 8192), (5, 264, 8200), (130, 520, 8192), (300, 776, 9000),
+                                   (129, 4096, 14336)])
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+def test_split_k_shapes(bi, M, N, K, out):
+    """Weights with few column tiles and K >= 8192 take the fixed two-way K
+    split (cluster of two CTAs, halves combined acc0 + acc1): parity with the
+    oracle on ragged shapes, and the last row alone gives the same bits."""
+    A = synth.normal_bf16((M, K), 1.0, M * 17 + K)
+    W = synth.normal_bf16((N, K), 0.02, N * 19 + K)
+    dt = torch.bfloat16 if out == "bf16" else torch.float32
+    C = _parity(bi, A, W, dt, what=f"split-K gemm {M}x{N}x{K} {out}")
+    C1 = bi.gemm(dev(A[-1:]), dev(W), dt)
+    assert same_bits(C1[0], C[-1])

@@ -36,7 +36,8 @@ def _split(bi, x32):
     return hi, lo
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 8, 8), (130, 520, 200), (257, 1032, 4096), (64, 14336, 4096)])
+@pytest.mark.parametrize("M,N,K", [(1, 8, 8), (130, 520, 200), (257, 1032, 4096), (64, 14336, 4096),
+                                   (33, 4096, 14336)])  # the last takes the two-way K split
 def test_gemm_x2_parity(bi, M, N, K):
     g = torch.Generator().manual_seed(M + N + K)
     A = torch.randn(M, K, generator=g, dtype=torch.float64).float()
