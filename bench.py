@@ -41,7 +41,7 @@ COPIES = 3
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # dram__bytes_read.sum + dram__bytes_write.sum of one gemm_tcgen05_kernel<1>
 # launch at M=4096 K=4096 N=14336 (profiles/gemm_tcgen05_m4096_k4096_n14336.md)
-GEMM_TRAFFIC_BYTES = 155.250432e6 + 97.863936e6
+GEMM_TRAFFIC_BYTES = 155.398400e6 + 98.859008e6
 
 
 def parse():
@@ -53,7 +53,8 @@ def parse():
     ap.add_argument("--no-extras", action="store_true", help="skip attention/RMSNorm/cuBLAS legs")
     ap.add_argument("--study", default=None, choices=["precision"],
                     help="precision study: all-bf16 vs fp32 upcast vs bf16-MLP-only decoder")
-    ap.add_argument("--case", default=None, choices=["gemm", "gemm_m128", "attn", "rmsnorm", "forward"],
+    ap.add_argument("--case", default=None, choices=["gemm", "gemm_m128", "gemm_split", "attn", "rmsnorm",
+                                                     "forward"],
                     help="run 3 launches of one kernel on its workload and exit (for profilers)")
     return ap.parse_args()
 
@@ -494,11 +495,13 @@ def run_case(case):
         assert bi.bi_device_status(clear=True) == 0
         print("case forward: ok")
         return 0
-    if case in ("gemm", "gemm_m128"):
-        M = 4096 if case == "gemm" else 128
-        A = torch.randn(M, 4096, device="cuda", generator=g).to(torch.bfloat16)
-        W = (torch.randn(14336, 4096, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
-        C = torch.empty(M, 14336, dtype=torch.bfloat16, device="cuda")
+    if case in ("gemm", "gemm_m128", "gemm_split"):
+        # gemm_split: the K = 14336, N = 4096 weight, which takes the two-way K split
+        M = {"gemm": 4096, "gemm_m128": 128, "gemm_split": 2048}[case]
+        K, N = (14336, 4096) if case == "gemm_split" else (4096, 14336)
+        A = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
+        W = (torch.randn(N, K, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+        C = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
         fn = lambda: bi.bi_gemm(A, W, C)  # noqa: E731
     elif case == "attn":
         lens = synth.attention_lengths(32, 1, 8192, seed=0)
