@@ -44,7 +44,7 @@ constexpr int SPLIT = BI_ATTN_SPLIT;   // 512 keys
 constexpr int PAGE = BI_PAGE_SIZE;     // 16 keys
 constexpr int PAGES_PER_TILE = TILE / PAGE;
 constexpr uint32_t TILE_BYTES = 128 * 128 * 2;  // 32 KB: one K or V tile (128 keys x 128 d)
-constexpr int ITEM_RING = 32;                   // claimed work items in flight inside a CTA
+constexpr int ITEM_RING = 16;                   // claimed work items in flight inside a CTA
 constexpr int MAX_KV_BUF = 3;
 
 // Shared-memory layout. Prefill: Q (two buffers, one per work item in flight)
@@ -60,6 +60,7 @@ struct Lay {
   static constexpr int NK = DECODE ? 3 : 2;                 // K tile buffers
   static constexpr int NV = DECODE ? 3 : 2;                 // V tile buffers
   static constexpr int NP = DECODE ? 2 : 1;                 // P buffers
+  static constexpr int NS = DECODE ? 3 : 2;                 // S buffers in tensor memory
   static constexpr uint32_t HALF = DECODE ? 1024 : 16384;   // bytes between the 64-column halves of Q / P
   static constexpr uint32_t ROW_SBO = DECODE ? 0 : 1024;    // bytes between 8-row groups of Q / P
   static constexpr uint32_t QP_BYTES = 2 * HALF;            // one Q or P buffer
@@ -70,8 +71,8 @@ struct Lay {
   static constexpr uint32_t OFF_BAR = OFF_P + NP * QP_BYTES;
   static constexpr uint32_t OFF_RING = OFF_BAR + 256;   // producer's page-id ring [16 tiles][8 pages]
   static constexpr uint32_t OFF_RED = OFF_RING + 512;   // decode quarter exchange [2][4 warps][8 heads] fp32
-  static constexpr uint32_t OFF_ITEMS = OFF_RED + 256;  // item ring [32] int32, then one mbarrier per slot
-  static constexpr size_t SMEM_BYTES = 1024 + OFF_ITEMS + ITEM_RING * 4 + ITEM_RING * 8;
+  static constexpr uint32_t OFF_ITEMS = OFF_RED + 256;  // item ring [16] x 48 B, then one mbarrier per slot
+  static constexpr size_t SMEM_BYTES = 1024 + OFF_ITEMS + ITEM_RING * 48 + ITEM_RING * 8;
   static_assert(NK <= MAX_KV_BUF && NV <= MAX_KV_BUF, "barrier arrays hold 3 K and 3 V buffers");
   static_assert(OFF_Q % 1024 == 0 && OFF_P % 1024 == 0, "swizzled Q / P tiles need 1 KB alignment");
   static_assert(SMEM_BYTES <= 232448, "attention: shared memory above the 227 KB per-CTA limit");
@@ -79,9 +80,9 @@ struct Lay {
 // warps 0-3: one thread per MMA row (softmax, O rescale, partials)
 // warp 4: TMA producer; warp 5: TMEM allocator and MMA issuer
 constexpr int THREADS = 192;
-// tensor memory: S double buffer at columns [0,128) and [128,256), O at [256,384)
+// tensor memory: S buffers at columns [0,128), [128,256) and (decode) [256,384); O at [384,512)
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TMEM_O = 256;
+constexpr uint32_t TMEM_O = 384;  // S buffers at [0,128), [128,256) (and in decode [256,384))
 
 struct Params {
   const uint8_t* kc;  // bf16 key cache, 4 KB per (page, kv head) block
@@ -103,6 +104,14 @@ struct Params {
 struct Item {
   int s, b, g, r0, nb, L, q_lo, q_hi, key_lo, t0, ntiles;
 };
+
+// An entry of the shared item ring: the claimed index (-1: no more work) and
+// its decoded coordinates, so that no role repeats the global loads of item_at.
+struct RingItem {
+  int32_t idx;
+  Item it;
+};
+static_assert(sizeof(RingItem) == 48, "item ring entry");
 
 // Work item idx -> its coordinates; false when it has nothing to do. The kv
 // head varies fastest and the split slowest, so the persistent CTAs first take
@@ -168,10 +177,16 @@ __device__ __forceinline__ const uint8_t* block_src(const uint8_t* cache, int32_
 // Work items are claimed at run time: the producer's look-ahead cursor takes
 // the next index from a global counter (atomicAdd -- scheduling only, no
 // value is ever reduced through it), skips items with no work, and publishes
-// each claimed item (or -1 at the end) in a shared ring with one mbarrier per
-// slot; every other role walks the ring in order. Which CTA runs an item
-// never reaches its arithmetic. The look-ahead is bounded by the K/V buffers
-// (a dozen items at most), far inside the 32-slot ring.
+// each claimed item, decoded (or -1 at the end), in a shared ring with one
+// mbarrier per slot; every other role walks the ring in order. Which CTA runs
+// an item never reaches its arithmetic. The look-ahead is bounded by the
+// buffers: the claiming cursor runs at most PF_AHEAD + 1 tiles ahead of the K
+// loads, which run at most NK tiles ahead of QK^T, which runs at most NS
+// tiles ahead of the softmax, and the V loads trail the softmax by at most
+// NP tiles -- 13 tiles (so at most 13 items) in decode, 11 in prefill,
+// inside the 16-slot ring.
+// (Claiming one index ahead, to hide the atomic's latency, was measured
+// slower: a CTA holding an item it has not started delays the tail.)
 __device__ __forceinline__ int claim_item(const Params& p, int lane, Item& it) {
   while (true) {
     int v = 0;
@@ -191,23 +206,32 @@ struct Cursor {
 
 // Advances to the next tile; on a new item, reads ring entry n (waiting for
 // its publication). Returns false only when a wait timed out.
-__device__ __forceinline__ bool cursor_next(const Params& p, Cursor& c, const int32_t* ring,
+// Ring entry n once published (waits for it): false when the wait timed out.
+__device__ __forceinline__ bool ring_read(const Params& p, const RingItem* ring, uint64_t* ibar, int n,
+                                          volatile int* abort_flag, int& idx, Item& it) {
+  const int slot = n & (ITEM_RING - 1);
+  if (!mbar_wait(&ibar[slot], ((uint32_t)n / ITEM_RING) & 1u, p.status, abort_flag)) return false;
+  const volatile int32_t* e = reinterpret_cast<const volatile int32_t*>(&ring[slot]);
+  idx = e[0];
+  int* dst = reinterpret_cast<int*>(&it);
+#pragma unroll
+  for (int i = 0; i < 11; ++i) dst[i] = e[1 + i];
+  return true;
+}
+
+__device__ __forceinline__ bool cursor_next(const Params& p, Cursor& c, const RingItem* ring,
                                             uint64_t* ibar, volatile int* abort_flag) {
   if (c.valid && ++c.t < c.it.ntiles) return true;
   c.valid = false;
   c.t = 0;
   ++c.n;
-  const int slot = c.n & (ITEM_RING - 1);
-  if (!mbar_wait(&ibar[slot], ((uint32_t)c.n / ITEM_RING) & 1u, p.status, abort_flag)) return false;
-  const int idx = reinterpret_cast<const volatile int32_t*>(ring)[slot];
-  if (idx >= 0) {
-    item_at(p, idx, c.it, false);
-    c.valid = true;
-  }
+  int idx;
+  if (!ring_read(p, ring, ibar, c.n, abort_flag, idx, c.it)) return false;
+  c.valid = idx >= 0;
   return true;
 }
 
-__device__ __forceinline__ bool cursor_start(const Params& p, Cursor& c, const int32_t* ring,
+__device__ __forceinline__ bool cursor_start(const Params& p, Cursor& c, const RingItem* ring,
                                              uint64_t* ibar, volatile int* abort_flag) {
   c.n = -1;
   c.t = 0;
@@ -216,7 +240,7 @@ __device__ __forceinline__ bool cursor_start(const Params& p, Cursor& c, const i
 }
 
 // The producer's look-ahead cursor: claims and publishes items.
-__device__ __forceinline__ void claim_next(const Params& p, Cursor& c, int32_t* ring, uint64_t* ibar,
+__device__ __forceinline__ void claim_next(const Params& p, Cursor& c, RingItem* ring, uint64_t* ibar,
                                            int lane) {
   if (c.valid && ++c.t < c.it.ntiles) return;
   c.t = 0;
@@ -225,8 +249,12 @@ __device__ __forceinline__ void claim_next(const Params& p, Cursor& c, int32_t* 
   c.valid = idx >= 0;
   if (lane == 0) {
     const int slot = c.n & (ITEM_RING - 1);
-    reinterpret_cast<volatile int32_t*>(ring)[slot] = idx;
-    mbar_arrive(&ibar[slot]);
+    volatile int32_t* e = reinterpret_cast<volatile int32_t*>(&ring[slot]);
+    e[0] = idx;
+    const int* src = reinterpret_cast<const int*>(&c.it);
+#pragma unroll
+    for (int i = 0; i < 11; ++i) e[1 + i] = src[i];
+    mbar_arrive(&ibar[slot]);  // release: the entry is visible to whoever sees the phase
   }
 }
 
@@ -374,15 +402,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* k_empty = bars + 7;    // [NK]
   uint64_t* v_full = bars + 10;    // [NV]
   uint64_t* v_empty = bars + 13;   // [NV]
-  uint64_t* s_full = bars + 16;    // [2]
-  uint64_t* s_free = bars + 18;    // [2]
-  uint64_t* p_ready = bars + 20;   // [NP]
-  uint64_t* o_ready = bars + 22;   // [NP]: P V of the tile that read P buffer i is done
-  uint64_t* x_bar = bars + 24;     // decode: quarter exchange among the 4 softmax warps
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 25);
-  static_assert(26 * 8 <= 256, "barrier region");
-  int32_t* item_ring = reinterpret_cast<int32_t*>(smem + L::OFF_ITEMS);
-  uint64_t* item_bar = reinterpret_cast<uint64_t*>(smem + L::OFF_ITEMS + ITEM_RING * 4);
+  uint64_t* s_full = bars + 16;    // [NS]
+  uint64_t* s_free = bars + 19;    // [NS]
+  uint64_t* p_ready = bars + 22;   // [NP]
+  uint64_t* o_ready = bars + 24;   // [NP]: P V of the tile that read P buffer i is done
+  uint64_t* x_bar = bars + 26;     // decode: quarter exchange among the 4 softmax warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 27);
+  static_assert(28 * 8 <= 256, "barrier region");
+  RingItem* item_ring = reinterpret_cast<RingItem*>(smem + L::OFF_ITEMS);
+  uint64_t* item_bar = reinterpret_cast<uint64_t*>(smem + L::OFF_ITEMS + ITEM_RING * 48);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -392,6 +420,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
+    }
+    for (int i = 0; i < L::NS; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 128);
     }
@@ -547,11 +577,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       long long t_last = clock64();
       while ((sc.valid || nP < nS) && ok) {
         bool progressed = false;
-        if (sc.valid && nS - nP < 2) {
-          const int sb = nS & 1, kb = nS % NK, qb = qi & 1;
+        if (sc.valid && nS - nP < L::NS) {
+          const int sb = nS % L::NS, kb = nS % NK, qb = qi & 1;
           const bool ready = (sc.t != 0 || mbar_test(&q_full[qb], ((uint32_t)qi >> 1) & 1u)) &&
                              mbar_test(&k_full[kb], ((uint32_t)nS / NK) & 1u) &&
-                             mbar_test(&s_free[sb], (((uint32_t)nS >> 1) & 1u) ^ 1u);
+                             mbar_test(&s_free[sb], (((uint32_t)nS / L::NS) & 1u) ^ 1u);
           if (ready) {
             tc_fence_after();
             issue_s<DECODE>(tmem + sb * 128, sQ0 + qb * L::QP_BYTES, sK0 + kb * TILE_BYTES);
@@ -622,12 +652,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       return done;
     };
     for (int n = 0; ok; ++n) {
-      const int slot = n & (ITEM_RING - 1);
-      if (!mbar_wait(&item_bar[slot], ((uint32_t)n / ITEM_RING) & 1u, p.status, abort_flag)) break;
-      const int idx = reinterpret_cast<const volatile int32_t*>(item_ring)[slot];
-      if (idx < 0) break;
+      int idx;
       Item it;
-      item_at(p, idx, it, false);
+      if (!ring_read(p, item_ring, item_bar, n, abort_flag, idx, it)) break;
+      if (idx < 0) break;
       const int q_idx = it.q_lo + qr;
       const int pos = it.L - it.nb + q_idx;
       const bool row_valid = (decode ? lane < p.G : true) && (q_idx < it.q_hi) && (pos >= it.key_lo);
@@ -636,11 +664,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int tail = it.L % PAGE;
       float m = -INFINITY, l = 0.0f;
       for (int t = 0; t < it.ntiles; ++t, ++j) {
-        const int sb = j & 1;
+        const int sb = j % L::NS;
         const int kb0 = (it.t0 + t) * TILE;
         const bool need = row_valid && kb0 <= pos;
         const int nvalid = need ? min(TILE, pos + 1 - kb0) : 0;
-        if (!mbar_wait(&s_full[sb], ((uint32_t)j >> 1) & 1u, p.status, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&s_full[sb], ((uint32_t)j / L::NS) & 1u, p.status, abort_flag)) { ok = false; break; }
         tc_fence_after();
         float alpha = 1.0f, m_new = 0.0f;
         if constexpr (decode) {
