@@ -27,6 +27,7 @@ class PagedKV:
         self.free = synth.permutation(num_pages, seed).tolist()
         self.pages: dict[int, list[int]] = {}
         self.length: dict[int, int] = {}
+        self.refs: dict[int, int] = {}  # page id -> number of sequences whose table holds it
 
     def ensure(self, seq: int, length: int) -> None:
         pg = self.pages.setdefault(seq, [])
@@ -36,14 +37,39 @@ class PagedKV:
                 raise RuntimeError("KV cache out of pages")
             if len(pg) >= self.max_pages:
                 raise RuntimeError("sequence longer than max_pages_per_seq pages")
-            pg.append(self.free.pop(0))
+            page = self.free.pop(0)
+            self.refs[page] = 1
+            pg.append(page)
 
     def slot(self, seq: int, pos: int) -> int:
         return self.pages[seq][pos // PAGE] * PAGE + pos % PAGE
 
     def release(self, seq: int) -> None:
-        self.free.extend(self.pages.pop(seq, []))
+        for page in self.pages.pop(seq, []):
+            self.refs[page] -= 1
+            if self.refs[page] == 0:
+                del self.refs[page]
+                self.free.append(page)
         self.length.pop(seq, None)
+
+    def fork(self, src: int, dst: int, n_tokens: int) -> int:
+        """Prefix reuse: `dst` starts with the cached keys of the first
+        n_tokens of `src`, by sharing src's whole pages (the same page ids in
+        both block tables; nothing is copied). A partly filled last page is
+        not shared -- `dst` recomputes those tokens into pages of its own, so
+        no sequence ever writes into a page another one reads. Returns the
+        number of tokens `dst` now holds (n_tokens rounded down to a page).
+        Attention walks tiles and splits at absolute key offsets, so `dst`'s
+        outputs are the same bits as if it had computed the prefix itself."""
+        if dst in self.pages:
+            raise ValueError(f"sequence {dst} already exists")
+        n_tokens = min(n_tokens, self.length.get(src, 0))
+        shared = self.pages[src][: n_tokens // PAGE]
+        for page in shared:
+            self.refs[page] += 1
+        self.pages[dst] = list(shared)
+        self.length[dst] = len(shared) * PAGE
+        return self.length[dst]
 
 
 def make_batch(kv: PagedKV, chunks, tokens_of, device="cuda:0"):

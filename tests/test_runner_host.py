@@ -1,0 +1,55 @@
+"""Host bookkeeping of the forward's paged KV cache (no GPU): page
+allocation, prefix sharing between sequences and reference-counted release,
+and the batch assembly's slot arithmetic."""
+import pytest
+
+from invariant_deterministic_03_b200 import runner
+
+
+def _kv(num_pages=32):
+    return runner.PagedKV(n_layers=1, num_pages=num_pages, n_kv_heads=1, max_pages_per_seq=16, seed=3,
+                          device="cpu")
+
+
+def test_pages_come_from_a_seeded_permutation():
+    a, b = _kv(), _kv()
+    a.ensure(0, 40)
+    b.ensure(0, 40)
+    assert a.pages[0] == b.pages[0] and len(a.pages[0]) == 3
+    assert len(set(a.pages[0])) == 3
+    assert a.slot(0, 17) == a.pages[0][1] * 16 + 1
+
+
+def test_fork_shares_whole_pages_only():
+    kv = _kv()
+    kv.ensure(0, 50)
+    kv.length[0] = 50
+    held = kv.fork(0, 1, 45)                      # 45 tokens: two whole pages
+    assert held == 32
+    assert kv.pages[1] == kv.pages[0][:2]
+    assert kv.length[1] == 32
+    assert all(kv.refs[p] == 2 for p in kv.pages[0][:2]) and kv.refs[kv.pages[0][2]] == 1
+    kv.ensure(1, 40)                              # the fork's own tail page
+    assert kv.pages[1][2] not in kv.pages[0]
+    # never more than the source holds
+    assert kv.fork(0, 2, 1000) == 48
+    with pytest.raises(ValueError):
+        kv.fork(0, 1, 16)
+
+
+def test_release_frees_a_page_when_its_last_holder_goes():
+    kv = _kv()
+    kv.ensure(0, 64)
+    kv.length[0] = 64
+    kv.fork(0, 1, 64)
+    n_free = len(kv.free)
+    kv.release(0)
+    assert len(kv.free) == n_free                 # all four pages still held by sequence 1
+    kv.release(1)
+    assert len(kv.free) == n_free + 4 and not kv.refs
+
+
+def test_out_of_pages_is_an_error():
+    kv = _kv(num_pages=2)
+    with pytest.raises(RuntimeError):
+        kv.ensure(0, 33)
