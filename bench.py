@@ -39,7 +39,7 @@ SHAPES = [(4096, 14336), (14336, 4096)]          # (K, N)
 MS = [1 << i for i in range(13)]                 # 1 .. 4096
 COPIES = 3
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# dram__bytes_read.sum + dram__bytes_write.sum of one gemm_tcgen05_kernel<1>
+# dram__bytes_read.sum + dram__bytes_write.sum of one gemm_tcgen05_kernel<1, 0>
 # launch at M=4096 K=4096 N=14336 (profiles/gemm_tcgen05_m4096_k4096_n14336.md)
 GEMM_TRAFFIC_BYTES = 155.398400e6 + 98.859008e6
 
@@ -151,13 +151,21 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest x over all ranks (the slowest rank's time)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job rate of `world` replicas that each did flops_per_rank, over
+    the slowest rank's time ms."""
+    return flops_per_rank * world / (ms * 1e-3) / 1e12
 
 
 # --------------------------------------------------------------------------- workloads
@@ -622,7 +630,7 @@ def main():
     clocks = sampler.stop()
     ms_total = max_over_ranks(ms_total, world)
     ms_step = ms_total / args.steps
-    value = flops * world / (ms_step * 1e-3) / 1e12
+    value = whole_job_tflops(flops, world, ms_step)
 
     extras = {}
     table = sweep_table(torch, sw, reps=5)
@@ -636,7 +644,7 @@ def main():
     achieved = 2.0 * top["M"] * top["N"] * top["K"] / top["bi_ms"] / 1e9
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
                 "frac": achieved / peak_t, "traffic": GEMM_TRAFFIC_BYTES,
-                "kernel": "bi_gemm (gemm_tcgen05_kernel<1>), launch M=4096 K=4096 N=14336",
+                "kernel": "bi_gemm (gemm_tcgen05_kernel<1, 0>), launch M=4096 K=4096 N=14336",
                 "algorithmic_bytes": 2.0 * (top["M"] * top["K"] + top["N"] * top["K"] + top["M"] * top["N"]),
                 "peak_source": f"{peak_src} bf16 dense sustained",
                 "frac_of_burst": achieved / peaks.get("bf16_tflops", peak_t)}
@@ -676,10 +684,11 @@ def main():
                 "config": {"workload": "gemm sweep, Mistral-7B MLP shapes: M in {1,2,4,...,4096} x "
                                        "(K=4096,N=14336) and (K=14336,N=4096), bf16 in, fp32 accum, bf16 out",
                            "l2": "inputs larger than L2: weights rotate over 3 copies of 117 MB per shape",
-                           "tile": "128x256x64, tcgen05 M128 N256 K16, one tiling for all M",
+                           "tile": ("128x256x64, tcgen05 M128 N256 K16, one tiling for all M; K=14336 N=4096 "
+                                    "takes a fixed two-way K split (two-CTA cluster) at every M"),
                            "parallelism": f"replicas x{world}"},
                 "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
-                "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "e2e": {"value": whole_job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",
                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
                 "gpu_launches": launches}
         line.update(extras)
