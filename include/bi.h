@@ -81,6 +81,15 @@ const char* bi_last_error(void);
  * Returns BI_ERR_DEVICE_CHECK when the word was non-zero. */
 bi_status bi_device_status(int32_t* status, int32_t clear, void* stream);
 
+/* Self-check of the device wait bound (no counterpart on the pages; a test
+ * and diagnostic entry point). Launches one CTA whose threads wait on an
+ * mbarrier that nothing ever arrives on, through the same bounded wait the
+ * kernels use, giving up after `limit_cycles` SM clock cycles (1000 .. 2^32;
+ * the kernels use 2^32, about 2 s): the kernel then sets BI_DEV_WAIT_TIMEOUT
+ * in the status word and returns, leaving the context usable. Nothing faults,
+ * traps or hangs. BI_ERR_INVALID_ARG for a limit outside the range. */
+bi_status bi_check_wait_bound(int64_t limit_cycles, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* RMSNorm.  "Defeating Nondeterminism in LLM Inference", section
  * "Batch-invariant RMSNorm": the reference definition x * rsqrt(mean(x^2)) *

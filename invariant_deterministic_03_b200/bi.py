@@ -71,6 +71,7 @@ class Batch(ctypes.Structure):
 _SIGS = {
     "bi_last_error": (ctypes.c_char_p, []),
     "bi_device_status": (_i32, [ctypes.POINTER(_i32), _i32, _p]),
+    "bi_check_wait_bound": (_i32, [_i64, _p]),
     "bi_rmsnorm": (_i32, [_p, _p, _p, _i64, _i64, _f32, _p]),
     "bi_rmsnorm_f32in": (_i32, [_p, _p, _p, _i64, _i64, _f32, _p]),
     "bi_gemm": (_i32, [_p, _i64, _p, _i64, _p, _i64, _i32, _i64, _i64, _i64, _p]),
@@ -139,6 +140,11 @@ def bi_device_status(clear: bool = True, stream=None) -> int:
     if st not in (BI_OK, BI_ERR_DEVICE_CHECK):
         raise BIError("bi_device_status", st)
     return v.value
+
+
+def bi_check_wait_bound(limit_cycles: int, stream=None) -> None:
+    """Launches the wait-bound self-check (see include/bi.h)."""
+    _chk("bi_check_wait_bound", lib.bi_check_wait_bound(int(limit_cycles), _stream(stream)))
 
 
 def bi_rmsnorm(x, gamma, y, eps: float, stream=None) -> None:

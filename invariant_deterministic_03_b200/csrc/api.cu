@@ -6,6 +6,7 @@
 
 #include <mutex>
 
+#include "common.cuh"
 #include "host.h"
 
 namespace bi {
@@ -89,7 +90,41 @@ bi_status encode_tmap(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t rank
   return BI_OK;
 }
 
+// Self-check of the wait bound: thread 0 waits on an mbarrier that nothing
+// ever arrives on, through the same bounded wait every kernel uses, with a
+// short limit; it gives up, records BI_DEV_WAIT_TIMEOUT and raises the CTA's
+// abort flag, which releases the other threads' waits on the same barrier.
+__global__ void wait_bound_check_kernel(long long limit, int32_t* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  volatile int* ab = &abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_wait(&bar, 0, status, ab, limit);
+  } else {
+    mbar_wait(&bar, 0, status, ab, 2 * limit + 1000000);
+  }
+}
+
 }  // namespace bi
+
+extern "C" bi_status bi_check_wait_bound(int64_t limit_cycles, void* stream) {
+  if (limit_cycles < 1000 || limit_cycles > bi::kWaitLimitCycles)
+    return bi::fail(BI_ERR_INVALID_ARG, "check_wait_bound: limit %lld outside [1000, 2^32] cycles",
+                    (long long)limit_cycles);
+  bi_status st = bi::require_sm100();
+  if (st != BI_OK) return st;
+  bi::wait_bound_check_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(limit_cycles,
+                                                                              bi::status_word());
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return bi::cuda_fail(e, "check_wait_bound launch");
+  return BI_OK;
+}
 
 extern "C" const char* bi_last_error(void) { return bi::t_err; }
 

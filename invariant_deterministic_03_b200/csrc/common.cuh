@@ -90,13 +90,13 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 // (and sets BI_DEV_WAIT_TIMEOUT) when the wait runs past kWaitLimitCycles, or
 // at once when *abort is already set by another thread of the CTA.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status,
-                                          volatile int* abort) {
+                                          volatile int* abort, long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit) {
       set_status(status, BI_DEV_WAIT_TIMEOUT);
       *abort = 1;
       return false;

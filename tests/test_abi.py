@@ -131,3 +131,9 @@ def test_gemm_epilogue_host_checks(bi):
     assert sw(p, 64, p, 64, p, 8, 4, 16, 64, None) == bi.BI_ERR_SHAPE     # ldo < F
     assert sw(None, 64, p, 64, p, 16, 4, 16, 64, None) == bi.BI_ERR_INVALID_ARG
     assert sw(p, 64, p, 64, p, 16, 0, 16, 64, None) == bi.BI_OK           # M == 0: nothing to do
+
+
+def test_wait_bound_check_host_checks(bi):
+    assert bi.lib.bi_check_wait_bound(999, None) == bi.BI_ERR_INVALID_ARG
+    assert bi.lib.bi_check_wait_bound((1 << 32) + 1, None) == bi.BI_ERR_INVALID_ARG
+    assert b"limit" in bi.lib.bi_last_error()
