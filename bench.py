@@ -293,6 +293,28 @@ def attention_leg(bi, torch, synth, reps):
             "ms": ms, "kv_bytes": kv_bytes, "gbs": kv_bytes / ms / 1e6}
 
 
+def prefill_attention_leg(bi, torch, synth, reps):
+    """Causal prefill of four fresh 2048-token prompts (GQA 32/8, d 128) in one
+    bi_attn_prefill call: the prefill attention of the 7B forward leg.
+    FLOPs = 4 Hq d sum_i (p_i + 1) (QK^T and PV over the visible keys)."""
+    lens = [2048] * 4
+    lay = synth.PagedLayout(lens, seed=0)
+    g = torch.Generator("cuda").manual_seed(1)
+    kc = torch.randn(lay.num_pages, 8, 16, 128, device="cuda", generator=g).to(torch.bfloat16)
+    vc = torch.randn(lay.num_pages, 8, 128, 16, device="cuda", generator=g).to(torch.bfloat16)
+    n = sum(lens)
+    q = torch.randn(n, 32 * 128, device="cuda", generator=g).to(torch.bfloat16)
+    shape = bi.attn_shape(32, 8, lay.num_pages, lay.pages_per_seq, 4096)
+    ws = torch.empty(bi.bi_attn_workspace_size(shape, n), dtype=torch.uint8, device="cuda")
+    out = torch.empty(n, 32 * 128, dtype=torch.bfloat16, device="cuda")
+    bt, sl = lay.block_table.cuda(), torch.tensor(lens, dtype=torch.int32, device="cuda")
+    cu = torch.tensor([0, 2048, 4096, 6144, 8192], dtype=torch.int32, device="cuda")
+    ms = per_launch_ms(torch, lambda r=0: bi.bi_attn_prefill(q, cu, 2048, kc, vc, bt, sl, shape, out, ws), reps)
+    flops = 4.0 * 32 * 128 * sum(L * (L + 1) / 2 for L in lens)
+    return {"workload": "prefill, 4 x 2048-token prompts, causal, Hq=32, Hkv=8, d=128",
+            "ms": ms, "tflops": flops / ms / 1e9}
+
+
 def flash_decode_leg(torch, synth, reps):
     """The same decode workload through flash-attn's varlen kernel on K/V
     gathered into contiguous per-sequence rows: a non-invariant cost
@@ -664,6 +686,9 @@ def main():
         r = rmsnorm_leg(bi, torch, reps=10)
         r["frac"] = r["gbs"] / peaks["hbm_gbs"]
         extras["attn_decode"] = a
+        pa = prefill_attention_leg(bi, torch, synth, reps=5)
+        pa["frac"] = pa["tflops"] / peak_t
+        extras["attn_prefill"] = pa
         extras["rmsnorm"] = r
         extras["invariance"] = invariance_flags(torch, sw)
         extras["forward"] = forward_leg(torch, reps=5)
