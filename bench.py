@@ -419,27 +419,54 @@ def rmsnorm_leg(bi, torch, reps):
 def e2e_leg(bi, torch, sw, steps):
     """The same sweep through the C-ABI with HOST buffers: per step, each
     shape's weights and each launch's A rows go host->device from pinned
-    memory and each C comes back device->host, inside the timed region."""
+    memory and each C comes back device->host, inside the timed region.
+    Copies are pipelined on their own streams (host->device on one, the
+    GEMMs on the timing stream, device->host on a third, ordered by events),
+    so a launch's inputs arrive while earlier launches compute; every launch
+    has its own device buffers."""
     hA = {K: sw.A[K].cpu().pin_memory() for K, _ in SHAPES}
     hW = {(K, N): sw.W[(K, N)][0].cpu().pin_memory() for K, N in SHAPES}
-    hC = torch.empty(4096 * 14336, dtype=torch.bfloat16).pin_memory()
+    hC = {(K, N): torch.empty(sum(MS) * N, dtype=torch.bfloat16).pin_memory() for K, N in SHAPES}
     dW = {k: torch.empty_like(v[0]) for k, v in sw.W.items()}
-    dA = {K: torch.empty_like(sw.A[K]) for K, _ in SHAPES}
+    dA = {(K, M): torch.empty(M, K, dtype=torch.bfloat16, device="cuda") for K, _ in SHAPES for M in MS}
+    dC = {(N, M): torch.empty(M, N, dtype=torch.bfloat16, device="cuda") for _, N in SHAPES for M in MS}
     h2d = d2h = 0
     for K, N in SHAPES:
         h2d += N * K * 2
         for M in MS:
             h2d += M * K * 2
             d2h += M * N * 2
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
 
     def one():
+        start = torch.cuda.Event()
+        start.record(comp)
+        s_in.wait_event(start)
+        s_out.wait_event(start)
+        ready = {}
+        with torch.cuda.stream(s_in):
+            for K, N in SHAPES:
+                dW[(K, N)].copy_(hW[(K, N)], non_blocking=True)
+                for M in MS:
+                    dA[(K, M)].copy_(hA[K][:M], non_blocking=True)
+                    ev = torch.cuda.Event()
+                    ev.record(s_in)
+                    ready[(K, M)] = ev
         for K, N in SHAPES:
-            dW[(K, N)].copy_(hW[(K, N)], non_blocking=True)
+            off = 0
             for M in MS:
-                dA[K][:M].copy_(hA[K][:M], non_blocking=True)
-                C = sw.out(M, N)
-                bi.bi_gemm(dA[K][:M], dW[(K, N)], C)
-                hC[: M * N].view(M, N).copy_(C, non_blocking=True)
+                comp.wait_event(ready[(K, M)])
+                C = dC[(N, M)]
+                bi.bi_gemm(dA[(K, M)], dW[(K, N)], C)
+                done = torch.cuda.Event()
+                done.record(comp)
+                s_out.wait_event(done)
+                with torch.cuda.stream(s_out):
+                    hC[(K, N)][off: off + M * N].view(M, N).copy_(C, non_blocking=True)
+                off += M * N
+        comp.wait_stream(s_in)
+        comp.wait_stream(s_out)
 
     one()
     torch.cuda.synchronize()
