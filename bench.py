@@ -51,7 +51,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="bi", choices=["bi", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip attention/RMSNorm/cuBLAS legs")
-    ap.add_argument("--study", default=None, choices=["precision"],
+    ap.add_argument("--study", default=None, choices=["precision", "depth"],
                     help="precision study: all-bf16 vs fp32 upcast vs bf16-MLP-only decoder")
     ap.add_argument("--case", default=None, choices=["gemm", "gemm_m128", "gemm_split", "attn", "rmsnorm",
                                                      "forward"],
@@ -584,6 +584,48 @@ def run_case(case):
     return 0
 
 
+def run_depth_study(n_tok=16, depths=(1, 2, 4, 8, 16, 32)):
+    """Logit error against the fp64 oracle as a function of depth at the
+    Mistral-7B shape (random-init bf16 weights, std 0.02, seed 0; 16 uniform
+    random tokens, seed 1, decoded one at a time, every position compared):
+    the model cut after l layers (final norm and LM head applied to the
+    residual stream after layer l), with bf16 and with fp32 activations."""
+    import numpy as np
+    import torch
+    from invariant_deterministic_03_b200 import runner, synth
+    from oracle import fp64
+    torch.cuda.set_device(0)
+    cfg = dict(n_layers=max(depths), d_model=4096, n_q_heads=32, n_kv_heads=8, d_ff=14336, vocab=32000,
+               max_pos=4096, rms_eps=1e-6, rope_theta=1e4)
+    w = synth.model_weights(cfg, seed=0)
+    wd = {k: v.cuda().contiguous() for k, v in w.items()}
+    toks = synth.randint(n_tok, 0, cfg["vocab"] - 1, seed=1).tolist()
+    t0 = time.time()
+    ref = fp64.forward(fp64.ModelWeights(cfg, {k: synth.bf16_bits(v) for k, v in w.items()}), toks,
+                       depths=set(depths))
+    oracle_s = time.time() - t0
+    out = {"workload": f"Mistral-7B shape cut after l layers, random-init bf16, {n_tok} tokens teacher forced",
+           "oracle_seconds": oracle_s, "modes": {}}
+    for mode in ("bf16", "f32"):
+        rows = []
+        for l in depths:
+            c = dict(cfg, n_layers=l, precision=mode)
+            eng = runner.Engine(c, wd, num_pages=64, max_pages_per_seq=cfg["max_pos"] // 16,
+                                max_tokens=64, max_logits=4, seed=0)
+            lg = torch.cat([eng.step([(0, p, p + 1)], lambda _s: toks)[0] for p in range(n_tok)])
+            got = lg.double().cpu().numpy()
+            err = np.abs(got - ref[l])
+            rows.append({"layers": l, "max_abs": float(err.max()), "mean_abs": float(err.mean()),
+                         "rel_rms": float(np.linalg.norm(got - ref[l]) / np.linalg.norm(ref[l])),
+                         "logit_rms": float(np.sqrt(np.mean(ref[l] ** 2))),
+                         "top1_agree": float(np.mean(got.argmax(1) == ref[l].argmax(1)))})
+            del eng
+            torch.cuda.empty_cache()
+        out["modes"][mode] = rows
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def run_precision_study(n_prompts=512, prompt_len=256, oracle_prompts=4):
     """4-layer d=2048, 16-head (MHA), FFN 5632, vocab 32000 random-init decoder
     (std 0.02), 512 random prompts of 256 tokens, run in the three activation
@@ -655,6 +697,8 @@ def main():
     args = parse()
     if args.study == "precision":
         return run_precision_study()
+    if args.study == "depth":
+        return run_depth_study()
     if args.case:
         return run_case(args.case)
     if args.impl == "reference":

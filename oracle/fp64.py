@@ -238,8 +238,13 @@ class ModelWeights:
         return bf16_bits_to_f64(arr)
 
 
-def forward(weights: ModelWeights, tokens) -> np.ndarray:
+def forward(weights: ModelWeights, tokens, depths=None):
     """Logits [n, V] for every position of ONE sequence of token ids.
+
+    With `depths` (a collection of layer counts 0 .. n_layers), returns
+    instead {l: logits of the model cut after its first l layers}: the final
+    RMSNorm and LM head applied to the residual stream after layer l (the
+    same loop; depth n_layers is the plain result).
 
     The block is the pre-norm decoder the configuration names (RMSNorm, RoPE,
     grouped-query causal attention, SwiGLU MLP, untied LM head):
@@ -258,6 +263,13 @@ def forward(weights: ModelWeights, tokens) -> np.ndarray:
     pos = np.arange(n)
     scale = 1.0 / np.sqrt(dh)
     x = weights.get("embed")[tokens]                      # [n, D]
+
+    def head(x):
+        return gemm(rmsnorm(x, weights.get("final_norm"), eps), weights.get("lm_head"))
+
+    cut = {}
+    if depths is not None and 0 in depths:
+        cut[0] = head(x)
     for layer in range(c["n_layers"]):
         h = rmsnorm(x, weights.get("attn_norm", layer), eps)
         qkv = gemm(h, weights.get("w_qkv", layer))
@@ -271,5 +283,8 @@ def forward(weights: ModelWeights, tokens) -> np.ndarray:
         h = rmsnorm(x, weights.get("mlp_norm", layer), eps)
         gu = gemm(h, weights.get("w_gate_up", layer))
         x = x + gemm(swiglu(gu[:, :F], gu[:, F:]), weights.get("w_down", layer))
-    h = rmsnorm(x, weights.get("final_norm"), eps)
-    return gemm(h, weights.get("lm_head"))
+        if depths is not None and layer + 1 in depths:
+            cut[layer + 1] = head(x)
+    if depths is not None:
+        return cut
+    return head(x)

@@ -392,6 +392,24 @@ def test_forward_one_token_closed_form():
     np.testing.assert_allclose(fp64.forward(w, [tok])[0], want, rtol=1e-11, atol=1e-12)
 
 
+def test_forward_depth_cuts():
+    """Cutting the model after l layers: depth n_layers is the plain result
+    bit for bit, depth 0 is the final norm of the embedding times the LM
+    head, and depth l equals the full forward of the model built from the
+    first l layers alone."""
+    cfg = _tiny_cfg(L=3)
+    w = _tiny_weights(cfg, seed=4)
+    toks = [1, 9, 33, 2]
+    cuts = fp64.forward(w, toks, depths={0, 1, 3})
+    assert set(cuts) == {0, 1, 3}
+    assert np.array_equal(cuts[3], fp64.forward(w, toks))
+    E = fp64.bf16_bits_to_f64(w.a["embed"])
+    want0 = fp64.rmsnorm(E[toks], np.ones(cfg["d_model"]), cfg["rms_eps"]) @ fp64.bf16_bits_to_f64(w.a["lm_head"]).T
+    np.testing.assert_allclose(cuts[0], want0, rtol=1e-12, atol=1e-12)
+    one = fp64.ModelWeights(dict(cfg, n_layers=1), w.a)
+    np.testing.assert_allclose(cuts[1], fp64.forward(one, toks), rtol=0, atol=0)
+
+
 def test_bf16_rounding_helper():
     vals = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -2.5, 0.0, 3.4e38, 1e-40, np.inf])
     bits = fp64.f64_to_bf16_bits(vals)
