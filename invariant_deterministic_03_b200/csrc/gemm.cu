@@ -222,8 +222,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], 4);    // one arrive per epilogue warp
-      mbar_init(&xfer_full[a], 128);  // every epilogue thread of the peer
-      mbar_init(&xfer_free[a], 128);
+      mbar_init(&xfer_full[a], 4);  // lane 0 of each epilogue warp of the peer
+      mbar_init(&xfer_free[a], 4);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -402,10 +402,17 @@ __global__ void __launch_bounds__(THREADS, 1)
           uint32_t r[32];
           tmem_ld32(taddr + c * 32, r);
           tmem_ld_wait();
+          // One lane per warp waits (acquire) and arrives (release) at
+          // cluster scope; __syncwarp orders the other lanes' accesses
+          // around it (release and acquire are cumulative), so each hand-over
+          // costs one cluster fence per warp, not one per thread.
           if (send) {
             const int slot = nx_out & 1;  // a slot of the peer's staging area
-            if (!mbar_wait_cluster(&xfer_free[slot], (((uint32_t)nx_out >> 1) & 1u) ^ 1u, p.status,
-                                   abort_flag)) {
+            int w_ok = 1;
+            if (lane == 0)
+              w_ok = mbar_wait_cluster(&xfer_free[slot], (((uint32_t)nx_out >> 1) & 1u) ^ 1u, p.status,
+                                       abort_flag);
+            if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
               ok = false;
               break;
             }
@@ -416,11 +423,15 @@ __global__ void __launch_bounds__(THREADS, 1)
                 st_cluster_v4(dst + ((uint32_t)(j ^ (trow & 7)) << 4), r[4 * j], r[4 * j + 1],
                               r[4 * j + 2], r[4 * j + 3]);
             }
-            mbar_arrive_cluster(cluster_addr(&xfer_full[slot], peer));
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(cluster_addr(&xfer_full[slot], peer));
             ++nx_out;
           } else {
             const int slot = nx_in & 1;
-            if (!mbar_wait_cluster(&xfer_full[slot], ((uint32_t)nx_in >> 1) & 1u, p.status, abort_flag)) {
+            int w_ok = 1;
+            if (lane == 0)
+              w_ok = mbar_wait_cluster(&xfer_full[slot], ((uint32_t)nx_in >> 1) & 1u, p.status, abort_flag);
+            if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
               ok = false;
               break;
             }
@@ -435,7 +446,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 r[4 * j + 3] = __float_as_uint(__fadd_rn(__uint_as_float(r[4 * j + 3]), __uint_as_float(v.w)));
               }
             }
-            mbar_arrive_cluster(cluster_addr(&xfer_free[slot], peer));
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(cluster_addr(&xfer_free[slot], peer));
             ++nx_in;
             finish(c, r);
           }
