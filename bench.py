@@ -400,6 +400,21 @@ def forward_leg(torch, reps):
         n_tok = b["tokens"].shape[0]
         out[name] = {"tokens": n_tok, "ms": ms, "tokens_per_s": n_tok / ms * 1e3,
                      "tflops": n_tok * out["gflop_per_token_weights"] / ms / 1e3}
+        if name == "decode":
+            # the same step captured once in a CUDA graph (its ~330 launches
+            # replayed as one; a serving loop updates the batch tensors in place)
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                fn()
+            torch.cuda.current_stream().wait_stream(side)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                fn()
+            gms = per_launch_ms(torch, lambda r=0: graph.replay(), reps)
+            out[name]["graph_ms"] = gms
+            out[name]["graph_tokens_per_s"] = n_tok / gms * 1e3
+            del graph
     del eng, w
     torch.cuda.empty_cache()
     return out

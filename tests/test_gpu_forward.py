@@ -130,3 +130,34 @@ def test_greedy_generation_run_to_run(bi):
         assert int(torch.argmax(lg[0]).item()) == int(nxt[0].item())
     assert outs[0][0] == outs[1][0]
     assert same_bits(outs[0][1], outs[1][1])
+
+
+def test_decode_step_graph_replay_is_bitwise(bi):
+    """A decode step captured in a CUDA graph and replayed gives the same
+    logits bits and tokens as the eager call on the same inputs."""
+    from invariant_deterministic_03_b200 import runner
+    cfg = SMALL
+    w = synth.model_weights(cfg, seed=31)
+    eng, _ = _engine(cfg, w, seed=4)
+    toks = synth.randint(40, 0, cfg["vocab"] - 1, seed=32).tolist()
+    eng.step([(0, 0, 39), (1, 0, 20)], lambda s: toks)
+    b = runner.make_batch(eng.kv, [(0, 39, 40), (1, 20, 21)], lambda s: toks)
+    b["max_kv_len"] = cfg["max_pos"]
+    eager = torch.empty(2, cfg["vocab"], dtype=torch.float32, device="cuda:0")
+    eager_t = torch.empty(2, dtype=torch.int32, device="cuda:0")
+    eng.model.forward(b, eng.kv.k, eng.kv.v, eager, eager_t, eng.ws)
+    g_out = torch.empty_like(eager)
+    g_tok = torch.empty_like(eager_t)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        eng.model.forward(b, eng.kv.k, eng.kv.v, g_out, g_tok, eng.ws)
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        eng.model.forward(b, eng.kv.k, eng.kv.v, g_out, g_tok, eng.ws)
+    g_out.zero_()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert same_bits(g_out, eager) and torch.equal(g_tok, eager_t)
