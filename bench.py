@@ -370,7 +370,7 @@ def forward_setup(torch, cfg=FWD_CFG, seed=0):
          "w_gate_up": rnd(L, 2 * F, D), "w_down": rnd(L, D, F)}
     ctx = [1400] + synth.randint(63, 16, 2048, seed=2).tolist()
     fresh = [2048] * 4
-    pages = sum((c + 1 + 15) // 16 for c in ctx) + sum((f + 15) // 16 for f in fresh) + 64
+    pages = sum((c + 1 + 15) // 16 for c in ctx) + sum((f + 15) // 16 for f in fresh) + 4 * 32 + 64
     eng = runner.Engine(cfg, w, num_pages=pages, max_pages_per_seq=cfg["max_pos"] // 16,
                         max_tokens=8192, max_logits=64, seed=seed)
     toks = synth.randint(cfg["max_pos"], 0, V - 1, seed=3).tolist()
@@ -379,18 +379,25 @@ def forward_setup(torch, cfg=FWD_CFG, seed=0):
         eng.kv.length[s] = c
     decode = runner.make_batch(eng.kv, [(s, c, c + 1) for s, c in enumerate(ctx)], lambda s: toks)
     prefill = runner.make_batch(eng.kv, [(100 + i, 0, f) for i, f in enumerate(fresh)], lambda s: toks)
-    for b in (decode, prefill):
+    # a continuous-batching step: the 64 decode tokens plus four 512-token
+    # prompt chunks, laid out with the one-token chunks first (their attention
+    # in the decode kernel) and, for comparison, all through the prefill kernel
+    mixed_chunks = [(s, c, c + 1) for s, c in enumerate(ctx)] + [(200 + i, 0, 512) for i in range(4)]
+    mixed = runner.make_batch(eng.kv, mixed_chunks, lambda s: toks)
+    mixed_one_kernel = runner.make_batch(eng.kv, mixed_chunks, lambda s: toks, decode_first=False)
+    for b in (decode, prefill, mixed, mixed_one_kernel):
         b["max_kv_len"] = cfg["max_pos"]
-    return eng, w, decode, prefill
+    return eng, w, decode, prefill, mixed, mixed_one_kernel
 
 
 def forward_leg(torch, reps):
-    eng, w, decode, prefill = forward_setup(torch)
+    eng, w, decode, prefill, mixed, mixed_one = forward_setup(torch)
     out = {"workload": "Mistral-7B shape (32 layers, d 4096, 32/8 heads, FFN 14336, vocab 32000), "
                        "random-init bf16; decode: 64 requests (contexts 1400 + 63 x U[16,2048]); "
-                       "prefill: 4 x 2048-token prompts",
+                       "prefill: 4 x 2048-token prompts; mixed: the 64 decode tokens + 4 x 512-token chunks",
            "gflop_per_token_weights": 2.0 * sum(v.numel() for k, v in w.items() if k not in ("embed",)) / 1e9}
-    for name, b in (("decode", decode), ("prefill", prefill)):
+    for name, b in (("decode", decode), ("prefill", prefill), ("mixed", mixed),
+                    ("mixed_one_attention_kernel", mixed_one)):
         n_log = b["logits_rows"].shape[0]
         logits = torch.empty(n_log, FWD_CFG["vocab"], dtype=torch.float32, device="cuda")
         nxt = torch.empty(n_log, dtype=torch.int32, device="cuda")
@@ -557,7 +564,7 @@ def run_case(case):
     if case == "forward":
         # one decode step and one prefill step of the 7B-shape forward after a
         # warm-up of each (for a launch list of every kernel they run)
-        eng, _, decode, prefill = forward_setup(torch)
+        eng, _, decode, prefill, _, _ = forward_setup(torch)
         for b in (decode, prefill, decode, prefill):
             n_log = b["logits_rows"].shape[0]
             logits = torch.empty(n_log, FWD_CFG["vocab"], dtype=torch.float32, device="cuda")

@@ -253,9 +253,12 @@ bi_status bi_attn_decode_noalloc(const void* q, int64_t ldq, const void* k_cache
                                  void* stream);
 
 /* Prefill (chunked): sequence b owns query rows cu_q[b] .. cu_q[b+1]-1
- * (cu_q [B+1] int32 on the device, cu_q[0] = 0, cu_q[B] = n_tok); they are its
- * LAST n_b = cu_q[b+1]-cu_q[b] tokens, so row cu_q[b]+i sits at position
- * seq_lens[b] - n_b + i. max_q_len bounds n_b (host-side grid size). */
+ * (cu_q [B+1] int32 on the device, increasing, 0 <= cu_q[0], cu_q[B] <=
+ * n_tok); they are its LAST n_b = cu_q[b+1]-cu_q[b] tokens, so row cu_q[b]+i
+ * sits at position seq_lens[b] - n_b + i. max_q_len bounds n_b (host-side
+ * grid size). q and out span all n_tok rows; rows outside cu_q[0] ..
+ * cu_q[B]-1 are not read or written (so a call can cover a subset of a
+ * batch, e.g. the multi-token chunks after the batch's one-token ones). */
 bi_status bi_attn_prefill(const void* q, int64_t ldq, const int32_t* cu_q,
                           int32_t max_q_len, int64_t n_tok, const void* k_cache,
                           const void* v_cache, const int32_t* block_table,
@@ -392,7 +395,13 @@ typedef struct bi_model bi_model;
  *   cu_q [B+1] (rows of each sequence, contiguous and in order),
  *   seq_lens [B] (keys cached after this step), block_table [B][max_pages_per_seq],
  *   logits_rows [n_logits] (which token rows produce logits).
- * Host ints: max_q_len bounds cu_q[b+1]-cu_q[b]; max_kv_len bounds seq_lens. */
+ * Host ints: max_q_len bounds cu_q[b+1]-cu_q[b]; max_kv_len bounds seq_lens;
+ * n_decode (0 .. B): the first n_decode sequences each bring exactly one
+ * token (rows 0 .. n_decode-1); their attention runs in the decode kernel and
+ * the rest in the prefill kernel, which give the same bits for a row (0 sends
+ * every row through one kernel: the decode kernel when every chunk is one
+ * token, else the prefill kernel). A wrong n_decode gives wrong rows, never
+ * an out-of-range access. */
 typedef struct {
   const int32_t* tokens;
   const int32_t* positions;
@@ -407,6 +416,7 @@ typedef struct {
   int32_t max_kv_len;
   int32_t max_pages_per_seq;
   int64_t n_logits;
+  int32_t n_decode;
 } bi_batch;
 
 bi_status bi_model_create(const bi_model_config* cfg, const bi_model_weights* w,

@@ -65,7 +65,7 @@ class Batch(ctypes.Structure):
     _fields_ = [("tokens", _p), ("positions", _p), ("slot_mapping", _p), ("cu_q", _p),
                 ("seq_lens", _p), ("block_table", _p), ("logits_rows", _p), ("n_tok", _i64),
                 ("B", _i32), ("max_q_len", _i32), ("max_kv_len", _i32),
-                ("max_pages_per_seq", _i32), ("n_logits", _i64)]
+                ("max_pages_per_seq", _i32), ("n_logits", _i64), ("n_decode", _i32)]
 
 
 _SIGS = {
@@ -357,13 +357,14 @@ class Model:
     def forward(self, batch: dict, k_cache, v_cache, logits, next_tokens, ws, stream=None):
         """batch: device int32 tensors tokens, positions, slot_mapping, cu_q,
         seq_lens, block_table [B, P], logits_rows, plus host ints max_q_len,
-        max_kv_len."""
+        max_kv_len and (optional) n_decode: the number of leading one-token
+        sequences."""
         bt = batch["block_table"]
         b = Batch(_ptr(batch["tokens"]), _ptr(batch["positions"]), _ptr(batch["slot_mapping"]),
                   _ptr(batch["cu_q"]), _ptr(batch["seq_lens"]), _ptr(bt),
                   _ptr(batch["logits_rows"]), batch["tokens"].shape[0],
                   batch["seq_lens"].shape[0], batch["max_q_len"], batch["max_kv_len"],
-                  bt.shape[1], batch["logits_rows"].shape[0])
+                  bt.shape[1], batch["logits_rows"].shape[0], batch.get("n_decode", 0))
         _chk("bi_forward", lib.bi_forward(self.handle, ctypes.byref(b), _ptr(k_cache),
                                           _ptr(v_cache), k_cache.shape[1], _ptr(logits),
                                           _ptr(next_tokens), _ptr(ws),

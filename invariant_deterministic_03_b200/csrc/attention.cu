@@ -852,6 +852,7 @@ __global__ void attn_combine_kernel(const CombineParams p) {
   const int h = (int)(wid % p.Hq);
   int b, nb, qidx;
   if (p.cu_q) {
+    if (tok < p.cu_q[0] || tok >= p.cu_q[p.B]) return;  // a row this call does not cover
     int lo = 0, hi = p.B;  // find b with cu_q[b] <= tok < cu_q[b+1]
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;

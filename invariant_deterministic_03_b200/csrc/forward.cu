@@ -171,6 +171,8 @@ extern "C" bi_status bi_forward(const bi_model* m, const bi_batch* bt, void* k_c
   if (!b.tokens || !b.positions || !b.slot_mapping || !b.cu_q || !b.seq_lens || !b.block_table || (b.n_logits && !b.logits_rows))
     return fail(BI_ERR_INVALID_ARG, "forward: null batch array");
   if (b.max_kv_len > c.max_pos) return fail(BI_ERR_SHAPE, "forward: max_kv_len above max_pos");
+  if (b.n_decode < 0 || b.n_decode > b.B || b.n_decode > b.n_tok)
+    return fail(BI_ERR_INVALID_ARG, "forward: n_decode %d outside 0 .. B", b.n_decode);
   const fwd::Layout L = fwd::layout(c, b.n_tok, b.n_logits, b.max_kv_len);
   if (ws_bytes < L.total) return fail(BI_ERR_WORKSPACE, "forward: workspace %zu < %zu", ws_bytes, L.total);
   if (!aligned16(ws) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(logits))
@@ -247,16 +249,17 @@ extern "C" bi_status bi_forward(const bi_model* m, const bi_batch* bt, void* k_c
       BI_TRY(launch_rope(qkv, QKV, Hq + Hkv, b.positions, T, rope, c.max_pos, s));
       BI_TRY(launch_kv_append(qkv + (size_t)Hq * BI_HEAD_DIM, qkv + (size_t)(Hq + Hkv) * BI_HEAD_DIM,
                               QKV, b.slot_mapping, T, kc, vc, Hkv, num_pages, s));
-      if (T == b.B && b.max_q_len == 1) {
-        // every chunk is one token: the decode kernel, whose rows are the
-        // same bits as the prefill kernel's (same tiles, splits and per-row
-        // arithmetic)
-        BI_TRY(bi_attn_decode(qkv, QKV, kc, vc, b.block_table, b.seq_lens, b.B, &sh, att, D, attn_ws,
+      // one-token sequences go through the decode kernel, longer chunks
+      // through the prefill kernel; a row gets the same bits from either
+      // (same tiles, splits and per-row arithmetic)
+      const int32_t nd = (T == b.B && b.max_q_len == 1) ? b.B : b.n_decode;
+      if (nd > 0)
+        BI_TRY(bi_attn_decode(qkv, QKV, kc, vc, b.block_table, b.seq_lens, nd, &sh, att, D, attn_ws,
                               L.attn_ws_bytes, stream));
-      } else {
-        BI_TRY(bi_attn_prefill(qkv, QKV, b.cu_q, b.max_q_len, T, kc, vc, b.block_table, b.seq_lens,
-                               b.B, &sh, att, D, attn_ws, L.attn_ws_bytes, stream));
-      }
+      if (nd < b.B)
+        BI_TRY(bi_attn_prefill(qkv, QKV, b.cu_q + nd, b.max_q_len, T, kc, vc,
+                               b.block_table + (size_t)nd * b.max_pages_per_seq, b.seq_lens + nd, b.B - nd,
+                               &sh, att, D, attn_ws, L.attn_ws_bytes, stream));
       BI_TRY(bi_gemm(att, D, w_o, D, x, D, BI_F32_ADD, T, D, D, stream));  // x += O proj
     }
 

@@ -72,13 +72,24 @@ class PagedKV:
         return self.length[dst]
 
 
-def make_batch(kv: PagedKV, chunks, tokens_of, device="cuda:0"):
+def make_batch(kv: PagedKV, chunks, tokens_of, device="cuda:0", decode_first: bool = True):
     """chunks: list of (seq, start, end) -- tokens start..end-1 of `seq` are
     processed in this step (their keys are written, then attended). The keys
     0..start-1 must already be cached. Returns the device batch dict for
-    Model.forward with one logits row per chunk (its last token)."""
-    toks, pos, slots, cu, lens, rows = [], [], [], [0], [], []
-    for seq, s, e in chunks:
+    Model.forward with one logits row per chunk (its last token), in the order
+    of `chunks`. With decode_first, one-token chunks are laid out first and
+    counted in n_decode, so their attention runs in the decode kernel (a row's
+    bits do not depend on which kernel or which batch position computes it)."""
+    order = list(range(len(chunks)))
+    n_decode = 0
+    if decode_first:
+        one = [i for i, (_, s, e) in enumerate(chunks) if e - s == 1]
+        rest = [i for i, (_, s, e) in enumerate(chunks) if e - s != 1]
+        order, n_decode = one + rest, len(one)
+    toks, pos, slots, cu, lens = [], [], [], [0], []
+    last_row = {}
+    for i in order:
+        seq, s, e = chunks[i]
         if kv.length.get(seq, 0) != s:
             raise ValueError(f"sequence {seq}: cache holds {kv.length.get(seq, 0)} keys, chunk starts at {s}")
         kv.ensure(seq, e)
@@ -89,16 +100,17 @@ def make_batch(kv: PagedKV, chunks, tokens_of, device="cuda:0"):
             slots.append(kv.slot(seq, p))
         cu.append(cu[-1] + e - s)
         lens.append(e)
-        rows.append(cu[-1] - 1)
+        last_row[i] = cu[-1] - 1
+    rows = [last_row[i] for i in range(len(chunks))]
     bt = torch.full((len(chunks), kv.max_pages), -1, dtype=torch.int32)
-    for i, (seq, _, _) in enumerate(chunks):
-        pg = kv.pages[seq]
-        bt[i, : len(pg)] = torch.tensor(pg, dtype=torch.int32)
+    for j, i in enumerate(order):
+        pg = kv.pages[chunks[i][0]]
+        bt[j, : len(pg)] = torch.tensor(pg, dtype=torch.int32)
     i32 = lambda x: torch.tensor(x, dtype=torch.int32, device=device)  # noqa: E731
     batch = {"tokens": i32(toks), "positions": i32(pos), "slot_mapping": i32(slots),
              "cu_q": i32(cu), "seq_lens": i32(lens), "block_table": bt.to(device),
              "logits_rows": i32(rows), "max_q_len": max(e - s for _, s, e in chunks),
-             "max_kv_len": max(lens)}
+             "max_kv_len": max(lens), "n_decode": n_decode}
     return batch
 
 

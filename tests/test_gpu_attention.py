@@ -212,3 +212,30 @@ def test_bad_page_sets_status(bi):
     st = bi.bi_device_status(clear=True)
     assert st & 0x4
     assert torch.isfinite(out.float()).all()
+
+
+def test_mixed_batch_decode_then_prefill_subsets(bi):
+    """A batch of one-token sequences followed by longer chunks: the decode
+    kernel over the leading sequences plus the prefill kernel over the rest
+    (cu_q, seq_lens and block table offset to the subset) gives the same bits
+    as one prefill call over everything, and a subset call leaves the rows
+    it does not cover untouched."""
+    lens = [700, 33, 1300, 250, 513]
+    S = Seqs(bi, lens, 32, 8, seed=41)
+    shape = S.shape(bi)
+    chunks = [(0, 699, 700), (1, 32, 33), (2, 1000, 1300), (3, 200, 250), (4, 0, 513)]
+    whole = _prefill(bi, S, chunks, shape)
+    q = torch.cat([S.q[b][s:e].reshape(e - s, -1) for b, s, e in chunks])
+    n = q.shape[0]
+    cu = torch.tensor([0, 1, 2, 302, 352, 865], dtype=torch.int32)
+    bt = dev(S.layout.block_table[[b for b, _, _ in chunks]])
+    sl = dev(torch.tensor([e for _, _, e in chunks], dtype=torch.int32))
+    ws = torch.empty(bi.bi_attn_workspace_size(shape, n), dtype=torch.uint8, device="cuda:0")
+    out = torch.full((n, q.shape[1]), 7.0, dtype=torch.bfloat16, device="cuda:0")
+    nd = 2
+    bi.bi_attn_decode(dev(q), S.kc, S.vc, bt, sl[:nd], shape, out[:nd], ws)
+    marker = out[:nd].clone()
+    bi.bi_attn_prefill(dev(q), dev(cu[nd:]), 512, S.kc, S.vc, bt[nd:].contiguous(), sl[nd:].contiguous(),
+                       shape, out, ws)
+    assert same_bits(out[:nd], marker)               # the subset call left the decode rows alone
+    assert same_bits(out, whole)

@@ -53,3 +53,20 @@ def test_out_of_pages_is_an_error():
     kv = _kv(num_pages=2)
     with pytest.raises(RuntimeError):
         kv.ensure(0, 33)
+
+
+def test_make_batch_puts_one_token_chunks_first():
+    kv = _kv(num_pages=64)
+    for seq, n in [(0, 20), (1, 5), (2, 40)]:
+        kv.ensure(seq, n)
+        kv.length[seq] = n
+    toks = list(range(100))
+    chunks = [(2, 40, 48), (0, 20, 21), (1, 5, 6)]       # 8 tokens, then two one-token chunks
+    b = runner.make_batch(kv, chunks, lambda s: toks, device="cpu")
+    assert b["n_decode"] == 2
+    assert b["cu_q"].tolist() == [0, 1, 2, 10]           # the one-token chunks are rows 0 and 1
+    assert b["positions"].tolist()[:2] == [20, 5]
+    assert b["seq_lens"].tolist() == [21, 6, 48]
+    assert b["logits_rows"].tolist() == [9, 0, 1]        # logits stay in the order of `chunks`
+    b2 = runner.make_batch(kv, chunks, lambda s: toks, device="cpu", decode_first=False)
+    assert b2["n_decode"] == 0 and b2["logits_rows"].tolist() == [7, 8, 9]
