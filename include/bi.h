@@ -140,6 +140,29 @@ bi_status bi_gemm_swiglu(const void* A, int64_t lda, const void* W,
                          int64_t ldw, void* out, int64_t ldo, int64_t M,
                          int64_t F, int64_t K, void* stream);
 
+/* QKV projection with RoPE and the KV-cache write in its epilogue. W is the
+ * fused [(Hq + 2 Hkv) * 128, K] weight (q heads, then k heads, then v heads,
+ * 128 rows each, row stride ldw); qkv [M, (Hq + 2 Hkv) * 128] bf16 (row
+ * stride ldq). The result is the same bits as these three calls in order:
+ *   bi_gemm(A, lda, W, ldw, qkv, ldq, BI_BF16, M, (Hq + 2 Hkv) * 128, K);
+ *   bi_rope(qkv, ldq, Hq + Hkv, positions, M, cos_sin, max_pos);
+ *   bi_kv_append(k heads of qkv, v heads of qkv, ldq, slot_mapping, M, ...);
+ * i.e. qkv holds the rotated q and k heads and the plain v heads, and row
+ * m's k and v heads are in the caches at slot_mapping[m] (skipped when < 0;
+ * outside the cache: skipped and BI_DEV_BAD_SLOT). One launch when the
+ * weight takes no K split (every weight with K < 8192 or more than 37
+ * column tiles); otherwise the three steps run as three launches. cos_sin
+ * [max_pos, 64, 2] fp32 from bi_rope_table; caches as for bi_kv_append
+ * (num_pages pages, Hkv heads). Constraints as bi_gemm; caches and cos_sin
+ * 16-byte aligned. M == 0 is a no-op. */
+bi_status bi_gemm_qkv(const void* A, int64_t lda, const void* W, int64_t ldw,
+                      void* qkv, int64_t ldq, int64_t M, int64_t K,
+                      int32_t n_q_heads, int32_t n_kv_heads,
+                      const int32_t* positions, const float* cos_sin,
+                      int32_t max_pos, const int32_t* slot_mapping,
+                      void* k_cache, void* v_cache, int32_t num_pages,
+                      void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Paged KV cache.  "Defeating Nondeterminism in LLM Inference", section
  * "Batch-invariant attention": the cache and page table are updated BEFORE

@@ -76,6 +76,8 @@ _SIGS = {
     "bi_rmsnorm_f32in": (_i32, [_p, _p, _p, _i64, _i64, _f32, _p]),
     "bi_gemm": (_i32, [_p, _i64, _p, _i64, _p, _i64, _i32, _i64, _i64, _i64, _p]),
     "bi_gemm_swiglu": (_i32, [_p, _i64, _p, _i64, _p, _i64, _i64, _i64, _i64, _p]),
+    "bi_gemm_qkv": (_i32, [_p, _i64, _p, _i64, _p, _i64, _i64, _i64, _i32, _i32, _p, _p, _i32, _p, _p, _p,
+                           _i32, _p]),
     "bi_kv_append": (_i32, [_p, _p, _i64, _p, _i64, _p, _p, ctypes.POINTER(KVLayout), _p]),
     "bi_attn_workspace_size": (_i32, [ctypes.POINTER(AttnShape), _i64, ctypes.POINTER(_sz)]),
     "bi_attn_decode": (_i32, [_p, _i64, _p, _p, _p, _p, _i32, ctypes.POINTER(AttnShape), _p,
@@ -176,6 +178,21 @@ def bi_gemm_swiglu(A, W, out, stream=None) -> None:
         raise ValueError("bi_gemm_swiglu: W must have 2F rows")
     _chk("bi_gemm_swiglu", lib.bi_gemm_swiglu(_ptr(A), A.stride(0), _ptr(W), W.stride(0), _ptr(out),
                                               out.stride(0), M, F, K, _stream(stream)))
+
+
+def bi_gemm_qkv(A, W, qkv, n_q_heads: int, n_kv_heads: int, positions, cos_sin, max_pos: int,
+                slot_mapping, k_cache, v_cache, stream=None) -> None:
+    """qkv = A W^T with RoPE on the q and k heads and k / v written to the
+    paged caches (one layer's [num_pages, Hkv, ...] slices). A [M, K] bf16,
+    W [(Hq + 2 Hkv) * 128, K] bf16, qkv [M, (Hq + 2 Hkv) * 128] bf16,
+    positions / slot_mapping [M] int32, cos_sin the bi_rope_table of max_pos
+    positions."""
+    M, K = A.shape
+    num_pages = k_cache.shape[0]
+    _chk("bi_gemm_qkv", lib.bi_gemm_qkv(_ptr(A), A.stride(0), _ptr(W), W.stride(0), _ptr(qkv),
+                                        qkv.stride(0), M, K, n_q_heads, n_kv_heads, _ptr(positions),
+                                        _ptr(cos_sin), max_pos, _ptr(slot_mapping), _ptr(k_cache),
+                                        _ptr(v_cache), num_pages, _stream(stream)))
 
 
 def bi_gemm_x2(A_hi, A_lo, W, C, stream=None, add: bool = False) -> None:

@@ -41,6 +41,15 @@ __device__ __forceinline__ float swiglu_f32(float g, float u) {
   return __fmul_rn(silu, u);
 }
 
+// RoPE of one (i, i + 64) pair of a head ("rotate half"), fp32, each product
+// and sum rounded once: (a, b) -> (a c - b s, b c + a s). The stand-alone
+// RoPE kernel and the QKV GEMM's epilogue both call this, so they give the
+// same bits.
+__device__ __forceinline__ void rope_rotate(float a, float b, float c, float s, float& ra, float& rb) {
+  ra = __fsub_rn(__fmul_rn(a, c), __fmul_rn(b, s));
+  rb = __fadd_rn(__fmul_rn(b, c), __fmul_rn(a, s));
+}
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

@@ -203,6 +203,7 @@ extern "C" bi_status bi_forward(const bi_model* m, const bi_batch* bt, void* k_c
   const int Hq = c.n_q_heads, Hkv = c.n_kv_heads;
   const int64_t QKV = (int64_t)(Hq + 2 * Hkv) * BI_HEAD_DIM;
   const size_t cache_layer = (size_t)num_pages * Hkv * BI_PAGE_SIZE * BI_HEAD_DIM;
+  const bool qkv_fused = ((T + BI_GEMM_BM - 1) / BI_GEMM_BM) * ((QKV + BI_GEMM_BN - 1) / BI_GEMM_BN) >= num_sms();
 
   BI_TRY(bi_rope_table(rope, c.max_pos, c.rope_theta, stream));
   BI_TRY(launch_embed(b.tokens, T, static_cast<const bf16*>(m->w.embed), c.vocab, D, x, s));
@@ -244,11 +245,21 @@ extern "C" bi_status bi_forward(const bi_model* m, const bi_batch* bt, void* k_c
       bf16* kc = static_cast<bf16*>(k_cache) + (size_t)l * cache_layer;
       bf16* vc = static_cast<bf16*>(v_cache) + (size_t)l * cache_layer;
       BI_TRY(bi_rmsnorm_f32in(x, attn_norm, h, T, D, c.rms_eps, stream));
-      BI_TRY(bi_gemm(h, D, w_qkv, D, qkv, QKV, BI_BF16, T, QKV, D, stream));
-      // q and k heads are adjacent in a qkv row: one launch rotates both
-      BI_TRY(launch_rope(qkv, QKV, Hq + Hkv, b.positions, T, rope, c.max_pos, s));
-      BI_TRY(launch_kv_append(qkv + (size_t)Hq * BI_HEAD_DIM, qkv + (size_t)(Hq + Hkv) * BI_HEAD_DIM,
-                              QKV, b.slot_mapping, T, kc, vc, Hkv, num_pages, s));
+      // QKV projection, RoPE of the q and k heads, cache write: one launch
+      // when every SM gets at least one output tile (RoPE and the scattered
+      // cache stores then spread over all SMs and overlap later tiles'
+      // MMAs); for fewer tiles the epilogue work would sit on those few SMs
+      // after their only tile, so three launches are faster. Same bits.
+      if (qkv_fused) {
+        BI_TRY(bi_gemm_qkv(h, D, w_qkv, D, qkv, QKV, T, D, Hq, Hkv, b.positions, rope, c.max_pos,
+                           b.slot_mapping, kc, vc, num_pages, stream));
+      } else {
+        BI_TRY(bi_gemm(h, D, w_qkv, D, qkv, QKV, BI_BF16, T, QKV, D, stream));
+        // q and k heads are adjacent in a qkv row: one launch rotates both
+        BI_TRY(launch_rope(qkv, QKV, Hq + Hkv, b.positions, T, rope, c.max_pos, s));
+        BI_TRY(launch_kv_append(qkv + (size_t)Hq * BI_HEAD_DIM, qkv + (size_t)(Hq + Hkv) * BI_HEAD_DIM,
+                                QKV, b.slot_mapping, T, kc, vc, Hkv, num_pages, s));
+      }
       // one-token sequences go through the decode kernel, longer chunks
       // through the prefill kernel; a row gets the same bits from either
       // (same tiles, splits and per-row arithmetic)

@@ -90,6 +90,13 @@ struct Params {
   int32_t kb_per_rank; // k-blocks of rank 0 (rank 1 takes the rest)
   uint32_t a_bytes;    // bytes of one A copy: 128 rows, or M rounded up to 8 when M < 128
   int32_t* status;
+  // EPI_QKV only: RoPE of the q and k heads and the paged-cache write
+  const int32_t* pos;    // [M] absolute positions
+  const float* cs;       // [max_pos, 64, 2] cos / sin
+  const int32_t* slots;  // [M] cache slots (page * 16 + offset), < 0: padding row
+  bf16* kc;              // key cache, 4 KB per (page, kv head)
+  bf16* vc;              // value cache, same blocking, transposed per page
+  int32_t max_pos, num_pages, hq, hkv;
 };
 
 __device__ __forceinline__ void store_row_chunk(const Params& p, int row, int col0,
@@ -180,7 +187,108 @@ __device__ __forceinline__ void store_swiglu_chunk(const Params& p, int row, int
 //               (W rows f) and the same 128 up features (W rows F + f):
 //               C[m, f] = bf16(swiglu_f32(bf16(g), bf16(u))), the same
 //               rounding points as a bf16 GEMM followed by bi_swiglu.
-constexpr int EPI_STORE = 0, EPI_ADD = 1, EPI_SWIGLU = 2;
+constexpr int EPI_STORE = 0, EPI_ADD = 1, EPI_SWIGLU = 2, EPI_QKV = 3;
+
+// EPI_QKV: the fused [q | k | v] projection (heads of 128 columns, so a
+// 256-column tile is heads 2 nb and 2 nb + 1). Every element is first
+// rounded to bf16 as EPI_STORE does. q and k heads then rotate each pair
+// (i, i + 64) with the RoPE kernel's arithmetic (rope_rotate on the bf16
+// values and the fp32 table) and are stored rounded again; k and v heads are
+// also written to the paged caches at the row's slot, in the KV append's
+// layout:
+//   keys:   element (slot o, d) at (o/8)*1024 + (d/8)*64 + (o%8)*8 + d%8
+//   values: element (d, slot o) at (d/8)*128 + (o/8)*64 + (d%8)*8 + o%8
+// of the (page, kv head) block. The qkv rows and both caches end up with the
+// same bits as bi_gemm, then bi_rope over the q and k heads, then
+// bi_kv_append. The tensor-memory loads are warp-collective, so every lane
+// runs them; only rows < M store.
+__device__ __forceinline__ void qkv_tile(const Params& p, int row, int nb, uint32_t taddr) {
+  const bool live = row < p.M;
+  int pos = 0, slot = -1;
+  if (live) {
+    pos = p.pos[row];
+    slot = p.slots[row];
+  }
+  const bool rot = pos >= 0 && pos < p.max_pos;
+  const bool slot_bad = slot >= p.num_pages * BI_PAGE_SIZE;
+  const bool to_cache = live && slot >= 0 && !slot_bad;
+  const int sl = to_cache ? slot : 0;
+  const int page = sl / BI_PAGE_SIZE, o = sl % BI_PAGE_SIZE;
+  if (live && !rot && nb * 2 < p.hq + p.hkv) set_status(p.status, BI_DEV_BAD_TOKEN);
+  const int n_heads = p.hq + 2 * p.hkv;
+  bf16* crow = static_cast<bf16*>(p.C) + (size_t)(live ? row : 0) * p.ldc;
+#pragma unroll 1
+  for (int hh = 0; hh < 2; ++hh) {
+    const int H = nb * 2 + hh;
+    if (H >= n_heads) break;  // uniform across the warp
+    bf16* out = crow + (size_t)H * BI_HEAD_DIM;
+    if (H >= p.hq && live && slot_bad) set_status(p.status, BI_DEV_BAD_SLOT);
+    if (H < p.hq + p.hkv) {
+      const bool is_k = H >= p.hq;
+      bf16* kdst = p.kc + ((size_t)page * p.hkv + (is_k ? H - p.hq : 0)) * (BI_PAGE_SIZE * BI_HEAD_DIM) +
+                   (o >> 3) * 1024 + (o & 7) * 8;
+#pragma unroll 1
+      for (int j = 0; j < 2; ++j) {
+        uint32_t ra[32], rb[32];  // columns 32 j .. 32 j + 31 and their partners 64 further on
+        tmem_ld32(taddr + (hh * 4 + j) * 32, ra);
+        tmem_ld32(taddr + (hh * 4 + j + 2) * 32, rb);
+        tmem_ld_wait();
+        if (!live) continue;
+        const float* csp = p.cs + ((size_t)(rot ? pos : 0) * 64 + j * 32) * 2;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          float ya[8], yb[8];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float4 t = rot ? reinterpret_cast<const float4*>(csp + g * 16)[q] : make_float4(1.f, 0.f, 1.f, 0.f);
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int e = 2 * q + h2;
+              const float a = round_bf16(ra[8 * g + e]), b = round_bf16(rb[8 * g + e]);
+              if (rot) rope_rotate(a, b, h2 ? t.z : t.x, h2 ? t.w : t.y, ya[e], yb[e]);
+              else { ya[e] = a; yb[e] = b; }
+            }
+          }
+          const uint4 A = make_uint4(pack_bf16x2(ya[0], ya[1]), pack_bf16x2(ya[2], ya[3]),
+                                     pack_bf16x2(ya[4], ya[5]), pack_bf16x2(ya[6], ya[7]));
+          const uint4 B = make_uint4(pack_bf16x2(yb[0], yb[1]), pack_bf16x2(yb[2], yb[3]),
+                                     pack_bf16x2(yb[4], yb[5]), pack_bf16x2(yb[6], yb[7]));
+          const int d0 = j * 32 + g * 8;
+          *reinterpret_cast<uint4*>(out + d0) = A;
+          *reinterpret_cast<uint4*>(out + 64 + d0) = B;
+          if (is_k && to_cache) {
+            *reinterpret_cast<uint4*>(kdst + (d0 >> 3) * 64) = A;
+            *reinterpret_cast<uint4*>(kdst + ((d0 + 64) >> 3) * 64) = B;
+          }
+        }
+      }
+    } else {
+      bf16* vdst = p.vc + ((size_t)page * p.hkv + (H - p.hq - p.hkv)) * (BI_PAGE_SIZE * BI_HEAD_DIM) +
+                   (o >> 3) * 64 + (o & 7);
+#pragma unroll 1
+      for (int j = 0; j < 4; ++j) {
+        uint32_t r[32];
+        tmem_ld32(taddr + (hh * 4 + j) * 32, r);
+        tmem_ld_wait();
+        if (!live) continue;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const uint4 V = make_uint4(pack_bf16x2(__uint_as_float(r[8 * g + 0]), __uint_as_float(r[8 * g + 1])),
+                                     pack_bf16x2(__uint_as_float(r[8 * g + 2]), __uint_as_float(r[8 * g + 3])),
+                                     pack_bf16x2(__uint_as_float(r[8 * g + 4]), __uint_as_float(r[8 * g + 5])),
+                                     pack_bf16x2(__uint_as_float(r[8 * g + 6]), __uint_as_float(r[8 * g + 7])));
+          const int d0 = j * 32 + g * 8;
+          *reinterpret_cast<uint4*>(out + d0) = V;
+          if (to_cache) {
+            const bf16* v8 = reinterpret_cast<const bf16*>(&V);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) vdst[((d0 + e) >> 3) * 128 + ((d0 + e) & 7) * 8] = v8[e];
+          }
+        }
+      }
+    }
+  }
+}
 
 template <int TERMS, int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
@@ -363,7 +471,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           store_row_chunk(p, row, col_of(c), r);
         }
       };
-      if (CL == 1) {
+      if constexpr (EPI == EPI_QKV) {
+        qkv_tile(p, row, nb, taddr);  // never split (the host only fuses unsplit weights)
+      } else if (CL == 1) {
 #pragma unroll 1
         for (int q = 0; q < BN / 32; ++q) {
           // SwiGLU pairs gate chunk c with up chunk c + 4
@@ -555,12 +665,27 @@ static bi_status pair_clusters(int* out) {
   return BI_OK;
 }
 
-// N is the output width: the W rows for EPI_STORE / EPI_ADD, the feature
-// count F (W has 2F rows) for EPI_SWIGLU.
+struct QkvArgs {
+  const int32_t* pos;
+  const float* cs;
+  const int32_t* slots;
+  bf16* kc;
+  bf16* vc;
+  int32_t max_pos, num_pages, hq, hkv;
+};
+
+// The fixed K split of a weight: a function of its shape (N, K) only.
+static int split_of(int64_t N, int64_t K, bool swiglu) {
+  const int64_t cols = swiglu ? BN / 2 : BN;
+  return ((N + cols - 1) / cols <= SPLIT_MAX_TILES_N && K >= SPLIT_MIN_K) ? 2 : 1;
+}
+
+// N is the output width: the W rows for EPI_STORE / EPI_ADD / EPI_QKV, the
+// feature count F (W has 2F rows) for EPI_SWIGLU.
 template <int TERMS, int EPI>
 static bi_status launch(const void* A, const void* A2, int64_t lda, const void* W, int64_t ldw,
                         void* C, int64_t ldc, int32_t c_dtype, int64_t M, int64_t N, int64_t K,
-                        cudaStream_t s) {
+                        cudaStream_t s, const QkvArgs* qa = nullptr) {
   bi_status st;
   const int32_t c_f32 = c_dtype != BI_BF16;
   if (K == 0) {
@@ -606,9 +731,19 @@ static bi_status launch(const void* A, const void* A2, int64_t lda, const void* 
   p.n_blocks = (int32_t)((N + cols_per_tile - 1) / cols_per_tile);
   p.k_blocks = (int32_t)((K + BK - 1) / BK);
   p.status = status_word();
+  p.pos = qa ? qa->pos : nullptr;
+  p.cs = qa ? qa->cs : nullptr;
+  p.slots = qa ? qa->slots : nullptr;
+  p.kc = qa ? qa->kc : nullptr;
+  p.vc = qa ? qa->vc : nullptr;
+  p.max_pos = qa ? qa->max_pos : 0;
+  p.num_pages = qa ? qa->num_pages : 0;
+  p.hq = qa ? qa->hq : 0;
+  p.hkv = qa ? qa->hkv : 0;
   if ((st = set_smem_attr<TERMS, EPI>()) != BI_OK) return st;
   // the K split depends on the weight's shape only, never on M
-  p.split = (p.n_blocks <= SPLIT_MAX_TILES_N && K >= SPLIT_MIN_K) ? 2 : 1;
+  p.split = split_of(N, K, EPI == EPI_SWIGLU);
+  if (EPI == EPI_QKV && p.split != 1) return fail(BI_ERR_UNSUPPORTED, "gemm_qkv: split weight");
   p.kb_per_rank = (p.k_blocks + p.split - 1) / p.split;
   const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
   const int sms = num_sms();
@@ -664,6 +799,49 @@ extern "C" bi_status bi_gemm_swiglu(const void* A, int64_t lda, const void* W, i
   if ((st = require_sm100()) != BI_OK) return st;
   return gemm::launch<1, gemm::EPI_SWIGLU>(A, nullptr, lda, W, ldw, out, ldo, BI_BF16, M, F, K,
                                            static_cast<cudaStream_t>(stream));
+}
+
+namespace bi {
+bi_status launch_kv_append(const bf16* k, const bf16* v, int64_t ld_new, const int32_t* slots,
+                           int64_t n_tok, bf16* kc, bf16* vc, int Hkv, int num_pages,
+                           cudaStream_t s);
+bi_status launch_rope(bf16* x, int64_t ldx, int n_heads, const int32_t* pos, int64_t n_tok,
+                      const float* cs, int max_pos, cudaStream_t s);
+}  // namespace bi
+
+extern "C" bi_status bi_gemm_qkv(const void* A, int64_t lda, const void* W, int64_t ldw, void* qkv,
+                                 int64_t ldq, int64_t M, int64_t K, int32_t n_q_heads,
+                                 int32_t n_kv_heads, const int32_t* positions, const float* cos_sin,
+                                 int32_t max_pos, const int32_t* slot_mapping, void* k_cache,
+                                 void* v_cache, int32_t num_pages, void* stream) {
+  if (n_q_heads <= 0 || n_kv_heads <= 0 || n_q_heads > 4096 || n_kv_heads > 4096)
+    return fail(BI_ERR_INVALID_ARG, "gemm_qkv: bad head counts");
+  const int64_t N = (int64_t)(n_q_heads + 2 * n_kv_heads) * BI_HEAD_DIM;
+  bi_status st = gemm::check_args(A, lda, W, ldw, qkv, ldq, BI_BF16, M, N, K);
+  if (st != BI_OK) return st;
+  if (!positions || !cos_sin || !slot_mapping || !k_cache || !v_cache)
+    return fail(BI_ERR_INVALID_ARG, "gemm_qkv: null pointer");
+  if (max_pos <= 0 || num_pages <= 0) return fail(BI_ERR_INVALID_ARG, "gemm_qkv: bad max_pos / num_pages");
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(cos_sin))
+    return fail(BI_ERR_ALIGN, "gemm_qkv: caches and table must be 16-byte aligned");
+  if (M == 0) return BI_OK;
+  if ((st = require_sm100()) != BI_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  bf16* out = static_cast<bf16*>(qkv);
+  if (K == 0 || gemm::split_of(N, K, false) != 1) {
+    // the same steps as three launches: the fused epilogue handles unsplit weights only
+    if ((st = gemm::launch<1, gemm::EPI_STORE>(A, nullptr, lda, W, ldw, qkv, ldq, BI_BF16, M, N, K, s)) != BI_OK)
+      return st;
+    if ((st = launch_rope(out, ldq, n_q_heads + n_kv_heads, positions, M, cos_sin, max_pos, s)) != BI_OK)
+      return st;
+    return launch_kv_append(out + (size_t)n_q_heads * BI_HEAD_DIM,
+                            out + (size_t)(n_q_heads + n_kv_heads) * BI_HEAD_DIM, ldq, slot_mapping, M,
+                            static_cast<bf16*>(k_cache), static_cast<bf16*>(v_cache), n_kv_heads,
+                            num_pages, s);
+  }
+  gemm::QkvArgs qa{positions, cos_sin, slot_mapping, static_cast<bf16*>(k_cache),
+                   static_cast<bf16*>(v_cache), max_pos, num_pages, n_q_heads, n_kv_heads};
+  return gemm::launch<1, gemm::EPI_QKV>(A, nullptr, lda, W, ldw, qkv, ldq, BI_BF16, M, N, K, s, &qa);
 }
 
 extern "C" bi_status bi_gemm_x2(const void* A_hi, const void* A_lo, int64_t lda, const void* W,

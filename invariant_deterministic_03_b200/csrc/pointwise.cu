@@ -137,8 +137,7 @@ __global__ void rope_kernel(bf16* __restrict__ x, int64_t ldx, int n_heads,
   float ra[VEC], rb[VEC];
 #pragma unroll
   for (int j = 0; j < VEC; ++j) {
-    ra[j] = __fsub_rn(__fmul_rn(a[j], c[j]), __fmul_rn(b[j], sn[j]));
-    rb[j] = __fadd_rn(__fmul_rn(b[j], c[j]), __fmul_rn(a[j], sn[j]));
+    rope_rotate(a[j], b[j], c[j], sn[j], ra[j], rb[j]);
   }
   if constexpr (VEC == 8) {
     *reinterpret_cast<uint4*>(row + i0) = make_uint4(pack_bf16x2(ra[0], ra[1]), pack_bf16x2(ra[2], ra[3]),

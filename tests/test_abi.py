@@ -137,3 +137,22 @@ def test_wait_bound_check_host_checks(bi):
     assert bi.lib.bi_check_wait_bound(999, None) == bi.BI_ERR_INVALID_ARG
     assert bi.lib.bi_check_wait_bound((1 << 32) + 1, None) == bi.BI_ERR_INVALID_ARG
     assert b"limit" in bi.lib.bi_last_error()
+
+
+def test_gemm_qkv_host_checks(bi):
+    p = 0x1000
+    g = bi.lib.bi_gemm_qkv
+    ok = dict(A=p, lda=512, W=p, ldw=512, qkv=p, ldq=1024, M=4, K=512, hq=4, hkv=2, pos=p, cs=p,
+              max_pos=64, slots=p, kc=p, vc=p, pages=8, s=None)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return g(a["A"], a["lda"], a["W"], a["ldw"], a["qkv"], a["ldq"], a["M"], a["K"], a["hq"], a["hkv"],
+                 a["pos"], a["cs"], a["max_pos"], a["slots"], a["kc"], a["vc"], a["pages"], a["s"])
+    assert call(hq=0) == bi.BI_ERR_INVALID_ARG
+    assert call(ldq=512) == bi.BI_ERR_SHAPE            # ldq < (4 + 2 * 2) * 128
+    assert call(K=500, lda=504, ldw=504) == bi.BI_ERR_SHAPE   # K % 8
+    assert call(slots=None) == bi.BI_ERR_INVALID_ARG
+    assert call(max_pos=0) == bi.BI_ERR_INVALID_ARG
+    assert call(kc=p + 8) == bi.BI_ERR_ALIGN
+    assert call(M=0) == bi.BI_OK                        # nothing to do
