@@ -217,52 +217,61 @@ __device__ __forceinline__ void qkv_tile(const Params& p, int row, int nb, uint3
   if (live && !rot && nb * 2 < p.hq + p.hkv) set_status(p.status, BI_DEV_BAD_TOKEN);
   const int n_heads = p.hq + 2 * p.hkv;
   bf16* crow = static_cast<bf16*>(p.C) + (size_t)(live ? row : 0) * p.ldc;
+  // q / k heads of this tile rotate with the row's cos / sin: loaded once per
+  // 32-pair block for both heads, before the accumulator reads
+  const int n_rot = max(0, min(2, p.hq + p.hkv - nb * 2));  // leading heads of the tile that rotate
+  const float* csrow = p.cs + (size_t)(rot ? pos : 0) * 128;
 #pragma unroll 1
-  for (int hh = 0; hh < 2; ++hh) {
+  for (int j = 0; j < 2 && n_rot > 0; ++j) {
+    float4 t[16];  // cos / sin of pairs 32 j .. 32 j + 31
+#pragma unroll
+    for (int q = 0; q < 16; ++q)
+      t[q] = (live && rot) ? reinterpret_cast<const float4*>(csrow + j * 64)[q] : make_float4(1.f, 0.f, 1.f, 0.f);
+#pragma unroll 1
+    for (int hh = 0; hh < n_rot; ++hh) {
+      const int H = nb * 2 + hh;
+      const bool is_k = H >= p.hq;
+      bf16* out = crow + (size_t)H * BI_HEAD_DIM;
+      if (j == 0 && is_k && live && slot_bad) set_status(p.status, BI_DEV_BAD_SLOT);
+      bf16* kdst = p.kc + ((size_t)page * p.hkv + (is_k ? H - p.hq : 0)) * (BI_PAGE_SIZE * BI_HEAD_DIM) +
+                   (o >> 3) * 1024 + (o & 7) * 8;
+      uint32_t ra[32], rb[32];  // columns 32 j .. 32 j + 31 and their partners 64 further on
+      tmem_ld32(taddr + (hh * 4 + j) * 32, ra);
+      tmem_ld32(taddr + (hh * 4 + j + 2) * 32, rb);
+      tmem_ld_wait();
+      if (!live) continue;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        float ya[8], yb[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float4 c = t[g * 4 + (e >> 1)];
+          const float a = round_bf16(ra[8 * g + e]), b = round_bf16(rb[8 * g + e]);
+          if (rot) rope_rotate(a, b, (e & 1) ? c.z : c.x, (e & 1) ? c.w : c.y, ya[e], yb[e]);
+          else { ya[e] = a; yb[e] = b; }
+        }
+        const uint4 A = make_uint4(pack_bf16x2(ya[0], ya[1]), pack_bf16x2(ya[2], ya[3]),
+                                   pack_bf16x2(ya[4], ya[5]), pack_bf16x2(ya[6], ya[7]));
+        const uint4 B = make_uint4(pack_bf16x2(yb[0], yb[1]), pack_bf16x2(yb[2], yb[3]),
+                                   pack_bf16x2(yb[4], yb[5]), pack_bf16x2(yb[6], yb[7]));
+        const int d0 = j * 32 + g * 8;
+        *reinterpret_cast<uint4*>(out + d0) = A;
+        *reinterpret_cast<uint4*>(out + 64 + d0) = B;
+        if (is_k && to_cache) {
+          *reinterpret_cast<uint4*>(kdst + (d0 >> 3) * 64) = A;
+          *reinterpret_cast<uint4*>(kdst + ((d0 + 64) >> 3) * 64) = B;
+        }
+      }
+    }
+  }
+  // v heads of this tile: stored and written to the value cache
+#pragma unroll 1
+  for (int hh = n_rot; hh < 2; ++hh) {
     const int H = nb * 2 + hh;
     if (H >= n_heads) break;  // uniform across the warp
     bf16* out = crow + (size_t)H * BI_HEAD_DIM;
-    if (H >= p.hq && live && slot_bad) set_status(p.status, BI_DEV_BAD_SLOT);
-    if (H < p.hq + p.hkv) {
-      const bool is_k = H >= p.hq;
-      bf16* kdst = p.kc + ((size_t)page * p.hkv + (is_k ? H - p.hq : 0)) * (BI_PAGE_SIZE * BI_HEAD_DIM) +
-                   (o >> 3) * 1024 + (o & 7) * 8;
-#pragma unroll 1
-      for (int j = 0; j < 2; ++j) {
-        uint32_t ra[32], rb[32];  // columns 32 j .. 32 j + 31 and their partners 64 further on
-        tmem_ld32(taddr + (hh * 4 + j) * 32, ra);
-        tmem_ld32(taddr + (hh * 4 + j + 2) * 32, rb);
-        tmem_ld_wait();
-        if (!live) continue;
-        const float* csp = p.cs + ((size_t)(rot ? pos : 0) * 64 + j * 32) * 2;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          float ya[8], yb[8];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float4 t = rot ? reinterpret_cast<const float4*>(csp + g * 16)[q] : make_float4(1.f, 0.f, 1.f, 0.f);
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const int e = 2 * q + h2;
-              const float a = round_bf16(ra[8 * g + e]), b = round_bf16(rb[8 * g + e]);
-              if (rot) rope_rotate(a, b, h2 ? t.z : t.x, h2 ? t.w : t.y, ya[e], yb[e]);
-              else { ya[e] = a; yb[e] = b; }
-            }
-          }
-          const uint4 A = make_uint4(pack_bf16x2(ya[0], ya[1]), pack_bf16x2(ya[2], ya[3]),
-                                     pack_bf16x2(ya[4], ya[5]), pack_bf16x2(ya[6], ya[7]));
-          const uint4 B = make_uint4(pack_bf16x2(yb[0], yb[1]), pack_bf16x2(yb[2], yb[3]),
-                                     pack_bf16x2(yb[4], yb[5]), pack_bf16x2(yb[6], yb[7]));
-          const int d0 = j * 32 + g * 8;
-          *reinterpret_cast<uint4*>(out + d0) = A;
-          *reinterpret_cast<uint4*>(out + 64 + d0) = B;
-          if (is_k && to_cache) {
-            *reinterpret_cast<uint4*>(kdst + (d0 >> 3) * 64) = A;
-            *reinterpret_cast<uint4*>(kdst + ((d0 + 64) >> 3) * 64) = B;
-          }
-        }
-      }
-    } else {
+    if (live && slot_bad) set_status(p.status, BI_DEV_BAD_SLOT);
+    {
       bf16* vdst = p.vc + ((size_t)page * p.hkv + (H - p.hq - p.hkv)) * (BI_PAGE_SIZE * BI_HEAD_DIM) +
                    (o >> 3) * 64 + (o & 7);
 #pragma unroll 1
