@@ -31,7 +31,8 @@
 //
 // CTA layout (192 threads, one CTA per SM, persistent over tiles):
 //   warp 0      TMA producer: A [128 x 64] and W [256 x 64] tiles, 128-byte
-//               swizzle, into a 4-stage shared-memory ring (mbarrier full/empty).
+//               swizzle, into a 4-stage shared-memory ring (3 stages with two
+//               A operands; mbarrier full/empty).
 //               Small M (every CTA holds at most one tile, W streams through
 //               fewer SMs than the GPU has): W tiles are also prefetched into
 //               L2 W_PREFETCH stages ahead of the loads, and when M <= 128
@@ -42,8 +43,10 @@
 //   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators);
 //               lane 0 issues the MMAs and tcgen05.commit's
 //   warps 2..5  epilogue: tcgen05.ld the accumulator row by row (thread = row),
-//               round to bf16 (RNE) or keep fp32, store to global; then free
-//               the accumulator for the tile after next.
+//               round to bf16 (RNE) or keep fp32, store to global, or run one
+//               of the fused epilogues (EPI_ADD, EPI_SWIGLU, EPI_QKV below)
+//               on the finished values; then free the accumulator for the
+//               tile after next.
 // Every mbarrier wait is bounded (see common.cuh); a timeout sets a status
 // bit and the CTA winds down, releasing its tensor memory.
 #include <mutex>
