@@ -5,7 +5,10 @@
 // attention (split + ordered merge) -> O GEMM (fp32 out) -> residual add ->
 // RMSNorm -> gate/up GEMM -> SwiGLU -> down GEMM (fp32 out) -> residual add.
 // Then the final RMSNorm of the rows that want logits and the LM-head GEMM
-// with fp32 logits, and optionally the greedy argmax.
+// with fp32 logits, and optionally the greedy argmax. In the bf16 mode the
+// residual adds and SwiGLU run in the GEMM epilogues, and so do RoPE and the
+// cache append when the QKV projection has a tile for every SM; each fused
+// step keeps the separate kernel's rounding points, so the bits are the same.
 //
 // Every kernel computes each row (token) with an order that depends only on
 // that row's data and, for attention, on its sequence's cache, so a
