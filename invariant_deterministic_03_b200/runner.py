@@ -80,6 +80,13 @@ def make_batch(kv: PagedKV, chunks, tokens_of, device="cuda:0", decode_first: bo
     of `chunks`. With decode_first, one-token chunks are laid out first and
     counted in n_decode, so their attention runs in the decode kernel (a row's
     bits do not depend on which kernel or which batch position computes it)."""
+    if not chunks:
+        raise ValueError("empty batch")
+    for seq, s, e in chunks:
+        if e <= s:
+            raise ValueError(f"sequence {seq}: empty chunk {s}..{e}")
+    if len({seq for seq, _, _ in chunks}) != len(chunks):
+        raise ValueError("a sequence appears twice in one step")
     order = list(range(len(chunks)))
     n_decode = 0
     if decode_first:

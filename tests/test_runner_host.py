@@ -70,3 +70,18 @@ def test_make_batch_puts_one_token_chunks_first():
     assert b["logits_rows"].tolist() == [9, 0, 1]        # logits stay in the order of `chunks`
     b2 = runner.make_batch(kv, chunks, lambda s: toks, device="cpu", decode_first=False)
     assert b2["n_decode"] == 0 and b2["logits_rows"].tolist() == [7, 8, 9]
+
+
+def test_make_batch_rejects_malformed_steps():
+    kv = _kv(num_pages=64)
+    kv.ensure(0, 10)
+    kv.length[0] = 10
+    toks = list(range(100))
+    with pytest.raises(ValueError):
+        runner.make_batch(kv, [], lambda s: toks, device="cpu")
+    with pytest.raises(ValueError):
+        runner.make_batch(kv, [(0, 10, 10)], lambda s: toks, device="cpu")       # no tokens
+    with pytest.raises(ValueError):
+        runner.make_batch(kv, [(0, 10, 11), (0, 11, 12)], lambda s: toks, device="cpu")  # twice
+    with pytest.raises(ValueError):
+        runner.make_batch(kv, [(0, 9, 11)], lambda s: toks, device="cpu")        # cache holds 10
