@@ -18,10 +18,13 @@ Two independent views of every operation:
 bf16 tensors cross into the oracle as uint16 bit patterns or as float64
 arrays that hold bf16 values exactly (:func:`oracle.fp64.bf16_bits_to_f64`).
 
-Parity status: every function of :mod:`oracle.fp64` except ``forward`` is
-pinned by ``tests/test_oracle_pins.py`` against closed forms, exact rational
+Parity status: every function of :mod:`oracle.fp64` is pinned by
+``tests/test_oracle_pins.py`` against closed forms, exact rational
 arithmetic, brute force or the worked examples printed in "Defeating
-Nondeterminism in LLM Inference". ``forward`` is pinned only structurally
-(causality, identity blocks, one-token closed form): the pages print no logits
-for any model, so its end-to-end values are "parity unpinned".
+Nondeterminism in LLM Inference". ``forward`` is pinned structurally there
+(causality, identity blocks, one-token closed form) and end to end by
+``tests/test_oracle_forward_library.py`` against an independent library
+implementation of the same architecture (the ``transformers`` Mistral model
+in float64, same weights: agreement ~1e-6). The pages print no logits for
+any model, so no pin reproduces a number of theirs for it.
 """

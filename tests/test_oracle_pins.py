@@ -325,7 +325,7 @@ def test_argmax_ties_lowest_index():
 
 
 # ---------------------------------------------------------------------------
-# forward: structural pins (end-to-end values are parity unpinned)
+# forward: structural pins (end to end: tests/test_oracle_forward_library.py)
 
 def _tiny_cfg(L=2):
     return dict(n_layers=L, d_model=256, n_q_heads=2, n_kv_heads=1, d_ff=96,
