@@ -1,6 +1,8 @@
-"""The oracle's decoder forward against an independent implementation of the
-same architecture: the Mistral model of the `transformers` library, run in
-float64 on the CPU with the same weights (no GPU, no network).
+"""The oracle against independent library implementations, on the CPU (no
+GPU, no network): its decoder forward against the Mistral model of the
+`transformers` library run in float64 with the same weights, its attention
+against torch's float64 scaled_dot_product_attention, and its RMSNorm
+against torch's rms_norm.
 
 The forward the oracle writes out (pre-norm RMSNorm, rotate-half RoPE with
 theta 1e4 at absolute positions, grouped-query causal attention with q head
@@ -90,3 +92,33 @@ def test_library_comparison_catches_a_planted_mistake():
     with torch.no_grad():
         lib = _library_model(w)(torch.tensor([tokens])).logits[0].numpy()
     assert np.abs(ours - lib).max() > 1e-2
+
+
+def test_oracle_attention_matches_torch_sdpa():
+    """Causal GQA attention of a prefill chunk (queries at positions 37..63
+    over keys 0..63, Hq 8 / Hkv 2) against torch's float64
+    scaled_dot_product_attention with the same inclusive causal mask and the
+    same contiguous head grouping."""
+    rng = np.random.default_rng(5)
+    L, n, hq, hkv, d = 64, 27, 8, 2, 128
+    q = rng.standard_normal((n, hq, d))
+    k = rng.standard_normal((L, hkv, d))
+    v = rng.standard_normal((L, hkv, d))
+    pos = np.arange(L - n, L)
+    scale = 1.0 / np.sqrt(d)
+    ours, _ = fp64.attention(q, k, v, pos, scale)
+    qt = torch.from_numpy(q).permute(1, 0, 2)[None]                  # [1, Hq, n, d]
+    kt = torch.from_numpy(k).permute(1, 0, 2).repeat_interleave(hq // hkv, 0)[None]
+    vt = torch.from_numpy(v).permute(1, 0, 2).repeat_interleave(hq // hkv, 0)[None]
+    mask = torch.from_numpy(np.arange(L)[None, :] <= pos[:, None])     # [n, L], True = attend
+    lib = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=scale)
+    lib = lib[0].permute(1, 0, 2).numpy()
+    assert np.abs(ours - lib).max() <= 1e-12
+
+
+def test_oracle_rmsnorm_matches_torch():
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((9, 256)) * rng.uniform(0.01, 100, size=(9, 1))
+    g = rng.uniform(0.5, 1.5, size=256)
+    lib = torch.nn.functional.rms_norm(torch.from_numpy(x), (256,), torch.from_numpy(g), eps=1e-6).numpy()
+    assert np.abs(fp64.rmsnorm(x, g, 1e-6) - lib).max() <= 1e-12 * np.abs(lib).max()
