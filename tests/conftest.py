@@ -18,4 +18,7 @@ def cuda_device():
     import torch
     if not torch.cuda.is_available():
         pytest.fail("gpu test collected without a CUDA device")
+    # libbi.so in-tree, compiled only if a source is newer than it
+    from invariant_deterministic_03_b200 import build
+    build.build()
     return torch.device("cuda:0")

@@ -3,16 +3,24 @@ allocation, prefix sharing between sequences and reference-counted release,
 and the batch assembly's slot arithmetic."""
 import pytest
 
-from invariant_deterministic_03_b200 import runner
+
+@pytest.fixture(scope="module")
+def runner():
+    # the runner imports the ctypes binding, which wants libbi.so on disk
+    # (it is only loaded, never called, here)
+    from invariant_deterministic_03_b200 import build
+    build.build()
+    from invariant_deterministic_03_b200 import runner as mod
+    return mod
 
 
-def _kv(num_pages=32):
+def _kv(runner, num_pages=32):
     return runner.PagedKV(n_layers=1, num_pages=num_pages, n_kv_heads=1, max_pages_per_seq=16, seed=3,
                           device="cpu")
 
 
-def test_pages_come_from_a_seeded_permutation():
-    a, b = _kv(), _kv()
+def test_pages_come_from_a_seeded_permutation(runner):
+    a, b = _kv(runner), _kv(runner)
     a.ensure(0, 40)
     b.ensure(0, 40)
     assert a.pages[0] == b.pages[0] and len(a.pages[0]) == 3
@@ -20,8 +28,8 @@ def test_pages_come_from_a_seeded_permutation():
     assert a.slot(0, 17) == a.pages[0][1] * 16 + 1
 
 
-def test_fork_shares_whole_pages_only():
-    kv = _kv()
+def test_fork_shares_whole_pages_only(runner):
+    kv = _kv(runner)
     kv.ensure(0, 50)
     kv.length[0] = 50
     held = kv.fork(0, 1, 45)                      # 45 tokens: two whole pages
@@ -37,8 +45,8 @@ def test_fork_shares_whole_pages_only():
         kv.fork(0, 1, 16)
 
 
-def test_release_frees_a_page_when_its_last_holder_goes():
-    kv = _kv()
+def test_release_frees_a_page_when_its_last_holder_goes(runner):
+    kv = _kv(runner)
     kv.ensure(0, 64)
     kv.length[0] = 64
     kv.fork(0, 1, 64)
@@ -49,14 +57,14 @@ def test_release_frees_a_page_when_its_last_holder_goes():
     assert len(kv.free) == n_free + 4 and not kv.refs
 
 
-def test_out_of_pages_is_an_error():
-    kv = _kv(num_pages=2)
+def test_out_of_pages_is_an_error(runner):
+    kv = _kv(runner, num_pages=2)
     with pytest.raises(RuntimeError):
         kv.ensure(0, 33)
 
 
-def test_make_batch_puts_one_token_chunks_first():
-    kv = _kv(num_pages=64)
+def test_make_batch_puts_one_token_chunks_first(runner):
+    kv = _kv(runner, num_pages=64)
     for seq, n in [(0, 20), (1, 5), (2, 40)]:
         kv.ensure(seq, n)
         kv.length[seq] = n
@@ -72,8 +80,8 @@ def test_make_batch_puts_one_token_chunks_first():
     assert b2["n_decode"] == 0 and b2["logits_rows"].tolist() == [7, 8, 9]
 
 
-def test_make_batch_rejects_malformed_steps():
-    kv = _kv(num_pages=64)
+def test_make_batch_rejects_malformed_steps(runner):
+    kv = _kv(runner, num_pages=64)
     kv.ensure(0, 10)
     kv.length[0] = 10
     toks = list(range(100))
