@@ -288,3 +288,118 @@ def forward(weights: ModelWeights, tokens, depths=None):
     if depths is not None:
         return cut
     return head(x)
+
+
+# --------------------------------------------------------------------------
+# the forward with the storage roundings of a mixed-precision implementation
+
+def round_to(x, kind):
+    """x rounded to a storage format, returned in float64.
+
+    kind: None (kept in float64), "f32" (IEEE float32, nearest even),
+    "bf16" (bfloat16, nearest even) or "bf16x2" (an fp32 value carried as a
+    pair hi = bf16(v), lo = bf16(v - hi), v = f32(x); the value is hi + lo).
+    Pure encoding: no arithmetic of the method.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    if kind is None:
+        return x
+    if kind == "f32":
+        return x.astype(np.float32).astype(np.float64)
+    if kind == "bf16":
+        return bf16_bits_to_f64(f64_to_bf16_bits(x))
+    if kind == "bf16x2":
+        v = x.astype(np.float32).astype(np.float64)
+        hi = bf16_bits_to_f64(f64_to_bf16_bits(v))
+        lo = bf16_bits_to_f64(f64_to_bf16_bits(v - hi))
+        return hi + lo
+    raise ValueError(f"unknown storage format {kind!r}")
+
+
+# Storage format of each activation of the decoder forward, per precision
+# mode. The modes are the cross-vendor precision study's variants
+# (arXivDaily 2610.05458, abstract): all-bf16 activations, the full fp32
+# upcast, and the upcast with only the MLP blocks kept in bf16. READING: the
+# pages name the variants, not where each rounds; these are the points at
+# which a kernel stack stores an activation in a narrower format than fp64:
+#   h        RMSNorm output feeding a GEMM (attention block: "h_attn",
+#            MLP block: "h_mlp", final: "h_final")
+#   qkv      the QKV projection's output
+#   qk_rope  q and k after RoPE
+#   p        the unnormalised softmax weights exp(s - m) fed to P V (and
+#            summed into the softmax denominator)
+#   attn     the attention output feeding the O projection
+#   gu       gate and up projection outputs; act: silu(g) * u
+#   resid    the residual stream after each addition
+#   logits   the LM head's output
+ROUNDING = {
+    "bf16": dict(h_attn="bf16", qkv="bf16", qk_rope="bf16", p="bf16", attn="bf16",
+                 h_mlp="bf16", gu="bf16", act="bf16", resid="f32", h_final="bf16", logits="f32"),
+    "f32": dict(h_attn="bf16x2", qkv="f32", qk_rope="f32", p="f32", attn="bf16x2",
+                h_mlp="bf16x2", gu="f32", act="bf16x2", resid="f32", h_final="bf16x2", logits="f32"),
+    "bf16_mlp": dict(h_attn="bf16x2", qkv="f32", qk_rope="f32", p="f32", attn="bf16x2",
+                     h_mlp="bf16", gu="bf16", act="bf16", resid="f32", h_final="bf16x2", logits="f32"),
+}
+
+
+def attention_rounded(q, k, v, q_pos, scale: float, p_kind):
+    """attention() with the softmax weights exp(s - m) rounded to `p_kind`
+    before both the weighted sum of the values and the denominator (m the
+    row maximum): out = sum_j P_j v_j / sum_j P_j, P_j = round(exp(s_j - m))."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    n, hq, d = q.shape
+    L, hkv, _ = k.shape
+    group = hq // hkv
+    q_pos = np.asarray(q_pos, dtype=np.int64)
+    masked = np.arange(L)[None, :] > q_pos[:, None]
+    out = np.zeros((n, hq, d))
+    for h in range(hq):
+        g = h // group
+        s = (q[:, h, :] @ k[:, g, :].T) * scale
+        s = np.where(masked, -np.inf, s)
+        P = round_to(np.exp(s - np.max(s, axis=-1, keepdims=True)), p_kind)
+        out[:, h, :] = (P @ v[:, g, :]) / np.sum(P, axis=-1, keepdims=True)
+    return out
+
+
+def forward_rounded(weights: ModelWeights, tokens, rounding=None):
+    """forward() with each activation stored in the format `rounding` names
+    (a dict as in ROUNDING, or a mode name; None: every point kept in
+    float64, which is forward() itself). Every operation is the float64
+    definition; only the stored values are rounded."""
+    if isinstance(rounding, str):
+        rounding = ROUNDING[rounding]
+    r = dict.fromkeys(ROUNDING["bf16"], None)
+    if rounding:
+        r.update(rounding)
+    c = weights.cfg
+    D, hq, hkv, dh = c["d_model"], c["n_q_heads"], c["n_kv_heads"], 128
+    F = c["d_ff"]
+    eps, theta = c["rms_eps"], c["rope_theta"]
+    tokens = np.asarray(tokens, dtype=np.int64)
+    n = tokens.shape[0]
+    pos = np.arange(n)
+    scale = 1.0 / np.sqrt(dh)
+    x = round_to(weights.get("embed")[tokens], r["resid"])
+    for layer in range(c["n_layers"]):
+        h = round_to(rmsnorm(x, weights.get("attn_norm", layer), eps), r["h_attn"])
+        qkv = round_to(gemm(h, weights.get("w_qkv", layer)), r["qkv"])
+        q = qkv[:, : hq * dh].reshape(n, hq, dh)
+        k = qkv[:, hq * dh:(hq + hkv) * dh].reshape(n, hkv, dh)
+        v = qkv[:, (hq + hkv) * dh:].reshape(n, hkv, dh)
+        q = round_to(rope(q, pos, theta), r["qk_rope"])
+        k = round_to(rope(k, pos, theta), r["qk_rope"])
+        if r["p"] is None:
+            a, _ = attention(q, k, v, pos, scale)
+        else:
+            a = attention_rounded(q, k, v, pos, scale, r["p"])
+        a = round_to(a.reshape(n, hq * dh), r["attn"])
+        x = round_to(x + gemm(a, weights.get("w_o", layer)), r["resid"])
+        h = round_to(rmsnorm(x, weights.get("mlp_norm", layer), eps), r["h_mlp"])
+        gu = round_to(gemm(h, weights.get("w_gate_up", layer)), r["gu"])
+        act = round_to(swiglu(gu[:, :F], gu[:, F:]), r["act"])
+        x = round_to(x + gemm(act, weights.get("w_down", layer)), r["resid"])
+    h = round_to(rmsnorm(x, weights.get("final_norm"), eps), r["h_final"])
+    return round_to(gemm(h, weights.get("lm_head")), r["logits"])

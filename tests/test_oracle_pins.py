@@ -422,3 +422,192 @@ def test_bf16_rounding_helper():
     assert np.isinf(back[5])                  # past the largest finite bf16
     assert back[6] == pytest.approx(1e-40, rel=2 ** -6)
     assert np.isinf(back[7])
+
+
+# ---------------------------------------------------------------------------
+# The fixed float32 order of ordered.rmsnorm_f32 and ordered.attention_f32,
+# emulated bit for bit: every float32 operation of the C code is redone here
+# with exactly one rounding (fmaf exactly, through rational arithmetic; the
+# other operations with numpy float32 scalars, which round once; expf through
+# the same libm function the C oracle calls). Planted mistakes of order must
+# then fail to match, so the pins can tell orders apart.
+
+import ctypes  # noqa: E402
+
+_libm = ctypes.CDLL("libm.so.6")
+_libm.expf.restype = ctypes.c_float
+_libm.expf.argtypes = [ctypes.c_float]
+
+
+def _f32_nearest(q: Fraction) -> np.float32:
+    """The float32 nearest to the rational q (ties to even)."""
+    if q == 0:
+        return np.float32(0.0)
+    sign = -1 if q < 0 else 1
+    q = abs(q)
+    e = q.numerator.bit_length() - q.denominator.bit_length()
+    if Fraction(2) ** e > q:
+        e -= 1                                       # now 2^e <= q < 2^(e+1)
+    quantum = Fraction(2) ** (max(e, -126) - 23)     # 24 significant bits
+    n = q / quantum
+    fl = n.numerator // n.denominator
+    rem = n - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    return np.float32(sign * float(fl * quantum))
+
+
+def _fma(a, b, c) -> np.float32:
+    return _f32_nearest(Fraction(float(a)) * Fraction(float(b)) + Fraction(float(c)))
+
+
+def _rmsnorm_row_emulated(x, g, eps, order=None, fused=True, group_r_gamma=False):
+    D = len(x)
+    ss = np.float32(0.0)
+    for j in (range(D) if order is None else order):
+        ss = _fma(x[j], x[j], ss) if fused else np.float32(x[j] * x[j]) + ss
+    r = np.float32(1.0) / np.sqrt(ss / np.float32(D) + np.float32(eps))
+    if group_r_gamma:
+        return np.array([x[j] * (r * g[j]) for j in range(D)], dtype=np.float32)
+    return np.array([(x[j] * r) * g[j] for j in range(D)], dtype=np.float32)
+
+
+def test_rmsnorm_f32_order_bitwise():
+    """ordered.rmsnorm_f32: ss = fmaf(x_j, x_j, ss) for j = 0 .. D-1, then
+    r = 1 / sqrtf(ss / D + eps), y_j = (x_j r) g_j -- equal bit for bit to
+    the emulation; a reversed sum, an unfused multiply-add and x (r g) each
+    change some outputs."""
+    rng = np.random.default_rng(21)
+    M, D = 32, 48
+    X = (rng.standard_normal((M, D)) * np.exp(rng.uniform(-3, 3, (M, D)))).astype(np.float32)
+    g = rng.uniform(0.5, 1.5, D).astype(np.float32)
+    eps = 1e-6
+    y = ordered.rmsnorm_f32(X, g, eps)
+    want = np.stack([_rmsnorm_row_emulated(X[i], g, eps) for i in range(M)])
+    assert np.array_equal(y.view(np.uint32), want.view(np.uint32))
+    planted = {
+        "reversed sum": [_rmsnorm_row_emulated(X[i], g, eps, order=range(D - 1, -1, -1)) for i in range(M)],
+        "mul then add": [_rmsnorm_row_emulated(X[i], g, eps, fused=False) for i in range(M)],
+        "x (r g)": [_rmsnorm_row_emulated(X[i], g, eps, group_r_gamma=True) for i in range(M)],
+    }
+    for name, rows in planted.items():
+        assert not np.array_equal(np.stack(rows).view(np.uint32), y.view(np.uint32)), name
+
+
+def _attention_emulated(q, k, v, q_pos, scale, l_order="forward", one_pass=False):
+    n, hq, d = q.shape
+    hkv = k.shape[1]
+    group = hq // hkv
+    sc = np.float32(scale)
+    out = np.zeros((n, hq, d), np.float32)
+    for i in range(n):
+        last = int(q_pos[i])
+        for h in range(hq):
+            gg = h // group
+            s = []
+            for j in range(last + 1):
+                acc = np.float32(0.0)
+                for e in range(d):
+                    acc = _fma(q[i, h, e], k[j, gg, e], acc)
+                s.append(np.float32(acc * sc))
+            if one_pass:
+                # a running maximum with rescaling (an online softmax): a
+                # different order of operations from the two passes
+                m, l = np.float32(-np.inf), np.float32(0.0)
+                o = [np.float32(0.0)] * d
+                for j in range(last + 1):
+                    mn = max(m, s[j])
+                    a = np.float32(_libm.expf(float(np.float32(m - mn)))) if m != -np.inf else np.float32(0.0)
+                    p = np.float32(_libm.expf(float(np.float32(s[j] - mn))))
+                    l = np.float32(a * l) + p
+                    o = [_fma(p, v[j, gg, e], np.float32(a * o[e])) for e in range(d)]
+                    m = mn
+            else:
+                m = np.float32(-np.inf)
+                for j in range(last + 1):
+                    if s[j] > m:
+                        m = s[j]
+                p = [np.float32(_libm.expf(float(np.float32(s[j] - m)))) for j in range(last + 1)]
+                l = np.float32(0.0)
+                for j in (range(last + 1) if l_order == "forward" else range(last, -1, -1)):
+                    l = l + p[j]
+                o = [np.float32(0.0)] * d
+                for j in range(last + 1):
+                    o = [_fma(p[j], v[j, gg, e], o[e]) for e in range(d)]
+            out[i, h] = [o[e] / l for e in range(d)]
+    return out
+
+
+def test_attention_f32_order_bitwise():
+    """ordered.attention_f32: s_j = fmaf-dot(q, k_j) over d in order, times
+    scale; the maximum over all visible keys first; then p_j = expf(s_j - m),
+    l += p_j and o += p_j v_j (fmaf) for j = 0 .. p; o / l. Equal bit for bit
+    to the emulation; the denominator summed backwards, and a one-pass
+    online softmax, each change some outputs."""
+    rng = np.random.default_rng(22)
+    L, hq, hkv, d = 14, 2, 1, 8
+    q = (rng.standard_normal((3, hq, d)) * 2).astype(np.float32)
+    k = rng.standard_normal((L, hkv, d)).astype(np.float32)
+    v = rng.standard_normal((L, hkv, d)).astype(np.float32)
+    pos = [5, 9, 13]
+    got = ordered.attention_f32(q, k, v, pos, 0.35)
+    want = _attention_emulated(q, k, v, pos, 0.35)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+    for kw in ({"l_order": "backward"}, {"one_pass": True}):
+        assert not np.array_equal(_attention_emulated(q, k, v, pos, 0.35, **kw).view(np.uint32),
+                                  got.view(np.uint32)), kw
+
+
+# ---------------------------------------------------------------------------
+# forward_rounded: the fp64 forward with each activation stored in a narrower
+# format (the basis of the bf16 forward's tolerance)
+
+def test_round_to_formats():
+    x = np.array([1.0 + 2 ** -9 + 2 ** -20, -3.0e-3, 0.1, 1e-30])
+    np.testing.assert_array_equal(fp64.round_to(x, "bf16"), fp64.bf16_bits_to_f64(fp64.f64_to_bf16_bits(x)))
+    np.testing.assert_array_equal(fp64.round_to(x, "f32"), x.astype(np.float32).astype(np.float64))
+    np.testing.assert_array_equal(fp64.round_to(x, None), x)
+    # hi + lo carries 16 significant bits: error below 2^-16 relative, and
+    # exact for a value that already has that many
+    y = fp64.round_to(x, "bf16x2")
+    assert np.all(np.abs(y - x) <= 2.0 ** -16 * np.abs(x))
+    assert fp64.round_to(np.array([1.0 + 2 ** -15]), "bf16x2")[0] == 1.0 + 2 ** -15
+
+
+def test_forward_rounded_without_rounding_is_forward():
+    cfg = _tiny_cfg()
+    w = _tiny_weights(cfg, seed=7)
+    toks = [3, 1, 4, 1, 5, 9]
+    assert np.array_equal(fp64.forward_rounded(w, toks, None), fp64.forward(w, toks))
+    assert np.array_equal(fp64.forward_rounded(w, toks, {}), fp64.forward(w, toks))
+
+
+def test_forward_rounded_every_point_is_live():
+    """Each storage point, rounded alone to bf16, moves the logits (a point
+    the function silently skipped would leave them unchanged), and all of
+    the bf16 mode together moves them by about the quadrature sum of the
+    single points' errors (independent roundings add in quadrature)."""
+    cfg = _tiny_cfg()
+    w = _tiny_weights(cfg, seed=8)
+    toks = [7, 2, 40, 11, 2, 33, 19, 5]
+    ref = fp64.forward(w, toks)
+    sq = 0.0
+    for point in fp64.ROUNDING["bf16"]:
+        err = fp64.forward_rounded(w, toks, {point: "bf16"}) - ref
+        assert np.max(np.abs(err)) > 0, point
+        sq += np.sum(err ** 2)
+    all_err = fp64.forward_rounded(w, toks, dict.fromkeys(fp64.ROUNDING["bf16"], "bf16")) - ref
+    ratio = np.sum(all_err ** 2) / sq
+    assert 0.5 < ratio < 2.0, ratio
+
+
+def test_forward_rounded_modes_order():
+    """fp32 activations (hi/lo pairs into the GEMMs) are far closer to fp64
+    than bf16 activations; bf16 MLP blocks alone fall in between."""
+    cfg = _tiny_cfg()
+    w = _tiny_weights(cfg, seed=9)
+    toks = list(range(1, 30, 3))
+    ref = fp64.forward(w, toks)
+    e = {m: np.max(np.abs(fp64.forward_rounded(w, toks, m) - ref)) for m in fp64.ROUNDING}
+    assert e["f32"] < e["bf16_mlp"] < e["bf16"]
+    assert e["f32"] < 1e-2 * e["bf16"]
