@@ -40,8 +40,10 @@ MS = [1 << i for i in range(13)]                 # 1 .. 4096
 COPIES = 3
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # dram__bytes_read.sum + dram__bytes_write.sum of one gemm_tcgen05_kernel<1, 0>
-# launch at M=4096 K=4096 N=14336 (profiles/gemm_tcgen05_m4096_k4096_n14336.md)
-GEMM_TRAFFIC_BYTES = 155.467776e6 + 100.073216e6
+# launch at M=4096 K=4096 N=14336 (profiles/gemm_tcgen05_m4096_k4096_n14336.md);
+# None until the current kernel has been captured
+GEMM_TRAFFIC_BYTES = None
+RMS_MS = [1 << i for i in range(13)] + [16384, 65536]   # RMSNorm bandwidth sweep, D = 4096
 
 
 def parse():
@@ -53,8 +55,8 @@ def parse():
     ap.add_argument("--no-extras", action="store_true", help="skip attention/RMSNorm/cuBLAS legs")
     ap.add_argument("--study", default=None, choices=["precision", "depth"],
                     help="precision study: all-bf16 vs fp32 upcast vs bf16-MLP-only decoder")
-    ap.add_argument("--case", default=None, choices=["gemm", "gemm_m128", "gemm_split", "attn", "rmsnorm",
-                                                     "forward"],
+    ap.add_argument("--case", default=None, choices=["gemm", "gemm_m128", "gemm_k14336", "attn",
+                                                     "attn_prefill", "rmsnorm", "forward"],
                     help="run 3 launches of one kernel on its workload and exit (for profilers)")
     return ap.parse_args()
 
@@ -311,8 +313,23 @@ def prefill_attention_leg(bi, torch, synth, reps):
     cu = torch.tensor([0, 2048, 4096, 6144, 8192], dtype=torch.int32, device="cuda")
     ms = per_launch_ms(torch, lambda r=0: bi.bi_attn_prefill(q, cu, 2048, kc, vc, bt, sl, shape, out, ws), reps)
     flops = 4.0 * 32 * 128 * sum(L * (L + 1) / 2 for L in lens)
-    return {"workload": "prefill, 4 x 2048-token prompts, causal, Hq=32, Hkv=8, d=128",
-            "ms": ms, "tflops": flops / ms / 1e9}
+    res = {"workload": "prefill, 4 x 2048-token prompts, causal, Hq=32, Hkv=8, d=128",
+           "ms": ms, "tflops": flops / ms / 1e9}
+    # torch SDPA on the same prompts with K / V gathered into contiguous
+    # [batch, heads, keys, d] tensors (GQA by enable_gqa): a non-invariant
+    # cost reference, not part of the path
+    try:
+        qs = torch.randn(4, 32, 2048, 128, device="cuda", generator=g).to(torch.bfloat16)
+        ks = torch.randn(4, 8, 2048, 128, device="cuda", generator=g).to(torch.bfloat16)
+        vs = torch.randn(4, 8, 2048, 128, device="cuda", generator=g).to(torch.bfloat16)
+        F = torch.nn.functional
+        fn = lambda r=0: F.scaled_dot_product_attention(qs, ks, vs, is_causal=True, enable_gqa=True)  # noqa: E731
+        tms = per_launch_ms(torch, fn, reps)
+        res["torch_sdpa"] = {"kernel": "torch scaled_dot_product_attention (causal, enable_gqa, contiguous K/V)",
+                             "ms": tms, "tflops": flops / tms / 1e9}
+    except Exception as e:  # noqa: BLE001
+        res["torch_sdpa"] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
+    return res
 
 
 def flash_decode_leg(torch, synth, reps):
@@ -428,6 +445,10 @@ def forward_leg(torch, reps):
 
 
 def rmsnorm_leg(bi, torch, reps):
+    """bi_rmsnorm at 65536 x 4096 (the HBM-bound claim), torch's rms_norm on
+    the same tensors as the non-invariant cost reference, and the bandwidth
+    sweep over M in {1, 2, 4, ..., 4096, 16384, 65536} at D = 4096 with each
+    smaller M's rows compared bitwise with the same rows at M = 65536."""
     M, D = 65536, 4096
     g = torch.Generator("cuda").manual_seed(2)
     x = torch.randn(M, D, device="cuda", generator=g).to(torch.bfloat16)
@@ -435,7 +456,26 @@ def rmsnorm_leg(bi, torch, reps):
     y = torch.empty_like(x)
     ms = per_launch_ms(torch, lambda r=0: bi.bi_rmsnorm(x, gamma, y, 1e-6), reps)
     by = 4.0 * M * D + 2 * D
-    return {"workload": "M=65536, D=4096 bf16", "ms": ms, "bytes": by, "gbs": by / ms / 1e6}
+    yt = torch.empty_like(x)
+    tms = per_launch_ms(torch, lambda r=0: yt.copy_(torch.nn.functional.rms_norm(x, (D,), gamma, 1e-6)), reps)
+    tms_only = per_launch_ms(torch, lambda r=0: torch.nn.functional.rms_norm(x, (D,), gamma, 1e-6), reps)
+    sweep, bitwise = [], True
+    for m in RMS_MS:
+        xm, ym = x[:m], y[:m]
+        t = per_launch_ms(torch, lambda r=0, xm=xm, ym=ym: bi.bi_rmsnorm(xm, gamma, ym, 1e-6), reps)
+        b = 4.0 * m * D + 2 * D
+        sweep.append({"M": m, "ms": round(t, 5), "gbs": round(b / t / 1e6, 1)})
+    full = torch.empty_like(x)
+    bi.bi_rmsnorm(x, gamma, full, 1e-6)
+    for m in RMS_MS:
+        part = torch.empty(m, D, dtype=torch.bfloat16, device="cuda")
+        bi.bi_rmsnorm(x[:m], gamma, part, 1e-6)
+        bitwise &= same_bits(part, full[:m])
+    return {"workload": "M=65536, D=4096 bf16", "ms": ms, "bytes": by, "gbs": by / ms / 1e6,
+            "torch_rms_norm": {"kernel": "torch.nn.functional.rms_norm (bf16, not batch-invariant by contract)",
+                               "ms": tms_only, "gbs": by / tms_only / 1e6,
+                               "ms_with_copy_into_preallocated": tms},
+            "sweep_d4096": sweep, "sweep_rows_bitwise_across_M": bool(bitwise)}
 
 
 def e2e_leg(bi, torch, sw, steps):
@@ -502,53 +542,136 @@ def e2e_leg(bi, torch, sw, steps):
     return ms, h2d, d2h
 
 
-def cpu_baseline_leg(target_s=10.0):
-    """The oracle's fp64 GEMM (numpy matmul) on a bounded sample of the sweep
-    workload: the first r rows of A for both shapes, r sized for ~10 s."""
+def _cpu_inputs():
+    """Seeded synthetic inputs of the CPU samples, as the float32 arrays the
+    C oracle reads (bf16 values, so they are the GPU workload's values)."""
     import numpy as np
-    import torch
-    from oracle import fp64
     from invariant_deterministic_03_b200 import synth
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
-    except Exception:
-        threads = os.cpu_count()
-    mats = {}
+    from oracle import fp64
+
+    def f32(t):
+        return fp64.bf16_bits_to_f64(synth.bf16_bits(t)).astype(np.float32)
+    d = {"W": {(K, N): f32(synth.normal_bf16((N, K), 0.02, 7 + K)) for K, N in SHAPES},
+         "A": {K: f32(synth.normal_bf16((64, K), 1.0, 8 + K)) for K, _ in SHAPES},
+         "x1": f32(synth.normal_bf16((64, 512), 1.0, 0)),
+         "g1": f32(synth.uniform_bf16((512,), 0.5, 1.5, 1000)),
+         "w1": f32(synth.normal_bf16((512, 1024), 1.0 / math.sqrt(512), 2)).T.copy(),
+         "x4096": f32(synth.normal_bf16((4096, 4096), 1.0, 3)),
+         "g4096": f32(synth.uniform_bf16((4096,), 0.5, 1.5, 4))}
+    return d
+
+
+def cpu_gemm_sample(ordered, d, threads, rows_per_thread):
+    """The fixed-order C oracle's GEMM (fmaf left to right over k, one output
+    element per thread) on the first `threads * rows_per_thread` rows of A
+    for both sweep shapes. Returns (flops, seconds, rows)."""
+    ordered.set_threads(threads)
+    rows = threads * rows_per_thread
+    t0 = time.perf_counter()
+    flops = 0.0
     for K, N in SHAPES:
-        W = fp64.bf16_bits_to_f64(synth.bf16_bits(synth.normal_bf16((N, K), 0.02, 7)))
-        A = fp64.bf16_bits_to_f64(synth.bf16_bits(synth.normal_bf16((512, K), 1.0, 8)))
-        mats[(K, N)] = (A, W)
-    rows, spent, flops, passes = 512, 0.0, 0.0, 0
-    t_start = time.perf_counter()
-    while spent < target_s:
-        for (K, N), (A, W) in mats.items():
-            fp64.gemm(A[:rows], W)
-            flops += 2.0 * rows * N * K
-        passes += 1
-        spent = time.perf_counter() - t_start
-    return {"value": flops / spent / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": f"oracle fp64 GEMM (numpy matmul) of the first {rows} rows of A against W for both "
-                      f"sweep shapes, repeated {passes} times, {spent:.1f} s of CPU work"}
+        ordered.gemm_f32(d["A"][K][:rows], d["W"][(K, N)])
+        flops += 2.0 * rows * N * K
+    return flops, time.perf_counter() - t0, rows
+
+
+def cpu_baseline_leg():
+    """The oracle's fixed-order float32 C path (oracle/ordered.c) timed on this
+    host's cores, at one thread and at all of them, on bounded samples of the
+    workloads: C1 (RMSNorm then GEMM, 64 x 512 -> 1024, whole), C1' (RMSNorm,
+    D = 4096, a 4096-row sample), C2 (the GEMM sweep, a row sample of both
+    shapes: rows below 256, as the small-M launches have), C3 (decode
+    attention over the 32 sequences of lengths U[1, 8192]: a 4-sequence
+    sample at one thread, all 32 at all cores). ~20 s of CPU work."""
+    import numpy as np
+    from invariant_deterministic_03_b200 import synth
+    from oracle import ordered
+    cores = ordered.max_threads()
+    d = _cpu_inputs()
+    legs = {}
+    # C2: GEMM sweep rows
+    fl1, t1, r1 = cpu_gemm_sample(ordered, d, 1, 2)
+    flA, tA, rA = cpu_gemm_sample(ordered, d, cores, 2)
+    legs["c2_gemm"] = {"unit": "TFLOP/s", "one_thread": fl1 / t1 / 1e12, "all_cores": flA / tA / 1e12,
+                       "sample": f"rows 0..{r1 - 1} (1 thread) and 0..{rA - 1} ({cores} threads) of A "
+                                 "against W for (K=4096,N=14336) and (K=14336,N=4096)"}
+    # C1: RMSNorm then GEMM, whole
+    c1 = {}
+    for th in (1, cores):
+        ordered.set_threads(th)
+        t0 = time.perf_counter()
+        reps = 5
+        for _ in range(reps):
+            n = ordered.rmsnorm_f32(d["x1"], d["g1"], 1e-6)
+            ordered.gemm_f32(n, d["w1"])
+        c1[th] = (time.perf_counter() - t0) / reps
+    legs["c1_rmsnorm_gemm"] = {"unit": "us", "one_thread": c1[1] * 1e6, "all_cores": c1[cores] * 1e6,
+                               "sample": "whole: X[64,512], gamma[512], W[512,1024] (5 repetitions)"}
+    # C1': RMSNorm bandwidth, algorithmic bf16 bytes (4 M D + 2 D) / time
+    rm = {}
+    for th in (1, cores):
+        ordered.set_threads(th)
+        t0 = time.perf_counter()
+        ordered.rmsnorm_f32(d["x4096"], d["g4096"], 1e-6)
+        rm[th] = time.perf_counter() - t0
+    by = 4.0 * 4096 * 4096 + 2 * 4096
+    legs["c1p_rmsnorm"] = {"unit": "GB/s", "one_thread": by / rm[1] / 1e9, "all_cores": by / rm[cores] / 1e9,
+                           "sample": "4096 rows of D = 4096 (bytes counted as the bf16 op's 4 M D + 2 D)"}
+    # C3: decode attention, algorithmic K/V bytes (L x 8 x 128 x 2 x 2 per sequence)
+    lens = synth.attention_lengths(32, 1, 8192, seed=0)
+    rng = np.random.default_rng(0)
+    q = rng.standard_normal((1, 32, 128)).astype(np.float32)
+    kv = rng.standard_normal((8192, 8, 128)).astype(np.float32)
+    at = {}
+    for th, seqs in ((1, lens[:4]), (cores, lens)):
+        ordered.set_threads(th)
+        t0 = time.perf_counter()
+        for L in seqs:
+            ordered.attention_f32(q, kv[:L], kv[:L], [L - 1], 1.0 / math.sqrt(128), threads=th)
+        at[th] = (sum(seqs) * 8 * 128 * 2 * 2, time.perf_counter() - t0)
+    legs["c3_decode_attention"] = {"unit": "GB/s", "one_thread": at[1][0] / at[1][1] / 1e9,
+                                   "all_cores": at[cores][0] / at[cores][1] / 1e9,
+                                   "sample": f"sequences of lengths {lens[:4]} (1 thread); all 32 ({cores} threads)"}
+    ordered.set_threads(cores)
+    return {"value": legs["c2_gemm"]["all_cores"], "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": (f"fixed-order float32 C oracle (fmaf left to right), GEMM sweep row sample "
+                       f"({legs['c2_gemm']['sample']}), {cores} threads; 1-thread and the C1, C1', C3 "
+                       "figures under legs"),
+            "legs": legs}
 
 
 # --------------------------------------------------------------------------- main
 
 def run_reference(args):
+    """The reference arm: the oracle (fixed-order float32 C path) on the
+    host's cores, each step a bounded row sample of the GEMM sweep."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    cb = cpu_baseline_leg(target_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)))
-    line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "TFLOP/s",
+    from oracle import ordered
+    d = _cpu_inputs()
+    cores = ordered.max_threads()
+    for _ in range(args.warmup):
+        cpu_gemm_sample(ordered, d, cores, 1)
+    fl = sec = 0.0
+    for _ in range(args.steps):
+        f, t, rows = cpu_gemm_sample(ordered, d, cores, 1)
+        fl += f
+        sec += t
+    value = fl / sec / 1e12
+    sample = (f"fixed-order float32 C oracle GEMM, rows 0..{rows - 1} of A against W for both sweep "
+              f"shapes per step, {cores} threads")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "ms_per_step": sec / max(1, args.steps) * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": "gemm sweep, Mistral-7B MLP shapes: M in 1..4096 (powers of 2) x "
-                                   "(K=4096,N=14336) and (K=14336,N=4096); oracle runs a bounded row sample",
+                                   "(K=4096,N=14336) and (K=14336,N=4096); the oracle runs a bounded row sample",
                        "world_size": world},
-            "cpu_baseline": cb,
-            "e2e": {"value": cb["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -574,10 +697,9 @@ def run_case(case):
         assert bi.bi_device_status(clear=True) == 0
         print("case forward: ok")
         return 0
-    if case in ("gemm", "gemm_m128", "gemm_split"):
-        # gemm_split: the K = 14336, N = 4096 weight, which takes the two-way K split
-        M = {"gemm": 4096, "gemm_m128": 128, "gemm_split": 2048}[case]
-        K, N = (14336, 4096) if case == "gemm_split" else (4096, 14336)
+    if case in ("gemm", "gemm_m128", "gemm_k14336"):
+        M = {"gemm": 4096, "gemm_m128": 128, "gemm_k14336": 2048}[case]
+        K, N = (14336, 4096) if case == "gemm_k14336" else (4096, 14336)
         A = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
         W = (torch.randn(N, K, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
         C = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
@@ -593,6 +715,18 @@ def run_case(case):
         out = torch.empty(32, 32 * 128, dtype=torch.bfloat16, device="cuda")
         bt, sl = lay.block_table.cuda(), torch.tensor(lens, dtype=torch.int32, device="cuda")
         fn = lambda: bi.bi_attn_decode(q, kc, vc, bt, sl, shape, out, ws)  # noqa: E731
+    elif case == "attn_prefill":
+        lens = [2048] * 4
+        lay = synth.PagedLayout(lens, seed=0)
+        kc = torch.randn(lay.num_pages, 8, 16, 128, device="cuda", generator=g).to(torch.bfloat16)
+        vc = torch.randn(lay.num_pages, 8, 128, 16, device="cuda", generator=g).to(torch.bfloat16)
+        q = torch.randn(8192, 32 * 128, device="cuda", generator=g).to(torch.bfloat16)
+        shape = bi.attn_shape(32, 8, lay.num_pages, lay.pages_per_seq, 4096)
+        ws = torch.empty(bi.bi_attn_workspace_size(shape, 8192), dtype=torch.uint8, device="cuda")
+        out = torch.empty(8192, 32 * 128, dtype=torch.bfloat16, device="cuda")
+        bt, sl = lay.block_table.cuda(), torch.tensor(lens, dtype=torch.int32, device="cuda")
+        cu = torch.tensor([0, 2048, 4096, 6144, 8192], dtype=torch.int32, device="cuda")
+        fn = lambda: bi.bi_attn_prefill(q, cu, 2048, kc, vc, bt, sl, shape, out, ws)  # noqa: E731
     else:
         x = torch.randn(65536, 4096, device="cuda", generator=g).to(torch.bfloat16)
         gamma = torch.rand(4096, device="cuda", generator=g).to(torch.bfloat16)
@@ -650,10 +784,12 @@ def run_depth_study(n_tok=16, depths=(1, 2, 4, 8, 16, 32)):
 
 def run_precision_study(n_prompts=512, prompt_len=256, oracle_prompts=4):
     """4-layer d=2048, 16-head (MHA), FFN 5632, vocab 32000 random-init decoder
-    (std 0.02), 512 random prompts of 256 tokens, run in the three activation
-    precisions. Runtime: the whole workload on the GPU (prefill, device time).
-    Error: logits of every position of `oracle_prompts` prompts against the
-    fp64 oracle forward (teacher forced)."""
+    (std 0.02), 512 random prompts of 256 tokens, run in the four activation
+    precisions (bf16, fp16 -- the same weights converted to fp16 --, fp32
+    upcast, bf16 MLP only). Runtime: the whole workload on the GPU (prefill,
+    device time). Error: logits of every position of `oracle_prompts` prompts
+    against the fp64 oracle forward of the bf16 weights (teacher forced; the
+    fp16 variant's error includes its weights' conversion)."""
     import numpy as np
     import torch
     from invariant_deterministic_03_b200 import runner, synth
@@ -669,9 +805,11 @@ def run_precision_study(n_prompts=512, prompt_len=256, oracle_prompts=4):
            "modes": {}}
     ref = [fp64.forward(fp64.ModelWeights(cfg, {k: synth.bf16_bits(v) for k, v in w.items()}), prompts[i])
            for i in range(oracle_prompts)]
-    for mode in ["bf16", "f32", "bf16_mlp"]:
+    wd16 = {k: v.to(torch.float16) for k, v in wd.items()}
+    for mode in ["bf16", "f16", "f32", "bf16_mlp"]:
         c = dict(cfg, precision=mode)
-        eng = runner.Engine(c, wd, num_pages=per_step * prompt_len // 16 + 64, max_pages_per_seq=prompt_len // 16,
+        wm = wd16 if mode == "f16" else wd
+        eng = runner.Engine(c, wm, num_pages=per_step * prompt_len // 16 + 64, max_pages_per_seq=prompt_len // 16,
                             max_tokens=per_step * prompt_len, max_logits=per_step, seed=0)
         # logits of every position for the oracle prompts: one token per step
         errs, top1, top5 = [], [], []
@@ -687,7 +825,7 @@ def run_precision_study(n_prompts=512, prompt_len=256, oracle_prompts=4):
             top5.append(np.mean([len(set(t5g[j].tolist()) & set(t5r[j].tolist())) / 5 for j in range(prompt_len)]))
             eng.kv.release(10_000 + i)
         # runtime: the whole workload as prefill, 64 prompts per step
-        eng2 = runner.Engine(c, wd, num_pages=per_step * prompt_len // 16 + 64, max_pages_per_seq=prompt_len // 16,
+        eng2 = runner.Engine(c, wm, num_pages=per_step * prompt_len // 16 + 64, max_pages_per_seq=prompt_len // 16,
                              max_tokens=per_step * prompt_len, max_logits=per_step, seed=1)
         def one_pass():
             for s0 in range(0, n_prompts, per_step):
@@ -752,20 +890,27 @@ def main():
     big = [r for r in table if r["M"] >= 1024]
     big_fl = sum(2.0 * r["M"] * r["N"] * r["K"] for r in big)
     big_ms = sum(r["bi_ms"] for r in big)
-    peak_t = peaks.get("bf16_tflops_sustained") or peaks.get("bf16_tflops")
-    # the dominant kernel's largest launch of the step (M=4096, K=4096, N=14336):
-    # the launch the committed ncu capture measured
+    # each launch below is timed alone by CUDA events, so its roofline is the
+    # burst peak; the sustained figure is reported beside it
+    peak_t = peaks.get("bf16_tflops") or peaks.get("bf16_tflops_sustained")
+    peak_sus = peaks.get("bf16_tflops_sustained")
+    # the dominant kernel's largest launch of the step (M=4096, K=4096, N=14336)
     top = [r for r in table if r["M"] == 4096 and r["K"] == 4096][0]
     achieved = 2.0 * top["M"] * top["N"] * top["K"] / top["bi_ms"] / 1e9
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
                 "frac": achieved / peak_t, "traffic": GEMM_TRAFFIC_BYTES,
                 "kernel": "bi_gemm (gemm_tcgen05_kernel<1, 0>), launch M=4096 K=4096 N=14336",
                 "algorithmic_bytes": 2.0 * (top["M"] * top["K"] + top["N"] * top["K"] + top["M"] * top["N"]),
-                "peak_source": f"{peak_src} bf16 dense sustained",
-                "frac_of_burst": achieved / peaks.get("bf16_tflops", peak_t)}
-    extras["roofline_m_ge_1024"] = {"achieved": big_fl / big_ms / 1e9, "unit": "TFLOP/s",
-                                    "frac": big_fl / big_ms / 1e9 / peak_t,
-                                    "launches": "M in {1024, 2048, 4096} x both shapes"}
+                "peak_source": f"{peak_src} bf16 dense burst (launch timed alone)",
+                "frac_of_sustained": achieved / peak_sus if peak_sus else None}
+    per_launch = [{"M": r["M"], "K": r["K"], "N": r["N"], "tflops": round(r["bi_tflops"], 1),
+                   "frac": round(r["bi_tflops"] / peak_t, 3), "meets_0.70": r["bi_tflops"] / peak_t >= 0.70}
+                  for r in big]
+    agg = big_fl / big_ms / 1e9
+    extras["roofline_m_ge_1024"] = {"achieved": agg, "unit": "TFLOP/s", "peak": peak_t,
+                                    "frac": agg / peak_t, "meets_0.70": agg / peak_t >= 0.70,
+                                    "launches": "M in {1024, 2048, 4096} x both shapes, each timed alone",
+                                    "per_launch": per_launch}
     bi_sum = sum(r["bi_ms"] for r in table)
     th_sum = sum(r["cublas_ms"] for r in table)
     extras["sweep"] = [{k: (round(v, 4) if isinstance(v, float) else v) for k, v in r.items()} for r in table]
@@ -781,6 +926,7 @@ def main():
         extras["attn_decode"] = a
         pa = prefill_attention_leg(bi, torch, synth, reps=5)
         pa["frac"] = pa["tflops"] / peak_t
+        pa["peak"] = peak_t
         extras["attn_prefill"] = pa
         extras["rmsnorm"] = r
         extras["invariance"] = invariance_flags(torch, sw)
@@ -802,8 +948,9 @@ def main():
                 "config": {"workload": "gemm sweep, Mistral-7B MLP shapes: M in {1,2,4,...,4096} x "
                                        "(K=4096,N=14336) and (K=14336,N=4096), bf16 in, fp32 accum, bf16 out",
                            "l2": "inputs larger than L2: weights rotate over 3 copies of 117 MB per shape",
-                           "tile": ("128x256x64, tcgen05 M128 N256 K16, one tiling for all M; K=14336 N=4096 "
-                                    "takes a fixed two-way K split (two-CTA cluster) at every M"),
+                           "tile": ("256x256x64 output tile per CTA pair (two-CTA cluster, 128 rows each), "
+                                    "tcgen05.mma.cta_group::2 M256 N256 K16; one tiling for every M, N, K; "
+                                    "no split-K, no stream-K"),
                            "parallelism": f"replicas x{world}"},
                 "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
                 "e2e": {"value": whole_job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",

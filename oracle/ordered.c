@@ -176,4 +176,29 @@ void attention_f32(const float* q, const float* k, const float* v,
   }
 }
 
+/* ---- threads ------------------------------------------------------------- */
+
+/* OpenMP threads the parallel loops above use (timing only: every output
+ * element is computed by one thread in the order written, so the results do
+ * not depend on it). */
+#ifdef _OPENMP
+extern void omp_set_num_threads(int);
+extern int omp_get_max_threads(void);
+#endif
+void ordered_set_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
+int ordered_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
 int ordered_abi_version(void) { return 1; }

@@ -46,6 +46,8 @@ def lib() -> ctypes.CDLL:
         _lib.gemm_f32.argtypes = [p, p, p, i64, i64, i64]
         _lib.attention_f32.argtypes = [p, p, p, p, i64, i64, i64, i64, i64,
                                        f32, p, p, i64]
+        _lib.ordered_set_threads.argtypes = [ctypes.c_int]
+        _lib.ordered_max_threads.restype = ctypes.c_int
     return _lib
 
 
@@ -106,14 +108,25 @@ def gemm_f32(A, W) -> np.ndarray:
     return C
 
 
-def attention_f32(q, k, v, q_pos, scale: float) -> np.ndarray:
+def set_threads(n: int) -> None:
+    """OpenMP threads of the parallel loops (timing only; results do not
+    depend on it)."""
+    lib().ordered_set_threads(int(n))
+
+
+def max_threads() -> int:
+    return int(lib().ordered_max_threads())
+
+
+def attention_f32(q, k, v, q_pos, scale: float, threads: int | None = None) -> np.ndarray:
     q = _c(q, np.float32)
     k = _c(k, np.float32)
     v = _c(v, np.float32)
     pos = _c(q_pos, np.int32)
     n, hq, d = q.shape
     L, hkv, _ = k.shape
-    threads = max(1, os.cpu_count() or 1)
+    if threads is None:
+        threads = max(1, os.cpu_count() or 1)
     scratch = np.empty((threads, max(L, 1)), np.float32)
     out = np.empty_like(q)
     lib().attention_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(pos), n, L, hq, hkv, d,
