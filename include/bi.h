@@ -20,7 +20,10 @@
  *    non-BI_OK return nothing was enqueued and bi_last_error() (thread-local)
  *    holds a one-line reason.
  *  - No entry point allocates device memory. Scratch space is a caller-owned
- *    workspace whose size comes from the matching *_workspace_size query.
+ *    workspace whose size comes from the matching *_workspace_size query,
+ *    with one exception: bi_attn_decode_noalloc takes no workspace and uses
+ *    a fixed static device array of the library instead, shared by all calls
+ *    on a device.
  *  - Data that only the device can see (page ids, slot ids, sequence lengths)
  *    is range-checked inside the kernels: an out-of-range value skips the
  *    access and sets a bit of the library's device status word, read with
@@ -62,7 +65,7 @@ typedef enum { BI_BF16 = 0, BI_F32 = 1, BI_F32_ADD = 2 } bi_dtype;
 #define BI_PAGE_SIZE 16   /* tokens per KV-cache page */
 #define BI_ATTN_TILE 128  /* keys per attention tile, at absolute key offsets */
 #define BI_ATTN_SPLIT 512 /* keys per KV split (fixed split SIZE, not count) */
-#define BI_GEMM_BM 128    /* GEMM output tile rows */
+#define BI_GEMM_BM 256    /* GEMM output tile rows (a CTA pair, 128 rows each) */
 #define BI_GEMM_BN 256    /* GEMM output tile columns */
 #define BI_GEMM_BK 64     /* GEMM K stage */
 
@@ -120,20 +123,32 @@ bi_status bi_rmsnorm_f32in(const float* x, const void* gamma, void* y,
  *
  * A [M, K] bf16 (row stride lda), W [N, K] bf16 (row stride ldw), C [M, N]
  * (row stride ldc) bf16 (c_dtype = BI_BF16, round-to-nearest-even) or fp32
- * (BI_F32). Products are exact, accumulation is fp32 in tensor memory, one
- * tcgen05.mma kind::f16 shape (128 x 256 x 16), K walked 0, 16, 32, ... in
- * order whatever M is. Needs K % 8 == 0, N % 8 == 0, lda/ldw/ldc % 8 == 0,
- * A, W, C 16-byte aligned. M == 0 or N == 0 is a no-op. K == 0 writes zeros. */
+ * (BI_F32). Products are exact, accumulation is fp32 in tensor memory. One
+ * configuration for every shape: 256 x 256 output tiles, each computed by a
+ * pair of CTAs (a two-CTA cluster, 128 rows each) with one tcgen05.mma
+ * kind::f16 shape (cta_group::2, 256 x 256 x 16), K walked 0, 16, 32, ... in
+ * order inside the pair whatever M is. Needs K % 8 == 0, N % 8 == 0,
+ * lda/ldw/ldc % 8 == 0, A, W, C 16-byte aligned. M == 0 or N == 0 is a
+ * no-op. K == 0 writes zeros. */
 bi_status bi_gemm(const void* A, int64_t lda, const void* W, int64_t ldw,
                   void* C, int64_t ldc, int32_t c_dtype, int64_t M, int64_t N,
                   int64_t K, void* stream);
+
+/* bi_gemm with fp16 A and W (C fp16 for BI_BF16's slot, i.e. the 16-bit
+ * output, or fp32 / fp32-add): the GEMM of the FP16 variant of the
+ * cross-vendor paper's precision study (arXiv 2610.05458, abstract). The
+ * same tiles, instruction shape (kind::f16 with fp16 operands) and K order;
+ * the same constraints. */
+bi_status bi_gemm_f16(const void* A, int64_t lda, const void* W, int64_t ldw,
+                      void* C, int64_t ldc, int32_t c_dtype, int64_t M,
+                      int64_t N, int64_t K, void* stream);
 
 /* Gate/up projection with the SwiGLU activation in its epilogue. W is
  * [2F, K] (row stride ldw): gate rows 0..F-1, then up rows F..2F-1, as a
  * fused nn.Linear. out [M, F] bf16 (row stride ldo):
  *   g = bf16(A Wg^T), u = bf16(A Wu^T) exactly as bi_gemm computes them,
  *   out = bf16(g / (1 + e^-g) * u) in fp32 (the same steps as bi_swiglu).
- * Each 128 x 256 tile holds 128 gate and the matching 128 up columns, so the
+ * Each 256 x 256 tile holds 128 gate and the matching 128 up columns, so the
  * per-element reduction is bi_gemm's, whatever M is. Constraints as bi_gemm
  * with N = F. */
 bi_status bi_gemm_swiglu(const void* A, int64_t lda, const void* W,
@@ -149,9 +164,8 @@ bi_status bi_gemm_swiglu(const void* A, int64_t lda, const void* W,
  *   bi_kv_append(k heads of qkv, v heads of qkv, ldq, slot_mapping, M, ...);
  * i.e. qkv holds the rotated q and k heads and the plain v heads, and row
  * m's k and v heads are in the caches at slot_mapping[m] (skipped when < 0;
- * outside the cache: skipped and BI_DEV_BAD_SLOT). One launch when the
- * weight takes no K split (every weight with K < 8192 or more than 37
- * column tiles); otherwise the three steps run as three launches. cos_sin
+ * outside the cache: skipped and BI_DEV_BAD_SLOT). One launch (K == 0: the
+ * zeros, then the RoPE and append steps as separate launches). cos_sin
  * [max_pos, 64, 2] fp32 from bi_rope_table; caches as for bi_kv_append
  * (num_pages pages, Hkv heads). Constraints as bi_gemm; caches and cos_sin
  * 16-byte aligned. M == 0 is a no-op. */
@@ -338,8 +352,9 @@ bi_status bi_argmax(const float* logits, int64_t rows, int64_t V, int64_t ld,
 
 /* C = (A_hi + A_lo) W^T: both terms meet the same bf16 W tile; per output
  * element, each 64-wide K stage adds its 4 hi K-steps then its 4 lo K-steps,
- * stages in K order. One fixed configuration for every shape (128 x 256
- * tile). Same constraints as bi_gemm; A_hi and A_lo share lda. */
+ * stages in K order. One fixed configuration for every shape (bi_gemm's
+ * 256 x 256 CTA-pair tile). Same constraints as bi_gemm; A_hi and A_lo
+ * share lda. */
 bi_status bi_gemm_x2(const void* A_hi, const void* A_lo, int64_t lda,
                      const void* W, int64_t ldw, void* C, int64_t ldc,
                      int32_t c_dtype, int64_t M, int64_t N, int64_t K,
@@ -375,10 +390,16 @@ bi_status bi_attn_f32(const float* q, int64_t ldq, const int32_t* cu_q,
  * logits. precision selects the activation path:
  *   BI_PREC_BF16      bf16 activations, bf16 KV cache (bi_kv_layout)
  *   BI_PREC_F32       fp32 activations everywhere, fp32 KV cache
- *   BI_PREC_BF16_MLP  fp32 activations except the MLP block, fp32 KV cache */
+ *   BI_PREC_BF16_MLP  fp32 activations except the MLP block, fp32 KV cache
+ *   BI_PREC_F16       the bf16 path with fp16 in place of bf16 everywhere:
+ *                     fp16 weights (all arrays of bi_model_weights), fp16
+ *                     activations and KV cache (bi_kv_layout), fp16 P in
+ *                     attention; the FP16 variant of the cross-vendor
+ *                     paper's precision study (arXiv 2610.05458, abstract) */
 #define BI_PREC_BF16 0
 #define BI_PREC_F32 1
 #define BI_PREC_BF16_MLP 2
+#define BI_PREC_F16 3
 typedef struct {
   int32_t n_layers;
   int32_t d_model;     /* D */
@@ -392,7 +413,8 @@ typedef struct {
   int32_t precision; /* BI_PREC_* */
 } bi_model_config;
 
-/* Caller-owned device weights, bf16, nn.Linear layout [out, in]. Per layer l
+/* Caller-owned device weights, bf16 (fp16 for BI_PREC_F16), nn.Linear layout
+ * [out, in]. Per layer l
  * the arrays hold n_layers consecutive blocks:
  *   attn_norm [L][D], w_qkv [L][(Hq + 2 Hkv) * 128][D] (rows: q heads, then k
  *   heads, then v heads), w_o [L][D][Hq * 128], mlp_norm [L][D],
@@ -454,7 +476,8 @@ bi_status bi_forward_workspace_size(const bi_model* m, int64_t max_tokens,
 
 /* k_cache / v_cache: num_layers consecutive caches, layer l at offset
  * l * num_pages * Hkv * 16 * 128 elements; bf16 in bi_kv_layout for
- * BI_PREC_BF16, fp32 [num_pages, Hkv, 16, 128] (k and v alike) otherwise. logits
+ * BI_PREC_BF16, fp16 in bi_kv_layout for BI_PREC_F16, fp32 [num_pages, Hkv,
+ * 16, 128] (k and v alike) otherwise. logits
  * [n_logits, V] fp32; next_tokens [n_logits] int32 (nullable) = greedy argmax. */
 bi_status bi_forward(const bi_model* m, const bi_batch* batch, void* k_cache,
                      void* v_cache, int32_t num_pages, float* logits,

@@ -30,10 +30,10 @@ lib = ctypes.CDLL(LIB_PATH)
 BI_OK, BI_ERR_INVALID_ARG, BI_ERR_SHAPE, BI_ERR_ALIGN, BI_ERR_WORKSPACE, \
     BI_ERR_UNSUPPORTED, BI_ERR_CUDA, BI_ERR_DEVICE_CHECK = range(8)
 BI_BF16, BI_F32, BI_F32_ADD = 0, 1, 2
-BI_PREC_BF16, BI_PREC_F32, BI_PREC_BF16_MLP = 0, 1, 2
-PRECISIONS = {"bf16": BI_PREC_BF16, "f32": BI_PREC_F32, "bf16_mlp": BI_PREC_BF16_MLP}
+BI_PREC_BF16, BI_PREC_F32, BI_PREC_BF16_MLP, BI_PREC_F16 = 0, 1, 2, 3
+PRECISIONS = {"bf16": BI_PREC_BF16, "f32": BI_PREC_F32, "bf16_mlp": BI_PREC_BF16_MLP, "f16": BI_PREC_F16}
 HEAD_DIM, PAGE_SIZE, ATTN_TILE, ATTN_SPLIT = 128, 16, 128, 512
-GEMM_BM, GEMM_BN, GEMM_BK = 128, 256, 64
+GEMM_BM, GEMM_BN, GEMM_BK = 256, 256, 64
 
 _p, _i32, _i64, _f32, _f64, _sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64,
                                    ctypes.c_float, ctypes.c_double, ctypes.c_size_t)
@@ -75,6 +75,7 @@ _SIGS = {
     "bi_rmsnorm": (_i32, [_p, _p, _p, _i64, _i64, _f32, _p]),
     "bi_rmsnorm_f32in": (_i32, [_p, _p, _p, _i64, _i64, _f32, _p]),
     "bi_gemm": (_i32, [_p, _i64, _p, _i64, _p, _i64, _i32, _i64, _i64, _i64, _p]),
+    "bi_gemm_f16": (_i32, [_p, _i64, _p, _i64, _p, _i64, _i32, _i64, _i64, _i64, _p]),
     "bi_gemm_swiglu": (_i32, [_p, _i64, _p, _i64, _p, _i64, _i64, _i64, _i64, _p]),
     "bi_gemm_qkv": (_i32, [_p, _i64, _p, _i64, _p, _i64, _i64, _i64, _i32, _i32, _p, _p, _i32, _p, _p, _p,
                            _i32, _p]),
@@ -157,16 +158,23 @@ def bi_rmsnorm(x, gamma, y, eps: float, stream=None) -> None:
 
 def bi_gemm(A, W, C, stream=None, add: bool = False) -> None:
     """C = A W^T (or, add=True with fp32 C, C += A W^T). A [M, K] bf16, W [N, K]
-    bf16, C [M, N] bf16 or fp32 (row strides taken from the tensors)."""
+    bf16, C [M, N] bf16 or fp32 (row strides taken from the tensors). fp16 A
+    and W go to bi_gemm_f16 (C fp16 or fp32)."""
     M, K = A.shape
     N = W.shape[0]
+    f16 = A.dtype == torch.float16
+    if (W.dtype == torch.float16) != f16:
+        raise ValueError("bi_gemm: A and W must both be bf16 or both fp16")
     cdt = BI_F32 if C.dtype == torch.float32 else BI_BF16
+    if cdt == BI_BF16 and C.dtype != A.dtype:
+        raise ValueError("bi_gemm: a 16-bit C must have A's type")
     if add:
         if cdt != BI_F32:
             raise ValueError("bi_gemm(add=True) needs an fp32 C")
         cdt = BI_F32_ADD
-    _chk("bi_gemm", lib.bi_gemm(_ptr(A), A.stride(0), _ptr(W), W.stride(0), _ptr(C), C.stride(0),
-                                cdt, M, N, K, _stream(stream)))
+    fn = "bi_gemm_f16" if f16 else "bi_gemm"
+    _chk(fn, getattr(lib, fn)(_ptr(A), A.stride(0), _ptr(W), W.stride(0), _ptr(C), C.stride(0),
+                              cdt, M, N, K, _stream(stream)))
 
 
 def bi_gemm_swiglu(A, W, out, stream=None) -> None:
@@ -258,9 +266,34 @@ def bi_attn_workspace_size(shape: AttnShape, max_tokens: int) -> int:
     return n.value
 
 
+def _check_attn_args(q, k_cache, v_cache, block_table, seq_lens, shape: AttnShape, out, n_rows: int,
+                     where: str) -> None:
+    """Host-side agreement of the tensors with the shape fields the kernels
+    trust (the kernels range-check only what the device alone can see)."""
+    B = seq_lens.shape[0]
+    width = shape.num_q_heads * HEAD_DIM
+    if q.shape[0] < n_rows or out.shape[0] < n_rows:
+        raise ValueError(f"{where}: q / out have fewer than {n_rows} rows")
+    if q.shape[-1] < width or out.shape[-1] < width or q.stride(-1) != 1 or out.stride(-1) != 1:
+        raise ValueError(f"{where}: q / out rows must hold {width} contiguous elements")
+    for name, c in (("k_cache", k_cache), ("v_cache", v_cache)):
+        if c.shape[0] < shape.num_pages or not c.is_contiguous():
+            raise ValueError(f"{where}: {name} holds fewer than num_pages={shape.num_pages} pages "
+                             "or is not contiguous")
+        if c.numel() < shape.num_pages * shape.num_kv_heads * PAGE_SIZE * HEAD_DIM:
+            raise ValueError(f"{where}: {name} smaller than num_pages x num_kv_heads blocks")
+    if block_table.dim() != 2 or block_table.shape[0] < B or block_table.shape[1] < shape.max_pages_per_seq \
+            or block_table.stride(0) != shape.max_pages_per_seq or block_table.stride(1) != 1:
+        raise ValueError(f"{where}: block_table must be [>= B, max_pages_per_seq] with row stride "
+                         f"max_pages_per_seq={shape.max_pages_per_seq}")
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError(f"{where}: block_table and seq_lens must be int32")
+
+
 def bi_attn_decode(q, k_cache, v_cache, block_table, seq_lens, shape: AttnShape, out, ws,
                    stream=None) -> None:
     B = seq_lens.shape[0]
+    _check_attn_args(q, k_cache, v_cache, block_table, seq_lens, shape, out, B, "bi_attn_decode")
     _chk("bi_attn_decode", lib.bi_attn_decode(
         _ptr(q), q.stride(0), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens), B,
         ctypes.byref(shape), _ptr(out), out.stride(0), _ptr(ws),
@@ -272,6 +305,7 @@ def bi_attn_decode_noalloc(q, k_cache, v_cache, block_table, seq_lens, shape: At
     """bi_attn_decode without a workspace argument: for callers that cannot
     allocate device memory; uses the library's fixed 16 MiB device scratch."""
     B = seq_lens.shape[0]
+    _check_attn_args(q, k_cache, v_cache, block_table, seq_lens, shape, out, B, "bi_attn_decode_noalloc")
     _chk("bi_attn_decode_noalloc", lib.bi_attn_decode_noalloc(
         _ptr(q), q.stride(0), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens), B,
         ctypes.byref(shape), _ptr(out), out.stride(0), _stream(stream)))
@@ -280,6 +314,9 @@ def bi_attn_decode_noalloc(q, k_cache, v_cache, block_table, seq_lens, shape: At
 def bi_attn_prefill(q, cu_q, max_q_len: int, k_cache, v_cache, block_table, seq_lens,
                     shape: AttnShape, out, ws, stream=None) -> None:
     B = seq_lens.shape[0]
+    _check_attn_args(q, k_cache, v_cache, block_table, seq_lens, shape, out, q.shape[0], "bi_attn_prefill")
+    if cu_q.shape[0] < B + 1 or cu_q.dtype != torch.int32:
+        raise ValueError("bi_attn_prefill: cu_q must be int32 with B + 1 entries")
     _chk("bi_attn_prefill", lib.bi_attn_prefill(
         _ptr(q), q.stride(0), _ptr(cu_q), max_q_len, q.shape[0], _ptr(k_cache), _ptr(v_cache),
         _ptr(block_table), _ptr(seq_lens), B, ctypes.byref(shape), _ptr(out), out.stride(0),
@@ -323,7 +360,9 @@ def rmsnorm(x, gamma, eps: float):
     return y
 
 
-def gemm(A, W, out_dtype=torch.bfloat16):
+def gemm(A, W, out_dtype=None):
+    if out_dtype is None:
+        out_dtype = A.dtype
     C = torch.empty((A.shape[0], W.shape[0]), dtype=out_dtype, device=A.device)
     bi_gemm(A, W, C)
     return C
@@ -332,13 +371,15 @@ def gemm(A, W, out_dtype=torch.bfloat16):
 def new_kv_cache(num_pages: int, num_kv_heads: int, device, n_layers: int = 1, zero=True,
                  precision: int = BI_PREC_BF16):
     """bf16 mode: k [L, pages, Hkv, 16, 128] and v [L, pages, Hkv, 128, 16] bf16
-    (v transposed per page). fp32 modes: k and v [L, pages, Hkv, 16, 128] fp32."""
+    (v transposed per page); the fp16 mode the same in fp16. fp32 modes: k and
+    v [L, pages, Hkv, 16, 128] fp32."""
     f = torch.zeros if zero else torch.empty
-    if precision != BI_PREC_BF16:
+    if precision in (BI_PREC_F32, BI_PREC_BF16_MLP):
         shp = (n_layers, num_pages, num_kv_heads, PAGE_SIZE, HEAD_DIM)
         return f(shp, dtype=torch.float32, device=device), f(shp, dtype=torch.float32, device=device)
-    k = f((n_layers, num_pages, num_kv_heads, PAGE_SIZE, HEAD_DIM), dtype=torch.bfloat16, device=device)
-    v = f((n_layers, num_pages, num_kv_heads, HEAD_DIM, PAGE_SIZE), dtype=torch.bfloat16, device=device)
+    dt = torch.float16 if precision == BI_PREC_F16 else torch.bfloat16
+    k = f((n_layers, num_pages, num_kv_heads, PAGE_SIZE, HEAD_DIM), dtype=dt, device=device)
+    v = f((n_layers, num_pages, num_kv_heads, HEAD_DIM, PAGE_SIZE), dtype=dt, device=device)
     return k, v
 
 
@@ -351,6 +392,10 @@ class Model:
         self.weights = weights  # keep the tensors alive
         prec = cfg.get("precision", "bf16")
         self.precision = PRECISIONS[prec] if isinstance(prec, str) else int(prec)
+        want = torch.float16 if self.precision == BI_PREC_F16 else torch.bfloat16
+        bad = [n for n, _ in ModelWeights._fields_ if weights[n].dtype != want]
+        if bad:
+            raise ValueError(f"Model: weights {bad} must be {want} for precision {prec!r}")
         c = ModelConfig(cfg["n_layers"], cfg["d_model"], cfg["n_q_heads"], cfg["n_kv_heads"],
                         cfg["d_ff"], cfg["vocab"], cfg["max_pos"], cfg["rms_eps"],
                         cfg["rope_theta"], self.precision)

@@ -67,7 +67,7 @@ def build(force: bool = False, debug: bool = False, verbose: bool = False) -> st
     objs = [os.path.join(BUILD, s.replace(".cu", ".o")) for s in SOURCES]
     if todo or not os.path.exists(LIB):
         cmd = [nvcc(), *ARCH, "-shared", "-cudart", "shared", "-o", LIB, *objs,
-               "-Xlinker", "-rpath=/usr/local/cuda/lib64"]
+               "-Xlinker", "-rpath=/usr/local/cuda/lib64", "-Xlinker", "--no-undefined"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

@@ -16,13 +16,17 @@
 //    pass merges them in split order (section "When are atomic adds
 //    needed?": split reduction plus a serial finishing reduction).
 //
-// Split kernel: one CTA per (split s, sequence b, query block, kv head g).
-// The CTA's 128 MMA rows are (query, q head of group g) pairs. Per tile:
-//   S  = Q K^T            tcgen05.mma M128 N128 K16 x8, fp32 in TMEM
-//   per row (one thread): m' = max(m, max_j s_j log2e*scale), alpha = 2^(m-m'),
-//        P_j = bf16(2^(s_j - m')), l = alpha*l + sum_j P_j (j = 0..127 in order)
-//   PV = P V              tcgen05.mma M128 N128 K16 x8 (one 16-key page per MMA)
-//   O  = fma(alpha, O, PV) per element, in registers.
+// Split kernel: persistent, one CTA per SM, working through items (split s,
+// sequence b, query block, kv head g) claimed at run time. The CTA's 128 MMA
+// rows are (query, q head of group g) pairs. Per 128-key tile:
+//   S  = Q K^T            tcgen05.mma M128 N128 K16 x8, fp32 in tensor memory
+//   per row: m' = the row's reference maximum (log2 domain; see
+//        new_reference), alpha = 2^(m-m'), P_j = bf16(2^(s_j - m')),
+//        l = alpha*l + sum_j P_j (four 32-key quarters, each left to right)
+//   O  = alpha*O          in tensor memory (skipped when alpha == 1)
+//   O += P V              tcgen05.mma M128 N128 K16 x8 (one 16-key page per MMA),
+//                         O accumulated in tensor memory
+// At the end of a split the unnormalised O and (m, l) go to the workspace.
 // A row takes part only in tiles whose first key is <= its position, so the
 // update sequence of a row is a function of (position, split) alone.
 // Masked keys get P = 0 by selection (never by arithmetic on -inf), and
@@ -32,6 +36,8 @@
 // Each (page, kv head) block of the cache is stored in the tensor core's
 // canonical K-major no-swizzle order (8 x 16-byte core matrices), so a tile is
 // 8 + 8 contiguous 4 KB bulk copies straight into MMA operand layout.
+#include <mutex>
+
 #include "common.cuh"
 #include "host.h"
 
@@ -75,8 +81,7 @@ struct Lay {
   static constexpr uint32_t OFF_P = OFF_Q + NQ * QP_BYTES;
   static constexpr uint32_t OFF_BAR = OFF_P + NP * QP_BYTES;
   static constexpr uint32_t OFF_RING = OFF_BAR + 256;   // producer's page-id ring [16 tiles][8 pages]
-  static constexpr uint32_t OFF_RED = OFF_RING + 512;   // decode quarter exchange [2][4 warps][8 heads] fp32
-  static constexpr uint32_t OFF_ITEMS = OFF_RED + 256;  // item ring [16] x 48 B, then one mbarrier per slot
+  static constexpr uint32_t OFF_ITEMS = OFF_RING + 512;  // item ring [16] x 48 B, then one mbarrier per slot
   static constexpr size_t SMEM_BYTES = 1024 + OFF_ITEMS + ITEM_RING * 48 + ITEM_RING * 8;
   static_assert(NK <= MAX_KV_BUF && NV <= MAX_KV_BUF, "barrier arrays hold 3 K and 3 V buffers");
   static_assert(OFF_Q % 1024 == 0 && OFF_P % 1024 == 0, "swizzled Q / P tiles need 1 KB alignment");
@@ -90,8 +95,8 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_O = 384;  // S buffers at [0,128), [128,256) (and in decode [256,384))
 
 struct Params {
-  const uint8_t* kc;  // bf16 key cache, 4 KB per (page, kv head) block
-  const uint8_t* vc;  // bf16 value cache, same blocking
+  const uint8_t* kc;  // 16-bit key cache, 4 KB per (page, kv head) block
+  const uint8_t* vc;  // 16-bit value cache, same blocking
   const int32_t* block_table;
   const int32_t* seq_lens;
   const int32_t* cu_q;  // null: decode (one query per sequence, row b)
@@ -271,31 +276,31 @@ static_assert(PF_RING * 8 * 4 <= 512, "page-id ring overflows its region");
 // K: 8 page blocks of 16 keys, canonical no-swizzle K-major: core matrices of
 // 8 keys x 8 d (128 B), d-chunks 128 B apart (LBO), 8-key groups 2 KB apart
 // (SBO, uniform across the blocks of a tile).
-template <bool DECODE>
+template <bool DECODE, typename ET>
 __device__ __forceinline__ void issue_s(uint32_t tmem_s, uint32_t q_addr, uint32_t k_addr) {
   using L = Lay<DECODE>;
-  constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
+  constexpr uint32_t idesc = idesc_f32acc(128, 128, E16<ET>::kMmaFormat);
 #pragma unroll
   for (int kk = 0; kk < HD / 16; ++kk) {
     const uint32_t qoff = (kk >> 2) * L::HALF + (kk & 3) * 32;
-    mma_bf16(tmem_s, smem_desc(q_addr + qoff, 16, L::ROW_SBO, 2), smem_desc(k_addr + kk * 256, 128, 2048, 0),
+    mma_f16k(tmem_s, smem_desc(q_addr + qoff, 16, L::ROW_SBO, 2), smem_desc(k_addr + kk * 256, 128, 2048, 0),
              idesc, kk != 0);
   }
 }
 
 // O (+)= P V: accumulate = 0 on the first tile of a split, 1 after.
-template <bool DECODE>
+template <bool DECODE, typename ET>
 __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t p_addr, uint32_t v_addr,
                                          bool accumulate) {
   using L = Lay<DECODE>;
-  constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
+  constexpr uint32_t idesc = idesc_f32acc(128, 128, E16<ET>::kMmaFormat);
 #pragma unroll
   for (int j = 0; j < PAGES_PER_TILE; ++j) {
     const uint32_t poff = (j >> 2) * L::HALF + (j & 3) * 32;
     // V page block j (16 keys = one K step): canonical no-swizzle K-major with
     // rows = d: core matrices of 8 d x 8 keys, key-chunks 128 B apart (LBO),
     // 8-d groups 256 B apart (SBO).
-    mma_bf16(tmem_o, smem_desc(p_addr + poff, 16, L::ROW_SBO, 2),
+    mma_f16k(tmem_o, smem_desc(p_addr + poff, 16, L::ROW_SBO, 2),
              smem_desc(v_addr + j * BLOCK_BYTES, 128, 256, 0), idesc, (accumulate || j != 0) ? 1u : 0u);
   }
 }
@@ -308,10 +313,12 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// One quarter (32 keys) of a row's tile: P_c = bf16(2^(S_c * scale_log2 -
-// m)) for c < nvalid (else 0), packed two per word into P[0..15], and the
-// quarter sum of the bf16 values, added left to right. Decode and prefill both
-// build a row from exactly these quarters, so their arithmetic is the same.
+// One quarter (32 keys) of a row's tile: P_c = r16(2^(S_c * scale_log2 -
+// m)) for c < nvalid (else 0), r16 the rounding to the 16-bit element type,
+// packed two per word into P[0..15], and the quarter sum of the rounded
+// values, added left to right. Decode and prefill both build a row from
+// exactly these quarters, so their arithmetic is the same.
+template <typename ET>
 __device__ __forceinline__ float quarter_p(const uint32_t (&S)[32], int nvalid, float neg_m,
                                            float scale_log2, uint32_t (&P)[16]) {
   float q = 0.0f;
@@ -321,9 +328,9 @@ __device__ __forceinline__ float quarter_p(const uint32_t (&S)[32], int nvalid, 
     // select, so no branch serialises the loop
     const float e0 = ex2_approx(__fmaf_rn(__uint_as_float(S[2 * c2]), scale_log2, neg_m));
     const float e1 = ex2_approx(__fmaf_rn(__uint_as_float(S[2 * c2 + 1]), scale_log2, neg_m));
-    const uint32_t pk = pack_bf16x2(2 * c2 < nvalid ? e0 : 0.0f, 2 * c2 + 1 < nvalid ? e1 : 0.0f);
-    q = __fadd_rn(q, __uint_as_float(pk << 16));          // bf16 of element 2*c2
-    q = __fadd_rn(q, __uint_as_float(pk & 0xffff0000u));  // bf16 of element 2*c2+1
+    const uint32_t pk = E16<ET>::pack2(2 * c2 < nvalid ? e0 : 0.0f, 2 * c2 + 1 < nvalid ? e1 : 0.0f);
+    q = __fadd_rn(q, E16<ET>::lo(pk));  // rounded element 2*c2
+    q = __fadd_rn(q, E16<ET>::hi(pk));  // rounded element 2*c2+1
     P[c2] = pk;
   }
   return q;
@@ -391,7 +398,7 @@ __device__ __forceinline__ void drain(uint64_t* bar, int fills) {
 //                             P_j = bf16(2^(s_j - m')), l = alpha*l + sum_j P_j,
 //                             O = alpha*O (fp32, skipped when alpha == 1), O += P V (MMA)
 // sums over j run j = 0..127 in order; masked keys have P_j = 0 by selection.
-template <bool DECODE>
+template <bool DECODE, typename ET>
 __global__ void __launch_bounds__(THREADS, 1)
     attn_split_kernel(const __grid_constant__ CUtensorMap tmQ, const Params p) {
   using L = Lay<DECODE>;
@@ -411,7 +418,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* s_free = bars + 19;    // [NS]
   uint64_t* p_ready = bars + 22;   // [NP]
   uint64_t* o_ready = bars + 24;   // [NP]: P V of the tile that read P buffer i is done
-  uint64_t* x_bar = bars + 26;     // decode: quarter exchange among the 4 softmax warps
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 27);
   static_assert(28 * 8 <= 256, "barrier region");
   RingItem* item_ring = reinterpret_cast<RingItem*>(smem + L::OFF_ITEMS);
@@ -442,7 +448,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&p_ready[i], 128);
       mbar_init(&o_ready[i], 1);
     }
-    mbar_init(x_bar, 128);
     for (int i = 0; i < ITEM_RING; ++i) mbar_init(&item_bar[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -591,7 +596,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                              mbar_test(&s_free[sb], (((uint32_t)nS / L::NS) & 1u) ^ 1u);
           if (ready) {
             tc_fence_after();
-            issue_s<DECODE>(tmem + sb * 128, sQ0 + qb * L::QP_BYTES, sK0 + kb * TILE_BYTES);
+            issue_s<DECODE, ET>(tmem + sb * 128, sQ0 + qb * L::QP_BYTES, sK0 + kb * TILE_BYTES);
             mma_commit(&s_full[sb]);
             mma_commit(&k_empty[kb]);
             if (sc.t == sc.it.ntiles - 1) mma_commit(&q_empty[qb]);  // Q is read by QK^T only
@@ -609,7 +614,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               mbar_test(&v_full[vb], ((uint32_t)nP / NV) & 1u)) {
             const uint32_t bit = 1u << (nP & 31);
             tc_fence_after();
-            issue_pv<DECODE>(tmem + TMEM_O, sP + pb * L::QP_BYTES, sV0 + vb * TILE_BYTES, (acc_bits & bit) != 0);
+            issue_pv<DECODE, ET>(tmem + TMEM_O, sP + pb * L::QP_BYTES, sV0 + vb * TILE_BYTES, (acc_bits & bit) != 0);
             mma_commit(&o_ready[pb]);
             mma_commit(&v_empty[vb]);
             ++nP;
@@ -631,17 +636,20 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ------------------------------------------------ softmax warps 0-3
     // Prefill layout: thread r owns MMA row r = (query r / G, head r % G) and
     // all 128 keys of a tile (its four quarters in turn).
-    // Decode layout (one query per item): the item's G head rows are loaded
-    // into rows 32w + i of every warp w (identical rows, identical S), and
-    // warp w computes quarter w (keys 32w .. 32w+31) of every head i < G;
-    // quarter maxima and quarter sums are exchanged through shared memory.
+    // Decode layout (one query per item): Q holds one 8-row core-matrix group
+    // (row i = head i < G) that the MMA repeats over all 128 rows, so tensor
+    // memory lane 32w + l holds head l % 8 for every warp w. Lane l of warp w
+    // takes head l % 8 and quarter l / 8 (keys 32 (l/8) .. +31) when that head
+    // belongs to the warp (head % 4 == w): the four lanes of a head in one
+    // warp combine their quarters by shuffles, so no warp waits for another.
     constexpr bool decode = DECODE;
     const int r = threadIdx.x;  // 0..127 == TMEM lane
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const int qr = decode ? 0 : r / p.G;
-    const int hj = decode ? lane : r - qr * p.G;
-    float* red = reinterpret_cast<float*>(smem + L::OFF_RED);  // [2][4 warps][8 head rows]
-    int j = 0, xc = 0;
+    const int hj = decode ? (lane & 7) : r - qr * p.G;
+    const int quarter_of_lane = lane >> 3;  // decode: this lane's quarter of the keys
+    const bool lane_owns = decode ? ((lane & 7) < p.G && (lane & 3) == warp) : true;
+    int j = 0;
     bool ok = true;
     // waits until the P V product of tile jj (counted across this CTA's items) is done
     auto pv_done = [&](int jj) -> bool {
@@ -649,12 +657,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       return true;
     };
-    auto exchange = [&](float v, int which) -> bool {
-      if (lane < 8) red[(which * 4 + warp) * 8 + lane] = v;
-      mbar_arrive(x_bar);
-      const bool done = mbar_wait(x_bar, (uint32_t)xc & 1u, p.status, abort_flag);
-      ++xc;
-      return done;
+    // decode: the 32 columns of quarter `quarter_of_lane` of this lane's tensor
+    // memory row at column base `col` (warp-collective loads of all four
+    // quarters; each lane keeps its own)
+    auto load_own_quarter = [&](uint32_t col, uint32_t (&out)[32]) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t tmp[32];
+        tmem_ld32(tmem + col + lane_off + c * 32, tmp);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) out[i] = quarter_of_lane == c ? tmp[i] : out[i];
+      }
     };
     for (int n = 0; ok; ++n) {
       int idx;
@@ -663,7 +677,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (idx < 0) break;
       const int q_idx = it.q_lo + qr;
       const int pos = it.L - it.nb + q_idx;
-      const bool row_valid = (decode ? lane < p.G : true) && (q_idx < it.q_hi) && (pos >= it.key_lo);
+      const bool row_valid = lane_owns && (q_idx < it.q_hi) && (pos >= it.key_lo);
       const bool warp_valid = decode ? true : __any_sync(0xffffffffu, row_valid);
       const int last_page = (it.L - 1) / PAGE;
       const int tail = it.L % PAGE;
@@ -677,42 +691,52 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         float alpha = 1.0f, m_new = 0.0f;
         if constexpr (decode) {
-          // ---- decode layout: this warp's quarter of every head row
+          // ---- decode layout: this lane's quarter of its head's row
           uint32_t S[32], P[16];
-          tmem_ld32(tmem + sb * 128 + lane_off + warp * 32, S);
-          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) S[i] = 0u;
+          load_own_quarter(sb * 128, S);
           tc_fence_before();
           mbar_arrive(&s_free[sb]);
-          const int nq = min(32, max(0, nvalid - warp * 32));
-          if (!exchange(quarter_max(S, nq), 0)) { ok = false; break; }
-          float mraw = -INFINITY;
-#pragma unroll
-          for (int w = 0; w < 4; ++w) mraw = fmaxf(mraw, red[w * 8 + (lane & 7)]);
+          const int nq = min(32, max(0, nvalid - quarter_of_lane * 32));
+          // the row maximum over the four quarters (exact, any order)
+          float mraw = quarter_max(S, nq);
+          mraw = fmaxf(mraw, __shfl_xor_sync(0xffffffffu, mraw, 8));
+          mraw = fmaxf(mraw, __shfl_xor_sync(0xffffffffu, mraw, 16));
           if (need) {
             m_new = new_reference(m, __fmul_rn(mraw, p.scale_log2), t);
             alpha = ex2_approx(__fsub_rn(m, m_new));
           }
-          const float qs = quarter_p(S, nq, -m_new, p.scale_log2, P);
-          if (!exchange(qs, 1)) { ok = false; break; }
+          const float qs = quarter_p<ET>(S, nq, -m_new, p.scale_log2, P);
+          // quarter sums of the head, in quarter order, as in prefill
+          const int h0 = lane & 7;
+          const float q0 = __shfl_sync(0xffffffffu, qs, h0);
+          const float q1 = __shfl_sync(0xffffffffu, qs, h0 + 8);
+          const float q2 = __shfl_sync(0xffffffffu, qs, h0 + 16);
+          const float q3 = __shfl_sync(0xffffffffu, qs, h0 + 24);
           if (need) {
-            const float lsum = __fadd_rn(__fadd_rn(__fadd_rn(red[32 + lane], red[32 + 8 + lane]),
-                                                   red[32 + 16 + lane]), red[32 + 24 + lane]);
+            const float lsum = __fadd_rn(__fadd_rn(__fadd_rn(q0, q1), q2), q3);
             l = (t == 0) ? lsum : __fadd_rn(__fmul_rn(alpha, l), lsum);
             m = m_new;
           }
           // P buffer j % NP was last read by the P V of tile j - NP
           if (j >= L::NP && !pv_done(j - L::NP)) { ok = false; break; }
-          if (lane < p.G) store_p_chunks(smem + OFF_P + (j % L::NP) * L::QP_BYTES, L::HALF, lane, warp, P);
+          if (lane_owns) store_p_chunks(smem + OFF_P + (j % L::NP) * L::QP_BYTES, L::HALF, h0, quarter_of_lane, P);
           if (t > 0 && __any_sync(0xffffffffu, need && alpha != 1.0f)) {
-            // O may be rescaled only once the P V of tile j-1 has landed in it
+            // O may be rescaled only once the P V of tile j-1 has landed in
+            // it; each lane scales its whole row (all four quarters), so every
+            // copy of a head's row that a lane of this warp owns stays whole
             if (L::NP > 1 && !pv_done(j - 1)) { ok = false; break; }
-            uint32_t o[32];
-            tmem_ld32(tmem + TMEM_O + lane_off + warp * 32, o);
-            tmem_ld_wait();
             const float a = need ? alpha : 1.0f;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              uint32_t o[32];
+              tmem_ld32(tmem + TMEM_O + lane_off + c * 32, o);
+              tmem_ld_wait();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__fmul_rn(__uint_as_float(o[c]), a));
-            tmem_st32(tmem + TMEM_O + lane_off + warp * 32, o);
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__fmul_rn(__uint_as_float(o[i]), a));
+              tmem_st32(tmem + TMEM_O + lane_off + c * 32, o);
+            }
             tmem_st_wait();
           }
         } else {
@@ -741,7 +765,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             float qs[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-              qs[q] = quarter_p(*reinterpret_cast<uint32_t(*)[32]>(&S[q * 32]),
+              qs[q] = quarter_p<ET>(*reinterpret_cast<uint32_t(*)[32]>(&S[q * 32]),
                                 min(32, max(0, nvalid - q * 32)), -m_new, p.scale_log2,
                                 *reinterpret_cast<uint32_t(*)[16]>(&P[q * 16]));
             if (need) {
@@ -796,16 +820,17 @@ __global__ void __launch_bounds__(THREADS, 1)
       const size_t widx = ((size_t)(it.r0 + q_idx) * p.Hq + (size_t)(it.g * p.G + hj)) * p.n_split_max + it.s;
       if constexpr (decode) {
         uint32_t o[32];
-        tmem_ld32(tmem + TMEM_O + lane_off + warp * 32, o);
-        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = 0u;
+        load_own_quarter(TMEM_O, o);
         if (row_valid) {
-          float* dst = p.ws_o + widx * HD + warp * 32;
+          float* dst = p.ws_o + widx * HD + quarter_of_lane * 32;
 #pragma unroll
           for (int c4 = 0; c4 < 8; ++c4)
             reinterpret_cast<float4*>(dst)[c4] =
                 make_float4(__uint_as_float(o[4 * c4]), __uint_as_float(o[4 * c4 + 1]),
                             __uint_as_float(o[4 * c4 + 2]), __uint_as_float(o[4 * c4 + 3]));
-          if (warp == 0) *reinterpret_cast<float2*>(p.ws_ml + widx * 2) = make_float2(m, l);
+          if (quarter_of_lane == 0) *reinterpret_cast<float2*>(p.ws_ml + widx * 2) = make_float2(m, l);
         }
       } else if (warp_valid) {
         float* dst = p.ws_o + widx * HD;
@@ -844,11 +869,12 @@ struct CombineParams {
   const float* ws_ml;
   const int32_t* seq_lens;
   const int32_t* cu_q;  // null: decode
-  bf16* out;
+  void* out;  // 16-bit rows (the element type of the kernel)
   int64_t ldo;
   int32_t n_tok, B, Hq, n_split_max, max_kv_len;
 };
 
+template <typename ET>
 __global__ void attn_combine_kernel(const CombineParams p) {
   const int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -873,7 +899,7 @@ __global__ void attn_combine_kernel(const CombineParams p) {
     qidx = 0;
   }
   const int L = p.seq_lens[b];
-  bf16* dst = p.out + (size_t)tok * p.ldo + (size_t)h * HD + lane * 4;
+  uint16_t* dst = static_cast<uint16_t*>(p.out) + (size_t)tok * p.ldo + (size_t)h * HD + lane * 4;
   if (L < nb || L > p.max_kv_len || nb <= 0) {  // flagged by the split kernel; write zeros
     *reinterpret_cast<uint2*>(dst) = make_uint2(0u, 0u);
     return;
@@ -898,7 +924,7 @@ __global__ void attn_combine_kernel(const CombineParams p) {
   // + 0.0f turns a -0 into +0, so a zero's sign cannot depend on the split path
   const float y0 = __fadd_rn(__fdiv_rn(o0, Lsum), 0.0f), y1 = __fadd_rn(__fdiv_rn(o1, Lsum), 0.0f);
   const float y2 = __fadd_rn(__fdiv_rn(o2, Lsum), 0.0f), y3 = __fadd_rn(__fdiv_rn(o3, Lsum), 0.0f);
-  *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(y0, y1), pack_bf16x2(y2, y3));
+  *reinterpret_cast<uint2*>(dst) = make_uint2(E16<ET>::pack2(y0, y1), E16<ET>::pack2(y2, y3));
 }
 
 // partial O [n_tok][Hq][n_split][128] fp32, then (m, l) pairs, then (256-byte
@@ -929,6 +955,7 @@ static bi_status check_shape(const bi_attn_shape* sh) {
   return BI_OK;
 }
 
+template <typename ET>
 static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t max_q_len,
                      int64_t n_tok, const void* k_cache, const void* v_cache,
                      const int32_t* block_table, const int32_t* seq_lens, int32_t B,
@@ -961,7 +988,7 @@ static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t ma
     uint64_t dims[3] = {(uint64_t)HD, (uint64_t)Hq, (uint64_t)n_tok};
     uint64_t strides[2] = {(uint64_t)HD * 2, (uint64_t)ldq * 2};
     uint32_t box[3] = {64, (uint32_t)G, cu_q ? (uint32_t)QR : 1u};
-    if ((st = encode_tmap(&tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims,
+    if ((st = encode_tmap(&tmQ, E16<ET>::kTmap, 3, const_cast<void*>(q), dims,
                           strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != BI_OK)
       return st;
   }
@@ -990,26 +1017,32 @@ static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t ma
   p.scale_log2 = (float)((double)sh->scale * 1.4426950408889634);  // scale * log2(e)
   p.status = status_word();
 
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (!attr_set[dev & 63]) {
-    cudaError_t e = cudaFuncSetAttribute(attn_split_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)Lay<true>::SMEM_BYTES);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attn_split_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)Lay<false>::SMEM_BYTES);
-    if (e != cudaSuccess) return cuda_fail(e, "attention: smem attribute");
-    attr_set[dev & 63] = true;
+  {
+    // once per device, under a lock (calls may come from several host threads)
+    static bool attr_set[64] = {false};
+    static std::mutex mu;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return fail(BI_ERR_UNSUPPORTED, "attention: device id %d out of range", dev);
+    std::lock_guard<std::mutex> lk(mu);
+    if (!attr_set[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(attn_split_kernel<true, ET>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)Lay<true>::SMEM_BYTES);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(attn_split_kernel<false, ET>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)Lay<false>::SMEM_BYTES);
+      if (e != cudaSuccess) return cuda_fail(e, "attention: smem attribute");
+      attr_set[dev] = true;
+    }
   }
   const int sms = num_sms();
   const int grid = (int)(total_items < sms ? total_items : sms);
   cudaError_t me = cudaMemsetAsync(p.work_counter, 0, sizeof(int32_t), stream);
   if (me != cudaSuccess) return cuda_fail(me, "attention: work counter reset");
   if (cu_q)
-    attn_split_kernel<false><<<grid, THREADS, Lay<false>::SMEM_BYTES, stream>>>(tmQ, p);
+    attn_split_kernel<false, ET><<<grid, THREADS, Lay<false>::SMEM_BYTES, stream>>>(tmQ, p);
   else
-    attn_split_kernel<true><<<grid, THREADS, Lay<true>::SMEM_BYTES, stream>>>(tmQ, p);
+    attn_split_kernel<true, ET><<<grid, THREADS, Lay<true>::SMEM_BYTES, stream>>>(tmQ, p);
   BI_CHECK_LAUNCH("attention split launch");
 
   CombineParams c;
@@ -1017,7 +1050,7 @@ static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t ma
   c.ws_ml = p.ws_ml;
   c.seq_lens = seq_lens;
   c.cu_q = cu_q;
-  c.out = static_cast<bf16*>(out);
+  c.out = out;
   c.ldo = ldo;
   c.n_tok = (int32_t)n_tok;
   c.B = B;
@@ -1026,12 +1059,31 @@ static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t ma
   c.max_kv_len = sh->max_kv_len;
   const int64_t warps = n_tok * Hq;
   const int blocks = (int)((warps + 7) / 8);
-  attn_combine_kernel<<<blocks, 256, 0, stream>>>(c);
+  attn_combine_kernel<ET><<<blocks, 256, 0, stream>>>(c);
   BI_CHECK_LAUNCH("attention combine launch");
   return BI_OK;
 }
 
 }  // namespace attn
+
+// The FP16 variant (fp16 Q, caches, P and output) for the forward's FP16
+// precision mode; the same kernels as bi_attn_decode / bi_attn_prefill.
+bi_status attn_decode_f16(const void* q, int64_t ldq, const void* k_cache, const void* v_cache,
+                          const int32_t* block_table, const int32_t* seq_lens, int32_t B,
+                          const bi_attn_shape* shape, void* out, int64_t ldo, void* ws, size_t ws_bytes,
+                          cudaStream_t s) {
+  return attn::run<f16>(q, ldq, nullptr, 1, B, k_cache, v_cache, block_table, seq_lens, B, shape, out, ldo,
+                        ws, ws_bytes, s);
+}
+
+bi_status attn_prefill_f16(const void* q, int64_t ldq, const int32_t* cu_q, int32_t max_q_len, int64_t n_tok,
+                           const void* k_cache, const void* v_cache, const int32_t* block_table,
+                           const int32_t* seq_lens, int32_t B, const bi_attn_shape* shape, void* out,
+                           int64_t ldo, void* ws, size_t ws_bytes, cudaStream_t s) {
+  if (!cu_q) return fail(BI_ERR_INVALID_ARG, "attn_prefill: cu_q is null");
+  return attn::run<f16>(q, ldq, cu_q, max_q_len, n_tok, k_cache, v_cache, block_table, seq_lens, B, shape, out,
+                        ldo, ws, ws_bytes, s);
+}
 }  // namespace bi
 
 using namespace bi;
@@ -1051,7 +1103,7 @@ extern "C" bi_status bi_attn_decode(const void* q, int64_t ldq, const void* k_ca
                                     const int32_t* seq_lens, int32_t B, const bi_attn_shape* shape,
                                     void* out, int64_t ldo, void* ws, size_t ws_bytes,
                                     void* stream) {
-  return attn::run(q, ldq, nullptr, 1, B, k_cache, v_cache, block_table, seq_lens, B, shape, out,
+  return attn::run<bf16>(q, ldq, nullptr, 1, B, k_cache, v_cache, block_table, seq_lens, B, shape, out,
                    ldo, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
@@ -1062,6 +1114,6 @@ extern "C" bi_status bi_attn_prefill(const void* q, int64_t ldq, const int32_t* 
                                      const bi_attn_shape* shape, void* out, int64_t ldo, void* ws,
                                      size_t ws_bytes, void* stream) {
   if (!cu_q) return fail(BI_ERR_INVALID_ARG, "attn_prefill: cu_q is null");
-  return attn::run(q, ldq, cu_q, max_q_len, n_tok, k_cache, v_cache, block_table, seq_lens, B,
+  return attn::run<bf16>(q, ldq, cu_q, max_q_len, n_tok, k_cache, v_cache, block_table, seq_lens, B,
                    shape, out, ldo, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }

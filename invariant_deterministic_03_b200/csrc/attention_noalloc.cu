@@ -12,10 +12,15 @@
 // nothing is allocated per call.
 //
 // The array's name means nothing to host code (there it is a host-side
-// stand-in, not a device address), so the device address is looked up once
-// per device with cudaGetSymbolAddress and cached; that lookup happens on the
-// first call on each device, which should therefore come before any stream
-// capture.
+// stand-in, not a device address), so the device address is looked up with
+// cudaGetSymbolAddress, with the device current, once per device and CUDA
+// context, and cached; the cache is keyed by the current context, so a
+// context that was destroyed and re-created (cudaDeviceReset, a released
+// primary context) gets a fresh lookup instead of a stale address. The
+// lookup happens on the first call in each context, which should therefore
+// come before any stream capture.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -28,21 +33,38 @@ static __device__ __align__(256) uint8_t g_attn_scratch[BI_ATTN_NOALLOC_SCRATCH_
 
 constexpr int kMaxDev = 64;
 static std::mutex g_mu;
+static CUcontext g_ctx[kMaxDev];        // context the cached address belongs to
 static void* g_scratch_ptr[kMaxDev];
+static PFN_cuCtxGetCurrent_v4000 g_get_ctx = nullptr;
 
-// Device address of this device's scratch array (looked up once per device,
-// with that device current).
+// Device address of the scratch array in the current device's current
+// context (looked up once per device and context, with that device current).
 static bi_status scratch_address(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "attn_decode_noalloc: cudaGetDevice");
   if (dev < 0 || dev >= kMaxDev) return fail(BI_ERR_UNSUPPORTED, "attn_decode_noalloc: device id %d out of range", dev);
   std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (!g_get_ctx) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    e = cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+      return fail(BI_ERR_UNSUPPORTED, "attn_decode_noalloc: cuCtxGetCurrent unavailable");
+    g_get_ctx = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+  }
+  CUcontext ctx = nullptr;
+  if (g_get_ctx(&ctx) != CUDA_SUCCESS) ctx = nullptr;
+  if (!ctx || !g_scratch_ptr[dev] || g_ctx[dev] != ctx) {
+    // the lookup also makes the device's primary context current when no
+    // context is yet (the runtime initialises it on first use)
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_attn_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "attn_decode_noalloc: cudaGetSymbolAddress");
+    if (g_get_ctx(&ctx) != CUDA_SUCCESS || !ctx)
+      return fail(BI_ERR_CUDA, "attn_decode_noalloc: no current CUDA context");
     g_scratch_ptr[dev] = p;
+    g_ctx[dev] = ctx;
   }
   *out = g_scratch_ptr[dev];
   return BI_OK;

@@ -7,6 +7,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -269,18 +270,22 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
   return d;
 }
 
-// Instruction descriptor of tcgen05.mma kind::f16 with bf16 A and B (both
-// K-major), fp32 accumulator, M x N tile.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+// Instruction descriptor of tcgen05.mma kind::f16 with 16-bit A and B of
+// operand format `fmt` (0: fp16, 1: bf16; A and B always the same type), both
+// K-major, fp32 accumulator, M x N tile.
+__host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, uint32_t fmt) {
   return (1u << 4)                        // D format: f32
-         | (1u << 7)                      // A format: bf16
-         | (1u << 10)                     // B format: bf16
+         | (fmt << 7)                     // A format
+         | (fmt << 10)                    // B format
          | ((uint32_t)(N >> 3) << 17)     // N / 8
          | ((uint32_t)(M >> 4) << 24);    // M / 16
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread.
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) { return idesc_f32acc(M, N, 1u); }
+
+// D[tmem] (+)= A[smem] * B[smem]^T (kind::f16: fp16 or bf16 operands, as the
+// instruction descriptor says), issued by one thread.
+__device__ __forceinline__ void mma_f16k(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                          uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -295,6 +300,62 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
           smem_u32(bar))
+      : "memory");
+}
+
+// ---------------------------------------------------------------- CTA pairs
+// A pair of CTAs (a two-CTA cluster) computes one 256-row MMA: each CTA holds
+// half of the A rows and half of the B rows in its own shared memory and its
+// half of the accumulator in its own tensor memory; the even CTA (rank 0)
+// issues the MMAs for both.
+
+// Tensor-memory allocation owned by both CTAs of the pair: one warp of EACH
+// CTA executes these together.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// D (+)= A * B^T over the pair (kind::f16: fp16 or bf16 operands, as the
+// instruction descriptor says), issued by one thread of rank 0; the
+// descriptors name the same shared-memory offsets in both CTAs.
+__device__ __forceinline__ void mma_f16k_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on the mbarrier at shared::cluster address `bar` (either CTA of the
+// pair) once every pair MMA issued so far by this thread is done.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+// TMA tiled load into this CTA's shared memory whose completion (bytes) is
+// counted on the mbarrier at shared::cluster address `bar`, which may belong
+// to the other CTA of the pair. No cluster multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar,
+                                                 int32_t c0, int32_t c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.cta_group::2"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
       : "memory");
 }
 
@@ -337,5 +398,43 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // round to nearest even
   return *reinterpret_cast<uint32_t*>(&v);
 }
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);  // round to nearest even
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+typedef __half f16;
+
+// The 16-bit element type of activations, weights and the KV cache: bf16 (the
+// library's default) or fp16 (the FP16 variant of the precision study). Every
+// kernel that rounds to or reads a 16-bit value goes through these, so both
+// types share every other instruction.
+template <typename T>
+struct E16;
+
+template <>
+struct E16<bf16> {
+  static constexpr uint32_t kMmaFormat = 1;  // tcgen05 kind::f16 operand format
+  static constexpr CUtensorMapDataType kTmap = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  static __device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16x2(lo, hi); }
+  static __device__ __forceinline__ float round(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
+  static __device__ __forceinline__ float lo(uint32_t w) { return __uint_as_float(w << 16); }
+  static __device__ __forceinline__ float hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+  static __device__ __forceinline__ float to_f32(bf16 v) { return __bfloat162float(v); }
+  static __device__ __forceinline__ bf16 from_f32(float v) { return __float2bfloat16_rn(v); }
+};
+
+template <>
+struct E16<f16> {
+  static constexpr uint32_t kMmaFormat = 0;
+  static constexpr CUtensorMapDataType kTmap = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  static __device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_f16x2(lo, hi); }
+  static __device__ __forceinline__ float round(float v) { return __half2float(__float2half_rn(v)); }
+  static __device__ __forceinline__ float lo(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu))); }
+  static __device__ __forceinline__ float hi(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
+  static __device__ __forceinline__ float to_f32(f16 v) { return __half2float(v); }
+  static __device__ __forceinline__ f16 from_f32(float v) { return __float2half_rn(v); }
+};
 
 }  // namespace bi

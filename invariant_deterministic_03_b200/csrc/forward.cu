@@ -26,13 +26,36 @@
 #include "host.h"
 
 namespace bi {
-bi_status launch_kv_append(const bf16* k, const bf16* v, int64_t ld_new, const int32_t* slots,
-                           int64_t n_tok, bf16* kc, bf16* vc, int Hkv, int num_pages,
+bi_status launch_kv_append(const uint16_t* k, const uint16_t* v, int64_t ld_new, const int32_t* slots,
+                           int64_t n_tok, uint16_t* kc, uint16_t* vc, int Hkv, int num_pages,
                            cudaStream_t s);
-bi_status launch_embed(const int32_t* tok, int64_t n_tok, const bf16* table, int64_t vocab,
+template <typename ET>
+bi_status launch_embed(const int32_t* tok, int64_t n_tok, const ET* table, int64_t vocab,
                        int64_t D, float* out, cudaStream_t s);
-bi_status launch_rope(bf16* x, int64_t ldx, int n_heads, const int32_t* pos, int64_t n_tok,
+template <typename ET>
+bi_status launch_rope(ET* x, int64_t ldx, int n_heads, const int32_t* pos, int64_t n_tok,
                       const float* cs, int max_pos, cudaStream_t s);
+template <typename ET>
+bi_status gemm_e16(const void* A, int64_t lda, const void* W, int64_t ldw, void* C, int64_t ldc,
+                   int32_t c_dtype, int64_t M, int64_t N, int64_t K, cudaStream_t s);
+template <typename ET>
+bi_status gemm_swiglu_e16(const void* A, int64_t lda, const void* W, int64_t ldw, void* out,
+                          int64_t ldo, int64_t M, int64_t F, int64_t K, cudaStream_t s);
+template <typename ET>
+bi_status gemm_qkv_e16(const void* A, int64_t lda, const void* W, int64_t ldw, void* qkv, int64_t ldq,
+                       int64_t M, int64_t K, int32_t n_q_heads, int32_t n_kv_heads, const int32_t* positions,
+                       const float* cos_sin, int32_t max_pos, const int32_t* slot_mapping, void* k_cache,
+                       void* v_cache, int32_t num_pages, cudaStream_t s);
+bi_status rmsnorm_f32in_f16(const float* x, const void* gamma, void* y, int64_t M, int64_t D, float eps,
+                            cudaStream_t s);
+bi_status attn_decode_f16(const void* q, int64_t ldq, const void* k_cache, const void* v_cache,
+                          const int32_t* block_table, const int32_t* seq_lens, int32_t B,
+                          const bi_attn_shape* shape, void* out, int64_t ldo, void* ws, size_t ws_bytes,
+                          cudaStream_t s);
+bi_status attn_prefill_f16(const void* q, int64_t ldq, const int32_t* cu_q, int32_t max_q_len, int64_t n_tok,
+                           const void* k_cache, const void* v_cache, const int32_t* block_table,
+                           const int32_t* seq_lens, int32_t B, const bi_attn_shape* shape, void* out,
+                           int64_t ldo, void* ws, size_t ws_bytes, cudaStream_t s);
 bi_status launch_argmax(const float* logits, int64_t rows, int64_t V, int64_t ld, int32_t* idx,
                         cudaStream_t s);
 bi_status launch_split(const float* x, int64_t n, bf16* hi, bf16* lo, cudaStream_t s);
@@ -133,7 +156,8 @@ extern "C" bi_status bi_model_create(const bi_model_config* cfg, const bi_model_
   if (G != 1 && G != 2 && G != 4 && G != 8) return fail(BI_ERR_SHAPE, "model_create: q heads per kv head must be 1, 2, 4 or 8");
   if (c.d_ff % 8 || c.vocab % 8) return fail(BI_ERR_SHAPE, "model_create: d_ff and vocab must be multiples of 8");
   if (!(c.rms_eps >= 0.0f) || !(c.rope_theta > 1.0)) return fail(BI_ERR_INVALID_ARG, "model_create: bad eps or rope_theta");
-  if (c.precision != BI_PREC_BF16 && c.precision != BI_PREC_F32 && c.precision != BI_PREC_BF16_MLP)
+  if (c.precision != BI_PREC_BF16 && c.precision != BI_PREC_F32 && c.precision != BI_PREC_BF16_MLP &&
+      c.precision != BI_PREC_F16)
     return fail(BI_ERR_INVALID_ARG, "model_create: unknown precision %d", c.precision);
   if (!w->embed || !w->final_norm || !w->lm_head) return fail(BI_ERR_INVALID_ARG, "model_create: missing weights");
   if (c.n_layers > 0 && (!w->attn_norm || !w->w_qkv || !w->w_o || !w->mlp_norm || !w->w_gate_up || !w->w_down))
@@ -200,16 +224,19 @@ extern "C" bi_status bi_forward(const bi_model* m, const bi_batch* bt, void* k_c
   float* rope = reinterpret_cast<float*>(base + L.rope);
   void* attn_ws = base + L.attn_ws;
 
-  const bool attn_f32 = c.precision != BI_PREC_BF16;  // attention block (and LM head) upcast
+  const bool f16m = c.precision == BI_PREC_F16;       // the 16-bit path in fp16
+  const bool attn_f32 = c.precision == BI_PREC_F32 || c.precision == BI_PREC_BF16_MLP;  // attention block (and LM head) upcast
   const bool mlp_f32 = c.precision == BI_PREC_F32;    // MLP block upcast
   const int64_t T = b.n_tok, D = c.d_model, F = c.d_ff;
   const int Hq = c.n_q_heads, Hkv = c.n_kv_heads;
   const int64_t QKV = (int64_t)(Hq + 2 * Hkv) * BI_HEAD_DIM;
   const size_t cache_layer = (size_t)num_pages * Hkv * BI_PAGE_SIZE * BI_HEAD_DIM;
-  const bool qkv_fused = ((T + BI_GEMM_BM - 1) / BI_GEMM_BM) * ((QKV + BI_GEMM_BN - 1) / BI_GEMM_BN) >= num_sms();
+  // a pair of CTAs per 256 x BI_GEMM_BN output tile
+  const bool qkv_fused = ((T + BI_GEMM_BM - 1) / BI_GEMM_BM) * ((QKV + BI_GEMM_BN - 1) / BI_GEMM_BN) >= num_sms() / 2;
 
   BI_TRY(bi_rope_table(rope, c.max_pos, c.rope_theta, stream));
-  BI_TRY(launch_embed(b.tokens, T, static_cast<const bf16*>(m->w.embed), c.vocab, D, x, s));
+  if (f16m) BI_TRY(launch_embed<f16>(b.tokens, T, static_cast<const f16*>(m->w.embed), c.vocab, D, x, s));
+  else BI_TRY(launch_embed<bf16>(b.tokens, T, static_cast<const bf16*>(m->w.embed), c.vocab, D, x, s));
 
   bi_attn_shape sh;
   sh.num_q_heads = Hq;
@@ -245,22 +272,28 @@ extern "C" bi_status bi_forward(const bi_model* m, const bi_batch* bt, void* k_c
       BI_TRY(launch_split(att32, T * D, att, att_lo, s));
       BI_TRY(bi_gemm_x2(att, att_lo, D, w_o, D, x, D, BI_F32_ADD, T, D, D, stream));  // x += O proj
     } else {
-      bf16* kc = static_cast<bf16*>(k_cache) + (size_t)l * cache_layer;
-      bf16* vc = static_cast<bf16*>(v_cache) + (size_t)l * cache_layer;
-      BI_TRY(bi_rmsnorm_f32in(x, attn_norm, h, T, D, c.rms_eps, stream));
+      uint16_t* kc = static_cast<uint16_t*>(k_cache) + (size_t)l * cache_layer;
+      uint16_t* vc = static_cast<uint16_t*>(v_cache) + (size_t)l * cache_layer;
+      BI_TRY(f16m ? rmsnorm_f32in_f16(x, attn_norm, h, T, D, c.rms_eps, s)
+                  : bi_rmsnorm_f32in(x, attn_norm, h, T, D, c.rms_eps, stream));
       // QKV projection, RoPE of the q and k heads, cache write: one launch
       // when every SM gets at least one output tile (RoPE and the scattered
       // cache stores then spread over all SMs and overlap later tiles'
       // MMAs); for fewer tiles the epilogue work would sit on those few SMs
       // after their only tile, so three launches are faster. Same bits.
       if (qkv_fused) {
-        BI_TRY(bi_gemm_qkv(h, D, w_qkv, D, qkv, QKV, T, D, Hq, Hkv, b.positions, rope, c.max_pos,
-                           b.slot_mapping, kc, vc, num_pages, stream));
+        BI_TRY(f16m ? gemm_qkv_e16<f16>(h, D, w_qkv, D, qkv, QKV, T, D, Hq, Hkv, b.positions, rope, c.max_pos,
+                                        b.slot_mapping, kc, vc, num_pages, s)
+                    : gemm_qkv_e16<bf16>(h, D, w_qkv, D, qkv, QKV, T, D, Hq, Hkv, b.positions, rope, c.max_pos,
+                                         b.slot_mapping, kc, vc, num_pages, s));
       } else {
-        BI_TRY(bi_gemm(h, D, w_qkv, D, qkv, QKV, BI_BF16, T, QKV, D, stream));
+        BI_TRY(f16m ? gemm_e16<f16>(h, D, w_qkv, D, qkv, QKV, BI_BF16, T, QKV, D, s)
+                    : gemm_e16<bf16>(h, D, w_qkv, D, qkv, QKV, BI_BF16, T, QKV, D, s));
         // q and k heads are adjacent in a qkv row: one launch rotates both
-        BI_TRY(launch_rope(qkv, QKV, Hq + Hkv, b.positions, T, rope, c.max_pos, s));
-        BI_TRY(launch_kv_append(qkv + (size_t)Hq * BI_HEAD_DIM, qkv + (size_t)(Hq + Hkv) * BI_HEAD_DIM,
+        if (f16m) BI_TRY(launch_rope<f16>(reinterpret_cast<f16*>(qkv), QKV, Hq + Hkv, b.positions, T, rope, c.max_pos, s));
+        else BI_TRY(launch_rope<bf16>(qkv, QKV, Hq + Hkv, b.positions, T, rope, c.max_pos, s));
+        BI_TRY(launch_kv_append(reinterpret_cast<const uint16_t*>(qkv + (size_t)Hq * BI_HEAD_DIM),
+                                reinterpret_cast<const uint16_t*>(qkv + (size_t)(Hq + Hkv) * BI_HEAD_DIM),
                                 QKV, b.slot_mapping, T, kc, vc, Hkv, num_pages, s));
       }
       // one-token sequences go through the decode kernel, longer chunks
@@ -268,13 +301,19 @@ extern "C" bi_status bi_forward(const bi_model* m, const bi_batch* bt, void* k_c
       // (same tiles, splits and per-row arithmetic)
       const int32_t nd = (T == b.B && b.max_q_len == 1) ? b.B : b.n_decode;
       if (nd > 0)
-        BI_TRY(bi_attn_decode(qkv, QKV, kc, vc, b.block_table, b.seq_lens, nd, &sh, att, D, attn_ws,
-                              L.attn_ws_bytes, stream));
+        BI_TRY(f16m ? attn_decode_f16(qkv, QKV, kc, vc, b.block_table, b.seq_lens, nd, &sh, att, D, attn_ws,
+                                      L.attn_ws_bytes, s)
+                    : bi_attn_decode(qkv, QKV, kc, vc, b.block_table, b.seq_lens, nd, &sh, att, D, attn_ws,
+                                     L.attn_ws_bytes, stream));
       if (nd < b.B)
-        BI_TRY(bi_attn_prefill(qkv, QKV, b.cu_q + nd, b.max_q_len, T, kc, vc,
-                               b.block_table + (size_t)nd * b.max_pages_per_seq, b.seq_lens + nd, b.B - nd,
-                               &sh, att, D, attn_ws, L.attn_ws_bytes, stream));
-      BI_TRY(bi_gemm(att, D, w_o, D, x, D, BI_F32_ADD, T, D, D, stream));  // x += O proj
+        BI_TRY(f16m ? attn_prefill_f16(qkv, QKV, b.cu_q + nd, b.max_q_len, T, kc, vc,
+                                       b.block_table + (size_t)nd * b.max_pages_per_seq, b.seq_lens + nd, b.B - nd,
+                                       &sh, att, D, attn_ws, L.attn_ws_bytes, s)
+                    : bi_attn_prefill(qkv, QKV, b.cu_q + nd, b.max_q_len, T, kc, vc,
+                                      b.block_table + (size_t)nd * b.max_pages_per_seq, b.seq_lens + nd, b.B - nd,
+                                      &sh, att, D, attn_ws, L.attn_ws_bytes, stream));
+      BI_TRY(f16m ? gemm_e16<f16>(att, D, w_o, D, x, D, BI_F32_ADD, T, D, D, s)
+                  : bi_gemm(att, D, w_o, D, x, D, BI_F32_ADD, T, D, D, stream));  // x += O proj
     }
 
     // ---- MLP block
@@ -284,9 +323,13 @@ extern "C" bi_status bi_forward(const bi_model* m, const bi_batch* bt, void* k_c
       BI_TRY(launch_swiglu_split(gu32, T, F, act, act_lo, s));
       BI_TRY(bi_gemm_x2(act, act_lo, F, w_d, F, x, D, BI_F32_ADD, T, D, F, stream));  // x += down proj
     } else {
-      BI_TRY(bi_rmsnorm_f32in(x, mlp_norm, h, T, D, c.rms_eps, stream));
-      BI_TRY(bi_gemm_swiglu(h, D, w_gu, D, act, F, T, F, D, stream));  // act = swiglu(gate, up)
-      BI_TRY(bi_gemm(act, F, w_d, F, x, D, BI_F32_ADD, T, D, F, stream));  // x += down proj
+      BI_TRY(f16m ? rmsnorm_f32in_f16(x, mlp_norm, h, T, D, c.rms_eps, s)
+                  : bi_rmsnorm_f32in(x, mlp_norm, h, T, D, c.rms_eps, stream));
+      // act = swiglu(gate, up); x += down proj
+      BI_TRY(f16m ? gemm_swiglu_e16<f16>(h, D, w_gu, D, act, F, T, F, D, s)
+                  : gemm_swiglu_e16<bf16>(h, D, w_gu, D, act, F, T, F, D, s));
+      BI_TRY(f16m ? gemm_e16<f16>(act, F, w_d, F, x, D, BI_F32_ADD, T, D, F, s)
+                  : gemm_e16<bf16>(act, F, w_d, F, x, D, BI_F32_ADD, T, D, F, s));
     }
   }
   if (b.n_logits == 0) return BI_OK;
@@ -298,8 +341,10 @@ extern "C" bi_status bi_forward(const bi_model* m, const bi_batch* bt, void* k_c
     BI_TRY(bi_gemm_x2(hl, hl_lo, D, m->w.lm_head, D, logits, c.vocab, BI_F32, b.n_logits, c.vocab, D,
                       stream));
   } else {
-    BI_TRY(bi_rmsnorm_f32in(xl, m->w.final_norm, hl, b.n_logits, D, c.rms_eps, stream));
-    BI_TRY(bi_gemm(hl, D, m->w.lm_head, D, logits, c.vocab, BI_F32, b.n_logits, c.vocab, D, stream));
+    BI_TRY(f16m ? rmsnorm_f32in_f16(xl, m->w.final_norm, hl, b.n_logits, D, c.rms_eps, s)
+                : bi_rmsnorm_f32in(xl, m->w.final_norm, hl, b.n_logits, D, c.rms_eps, stream));
+    BI_TRY(f16m ? gemm_e16<f16>(hl, D, m->w.lm_head, D, logits, c.vocab, BI_F32, b.n_logits, c.vocab, D, s)
+                : gemm_e16<bf16>(hl, D, m->w.lm_head, D, logits, c.vocab, BI_F32, b.n_logits, c.vocab, D, s));
   }
   if (next_tokens) BI_TRY(launch_argmax(logits, b.n_logits, c.vocab, c.vocab, next_tokens, s));
   return BI_OK;

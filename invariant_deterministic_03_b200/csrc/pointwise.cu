@@ -23,10 +23,11 @@ namespace pw {
 //   keys:   element (slot o, d) at (o/8)*1024 + (d/8)*64 + (o%8)*8 + d%8
 //   values: element (d, slot o) at (d/8)*128 + (o/8)*64 + (d%8)*8 + o%8
 // (element offsets inside the block; 8 x 8 core matrices of 128 bytes).
-__global__ void kv_append_kernel(const bf16* __restrict__ k_new, const bf16* __restrict__ v_new,
+// The copy moves 16-bit elements as bits, so it serves bf16 and fp16 caches.
+__global__ void kv_append_kernel(const uint16_t* __restrict__ k_new, const uint16_t* __restrict__ v_new,
                                  int64_t ld_new, const int32_t* __restrict__ slots, int64_t n_tok,
-                                 int Hkv, int num_pages, bf16* __restrict__ kc,
-                                 bf16* __restrict__ vc, int32_t* status) {
+                                 int Hkv, int num_pages, uint16_t* __restrict__ kc,
+                                 uint16_t* __restrict__ vc, int32_t* status) {
   const int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (wid >= n_tok * Hkv) return;
@@ -39,13 +40,13 @@ __global__ void kv_append_kernel(const bf16* __restrict__ k_new, const bf16* __r
     return;
   }
   const int page = slot / BI_PAGE_SIZE, o = slot % BI_PAGE_SIZE;
-  const bf16* ksrc = k_new + t * ld_new + (int64_t)g * BI_HEAD_DIM;
-  const bf16* vsrc = v_new + t * ld_new + (int64_t)g * BI_HEAD_DIM;
+  const uint16_t* ksrc = k_new + t * ld_new + (int64_t)g * BI_HEAD_DIM;
+  const uint16_t* vsrc = v_new + t * ld_new + (int64_t)g * BI_HEAD_DIM;
   const size_t blk = ((size_t)page * Hkv + g) * (BI_PAGE_SIZE * BI_HEAD_DIM);
   const int d0 = lane * 4;  // this lane's 4 consecutive d values (one core-matrix row half)
   const uint2 kv = reinterpret_cast<const uint2*>(ksrc)[lane];
   *reinterpret_cast<uint2*>(kc + blk + (o >> 3) * 1024 + (d0 >> 3) * 64 + (o & 7) * 8 + (d0 & 7)) = kv;
-  bf16* vdst = vc + blk + (o >> 3) * 64 + (o & 7);
+  uint16_t* vdst = vc + blk + (o >> 3) * 64 + (o & 7);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int d = d0 + i;
@@ -53,8 +54,9 @@ __global__ void kv_append_kernel(const bf16* __restrict__ k_new, const bf16* __r
   }
 }
 
-// ---- embedding gather into the fp32 residual stream
-__global__ void embed_kernel(const int32_t* __restrict__ tokens, const bf16* __restrict__ table,
+// ---- embedding gather into the fp32 residual stream (16-bit table, exact)
+template <typename ET>
+__global__ void embed_kernel(const int32_t* __restrict__ tokens, const ET* __restrict__ table,
                              int64_t vocab, int D, float* __restrict__ out, int32_t* status) {
   const int64_t t = blockIdx.x;
   const int32_t id = tokens[t];
@@ -64,12 +66,11 @@ __global__ void embed_kernel(const int32_t* __restrict__ tokens, const bf16* __r
     float v[8];
     if (ok) {
       const uint4 u = reinterpret_cast<const uint4*>(table + (size_t)id * D)[c];
-      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(h[i]);
-        v[2 * i] = f.x;
-        v[2 * i + 1] = f.y;
+        v[2 * i] = E16<ET>::lo(w[i]);
+        v[2 * i + 1] = E16<ET>::hi(w[i]);
       }
     } else {
 #pragma unroll
@@ -96,8 +97,8 @@ __global__ void rope_table_kernel(float* __restrict__ cs, int max_pos, double th
 // grid (token, head-pair block): each thread rotates 8 consecutive pairs
 // (i, i + 64), i = i0 .. i0+7, of one head with 16-byte accesses (rows
 // 16-byte aligned), or one pair (VEC == 1)
-template <int VEC>
-__global__ void rope_kernel(bf16* __restrict__ x, int64_t ldx, int n_heads,
+template <int VEC, typename ET>
+__global__ void rope_kernel(ET* __restrict__ x, int64_t ldx, int n_heads,
                             const int32_t* __restrict__ pos, const float* __restrict__ cs,
                             int max_pos, int32_t* status) {
   constexpr int PER_HEAD = 64 / VEC;
@@ -110,15 +111,15 @@ __global__ void rope_kernel(bf16* __restrict__ x, int64_t ldx, int n_heads,
     if (k == 0) set_status(status, BI_DEV_BAD_TOKEN);
     return;
   }
-  bf16* row = x + t * ldx + (int64_t)h * BI_HEAD_DIM;
+  ET* row = x + t * ldx + (int64_t)h * BI_HEAD_DIM;
   const float* csp = cs + ((size_t)p * 64 + i0) * 2;
   float a[VEC], b[VEC], c[VEC], sn[VEC];
   if constexpr (VEC == 8) {
     const uint4 av = *reinterpret_cast<const uint4*>(row + i0), bv = *reinterpret_cast<const uint4*>(row + i0 + 64);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      a[j] = __bfloat162float(reinterpret_cast<const bf16*>(&av)[j]);
-      b[j] = __bfloat162float(reinterpret_cast<const bf16*>(&bv)[j]);
+      a[j] = E16<ET>::to_f32(reinterpret_cast<const ET*>(&av)[j]);
+      b[j] = E16<ET>::to_f32(reinterpret_cast<const ET*>(&bv)[j]);
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -129,8 +130,8 @@ __global__ void rope_kernel(bf16* __restrict__ x, int64_t ldx, int n_heads,
       sn[2 * j + 1] = q.w;
     }
   } else {
-    a[0] = __bfloat162float(row[i0]);
-    b[0] = __bfloat162float(row[i0 + 64]);
+    a[0] = E16<ET>::to_f32(row[i0]);
+    b[0] = E16<ET>::to_f32(row[i0 + 64]);
     c[0] = csp[0];
     sn[0] = csp[1];
   }
@@ -140,13 +141,14 @@ __global__ void rope_kernel(bf16* __restrict__ x, int64_t ldx, int n_heads,
     rope_rotate(a[j], b[j], c[j], sn[j], ra[j], rb[j]);
   }
   if constexpr (VEC == 8) {
-    *reinterpret_cast<uint4*>(row + i0) = make_uint4(pack_bf16x2(ra[0], ra[1]), pack_bf16x2(ra[2], ra[3]),
-                                                     pack_bf16x2(ra[4], ra[5]), pack_bf16x2(ra[6], ra[7]));
-    *reinterpret_cast<uint4*>(row + i0 + 64) = make_uint4(pack_bf16x2(rb[0], rb[1]), pack_bf16x2(rb[2], rb[3]),
-                                                          pack_bf16x2(rb[4], rb[5]), pack_bf16x2(rb[6], rb[7]));
+    using E = E16<ET>;
+    *reinterpret_cast<uint4*>(row + i0) = make_uint4(E::pack2(ra[0], ra[1]), E::pack2(ra[2], ra[3]),
+                                                     E::pack2(ra[4], ra[5]), E::pack2(ra[6], ra[7]));
+    *reinterpret_cast<uint4*>(row + i0 + 64) = make_uint4(E::pack2(rb[0], rb[1]), E::pack2(rb[2], rb[3]),
+                                                          E::pack2(rb[4], rb[5]), E::pack2(rb[6], rb[7]));
   } else {
-    row[i0] = __float2bfloat16_rn(ra[0]);
-    row[i0 + 64] = __float2bfloat16_rn(rb[0]);
+    row[i0] = E16<ET>::from_f32(ra[0]);
+    row[i0 + 64] = E16<ET>::from_f32(rb[0]);
   }
 }
 
@@ -219,8 +221,8 @@ __global__ void argmax_kernel(const float* __restrict__ logits, int64_t V, int64
 
 }  // namespace pw
 
-bi_status launch_kv_append(const bf16* k, const bf16* v, int64_t ld_new, const int32_t* slots,
-                           int64_t n_tok, bf16* kc, bf16* vc, int Hkv, int num_pages,
+bi_status launch_kv_append(const uint16_t* k, const uint16_t* v, int64_t ld_new, const int32_t* slots,
+                           int64_t n_tok, uint16_t* kc, uint16_t* vc, int Hkv, int num_pages,
                            cudaStream_t s) {
   const int64_t warps = n_tok * Hkv;
   const int64_t blocks = (warps + 7) / 8;
@@ -230,25 +232,31 @@ bi_status launch_kv_append(const bf16* k, const bf16* v, int64_t ld_new, const i
   return BI_OK;
 }
 
-bi_status launch_embed(const int32_t* tok, int64_t n_tok, const bf16* table, int64_t vocab,
+template <typename ET>
+bi_status launch_embed(const int32_t* tok, int64_t n_tok, const ET* table, int64_t vocab,
                        int64_t D, float* out, cudaStream_t s) {
-  pw::embed_kernel<<<(unsigned)n_tok, 128, 0, s>>>(tok, table, vocab, (int)D, out, status_word());
+  pw::embed_kernel<ET><<<(unsigned)n_tok, 128, 0, s>>>(tok, table, vocab, (int)D, out, status_word());
   BI_CHECK_LAUNCH("embed launch");
   return BI_OK;
 }
+template bi_status launch_embed<bf16>(const int32_t*, int64_t, const bf16*, int64_t, int64_t, float*, cudaStream_t);
+template bi_status launch_embed<f16>(const int32_t*, int64_t, const f16*, int64_t, int64_t, float*, cudaStream_t);
 
-bi_status launch_rope(bf16* x, int64_t ldx, int n_heads, const int32_t* pos, int64_t n_tok,
+template <typename ET>
+bi_status launch_rope(ET* x, int64_t ldx, int n_heads, const int32_t* pos, int64_t n_tok,
                       const float* cs, int max_pos, cudaStream_t s) {
   if (n_tok == 0) return BI_OK;
   const bool vec = ldx % 8 == 0 && aligned16(x);
   const int64_t per_tok = (int64_t)n_heads * (vec ? 8 : 64);
   const dim3 grid((unsigned)n_tok, (unsigned)((per_tok + 255) / 256));
   if (n_tok > 0x7fffffff || grid.y > 65535) return fail(BI_ERR_SHAPE, "rope: size out of range");
-  if (vec) pw::rope_kernel<8><<<grid, 256, 0, s>>>(x, ldx, n_heads, pos, cs, max_pos, status_word());
-  else pw::rope_kernel<1><<<grid, 256, 0, s>>>(x, ldx, n_heads, pos, cs, max_pos, status_word());
+  if (vec) pw::rope_kernel<8, ET><<<grid, 256, 0, s>>>(x, ldx, n_heads, pos, cs, max_pos, status_word());
+  else pw::rope_kernel<1, ET><<<grid, 256, 0, s>>>(x, ldx, n_heads, pos, cs, max_pos, status_word());
   BI_CHECK_LAUNCH("rope launch");
   return BI_OK;
 }
+template bi_status launch_rope<bf16>(bf16*, int64_t, int, const int32_t*, int64_t, const float*, int, cudaStream_t);
+template bi_status launch_rope<f16>(f16*, int64_t, int, const int32_t*, int64_t, const float*, int, cudaStream_t);
 
 bi_status launch_swiglu(const bf16* gu, int64_t n_tok, int64_t F, bf16* out, cudaStream_t s) {
   const bool vec = F % 8 == 0 && aligned16(gu) && aligned16(out);
@@ -299,9 +307,9 @@ extern "C" bi_status bi_kv_append(const void* k_new, const void* v_new, int64_t 
     return fail(BI_ERR_ALIGN, "kv_append: rows must be 16-byte aligned");
   if (n_tok == 0) return BI_OK;
   if ((st = require_sm100()) != BI_OK) return st;
-  return launch_kv_append(static_cast<const bf16*>(k_new), static_cast<const bf16*>(v_new), ld_new,
-                          slot_mapping, n_tok, static_cast<bf16*>(k_cache),
-                          static_cast<bf16*>(v_cache), kv->num_kv_heads, kv->num_pages,
+  return launch_kv_append(static_cast<const uint16_t*>(k_new), static_cast<const uint16_t*>(v_new), ld_new,
+                          slot_mapping, n_tok, static_cast<uint16_t*>(k_cache),
+                          static_cast<uint16_t*>(v_cache), kv->num_kv_heads, kv->num_pages,
                           static_cast<cudaStream_t>(stream));
 }
 
@@ -314,7 +322,7 @@ extern "C" bi_status bi_embed(const int32_t* tokens, int64_t n_tok, const void* 
   if (n_tok == 0) return BI_OK;
   bi_status st = require_sm100();
   if (st != BI_OK) return st;
-  return launch_embed(tokens, n_tok, static_cast<const bf16*>(table), vocab, D, out,
+  return launch_embed<bf16>(tokens, n_tok, static_cast<const bf16*>(table), vocab, D, out,
                       static_cast<cudaStream_t>(stream));
 }
 
@@ -337,7 +345,7 @@ extern "C" bi_status bi_rope(void* x, int64_t ldx, int32_t n_heads, const int32_
   if (n_tok == 0) return BI_OK;
   bi_status st = require_sm100();
   if (st != BI_OK) return st;
-  return launch_rope(static_cast<bf16*>(x), ldx, n_heads, positions, n_tok, cos_sin, max_pos,
+  return launch_rope<bf16>(static_cast<bf16*>(x), ldx, n_heads, positions, n_tok, cos_sin, max_pos,
                      static_cast<cudaStream_t>(stream));
 }
 

@@ -36,6 +36,19 @@ struct Row8<bf16> {
 };
 
 template <>
+struct Row8<f16> {
+  static __device__ __forceinline__ void load(const f16* p, float (&v)[8]) {
+    uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = E16<f16>::lo(w[i]);
+      v[2 * i + 1] = E16<f16>::hi(w[i]);
+    }
+  }
+};
+
+template <>
 struct Row8<float> {
   static __device__ __forceinline__ void load(const float* p, float (&v)[8]) {
     float4 a = *reinterpret_cast<const float4*>(p);
@@ -47,11 +60,13 @@ struct Row8<float> {
 
 // CPT = chunks per thread (compile-time so the row stays in registers).
 // SPLIT: write the fp32 result as a bf16 pair (y = bf16(v), y_lo = bf16(v - y))
-// for the fp32-activation path; otherwise y = bf16(v).
-template <typename Tin, int CPT, bool SPLIT>
+// for the fp32-activation path; otherwise y = r16(v), r16 the rounding to
+// the 16-bit output type ET (bf16, or fp16 for the FP16 variant; gamma has
+// the same type).
+template <typename Tin, int CPT, bool SPLIT, typename ET>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const Tin* __restrict__ x,
-                                                      const bf16* __restrict__ gamma,
-                                                      bf16* __restrict__ y, bf16* __restrict__ y_lo,
+                                                      const ET* __restrict__ gamma,
+                                                      ET* __restrict__ y, ET* __restrict__ y_lo,
                                                       int D, float eps) {
   __shared__ float warp_sum[32];
   __shared__ float row_scale;
@@ -60,7 +75,7 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const Tin* __restrict__ x,
   const int nchunks = D >> 3;
   const size_t row = blockIdx.x;
   const Tin* xr = x + row * (size_t)D;
-  bf16* yr = y + row * (size_t)D;
+  ET* yr = y + row * (size_t)D;
 
   float v[CPT][8];
   float ss = 0.0f;
@@ -91,7 +106,7 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const Tin* __restrict__ x,
     int c = t + i * T;
     if (c < nchunks) {
       float g[8];
-      Row8<bf16>::load(gamma + c * 8, g);
+      Row8<ET>::load(gamma + c * 8, g);
       uint4 o, olo;
       uint32_t* op = reinterpret_cast<uint32_t*>(&o);
       uint32_t* olp = reinterpret_cast<uint32_t*>(&olo);
@@ -99,7 +114,7 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const Tin* __restrict__ x,
       for (int e = 0; e < 4; ++e) {
         const float a = __fmul_rn(__fmul_rn(v[i][2 * e], r), g[2 * e]);
         const float b = __fmul_rn(__fmul_rn(v[i][2 * e + 1], r), g[2 * e + 1]);
-        op[e] = pack_bf16x2(a, b);
+        op[e] = E16<ET>::pack2(a, b);
         if (SPLIT) {
           const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162*>(&op[e]);
           const float2 hf = __bfloat1622float2(hb);
@@ -124,18 +139,18 @@ static void rms_geometry(int64_t D, int* threads, int* cpt) {
   *cpt = p;
 }
 
-template <typename Tin, bool SPLIT = false>
-static bi_status launch_rms(const Tin* x, const bf16* g, bf16* y, int64_t M, int64_t D, float eps,
-                            cudaStream_t s, bf16* y_lo = nullptr) {
+template <typename Tin, bool SPLIT = false, typename ET = bf16>
+static bi_status launch_rms(const Tin* x, const ET* g, ET* y, int64_t M, int64_t D, float eps,
+                            cudaStream_t s, ET* y_lo = nullptr) {
   int T, cpt;
   rms_geometry(D, &T, &cpt);
   dim3 grid((unsigned)M), block(T);
   switch (cpt) {
-    case 1: rmsnorm_kernel<Tin, 1, SPLIT><<<grid, block, 0, s>>>(x, g, y, y_lo, (int)D, eps); break;
-    case 2: rmsnorm_kernel<Tin, 2, SPLIT><<<grid, block, 0, s>>>(x, g, y, y_lo, (int)D, eps); break;
-    case 4: rmsnorm_kernel<Tin, 4, SPLIT><<<grid, block, 0, s>>>(x, g, y, y_lo, (int)D, eps); break;
-    case 8: rmsnorm_kernel<Tin, 8, SPLIT><<<grid, block, 0, s>>>(x, g, y, y_lo, (int)D, eps); break;
-    case 16: rmsnorm_kernel<Tin, 16, SPLIT><<<grid, block, 0, s>>>(x, g, y, y_lo, (int)D, eps); break;
+    case 1: rmsnorm_kernel<Tin, 1, SPLIT, ET><<<grid, block, 0, s>>>(x, g, y, y_lo, (int)D, eps); break;
+    case 2: rmsnorm_kernel<Tin, 2, SPLIT, ET><<<grid, block, 0, s>>>(x, g, y, y_lo, (int)D, eps); break;
+    case 4: rmsnorm_kernel<Tin, 4, SPLIT, ET><<<grid, block, 0, s>>>(x, g, y, y_lo, (int)D, eps); break;
+    case 8: rmsnorm_kernel<Tin, 8, SPLIT, ET><<<grid, block, 0, s>>>(x, g, y, y_lo, (int)D, eps); break;
+    case 16: rmsnorm_kernel<Tin, 16, SPLIT, ET><<<grid, block, 0, s>>>(x, g, y, y_lo, (int)D, eps); break;
     default: return fail(BI_ERR_SHAPE, "rmsnorm: D=%lld unsupported", (long long)D);
   }
   BI_CHECK_LAUNCH("rmsnorm launch");
@@ -151,6 +166,16 @@ static bi_status check_rms(const void* x, const void* gamma, const void* y, int6
   if (!(eps >= 0.0f)) return fail(BI_ERR_INVALID_ARG, "rmsnorm: eps must be >= 0");
   if (!aligned16(x) || !aligned16(gamma) || !aligned16(y)) return fail(BI_ERR_ALIGN, "rmsnorm: pointers must be 16-byte aligned");
   return BI_OK;
+}
+
+// fp32 rows (the residual stream) to fp16 rows: the FP16 precision mode of
+// the forward.
+bi_status rmsnorm_f32in_f16(const float* x, const void* gamma, void* y, int64_t M, int64_t D, float eps,
+                            cudaStream_t s) {
+  bi_status st = check_rms(x, gamma, y, M, D, eps);
+  if (st != BI_OK || M == 0) return st;
+  if ((st = require_sm100()) != BI_OK) return st;
+  return launch_rms<float, false, f16>(x, static_cast<const f16*>(gamma), static_cast<f16*>(y), M, D, eps, s);
 }
 
 }  // namespace bi

@@ -48,7 +48,8 @@ def permutation(n: int, seed: int) -> torch.Tensor:
 
 
 def bf16_bits(t: torch.Tensor):
-    """bf16 tensor -> numpy uint16 bit patterns (the oracle's input form)."""
+    """16-bit (bf16 or fp16) tensor -> numpy uint16 bit patterns (the
+    oracle's input form)."""
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view("uint16")
 
 
@@ -107,3 +108,8 @@ def model_weights(cfg: dict, seed: int, std: float = 0.02) -> dict:
     w["w_gate_up"] = torch.stack([normal_bf16((2 * F, D), std, seed * 100 + 12 + 5 * l) for l in range(L)]) if L else torch.empty(0, 2 * F, D, dtype=torch.bfloat16)
     w["w_down"] = torch.stack([normal_bf16((D, F), std, seed * 100 + 13 + 5 * l) for l in range(L)]) if L else torch.empty(0, D, F, dtype=torch.bfloat16)
     return w
+
+
+def to_f16(weights: dict) -> dict:
+    """The same weights in fp16 (nearest), for the FP16 precision variant."""
+    return {k: v.to(torch.float16) for k, v in weights.items()}

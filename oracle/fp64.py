@@ -29,6 +29,11 @@ def bf16_bits_to_f64(bits) -> np.ndarray:
     return u.view(np.float32).astype(np.float64)
 
 
+def f16_bits_to_f64(bits) -> np.ndarray:
+    """uint16 IEEE half bit patterns -> float64 holding the exact same values."""
+    return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
 def f64_to_bf16_bits(x) -> np.ndarray:
     """float64 -> nearest bf16 (round to nearest, ties to even) as uint16.
 
@@ -220,8 +225,9 @@ def argmax_first(x) -> np.ndarray:
 # dense decoder forward
 
 class ModelWeights:
-    """bf16 weights of a dense pre-norm decoder, held as uint16 bit patterns
-    (numpy), converted to float64 one matrix at a time.
+    """16-bit weights of a dense pre-norm decoder (bf16, or fp16 with
+    fmt="f16"), held as uint16 bit patterns (numpy), converted to float64 one
+    matrix at a time.
 
     Arrays (nn.Linear layout [out, in]):
       embed [V, D], attn_norm [L, D], w_qkv [L, (Hq + 2 Hkv) d, D],
@@ -229,13 +235,14 @@ class ModelWeights:
       w_down [L, D, F], final_norm [D], lm_head [V, D].
     """
 
-    def __init__(self, cfg: dict, arrays: dict):
+    def __init__(self, cfg: dict, arrays: dict, fmt: str = "bf16"):
         self.cfg = cfg
         self.a = arrays
+        self.fmt = fmt
 
     def get(self, name, layer=None) -> np.ndarray:
         arr = self.a[name] if layer is None else self.a[name][layer]
-        return bf16_bits_to_f64(arr)
+        return f16_bits_to_f64(arr) if self.fmt == "f16" else bf16_bits_to_f64(arr)
 
 
 def forward(weights: ModelWeights, tokens, depths=None):
@@ -297,8 +304,9 @@ def round_to(x, kind):
     """x rounded to a storage format, returned in float64.
 
     kind: None (kept in float64), "f32" (IEEE float32, nearest even),
-    "bf16" (bfloat16, nearest even) or "bf16x2" (an fp32 value carried as a
-    pair hi = bf16(v), lo = bf16(v - hi), v = f32(x); the value is hi + lo).
+    "bf16" (bfloat16, nearest even), "f16" (IEEE half, nearest even) or
+    "bf16x2" (an fp32 value carried as a pair hi = bf16(v), lo = bf16(v -
+    hi), v = f32(x); the value is hi + lo).
     Pure encoding: no arithmetic of the method.
     """
     x = np.asarray(x, dtype=np.float64)
@@ -308,6 +316,9 @@ def round_to(x, kind):
         return x.astype(np.float32).astype(np.float64)
     if kind == "bf16":
         return bf16_bits_to_f64(f64_to_bf16_bits(x))
+    if kind == "f16":
+        with np.errstate(over="ignore"):
+            return x.astype(np.float16).astype(np.float64)
     if kind == "bf16x2":
         v = x.astype(np.float32).astype(np.float64)
         hi = bf16_bits_to_f64(f64_to_bf16_bits(v))
@@ -318,8 +329,9 @@ def round_to(x, kind):
 
 # Storage format of each activation of the decoder forward, per precision
 # mode. The modes are the cross-vendor precision study's variants
-# (arXivDaily 2610.05458, abstract): all-bf16 activations, the full fp32
-# upcast, and the upcast with only the MLP blocks kept in bf16. READING: the
+# (arXivDaily 2610.05458, abstract): all-bf16 activations, all-fp16
+# activations, the full fp32 upcast, and the upcast with only the MLP blocks
+# kept in bf16. READING: the
 # pages name the variants, not where each rounds; these are the points at
 # which a kernel stack stores an activation in a narrower format than fp64:
 #   h        RMSNorm output feeding a GEMM (attention block: "h_attn",
@@ -335,6 +347,8 @@ def round_to(x, kind):
 ROUNDING = {
     "bf16": dict(h_attn="bf16", qkv="bf16", qk_rope="bf16", p="bf16", attn="bf16",
                  h_mlp="bf16", gu="bf16", act="bf16", resid="f32", h_final="bf16", logits="f32"),
+    "f16": dict(h_attn="f16", qkv="f16", qk_rope="f16", p="f16", attn="f16",
+                h_mlp="f16", gu="f16", act="f16", resid="f32", h_final="f16", logits="f32"),
     "f32": dict(h_attn="bf16x2", qkv="f32", qk_rope="f32", p="f32", attn="bf16x2",
                 h_mlp="bf16x2", gu="f32", act="bf16x2", resid="f32", h_final="bf16x2", logits="f32"),
     "bf16_mlp": dict(h_attn="bf16x2", qkv="f32", qk_rope="f32", p="f32", attn="bf16x2",

@@ -6,15 +6,21 @@ FFN 14336 SwiGLU, RoPE theta 1e4, vocab 32000), random-init bf16 weights
 that varies chunk sizes -- the request's logits (fp32) and tokens must be the
 same bits every time ("Defeating Nondeterminism in LLM Inference", section
 "Batch invariance and determinism": a request's output must not depend on
-the server's load). A short teacher-forced prefix is also checked against
-the fp64 oracle in the fp32-activation mode."""
+the server's load). The whole request (1400 prompt + 128 generated tokens)
+is also teacher-forced against the fp64 oracle at every position: the
+fp32-activation mode within 1e-2, the bf16 mode within 1.5x the error of the
+fp64 forward with bf16 storage at the same points (the cross-vendor paper's
+abstract reports the logit error of the two precisions)."""
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
 
 from invariant_deterministic_03_b200 import synth
 from oracle import fp64
-from tests.gpu_common import f64, same_bits
+from tests.gpu_common import all_position_logits, emulated_logit_bounds, f64, same_bits
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -29,10 +35,10 @@ def weights():
     return w, {k: v.cuda().contiguous() for k, v in w.items()}
 
 
-def _engine(cfg, wd, seed, max_tokens, pages=10240):
+def _engine(cfg, wd, seed, max_tokens, pages=10240, max_logits=64):
     from invariant_deterministic_03_b200 import runner
     return runner.Engine(cfg, wd, num_pages=pages, max_pages_per_seq=cfg["max_pos"] // 16,
-                         max_tokens=max_tokens, max_logits=64, seed=seed)
+                         max_tokens=max_tokens, max_logits=max_logits, seed=seed)
 
 
 def _serve(cfg, wd, others, sched_seed, engine_seed):
@@ -97,15 +103,47 @@ def test_config4_bitwise_across_cobatching(weights):
     assert tk == ref_toks and same_bits(lg, ref_logits)
 
 
-def test_config4_fp32_mode_prefix_vs_fp64(weights):
-    """fp32-activation mode, teacher forced on the first 24 prompt tokens:
-    max |logit - fp64| <= 1e-2 at the full 32-layer depth."""
+def test_config4_whole_request_vs_fp64(weights):
+    """Teacher forced over the whole request: the 1400 prompt tokens and the
+    128 tokens the bf16 path generates greedily, 1528 positions, against the
+    fp64 oracle forward. fp32-activation mode: max |logit - fp64| <= 1e-2 at
+    every position. bf16 mode: within 1.5x the rounding emulation's error;
+    and its teacher-forced rows at the 128 decode positions are the same bits
+    the decode steps produced (chunked prefill == decode). The errors are
+    written to $BI_RECORD_DIR/logit_error_7b_1400p128.json when that is set."""
     w, wd = weights
-    cfg = dict(CFG, precision="f32")
-    n = 24
-    toks = synth.randint(PROMPT, 0, CFG["vocab"] - 1, seed=1).tolist()[:n]
-    eng = _engine(cfg, wd, seed=9, max_tokens=256, pages=64)
-    lg = torch.cat([eng.step([(0, p, p + 1)], lambda s: toks)[0] for p in range(n)])
-    ref = fp64.forward(fp64.ModelWeights(CFG, {k: synth.bf16_bits(v) for k, v in w.items()}), toks)
-    err = np.abs(f64(lg) - ref)
-    assert err.max() <= 1e-2, f"max abs logit error {err.max():.3e}"
+    ref_logits, gen = _serve(CFG, wd, [], sched_seed=100, engine_seed=0)
+    prompt = synth.randint(PROMPT, 0, CFG["vocab"] - 1, seed=1).tolist()
+    seq = prompt + list(gen)                                  # 1528 tokens
+    ow = fp64.ModelWeights(CFG, {k: synth.bf16_bits(v) for k, v in w.items()})
+    ref = fp64.forward(ow, seq)                               # [1528, V]
+    rec = {"workload": "Mistral-7B shape, random-init bf16 (seed 0), 1400-token prompt (seed 1) + "
+                       "128 greedy tokens of the bf16 path, teacher forced, every position",
+           "positions": len(seq)}
+    got = {}
+    for mode in ("f32", "bf16"):
+        eng = _engine(dict(CFG, precision=mode), wd, seed=21, max_tokens=512, pages=256, max_logits=512)
+        lg = all_position_logits(eng, seq, 512)
+        torch.cuda.synchronize()
+        got[mode] = lg
+        d = f64(lg) - ref
+        rec[mode] = {"max_abs": float(np.max(np.abs(d))), "mean_abs": float(np.mean(np.abs(d))),
+                     "global_rel": float(np.linalg.norm(d) / np.linalg.norm(ref)),
+                     "top1_agreement": float(np.mean(f64(lg).argmax(1) == ref.argmax(1)))}
+        del eng
+        torch.cuda.empty_cache()
+    max_abs, grel, emu = emulated_logit_bounds(ow, seq, "bf16", ref)
+    rec["bf16"]["emulated"] = emu
+    rec["bf16"]["bound_max_abs"] = max_abs
+    rec["f32"]["bound_max_abs"] = 1e-2
+    rec["logit_rms"] = float(np.sqrt(np.mean(ref ** 2)))
+    out_dir = os.environ.get("BI_RECORD_DIR")
+    if out_dir:
+        os.makedirs(out_dir, exist_ok=True)
+        with open(os.path.join(out_dir, "logit_error_7b_1400p128.json"), "w") as f:
+            json.dump(rec, f, indent=1)
+    assert rec["f32"]["max_abs"] <= 1e-2, rec["f32"]
+    assert rec["bf16"]["max_abs"] <= max_abs, rec["bf16"]
+    assert rec["bf16"]["global_rel"] <= grel, rec["bf16"]
+    # positions 1399 .. 1526 predicted the generated tokens in the decode steps
+    assert same_bits(got["bf16"][PROMPT - 1:PROMPT - 1 + NEW], ref_logits)

@@ -47,8 +47,12 @@ def test_config1_rmsnorm_then_gemm(bi):
         assert same_bits(Cp, C[perm.cuda()])
 
 
+# M straddles the pair tile's row halves (128 rows per CTA, 256 per pair):
+# 129 and 255 leave part of the second CTA's rows live, 256 fills the pair,
+# 257 and 383 start a second pair tile
 @pytest.mark.parametrize("M,N,K", [(1, 8, 8), (5, 264, 72), (130, 520, 200), (257, 1032, 1000),
-                                   (128, 256, 64), (300, 776, 4104), (2, 16, 4096)])
+                                   (128, 256, 64), (300, 776, 4104), (2, 16, 4096), (129, 136, 64),
+                                   (255, 384, 136), (256, 128, 520), (383, 264, 264)])
 @pytest.mark.parametrize("out", ["bf16", "f32"])
 def test_ragged_shapes(bi, M, N, K, out):
     A = synth.normal_bf16((M, K), 1.0, M * 7 + K)
@@ -132,13 +136,31 @@ def test_linspace_batch_invariance_demo(bi):
 @pytest.mark.parametrize("M,N,K", [(1, 8, 8192), (5, 264, 8200), (130, 520, 8192), (300, 776, 9000),
                                    (129, 4096, 14336)])
 @pytest.mark.parametrize("out", ["bf16", "f32"])
-def test_split_k_shapes(bi, M, N, K, out):
-    """Weights with few column tiles and K >= 8192 take the fixed two-way K
-    split (cluster of two CTAs, halves combined acc0 + acc1): parity with the
+def test_long_k_shapes(bi, M, N, K, out):
+    """Narrow weights with a long K (the down projection's shape class): the
+    whole K loop of a tile stays in one CTA pair, in order; parity with the
     oracle on ragged shapes, and the last row alone gives the same bits."""
     A = synth.normal_bf16((M, K), 1.0, M * 17 + K)
     W = synth.normal_bf16((N, K), 0.02, N * 19 + K)
     dt = torch.bfloat16 if out == "bf16" else torch.float32
-    C = _parity(bi, A, W, dt, what=f"split-K gemm {M}x{N}x{K} {out}")
+    C = _parity(bi, A, W, dt, what=f"long-K gemm {M}x{N}x{K} {out}")
+    C1 = bi.gemm(dev(A[-1:]), dev(W), dt)
+    assert same_bits(C1[0], C[-1])
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 8, 8), (130, 520, 200), (257, 1032, 1000), (300, 776, 4104)])
+@pytest.mark.parametrize("out", ["f16", "f32"])
+def test_f16_gemm_parity_and_rows(bi, M, N, K, out):
+    """bi_gemm_f16 (the FP16 variant's GEMM: fp16 A and W, the same pair tile
+    and K order): parity with the oracle, and the last row alone gives the
+    same bits."""
+    A = synth.normal_bf16((M, K), 1.0, M * 29 + K).to(torch.float16)
+    W = synth.normal_bf16((N, K), 0.02, N * 31 + K).to(torch.float16)
+    dt = torch.float16 if out == "f16" else torch.float32
+    C = bi.gemm(dev(A), dev(W), dt)
+    a = fp64.f16_bits_to_f64(synth.bf16_bits(A))
+    w = fp64.f16_bits_to_f64(synth.bf16_bits(W))
+    got = fp64.f16_bits_to_f64(synth.bf16_bits(C.cpu())) if out == "f16" else f64(C)
+    check(got, fp64.gemm(a, w), fp64.gemm_reduction_scale(a, w), KAPPA, what=f"f16 gemm {M}x{N}x{K} {out}")
     C1 = bi.gemm(dev(A[-1:]), dev(W), dt)
     assert same_bits(C1[0], C[-1])

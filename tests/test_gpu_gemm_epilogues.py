@@ -29,9 +29,9 @@ def bi(cuda_device):
     return mod
 
 
-# the last two also take the fixed two-way K split (few column tiles, K >= 8192)
+# ragged shapes, rows on both CTAs of a pair tile, and long K on narrow weights
 SHAPES = [(1, 8, 8), (5, 264, 72), (130, 520, 200), (300, 776, 4104), (129, 4096, 4096),
-          (7, 264, 8200), (130, 4096, 14336)]
+          (7, 264, 8200), (130, 4096, 14336), (255, 136, 520), (257, 264, 136)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)
@@ -66,7 +66,8 @@ def test_gemm_add_k0_leaves_c(bi):
 
 
 @pytest.mark.parametrize("M,F,K", [(1, 8, 8), (5, 128, 64), (130, 136, 200), (300, 520, 4104),
-                                   (64, 1024, 512), (9, 136, 8192), (130, 520, 9000)])
+                                   (64, 1024, 512), (9, 136, 8192), (130, 520, 9000), (200, 136, 136),
+                                   (257, 72, 64)])
 def test_gemm_swiglu(bi, M, F, K):
     A = synth.normal_bf16((M, K), 1.0, M * 13 + K)
     W = synth.normal_bf16((2 * F, K), 0.05, F * 7 + K)

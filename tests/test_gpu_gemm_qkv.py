@@ -6,8 +6,8 @@ Nondeterminism in LLM Inference", section "How do we make kernels
 batch-invariant?": a pointwise step fused into the producer keeps each
 element's arithmetic, and the cache is still written before attention
 reads it). Shapes cover the 7B head layout, ragged K, head counts whose
-tiles mix q and k heads, a weight that takes the fixed K split (three
-launches), padding rows, and bad slots and positions."""
+tiles mix q and k heads, a long K, row counts on both CTAs of a pair
+tile, padding rows, and bad slots and positions."""
 import numpy as np
 import pytest
 import torch
@@ -71,7 +71,7 @@ def _case(bi, table, M, K, Hq, Hkv, seed, slots=None, positions=None, num_pages=
 
 @pytest.mark.parametrize("M,K,Hq,Hkv", [(1, 4096, 32, 8), (7, 4096, 32, 8), (130, 4096, 32, 8),
                                         (5, 72, 4, 2), (64, 200, 3, 1), (33, 520, 5, 3),
-                                        (17, 8200, 4, 2)])
+                                        (17, 8200, 4, 2), (200, 136, 6, 2), (300, 264, 4, 1)])
 def test_fused_equals_three_steps(bi, table, M, K, Hq, Hkv):
     st1, st2, _, _ = _case(bi, table, M, K, Hq, Hkv, seed=M * 31 + K)
     assert st1 == 0 and st2 == 0

@@ -4,11 +4,13 @@ bitwise, as computing its whole prompt itself ("Defeating Nondeterminism in
 LLM Inference", section "Batch-invariant attention": keys are reduced at the
 same absolute tile and split boundaries whether they were cached earlier or
 belong to the chunk in flight)."""
+import numpy as np
 import pytest
 import torch
 
 from invariant_deterministic_03_b200 import synth
-from tests.gpu_common import same_bits
+from oracle import fp64
+from tests.gpu_common import emulated_logit_bounds, f64, same_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -64,6 +66,14 @@ def test_prefix_reuse_is_bitwise(cuda_device, cfg, prefix, suffix):
     rows, new = _prefill_then_decode(eng, 1, b_toks, held, [17, 128, 1024], 6)
     assert new == ref_new
     assert same_bits(rows, ref_rows)
+    # and against the fp64 oracle, teacher forced on the forked request's
+    # tokens: row i is the logits at position len(b_toks) - 1 + i
+    seq = b_toks + new[:-1]
+    ow = fp64.ModelWeights(cfg, {k: synth.bf16_bits(v) for k, v in w.items()})
+    ref = fp64.forward(ow, seq)
+    max_abs, _, emu = emulated_logit_bounds(ow, seq, "bf16", ref)
+    err = np.max(np.abs(f64(rows) - ref[len(b_toks) - 1:]))
+    assert err <= max_abs, f"max abs logit error {err:.3e} (emulated {emu['max_abs']:.3e})"
 
     # releasing the source keeps the shared pages alive for the fork
     eng.kv.release(0)

@@ -572,6 +572,14 @@ def test_round_to_formats():
     y = fp64.round_to(x, "bf16x2")
     assert np.all(np.abs(y - x) <= 2.0 ** -16 * np.abs(x))
     assert fp64.round_to(np.array([1.0 + 2 ** -15]), "bf16x2")[0] == 1.0 + 2 ** -15
+    # IEEE half: 11 significant bits, ties to even, overflow past 65504,
+    # subnormal quantum 2^-24
+    h = fp64.round_to(np.array([1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11, 65504.0, 65520.0, 2.0 ** -25,
+                                1.5 * 2.0 ** -24, -2.5]), "f16")
+    assert list(h[:4]) == [1.0, 1 + 2.0 ** -9, 65504.0, np.inf]
+    assert list(h[4:]) == [0.0, 2.0 ** -23, -2.5]
+    bits = np.array([0x3C00, 0xC000, 0x0001, 0x7BFF], dtype=np.uint16)
+    np.testing.assert_array_equal(fp64.f16_bits_to_f64(bits), [1.0, -2.0, 2.0 ** -24, 65504.0])
 
 
 def test_forward_rounded_without_rounding_is_forward():

@@ -47,12 +47,10 @@ def _with_workspace(bi, q, kc, vc, bt, sl, shape):
 
 
 def _noalloc(bi, q, kc, vc, bt, sl, shape):
+    """Through the Python binding (which checks the tensors against the shape
+    and calls the C entry point)."""
     out = torch.full_like(q, float("nan"))
-    st = bi.lib.bi_attn_decode_noalloc(q.data_ptr(), q.stride(0), kc.data_ptr(), vc.data_ptr(),
-                                       bt.data_ptr(), sl.data_ptr(), q.shape[0], ctypes.byref(shape),
-                                       out.data_ptr(), out.stride(0),
-                                       torch.cuda.current_stream().cuda_stream)
-    assert st == bi.BI_OK, bi.lib.bi_last_error()
+    bi.bi_attn_decode_noalloc(q, kc, vc, bt, sl, shape, out)
     return out
 
 
@@ -67,6 +65,19 @@ def test_noalloc_decode_matches_workspace_decode_twice(bi):
         check(f64(got), f64(ref), what=f"noalloc call {i + 1}")
         assert same_bits(got, ref)
     assert bi.bi_device_status(clear=True) == 0
+
+
+def test_noalloc_binding_rejects_mismatched_tensors(bi):
+    """The binding refuses tensors that disagree with the shape fields the
+    kernel trusts, before anything reaches the device."""
+    q, kc, vc, bt, sl, shape = _decode_case(bi, [5, 6], seed=51)
+    out = torch.empty_like(q)
+    with pytest.raises(ValueError):
+        bi.bi_attn_decode_noalloc(q[:1], kc, vc, bt, sl, shape, out)          # fewer q rows than B
+    with pytest.raises(ValueError):
+        bi.bi_attn_decode_noalloc(q, kc[:1], vc, bt, sl, shape, out)          # cache below num_pages
+    with pytest.raises(ValueError):
+        bi.bi_attn_decode_noalloc(q, kc, vc, bt[:, :1], sl, shape, out)       # block table too narrow
 
 
 def test_noalloc_rejects_sizes_past_the_scratch(bi):
