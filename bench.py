@@ -39,10 +39,9 @@ SHAPES = [(4096, 14336), (14336, 4096)]          # (K, N)
 MS = [1 << i for i in range(13)]                 # 1 .. 4096
 COPIES = 3
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# dram__bytes_read.sum + dram__bytes_write.sum of one gemm_tcgen05_kernel<1, 0>
-# launch at M=4096 K=4096 N=14336 (profiles/gemm_tcgen05_m4096_k4096_n14336.md);
-# None until the current kernel has been captured
-GEMM_TRAFFIC_BYTES = None
+# dram__bytes_read.sum + dram__bytes_write.sum of one gemm_tcgen05_kernel<1, 0, bf16>
+# launch at M=4096 K=4096 N=14336 (profiles/gemm_tcgen05_m4096_k4096_n14336.md)
+GEMM_TRAFFIC_BYTES = 171.912960e6 + 100.647936e6
 RMS_MS = [1 << i for i in range(13)] + [16384, 65536]   # RMSNorm bandwidth sweep, D = 4096
 
 
@@ -899,7 +898,7 @@ def main():
     achieved = 2.0 * top["M"] * top["N"] * top["K"] / top["bi_ms"] / 1e9
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
                 "frac": achieved / peak_t, "traffic": GEMM_TRAFFIC_BYTES,
-                "kernel": "bi_gemm (gemm_tcgen05_kernel<1, 0>), launch M=4096 K=4096 N=14336",
+                "kernel": "bi_gemm (gemm_tcgen05_kernel<1, 0, bf16>), launch M=4096 K=4096 N=14336",
                 "algorithmic_bytes": 2.0 * (top["M"] * top["K"] + top["N"] * top["K"] + top["M"] * top["N"]),
                 "peak_source": f"{peak_src} bf16 dense burst (launch timed alone)",
                 "frac_of_sustained": achieved / peak_sus if peak_sus else None}

@@ -39,10 +39,10 @@ def _rows(V):
             r[t % V] = 9.5
         rows.append(r)
     r = rng.standard_normal(V).astype(np.float32)
-    r[[V - 1, 4, V // 2]] = np.nan
-    rows.append(r)                                   # first NaN: index 4
+    r[[V - 1, min(4, V - 2), V // 2]] = np.nan
+    rows.append(r)                                   # the first NaN wins
     r = rng.standard_normal(V).astype(np.float32)
-    r[7] = np.inf
+    r[min(7, V - 1)] = np.inf
     r[V - 3] = np.nan
     rows.append(r)                                   # NaN above +inf
     rows.append(np.full(V, -np.inf, np.float32))     # all -inf: index 0

@@ -77,7 +77,7 @@ def test_noalloc_binding_rejects_mismatched_tensors(bi):
     with pytest.raises(ValueError):
         bi.bi_attn_decode_noalloc(q, kc[:1], vc, bt, sl, shape, out)          # cache below num_pages
     with pytest.raises(ValueError):
-        bi.bi_attn_decode_noalloc(q, kc, vc, bt[:, :1], sl, shape, out)       # block table too narrow
+        bi.bi_attn_decode_noalloc(q, kc, vc, bt[:1], sl, shape, out)          # block table rows below B
 
 
 def test_noalloc_rejects_sizes_past_the_scratch(bi):
