@@ -21,12 +21,15 @@
 // rows are (query, q head of group g) pairs. Per 128-key tile:
 //   S  = Q K^T            tcgen05.mma M128 N128 K16 x8, fp32 in tensor memory
 //   per row: m' = the row's reference maximum (log2 domain; see
-//        new_reference), alpha = 2^(m-m'), P_j = bf16(2^(s_j - m')),
-//        l = alpha*l + sum_j P_j (four 32-key quarters, each left to right)
+//        new_reference), alpha = 2^(m-m'), P_j = r16(2^(s_j - m')) (r16:
+//        rounding to the 16-bit element type), and for each 32-key quarter q
+//        l_q = alpha*l_q + (the quarter's P_j summed left to right)
 //   O  = alpha*O          in tensor memory (skipped when alpha == 1)
 //   O += P V              tcgen05.mma M128 N128 K16 x8 (one 16-key page per MMA),
 //                         O accumulated in tensor memory
-// At the end of a split the unnormalised O and (m, l) go to the workspace.
+// At the end of a split the unnormalised O, m and l = ((l_0 + l_1) + l_2) +
+// l_3 go to the workspace. Decode (one query per item) and prefill (chunks)
+// run exactly this arithmetic per row, in two layouts of the softmax work.
 // A row takes part only in tiles whose first key is <= its position, so the
 // update sequence of a row is a function of (position, split) alone.
 // Masked keys get P = 0 by selection (never by arithmetic on -inf), and
@@ -81,7 +84,8 @@ struct Lay {
   static constexpr uint32_t OFF_P = OFF_Q + NQ * QP_BYTES;
   static constexpr uint32_t OFF_BAR = OFF_P + NP * QP_BYTES;
   static constexpr uint32_t OFF_RING = OFF_BAR + 256;   // producer's page-id ring [16 tiles][8 pages]
-  static constexpr uint32_t OFF_ITEMS = OFF_RING + 512;  // item ring [16] x 48 B, then one mbarrier per slot
+  static constexpr uint32_t OFF_RED = OFF_RING + 512;   // decode quarter exchange [2 slots][4 warps][8 heads] fp32
+  static constexpr uint32_t OFF_ITEMS = OFF_RED + (DECODE ? 256 : 0);  // item ring [16] x 48 B, then one mbarrier per slot
   static constexpr size_t SMEM_BYTES = 1024 + OFF_ITEMS + ITEM_RING * 48 + ITEM_RING * 8;
   static_assert(NK <= MAX_KV_BUF && NV <= MAX_KV_BUF, "barrier arrays hold 3 K and 3 V buffers");
   static_assert(OFF_Q % 1024 == 0 && OFF_P % 1024 == 0, "swizzled Q / P tiles need 1 KB alignment");
@@ -381,8 +385,9 @@ __device__ __forceinline__ void drain(uint64_t* bar, int fills) {
   }
 }
 
-// Split kernel. Persistent: one CTA per SM walks work items idx = blockIdx.x,
-// blockIdx.x + gridDim.x, ...; the three roles walk the same item sequence.
+// Split kernel. Persistent: one CTA per SM takes work items as they are
+// claimed at run time (claim_item); the three roles walk the same item
+// sequence through the shared item ring.
 // Tiles j are counted across items. The producer keeps K and V loads apart
 // (a K buffer is free once its QK^T is done, a V buffer once its PV is done)
 // and the MMA warp issues S(j) = Q K_j^T and O += P_j V_j as soon as each is
@@ -390,14 +395,16 @@ __device__ __forceinline__ void drain(uint64_t* bar, int fills) {
 // DECODE selects the softmax layout (see below); both layouts run the same
 // per-row arithmetic.
 //
-// Row arithmetic (thread = row, fixed order, same in decode and prefill):
+// Row arithmetic (fixed order, the same in decode and prefill):
 //   first tile of the split:  m = max_j s_j (log2 domain, s_j = S_ij * scale*log2e),
-//                             P_j = bf16(2^(s_j - m)), l = sum_j P_j, O = P V
+//                             P_j = r16(2^(s_j - m)), l_q = sum_{j in quarter q} P_j, O = P V
 //   later tiles:              c = max(m, max_j s_j); m' = m if c - m <= 8 else c
 //                             (new_reference), alpha = 2^(m - m'),
-//                             P_j = bf16(2^(s_j - m')), l = alpha*l + sum_j P_j,
+//                             P_j = r16(2^(s_j - m')), l_q = alpha*l_q + sum_{j in q} P_j,
 //                             O = alpha*O (fp32, skipped when alpha == 1), O += P V (MMA)
-// sums over j run j = 0..127 in order; masked keys have P_j = 0 by selection.
+//   end of the split:         l = ((l_0 + l_1) + l_2) + l_3
+// sums over j run left to right inside each 32-key quarter; masked keys have
+// P_j = 0 by selection.
 template <bool DECODE, typename ET>
 __global__ void __launch_bounds__(THREADS, 1)
     attn_split_kernel(const __grid_constant__ CUtensorMap tmQ, const Params p) {
@@ -418,6 +425,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* s_free = bars + 19;    // [NS]
   uint64_t* p_ready = bars + 22;   // [NP]
   uint64_t* o_ready = bars + 24;   // [NP]: P V of the tile that read P buffer i is done
+  uint64_t* x_bar = bars + 26;     // decode: quarter exchange among the 4 softmax warps
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 27);
   static_assert(28 * 8 <= 256, "barrier region");
   RingItem* item_ring = reinterpret_cast<RingItem*>(smem + L::OFF_ITEMS);
@@ -448,6 +456,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&p_ready[i], 128);
       mbar_init(&o_ready[i], 1);
     }
+    mbar_init(x_bar, 128);
     for (int i = 0; i < ITEM_RING; ++i) mbar_init(&item_bar[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -636,20 +645,22 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ------------------------------------------------ softmax warps 0-3
     // Prefill layout: thread r owns MMA row r = (query r / G, head r % G) and
     // all 128 keys of a tile (its four quarters in turn).
-    // Decode layout (one query per item): Q holds one 8-row core-matrix group
-    // (row i = head i < G) that the MMA repeats over all 128 rows, so tensor
-    // memory lane 32w + l holds head l % 8 for every warp w. Lane l of warp w
-    // takes head l % 8 and quarter l / 8 (keys 32 (l/8) .. +31) when that head
-    // belongs to the warp (head % 4 == w): the four lanes of a head in one
-    // warp combine their quarters by shuffles, so no warp waits for another.
+    // Decode layout (one query per item): the item's G head rows are loaded
+    // into rows 32w + i of every warp w (identical rows, identical S), and
+    // warp w computes quarter w (keys 32w .. 32w+31) of every head i < G;
+    // quarter maxima are exchanged through shared memory once per tile, and
+    // each warp keeps its quarter's running sum l_q, so the quarter sums are
+    // exchanged once per split. (A layout in which the four lanes of a head in
+    // one warp each take a quarter and combine by shuffles was measured
+    // slower: each lane then needs its own column range, four tensor-memory
+    // loads per tile instead of one.)
     constexpr bool decode = DECODE;
     const int r = threadIdx.x;  // 0..127 == TMEM lane
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const int qr = decode ? 0 : r / p.G;
-    const int hj = decode ? (lane & 7) : r - qr * p.G;
-    const int quarter_of_lane = lane >> 3;  // decode: this lane's quarter of the keys
-    const bool lane_owns = decode ? ((lane & 7) < p.G && (lane & 3) == warp) : true;
-    int j = 0;
+    const int hj = decode ? lane : r - qr * p.G;
+    float* red = reinterpret_cast<float*>(smem + L::OFF_RED);  // decode: [2 slots][4 warps][8 head rows]
+    int j = 0, xc = 0;
     bool ok = true;
     // waits until the P V product of tile jj (counted across this CTA's items) is done
     auto pv_done = [&](int jj) -> bool {
@@ -657,18 +668,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       return true;
     };
-    // decode: the 32 columns of quarter `quarter_of_lane` of this lane's tensor
-    // memory row at column base `col` (warp-collective loads of all four
-    // quarters; each lane keeps its own)
-    auto load_own_quarter = [&](uint32_t col, uint32_t (&out)[32]) {
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t tmp[32];
-        tmem_ld32(tmem + col + lane_off + c * 32, tmp);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) out[i] = quarter_of_lane == c ? tmp[i] : out[i];
-      }
+    // Exchange k writes and reads slot k & 1 of the shared buffer: a warp can
+    // be at most one exchange ahead of another (it passes exchange k + 1
+    // only once every warp has arrived there, i.e. has read exchange k), so
+    // two slots keep a fast warp from overwriting values a slow one still
+    // reads. Returns the slot's base (or -1 when the wait timed out).
+    auto exchange = [&](float v) -> int {
+      const int which = xc & 1;
+      if (lane < 8) red[(which * 4 + warp) * 8 + lane] = v;
+      mbar_arrive(x_bar);
+      const bool done = mbar_wait(x_bar, (uint32_t)xc & 1u, p.status, abort_flag);
+      ++xc;
+      return done ? which * 32 : -1;
     };
     for (int n = 0; ok; ++n) {
       int idx;
@@ -677,11 +688,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (idx < 0) break;
       const int q_idx = it.q_lo + qr;
       const int pos = it.L - it.nb + q_idx;
-      const bool row_valid = lane_owns && (q_idx < it.q_hi) && (pos >= it.key_lo);
+      const bool row_valid = (decode ? lane < p.G : true) && (q_idx < it.q_hi) && (pos >= it.key_lo);
       const bool warp_valid = decode ? true : __any_sync(0xffffffffu, row_valid);
       const int last_page = (it.L - 1) / PAGE;
       const int tail = it.L % PAGE;
-      float m = -INFINITY, l = 0.0f;
+      float m = -INFINITY, l = 0.0f;  // l: decode, this warp's quarter sum
+      float lq[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // prefill: the row's four quarter sums
       for (int t = 0; t < it.ntiles; ++t, ++j) {
         const int sb = j % L::NS;
         const int kb0 = (it.t0 + t) * TILE;
@@ -691,52 +703,40 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         float alpha = 1.0f, m_new = 0.0f;
         if constexpr (decode) {
-          // ---- decode layout: this lane's quarter of its head's row
+          // ---- decode layout: this warp's quarter of every head row
           uint32_t S[32], P[16];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) S[i] = 0u;
-          load_own_quarter(sb * 128, S);
+          tmem_ld32(tmem + sb * 128 + lane_off + warp * 32, S);
+          tmem_ld_wait();
           tc_fence_before();
           mbar_arrive(&s_free[sb]);
-          const int nq = min(32, max(0, nvalid - quarter_of_lane * 32));
-          // the row maximum over the four quarters (exact, any order)
-          float mraw = quarter_max(S, nq);
-          mraw = fmaxf(mraw, __shfl_xor_sync(0xffffffffu, mraw, 8));
-          mraw = fmaxf(mraw, __shfl_xor_sync(0xffffffffu, mraw, 16));
+          const int nq = min(32, max(0, nvalid - warp * 32));
+          const int xm = exchange(quarter_max(S, nq));
+          if (xm < 0) { ok = false; break; }
+          float mraw = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) mraw = fmaxf(mraw, red[xm + w * 8 + (lane & 7)]);
           if (need) {
             m_new = new_reference(m, __fmul_rn(mraw, p.scale_log2), t);
             alpha = ex2_approx(__fsub_rn(m, m_new));
           }
           const float qs = quarter_p<ET>(S, nq, -m_new, p.scale_log2, P);
-          // quarter sums of the head, in quarter order, as in prefill
-          const int h0 = lane & 7;
-          const float q0 = __shfl_sync(0xffffffffu, qs, h0);
-          const float q1 = __shfl_sync(0xffffffffu, qs, h0 + 8);
-          const float q2 = __shfl_sync(0xffffffffu, qs, h0 + 16);
-          const float q3 = __shfl_sync(0xffffffffu, qs, h0 + 24);
           if (need) {
-            const float lsum = __fadd_rn(__fadd_rn(__fadd_rn(q0, q1), q2), q3);
-            l = (t == 0) ? lsum : __fadd_rn(__fmul_rn(alpha, l), lsum);
+            l = (t == 0) ? qs : __fadd_rn(__fmul_rn(alpha, l), qs);  // this warp's quarter
             m = m_new;
           }
           // P buffer j % NP was last read by the P V of tile j - NP
           if (j >= L::NP && !pv_done(j - L::NP)) { ok = false; break; }
-          if (lane_owns) store_p_chunks(smem + OFF_P + (j % L::NP) * L::QP_BYTES, L::HALF, h0, quarter_of_lane, P);
+          if (lane < p.G) store_p_chunks(smem + OFF_P + (j % L::NP) * L::QP_BYTES, L::HALF, lane, warp, P);
           if (t > 0 && __any_sync(0xffffffffu, need && alpha != 1.0f)) {
-            // O may be rescaled only once the P V of tile j-1 has landed in
-            // it; each lane scales its whole row (all four quarters), so every
-            // copy of a head's row that a lane of this warp owns stays whole
+            // O may be rescaled only once the P V of tile j-1 has landed in it
             if (L::NP > 1 && !pv_done(j - 1)) { ok = false; break; }
+            uint32_t o[32];
+            tmem_ld32(tmem + TMEM_O + lane_off + warp * 32, o);
+            tmem_ld_wait();
             const float a = need ? alpha : 1.0f;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-              uint32_t o[32];
-              tmem_ld32(tmem + TMEM_O + lane_off + c * 32, o);
-              tmem_ld_wait();
 #pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__fmul_rn(__uint_as_float(o[i]), a));
-              tmem_st32(tmem + TMEM_O + lane_off + c * 32, o);
-            }
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__fmul_rn(__uint_as_float(o[c]), a));
+            tmem_st32(tmem + TMEM_O + lane_off + warp * 32, o);
             tmem_st_wait();
           }
         } else {
@@ -769,8 +769,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                                 min(32, max(0, nvalid - q * 32)), -m_new, p.scale_log2,
                                 *reinterpret_cast<uint32_t(*)[16]>(&P[q * 16]));
             if (need) {
-              const float lsum = __fadd_rn(__fadd_rn(__fadd_rn(qs[0], qs[1]), qs[2]), qs[3]);
-              l = (t == 0) ? lsum : __fadd_rn(__fmul_rn(alpha, l), lsum);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) lq[q] = (t == 0) ? qs[q] : __fadd_rn(__fmul_rn(alpha, lq[q]), qs[q]);
               m = m_new;
             }
           }
@@ -819,22 +819,28 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!pv_done(j - 1)) { ok = false; break; }
       const size_t widx = ((size_t)(it.r0 + q_idx) * p.Hq + (size_t)(it.g * p.G + hj)) * p.n_split_max + it.s;
       if constexpr (decode) {
+        // the row's sum: its four quarter sums, in quarter order
+        const int xl = exchange(l);
+        if (xl < 0) { ok = false; break; }
+        const int h8 = lane & 7;
+        const float lrow = __fadd_rn(__fadd_rn(__fadd_rn(red[xl + h8], red[xl + 8 + h8]), red[xl + 16 + h8]),
+                                     red[xl + 24 + h8]);
         uint32_t o[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = 0u;
-        load_own_quarter(TMEM_O, o);
+        tmem_ld32(tmem + TMEM_O + lane_off + warp * 32, o);
+        tmem_ld_wait();
         if (row_valid) {
-          float* dst = p.ws_o + widx * HD + quarter_of_lane * 32;
+          float* dst = p.ws_o + widx * HD + warp * 32;
 #pragma unroll
           for (int c4 = 0; c4 < 8; ++c4)
             reinterpret_cast<float4*>(dst)[c4] =
                 make_float4(__uint_as_float(o[4 * c4]), __uint_as_float(o[4 * c4 + 1]),
                             __uint_as_float(o[4 * c4 + 2]), __uint_as_float(o[4 * c4 + 3]));
-          if (quarter_of_lane == 0) *reinterpret_cast<float2*>(p.ws_ml + widx * 2) = make_float2(m, l);
+          if (warp == 0) *reinterpret_cast<float2*>(p.ws_ml + widx * 2) = make_float2(m, lrow);
         }
       } else if (warp_valid) {
         float* dst = p.ws_o + widx * HD;
-        if (row_valid) *reinterpret_cast<float2*>(p.ws_ml + widx * 2) = make_float2(m, l);
+        const float lrow = __fadd_rn(__fadd_rn(__fadd_rn(lq[0], lq[1]), lq[2]), lq[3]);
+        if (row_valid) *reinterpret_cast<float2*>(p.ws_ml + widx * 2) = make_float2(m, lrow);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint32_t o[32];
