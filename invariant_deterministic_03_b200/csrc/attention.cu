@@ -56,25 +56,29 @@ constexpr uint32_t TILE_BYTES = 128 * 128 * 2;  // 32 KB: one K or V tile (128 k
 constexpr int ITEM_RING = 16;                   // claimed work items in flight inside a CTA
 constexpr int MAX_KV_BUF = 3;
 
-// Shared-memory layout. Prefill: Q (one buffer, released after an item's
-// last Q K^T so the next item's Q loads while its softmax finishes) and P are
-// full 128-row tiles, three K buffers and two V buffers (one Q buffer less and
-// a third K buffer measured ~2 % faster than two of each: the K copies land
-// 1.5-3 us after issue and gate Q K^T). Decode: the MMA rows
-// that matter are the G <= 8 head rows of one query, so Q and P keep just one
-// 8-row core-matrix group per 64-column half and the MMA operand descriptor
-// repeats it for all 16 groups (8-row-group stride 0): the same 128-row MMA
-// reads the same values in every row that matters, and the ~90 KB saved buy a
-// third K and a third V buffer and a second P buffer (so the softmax of tile
-// j+1 can store its P while the P V product of tile j still runs); decode
-// keeps two compact Q buffers.
+// Shared-memory layout. Prefill: Q and P are full 128-row tiles, one buffer
+// each (Q is released after an item's last Q K^T, so the next item's Q loads
+// while its softmax finishes), two K and three V buffers (the V copies are
+// the ones the P V products wait for; two K and three V measured ~2 % faster
+// than three K and two V). Decode: the MMA rows that matter are the G <= 8
+// head rows of one query, so Q and P keep just one 8-row core-matrix group
+// per 64-column half and the MMA operand descriptor repeats it for all 16
+// groups (8-row-group stride 0): the same 128-row MMA reads the same values
+// in every row that matters, and the ~90 KB saved buy a third K and a third
+// V buffer and a second P buffer (so the softmax of tile j+1 can store its P
+// while the P V product of tile j still runs); decode keeps two compact Q
+// buffers.
 template <bool DECODE>
 struct Lay {
-  static constexpr int NK = 3;                              // K tile buffers
+  static constexpr int NK = DECODE ? 3 : 2;                 // K tile buffers
   static constexpr int NQ = DECODE ? 2 : 1;                 // Q buffers
-  static constexpr int NV = DECODE ? 3 : 2;                 // V tile buffers
+  static constexpr int NV = 3;                              // V tile buffers
   static constexpr int NP = DECODE ? 2 : 1;                 // P buffers
   static constexpr int NS = DECODE ? 3 : 2;                 // S buffers in tensor memory
+  static constexpr int SOFTMAX_WARPS = DECODE ? 4 : 16;     // one 32-key quarter of 32 rows each
+  static constexpr int SOFTMAX_THREADS = SOFTMAX_WARPS * 32;
+  static constexpr int PRODUCER_WARP = SOFTMAX_WARPS;       // then the MMA / tensor-memory warp, the scheduler warp
+  static constexpr int THREADS = SOFTMAX_THREADS + 96;
   static constexpr uint32_t HALF = DECODE ? 1024 : 16384;   // bytes between the 64-column halves of Q / P
   static constexpr uint32_t ROW_SBO = DECODE ? 0 : 1024;    // bytes between 8-row groups of Q / P
   static constexpr uint32_t QP_BYTES = 2 * HALF;            // one Q or P buffer
@@ -91,12 +95,15 @@ struct Lay {
   static_assert(OFF_Q % 1024 == 0 && OFF_P % 1024 == 0, "swizzled Q / P tiles need 1 KB alignment");
   static_assert(SMEM_BYTES <= 232448, "attention: shared memory above the 227 KB per-CTA limit");
 };
-// warps 0-3: one thread per MMA row (softmax, O rescale, partials)
-// warp 4: TMA producer; warp 5: TMEM allocator and MMA issuer
-constexpr int THREADS = 192;
-// tensor memory: S buffers at columns [0,128), [128,256) and (decode) [256,384); O at [384,512)
+// Warps 0 .. SOFTMAX_WARPS-1: softmax, O rescale and partials (one 32-key
+// quarter of 32 MMA rows per warp); then the TMA producer warp, the
+// tensor-memory allocator and MMA issuer warp, and the scheduler warp.
+// Tensor memory: S buffers at columns [0,128), [128,256) and (decode)
+// [256,384); in prefill columns [256,264) carry the quarter exchange; O at
+// [384,512).
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TMEM_O = 384;  // S buffers at [0,128), [128,256) (and in decode [256,384))
+constexpr uint32_t TMEM_X = 256;
+constexpr uint32_t TMEM_O = 384;
 
 struct Params {
   const uint8_t* kc;  // 16-bit key cache, 4 KB per (page, kv head) block
@@ -112,6 +119,7 @@ struct Params {
   int32_t* work_counter;  // next unclaimed work item (zeroed before the launch)
   float scale_log2;
   int32_t* status;
+  int32_t ws_wide;  // ws_o is 32-byte aligned: partial rows go out in 256-bit stores
 };
 
 // One unit of work: (split s, sequence b, query block, kv head g).
@@ -188,19 +196,12 @@ __device__ __forceinline__ const uint8_t* block_src(const uint8_t* cache, int32_
   return pid < 0 ? g_attn_zero_block : cache + ((size_t)pid * Hkv + g) * BLOCK_BYTES;
 }
 
-// Work items are claimed at run time: the producer's look-ahead cursor takes
-// the next index from a global counter (atomicAdd -- scheduling only, no
-// value is ever reduced through it), skips items with no work, and publishes
-// each claimed item, decoded (or -1 at the end), in a shared ring with one
-// mbarrier per slot; every other role walks the ring in order. Which CTA runs
-// an item never reaches its arithmetic. The look-ahead is bounded by the
-// buffers: the claiming cursor runs at most PF_AHEAD + 1 tiles ahead of the K
-// loads, which run at most NK tiles ahead of QK^T, which runs at most NS
-// tiles ahead of the softmax, and the V loads trail the softmax by at most
-// NP tiles -- 13 tiles (so at most 13 items) in decode, 11 in prefill,
-// inside the 16-slot ring.
-// (Claiming one index ahead, to hide the atomic's latency, was measured
-// slower: a CTA holding an item it has not started delays the tail.)
+// Work items are claimed at run time: the scheduler warp takes the next
+// index from a global counter (atomicAdd -- scheduling only, no value is ever
+// reduced through it), skips items with no work, and publishes each claimed
+// item, decoded (or -1 at the end), in a shared ring with one mbarrier per
+// slot; every other role walks the ring in order. Which CTA runs an item
+// never reaches its arithmetic.
 __device__ __forceinline__ int claim_item(const Params& p, int lane, Item& it) {
   while (true) {
     int v = 0;
@@ -253,28 +254,26 @@ __device__ __forceinline__ bool cursor_start(const Params& p, Cursor& c, const R
   return cursor_next(p, c, ring, ibar, abort_flag);
 }
 
-// The producer's look-ahead cursor: claims and publishes items.
-__device__ __forceinline__ void claim_next(const Params& p, Cursor& c, RingItem* ring, uint64_t* ibar,
-                                           int lane) {
-  if (c.valid && ++c.t < c.it.ntiles) return;
-  c.t = 0;
-  ++c.n;
-  const int idx = claim_item(p, lane, c.it);
-  c.valid = idx >= 0;
-  if (lane == 0) {
-    const int slot = c.n & (ITEM_RING - 1);
-    volatile int32_t* e = reinterpret_cast<volatile int32_t*>(&ring[slot]);
-    e[0] = idx;
-    const int* src = reinterpret_cast<const int*>(&c.it);
-#pragma unroll
-    for (int i = 0; i < 11; ++i) e[1 + i] = src[i];
-    mbar_arrive(&ibar[slot]);  // release: the entry is visible to whoever sees the phase
-  }
-}
-
-constexpr int PF_AHEAD = 4;   // page-table lookups run this many tiles ahead of the K loads
-constexpr int PF_RING = 16;   // looked-up page ids, from the oldest V load to the newest lookup
+constexpr int PF_AHEAD = 4;     // page-table lookups run this many tiles ahead of the K loads
+constexpr int PF_RING = 16;     // looked-up page ids, from the oldest V load to the newest lookup
+constexpr int SCHED_AHEAD = 1;  // ring entries the scheduler publishes ahead of the page look-ahead
 static_assert(PF_RING * 8 * 4 <= 512, "page-id ring overflows its region");
+// Ring bounds. With j the tile the softmax is on: S(n) is issued only once
+// the softmax has read S(n - NS), K(n) only once S(n - NK) is done, and the
+// look-ahead is PF_AHEAD tiles past the K copies, so it is at most NS + NK +
+// PF_AHEAD tiles past j; the softmax passes tile j only after the P V of
+// tile j - NP was issued, so every V copy up to j - NP + 1 is out. Every role
+// reads its items from the ring in order and every item has a tile, so from
+// the slowest reader to the look-ahead there are at most NS + NK + PF_AHEAD +
+// NP - 1 tiles (11 in decode, 8 in prefill), and the scheduler adds
+// SCHED_AHEAD entries; both rings hold 16.
+template <bool DECODE>
+constexpr bool rings_fit() {
+  using L = Lay<DECODE>;
+  return L::NS + L::NK + PF_AHEAD + L::NP - 1 + SCHED_AHEAD <= ITEM_RING &&
+         L::NS + L::NK + PF_AHEAD + L::NP - 1 < PF_RING;
+}
+static_assert(rings_fit<true>() && rings_fit<false>(), "item or page-id ring too small for the look-ahead");
 
 // S = Q K^T. Q: 128 rows x 128 d, 128-byte swizzle in two 64-column halves.
 // K: 8 page blocks of 16 keys, canonical no-swizzle K-major: core matrices of
@@ -320,7 +319,8 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // One quarter (32 keys) of a row's tile: P_c = r16(2^(S_c * scale_log2 -
 // m)) for c < nvalid (else 0), r16 the rounding to the 16-bit element type,
 // packed two per word into P[0..15], and the quarter sum of the rounded
-// values, added left to right. Decode and prefill both build a row from
+// values, added left to right. P may alias S[0..15]: word c2 of P is written
+// after S[2 c2] and S[2 c2 + 1], the last elements it depends on, are read. Decode and prefill both build a row from
 // exactly these quarters, so their arithmetic is the same.
 template <typename ET>
 __device__ __forceinline__ float quarter_p(const uint32_t (&S)[32], int nvalid, float neg_m,
@@ -355,11 +355,18 @@ __device__ __forceinline__ float new_reference(float m, float tile_max, int t) {
   return (t > 0 && __fsub_rn(mc, m) <= RESCALE_LOG2) ? m : mc;
 }
 
+// The maximum of a quarter's first nvalid scores (-inf when none), by a
+// pairwise tree (depth 5 instead of a 32-long chain): max is exact, so any
+// order gives the same value for non-NaN scores; masked keys enter as -inf.
 __device__ __forceinline__ float quarter_max(const uint32_t (&S)[32], int nvalid) {
-  float m = -INFINITY;
+  float v[32];
 #pragma unroll
-  for (int c = 0; c < 32; ++c) m = fmaxf(m, c < nvalid ? __uint_as_float(S[c]) : -INFINITY);
-  return m;
+  for (int c = 0; c < 32; ++c) v[c] = c < nvalid ? __uint_as_float(S[c]) : -INFINITY;
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+    for (int c = 0; c < w; ++c) v[c] = fmaxf(v[c], v[c + w]);
+  return v[0];
 }
 
 // P row `row`, keys 32*quarter .. +31, into the 128-byte-swizzled P tile whose
@@ -406,7 +413,7 @@ __device__ __forceinline__ void drain(uint64_t* bar, int fills) {
 // sums over j run left to right inside each 32-key quarter; masked keys have
 // P_j = 0 by selection.
 template <bool DECODE, typename ET>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(Lay<DECODE>::THREADS, 1)
     attn_split_kernel(const __grid_constant__ CUtensorMap tmQ, const Params p) {
   using L = Lay<DECODE>;
   constexpr int NK = L::NK, NV = L::NV;
@@ -425,9 +432,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* s_free = bars + 19;    // [NS]
   uint64_t* p_ready = bars + 22;   // [NP]
   uint64_t* o_ready = bars + 24;   // [NP]: P V of the tile that read P buffer i is done
-  uint64_t* x_bar = bars + 26;     // decode: quarter exchange among the 4 softmax warps
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 27);
-  static_assert(28 * 8 <= 256, "barrier region");
+  uint64_t* x_bar = bars + 26;     // quarter exchange: decode [1], prefill [4] (one per lane group)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 30);
+  // ring entry (item) the producer's page look-ahead is on; the scheduler stays
+  // at most SCHED_AHEAD entries in front of it
+  volatile int* pf_item = reinterpret_cast<volatile int*>(bars + 31);
+  static_assert(32 * 8 <= 256, "barrier region");
   RingItem* item_ring = reinterpret_cast<RingItem*>(smem + L::OFF_ITEMS);
   uint64_t* item_bar = reinterpret_cast<uint64_t*>(smem + L::OFF_ITEMS + ITEM_RING * 48);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -442,7 +452,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int i = 0; i < L::NS; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
+      mbar_init(&s_free[i], L::SOFTMAX_THREADS);
     }
     for (int i = 0; i < NK; ++i) {
       mbar_init(&k_full[i], 1);
@@ -453,15 +463,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&v_empty[i], 1);
     }
     for (int i = 0; i < L::NP; ++i) {
-      mbar_init(&p_ready[i], 128);
+      mbar_init(&p_ready[i], L::SOFTMAX_THREADS);
       mbar_init(&o_ready[i], 1);
     }
-    mbar_init(x_bar, 128);
+    for (int i = 0; i < (DECODE ? 1 : 4); ++i) mbar_init(&x_bar[i], 128);
     for (int i = 0; i < ITEM_RING; ++i) mbar_init(&item_bar[i], 1);
     *abort_flag = 0;
+    *pf_item = -1;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == L::PRODUCER_WARP + 1) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
@@ -470,32 +481,39 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == L::PRODUCER_WARP) {
     // ------------------------------------------------ producer warp
-    // Lane 0 owns the barriers and the Q loads; lanes 0..7 each look up one
-    // page of a tile and issue that page's 4 KB copy, so a tile's eight
-    // copies go out together. All lanes walk the same cursors.
+    // Lane 0 owns the barriers and the Q loads; lanes 0..7 each own one page
+    // of a tile: its block-table entry is fetched PF_AHEAD tiles early by
+    // cp.async into the page-id ring (one commit group per tile), checked
+    // when the tile's K copies are issued, and each lane issues its page's
+    // 4 KB copy, so a tile's eight copies go out together. All lanes walk
+    // the same cursors (kc: K copies, vc: V copies, pf: page look-ahead).
     if (lane == 0) prefetch_tmap(&tmQ);
     const uint32_t q_bytes = 2u * 64u * 2u * (uint32_t)(p.G * p.q_box);
     int32_t* ring = reinterpret_cast<int32_t*>(smem + L::OFF_RING);  // [PF_RING][8]
+    // lanes 0..7: the block-table entries of the pf cursor's tile into a ring slot
+    auto lookup_pages = [&](const Cursor& c, int32_t* slot) {
+      if (lane < PAGES_PER_TILE) {
+        const int i = min((c.it.t0 + c.t) * PAGES_PER_TILE + lane, p.max_pages - 1);
+        cp_async4(slot + lane, p.block_table + (size_t)c.it.b * p.max_pages + i);
+      }
+    };
     Cursor kc, vc, pf;
-    pf.n = -1;
-    pf.t = 0;
-    pf.valid = false;
-    claim_next(p, pf, item_ring, item_bar, lane);  // publishes ring entry 0
-    bool ok = cursor_start(p, kc, item_ring, item_bar, abort_flag);
+    bool ok = cursor_start(p, pf, item_ring, item_bar, abort_flag);
+    if (lane == 0) *pf_item = pf.n;
+    if (ok) ok = cursor_start(p, kc, item_ring, item_bar, abort_flag);
     vc = kc;
     int nk = 0, nv = 0, npf = 0, qi = 0;
-    int q_fills[2] = {0, 0}, k_fills[NK] = {}, v_fills[NV] = {};
-    for (; pf.valid && npf < PF_AHEAD; ++npf, claim_next(p, pf, item_ring, item_bar, lane))
-      if (lane < PAGES_PER_TILE)
-        ring[(npf & (PF_RING - 1)) * 8 + lane] =
-            page_valid(p, pf.it.L, pf.it.t0 + pf.t, lane, tile_page_raw(p, pf.it.b, pf.it.t0 + pf.t, lane));
-    // one lookup in flight: its load is issued now and its result is checked
-    // and stored one K issue later, off the issue path
-    bool la_pending = false;
-    int32_t la_pid = -1;
-    int la_slot = 0, la_L = 0, la_tile = 0;
+    for (int i = 0; i < PF_AHEAD; ++i) {  // the first PF_AHEAD tiles' lookups
+      if (ok && pf.valid) {
+        lookup_pages(pf, ring + (npf & (PF_RING - 1)) * 8);
+        ++npf;
+        if (!cursor_next(p, pf, item_ring, item_bar, abort_flag)) ok = false;
+        if (lane == 0) *pf_item = pf.n;
+      }
+      cp_async_commit();  // one group per tile slot, empty past the last tile
+    }
     long long t_last = clock64();
     while ((kc.valid || vc.valid) && ok) {
       bool progressed = false;
@@ -517,29 +535,28 @@ __global__ void __launch_bounds__(THREADS, 1)
               tma_load_3d(qdst, &tmQ, &q_full[qb], 0, kc.it.g * p.G, kc.it.r0 + kc.it.q_lo);
               tma_load_3d(qdst + L::HALF, &tmQ, &q_full[qb], 64, kc.it.g * p.G, kc.it.r0 + kc.it.q_lo);
             }
-            ++q_fills[qb];
             ++qi;
           }
-          if (la_pending) {
-            if (lane < PAGES_PER_TILE) ring[la_slot * 8 + lane] = page_valid(p, la_L, la_tile, lane, la_pid);
-            la_pending = false;
+          // this tile's lookups (committed PF_AHEAD groups ago) have landed
+          cp_async_wait<PF_AHEAD - 1>();
+          int32_t* kslot = ring + (nk & (PF_RING - 1)) * 8;
+          int32_t pid = -1;
+          if (lane < PAGES_PER_TILE) {
+            pid = page_valid(p, kc.it.L, kc.it.t0 + kc.t, lane, kslot[lane]);
+            kslot[lane] = pid;  // the checked id, for this tile's V copy
           }
-          if (pf.valid) {  // keep the page lookups PF_AHEAD tiles ahead
-            la_tile = pf.it.t0 + pf.t;
-            la_L = pf.it.L;
-            la_slot = npf & (PF_RING - 1);
-            la_pid = lane < PAGES_PER_TILE ? tile_page_raw(p, pf.it.b, la_tile, lane) : -1;
-            la_pending = true;
+          if (pf.valid) {  // keep the lookups PF_AHEAD tiles ahead
+            lookup_pages(pf, ring + (npf & (PF_RING - 1)) * 8);
             ++npf;
-            claim_next(p, pf, item_ring, item_bar, lane);
+            if (!cursor_next(p, pf, item_ring, item_bar, abort_flag)) ok = false;
+            if (lane == 0) *pf_item = pf.n;
           }
+          cp_async_commit();
           if (lane == 0) mbar_arrive_expect_tx(&k_full[kb], TILE_BYTES);
           __syncwarp();
           if (lane < PAGES_PER_TILE)
-            bulk_load(smem + OFF_K + kb * TILE_BYTES + lane * BLOCK_BYTES,
-                      block_src(p.kc, ring[(nk & (PF_RING - 1)) * 8 + lane], p.Hkv, kc.it.g), BLOCK_BYTES,
-                      &k_full[kb]);
-          ++k_fills[kb];
+            bulk_load(smem + OFF_K + kb * TILE_BYTES + lane * BLOCK_BYTES, block_src(p.kc, pid, p.Hkv, kc.it.g),
+                      BLOCK_BYTES, &k_full[kb]);
           ++nk;
           if (!cursor_next(p, kc, item_ring, item_bar, abort_flag)) ok = false;
           progressed = true;
@@ -556,7 +573,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             bulk_load(smem + OFF_V + vb * TILE_BYTES + lane * BLOCK_BYTES,
                       block_src(p.vc, ring[(nv & (PF_RING - 1)) * 8 + lane], p.Hkv, vc.it.g), BLOCK_BYTES,
                       &v_full[vb]);
-          ++v_fills[vb];
           ++nv;
           if (!cursor_next(p, vc, item_ring, item_bar, abort_flag)) ok = false;
           progressed = true;
@@ -576,15 +592,57 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (__shfl_sync(0xffffffffu, stop, 0)) ok = false;
     }
-    // publish the rest of the claims up to the end marker: consumers may still
-    // be waiting for ring entries the look-ahead has not reached
-    while (ok && pf.valid) claim_next(p, pf, item_ring, item_bar, lane);
+    cp_async_wait<0>();  // no lookup still landing in shared memory
     if (!ok && lane == 0) {
-      for (int i = 0; i < 2; ++i) drain(&q_full[i], q_fills[i]);
-      for (int i = 0; i < NK; ++i) drain(&k_full[i], k_fills[i]);
-      for (int i = 0; i < NV; ++i) drain(&v_full[i], v_fills[i]);
+      // buffer i of a ring of nb took the copies numbered i, i + nb, ... below the count
+      auto fills = [](int count, int i, int nb) { return (count - i + nb - 1) / nb; };
+      for (int i = 0; i < L::NQ; ++i) drain(&q_full[i], fills(qi, i, L::NQ));
+      for (int i = 0; i < NK; ++i) drain(&k_full[i], fills(nk, i, NK));
+      for (int i = 0; i < NV; ++i) drain(&v_full[i], fills(nv, i, NV));
     }
-  } else if (warp == 5) {
+  } else if (warp == L::PRODUCER_WARP + 2) {
+    // ------------------------------------------------ scheduler warp
+    // Claims work items (claim_item) and publishes each, decoded, as the next
+    // ring entry (the end marker -1 last), at most SCHED_AHEAD entries in
+    // front of the one the producer's page look-ahead is on: the claim's
+    // atomic and the item's global loads overlap the copies instead of
+    // stalling the producer.
+    long long t_last = clock64();
+    for (int n = 0;; ++n) {
+      int go;
+      do {  // 0: wait for the look-ahead, 1: claim, 2: stop
+        go = 0;
+        if (lane == 0) {
+          if (n <= *pf_item + SCHED_AHEAD) {
+            go = 1;
+          } else if (*abort_flag) {
+            go = 2;
+          } else if (clock64() - t_last > kWaitLimitCycles) {
+            set_status(p.status, BI_DEV_WAIT_TIMEOUT);
+            *abort_flag = 1;
+            go = 2;
+          } else {
+            __nanosleep(64);
+          }
+        }
+        go = __shfl_sync(0xffffffffu, go, 0);
+      } while (go == 0);
+      if (go == 2) break;
+      Item it;
+      const int idx = claim_item(p, lane, it);
+      if (lane == 0) {
+        const int slot = n & (ITEM_RING - 1);
+        volatile int32_t* e = reinterpret_cast<volatile int32_t*>(&item_ring[slot]);
+        e[0] = idx;
+        const int* src = reinterpret_cast<const int*>(&it);
+#pragma unroll
+        for (int i = 0; i < 11; ++i) e[1 + i] = src[i];
+        mbar_arrive(&item_bar[slot]);  // release: the entry is visible to whoever sees the phase
+      }
+      t_last = clock64();
+      if (idx < 0) break;
+    }
+  } else if (warp == L::PRODUCER_WARP + 1) {
     // ------------------------------------------------ MMA issuer (one thread)
     if (lane == 0) {
       const uint32_t sQ0 = smem_u32(smem + OFF_Q), sK0 = smem_u32(smem + OFF_K);
@@ -642,24 +700,28 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
   } else {
-    // ------------------------------------------------ softmax warps 0-3
-    // Prefill layout: thread r owns MMA row r = (query r / G, head r % G) and
-    // all 128 keys of a tile (its four quarters in turn).
-    // Decode layout (one query per item): the item's G head rows are loaded
-    // into rows 32w + i of every warp w (identical rows, identical S), and
-    // warp w computes quarter w (keys 32w .. 32w+31) of every head i < G;
-    // quarter maxima are exchanged through shared memory once per tile, and
-    // each warp keeps its quarter's running sum l_q, so the quarter sums are
-    // exchanged once per split. (A layout in which the four lanes of a head in
-    // one warp each take a quarter and combine by shuffles was measured
-    // slower: each lane then needs its own column range, four tensor-memory
-    // loads per tile instead of one.)
+    // ------------------------------------------------ softmax warps
+    // Warp w owns one 32-key quarter of the S and P columns (and the same 32
+    // d columns of O) for the 32 MMA rows of its tensor-memory lane group.
+    // Prefill: 16 warps; lane group w % 4 (rows 32 (w % 4) .. +31), quarter
+    // w / 4; MMA row r = (query r / G, head r % G).
+    // Decode (one query per item): 4 warps; the item's G head rows are loaded
+    // into rows 32w + i of every lane group (identical rows, identical S), and
+    // warp w takes quarter w of every head i < G.
+    // The four quarters of a row meet in exchange(): their maxima once per
+    // tile and their sums l_q once per split. (In decode a layout in which the
+    // four lanes of a head in one warp each take a quarter and combine by
+    // shuffles was measured slower: each lane then needs its own column
+    // range, four tensor-memory loads per tile instead of one.)
     constexpr bool decode = DECODE;
-    const int r = threadIdx.x;  // 0..127 == TMEM lane
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int rg = decode ? warp : (warp & 3);        // tensor-memory lane group
+    const int quarter = decode ? warp : (warp >> 2);  // columns 32 quarter .. +31
+    const uint32_t lane_off = (uint32_t)(rg * 32) << 16;
+    const int r = decode ? lane : rg * 32 + lane;     // prefill: the MMA row
     const int qr = decode ? 0 : r / p.G;
     const int hj = decode ? lane : r - qr * p.G;
     float* red = reinterpret_cast<float*>(smem + L::OFF_RED);  // decode: [2 slots][4 warps][8 head rows]
+    uint64_t* xbar = decode ? x_bar : &x_bar[rg];
     int j = 0, xc = 0;
     bool ok = true;
     // waits until the P V product of tile jj (counted across this CTA's items) is done
@@ -668,18 +730,40 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       return true;
     };
-    // Exchange k writes and reads slot k & 1 of the shared buffer: a warp can
-    // be at most one exchange ahead of another (it passes exchange k + 1
-    // only once every warp has arrived there, i.e. has read exchange k), so
-    // two slots keep a fast warp from overwriting values a slow one still
-    // reads. Returns the slot's base (or -1 when the wait timed out).
-    auto exchange = [&](float v) -> int {
+    // The four warps that share this thread's row each contribute v, the
+    // value of their quarter; x[q] receives quarter q's value for the row.
+    // Decode meets in shared memory (its four warps sit in different lane
+    // groups), prefill in tensor-memory columns TMEM_X .. +7 of the lane group
+    // (shared memory is full). Exchange k uses slot k & 1: a warp can be at
+    // most one exchange ahead of another (it passes exchange k + 1 only once
+    // every warp has arrived there, i.e. has read exchange k), so two slots
+    // keep a fast warp from overwriting values a slow one still reads.
+    // False when the wait timed out.
+    auto exchange = [&](float v, float (&x)[4]) -> bool {
       const int which = xc & 1;
-      if (lane < 8) red[(which * 4 + warp) * 8 + lane] = v;
-      mbar_arrive(x_bar);
-      const bool done = mbar_wait(x_bar, (uint32_t)xc & 1u, p.status, abort_flag);
+      if constexpr (decode) {
+        if (lane < 8) red[(which * 4 + warp) * 8 + lane] = v;
+      } else {
+        tmem_st1(tmem + lane_off + TMEM_X + which * 4 + quarter, __float_as_uint(v));
+        tmem_st_wait();
+        tc_fence_before();
+      }
+      mbar_arrive(xbar);
+      const bool done = mbar_wait(xbar, (uint32_t)xc & 1u, p.status, abort_flag);
       ++xc;
-      return done ? which * 32 : -1;
+      if (!done) return false;
+      if constexpr (decode) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) x[w] = red[(which * 4 + w) * 8 + (lane & 7)];
+      } else {
+        tc_fence_after();
+        uint32_t u[4];
+        tmem_ld4(tmem + lane_off + TMEM_X + which * 4, u);
+        tmem_ld_wait();
+#pragma unroll
+        for (int w = 0; w < 4; ++w) x[w] = __uint_as_float(u[w]);
+      }
+      return true;
     };
     for (int n = 0; ok; ++n) {
       int idx;
@@ -689,121 +773,77 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int q_idx = it.q_lo + qr;
       const int pos = it.L - it.nb + q_idx;
       const bool row_valid = (decode ? lane < p.G : true) && (q_idx < it.q_hi) && (pos >= it.key_lo);
+      // the same for the four warps of a lane group (they hold the same rows)
       const bool warp_valid = decode ? true : __any_sync(0xffffffffu, row_valid);
       const int last_page = (it.L - 1) / PAGE;
       const int tail = it.L % PAGE;
-      float m = -INFINITY, l = 0.0f;  // l: decode, this warp's quarter sum
-      float lq[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // prefill: the row's four quarter sums
+      // the tile of this item whose last page holds slots past the sequence end (-1: none)
+      const int zero_t = tail != 0 ? last_page / PAGES_PER_TILE - it.t0 : -1;
+      const uint32_t zero_off = (uint32_t)(last_page % PAGES_PER_TILE) * BLOCK_BYTES;
+      const size_t widx = ((size_t)(it.r0 + q_idx) * p.Hq + (size_t)(it.g * p.G + hj)) * p.n_split_max + it.s;
+      float m = -INFINITY, l = 0.0f;  // l: this warp's quarter sum l_q
       for (int t = 0; t < it.ntiles; ++t, ++j) {
         const int sb = j % L::NS;
         const int kb0 = (it.t0 + t) * TILE;
         const bool need = row_valid && kb0 <= pos;
         const int nvalid = need ? min(TILE, pos + 1 - kb0) : 0;
+        const int nq = min(32, max(0, nvalid - quarter * 32));
         if (!mbar_wait(&s_full[sb], ((uint32_t)j / L::NS) & 1u, p.status, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        float alpha = 1.0f, m_new = 0.0f;
-        if constexpr (decode) {
-          // ---- decode layout: this warp's quarter of every head row
-          uint32_t S[32], P[16];
-          tmem_ld32(tmem + sb * 128 + lane_off + warp * 32, S);
+        float alpha = 1.0f;
+        // P is packed (two 16-bit values per word) into S[0..15] as S is consumed
+        uint32_t S[32];
+        uint32_t(&P)[16] = *reinterpret_cast<uint32_t(*)[16]>(&S[0]);
+        if (warp_valid) {
+          tmem_ld32(tmem + sb * 128 + lane_off + quarter * 32, S);
           tmem_ld_wait();
-          tc_fence_before();
-          mbar_arrive(&s_free[sb]);
-          const int nq = min(32, max(0, nvalid - warp * 32));
-          const int xm = exchange(quarter_max(S, nq));
-          if (xm < 0) { ok = false; break; }
+        }
+        tc_fence_before();
+        mbar_arrive(&s_free[sb]);
+        if (warp_valid) {
+          float xm[4];
+          if (!exchange(quarter_max(S, nq), xm)) { ok = false; break; }
           float mraw = -INFINITY;
 #pragma unroll
-          for (int w = 0; w < 4; ++w) mraw = fmaxf(mraw, red[xm + w * 8 + (lane & 7)]);
+          for (int q = 0; q < 4; ++q) mraw = fmaxf(mraw, xm[q]);
+          float m_new = 0.0f;
           if (need) {
             m_new = new_reference(m, __fmul_rn(mraw, p.scale_log2), t);
             alpha = ex2_approx(__fsub_rn(m, m_new));
           }
           const float qs = quarter_p<ET>(S, nq, -m_new, p.scale_log2, P);
           if (need) {
-            l = (t == 0) ? qs : __fadd_rn(__fmul_rn(alpha, l), qs);  // this warp's quarter
+            l = (t == 0) ? qs : __fadd_rn(__fmul_rn(alpha, l), qs);
             m = m_new;
           }
-          // P buffer j % NP was last read by the P V of tile j - NP
-          if (j >= L::NP && !pv_done(j - L::NP)) { ok = false; break; }
-          if (lane < p.G) store_p_chunks(smem + OFF_P + (j % L::NP) * L::QP_BYTES, L::HALF, lane, warp, P);
+        }
+        // P buffer j % NP was last read by the P V of tile j - NP
+        if (j >= L::NP && !pv_done(j - L::NP)) { ok = false; break; }
+        if (warp_valid) {
+          if (decode ? lane < p.G : true)
+            store_p_chunks(smem + OFF_P + (j % L::NP) * L::QP_BYTES, L::HALF, r, quarter, P);
+          // rescale this warp's 32 columns of O in tensor memory (not on the
+          // split's first tile, whose P V overwrites O)
           if (t > 0 && __any_sync(0xffffffffu, need && alpha != 1.0f)) {
             // O may be rescaled only once the P V of tile j-1 has landed in it
             if (L::NP > 1 && !pv_done(j - 1)) { ok = false; break; }
             uint32_t o[32];
-            tmem_ld32(tmem + TMEM_O + lane_off + warp * 32, o);
+            tmem_ld32(tmem + TMEM_O + lane_off + quarter * 32, o);
             tmem_ld_wait();
             const float a = need ? alpha : 1.0f;
 #pragma unroll
             for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__fmul_rn(__uint_as_float(o[c]), a));
-            tmem_st32(tmem + TMEM_O + lane_off + warp * 32, o);
+            tmem_st32(tmem + TMEM_O + lane_off + quarter * 32, o);
             tmem_st_wait();
           }
-        } else {
-          // ---- prefill layout: all four quarters of row r
-          uint32_t S[128];
-          if (warp_valid) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              tmem_ld32(tmem + sb * 128 + lane_off + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&S[q * 32]));
-            tmem_ld_wait();
-          }
-          tc_fence_before();
-          mbar_arrive(&s_free[sb]);
-          // P is packed (2 bf16 per word) into S[0..63] as S is consumed
-          uint32_t* P = S;
-          if (warp_valid) {
-            float mraw = -INFINITY;
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              mraw = fmaxf(mraw, quarter_max(*reinterpret_cast<uint32_t(*)[32]>(&S[q * 32]),
-                                             min(32, max(0, nvalid - q * 32))));
-            if (need) {
-              m_new = new_reference(m, __fmul_rn(mraw, p.scale_log2), t);
-              alpha = ex2_approx(__fsub_rn(m, m_new));
-            }
-            float qs[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              qs[q] = quarter_p<ET>(*reinterpret_cast<uint32_t(*)[32]>(&S[q * 32]),
-                                min(32, max(0, nvalid - q * 32)), -m_new, p.scale_log2,
-                                *reinterpret_cast<uint32_t(*)[16]>(&P[q * 16]));
-            if (need) {
-#pragma unroll
-              for (int q = 0; q < 4; ++q) lq[q] = (t == 0) ? qs[q] : __fadd_rn(__fmul_rn(alpha, lq[q]), qs[q]);
-              m = m_new;
-            }
-          }
-          // the P V that last read this P buffer (one buffer: tile j-1) must be
-          // done before P and O are touched
-          if (j >= L::NP && !pv_done(j - L::NP)) { ok = false; break; }
-          static_assert(DECODE || L::NP == 1, "prefill rescales O right after the P buffer wait");
-          if (warp_valid) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              store_p_chunks(smem + OFF_P, L::HALF, r, q, *reinterpret_cast<uint32_t(*)[16]>(&P[q * 16]));
-            // rescale O in tensor memory (not on the split's first tile, whose P V overwrites O)
-            if (t > 0 && __any_sync(0xffffffffu, need && alpha != 1.0f)) {
-              const float a = need ? alpha : 1.0f;
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                uint32_t o[32];
-                tmem_ld32(tmem + TMEM_O + lane_off + q * 32, o);
-                tmem_ld_wait();
-#pragma unroll
-                for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__fmul_rn(__uint_as_float(o[c]), a));
-                tmem_st32(tmem + TMEM_O + lane_off + q * 32, o);
-              }
-              tmem_st_wait();
-            }
-          }
         }
-        // zero V slots at or past the sequence end inside this tile's last page
-        if (tail != 0 && last_page / PAGES_PER_TILE == it.t0 + t) {
+        // zero V slots at or past the sequence end inside this tile's last
+        // page (threads 0..127: value row d = thread)
+        if (threadIdx.x < 128 && t == zero_t) {
           const int vb = j % NV;
           if (!mbar_wait(&v_full[vb], ((uint32_t)j / NV) & 1u, p.status, abort_flag)) { ok = false; break; }
-          uint8_t* vblk = smem + OFF_V + vb * TILE_BYTES + (last_page % PAGES_PER_TILE) * BLOCK_BYTES;
-          const int d = r;  // value row d of the block
+          uint8_t* vblk = smem + OFF_V + vb * TILE_BYTES + zero_off;
+          const int d = threadIdx.x;
           for (int slot = tail; slot < PAGE; ++slot) {
             const uint32_t off = (uint32_t)(d >> 3) * 256u + (uint32_t)(slot >> 3) * 128u +
                                  (uint32_t)(d & 7) * 16u + (uint32_t)(slot & 7) * 2u;
@@ -817,42 +857,17 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!ok) break;
       // end of the split: unnormalised O, m, l of every valid row
       if (!pv_done(j - 1)) { ok = false; break; }
-      const size_t widx = ((size_t)(it.r0 + q_idx) * p.Hq + (size_t)(it.g * p.G + hj)) * p.n_split_max + it.s;
-      if constexpr (decode) {
+      if (warp_valid) {
         // the row's sum: its four quarter sums, in quarter order
-        const int xl = exchange(l);
-        if (xl < 0) { ok = false; break; }
-        const int h8 = lane & 7;
-        const float lrow = __fadd_rn(__fadd_rn(__fadd_rn(red[xl + h8], red[xl + 8 + h8]), red[xl + 16 + h8]),
-                                     red[xl + 24 + h8]);
+        float xl[4];
+        if (!exchange(l, xl)) { ok = false; break; }
+        const float lrow = __fadd_rn(__fadd_rn(__fadd_rn(xl[0], xl[1]), xl[2]), xl[3]);
         uint32_t o[32];
-        tmem_ld32(tmem + TMEM_O + lane_off + warp * 32, o);
+        tmem_ld32(tmem + TMEM_O + lane_off + quarter * 32, o);
         tmem_ld_wait();
         if (row_valid) {
-          float* dst = p.ws_o + widx * HD + warp * 32;
-#pragma unroll
-          for (int c4 = 0; c4 < 8; ++c4)
-            reinterpret_cast<float4*>(dst)[c4] =
-                make_float4(__uint_as_float(o[4 * c4]), __uint_as_float(o[4 * c4 + 1]),
-                            __uint_as_float(o[4 * c4 + 2]), __uint_as_float(o[4 * c4 + 3]));
-          if (warp == 0) *reinterpret_cast<float2*>(p.ws_ml + widx * 2) = make_float2(m, lrow);
-        }
-      } else if (warp_valid) {
-        float* dst = p.ws_o + widx * HD;
-        const float lrow = __fadd_rn(__fadd_rn(__fadd_rn(lq[0], lq[1]), lq[2]), lq[3]);
-        if (row_valid) *reinterpret_cast<float2*>(p.ws_ml + widx * 2) = make_float2(m, lrow);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t o[32];
-          tmem_ld32(tmem + TMEM_O + lane_off + q * 32, o);
-          tmem_ld_wait();
-          if (row_valid) {
-#pragma unroll
-            for (int c4 = 0; c4 < 8; ++c4)
-              reinterpret_cast<float4*>(dst + q * 32)[c4] =
-                  make_float4(__uint_as_float(o[4 * c4]), __uint_as_float(o[4 * c4 + 1]),
-                              __uint_as_float(o[4 * c4 + 2]), __uint_as_float(o[4 * c4 + 3]));
-          }
+          st_global_f32x32(p.ws_o + widx * HD + quarter * 32, o, p.ws_wide != 0);
+          if (quarter == 0) *reinterpret_cast<float2*>(p.ws_ml + widx * 2) = make_float2(m, lrow);
         }
       }
       tc_fence_before();
@@ -862,7 +877,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) {
+  if (warp == L::PRODUCER_WARP + 1) {
     __syncwarp();
     tmem_dealloc(tmem, TMEM_COLS);
   }
@@ -1022,6 +1037,7 @@ static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t ma
   p.work_counter = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + ws_counter_offset(n_tok, Hq, n_split));
   p.scale_log2 = (float)((double)sh->scale * 1.4426950408889634);  // scale * log2(e)
   p.status = status_word();
+  p.ws_wide = (reinterpret_cast<uintptr_t>(p.ws_o) & 31) == 0;
 
   {
     // once per device, under a lock (calls may come from several host threads)
@@ -1046,9 +1062,9 @@ static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t ma
   cudaError_t me = cudaMemsetAsync(p.work_counter, 0, sizeof(int32_t), stream);
   if (me != cudaSuccess) return cuda_fail(me, "attention: work counter reset");
   if (cu_q)
-    attn_split_kernel<false, ET><<<grid, THREADS, Lay<false>::SMEM_BYTES, stream>>>(tmQ, p);
+    attn_split_kernel<false, ET><<<grid, Lay<false>::THREADS, Lay<false>::SMEM_BYTES, stream>>>(tmQ, p);
   else
-    attn_split_kernel<true, ET><<<grid, THREADS, Lay<true>::SMEM_BYTES, stream>>>(tmQ, p);
+    attn_split_kernel<true, ET><<<grid, Lay<true>::THREADS, Lay<true>::SMEM_BYTES, stream>>>(tmQ, p);
   BI_CHECK_LAUNCH("attention split launch");
 
   CombineParams c;

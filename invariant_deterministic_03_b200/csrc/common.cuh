@@ -328,6 +328,19 @@ __device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
                : "memory");
 }
 
+// Arrive on the mbarrier at the same shared-memory offset in both CTAs of
+// the pair (`bar_local`: this CTA's copy) once every pair MMA issued so far by
+// this thread is done: one commit signalling both CTAs (cta mask 0b11). This
+// is the tensor core's completion signal, not a memory load.
+__device__ __forceinline__ void mma_commit_pair_both(uint32_t bar_local) {
+  const uint16_t both = 3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          bar_local),
+      "h"(both)
+      : "memory");
+}
+
 // TMA tiled load into this CTA's shared memory whose completion (bytes) is
 // counted on the mbarrier at shared::cluster address `bar`, which may belong
 // to the other CTA of the pair. No cluster multicast.
@@ -352,6 +365,50 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
+}
+
+// 32 consecutive fp32 values to global memory: four 256-bit stores when
+// `wide` (dst 32-byte aligned: each lane then writes whole 32-byte sectors),
+// else eight 128-bit stores (dst 16-byte aligned).
+__device__ __forceinline__ void st_global_f32x32(float* dst, const uint32_t (&v)[32], bool wide) {
+  if (wide) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + 8 * i), "r"(v[8 * i]),
+                   "r"(v[8 * i + 1]), "r"(v[8 * i + 2]), "r"(v[8 * i + 3]), "r"(v[8 * i + 4]), "r"(v[8 * i + 5]),
+                   "r"(v[8 * i + 6]), "r"(v[8 * i + 7])
+                   : "memory");
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 4 * i), "r"(v[4 * i]), "r"(v[4 * i + 1]),
+                   "r"(v[4 * i + 2]), "r"(v[4 * i + 3])
+                   : "memory");
+  }
+}
+
+// 4-byte asynchronous copy global -> shared (cp.async; completion tracked
+// per thread in commit groups).
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Waits until at most N of this thread's most recent commit groups are pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Store one 32-bit column of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
+}
+
+// Load 4 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t (&r)[4]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
 }
 
 // Store 32 consecutive fp32 columns of this thread's TMEM lane.

@@ -32,7 +32,11 @@
 //               rows past M, never stored, read whatever the stage held; no
 //               row of the product depends on another row).
 //   warp 1      allocates 2 x BN tensor-memory columns (two accumulators) for
-//               the pair; on rank 0 lane 0 issues the MMAs and commits
+//               the pair; on rank 0 lane 0 issues the MMAs and commits, each
+//               commit one tcgen05.commit multicast to the same barrier in
+//               both CTAs (stage free, accumulator full), which each CTA
+//               waits on at CTA scope (one commit to both measured ~5 %
+//               faster than a commit per CTA with cluster-scope waits)
 //   warps 2..5  epilogue of this CTA's 128 rows: tcgen05.ld the accumulator
 //               row by row (thread = row), round to bf16 (RNE) or keep fp32,
 //               store to global, or run one of the fused epilogues (EPI_ADD,
@@ -380,7 +384,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int w_row = EPI == EPI_SWIGLU ? (int)rank * p.N + nb * (BN / 2) : nb * BN + (int)rank * (BN / 2);
         for (int kb = 0; kb < pf && kb < p.k_blocks; ++kb) tma_prefetch_2d(&tmB, kb * BK, w_row);
         for (int kb = 0; kb < p.k_blocks; ++kb) {
-          if (!mbar_wait_cluster(&empty[stage], phase ^ 1, p.status, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&empty[stage], phase ^ 1, p.status, abort_flag)) { ok = false; break; }
           if (pf && kb + pf < p.k_blocks) tma_prefetch_2d(&tmB, (kb + pf) * BK, w_row);
           uint8_t* sa = tiles + stage * STAGE_BYTES;
           const uint32_t fb = cluster_addr(&full[stage], 0);
@@ -446,14 +450,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           issued = true;
           // frees the stage in both CTAs once these MMAs retire
-          mma_commit_pair(cluster_addr(&empty[stage], 0));
-          mma_commit_pair(cluster_addr(&empty[stage], 1));
+          mma_commit_pair_both(smem_u32(&empty[stage]));
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
         // accumulator complete, in both CTAs' tensor memory
-        mma_commit_pair(cluster_addr(&acc_full[acc], 0));
-        mma_commit_pair(cluster_addr(&acc_full[acc], 1));
+        mma_commit_pair_both(smem_u32(&acc_full[acc]));
         if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       }
       if (!ok && issued) {
@@ -474,7 +476,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint32_t acc_phase = 0;
     for (int tile = tile0; tile < num_tiles; tile += tile_step) {
       const int mb = tile % p.m_blocks, nb = tile / p.m_blocks;
-      if (!mbar_wait_cluster(&acc_full[acc], acc_phase, p.status, abort_flag)) break;
+      if (!mbar_wait(&acc_full[acc], acc_phase, p.status, abort_flag)) break;
       tc_fence_after();
       const int row = mb * BM + (int)rank * BM_CTA + trow;
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;

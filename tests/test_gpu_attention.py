@@ -117,6 +117,33 @@ def test_decode_equals_chunked_prefill(bi, Hq, Hkv):
             assert same_bits(out, dec[s0:e0]), f"chunk {chunk} at {s0}"
 
 
+def test_workspace_alignment_does_not_change_bits(bi):
+    """The split kernel writes its partial rows with 256-bit stores when the
+    workspace is 32-byte aligned and 128-bit stores when it is only 16-byte
+    aligned; both give the same bits, for decode and prefill."""
+    lens = [5, 600, 1300]
+    S = Seqs(bi, lens, 32, 8, seed=11)
+    shape = S.shape(bi)
+    q_rows = dev(torch.stack([S.q[b][L - 1].reshape(-1) for b, L in enumerate(lens)]))
+    sl = dev(torch.tensor(lens, dtype=torch.int32))
+    n = bi.bi_attn_workspace_size(shape, 1300)
+    big = torch.empty(n + 64, dtype=torch.uint8, device="cuda:0")
+    assert big.data_ptr() % 32 == 0
+    outs = []
+    for off in (0, 16):
+        ws = big[off:off + n]
+        dec = torch.empty(len(lens), q_rows.shape[1], dtype=torch.bfloat16, device="cuda:0")
+        bi.bi_attn_decode(q_rows, S.kc, S.vc, S.bt, sl, shape, dec, ws)
+        q = dev(S.q[2].reshape(1300, -1))
+        pre = torch.empty_like(q)
+        bi.bi_attn_prefill(q, dev(torch.tensor([0, 1300], dtype=torch.int32)), 1300, S.kc, S.vc,
+                           S.bt[2:3].contiguous(), sl[2:3].contiguous(), shape, pre, ws)
+        outs.append((dec, pre))
+    assert same_bits(outs[0][0], outs[1][0])
+    assert same_bits(outs[0][1], outs[1][1])
+    assert same_bits(outs[0][1][-1], outs[0][0][2])     # the last prompt row is the decode row
+
+
 def test_batch_composition(bi):
     """A sequence's rows are the same bits alone, co-batched with others of
     mixed lengths and chunk sizes, and at a different batch position."""
