@@ -73,7 +73,8 @@ typedef enum { BI_BF16 = 0, BI_F32 = 1, BI_F32_ADD = 2 } bi_dtype;
 #define BI_DEV_WAIT_TIMEOUT 0x1 /* a bounded mbarrier wait ran out */
 #define BI_DEV_BAD_SLOT 0x2     /* slot_mapping entry outside the cache */
 #define BI_DEV_BAD_PAGE 0x4     /* block_table entry outside the cache */
-#define BI_DEV_BAD_SEQLEN 0x8   /* seq_lens entry outside [n_query, max_kv_len] */
+#define BI_DEV_BAD_SEQLEN 0x8   /* seq_lens entry outside [n_query, max_kv_len], or a prefill
+                                   chunk with more than max_q_len rows */
 #define BI_DEV_BAD_TOKEN 0x10   /* token id outside the vocabulary */
 
 /* Thread-local description of the last failure on this host thread. */
@@ -231,7 +232,9 @@ bi_status bi_kv_append(const void* k_new, const void* v_new, int64_t ld_new,
  * q rows: token t, head h at q + t*ldq + h*128 (bf16). out likewise with ldo.
  * block_table [B, max_pages_per_seq] int32 (page ids, in key order),
  * seq_lens [B] int32 = number of keys in the cache for sequence b, INCLUDING
- * the tokens queried in this call (they were appended first). */
+ * the tokens queried in this call (they were appended first). A seq_lens
+ * entry outside [queried tokens, max_kv_len] sets BI_DEV_BAD_SEQLEN and the
+ * sequence's rows are written as zeros. */
 typedef struct {
   int32_t num_q_heads;       /* Hq */
   int32_t num_kv_heads;      /* Hkv; Hq / Hkv must be 1, 2, 4 or 8 */
@@ -293,7 +296,9 @@ bi_status bi_attn_decode_noalloc(const void* q, int64_t ldq, const void* k_cache
  * (cu_q [B+1] int32 on the device, increasing, 0 <= cu_q[0], cu_q[B] <=
  * n_tok); they are its LAST n_b = cu_q[b+1]-cu_q[b] tokens, so row cu_q[b]+i
  * sits at position seq_lens[b] - n_b + i. max_q_len bounds n_b (host-side
- * grid size). q and out span all n_tok rows; rows outside cu_q[0] ..
+ * grid size; a longer chunk sets BI_DEV_BAD_SEQLEN and its rows past the
+ * covered ones are written as zeros). q and out span all n_tok rows; rows
+ * outside cu_q[0] ..
  * cu_q[B]-1 are not read or written (so a call can cover a subset of a
  * batch, e.g. the multi-token chunks after the batch's one-token ones). */
 bi_status bi_attn_prefill(const void* q, int64_t ldq, const int32_t* cu_q,

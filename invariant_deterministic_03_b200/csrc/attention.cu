@@ -54,7 +54,6 @@ constexpr int PAGE = BI_PAGE_SIZE;     // 16 keys
 constexpr int PAGES_PER_TILE = TILE / PAGE;
 constexpr uint32_t TILE_BYTES = 128 * 128 * 2;  // 32 KB: one K or V tile (128 keys x 128 d)
 constexpr int ITEM_RING = 16;                   // claimed work items in flight inside a CTA
-constexpr int MAX_KV_BUF = 3;
 
 // Shared-memory layout. Prefill: Q and P are full 128-row tiles, one buffer
 // each (Q is released after an item's last Q K^T, so the next item's Q loads
@@ -91,7 +90,7 @@ struct Lay {
   static constexpr uint32_t OFF_RED = OFF_RING + 512;   // decode quarter exchange [2 slots][4 warps][8 heads] fp32
   static constexpr uint32_t OFF_ITEMS = OFF_RED + (DECODE ? 256 : 0);  // item ring [16] x 48 B, then one mbarrier per slot
   static constexpr size_t SMEM_BYTES = 1024 + OFF_ITEMS + ITEM_RING * 48 + ITEM_RING * 8;
-  static_assert(NK <= MAX_KV_BUF && NV <= MAX_KV_BUF, "barrier arrays hold 3 K and 3 V buffers");
+  static_assert(NK + NV <= 6, "barrier area holds six K / V buffers");
   static_assert(OFF_Q % 1024 == 0 && OFF_P % 1024 == 0, "swizzled Q / P tiles need 1 KB alignment");
   static_assert(SMEM_BYTES <= 232448, "attention: shared memory above the 227 KB per-CTA limit");
 };
@@ -153,6 +152,9 @@ __device__ __forceinline__ bool item_at(const Params& p, int idx, Item& it, bool
     it.r0 = it.b;
     it.nb = 1;
   }
+  // a chunk with more rows than max_q_len (the grid covers max_q_len rows)
+  if (report && jb == 0 && it.s == 0 && it.g == 0 && it.nb > p.qblocks * p.QR)
+    set_status(p.status, BI_DEV_BAD_SEQLEN);
   if (it.nb <= 0 || jb * p.QR >= it.nb) return false;
   if (it.L < it.nb || it.L > p.max_kv_len || it.r0 < 0 || it.r0 + it.nb > p.n_tok) {
     if (report && it.s == 0 && jb == 0 && it.g == 0) set_status(p.status, BI_DEV_BAD_SEQLEN);
@@ -422,17 +424,18 @@ __global__ void __launch_bounds__(Lay<DECODE>::THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
-  uint64_t* q_full = bars + 0;     // [2]
-  uint64_t* q_empty = bars + 2;    // [2]
-  uint64_t* k_full = bars + 4;     // [NK]
-  uint64_t* k_empty = bars + 7;    // [NK]
-  uint64_t* v_full = bars + 10;    // [NV]
-  uint64_t* v_empty = bars + 13;   // [NV]
-  uint64_t* s_full = bars + 16;    // [NS]
-  uint64_t* s_free = bars + 19;    // [NS]
-  uint64_t* p_ready = bars + 22;   // [NP]
-  uint64_t* o_ready = bars + 24;   // [NP]: P V of the tile that read P buffer i is done
-  uint64_t* x_bar = bars + 26;     // quarter exchange: decode [1], prefill [4] (one per lane group)
+  uint64_t* q_full = bars + 0;                // [2]
+  uint64_t* q_empty = bars + 2;               // [2]
+  uint64_t* k_full = bars + 4;                // [NK]
+  uint64_t* k_empty = k_full + NK;            // [NK]
+  uint64_t* v_full = k_empty + NK;            // [NV]
+  uint64_t* v_empty = v_full + NV;            // [NV]
+  uint64_t* s_full = bars + 16;               // [NS]
+  uint64_t* s_free = bars + 19;               // [NS]
+  uint64_t* p_ready = bars + 22;              // [NP]
+  uint64_t* o_ready = bars + 24;              // [NP]: P V of the tile that read P buffer i is done
+  uint64_t* x_bar = bars + 26;                // quarter exchange: decode [1], prefill [4] (one per lane group)
+  static_assert(4 + 2 * (NK + NV) <= 16, "K / V barriers overlap the S barriers");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 30);
   // ring entry (item) the producer's page look-ahead is on; the scheduler stays
   // at most SCHED_AHEAD entries in front of it
@@ -893,6 +896,7 @@ struct CombineParams {
   void* out;  // 16-bit rows (the element type of the kernel)
   int64_t ldo;
   int32_t n_tok, B, Hq, n_split_max, max_kv_len;
+  int32_t max_rows;  // rows per sequence the split kernel covers (qblocks x rows per block)
 };
 
 template <typename ET>
@@ -921,7 +925,7 @@ __global__ void attn_combine_kernel(const CombineParams p) {
   }
   const int L = p.seq_lens[b];
   uint16_t* dst = static_cast<uint16_t*>(p.out) + (size_t)tok * p.ldo + (size_t)h * HD + lane * 4;
-  if (L < nb || L > p.max_kv_len || nb <= 0) {  // flagged by the split kernel; write zeros
+  if (L < nb || L > p.max_kv_len || nb <= 0 || qidx >= p.max_rows) {  // flagged by the split kernel; zeros
     *reinterpret_cast<uint2*>(dst) = make_uint2(0u, 0u);
     return;
   }
@@ -1079,6 +1083,7 @@ static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t ma
   c.Hq = Hq;
   c.n_split_max = n_split;
   c.max_kv_len = sh->max_kv_len;
+  c.max_rows = qblocks * QR;
   const int64_t warps = n_tok * Hq;
   const int blocks = (int)((warps + 7) / 8);
   attn_combine_kernel<ET><<<blocks, 256, 0, stream>>>(c);

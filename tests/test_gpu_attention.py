@@ -262,7 +262,27 @@ def test_mixed_batch_decode_then_prefill_subsets(bi):
     nd = 2
     bi.bi_attn_decode(dev(q), S.kc, S.vc, bt, sl[:nd], shape, out[:nd], ws)
     marker = out[:nd].clone()
-    bi.bi_attn_prefill(dev(q), dev(cu[nd:]), 512, S.kc, S.vc, bt[nd:].contiguous(), sl[nd:].contiguous(),
+    max_q = max(e - s for _, s, e in chunks[nd:])   # 513: bounds every chunk's rows
+    bi.bi_attn_prefill(dev(q), dev(cu[nd:]), max_q, S.kc, S.vc, bt[nd:].contiguous(), sl[nd:].contiguous(),
                        shape, out, ws)
     assert same_bits(out[:nd], marker)               # the subset call left the decode rows alone
     assert same_bits(out, whole)
+    assert bi.bi_device_status(clear=True) == 0
+
+
+def test_chunk_longer_than_max_q_len_is_reported(bi):
+    """max_q_len sizes the grid on the host; a chunk with more rows than it
+    (only visible on the device) sets BI_DEV_BAD_SEQLEN instead of passing
+    silently."""
+    lens = [513]
+    S = Seqs(bi, lens, 32, 8, seed=43)
+    shape = S.shape(bi)
+    q = dev(S.q[0].reshape(513, -1))
+    ws = torch.empty(bi.bi_attn_workspace_size(shape, 513), dtype=torch.uint8, device="cuda:0")
+    out = torch.empty_like(q)
+    bi.bi_device_status(clear=True)
+    bi.bi_attn_prefill(q, dev(torch.tensor([0, 513], dtype=torch.int32)), 512, S.kc, S.vc, S.bt,
+                       dev(torch.tensor([513], dtype=torch.int32)), shape, out, ws)
+    torch.cuda.synchronize()
+    assert bi.bi_device_status(clear=True) & 0x8      # BI_DEV_BAD_SEQLEN
+    assert not out[512:].float().abs().any()          # the row past max_q_len rows: zeros
