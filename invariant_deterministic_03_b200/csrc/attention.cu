@@ -899,13 +899,9 @@ struct CombineParams {
   int32_t max_rows;  // rows per sequence the split kernel covers (qblocks x rows per block)
 };
 
+// One (token, head) row, by one warp.
 template <typename ET>
-__global__ void attn_combine_kernel(const CombineParams p) {
-  const int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (wid >= (int64_t)p.n_tok * p.Hq) return;
-  const int tok = (int)(wid / p.Hq);
-  const int h = (int)(wid % p.Hq);
+__device__ __forceinline__ void combine_row(const CombineParams& p, int tok, int h, int lane) {
   int b, nb, qidx;
   if (p.cu_q) {
     if (tok < p.cu_q[0] || tok >= p.cu_q[p.B]) return;  // a row this call does not cover
@@ -932,24 +928,62 @@ __global__ void attn_combine_kernel(const CombineParams p) {
   const int pos = L - nb + qidx;
   const int n = pos / SPLIT + 1;
   const size_t base = ((size_t)tok * p.Hq + h) * p.n_split_max;
-  float M = -INFINITY;
-  for (int s = 0; s < n; ++s) M = fmaxf(M, p.ws_ml[(base + s) * 2]);
+  // Lane s holds split s's (m, l) (splits 32 at a time); M is their maximum
+  // (exact in any order), taken across the warp by shuffles.
+  float2 ml0 = make_float2(-INFINITY, 0.0f);  // splits 0 .. 31, kept for the sums
+  if (lane < n) ml0 = *reinterpret_cast<const float2*>(p.ws_ml + (base + lane) * 2);
+  float M = ml0.x;
+  for (int c = 32; c < n; c += 32)
+    if (c + lane < n) M = fmaxf(M, p.ws_ml[(base + c + lane) * 2]);
+#pragma unroll
+  for (int d = 16; d; d >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, d));
+  // The sums in split order s = 0 .. n-1; the O rows of four splits are
+  // loaded before their four fused multiply-adds, so the loads overlap.
   float Lsum = 0.0f;
   float o0 = 0.0f, o1 = 0.0f, o2 = 0.0f, o3 = 0.0f;
-  for (int s = 0; s < n; ++s) {
-    const float2 ml = *reinterpret_cast<const float2*>(p.ws_ml + (base + s) * 2);
-    const float w = exp2f(__fsub_rn(ml.x, M));
-    Lsum = __fmaf_rn(w, ml.y, Lsum);
-    const float4 o = *reinterpret_cast<const float4*>(p.ws_o + (base + s) * HD + lane * 4);
-    o0 = __fmaf_rn(w, o.x, o0);
-    o1 = __fmaf_rn(w, o.y, o1);
-    o2 = __fmaf_rn(w, o.z, o2);
-    o3 = __fmaf_rn(w, o.w, o3);
+  for (int c = 0; c < n; c += 32) {
+    float2 ml = ml0;
+    if (c > 0) ml = c + lane < n ? *reinterpret_cast<const float2*>(p.ws_ml + (base + c + lane) * 2)
+                                 : make_float2(-INFINITY, 0.0f);
+    const float w_lane = c + lane < n ? exp2f(__fsub_rn(ml.x, M)) : 0.0f;  // split c + lane's weight
+    const int cn = min(32, n - c);
+    for (int k0 = 0; k0 < cn; k0 += 4) {
+      float4 ov[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (k0 + k < cn) ov[k] = *reinterpret_cast<const float4*>(p.ws_o + (base + c + k0 + k) * HD + lane * 4);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (k0 + k < cn) {  // the same for the whole warp
+          const float w = __shfl_sync(0xffffffffu, w_lane, k0 + k);
+          const float l = __shfl_sync(0xffffffffu, ml.y, k0 + k);
+          Lsum = __fmaf_rn(w, l, Lsum);
+          o0 = __fmaf_rn(w, ov[k].x, o0);
+          o1 = __fmaf_rn(w, ov[k].y, o1);
+          o2 = __fmaf_rn(w, ov[k].z, o2);
+          o3 = __fmaf_rn(w, ov[k].w, o3);
+        }
+      }
+    }
   }
   // + 0.0f turns a -0 into +0, so a zero's sign cannot depend on the split path
   const float y0 = __fadd_rn(__fdiv_rn(o0, Lsum), 0.0f), y1 = __fadd_rn(__fdiv_rn(o1, Lsum), 0.0f);
   const float y2 = __fadd_rn(__fdiv_rn(o2, Lsum), 0.0f), y3 = __fadd_rn(__fdiv_rn(o3, Lsum), 0.0f);
   *reinterpret_cast<uint2*>(dst) = make_uint2(E16<ET>::pack2(y0, y1), E16<ET>::pack2(y2, y3));
+}
+
+// A grid of a few CTAs per SM whose warps stride over the (token, head) rows
+// (tens of thousands of one-row CTAs cost more in scheduling than the rows).
+template <typename ET>
+__global__ void __launch_bounds__(256, 4) attn_combine_kernel(const CombineParams p) {
+  // launched as a programmatic dependent of the split kernel: wait until that
+  // grid has completed and its writes are visible
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = (int64_t)p.n_tok * p.Hq;
+  const int64_t step = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); wid < rows; wid += step)
+    combine_row<ET>(p, (int)(wid / p.Hq), (int)(wid % p.Hq), lane);
 }
 
 // partial O [n_tok][Hq][n_split][128] fp32, then (m, l) pairs, then (256-byte
@@ -1085,8 +1119,23 @@ static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t ma
   c.max_kv_len = sh->max_kv_len;
   c.max_rows = qblocks * QR;
   const int64_t warps = n_tok * Hq;
-  const int blocks = (int)((warps + 7) / 8);
-  attn_combine_kernel<ET><<<blocks, 256, 0, stream>>>(c);
+  const int64_t want = (warps + 7) / 8;
+  const int blocks = (int)(want < (int64_t)num_sms() * 4 ? want : (int64_t)num_sms() * 4);
+  // programmatic dependent launch: the combine is launched as the split
+  // kernel's CTAs exit (no explicit trigger: an early one measured slower for
+  // prefill) and starts its work only once the split grid is done
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t ce = cudaLaunchKernelEx(&cfg, attn_combine_kernel<ET>, c);
+  if (ce != cudaSuccess) return cuda_fail(ce, "attention combine launch");
   BI_CHECK_LAUNCH("attention combine launch");
   return BI_OK;
 }
