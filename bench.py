@@ -41,7 +41,7 @@ COPIES = 3
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # dram__bytes_read.sum + dram__bytes_write.sum of one gemm_tcgen05_kernel<1, 0, bf16>
 # launch at M=4096 K=4096 N=14336 (profiles/gemm_tcgen05_m4096_k4096_n14336.md)
-GEMM_TRAFFIC_BYTES = 171.912960e6 + 100.647936e6
+GEMM_TRAFFIC_BYTES = 172.939008e6 + 98.600704e6
 RMS_MS = [1 << i for i in range(13)] + [16384, 65536]   # RMSNorm bandwidth sweep, D = 4096
 
 
