@@ -868,9 +868,56 @@ __global__ void __launch_bounds__(Lay<DECODE>::THREADS, 1)
         uint32_t o[32];
         tmem_ld32(tmem + TMEM_O + lane_off + quarter * 32, o);
         tmem_ld_wait();
-        if (row_valid) {
-          st_global_f32x32(p.ws_o + widx * HD + quarter * 32, o, p.ws_wide != 0);
-          if (quarter == 0) *reinterpret_cast<float2*>(p.ws_ml + widx * 2) = make_float2(m, lrow);
+        if (row_valid && quarter == 0) *reinterpret_cast<float2*>(p.ws_ml + widx * 2) = make_float2(m, lrow);
+        if constexpr (decode) {
+          if (row_valid) st_global_f32x32(p.ws_o + widx * HD + quarter * 32, o, p.ws_wide != 0);
+        } else {
+          // The warp's 32 rows go out as 128-byte row pieces, four lanes per
+          // row: within each group of four lanes the 8-column chunks are
+          // transposed (two exchange stages, lanes i ^ 2 then i ^ 1), after
+          // which lane 4a + c holds chunk c of rows 4a .. 4a + 3 in its slots
+          // 0 .. 3 (o[8k .. 8k + 7] = row 4a + k). Store k then writes row
+          // 4a + k whole from its four lanes (same bytes as one row per lane,
+          // a quarter of the memory requests).
+          const int i4 = lane & 3;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {  // lanes i, i ^ 2 swap chunks {2, 3} / {0, 1}
+            const bool hi = (i4 & 2) != 0;
+            const uint32_t recv = __shfl_xor_sync(0xffffffffu, hi ? o[e] : o[16 + e], 2);
+            if (hi) o[e] = recv; else o[16 + e] = recv;
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {  // lanes i, i ^ 1 swap slots {1, 3} / {0, 2}
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const bool odd = (i4 & 1) != 0;
+              const int even_slot = h * 16 + e, odd_slot = h * 16 + 8 + e;
+              const uint32_t recv = __shfl_xor_sync(0xffffffffu, odd ? o[even_slot] : o[odd_slot], 1);
+              if (odd) o[even_slot] = recv; else o[odd_slot] = recv;
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int rk = rg * 32 + (lane & ~3) + k;  // the row this store writes
+            const int qk = it.q_lo + rk / p.G, hk = rk % p.G;
+            if (qk < it.q_hi && it.L - it.nb + qk >= it.key_lo) {
+              const size_t wk = ((size_t)(it.r0 + qk) * p.Hq + (size_t)(it.g * p.G + hk)) * p.n_split_max + it.s;
+              float* dst = p.ws_o + wk * HD + quarter * 32 + i4 * 8;
+              if (p.ws_wide) {
+                asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst),
+                             "r"(o[8 * k]), "r"(o[8 * k + 1]), "r"(o[8 * k + 2]), "r"(o[8 * k + 3]),
+                             "r"(o[8 * k + 4]), "r"(o[8 * k + 5]), "r"(o[8 * k + 6]), "r"(o[8 * k + 7])
+                             : "memory");
+              } else {
+                asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "r"(o[8 * k]),
+                             "r"(o[8 * k + 1]), "r"(o[8 * k + 2]), "r"(o[8 * k + 3])
+                             : "memory");
+                asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 4), "r"(o[8 * k + 4]),
+                             "r"(o[8 * k + 5]), "r"(o[8 * k + 6]), "r"(o[8 * k + 7])
+                             : "memory");
+              }
+            }
+          }
         }
       }
       tc_fence_before();
