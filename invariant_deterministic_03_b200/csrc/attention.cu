@@ -357,18 +357,27 @@ __device__ __forceinline__ float new_reference(float m, float tile_max, int t) {
   return (t > 0 && __fsub_rn(mc, m) <= RESCALE_LOG2) ? m : mc;
 }
 
-// The maximum of a quarter's first nvalid scores (-inf when none), by a
-// pairwise tree (depth 5 instead of a 32-long chain): max is exact, so any
-// order gives the same value for non-NaN scores; masked keys enter as -inf.
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// The maximum of a quarter's first nvalid scores (-inf when none), by a tree
+// of three-input maxima (17 operations, depth 4, instead of a 32-long chain):
+// max is exact, so any order gives the same value for non-NaN scores; masked
+// keys enter as -inf. With nvalid = 32 (a constant) no select is left.
 __device__ __forceinline__ float quarter_max(const uint32_t (&S)[32], int nvalid) {
   float v[32];
 #pragma unroll
   for (int c = 0; c < 32; ++c) v[c] = c < nvalid ? __uint_as_float(S[c]) : -INFINITY;
+  float a[11];
 #pragma unroll
-  for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-    for (int c = 0; c < w; ++c) v[c] = fmaxf(v[c], v[c + w]);
-  return v[0];
+  for (int k = 0; k < 10; ++k) a[k] = max3(v[3 * k], v[3 * k + 1], v[3 * k + 2]);
+  a[10] = fmaxf(v[30], v[31]);
+  const float b0 = max3(a[0], a[1], a[2]), b1 = max3(a[3], a[4], a[5]), b2 = max3(a[6], a[7], a[8]);
+  const float b3 = fmaxf(a[9], a[10]);
+  return fmaxf(max3(b0, b1, b2), b3);
 }
 
 // P row `row`, keys 32*quarter .. +31, into the 128-byte-swizzled P tile whose
@@ -805,7 +814,10 @@ __global__ void __launch_bounds__(Lay<DECODE>::THREADS, 1)
         mbar_arrive(&s_free[sb]);
         if (warp_valid) {
           float xm[4];
-          if (!exchange(quarter_max(S, nq), xm)) { ok = false; break; }
+          // prefill: a warp whose rows all see this whole quarter skips the
+          // masking selects (the same operations on the same values)
+          const bool full_q = !decode && __all_sync(0xffffffffu, nq >= 32);
+          if (!exchange(full_q ? quarter_max(S, 32) : quarter_max(S, nq), xm)) { ok = false; break; }
           float mraw = -INFINITY;
 #pragma unroll
           for (int q = 0; q < 4; ++q) mraw = fmaxf(mraw, xm[q]);
@@ -814,7 +826,8 @@ __global__ void __launch_bounds__(Lay<DECODE>::THREADS, 1)
             m_new = new_reference(m, __fmul_rn(mraw, p.scale_log2), t);
             alpha = ex2_approx(__fsub_rn(m, m_new));
           }
-          const float qs = quarter_p<ET>(S, nq, -m_new, p.scale_log2, P);
+          const float qs = full_q ? quarter_p<ET>(S, 32, -m_new, p.scale_log2, P)
+                                  : quarter_p<ET>(S, nq, -m_new, p.scale_log2, P);
           if (need) {
             l = (t == 0) ? qs : __fadd_rn(__fmul_rn(alpha, l), qs);
             m = m_new;
