@@ -144,6 +144,30 @@ def test_workspace_alignment_does_not_change_bits(bi):
     assert same_bits(outs[0][1][-1], outs[0][0][2])     # the last prompt row is the decode row
 
 
+def test_prefill_bench_workload_sampled(bi):
+    """The prefill workload the benchmark times, in the same launch: four
+    fresh 2048-token prompts, causal, GQA 32/8, one bi_attn_prefill call.
+    Sampled rows (split and tile boundaries, the diagonal, the last row)
+    match the fp64 oracle, and each equals, bit for bit, a decode of the same
+    position over the same cache."""
+    L, B = 2048, 4
+    S = Seqs(bi, [L] * B, 32, 8, seed=61)
+    shape = S.shape(bi)
+    out = _prefill(bi, S, [(b, 0, L) for b in range(B)], shape)
+    positions = [0, 127, 128, 511, 512, 1000, 1535, 2047]
+    for b in range(B):
+        o64, R = S.oracle(b, positions)
+        rows = out[b * L + torch.tensor(positions)]
+        check(f64(rows).reshape(len(positions), 32, D), o64, R, kappa=1.0, what=f"prefill b={b}")
+    # decode of the same positions: one query each, keys up to and including it
+    qd = torch.stack([S.q[b][p_].reshape(-1) for b in range(B) for p_ in positions])
+    bt = S.bt.repeat_interleave(len(positions), dim=0)
+    lens = [p_ + 1 for _ in range(B) for p_ in positions]
+    dec = _decode(bi, S, dev(qd), lens, bt, shape)
+    idx = torch.tensor([b * L + p_ for b in range(B) for p_ in positions])
+    assert same_bits(dec, out[idx])
+
+
 def test_batch_composition(bi):
     """A sequence's rows are the same bits alone, co-batched with others of
     mixed lengths and chunk sizes, and at a different batch position."""
