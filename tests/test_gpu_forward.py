@@ -135,10 +135,10 @@ def test_invariance_chunking_and_cobatching(bi):
         step += 1
     for p, row in got:
         assert same_bits(row, per_tok[p]), f"position {p}"
-    # a step of 999 tokens has 8 x 24 >= 148 QKV output tiles, so its QKV
-    # projection, RoPE and cache write run as one fused launch (the steps
-    # above, all under 148 tiles, run them as three launches); the keys it
-    # caches are then read by a decode step
+    # a step of 999 tokens has ceil(999 / 256) x 24 = 96 QKV pair tiles, at
+    # least one per two SMs, so its QKV projection, RoPE and cache write run
+    # as one fused launch (steps of up to 768 tokens, 72 pair tiles, run them
+    # as three launches); the keys it caches are then read by a decode step
     e4, _ = _engine(cfg, w, seed=8)
     other = synth.randint(700, 0, cfg["vocab"] - 1, seed=30).tolist()
     tok4 = lambda s: toks if s == 0 else other   # noqa: E731

@@ -69,7 +69,10 @@ def _case(bi, table, M, K, Hq, Hkv, seed, slots=None, positions=None, num_pages=
     return st1, st2, qkv1, kc1
 
 
+# (768, 4096, 32, 8) and (769, 4096, 32, 8): the 7B width on both sides of
+# the forward's switch from three launches to the fused one (72 / 96 pair tiles)
 @pytest.mark.parametrize("M,K,Hq,Hkv", [(1, 4096, 32, 8), (7, 4096, 32, 8), (130, 4096, 32, 8),
+                                        (768, 4096, 32, 8), (769, 4096, 32, 8),
                                         (5, 72, 4, 2), (64, 200, 3, 1), (33, 520, 5, 3),
                                         (17, 8200, 4, 2), (200, 136, 6, 2), (300, 264, 4, 1)])
 def test_fused_equals_three_steps(bi, table, M, K, Hq, Hkv):
