@@ -92,7 +92,7 @@ def test_decode_parity(bi, Hq, Hkv):
         check(f64(out[b]).reshape(1, Hq, D), o64, R, kappa=1.0, what=f"decode b={b} L={L}")
 
 
-@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (8, 8)])
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (8, 8), (16, 8), (64, 8)])
 def test_decode_equals_chunked_prefill(bi, Hq, Hkv):
     """Every token of a 1100-token sequence: decode (one token, its keys
     cached) == prefill in chunks of 1, 64 and 512 == whole prefill, bitwise;
