@@ -1032,18 +1032,139 @@ __device__ __forceinline__ void combine_row(const CombineParams& p, int tok, int
   *reinterpret_cast<uint2*>(dst) = make_uint2(E16<ET>::pack2(y0, y1), E16<ET>::pack2(y2, y3));
 }
 
+// A row's place in the finishing pass: 0 not covered by this call, 1 zeros
+// (flagged by the split kernel), 2 n <= 4 splits, 3 more.
+struct CombRow {
+  int kind, n, tok, h;
+  size_t base;
+  uint16_t* dst;
+};
+
+__device__ __forceinline__ CombRow comb_setup(const CombineParams& p, int64_t wid, int lane) {
+  CombRow r;
+  r.tok = (int)(wid / p.Hq);
+  r.h = (int)(wid % p.Hq);
+  r.kind = 0;
+  r.n = 0;
+  r.base = 0;
+  r.dst = nullptr;
+  int b, nb, qidx;
+  if (p.cu_q) {
+    if (r.tok < p.cu_q[0] || r.tok >= p.cu_q[p.B]) return r;  // a row this call does not cover
+    int lo = 0, hi = p.B;  // find b with cu_q[b] <= tok < cu_q[b+1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (p.cu_q[mid] <= r.tok) lo = mid; else hi = mid;
+    }
+    b = lo;
+    nb = p.cu_q[b + 1] - p.cu_q[b];
+    qidx = r.tok - p.cu_q[b];
+    if (p.cu_q[b] < 0 || p.cu_q[b + 1] > p.n_tok) nb = 0;  // malformed cu_q: zeros
+  } else {
+    b = r.tok;
+    nb = 1;
+    qidx = 0;
+  }
+  const int L = p.seq_lens[b];
+  r.dst = static_cast<uint16_t*>(p.out) + (size_t)r.tok * p.ldo + (size_t)r.h * HD + lane * 4;
+  if (L < nb || L > p.max_kv_len || nb <= 0 || qidx >= p.max_rows) {
+    r.kind = 1;
+    return r;
+  }
+  r.n = (L - nb + qidx) / SPLIT + 1;
+  r.base = ((size_t)r.tok * p.Hq + r.h) * p.n_split_max;
+  r.kind = r.n <= 4 ? 2 : 3;
+  return r;
+}
+
+// A short row's loads, issued asynchronously (cp.async) into this lane's own
+// shared-memory slots: its 16 bytes of each split's O row, and (lane s < n)
+// split s's (m, l). One commit group per row.
+__device__ __forceinline__ void comb_issue(const CombineParams& p, const CombRow& r, int lane, float4* so,
+                                           float2* sml) {
+  if (r.kind == 2) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (k < r.n)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(smem_u32(so + k * 32 + lane)),
+                     "l"(p.ws_o + (r.base + k) * HD + lane * 4)
+                     : "memory");
+    if (lane < r.n)
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(sml + lane)),
+                   "l"(p.ws_ml + (r.base + lane) * 2)
+                   : "memory");
+  }
+  cp_async_commit();
+}
+
+// The merge of a short row from the lane's own slots: the same operations as
+// combine_row (M over the splits' m by shuffles, weights 2^(m_s - M), sums in
+// split order, y = o / L + 0).
+template <typename ET>
+__device__ __forceinline__ void comb_short(const CombRow& r, int lane, const float4* so, const float2* sml) {
+  const float2 ml = lane < r.n ? sml[lane] : make_float2(-INFINITY, 0.0f);
+  float M = ml.x;
+#pragma unroll
+  for (int d = 16; d; d >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, d));
+  const float w_lane = lane < r.n ? exp2f(__fsub_rn(ml.x, M)) : 0.0f;
+  float Lsum = 0.0f;
+  float o0 = 0.0f, o1 = 0.0f, o2 = 0.0f, o3 = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    if (k < r.n) {  // the same for the whole warp
+      const float w = __shfl_sync(0xffffffffu, w_lane, k);
+      const float l = __shfl_sync(0xffffffffu, ml.y, k);
+      const float4 o = so[k * 32 + lane];
+      Lsum = __fmaf_rn(w, l, Lsum);
+      o0 = __fmaf_rn(w, o.x, o0);
+      o1 = __fmaf_rn(w, o.y, o1);
+      o2 = __fmaf_rn(w, o.z, o2);
+      o3 = __fmaf_rn(w, o.w, o3);
+    }
+  }
+  const float y0 = __fadd_rn(__fdiv_rn(o0, Lsum), 0.0f), y1 = __fadd_rn(__fdiv_rn(o1, Lsum), 0.0f);
+  const float y2 = __fadd_rn(__fdiv_rn(o2, Lsum), 0.0f), y3 = __fadd_rn(__fdiv_rn(o3, Lsum), 0.0f);
+  *reinterpret_cast<uint2*>(r.dst) = make_uint2(E16<ET>::pack2(y0, y1), E16<ET>::pack2(y2, y3));
+}
+
 // A grid of a few CTAs per SM whose warps stride over the (token, head) rows
 // (tens of thousands of one-row CTAs cost more in scheduling than the rows).
+// A warp issues the next row's loads (cp.async into its own shared-memory
+// slots, double-buffered) before merging the current row, so two rows' loads
+// are in flight per warp without holding them in registers. Rows with more
+// than four splits are merged from global memory (combine_row).
 template <typename ET>
 __global__ void __launch_bounds__(256, 4) attn_combine_kernel(const CombineParams p) {
+  __shared__ __align__(16) float4 s_o[8][2][4 * 32];  // [warp][buffer][split * 32 + lane]
+  __shared__ __align__(16) float2 s_ml[8][2][32];     // [warp][buffer][lane = split]
   // launched as a programmatic dependent of the split kernel: wait until that
   // grid has completed and its writes are visible
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int64_t rows = (int64_t)p.n_tok * p.Hq;
   const int64_t step = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); wid < rows; wid += step)
-    combine_row<ET>(p, (int)(wid / p.Hq), (int)(wid % p.Hq), lane);
+  int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + w;
+  if (wid >= rows) return;
+  CombRow cur = comb_setup(p, wid, lane);
+  int buf = 0;
+  comb_issue(p, cur, lane, s_o[w][0], s_ml[w][0]);
+  for (; wid < rows; wid += step) {
+    CombRow nxt;
+    nxt.kind = 0;
+    if (wid + step < rows) nxt = comb_setup(p, wid + step, lane);
+    comb_issue(p, nxt, lane, s_o[w][buf ^ 1], s_ml[w][buf ^ 1]);
+    cp_async_wait<1>();  // this lane's copies of the current row have landed
+    if (cur.kind == 1) {
+      *reinterpret_cast<uint2*>(cur.dst) = make_uint2(0u, 0u);
+    } else if (cur.kind == 2) {
+      comb_short<ET>(cur, lane, s_o[w][buf], s_ml[w][buf]);
+    } else if (cur.kind == 3) {
+      combine_row<ET>(p, cur.tok, cur.h, lane);
+    }
+    cur = nxt;
+    buf ^= 1;
+  }
+  cp_async_wait<0>();
 }
 
 // partial O [n_tok][Hq][n_split][128] fp32, then (m, l) pairs, then (256-byte
