@@ -946,8 +946,9 @@ __global__ void __launch_bounds__(Lay<DECODE>::THREADS, 1)
   }
 }
 
-// Finishing pass: one warp per (query token, q head); lane owns 4 of the 128
-// output elements. Splits merged strictly in order s = 0 .. n-1.
+// Finishing pass: a (query token, q head) row is merged by one warp, lane
+// owning 4 of the 128 output elements. Splits merged strictly in order s = 0
+// .. n-1.
 struct CombineParams {
   const float* ws_o;
   const float* ws_ml;
@@ -957,6 +958,7 @@ struct CombineParams {
   int64_t ldo;
   int32_t n_tok, B, Hq, n_split_max, max_kv_len;
   int32_t max_rows;  // rows per sequence the split kernel covers (qblocks x rows per block)
+  int32_t hpu;       // heads of one query token per unit of work (1 .. 16)
 };
 
 // One (token, head) row, by one warp.
@@ -1032,49 +1034,66 @@ __device__ __forceinline__ void combine_row(const CombineParams& p, int tok, int
   *reinterpret_cast<uint2*>(dst) = make_uint2(E16<ET>::pack2(y0, y1), E16<ET>::pack2(y2, y3));
 }
 
-// A row's place in the finishing pass: 0 not covered by this call, 1 zeros
-// (flagged by the split kernel), 2 n <= 4 splits, 3 more.
-struct CombRow {
-  int kind, n, tok, h;
-  size_t base;
-  uint16_t* dst;
+// A query token's place in the finishing pass (every head of a token is the
+// same case): 0 nothing to do (not covered by this call), 1 zeros (flagged by
+// the split kernel), 2 n <= 4 splits, 3 more.
+struct CombTok {
+  int kind, n, tok;
 };
 
-__device__ __forceinline__ CombRow comb_setup(const CombineParams& p, int64_t wid, int lane) {
-  CombRow r;
-  r.tok = (int)(wid / p.Hq);
-  r.h = (int)(wid % p.Hq);
-  r.kind = 0;
-  r.n = 0;
-  r.base = 0;
-  r.dst = nullptr;
+__device__ __forceinline__ CombTok comb_token(const CombineParams& p, int tok) {
+  CombTok t;
+  t.tok = tok;
+  t.kind = 0;
+  t.n = 0;
   int b, nb, qidx;
   if (p.cu_q) {
-    if (r.tok < p.cu_q[0] || r.tok >= p.cu_q[p.B]) return r;  // a row this call does not cover
+    if (tok < p.cu_q[0] || tok >= p.cu_q[p.B]) return t;  // a token this call does not cover
     int lo = 0, hi = p.B;  // find b with cu_q[b] <= tok < cu_q[b+1]
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
-      if (p.cu_q[mid] <= r.tok) lo = mid; else hi = mid;
+      if (p.cu_q[mid] <= tok) lo = mid; else hi = mid;
     }
     b = lo;
     nb = p.cu_q[b + 1] - p.cu_q[b];
-    qidx = r.tok - p.cu_q[b];
+    qidx = tok - p.cu_q[b];
     if (p.cu_q[b] < 0 || p.cu_q[b + 1] > p.n_tok) nb = 0;  // malformed cu_q: zeros
   } else {
-    b = r.tok;
+    b = tok;
     nb = 1;
     qidx = 0;
   }
   const int L = p.seq_lens[b];
-  r.dst = static_cast<uint16_t*>(p.out) + (size_t)r.tok * p.ldo + (size_t)r.h * HD + lane * 4;
   if (L < nb || L > p.max_kv_len || nb <= 0 || qidx >= p.max_rows) {
-    r.kind = 1;
-    return r;
+    t.kind = 1;
+    return t;
   }
-  r.n = (L - nb + qidx) / SPLIT + 1;
-  r.base = ((size_t)r.tok * p.Hq + r.h) * p.n_split_max;
-  r.kind = r.n <= 4 ? 2 : 3;
+  t.n = (L - nb + qidx) / SPLIT + 1;
+  t.kind = t.n <= 4 ? 2 : 3;
+  return t;
+}
+
+// One (token, head) row of the finishing pass and its token's case.
+struct CombRow {
+  int kind, n, tok, h;
+};
+
+__device__ __forceinline__ CombRow comb_row(const CombTok& t, int h) {
+  CombRow r;
+  r.kind = t.kind;
+  r.n = t.n;
+  r.tok = t.tok;
+  r.h = h;
   return r;
+}
+
+// The row's first partial (split 0) in the workspace, and this lane's 4
+// output elements.
+__device__ __forceinline__ size_t comb_base(const CombineParams& p, const CombRow& r) {
+  return ((size_t)r.tok * p.Hq + r.h) * p.n_split_max;
+}
+__device__ __forceinline__ uint16_t* comb_dst(const CombineParams& p, const CombRow& r, int lane) {
+  return static_cast<uint16_t*>(p.out) + (size_t)r.tok * p.ldo + (size_t)r.h * HD + lane * 4;
 }
 
 // A short row's loads, issued asynchronously (cp.async) into this lane's own
@@ -1083,15 +1102,16 @@ __device__ __forceinline__ CombRow comb_setup(const CombineParams& p, int64_t wi
 __device__ __forceinline__ void comb_issue(const CombineParams& p, const CombRow& r, int lane, float4* so,
                                            float2* sml) {
   if (r.kind == 2) {
+    const size_t base = comb_base(p, r);
 #pragma unroll
     for (int k = 0; k < 4; ++k)
       if (k < r.n)
         asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(smem_u32(so + k * 32 + lane)),
-                     "l"(p.ws_o + (r.base + k) * HD + lane * 4)
+                     "l"(p.ws_o + (base + k) * HD + lane * 4)
                      : "memory");
     if (lane < r.n)
       asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(sml + lane)),
-                   "l"(p.ws_ml + (r.base + lane) * 2)
+                   "l"(p.ws_ml + (base + lane) * 2)
                    : "memory");
   }
   cp_async_commit();
@@ -1101,7 +1121,8 @@ __device__ __forceinline__ void comb_issue(const CombineParams& p, const CombRow
 // combine_row (M over the splits' m by shuffles, weights 2^(m_s - M), sums in
 // split order, y = o / L + 0).
 template <typename ET>
-__device__ __forceinline__ void comb_short(const CombRow& r, int lane, const float4* so, const float2* sml) {
+__device__ __forceinline__ void comb_short(const CombineParams& p, const CombRow& r, int lane, const float4* so,
+                                           const float2* sml) {
   const float2 ml = lane < r.n ? sml[lane] : make_float2(-INFINITY, 0.0f);
   float M = ml.x;
 #pragma unroll
@@ -1124,15 +1145,18 @@ __device__ __forceinline__ void comb_short(const CombRow& r, int lane, const flo
   }
   const float y0 = __fadd_rn(__fdiv_rn(o0, Lsum), 0.0f), y1 = __fadd_rn(__fdiv_rn(o1, Lsum), 0.0f);
   const float y2 = __fadd_rn(__fdiv_rn(o2, Lsum), 0.0f), y3 = __fadd_rn(__fdiv_rn(o3, Lsum), 0.0f);
-  *reinterpret_cast<uint2*>(r.dst) = make_uint2(E16<ET>::pack2(y0, y1), E16<ET>::pack2(y2, y3));
+  *reinterpret_cast<uint2*>(comb_dst(p, r, lane)) = make_uint2(E16<ET>::pack2(y0, y1), E16<ET>::pack2(y2, y3));
 }
 
-// A grid of a few CTAs per SM whose warps stride over the (token, head) rows
-// (tens of thousands of one-row CTAs cost more in scheduling than the rows).
-// A warp issues the next row's loads (cp.async into its own shared-memory
-// slots, double-buffered) before merging the current row, so two rows' loads
-// are in flight per warp without holding them in registers. Rows with more
-// than four splits are merged from global memory (combine_row).
+// A grid of a few CTAs per SM whose warps stride over units of one query
+// token and up to p.hpu of its heads (tens of thousands of one-row CTAs
+// cost more in scheduling than the rows); the token's sequence and split
+// count are looked up once per unit. A warp walks its rows (the heads of a
+// unit, then the next unit's) and issues the next row's loads (cp.async into
+// its own shared-memory slots, double-buffered) before merging the current
+// row, so two rows' loads are in flight per warp without holding them in
+// registers. Rows with more than four splits are merged from global memory
+// (combine_row).
 template <typename ET>
 __global__ void __launch_bounds__(256, 4) attn_combine_kernel(const CombineParams p) {
   __shared__ __align__(16) float4 s_o[8][2][4 * 32];  // [warp][buffer][split * 32 + lane]
@@ -1141,28 +1165,45 @@ __global__ void __launch_bounds__(256, 4) attn_combine_kernel(const CombineParam
   // grid has completed and its writes are visible
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int64_t rows = (int64_t)p.n_tok * p.Hq;
+  const int hch = (p.Hq + p.hpu - 1) / p.hpu;  // units per token
+  const int64_t units = (int64_t)p.n_tok * hch;
   const int64_t step = (int64_t)gridDim.x * (blockDim.x >> 5);
-  int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + w;
-  if (wid >= rows) return;
-  CombRow cur = comb_setup(p, wid, lane);
+  int64_t u = (int64_t)blockIdx.x * (blockDim.x >> 5) + w;
+  if (u >= units) return;
+  // row cursor: unit u, head h of [h .. h_end)
+  CombTok t = comb_token(p, (int)(u / hch));
+  int h = (int)(u % hch) * p.hpu;
+  int h_end = min(h + p.hpu, p.Hq);
+  auto advance = [&]() -> bool {  // to the next row; false past the last
+    if (++h < h_end) return true;
+    u += step;
+    if (u >= units) return false;
+    t = comb_token(p, (int)(u / hch));
+    h = (int)(u % hch) * p.hpu;
+    h_end = min(h + p.hpu, p.Hq);
+    return true;
+  };
+  CombRow cur = comb_row(t, h);
   int buf = 0;
   comb_issue(p, cur, lane, s_o[w][0], s_ml[w][0]);
-  for (; wid < rows; wid += step) {
+  bool more = advance();
+  while (true) {
     CombRow nxt;
     nxt.kind = 0;
-    if (wid + step < rows) nxt = comb_setup(p, wid + step, lane);
+    if (more) nxt = comb_row(t, h);
     comb_issue(p, nxt, lane, s_o[w][buf ^ 1], s_ml[w][buf ^ 1]);
     cp_async_wait<1>();  // this lane's copies of the current row have landed
     if (cur.kind == 1) {
-      *reinterpret_cast<uint2*>(cur.dst) = make_uint2(0u, 0u);
+      *reinterpret_cast<uint2*>(comb_dst(p, cur, lane)) = make_uint2(0u, 0u);
     } else if (cur.kind == 2) {
-      comb_short<ET>(cur, lane, s_o[w][buf], s_ml[w][buf]);
+      comb_short<ET>(p, cur, lane, s_o[w][buf], s_ml[w][buf]);
     } else if (cur.kind == 3) {
       combine_row<ET>(p, cur.tok, cur.h, lane);
     }
+    if (!more) break;
     cur = nxt;
     buf ^= 1;
+    more = advance();
   }
   cp_async_wait<0>();
 }
@@ -1299,7 +1340,18 @@ static bi_status run(const void* q, int64_t ldq, const int32_t* cu_q, int32_t ma
   c.n_split_max = n_split;
   c.max_kv_len = sh->max_kv_len;
   c.max_rows = qblocks * QR;
-  const int64_t warps = n_tok * Hq;
+  // Heads per unit: the largest of 16, 8, 4, 2 that still leaves a unit for
+  // every warp of the grid (four CTAs of eight warps per SM), else 1. Units
+  // decide only which warp merges a row, never how.
+  const int64_t grid_warps = (int64_t)sms * 4 * 8;
+  c.hpu = 1;
+  for (int hpu = 16; hpu > 1; hpu >>= 1) {
+    if (n_tok * ((Hq + hpu - 1) / hpu) >= grid_warps) {
+      c.hpu = hpu;
+      break;
+    }
+  }
+  const int64_t warps = n_tok * ((Hq + c.hpu - 1) / c.hpu);  // one per (token, head unit)
   const int64_t want = (warps + 7) / 8;
   const int blocks = (int)(want < (int64_t)num_sms() * 4 ? want : (int64_t)num_sms() * 4);
   // programmatic dependent launch: the combine is launched as the split

@@ -168,6 +168,25 @@ def test_prefill_bench_workload_sampled(bi):
     assert same_bits(dec, out[idx])
 
 
+def test_finishing_pass_work_units_do_not_change_bits(bi):
+    """The finishing pass hands a warp units of one token and up to 16 of its
+    heads when the call has rows enough, else one row per warp. With 24 q
+    heads a 2400-token prefill takes 16-head units, the second one ragged (8
+    heads); the same rows from 300-token chunks (one row per warp) are the
+    same bits, and sampled rows match the fp64 oracle."""
+    L = 2400
+    S = Seqs(bi, [L], 24, 6, seed=71)
+    shape = S.shape(bi)
+    whole = _prefill(bi, S, [(0, 0, L)], shape)
+    for s0 in range(0, L, 300):
+        part = _prefill(bi, S, [(0, s0, s0 + 300)], shape)
+        assert same_bits(part, whole[s0:s0 + 300]), f"chunk at {s0}"
+    positions = [0, 511, 512, 1535, 1536, 2047, 2048, 2399]
+    o64, R = S.oracle(0, positions)
+    check(f64(whole[torch.tensor(positions)]).reshape(len(positions), 24, D), o64, R, kappa=1.0,
+          what="prefill 24 heads")
+
+
 def test_batch_composition(bi):
     """A sequence's rows are the same bits alone, co-batched with others of
     mixed lengths and chunk sizes, and at a different batch position."""
