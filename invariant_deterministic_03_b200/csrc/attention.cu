@@ -1186,8 +1186,10 @@ __global__ void __launch_bounds__(256, 4) attn_combine_kernel(const CombineParam
   CombRow cur = comb_row(t, h);
   int buf = 0;
   comb_issue(p, cur, lane, s_o[w][0], s_ml[w][0]);
-  bool more = advance();
-  while (true) {
+  // every pass merges the current row; the loop ends after the row at which
+  // the cursor (advance) ran past this warp's last unit
+  bool more = advance(), last = false;
+  do {
     CombRow nxt;
     nxt.kind = 0;
     if (more) nxt = comb_row(t, h);
@@ -1200,11 +1202,11 @@ __global__ void __launch_bounds__(256, 4) attn_combine_kernel(const CombineParam
     } else if (cur.kind == 3) {
       combine_row<ET>(p, cur.tok, cur.h, lane);
     }
-    if (!more) break;
+    last = !more;
     cur = nxt;
     buf ^= 1;
-    more = advance();
-  }
+    if (more) more = advance();
+  } while (!last);
   cp_async_wait<0>();
 }
 
