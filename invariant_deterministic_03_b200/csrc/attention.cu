@@ -55,11 +55,12 @@ constexpr int PAGES_PER_TILE = TILE / PAGE;
 constexpr uint32_t TILE_BYTES = 128 * 128 * 2;  // 32 KB: one K or V tile (128 keys x 128 d)
 constexpr int ITEM_RING = 16;                   // claimed work items in flight inside a CTA
 
-// Shared-memory layout. Prefill: Q and P are full 128-row tiles, one buffer
-// each (Q is released after an item's last Q K^T, so the next item's Q loads
-// while its softmax finishes), two K and three V buffers (the V copies are
-// the ones the P V products wait for; two K and three V measured ~2 % faster
-// than three K and two V). Decode: the MMA rows that matter are the G <= 8
+// Shared-memory layout. Prefill: Q and P are full 128-row tiles; two Q
+// buffers (the next item's Q loads while the current item runs), one P
+// buffer, two K and two V buffers (seven 32 KB tiles fill the 227 KB: two Q
+// and two V measured 1.6 % faster than one Q and three V, one Q and three V
+// ~2 % faster than one Q, three K and two V, and a second P buffer in place
+// of the third V gained nothing). Decode: the MMA rows that matter are the G <= 8
 // head rows of one query, so Q and P keep just one 8-row core-matrix group
 // per 64-column half and the MMA operand descriptor repeats it for all 16
 // groups (8-row-group stride 0): the same 128-row MMA reads the same values
@@ -70,8 +71,8 @@ constexpr int ITEM_RING = 16;                   // claimed work items in flight 
 template <bool DECODE>
 struct Lay {
   static constexpr int NK = DECODE ? 3 : 2;                 // K tile buffers
-  static constexpr int NQ = DECODE ? 2 : 1;                 // Q buffers
-  static constexpr int NV = 3;                              // V tile buffers
+  static constexpr int NQ = 2;                              // Q buffers
+  static constexpr int NV = DECODE ? 3 : 2;                 // V tile buffers
   static constexpr int NP = DECODE ? 2 : 1;                 // P buffers
   static constexpr int NS = DECODE ? 3 : 2;                 // S buffers in tensor memory
   static constexpr int SOFTMAX_WARPS = DECODE ? 4 : 16;     // one 32-key quarter of 32 rows each
