@@ -187,6 +187,30 @@ def test_finishing_pass_work_units_do_not_change_bits(bi):
           what="prefill 24 heads")
 
 
+def test_flagged_sequence_inside_work_units(bi):
+    """A call large enough for 16-head units in the finishing pass, with one
+    sequence whose length exceeds max_kv_len: that sequence's rows are zeros
+    and BI_DEV_BAD_SEQLEN is set, and every other row is the same bits as in
+    a call without it (8-head units)."""
+    L = 600
+    S = Seqs(bi, [L] * 4, 32, 8, seed=73)
+    shape = S.shape(bi)
+    q = dev(torch.cat([S.q[b].reshape(L, -1) for b in range(4)]))
+    cu = dev(torch.tensor([0, L, 2 * L, 3 * L, 4 * L], dtype=torch.int32))
+    ws = torch.empty(bi.bi_attn_workspace_size(shape, 4 * L), dtype=torch.uint8, device="cuda:0")
+    out = torch.empty_like(q)
+    bi.bi_device_status(clear=True)
+    bi.bi_attn_prefill(q, cu, L, S.kc, S.vc, S.bt, dev(torch.tensor([L, L, 5000, L], dtype=torch.int32)),
+                       shape, out, ws)
+    torch.cuda.synchronize()
+    assert bi.bi_device_status(clear=True) & 0x8      # BI_DEV_BAD_SEQLEN
+    assert not out[2 * L:3 * L].float().abs().any()
+    good = _prefill(bi, S, [(0, 0, L), (1, 0, L), (3, 0, L)], shape)
+    assert bi.bi_device_status(clear=True) == 0
+    assert same_bits(out[:2 * L], good[:2 * L])
+    assert same_bits(out[3 * L:], good[2 * L:])
+
+
 def test_batch_composition(bi):
     """A sequence's rows are the same bits alone, co-batched with others of
     mixed lengths and chunk sizes, and at a different batch position."""
