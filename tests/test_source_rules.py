@@ -5,7 +5,8 @@ status bit, never a dead context); no device allocation inside the library
 mbarrier carries the cycle limit on its own line, and the only open-ended
 loops are the two bounded-wait helpers (each returns on the cycle limit or
 the CTA's abort flag) and the work-claiming loop (its counter only grows,
-up to the item count).
+up to the item count); no TMA or bulk copy uses cluster multicast (the one
+multicast is the tcgen05.commit that signals both CTAs of a GEMM pair).
 """
 import os
 import re
@@ -54,3 +55,12 @@ def test_every_spin_wait_is_bounded():
                 assert "kWaitLimitCycles" in line, f"{f}:{n}: unbounded mbarrier poll"
             if re.search(r"while\s*\(\s*(true|1)\s*\)|for\s*\(\s*;\s*;\s*\)", line):
                 assert current in OPEN_LOOP_OK, f"{f}:{n}: open-ended loop in {current}"
+
+
+def test_no_multicast_copies():
+    for f, text in _sources():
+        for n, line in enumerate(_code(text).split("\n"), 1):
+            if "multicast" in line:
+                assert "tcgen05.commit" in line, f"{f}:{n}: multicast outside tcgen05.commit"
+            if re.search(r"cp\.async\.bulk", line):
+                assert "multicast" not in line, f"{f}:{n}: bulk copy with multicast"
