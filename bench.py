@@ -500,6 +500,37 @@ def rmsnorm_leg(bi, torch, reps):
             "sweep_d4096": sweep, "sweep_rows_bitwise_across_M": bool(bitwise)}
 
 
+def rmsnorm_fold_leg(bi, torch, reps):
+    """The 7B QKV projection after its RMSNorm at decode sizes: bi_gemm_rmsnorm
+    (the norm applied while the GEMM writes its A stages) against
+    bi_rmsnorm_f32in followed by bi_gemm, which gives the same bits; the
+    weights rotate over three copies so no call reads them from L2; calls
+    back to back."""
+    K, N = 4096, 6144
+    g = torch.Generator("cuda").manual_seed(4)
+    Ws = [(torch.randn(N, K, device="cuda", generator=g) * 0.02).to(torch.bfloat16) for _ in range(3)]
+    gamma = torch.rand(K, device="cuda", generator=g).to(torch.bfloat16)
+    rows = []
+    for M in (64, 256):
+        x = torch.randn(M, K, device="cuda", generator=g)
+        C = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        C2 = torch.empty_like(C)
+        h = torch.empty(M, K, dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(bi.bi_gemm_rmsnorm_workspace_size(M, K), dtype=torch.uint8, device="cuda")
+        fused = back_to_back_ms(torch, lambda r=0: bi.bi_gemm_rmsnorm(x, gamma, 1e-6, Ws[r % 3], C, ws), reps)
+
+        def unfused_call(r=0):
+            bi.bi_rmsnorm(x, gamma, h, 1e-6)
+            bi.bi_gemm(h, Ws[r % 3], C2)
+        unfused = back_to_back_ms(torch, unfused_call, reps)
+        bi.bi_gemm_rmsnorm(x, gamma, 1e-6, Ws[0], C, ws)
+        unfused_call(0)
+        rows.append({"M": M, "fused_us": round(fused * 1e3, 2), "unfused_us": round(unfused * 1e3, 2),
+                     "same_bits": bool(same_bits(C, C2))})
+    return {"workload": "QKV projection of the 7B shape (K=4096, N=6144) on fp32 rows after RMSNorm",
+            "rows": rows}
+
+
 def e2e_leg(bi, torch, sw, steps):
     """The same sweep through the C-ABI with HOST buffers: per step, each
     shape's weights and each launch's A rows go host->device from pinned
@@ -952,6 +983,7 @@ def main():
         pa["peak"] = peak_t
         extras["attn_prefill"] = pa
         extras["rmsnorm"] = r
+        extras["rmsnorm_fold"] = rmsnorm_fold_leg(bi, torch, reps=50)
         extras["invariance"] = invariance_flags(torch, sw)
         extras["forward"] = forward_leg(torch, reps=5)
 

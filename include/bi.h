@@ -178,6 +178,36 @@ bi_status bi_gemm_qkv(const void* A, int64_t lda, const void* W, int64_t ldw,
                       void* k_cache, void* v_cache, int32_t num_pages,
                       void* stream);
 
+/* RMSNorm folded into the next GEMM's A operand ("Defeating Nondeterminism
+ * in LLM Inference", sections "Batch-invariant RMSNorm" and "Batch-invariant
+ * matmul": the norm's per-row reduction and the matmul's per-element K loop
+ * keep their own fixed orders, so the fused op is batch-invariant too).
+ *   bi_gemm_rmsnorm:        C = bi_gemm(bi_rmsnorm_f32in(x, gamma, eps), W)
+ *   bi_gemm_rmsnorm_swiglu: out = bi_gemm_swiglu(bi_rmsnorm_f32in(x, ...), W)
+ * with exactly those calls' bits. x fp32 [M, K] contiguous (the residual
+ * stream), gamma [K] bf16, W [N, K] (swiglu: [2F, K]) bf16 with row stride
+ * ldw; C [M, N] bf16 or fp32 (c_dtype BI_BF16 / BI_F32), out [M, F] bf16.
+ * When every output tile has a CTA pair of its own (small M), the GEMM's
+ * otherwise idle epilogue warps write r16((x r_i) gamma) into each A stage
+ * (after a pass computing r_i by bi_rmsnorm_f32in's reduction); otherwise
+ * the normed rows go through the workspace and the plain GEMM runs. ws:
+ * caller-owned device memory of bi_gemm_rmsnorm_workspace_size(M, K) bytes,
+ * 16-byte aligned. Constraints as bi_gemm, K (the normed width) <= 32768,
+ * x and gamma 16-byte aligned. M == 0 or N == 0 is a no-op. Measured on
+ * B200 the folded path is slower than the two calls (0.097 vs 0.031 ms for
+ * the 7B QKV projection at M = 64): the GEMM's SMs then read the fp32 rows,
+ * twice the bytes of the bf16 normed rows, next to the weights they stream;
+ * bi_forward uses the two calls. */
+bi_status bi_gemm_rmsnorm_workspace_size(int64_t M, int64_t K, size_t* bytes);
+bi_status bi_gemm_rmsnorm(const float* x, const void* gamma, float eps,
+                          const void* W, int64_t ldw, void* C, int64_t ldc,
+                          int32_t c_dtype, int64_t M, int64_t N, int64_t K,
+                          void* ws, size_t ws_bytes, void* stream);
+bi_status bi_gemm_rmsnorm_swiglu(const float* x, const void* gamma, float eps,
+                                 const void* W, int64_t ldw, void* out,
+                                 int64_t ldo, int64_t M, int64_t F, int64_t K,
+                                 void* ws, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Paged KV cache.  "Defeating Nondeterminism in LLM Inference", section
  * "Batch-invariant attention": the cache and page table are updated BEFORE

@@ -79,6 +79,9 @@ _SIGS = {
     "bi_gemm_swiglu": (_i32, [_p, _i64, _p, _i64, _p, _i64, _i64, _i64, _i64, _p]),
     "bi_gemm_qkv": (_i32, [_p, _i64, _p, _i64, _p, _i64, _i64, _i64, _i32, _i32, _p, _p, _i32, _p, _p, _p,
                            _i32, _p]),
+    "bi_gemm_rmsnorm_workspace_size": (_i32, [_i64, _i64, ctypes.POINTER(_sz)]),
+    "bi_gemm_rmsnorm": (_i32, [_p, _p, _f32, _p, _i64, _p, _i64, _i32, _i64, _i64, _i64, _p, _sz, _p]),
+    "bi_gemm_rmsnorm_swiglu": (_i32, [_p, _p, _f32, _p, _i64, _p, _i64, _i64, _i64, _i64, _p, _sz, _p]),
     "bi_kv_append": (_i32, [_p, _p, _i64, _p, _i64, _p, _p, ctypes.POINTER(KVLayout), _p]),
     "bi_attn_workspace_size": (_i32, [ctypes.POINTER(AttnShape), _i64, ctypes.POINTER(_sz)]),
     "bi_attn_decode": (_i32, [_p, _i64, _p, _p, _p, _p, _i32, ctypes.POINTER(AttnShape), _p,
@@ -175,6 +178,45 @@ def bi_gemm(A, W, C, stream=None, add: bool = False) -> None:
     fn = "bi_gemm_f16" if f16 else "bi_gemm"
     _chk(fn, getattr(lib, fn)(_ptr(A), A.stride(0), _ptr(W), W.stride(0), _ptr(C), C.stride(0),
                               cdt, M, N, K, _stream(stream)))
+
+
+def bi_gemm_rmsnorm_workspace_size(M: int, K: int) -> int:
+    n = _sz(0)
+    _chk("bi_gemm_rmsnorm_workspace_size", lib.bi_gemm_rmsnorm_workspace_size(M, K, ctypes.byref(n)))
+    return n.value
+
+
+def _check_fold_args(x, gamma, W, out, ws, rows_w: int, where: str) -> None:
+    M, K = x.shape
+    if x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError(f"{where}: x must be contiguous fp32 [M, K]")
+    if gamma.numel() < K or W.shape[0] < rows_w or W.shape[1] < K or out.shape[0] < M:
+        raise ValueError(f"{where}: gamma / W / out smaller than the shapes")
+    if ws.numel() * ws.element_size() < bi_gemm_rmsnorm_workspace_size(M, K):
+        raise ValueError(f"{where}: workspace too small")
+
+
+def bi_gemm_rmsnorm(x, gamma, eps: float, W, C, ws, c_dtype: int = BI_BF16, stream=None) -> None:
+    """C = bi_gemm(bi_rmsnorm_f32in(x, gamma, eps), W) with the same bits. x [M, K]
+    fp32, gamma [K] bf16, W [N, K] bf16, C [M, N] bf16 or fp32, ws from
+    bi_gemm_rmsnorm_workspace_size(M, K)."""
+    M, K = x.shape
+    N = C.shape[1]
+    _check_fold_args(x, gamma, W, C, ws, N, "bi_gemm_rmsnorm")
+    _chk("bi_gemm_rmsnorm", lib.bi_gemm_rmsnorm(_ptr(x), _ptr(gamma), eps, _ptr(W), W.stride(0), _ptr(C),
+                                                C.stride(0), c_dtype, M, N, K, _ptr(ws),
+                                                ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def bi_gemm_rmsnorm_swiglu(x, gamma, eps: float, W, out, ws, stream=None) -> None:
+    """out = bi_gemm_swiglu(bi_rmsnorm_f32in(x, gamma, eps), W) with the same
+    bits. W [2F, K] bf16 (gate rows, then up rows), out [M, F] bf16."""
+    M, K = x.shape
+    F = out.shape[1]
+    _check_fold_args(x, gamma, W, out, ws, 2 * F, "bi_gemm_rmsnorm_swiglu")
+    _chk("bi_gemm_rmsnorm_swiglu", lib.bi_gemm_rmsnorm_swiglu(_ptr(x), _ptr(gamma), eps, _ptr(W), W.stride(0),
+                                                              _ptr(out), out.stride(0), M, F, K, _ptr(ws),
+                                                              ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def bi_gemm_swiglu(A, W, out, stream=None) -> None:

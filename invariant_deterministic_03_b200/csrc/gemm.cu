@@ -37,7 +37,9 @@
 //               both CTAs (stage free, accumulator full), which each CTA
 //               waits on at CTA scope (one commit to both measured ~5 %
 //               faster than a commit per CTA with cluster-scope waits)
-//   warps 2..5  epilogue of this CTA's 128 rows: tcgen05.ld the accumulator
+//   warps 2..5  (FOLD only, first) write the A stages from fp32 rows, see
+//               gemm_tcgen05_kernel; then
+//               epilogue of this CTA's 128 rows: tcgen05.ld the accumulator
 //               row by row (thread = row), round to bf16 (RNE) or keep fp32,
 //               store to global, or run one of the fused epilogues (EPI_ADD,
 //               EPI_SWIGLU, EPI_QKV below) on the finished values; then free
@@ -98,6 +100,12 @@ struct Params {
   uint16_t* kc;          // key cache (16-bit elements), 4 KB per (page, kv head)
   uint16_t* vc;          // value cache, same blocking, transposed per page
   int32_t max_pos, num_pages, hq, hkv;
+  // FOLD only: A[m, k] = r16((x[m, k] * r[m]) * gamma[k]), the RMSNorm of the
+  // fp32 rows x applied while the A tile is written to shared memory
+  const float* fx;       // [M, ldx] fp32 rows
+  int64_t ldx;
+  const float* fr;       // [M] row scales (rmsnorm_scales_f32)
+  const uint16_t* fg;    // [K] gamma, 16-bit (the element type)
 };
 
 template <typename ET>
@@ -307,7 +315,14 @@ __device__ __forceinline__ void qkv_tile(const Params& p, int row, int nb, uint3
   }
 }
 
-template <int TERMS, int EPI, typename ET>
+// FOLD (TERMS = 1, only when every pair holds at most one tile): warps 2..5
+// write each A stage themselves before their epilogue, as r16((x * r) * gamma)
+// from fp32 rows -- the operations of bi_rmsnorm_f32in, so A holds the same
+// bits as that kernel's output and the product is the same as bi_rmsnorm_f32in
+// then bi_gemm. Each of the 8 warps (4 per CTA) arrives on rank 0's "full"
+// barrier of the stage after its rows are written and fenced for the tensor
+// core; the W copies arrive as in the TMA path.
+template <int TERMS, int EPI, typename ET, bool FOLD = false>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmA2,
@@ -336,7 +351,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], FOLD ? 9 : 1);  // FOLD: + one arrival per A-writing warp of both CTAs
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -377,7 +392,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const bool a_live = a_row < p.M;
         // bytes landing on rank 0's full barrier per stage: both CTAs' copies
         const bool a1_live = mb * BM + BM_CTA < p.M;
-        const uint32_t tx = TERMS * p.a_bytes * (a1_live ? 2u : 1u) + 2u * B_BYTES;
+        const uint32_t tx = FOLD ? 2u * B_BYTES : TERMS * p.a_bytes * (a1_live ? 2u : 1u) + 2u * B_BYTES;
         // W rows of this CTA: BN/2 from nb * BN + rank * BN/2, or (SwiGLU)
         // BN/2 gate rows from nb * BN/2 (rank 0) or the matching up rows
         // from F + nb * BN/2 (rank 1)
@@ -389,7 +404,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           uint8_t* sa = tiles + stage * STAGE_BYTES;
           const uint32_t fb = cluster_addr(&full[stage], 0);
           if (rank == 0) mbar_arrive_expect_tx(&full[stage], tx);
-          if (a_live) {
+          if (!FOLD && a_live) {
             tma_load_2d_pair(sa, &tmA, fb, kb * BK, a_row);
             if (TERMS == 2) tma_load_2d_pair(sa + A_BYTES, &tmA2, fb, kb * BK, a_row);
           }
@@ -472,6 +487,89 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int quarter = warp & 3;
     const int trow = quarter * 32 + lane;  // accumulator row (TMEM lane) of this thread
     const uint32_t acc_empty0 = cluster_addr(acc_empty, 0);
+    if constexpr (FOLD) {
+      // A stages of this CTA's 128 rows (the pair's only tile). The 128
+      // threads of warps 2..5 share the rows below M: eight threads per row,
+      // one 16-byte chunk (8 columns) each, so a row's fp32 x is read in one
+      // coalesced 256-byte piece; a thread has at most 8 chunks per stage.
+      // Two register sets hold the loads of two stages, so a stage's loads
+      // are in flight while the one before it is converted.
+      constexpr int CH = 8;
+      bool ok = tile0 < num_tiles;
+      const int mb = ok ? tile0 % p.m_blocks : 0;
+      const int row_base = mb * BM + (int)rank * BM_CTA;
+      const int live = max(0, min(BM_CTA, p.M - row_base));
+      const int ct = (int)threadIdx.x - 64;          // 0 .. 127
+      const uint32_t full0 = cluster_addr(full, 0);  // rank 0's barriers
+      float4 xa[CH][2], xb[CH][2];
+      uint4 ga[CH], gb[CH];
+      float ra[CH], rb[CH];
+      // the loads of stage kb's chunks into one register set
+      auto load = [&](int kb, float4 (&x)[CH][2], uint4 (&g)[CH], float (&r)[CH]) {
+#pragma unroll
+        for (int j = 0; j < CH; ++j) {
+          const int c = ct + 128 * j;
+          const int row = c >> 3, k0 = kb * BK + (c & 7) * 8;
+          if (row < live && k0 < p.K) {  // K % 8 == 0: a chunk is wholly inside or outside
+            const float* xr = p.fx + (size_t)(row_base + row) * p.ldx + k0;
+            x[j][0] = *reinterpret_cast<const float4*>(xr);
+            x[j][1] = *reinterpret_cast<const float4*>(xr + 4);
+            g[j] = *reinterpret_cast<const uint4*>(p.fg + k0);
+            r[j] = p.fr[row_base + row];
+          }
+        }
+      };
+      // r16((x r) gamma) of stage kb's chunks into the stage's A tile
+      auto store = [&](int kb, uint8_t* sa, const float4 (&x)[CH][2], const uint4 (&g)[CH], const float (&r)[CH]) {
+#pragma unroll
+        for (int j = 0; j < CH; ++j) {
+          const int c = ct + 128 * j;
+          const int row = c >> 3, ch = c & 7, k0 = kb * BK + ch * 8;
+          if (row >= live) continue;  // rows past M are never stored; they keep stale values
+          uint4 o = make_uint4(0u, 0u, 0u, 0u);  // columns past K: zeros, as a TMA copy would fill
+          if (k0 < p.K) {
+            const float xv[8] = {x[j][0].x, x[j][0].y, x[j][0].z, x[j][0].w,
+                                 x[j][1].x, x[j][1].y, x[j][1].z, x[j][1].w};
+            const uint32_t g2[4] = {g[j].x, g[j].y, g[j].z, g[j].w};
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float lo = __fmul_rn(__fmul_rn(xv[2 * e], r[j]), E16<ET>::lo(g2[e]));
+              const float hi = __fmul_rn(__fmul_rn(xv[2 * e + 1], r[j]), E16<ET>::hi(g2[e]));
+              w[e] = E16<ET>::pack2(lo, hi);
+            }
+            o = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          // 128-byte swizzle of a 1024-byte aligned tile: chunk ch of row
+          // `row` sits at chunk ch ^ (row % 8) of the row
+          *reinterpret_cast<uint4*>(sa + row * 128 + ((ch ^ (row & 7)) << 4)) = o;
+        }
+      };
+      int stage = 0;
+      uint32_t phase = 0;
+      if (ok) load(0, xa, ga, ra);
+      if (ok && p.k_blocks > 1) load(1, xb, gb, rb);
+      for (int kb = 0; kb < p.k_blocks && ok; ++kb) {
+        const bool even = (kb & 1) == 0;
+        if (!mbar_wait(&empty[stage], phase ^ 1, p.status, abort_flag)) { ok = false; break; }
+        uint8_t* sa = tiles + stage * STAGE_BYTES;
+        if (even) store(kb, sa, xa, ga, ra);
+        else store(kb, sa, xb, gb, rb);
+        fence_proxy_async_smem();  // the writes, visible to the tensor core
+        __syncwarp();
+        if (lane == 0) {
+          if (rank == 0) mbar_arrive(&full[stage]);
+          else mbar_arrive_cluster(full0 + stage * 8);
+        }
+        // the loads of the stage two ahead into the registers just used,
+        // issued after the fence so that it does not wait for them
+        if (kb + 2 < p.k_blocks) {
+          if (even) load(kb + 2, xa, ga, ra);
+          else load(kb + 2, xb, gb, rb);
+        }
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = tile0; tile < num_tiles; tile += tile_step) {
@@ -561,7 +659,7 @@ static bi_status check_args(const void* A, int64_t lda, const void* W, int64_t l
   return BI_OK;
 }
 
-template <int TERMS, int EPI, typename ET>
+template <int TERMS, int EPI, typename ET, bool FOLD = false>
 static bi_status set_smem_attr() {
   static bool done[64] = {false};
   static std::mutex mu;
@@ -570,7 +668,7 @@ static bi_status set_smem_attr() {
   if (dev < 0 || dev >= 64) return fail(BI_ERR_UNSUPPORTED, "gemm: device id %d out of range", dev);
   std::lock_guard<std::mutex> lk(mu);
   if (!done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tcgen05_kernel<TERMS, EPI, ET>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_tcgen05_kernel<TERMS, EPI, ET, FOLD>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Cfg<TERMS>::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e, "gemm: smem attribute");
@@ -581,11 +679,11 @@ static bi_status set_smem_attr() {
 
 // How many CTA pairs of this kernel the device runs at once (queried once per
 // device).
-template <int TERMS, int EPI, typename ET>
+template <int TERMS, int EPI, typename ET, bool FOLD = false>
 static bi_status pair_slots(int* out) {
   static int cache[64] = {0};
   static std::mutex mu;
-  bi_status st = set_smem_attr<TERMS, EPI, ET>();
+  bi_status st = set_smem_attr<TERMS, EPI, ET, FOLD>();
   if (st != BI_OK) return st;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -604,7 +702,7 @@ static bi_status pair_slots(int* out) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    cudaError_t e = cudaOccupancyMaxActiveClusters(&n, gemm_tcgen05_kernel<TERMS, EPI, ET>, &cfg);
+    cudaError_t e = cudaOccupancyMaxActiveClusters(&n, gemm_tcgen05_kernel<TERMS, EPI, ET, FOLD>, &cfg);
     if (e != cudaSuccess) return cuda_fail(e, "gemm: cluster occupancy");
     if (n <= 0) return fail(BI_ERR_UNSUPPORTED, "gemm: no two-CTA cluster fits on this device");
     v = n;
@@ -622,12 +720,20 @@ struct QkvArgs {
   int32_t max_pos, num_pages, hq, hkv;
 };
 
+struct FoldArgs {
+  const float* x;
+  int64_t ldx;
+  const float* r;
+  const void* gamma;
+};
+
 // N is the output width: the W rows for EPI_STORE / EPI_ADD / EPI_QKV, the
-// feature count F (W has 2F rows) for EPI_SWIGLU.
-template <int TERMS, int EPI, typename ET>
+// feature count F (W has 2F rows) for EPI_SWIGLU. FOLD: A comes from fa (the
+// caller has checked that every pair holds at most one tile).
+template <int TERMS, int EPI, typename ET, bool FOLD = false>
 static bi_status launch(const void* A, const void* A2, int64_t lda, const void* W, int64_t ldw,
                         void* C, int64_t ldc, int32_t c_dtype, int64_t M, int64_t N, int64_t K,
-                        cudaStream_t s, const QkvArgs* qa = nullptr) {
+                        cudaStream_t s, const QkvArgs* qa = nullptr, const FoldArgs* fa = nullptr) {
   bi_status st;
   const int32_t c_f32 = c_dtype != BI_BF16;
   if (K == 0) {
@@ -638,7 +744,7 @@ static bi_status launch(const void* A, const void* A2, int64_t lda, const void* 
   }
   CUtensorMap tmA, tmA2, tmB;
   const uint32_t a_rows = M < BM_CTA ? (uint32_t)((M + 7) / 8 * 8) : (uint32_t)BM_CTA;
-  {
+  if (!FOLD) {
     uint64_t dims[2] = {(uint64_t)K, (uint64_t)M};
     uint64_t strides[1] = {(uint64_t)lda * 2};
     uint32_t box[2] = {BK, a_rows};
@@ -661,6 +767,7 @@ static bi_status launch(const void* A, const void* A2, int64_t lda, const void* 
                           strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != BI_OK)
       return st;
   }
+  if (FOLD) tmA = tmA2 = tmB;  // not read: the A stages are written by the kernel
   Params p;
   p.C = C;
   p.ldc = ldc;
@@ -682,10 +789,15 @@ static bi_status launch(const void* A, const void* A2, int64_t lda, const void* 
   p.num_pages = qa ? qa->num_pages : 0;
   p.hq = qa ? qa->hq : 0;
   p.hkv = qa ? qa->hkv : 0;
+  p.fx = fa ? fa->x : nullptr;
+  p.ldx = fa ? fa->ldx : 0;
+  p.fr = fa ? fa->r : nullptr;
+  p.fg = fa ? static_cast<const uint16_t*>(fa->gamma) : nullptr;
   p.a_bytes = a_rows * BK * 2;
   int slots = 0;
-  if ((st = pair_slots<TERMS, EPI, ET>(&slots)) != BI_OK) return st;
+  if ((st = pair_slots<TERMS, EPI, ET, FOLD>(&slots)) != BI_OK) return st;
   const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
+  if (FOLD && (tiles > slots || !fa)) return fail(BI_ERR_SHAPE, "gemm fold: more tiles than CTA pairs");
   p.w_prefetch = tiles <= slots ? W_PREFETCH : 0;
   const int64_t pairs = tiles < slots ? tiles : slots;
   cudaLaunchConfig_t cfg = {};
@@ -700,7 +812,7 @@ static bi_status launch(const void* A, const void* A2, int64_t lda, const void* 
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tcgen05_kernel<TERMS, EPI, ET>, tmA, tmA2, tmB, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tcgen05_kernel<TERMS, EPI, ET, FOLD>, tmA, tmA2, tmB, p);
   if (e != cudaSuccess) return cuda_fail(e, "gemm: cluster launch");
   BI_CHECK_LAUNCH("gemm launch");
   return BI_OK;
@@ -789,6 +901,78 @@ template bi_status gemm_qkv_e16<f16>(const void*, int64_t, const void*, int64_t,
                                      int32_t, int32_t, const int32_t*, const float*, int32_t, const int32_t*,
                                      void*, void*, int32_t, cudaStream_t);
 }  // namespace bi
+
+namespace bi {
+bi_status rmsnorm_scales_f32(const float* x, int64_t M, int64_t D, float eps, float* r, cudaStream_t s);
+
+namespace gemm {
+// Workspace of the RMSNorm-folded GEMM: the row scales (M fp32, 256-byte
+// rounded), then room for the normed rows (M x K bf16) used when the fold
+// does not apply.
+static size_t fold_ws_bytes(int64_t M, int64_t K) {
+  return (((size_t)M * 4 + 255) & ~(size_t)255) + (size_t)M * K * 2;
+}
+
+// C = (RMSNorm(x) with gamma) W^T, x fp32 [M, K] contiguous. When every CTA
+// pair holds at most one output tile the norm is applied inside the GEMM
+// (FOLD: the row scales first, by bi_rmsnorm_f32in's reduction, then the
+// GEMM writes r16((x r) gamma) into its A stages); otherwise the normed rows
+// go through the workspace (bi_rmsnorm_f32in, then the plain GEMM). Either
+// way the bits are those of bi_rmsnorm_f32in followed by bi_gemm (or
+// bi_gemm_swiglu for EPI_SWIGLU).
+template <int EPI>
+static bi_status rmsnorm_gemm(const float* x, const void* gamma, float eps, const void* W, int64_t ldw, void* C,
+                              int64_t ldc, int32_t c_dtype, int64_t M, int64_t N, int64_t K, void* ws,
+                              size_t ws_bytes, cudaStream_t s) {
+  if (!x || !gamma || !ws) return fail(BI_ERR_INVALID_ARG, "gemm_rmsnorm: null pointer");
+  bi_status st = check_args(ws, K, W, ldw, C, ldc, c_dtype, M, N, K);
+  if (st != BI_OK) return st;
+  if (c_dtype == BI_F32_ADD) return fail(BI_ERR_INVALID_ARG, "gemm_rmsnorm: c_dtype must be BI_BF16 or BI_F32");
+  if (EPI == EPI_SWIGLU && c_dtype != BI_BF16) return fail(BI_ERR_INVALID_ARG, "gemm_rmsnorm_swiglu: output is bf16");
+  if (K <= 0 || K > 32768) return fail(BI_ERR_SHAPE, "gemm_rmsnorm: K (the normed width) must be 8 .. 32768");
+  if (!aligned16(x) || !aligned16(gamma)) return fail(BI_ERR_ALIGN, "gemm_rmsnorm: x and gamma must be 16-byte aligned");
+  if (!(eps >= 0.0f)) return fail(BI_ERR_INVALID_ARG, "gemm_rmsnorm: eps must be >= 0");
+  if (ws_bytes < fold_ws_bytes(M, K)) return fail(BI_ERR_WORKSPACE, "gemm_rmsnorm: workspace %zu < %zu", ws_bytes,
+                                                  fold_ws_bytes(M, K));
+  if (M == 0 || N == 0) return BI_OK;
+  if ((st = require_sm100()) != BI_OK) return st;
+  float* r = static_cast<float*>(ws);
+  bf16* h = reinterpret_cast<bf16*>(static_cast<uint8_t*>(ws) + (((size_t)M * 4 + 255) & ~(size_t)255));
+  int slots = 0;
+  if ((st = pair_slots<1, EPI, bf16, true>(&slots)) != BI_OK) return st;
+  const int64_t cols_per_tile = EPI == EPI_SWIGLU ? BN / 2 : BN;
+  const int64_t tiles = ((M + BM - 1) / BM) * ((N + cols_per_tile - 1) / cols_per_tile);
+  if (tiles <= slots) {
+    if ((st = rmsnorm_scales_f32(x, M, K, eps, r, s)) != BI_OK) return st;
+    const FoldArgs fa{x, K, r, gamma};
+    return launch<1, EPI, bf16, true>(nullptr, nullptr, K, W, ldw, C, ldc, c_dtype, M, N, K, s, nullptr, &fa);
+  }
+  if ((st = bi_rmsnorm_f32in(x, gamma, h, M, K, eps, s)) != BI_OK) return st;
+  return launch<1, EPI, bf16>(h, nullptr, K, W, ldw, C, ldc, c_dtype, M, N, K, s);
+}
+}  // namespace gemm
+}  // namespace bi
+
+extern "C" bi_status bi_gemm_rmsnorm_workspace_size(int64_t M, int64_t K, size_t* bytes) {
+  if (!bytes || M < 0 || K < 0) return fail(BI_ERR_INVALID_ARG, "gemm_rmsnorm_workspace_size: bad arguments");
+  *bytes = gemm::fold_ws_bytes(M, K);
+  return BI_OK;
+}
+
+extern "C" bi_status bi_gemm_rmsnorm(const float* x, const void* gamma, float eps, const void* W, int64_t ldw,
+                                     void* C, int64_t ldc, int32_t c_dtype, int64_t M, int64_t N, int64_t K,
+                                     void* ws, size_t ws_bytes, void* stream) {
+  return gemm::rmsnorm_gemm<gemm::EPI_STORE>(x, gamma, eps, W, ldw, C, ldc, c_dtype, M, N, K, ws, ws_bytes,
+                                             static_cast<cudaStream_t>(stream));
+}
+
+extern "C" bi_status bi_gemm_rmsnorm_swiglu(const float* x, const void* gamma, float eps, const void* W,
+                                            int64_t ldw, void* out, int64_t ldo, int64_t M, int64_t F, int64_t K,
+                                            void* ws, size_t ws_bytes, void* stream) {
+  if (F > (1ll << 29)) return fail(BI_ERR_SHAPE, "gemm_rmsnorm_swiglu: F above 2^29");
+  return gemm::rmsnorm_gemm<gemm::EPI_SWIGLU>(x, gamma, eps, W, ldw, out, ldo, BI_BF16, M, F, K, ws, ws_bytes,
+                                              static_cast<cudaStream_t>(stream));
+}
 
 extern "C" bi_status bi_gemm(const void* A, int64_t lda, const void* W, int64_t ldw, void* C,
                              int64_t ldc, int32_t c_dtype, int64_t M, int64_t N, int64_t K,

@@ -62,12 +62,13 @@ struct Row8<float> {
 // SPLIT: write the fp32 result as a bf16 pair (y = bf16(v), y_lo = bf16(v - y))
 // for the fp32-activation path; otherwise y = r16(v), r16 the rounding to
 // the 16-bit output type ET (bf16, or fp16 for the FP16 variant; gamma has
-// the same type).
-template <typename Tin, int CPT, bool SPLIT, typename ET>
+// the same type). R_ONLY: write only the row's scale r to r_out[row] (the
+// same reduction, for a GEMM that applies the norm to its A operand).
+template <typename Tin, int CPT, bool SPLIT, typename ET, bool R_ONLY = false>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const Tin* __restrict__ x,
                                                       const ET* __restrict__ gamma,
                                                       ET* __restrict__ y, ET* __restrict__ y_lo,
-                                                      int D, float eps) {
+                                                      int D, float eps, float* __restrict__ r_out = nullptr) {
   __shared__ float warp_sum[32];
   __shared__ float row_scale;
   const int T = blockDim.x;
@@ -98,7 +99,9 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const Tin* __restrict__ x,
     const int nw = T >> 5;
     for (int w = 0; w < nw; ++w) total = total + warp_sum[w];
     row_scale = 1.0f / sqrtf(total / (float)D + eps);
+    if (R_ONLY) r_out[row] = row_scale;
   }
+  if (R_ONLY) return;
   __syncthreads();
   const float r = row_scale;
 #pragma unroll
@@ -165,6 +168,30 @@ static bi_status check_rms(const void* x, const void* gamma, const void* y, int6
   if (M > 0x7fffffffll) return fail(BI_ERR_SHAPE, "rmsnorm: M=%lld too large", (long long)M);
   if (!(eps >= 0.0f)) return fail(BI_ERR_INVALID_ARG, "rmsnorm: eps must be >= 0");
   if (!aligned16(x) || !aligned16(gamma) || !aligned16(y)) return fail(BI_ERR_ALIGN, "rmsnorm: pointers must be 16-byte aligned");
+  return BI_OK;
+}
+
+// The row scales r_i = 1 / sqrt(sum_j x_ij^2 / D + eps) of fp32 rows, by the
+// reduction bi_rmsnorm_f32in uses (same geometry, same order), into r[M].
+bi_status rmsnorm_scales_f32(const float* x, int64_t M, int64_t D, float eps, float* r, cudaStream_t s) {
+  if (!x || !r) return fail(BI_ERR_INVALID_ARG, "rmsnorm scales: null pointer");
+  if (M < 0 || D <= 0 || D % 8 != 0 || D > 32768 || M > 0x7fffffffll)
+    return fail(BI_ERR_SHAPE, "rmsnorm scales: bad sizes M=%lld D=%lld", (long long)M, (long long)D);
+  if (!(eps >= 0.0f)) return fail(BI_ERR_INVALID_ARG, "rmsnorm scales: eps must be >= 0");
+  if (!aligned16(x)) return fail(BI_ERR_ALIGN, "rmsnorm scales: x must be 16-byte aligned");
+  if (M == 0) return BI_OK;
+  int T, cpt;
+  rms_geometry(D, &T, &cpt);
+  dim3 grid((unsigned)M), block(T);
+  switch (cpt) {
+    case 1: rmsnorm_kernel<float, 1, false, bf16, true><<<grid, block, 0, s>>>(x, nullptr, nullptr, nullptr, (int)D, eps, r); break;
+    case 2: rmsnorm_kernel<float, 2, false, bf16, true><<<grid, block, 0, s>>>(x, nullptr, nullptr, nullptr, (int)D, eps, r); break;
+    case 4: rmsnorm_kernel<float, 4, false, bf16, true><<<grid, block, 0, s>>>(x, nullptr, nullptr, nullptr, (int)D, eps, r); break;
+    case 8: rmsnorm_kernel<float, 8, false, bf16, true><<<grid, block, 0, s>>>(x, nullptr, nullptr, nullptr, (int)D, eps, r); break;
+    case 16: rmsnorm_kernel<float, 16, false, bf16, true><<<grid, block, 0, s>>>(x, nullptr, nullptr, nullptr, (int)D, eps, r); break;
+    default: return fail(BI_ERR_SHAPE, "rmsnorm scales: D=%lld unsupported", (long long)D);
+  }
+  BI_CHECK_LAUNCH("rmsnorm scales launch");
   return BI_OK;
 }
 
