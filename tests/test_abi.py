@@ -156,3 +156,30 @@ def test_gemm_qkv_host_checks(bi):
     assert call(max_pos=0) == bi.BI_ERR_INVALID_ARG
     assert call(kc=p + 8) == bi.BI_ERR_ALIGN
     assert call(M=0) == bi.BI_OK                        # nothing to do
+
+
+def test_gemm_rmsnorm_host_checks(bi):
+    p = 0x1000
+    n = ctypes.c_size_t(0)
+    assert bi.lib.bi_gemm_rmsnorm_workspace_size(64, 4096, ctypes.byref(n)) == bi.BI_OK
+    assert n.value == 256 + 64 * 4096 * 2                   # row scales (256-byte rounded), then normed rows
+    assert bi.lib.bi_gemm_rmsnorm_workspace_size(-1, 8, ctypes.byref(n)) == bi.BI_ERR_INVALID_ARG
+    g = bi.lib.bi_gemm_rmsnorm
+    ok = dict(x=p, gamma=p, eps=1e-6, W=p, ldw=512, C=p, ldc=256, c=bi.BI_BF16, M=4, N=256, K=512, ws=p,
+              wsb=1 << 20, s=None)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return g(a["x"], a["gamma"], a["eps"], a["W"], a["ldw"], a["C"], a["ldc"], a["c"], a["M"], a["N"], a["K"],
+                 a["ws"], a["wsb"], a["s"])
+    assert call(x=None) == bi.BI_ERR_INVALID_ARG
+    assert call(ws=None) == bi.BI_ERR_INVALID_ARG
+    assert call(c=bi.BI_F32_ADD) == bi.BI_ERR_INVALID_ARG   # no accumulation into C
+    assert call(K=500, ldw=504) == bi.BI_ERR_SHAPE           # K % 8
+    assert call(gamma=p + 8) == bi.BI_ERR_ALIGN
+    assert call(eps=-1.0) == bi.BI_ERR_INVALID_ARG
+    assert call(wsb=100) == bi.BI_ERR_WORKSPACE
+    assert call(M=0) == bi.BI_OK                            # nothing to do
+    sw = bi.lib.bi_gemm_rmsnorm_swiglu
+    assert sw(p, p, 1e-6, p, 512, p, 256, 4, 256, 512, p, 100, None) == bi.BI_ERR_WORKSPACE
+    assert sw(p, p, 1e-6, p, 512, p, 256, 0, 256, 512, p, 1 << 20, None) == bi.BI_OK
