@@ -538,7 +538,9 @@ def e2e_leg(bi, torch, sw, steps):
     Copies are pipelined on their own streams (host->device on one, the
     GEMMs on the timing stream, device->host on a third, ordered by events),
     so a launch's inputs arrive while earlier launches compute; every launch
-    has its own device buffers."""
+    has its own device buffers. Within a shape the launches go from the
+    largest M down, so the step ends on small copies instead of the largest
+    product and its read-back."""
     hA = {K: sw.A[K].cpu().pin_memory() for K, _ in SHAPES}
     hW = {(K, N): sw.W[(K, N)][0].cpu().pin_memory() for K, N in SHAPES}
     hC = {(K, N): torch.empty(sum(MS) * N, dtype=torch.bfloat16).pin_memory() for K, N in SHAPES}
@@ -563,14 +565,14 @@ def e2e_leg(bi, torch, sw, steps):
         with torch.cuda.stream(s_in):
             for K, N in SHAPES:
                 dW[(K, N)].copy_(hW[(K, N)], non_blocking=True)
-                for M in MS:
+                for M in reversed(MS):
                     dA[(K, M)].copy_(hA[K][:M], non_blocking=True)
                     ev = torch.cuda.Event()
                     ev.record(s_in)
                     ready[(K, M)] = ev
         for K, N in SHAPES:
             off = 0
-            for M in MS:
+            for M in reversed(MS):
                 comp.wait_event(ready[(K, M)])
                 C = dC[(N, M)]
                 bi.bi_gemm(dA[(K, M)], dW[(K, N)], C)
